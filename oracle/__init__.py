@@ -1,0 +1,230 @@
+"""CPU oracle for record-and-replay discrete adjoints -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference leg may import this package.  The product (``discrete_adjoint_b200``)
+never imports it and shares no code with it.
+
+The oracle is ``oracle.cpp`` compiled with ``-ffp-contract=off`` (so the
+compiler never fuses a multiply and an add on its own: every fused
+multiply-add is an explicit ``std::fma`` at a site fixed by the floating-point
+contract) and loaded through ctypes.  What each entry computes, and the
+passage of GRADSOLVE (arXiv 2609.02876) it follows, is documented in
+``oracle.cpp``.
+
+Array conventions here: per-trajectory inputs are structure-of-arrays, ``p``
+``[np][n]``, ``u0`` ``[d][n]``, ``target``/``weight`` ``[nsave][d][n]``; the
+oracle's own mesh is trajectory-major, ``h`` ``[n][smax]``,
+``save_idx`` ``[n][nsave]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+SYSTEMS = {"lorenz": 1, "robertson": 2, "hires": 3, "node64": 4, "linear": 5}
+METHODS = {"tsit5": 1, "ros2": 2}
+DTYPES = {"f32": 1, "f64": 2}
+LOSSES = {"sumsq": 1, "linear": 2}
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source (g++, no fused contraction)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    cmd = ["g++", "-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+           "-pthread", "-o", _LIB + ".tmp", _SRC]
+    subprocess.run(cmd, check=True)
+    os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        L.or_record.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, f64, f64, i32, dp, f64, f64, f64,
+                                i32, dp, ip, ip, ip, ip, i32]
+        L.or_grad.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, ip, i32, dp, dp,
+                              i32, dp, dp, dp, dp, i32]
+        L.or_dirderiv.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, i32, dp, dp,
+                                  dp, dp, dp, dp, i32]
+        L.or_replay.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, i32, dp, dp,
+                                dp, dp, i32]
+        L.or_count_step.argtypes = [i32, i32, i32, i32, dp]
+        L.or_step.argtypes = [i32, i32, i32, i32, dp, dp, dp, f64, dp, dp]
+        L.or_rhs.argtypes = [i32, i32, dp, dp, dp, dp, dp]
+        L.or_tsit5_tableau.argtypes = [dp, dp, dp]
+        L.or_tsit5_tableau.restype = None
+        L.or_ros2_gamma.restype = f64
+        _lib = L
+    return _lib
+
+
+def _d(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _i(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+@dataclass
+class Mesh:
+    """The oracle's record: trajectory-major, zero padded."""
+    h: np.ndarray         # [n][smax] float64 (fp32 runs hold fp32 values)
+    nsteps: np.ndarray    # [n] int32
+    save_idx: np.ndarray  # [n][nsave] int32
+    status: np.ndarray    # [n] int32
+    nreject: np.ndarray   # [n] int32
+
+    @property
+    def smax(self) -> int:
+        return self.h.shape[1]
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def record(prob, smax: int, h0: float = 0.0, nthreads: int | None = None) -> Mesh:
+    """Adaptive record of every trajectory of ``prob`` (a ``workloads.Problem``)."""
+    L = lib()
+    n, nsave = prob.n, len(prob.tsave)
+    p, u0, W, ts = _f64(prob.p), _f64(prob.u0), _f64(prob.W), _f64(prob.tsave)
+    h = np.zeros((n, smax), np.float64)
+    nsteps = np.zeros(n, np.int32)
+    save_idx = np.zeros((n, max(nsave, 1)), np.int32)
+    status = np.zeros(n, np.int32)
+    nrej = np.zeros(n, np.int32)
+    rc = L.or_record(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, prob.d, prob.np_,
+                     _d(p), _d(u0), _d(W), prob.t0, prob.t1, nsave, _d(ts), prob.rtol, prob.atol, h0, smax,
+                     _d(h), _i(nsteps), _i(save_idx), _i(status), _i(nrej), nthreads or default_threads())
+    _check(rc, "record")
+    return Mesh(h, nsteps, save_idx[:, :nsave], status, nrej)
+
+
+def _mesh_args(mesh: Mesh):
+    h = np.ascontiguousarray(mesh.h, np.float64)
+    ns = np.ascontiguousarray(mesh.nsteps, np.int32)
+    si = np.ascontiguousarray(mesh.save_idx, np.int32)
+    return h, ns, si
+
+
+def grad(prob, mesh: Mesh, mode: str = "tape", nthreads: int | None = None):
+    """Exact gradient of the fixed-step replay loss.
+
+    mode ``"tape"``: reverse-mode AD (tape).  mode ``"dual"``: forward mode,
+    one dual-number pass per input (p and u0; not node64).
+    Returns dict(loss [n], dp [np][n], du0 [d][n], dW [64,64] or None).
+    """
+    L = lib()
+    n, d, npar = prob.n, prob.d, prob.np_
+    h, ns, si = _mesh_args(mesh)
+    st = np.ascontiguousarray(mesh.status, np.int32)
+    loss = np.zeros(n)
+    dp = np.zeros((npar, n))
+    du0 = np.zeros((d, n))
+    dW = np.zeros((64, 64)) if prob.system == "node64" else None
+    rc = L.or_grad(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, d, npar, _d(_f64(prob.p)),
+                   _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si), _i(st),
+                   LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), 0 if mode == "tape" else 1,
+                   _d(loss), _d(dp), _d(du0), _d(dW), nthreads or default_threads())
+    _check(rc, "grad")
+    return {"loss": loss, "dp": dp, "du0": du0, "dW": dW}
+
+
+def dirderiv(prob, mesh: Mesh, dir_p=None, dir_u0=None, dir_W=None, nthreads: int | None = None):
+    """Forward-mode directional derivative of each trajectory's loss, [n]."""
+    L = lib()
+    h, ns, si = _mesh_args(mesh)
+    out = np.zeros(prob.n)
+    rc = L.or_dirderiv(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], prob.n, prob.d, prob.np_,
+                       _d(_f64(prob.p)), _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h),
+                       _i(ns), _i(si), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)),
+                       _d(_f64(dir_p)), _d(_f64(dir_u0)), _d(_f64(dir_W)), _d(out), nthreads or default_threads())
+    _check(rc, "dirderiv")
+    return out
+
+
+def replay(prob, mesh: Mesh, nthreads: int | None = None):
+    """Plain replay: (loss [n], u_save [nsave][d][n])."""
+    L = lib()
+    h, ns, si = _mesh_args(mesh)
+    loss = np.zeros(prob.n)
+    us = np.zeros((si.shape[1], prob.d, prob.n))
+    rc = L.or_replay(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], prob.n, prob.d, prob.np_,
+                     _d(_f64(prob.p)), _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h),
+                     _i(ns), _i(si), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), _d(loss),
+                     _d(us), nthreads or default_threads())
+    _check(rc, "replay")
+    return loss, us
+
+
+def count_step(system: str, method: str, d: int, npar: int) -> dict:
+    """Arithmetic operations of one fixed replay step (no error estimate)."""
+    out = np.zeros(6)
+    lib().or_count_step(SYSTEMS[system], METHODS[method], d, npar, _d(out))
+    return dict(zip(["add", "mul", "fma", "div", "sqrt", "tanh"], out.astype(int).tolist()))
+
+
+def step(system: str, method: str, dtype: str, u, p, h: float, W=None):
+    """One step of the method: (u_new, error estimate, ok)."""
+    u = _f64(u)
+    pp = np.zeros(64)
+    if p is not None:
+        pp[: len(p)] = p
+    un = np.zeros_like(u)
+    er = np.zeros_like(u)
+    rc = lib().or_step(SYSTEMS[system], METHODS[method], DTYPES[dtype], len(u), _d(u), _d(pp), _d(_f64(W)),
+                       h, _d(un), _d(er))
+    return un, er, rc == 0
+
+
+def rhs(system: str, u, p, W=None):
+    """(f(u), analytic Jacobian or zeros) at one point, float64."""
+    u = _f64(u)
+    d = len(u)
+    f = np.zeros(d)
+    J = np.zeros((d, d)) if d <= 8 else None
+    lib().or_rhs(SYSTEMS[system], d, _d(u), _d(_f64(p)), _d(_f64(W)), _d(f), _d(J))
+    return f, J
+
+
+def tsit5_tableau():
+    c = np.zeros(7)
+    A = np.zeros((7, 6))
+    bt = np.zeros(7)
+    lib().or_tsit5_tableau(_d(c), _d(A), _d(bt))
+    return c, A, bt
+
+
+def ros2_gamma() -> float:
+    return float(lib().or_ros2_gamma())

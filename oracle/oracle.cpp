@@ -1,0 +1,900 @@
+// oracle.cpp -- plain, slow CPU oracle for record-and-replay discrete adjoints.
+//
+// TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or
+// call this file.  Only tests/, __graft_entry__.smoke() and bench.py's CPU
+// baseline / reference leg load the shared library built from it.  It shares no
+// code with the CUDA library: the step formulas below are written out a second
+// time from the method's definition and from the floating-point contract (the
+// operation order that both sides follow), not from the kernels.
+//
+// What it computes (GRADSOLVE, arXiv 2609.02876, abstract and the evolve.pub
+// review "Summary" / "Strengths: precisely scoped exactness claim"): an adaptive
+// solver records the step sizes it accepts; a fixed-step replay of those steps,
+// with the mesh held as data, defines the loss; the gradient is the exact
+// derivative of that replay (the discrete adjoint), excluding any derivative of
+// the step-size choices.
+//
+//   record()   the adaptive solve, step by step, plain scalar arithmetic.
+//   replay<S>  fixed-step replay over a recorded mesh, generic in the scalar S.
+//   grad       reverse-mode AD of replay<S> with a small operator-overloading
+//              tape (S = Rv<T>), i.e. the definition "derivative of the replay"
+//              written out, not a hand-derived adjoint.
+//   dirderiv   forward-mode dual numbers (S = Dv<T>) through the same replay:
+//              an independent second route to the same derivative.
+//   flops      a counting scalar (S = Cn) to count the replay's operations.
+//
+// Integrators: Tsitouras' 5(4) pair (Tsit5, Tsitouras 2011) and the
+// second-order Rosenbrock method ROS2 of Verwer, Spee, Blom & Hundsdorfer
+// (1999) with gamma = 1 + 1/sqrt(2).  Systems: Lorenz (DiffEqGPU "ad" example,
+// "Forward-mode automatic differentiation" listing), Robertson kinetics
+// (mass-action form of the reaction scheme A->B (k1), 2B->B+C (k2),
+// B+C->A+C (k3)), and the d=64 shared-weight system tanh(W u + b) - u.
+//
+// Parity pins for every function here live in tests/test_oracle_*.py.
+#include <algorithm>
+#include <cfloat>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <type_traits>
+#include <vector>
+
+namespace orc {
+
+// ---------------------------------------------------------------------------
+// Scalar types.  Every overload computes its VALUE with exactly the plain-T
+// operation (one rounding per +,-,*,/, one per fma), so replay<Rv<T>>,
+// replay<Dv<T>> and replay<T> produce bitwise identical forward values.
+// ---------------------------------------------------------------------------
+
+// ---- reverse mode: tape of nodes, each with up to three parents -----------
+template <class T>
+struct Node {
+  T v;
+  int32_t a, b, c;
+  T da, db, dc;
+};
+
+template <class T>
+struct Tape {
+  std::vector<Node<T>> nodes;
+  int32_t push(T v, int32_t a = -1, T da = 0, int32_t b = -1, T db = 0, int32_t c = -1, T dc = 0) {
+    nodes.push_back(Node<T>{v, a, b, c, da, db, dc});
+    return (int32_t)nodes.size() - 1;
+  }
+};
+
+template <class T>
+Tape<T>& tape() {
+  static thread_local Tape<T> t;
+  return t;
+}
+
+// A reverse-mode variable: value plus tape index (-1 = constant, no node).
+template <class T>
+struct Rv {
+  T v;
+  int32_t id;
+  Rv() : v(0), id(-1) {}
+  Rv(T x) : v(x), id(-1) {}  // constants carry no node
+  Rv(T x, int32_t i) : v(x), id(i) {}
+};
+
+template <class T>
+Rv<T> rv_node(T v, int32_t a, T da, int32_t b = -1, T db = 0, int32_t c = -1, T dc = 0) {
+  if (a < 0 && b < 0 && c < 0) return Rv<T>(v);
+  return Rv<T>(v, tape<T>().push(v, a, da, b, db, c, dc));
+}
+template <class T> Rv<T> operator+(Rv<T> x, Rv<T> y) { return rv_node<T>(x.v + y.v, x.id, 1, y.id, 1); }
+template <class T> Rv<T> operator-(Rv<T> x, Rv<T> y) { return rv_node<T>(x.v - y.v, x.id, 1, y.id, -1); }
+template <class T> Rv<T> operator*(Rv<T> x, Rv<T> y) { return rv_node<T>(x.v * y.v, x.id, y.v, y.id, x.v); }
+template <class T> Rv<T> operator/(Rv<T> x, Rv<T> y) {
+  T q = x.v / y.v;
+  return rv_node<T>(q, x.id, T(1) / y.v, y.id, -q / y.v);
+}
+template <class T> Rv<T> operator-(Rv<T> x) { return rv_node<T>(-x.v, x.id, -1); }
+template <class T> Rv<T> fma_(Rv<T> x, Rv<T> y, Rv<T> z) {
+  return rv_node<T>(std::fma(x.v, y.v, z.v), x.id, y.v, y.id, x.v, z.id, 1);
+}
+template <class T> Rv<T> sqrt_(Rv<T> x) {
+  T r = std::sqrt(x.v);
+  return rv_node<T>(r, x.id, T(0.5) / r);
+}
+template <class T> Rv<T> tanh_(Rv<T> x) {
+  T r = std::tanh(x.v);
+  return rv_node<T>(r, x.id, T(1) - r * r);
+}
+template <class T> T val(Rv<T> x) { return x.v; }
+
+// ---- forward mode: one tangent direction -----------------------------------
+template <class T>
+struct Dv {
+  T v, d;
+  Dv() : v(0), d(0) {}
+  Dv(T x) : v(x), d(0) {}
+  Dv(T x, T dx) : v(x), d(dx) {}
+};
+template <class T> Dv<T> operator+(Dv<T> x, Dv<T> y) { return Dv<T>(x.v + y.v, x.d + y.d); }
+template <class T> Dv<T> operator-(Dv<T> x, Dv<T> y) { return Dv<T>(x.v - y.v, x.d - y.d); }
+template <class T> Dv<T> operator*(Dv<T> x, Dv<T> y) { return Dv<T>(x.v * y.v, x.d * y.v + x.v * y.d); }
+template <class T> Dv<T> operator/(Dv<T> x, Dv<T> y) {
+  T q = x.v / y.v;
+  return Dv<T>(q, (x.d - q * y.d) / y.v);
+}
+template <class T> Dv<T> operator-(Dv<T> x) { return Dv<T>(-x.v, -x.d); }
+template <class T> Dv<T> fma_(Dv<T> x, Dv<T> y, Dv<T> z) {
+  return Dv<T>(std::fma(x.v, y.v, z.v), x.d * y.v + x.v * y.d + z.d);
+}
+template <class T> Dv<T> sqrt_(Dv<T> x) {
+  T r = std::sqrt(x.v);
+  return Dv<T>(r, x.d * (T(0.5) / r));
+}
+template <class T> Dv<T> tanh_(Dv<T> x) {
+  T r = std::tanh(x.v);
+  return Dv<T>(r, x.d * (T(1) - r * r));
+}
+template <class T> T val(Dv<T> x) { return x.v; }
+
+// ---- operation counter ------------------------------------------------------
+struct OpCount {
+  int64_t add = 0, mul = 0, fma = 0, div = 0, sqrt = 0, tanh = 0;
+};
+inline OpCount& opcount() {
+  static thread_local OpCount c;
+  return c;
+}
+struct Cn {
+  double v;
+  Cn() : v(0) {}
+  Cn(double x) : v(x) {}
+};
+inline Cn operator+(Cn x, Cn y) { opcount().add++; return Cn(x.v + y.v); }
+inline Cn operator-(Cn x, Cn y) { opcount().add++; return Cn(x.v - y.v); }
+inline Cn operator*(Cn x, Cn y) { opcount().mul++; return Cn(x.v * y.v); }
+inline Cn operator/(Cn x, Cn y) { opcount().div++; return Cn(x.v / y.v); }
+inline Cn operator-(Cn x) { return Cn(-x.v); }  // sign flip: not an arithmetic op
+inline Cn fma_(Cn x, Cn y, Cn z) { opcount().fma++; return Cn(std::fma(x.v, y.v, z.v)); }
+inline Cn sqrt_(Cn x) { opcount().sqrt++; return Cn(std::sqrt(x.v)); }
+inline Cn tanh_(Cn x) { opcount().tanh++; return Cn(std::tanh(x.v)); }
+inline double val(Cn x) { return x.v; }
+
+// ---- plain scalars -----------------------------------------------------------
+inline double fma_(double x, double y, double z) { return std::fma(x, y, z); }
+inline float fma_(float x, float y, float z) { return std::fma(x, y, z); }
+inline double sqrt_(double x) { return std::sqrt(x); }
+inline float sqrt_(float x) { return std::sqrt(x); }
+inline double tanh_(double x) { return std::tanh(x); }
+inline float tanh_(float x) { return std::tanh(x); }
+inline double val(double x) { return x; }
+inline float val(float x) { return x; }
+
+template <class S> struct base_of { using type = S; };
+template <class T> struct base_of<Rv<T>> { using type = T; };
+template <class T> struct base_of<Dv<T>> { using type = T; };
+template <> struct base_of<Cn> { using type = double; };
+
+// ---------------------------------------------------------------------------
+// Method constants.
+// ---------------------------------------------------------------------------
+enum { SYS_LORENZ = 1, SYS_ROBERTSON = 2, SYS_HIRES = 3, SYS_NODE64 = 4, SYS_LINEAR = 5 };
+enum { M_TSIT5 = 1, M_ROS2 = 2 };
+enum { DT_F32 = 1, DT_F64 = 2 };
+enum { LOSS_SUMSQ = 1, LOSS_LINEAR = 2 };
+enum { TRAJ_OK = 0, TRAJ_MAXSTEPS = 1, TRAJ_DTMIN = 2, TRAJ_NONFINITE = 3, TRAJ_SINGULAR = 4 };
+
+// Tsitouras (2011) 5(4) pair.  Row j of TS_A holds a_{j+1, m+1}; row 6 is the
+// propagating weight vector b (the method is FSAL: stage 7 is f(u_{n+1})).
+// TS_BT holds b - bhat, the weights of the embedded error estimate.
+static const double TS_C[7] = {0.0, 0.161, 0.327, 0.9, 0.9800255409045097, 1.0, 1.0};
+static const double TS_A[7][6] = {
+    {0, 0, 0, 0, 0, 0},
+    {0.161, 0, 0, 0, 0, 0},
+    {-0.008480655492356989, 0.335480655492357, 0, 0, 0, 0},
+    {2.897153057105493, -6.359448489975075, 4.3622954328695815, 0, 0, 0},
+    {5.325864828439257, -11.748883564062828, 7.4955393428898365, -0.09249506636175525, 0, 0},
+    {5.86145544294642, -12.92096931784711, 8.159367898576159, -0.071584973281401, -0.028269050394068383, 0},
+    {0.09646076681806523, 0.01, 0.4798896504144996, 1.379008574103742, -3.290069515436081, 2.324710524099774}};
+static const double TS_BT[7] = {-0.00178001105222577714, -0.0008164344596567469, 0.007880878010261995,
+                                -0.1447110071732629,     0.5823571654525552,     -0.45808210592918697,
+                                1.0 / 66.0};
+
+// ROS2 (Verwer et al. 1999): gamma = 1 + 1/sqrt(2), L-stable choice.
+static const double ROS2_GAMMA = 1.7071067811865475;  // 1 + 1/sqrt(2) rounded to double
+
+constexpr int DMAX = 64;
+
+// ---------------------------------------------------------------------------
+// Right-hand sides.  u: state (d), p: per-trajectory parameters (np),
+// W: shared weights (NODE64 only, row-major 64x64).
+// ---------------------------------------------------------------------------
+template <class S>
+void rhs(int sys, const S* u, const S* p, const S* W, S* out) {
+  if (sys == SYS_LORENZ) {
+    // du1 = sigma (u2 - u1); du2 = u1 (rho - u3) - u2; du3 = u1 u2 - beta u3
+    out[0] = p[0] * (u[1] - u[0]);
+    out[1] = fma_(u[0], p[1] - u[2], -u[1]);
+    out[2] = fma_(u[0], u[1], -(p[2] * u[2]));
+  } else if (sys == SYS_ROBERTSON) {
+    // rates r1 = k1 y1, r2 = k2 y2^2, r3 = k3 y2 y3
+    S r1 = p[0] * u[0];
+    S r2 = p[1] * (u[1] * u[1]);
+    S r3 = p[2] * (u[1] * u[2]);
+    out[0] = r3 - r1;
+    out[1] = (r1 - r3) - r2;
+    out[2] = r2;
+  } else if (sys == SYS_LINEAR) {
+    // scalar test equation u' = p u (pins only: closed forms exist)
+    out[0] = p[0] * u[0];
+  } else if (sys == SYS_NODE64) {
+    for (int r = 0; r < 64; ++r) {
+      S acc = p[r];
+      for (int c = 0; c < 64; ++c) acc = fma_(W[r * 64 + c], u[c], acc);
+      out[r] = tanh_(acc) - u[r];
+    }
+  }
+}
+
+// Analytic Jacobian df/du, row-major d x d (Rosenbrock path).
+template <class S>
+void jac(int sys, const S* u, const S* p, S* J) {
+  if (sys == SYS_ROBERTSON) {
+    S a = p[2] * u[2];           // k3 y3
+    S b = p[2] * u[1];           // k3 y2
+    S c = S(2) * (p[1] * u[1]);  // 2 k2 y2
+    J[0] = -p[0];
+    J[1] = a;
+    J[2] = b;
+    J[3] = p[0];
+    J[4] = -(a + c);
+    J[5] = -b;
+    J[6] = S(0);
+    J[7] = c;
+    J[8] = S(0);
+  } else if (sys == SYS_LINEAR) {
+    J[0] = p[0];
+  } else if (sys == SYS_LORENZ) {
+    J[0] = -p[0];
+    J[1] = p[0];
+    J[2] = S(0);
+    J[3] = p[1] - u[2];
+    J[4] = S(-1);
+    J[5] = -u[0];
+    J[6] = u[1];
+    J[7] = u[0];
+    J[8] = -p[2];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// One Tsit5 step of size h from u.  Stage j state: acc = a_j1 k1 + sum a_jm k_m
+// (an fma chain in increasing m), U_j = fma(h, acc, u).  u_new is stage 7.
+// If err != nullptr also returns the embedded error e = h * sum bt_j k_j.
+// ---------------------------------------------------------------------------
+template <class S>
+void tsit5_step(int sys, int d, const S* u, const S* p, const S* W, S h, S* unew, S* err) {
+  using T = typename base_of<S>::type;
+  S k[7][DMAX];
+  S U[DMAX];
+  rhs<S>(sys, u, p, W, k[0]);
+  for (int j = 1; j < 7; ++j) {
+    for (int c = 0; c < d; ++c) {
+      S acc = S(T(TS_A[j][0])) * k[0][c];
+      for (int m = 1; m < j; ++m) acc = fma_(S(T(TS_A[j][m])), k[m][c], acc);
+      U[c] = fma_(h, acc, u[c]);
+    }
+    if (j == 6) {
+      for (int c = 0; c < d; ++c) unew[c] = U[c];
+      if (!err) return;  // replay: the FSAL stage is the next step's first stage
+    }
+    rhs<S>(sys, U, p, W, k[j]);
+  }
+  for (int c = 0; c < d; ++c) {
+    S acc = S(T(TS_BT[0])) * k[0][c];
+    for (int m = 1; m < 7; ++m) acc = fma_(S(T(TS_BT[m])), k[m][c], acc);
+    err[c] = h * acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// LU with partial pivoting (largest |entry|, ties to the lowest row), Doolittle
+// right-looking order; multipliers stored below the diagonal.  Returns false on
+// an exactly zero or non-finite pivot.
+// ---------------------------------------------------------------------------
+template <class S>
+bool lu_factor(int d, S* M, int* P) {
+  using T = typename base_of<S>::type;
+  for (int i = 0; i < d; ++i) P[i] = i;
+  for (int k = 0; k < d; ++k) {
+    int piv = k;
+    for (int i = k + 1; i < d; ++i)
+      if (std::fabs(val(M[i * d + k])) > std::fabs(val(M[piv * d + k]))) piv = i;
+    if (piv != k) {
+      for (int j = 0; j < d; ++j) std::swap(M[k * d + j], M[piv * d + j]);
+      std::swap(P[k], P[piv]);
+    }
+    T pv = val(M[k * d + k]);
+    if (pv == T(0) || !std::isfinite(pv)) return false;
+    for (int i = k + 1; i < d; ++i) {
+      S l = M[i * d + k] / M[k * d + k];
+      M[i * d + k] = l;
+      for (int j = k + 1; j < d; ++j) M[i * d + j] = fma_(-l, M[k * d + j], M[i * d + j]);
+    }
+  }
+  return true;
+}
+
+template <class S>
+void lu_solve(int d, const S* LU, const int* P, const S* b, S* x) {
+  for (int i = 0; i < d; ++i) x[i] = b[P[i]];
+  for (int i = 1; i < d; ++i)
+    for (int j = 0; j < i; ++j) x[i] = fma_(-LU[i * d + j], x[j], x[i]);
+  for (int i = d - 1; i >= 0; --i) {
+    for (int j = i + 1; j < d; ++j) x[i] = fma_(-LU[i * d + j], x[j], x[i]);
+    x[i] = x[i] / LU[i * d + i];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// One ROS2 step (Verwer et al. 1999):
+//   M = I - gamma h J(u);  M k1 = f(u);  M k2 = f(u + h k1) - 2 k1;
+//   u_new = u + h (3/2 k1 + 1/2 k2);  error e = h/2 (k1 + k2)
+// (difference to the embedded first-order solution u + h k1).
+// Returns false when M is singular.
+// ---------------------------------------------------------------------------
+template <class S>
+bool ros2_step(int sys, int d, const S* u, const S* p, S h, S* unew, S* err) {
+  using T = typename base_of<S>::type;
+  S J[64];
+  S M[64];
+  int P[8];
+  jac<S>(sys, u, p, J);
+  S gh = S(T(ROS2_GAMMA)) * h;
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) M[i * d + j] = fma_(-gh, J[i * d + j], S(T(i == j ? 1 : 0)));
+  if (!lu_factor<S>(d, M, P)) return false;
+  S f0[8] = {}, k1[8] = {}, v[8] = {}, f1[8] = {}, r[8] = {}, k2[8] = {};
+  rhs<S>(sys, u, p, nullptr, f0);
+  lu_solve<S>(d, M, P, f0, k1);
+  for (int c = 0; c < d; ++c) v[c] = fma_(h, k1[c], u[c]);
+  rhs<S>(sys, v, p, nullptr, f1);
+  for (int c = 0; c < d; ++c) r[c] = fma_(S(T(-2)), k1[c], f1[c]);
+  lu_solve<S>(d, M, P, r, k2);
+  for (int c = 0; c < d; ++c) {
+    S acc = S(T(1.5)) * k1[c];
+    acc = fma_(S(T(0.5)), k2[c], acc);
+    unew[c] = fma_(h, acc, u[c]);
+  }
+  if (err)
+    for (int c = 0; c < d; ++c) err[c] = (h * S(T(0.5))) * (k1[c] + k2[c]);
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Adaptive recorder (plain scalar T).
+//
+// Error norm: err = sqrt( (1/d) sum_c (e_c / sc_c)^2 ), sc_c = atol + rtol *
+// max(|u_c|, |u_new_c|), accept iff err <= 1.  PI controller with error order
+// q (5 for Tsit5, 2 for ROS2): accepted -> fac = 0.9 err^(-0.7/q)
+// errprev^(0.4/q) clipped to [0.2, 10] (10 if err == 0), capped at 1 after a
+// rejection, errprev <- max(err, 1e-4); rejected -> fac = max(0.2, 0.9
+// err^(-1/q)) (0.2 if err is NaN).  The next proposal is fac * h_prop, where
+// h_prop is the unclipped proposal.  Steps are shortened to land exactly on
+// every save time and on t1; save_idx[k] is the number of accepted steps taken
+// when t reached tsave[k].  Starting step: Hairer, Norsett & Wanner I, II.4.
+// ---------------------------------------------------------------------------
+template <class T>
+struct RecordOut {
+  std::vector<T> h;
+  int nsteps = 0, nreject = 0, status = TRAJ_OK;
+  std::vector<int> save_idx;
+};
+
+template <class T>
+T rms_scaled(int d, const T* x, const T* sc) {
+  T s = 0;
+  for (int c = 0; c < d; ++c) {
+    T q = x[c] / sc[c];
+    s = std::fma(q, q, s);
+  }
+  return std::sqrt(s / T(d));
+}
+
+template <class T>
+T initial_step(int sys, int method, int d, const T* u0, const T* p, const T* W, T t0, T t1, T rtol,
+               T atol) {
+  T q = method == M_TSIT5 ? T(5) : T(2);
+  T sc[DMAX] = {}, f0[DMAX] = {}, u1[DMAX] = {}, f1[DMAX] = {}, df[DMAX] = {};
+  for (int c = 0; c < d; ++c) sc[c] = std::fma(rtol, std::fabs(u0[c]), atol);
+  rhs<T>(sys, u0, p, W, f0);
+  T d0 = rms_scaled<T>(d, u0, sc);
+  T d1 = rms_scaled<T>(d, f0, sc);
+  T h0 = (d0 < T(1e-5) || d1 < T(1e-5)) ? T(1e-6) : T(0.01) * (d0 / d1);
+  h0 = std::min(h0, t1 - t0);
+  for (int c = 0; c < d; ++c) u1[c] = std::fma(h0, f0[c], u0[c]);
+  rhs<T>(sys, u1, p, W, f1);
+  for (int c = 0; c < d; ++c) df[c] = f1[c] - f0[c];
+  T d2 = rms_scaled<T>(d, df, sc) / h0;
+  T dm = std::max(d1, d2);
+  T h1 = dm <= T(1e-15) ? std::max(T(1e-6), h0 * T(1e-3)) : std::pow(T(0.01) / dm, T(1) / q);
+  return std::min(std::min(T(100) * h0, h1), t1 - t0);
+}
+
+template <class T>
+RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, const T* W, T t0, T t1,
+                        int nsave, const T* tsave, T rtol, T atol, T h0user, int smax) {
+  RecordOut<T> out;
+  out.save_idx.assign(nsave, 0);
+  const T eps = std::numeric_limits<T>::epsilon();
+  const T q = method == M_TSIT5 ? T(5) : T(2);
+  T u[DMAX], un[DMAX], e[DMAX], sc[DMAX], f0[DMAX];
+  for (int c = 0; c < d; ++c) u[c] = u0[c];
+  rhs<T>(sys, u, p, W, f0);
+  for (int c = 0; c < d; ++c)
+    if (!std::isfinite(f0[c]) || !std::isfinite(u[c])) {
+      out.status = TRAJ_NONFINITE;
+      return out;
+    }
+  T hprop = h0user > T(0) ? h0user : initial_step<T>(sys, method, d, u0, p, W, t0, t1, rtol, atol);
+  if (!(hprop > T(0)) || !std::isfinite(hprop)) {
+    out.status = TRAJ_NONFINITE;
+    return out;
+  }
+  T t = t0, errprev = T(1);
+  bool prev_rej = false;
+  int kk = 0;
+  while (true) {
+    T tstop = kk < nsave ? tsave[kk] : t1;
+    if (hprop < T(16) * eps * std::fabs(t)) {
+      out.status = TRAJ_DTMIN;
+      return out;
+    }
+    // a step that would end at or within 4 eps of the next stop lands on it
+    T tn = t + hprop;
+    bool clipped = tn >= tstop - T(4) * eps * std::fabs(tstop);
+    T h = clipped ? tstop - t : hprop;
+    bool ok = method == M_TSIT5 ? (tsit5_step<T>(sys, d, u, p, W, h, un, e), true)
+                                : ros2_step<T>(sys, d, u, p, h, un, e);
+    if (!ok) {
+      out.status = TRAJ_SINGULAR;
+      return out;
+    }
+    for (int c = 0; c < d; ++c) sc[c] = std::fma(rtol, std::max(std::fabs(u[c]), std::fabs(un[c])), atol);
+    T err = rms_scaled<T>(d, e, sc);
+    if (err <= T(1)) {
+      if (out.nsteps >= smax) {
+        out.status = TRAJ_MAXSTEPS;
+        return out;
+      }
+      out.h.push_back(h);
+      out.nsteps++;
+      t = clipped ? tstop : tn;
+      for (int c = 0; c < d; ++c) u[c] = un[c];
+      while (kk < nsave && t == tsave[kk]) out.save_idx[kk++] = out.nsteps;
+      T fac;
+      if (err == T(0)) {
+        fac = T(10);
+      } else {
+        fac = (T(0.9) * std::pow(err, -T(0.7) / q)) * std::pow(errprev, T(0.4) / q);
+        fac = std::min(T(10), std::max(T(0.2), fac));
+      }
+      if (prev_rej) fac = std::min(fac, T(1));
+      errprev = std::max(err, T(1e-4));
+      prev_rej = false;
+      hprop = fac * hprop;
+      if (t >= t1) return out;  // the last step lands exactly on t1
+    } else {
+      out.nreject++;
+      if (out.nreject > smax) {
+        out.status = TRAJ_MAXSTEPS;
+        return out;
+      }
+      T fac = std::isnan(err) ? T(0.2) : std::max(T(0.2), T(0.9) * std::pow(err, -T(1) / q));
+      hprop = fac * hprop;
+      prev_rej = true;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fixed-step replay over a recorded mesh, returning the loss.
+//   SUMSQ:  L = sum_k sum_c (u_c(t_k) - target_kc)^2    (target NULL -> 0)
+//   LINEAR: L = sum_k sum_c w_kc u_c(t_k)
+// accumulated as an fma chain in (k, c) order.  The mesh h is data: no
+// derivative flows through it.
+// ---------------------------------------------------------------------------
+template <class S>
+S replay_loss(int sys, int method, int d, const S* u0, const S* p, const S* W, const double* h, int nsteps,
+              int nsave, const int* save_idx, int loss_kind, const double* tgt /*[nsave][d] or null*/,
+              const double* wgt /*[nsave][d]*/, S* u_save /*[nsave][d] or null*/) {
+  using T = typename base_of<S>::type;
+  S u[DMAX], un[DMAX];
+  for (int c = 0; c < d; ++c) u[c] = u0[c];
+  S L = S(T(0));
+  int kk = 0;
+  auto visit = [&](int s) {
+    while (kk < nsave && save_idx[kk] == s) {
+      for (int c = 0; c < d; ++c) {
+        if (u_save) u_save[kk * d + c] = u[c];
+        if (loss_kind == LOSS_SUMSQ) {
+          S dlt = tgt ? u[c] - S(T(tgt[kk * d + c])) : u[c];
+          L = fma_(dlt, dlt, L);
+        } else {
+          L = fma_(S(T(wgt[kk * d + c])), u[c], L);
+        }
+      }
+      kk++;
+    }
+  };
+  visit(0);
+  for (int s = 0; s < nsteps; ++s) {
+    S hs = S(T(h[s]));
+    if (method == M_TSIT5)
+      tsit5_step<S>(sys, d, u, p, W, hs, un, nullptr);
+    else
+      ros2_step<S>(sys, d, u, p, hs, un, nullptr);
+    for (int c = 0; c < d; ++c) u[c] = un[c];
+    visit(s + 1);
+  }
+  return L;
+}
+
+// ---------------------------------------------------------------------------
+// Problem description shared by the entry points below.
+// ---------------------------------------------------------------------------
+struct Prob {
+  int sys, method, dtype, d, np;
+  int64_t n;
+  const double *p, *u0, *W;  // [np][n], [d][n], [64*64]
+};
+
+struct Mesh {
+  int smax, nsave;
+  const double* h;      // [n][smax]
+  const int* nsteps;    // [n]
+  const int* save_idx;  // [n][nsave]
+};
+
+struct Loss {
+  int kind;
+  const double *target, *weight;  // [nsave][d][n] each (target may be null)
+};
+
+template <class F>
+void parallel_for(int64_t n, int nthreads, F fn) {
+  if (nthreads <= 1 || n < 2) {
+    fn(0, (int64_t)0, n);
+    return;
+  }
+  nthreads = (int)std::min<int64_t>(nthreads, n);
+  std::vector<std::thread> th;
+  int64_t chunk = (n + nthreads - 1) / nthreads;
+  for (int t = 0; t < nthreads; ++t) {
+    int64_t a = t * chunk, b = std::min(n, a + chunk);
+    if (a >= b) break;
+    th.emplace_back([=] { fn(t, a, b); });
+  }
+  for (auto& x : th) x.join();
+}
+
+// Per-trajectory gathers of target/weight rows into [nsave][d].
+inline void gather_kd(const double* src, int nsave, int d, int64_t n, int64_t i, double* dst) {
+  for (int k = 0; k < nsave; ++k)
+    for (int c = 0; c < d; ++c) dst[k * d + c] = src[((int64_t)k * d + c) * n + i];
+}
+
+// Reverse-mode gradient of one trajectory with the tape.  Outputs: loss, dp
+// (np), du0 (d) and, for NODE64, accumulates dW (64*64) into dW_acc.
+template <class T>
+void grad_one_tape(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, double* loss, double* dp,
+                   double* du0, double* dW_acc) {
+  using R = Rv<T>;
+  auto& tp = tape<T>();
+  tp.nodes.clear();
+  int d = P.d, np = P.np;
+  std::vector<R> u0(d), p(np), W;
+  for (int c = 0; c < d; ++c) {
+    T v = T(P.u0[(int64_t)c * P.n + i]);
+    u0[c] = R(v, tp.push(v));
+  }
+  for (int c = 0; c < np; ++c) {
+    T v = T(P.p[(int64_t)c * P.n + i]);
+    p[c] = R(v, tp.push(v));
+  }
+  if (P.sys == SYS_NODE64) {
+    W.resize(64 * 64);
+    for (int c = 0; c < 64 * 64; ++c) {
+      T v = T(P.W[c]);
+      W[c] = R(v, tp.push(v));
+    }
+  }
+  std::vector<double> tg(Mh.nsave * d, 0.0), wg(Mh.nsave * d, 0.0);
+  if (Ls.target) gather_kd(Ls.target, Mh.nsave, d, P.n, i, tg.data());
+  if (Ls.weight) gather_kd(Ls.weight, Mh.nsave, d, P.n, i, wg.data());
+  R L = replay_loss<R>(P.sys, P.method, d, u0.data(), p.data(), W.empty() ? nullptr : W.data(),
+                       Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave, Mh.save_idx + i * Mh.nsave, Ls.kind,
+                       Ls.target ? tg.data() : nullptr, wg.data(), nullptr);
+  *loss = double(L.v);
+  std::vector<T> adj(tp.nodes.size(), T(0));
+  if (L.id >= 0) adj[L.id] = T(1);
+  for (int64_t k = (int64_t)tp.nodes.size() - 1; k >= 0; --k) {
+    const Node<T>& nd = tp.nodes[k];
+    T a = adj[k];
+    if (a == T(0)) continue;
+    if (nd.a >= 0) adj[nd.a] += nd.da * a;
+    if (nd.b >= 0) adj[nd.b] += nd.db * a;
+    if (nd.c >= 0) adj[nd.c] += nd.dc * a;
+  }
+  for (int c = 0; c < d; ++c) du0[c] = double(u0[c].id >= 0 ? adj[u0[c].id] : T(0));
+  for (int c = 0; c < np; ++c) dp[c] = double(p[c].id >= 0 ? adj[p[c].id] : T(0));
+  if (dW_acc)
+    for (int c = 0; c < 64 * 64; ++c) dW_acc[c] += double(adj[W[c].id]);
+}
+
+// Forward-mode directional derivative of one trajectory's loss along
+// (dir_p, dir_u0, dir_W).
+// dir_p_i[np], dir_u0_i[d]: this trajectory's direction (null = zero).
+template <class T>
+double dirderiv_one(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, const double* dir_p_i,
+                    const double* dir_u0_i, const double* dir_W) {
+  using D = Dv<T>;
+  int d = P.d, np = P.np;
+  std::vector<D> u0(d), p(np), W;
+  for (int c = 0; c < d; ++c) u0[c] = D(T(P.u0[(int64_t)c * P.n + i]), dir_u0_i ? T(dir_u0_i[c]) : T(0));
+  for (int c = 0; c < np; ++c) p[c] = D(T(P.p[(int64_t)c * P.n + i]), dir_p_i ? T(dir_p_i[c]) : T(0));
+  if (P.sys == SYS_NODE64) {
+    W.resize(64 * 64);
+    for (int c = 0; c < 64 * 64; ++c) W[c] = D(T(P.W[c]), dir_W ? T(dir_W[c]) : T(0));
+  }
+  std::vector<double> tg(Mh.nsave * d, 0.0), wg(Mh.nsave * d, 0.0);
+  if (Ls.target) gather_kd(Ls.target, Mh.nsave, d, P.n, i, tg.data());
+  if (Ls.weight) gather_kd(Ls.weight, Mh.nsave, d, P.n, i, wg.data());
+  D L = replay_loss<D>(P.sys, P.method, d, u0.data(), p.data(), W.empty() ? nullptr : W.data(),
+                       Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave, Mh.save_idx + i * Mh.nsave, Ls.kind,
+                       Ls.target ? tg.data() : nullptr, wg.data(), nullptr);
+  return double(L.d);
+}
+
+template <class T>
+double loss_one(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, double* u_save) {
+  int d = P.d, np = P.np;
+  std::vector<T> u0(d), p(np), W, us(Mh.nsave * d);
+  for (int c = 0; c < d; ++c) u0[c] = T(P.u0[(int64_t)c * P.n + i]);
+  for (int c = 0; c < np; ++c) p[c] = T(P.p[(int64_t)c * P.n + i]);
+  if (P.sys == SYS_NODE64) {
+    W.resize(64 * 64);
+    for (int c = 0; c < 64 * 64; ++c) W[c] = T(P.W[c]);
+  }
+  std::vector<double> tg(Mh.nsave * d, 0.0), wg(Mh.nsave * d, 0.0);
+  if (Ls.target) gather_kd(Ls.target, Mh.nsave, d, P.n, i, tg.data());
+  if (Ls.weight) gather_kd(Ls.weight, Mh.nsave, d, P.n, i, wg.data());
+  T L = replay_loss<T>(P.sys, P.method, d, u0.data(), p.data(), W.empty() ? nullptr : W.data(),
+                       Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave, Mh.save_idx + i * Mh.nsave, Ls.kind,
+                       Ls.target ? tg.data() : nullptr, wg.data(), us.data());
+  if (u_save)
+    for (int k = 0; k < Mh.nsave; ++k)
+      for (int c = 0; c < d; ++c) u_save[((int64_t)k * d + c) * P.n + i] = double(us[k * d + c]);
+  return double(L);
+}
+
+int check_prob(const Prob& P) {
+  if (P.n < 0) return -1;
+  if (P.sys == SYS_LORENZ && (P.d != 3 || P.np != 3)) return -1;
+  if (P.sys == SYS_ROBERTSON && (P.d != 3 || P.np != 3)) return -1;
+  if (P.sys == SYS_NODE64 && (P.d != 64 || P.np != 64 || !P.W)) return -1;
+  if (P.sys == SYS_HIRES) return -4;  // not built: equations not available here
+  if (P.sys == SYS_LINEAR && (P.d != 1 || P.np != 1)) return -1;
+  if (P.sys < 1 || P.sys > 5) return -1;
+  if (P.method != M_TSIT5 && P.method != M_ROS2) return -1;
+  if (P.method == M_ROS2 && P.d > 8) return -4;
+  if (P.method == M_ROS2 && P.sys == SYS_NODE64) return -4;
+  if (P.dtype != DT_F32 && P.dtype != DT_F64) return -1;
+  return 0;
+}
+
+}  // namespace orc
+
+using namespace orc;
+
+extern "C" {
+
+// Adaptive record.  Mesh outputs are trajectory-major: h[n][smax] (zero padded,
+// values widened to double), save_idx[n][nsave].
+int or_record(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
+              const double* W, double t0, double t1, int nsave, const double* tsave, double rtol, double atol,
+              double h0, int smax, double* h, int* nsteps, int* save_idx, int* status, int* nreject,
+              int nthreads) {
+  Prob P{sys, method, dtype, d, np, n, p, u0, W};
+  int rc = check_prob(P);
+  if (rc) return rc;
+  parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
+    auto run = [&](auto tag) {
+      using T = decltype(tag);
+      std::vector<T> uu(d), pp(np), WW, ts(nsave);
+      for (int k = 0; k < nsave; ++k) ts[k] = T(tsave[k]);
+      if (sys == SYS_NODE64) {
+        WW.resize(4096);
+        for (int c = 0; c < 4096; ++c) WW[c] = T(W[c]);
+      }
+      for (int64_t i = a; i < b; ++i) {
+        for (int c = 0; c < d; ++c) uu[c] = T(u0[(int64_t)c * n + i]);
+        for (int c = 0; c < np; ++c) pp[c] = T(p[(int64_t)c * n + i]);
+        RecordOut<T> r = record_one<T>(sys, method, d, uu.data(), pp.data(), WW.empty() ? nullptr : WW.data(),
+                                       T(t0), T(t1), nsave, ts.data(), T(rtol), T(atol), T(h0), smax);
+        nsteps[i] = r.nsteps;
+        status[i] = r.status;
+        nreject[i] = r.nreject;
+        for (int s = 0; s < smax; ++s) h[i * smax + s] = s < r.nsteps ? double(r.h[s]) : 0.0;
+        for (int k = 0; k < nsave; ++k) save_idx[i * nsave + k] = r.save_idx[k];
+      }
+    };
+    if (dtype == DT_F64) run(double(0)); else run(float(0));
+  });
+  return 0;
+}
+
+// Gradient of the replay loss.  mode 0: reverse-mode tape.  mode 1: forward
+// mode, one dual-number pass per input direction (p and u0 only; not NODE64).
+// Trajectories with status != 0 get NaN outputs.  dW (NODE64) is the sum over
+// trajectories, accumulated per thread chunk and then in chunk order.
+int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
+            const double* W, int smax, int nsave, const double* h, const int* nsteps, const int* save_idx,
+            const int* status, int loss_kind, const double* target, const double* weight, int mode,
+            double* loss, double* dp, double* du0, double* dW, int nthreads) {
+  Prob P{sys, method, dtype, d, np, n, p, u0, W};
+  int rc = check_prob(P);
+  if (rc) return rc;
+  if (mode == 1 && sys == SYS_NODE64) return -4;
+  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  Loss Ls{loss_kind, target, weight};
+  int nt = std::max(1, nthreads);
+  std::vector<std::vector<double>> dWp(sys == SYS_NODE64 ? nt : 0, std::vector<double>(4096, 0.0));
+  const double nan = std::numeric_limits<double>::quiet_NaN();
+  parallel_for(n, nt, [&](int tid, int64_t a, int64_t b) {
+    std::vector<double> gp(np), gu(d), e_p(np), e_u(d);
+    for (int64_t i = a; i < b; ++i) {
+      if (status && status[i] != 0) {
+        loss[i] = nan;
+        for (int c = 0; c < np; ++c) dp[(int64_t)c * n + i] = nan;
+        for (int c = 0; c < d; ++c) du0[(int64_t)c * n + i] = nan;
+        continue;
+      }
+      double L;
+      if (mode == 0) {
+        double* acc = sys == SYS_NODE64 ? dWp[tid].data() : nullptr;
+        if (dtype == DT_F64)
+          grad_one_tape<double>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
+        else
+          grad_one_tape<float>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
+      } else {
+        // unit directions: the basis vectors of p, then of u0
+        L = dtype == DT_F64 ? loss_one<double>(P, Mh, Ls, i, nullptr) : loss_one<float>(P, Mh, Ls, i, nullptr);
+        for (int c = 0; c < np + d; ++c) {
+          std::fill(e_p.begin(), e_p.end(), 0.0);
+          std::fill(e_u.begin(), e_u.end(), 0.0);
+          (c < np ? e_p[c] : e_u[c - np]) = 1.0;
+          double g = dtype == DT_F64 ? dirderiv_one<double>(P, Mh, Ls, i, e_p.data(), e_u.data(), nullptr)
+                                     : dirderiv_one<float>(P, Mh, Ls, i, e_p.data(), e_u.data(), nullptr);
+          (c < np ? gp[c] : gu[c - np]) = g;
+        }
+      }
+      loss[i] = L;
+      for (int c = 0; c < np; ++c) dp[(int64_t)c * n + i] = gp[c];
+      for (int c = 0; c < d; ++c) du0[(int64_t)c * n + i] = gu[c];
+    }
+  });
+  if (dW && sys == SYS_NODE64) {
+    for (int c = 0; c < 4096; ++c) dW[c] = 0.0;
+    for (int t = 0; t < nt; ++t)
+      for (int c = 0; c < 4096; ++c) dW[c] += dWp[t][c];
+  }
+  return 0;
+}
+
+// Forward-mode directional derivative of each trajectory's loss along the
+// given input directions (any may be null = zero).  out[n].
+int or_dirderiv(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
+                const double* W, int smax, int nsave, const double* h, const int* nsteps, const int* save_idx,
+                int loss_kind, const double* target, const double* weight, const double* dir_p,
+                const double* dir_u0, const double* dir_W, double* out, int nthreads) {
+  Prob P{sys, method, dtype, d, np, n, p, u0, W};
+  int rc = check_prob(P);
+  if (rc) return rc;
+  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  Loss Ls{loss_kind, target, weight};
+  parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
+    std::vector<double> dpi(np, 0.0), dui(d, 0.0);
+    for (int64_t i = a; i < b; ++i) {
+      for (int c = 0; c < np; ++c) dpi[c] = dir_p ? dir_p[(int64_t)c * n + i] : 0.0;
+      for (int c = 0; c < d; ++c) dui[c] = dir_u0 ? dir_u0[(int64_t)c * n + i] : 0.0;
+      out[i] = dtype == DT_F64 ? dirderiv_one<double>(P, Mh, Ls, i, dpi.data(), dui.data(), dir_W)
+                               : dirderiv_one<float>(P, Mh, Ls, i, dpi.data(), dui.data(), dir_W);
+    }
+  });
+  return 0;
+}
+
+// Plain replay: loss[n] and, if u_save != null, the states at the save
+// points, u_save[nsave][d][n].
+int or_replay(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
+              const double* W, int smax, int nsave, const double* h, const int* nsteps, const int* save_idx,
+              int loss_kind, const double* target, const double* weight, double* loss, double* u_save,
+              int nthreads) {
+  Prob P{sys, method, dtype, d, np, n, p, u0, W};
+  int rc = check_prob(P);
+  if (rc) return rc;
+  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  Loss Ls{loss_kind, target, weight};
+  parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
+    for (int64_t i = a; i < b; ++i)
+      loss[i] = dtype == DT_F64 ? loss_one<double>(P, Mh, Ls, i, u_save) : loss_one<float>(P, Mh, Ls, i, u_save);
+  });
+  return 0;
+}
+
+// Operation counts of one fixed step of the given system/method, for the
+// roofline's algorithmic-work figure: out = {add, mul, fma, div, sqrt, tanh}.
+int or_count_step(int sys, int method, int d, int np, double* out6) {
+  std::vector<Cn> u(d, Cn(0.5)), p(np, Cn(1.0)), un(d), W;
+  if (sys == SYS_NODE64) W.assign(4096, Cn(0.01));
+  opcount() = OpCount();
+  Cn h(0.01);
+  if (method == M_TSIT5)
+    tsit5_step<Cn>(sys, d, u.data(), p.data(), W.empty() ? nullptr : W.data(), h, un.data(), nullptr);
+  else
+    ros2_step<Cn>(sys, d, u.data(), p.data(), h, un.data(), nullptr);
+  OpCount c = opcount();
+  out6[0] = double(c.add);
+  out6[1] = double(c.mul);
+  out6[2] = double(c.fma);
+  out6[3] = double(c.div);
+  out6[4] = double(c.sqrt);
+  out6[5] = double(c.tanh);
+  return 0;
+}
+
+// Low-level access for pins: one step of the method in double or float.
+int or_step(int sys, int method, int dtype, int d, const double* u, const double* p, const double* W, double h,
+            double* unew, double* err) {
+  auto run = [&](auto tag) {
+    using T = decltype(tag);
+    std::vector<T> uu(d), pp(64), WW, un(d), e(d);
+    for (int c = 0; c < d; ++c) uu[c] = T(u[c]);
+    for (int c = 0; c < 64; ++c) pp[c] = p ? T(p[c]) : T(0);
+    if (W) {
+      WW.resize(4096);
+      for (int c = 0; c < 4096; ++c) WW[c] = T(W[c]);
+    }
+    bool ok = method == M_TSIT5
+                  ? (tsit5_step<T>(sys, d, uu.data(), pp.data(), WW.empty() ? nullptr : WW.data(), T(h), un.data(), e.data()), true)
+                  : ros2_step<T>(sys, d, uu.data(), pp.data(), T(h), un.data(), e.data());
+    for (int c = 0; c < d; ++c) {
+      unew[c] = double(un[c]);
+      if (err) err[c] = double(e[c]);
+    }
+    return ok ? 0 : 4;
+  };
+  return dtype == DT_F64 ? run(double(0)) : run(float(0));
+}
+
+// The right-hand side and its analytic Jacobian at one point (double).
+int or_rhs(int sys, int d, const double* u, const double* p, const double* W, double* f, double* J) {
+  (void)d;
+  rhs<double>(sys, u, p, W, f);
+  if (J) jac<double>(sys, u, p, J);
+  return 0;
+}
+
+// Tableau export for the order-condition pins: c[7], A[7][6], bt[7].
+void or_tsit5_tableau(double* c, double* A, double* bt) {
+  for (int i = 0; i < 7; ++i) {
+    c[i] = TS_C[i];
+    bt[i] = TS_BT[i];
+    for (int j = 0; j < 6; ++j) A[i * 6 + j] = TS_A[i][j];
+  }
+}
+
+double or_ros2_gamma(void) { return ROS2_GAMMA; }
+
+}  // extern "C"

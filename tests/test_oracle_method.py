@@ -1,0 +1,222 @@
+"""Pins of the oracle's integrators against facts fixed outside the oracle.
+
+* Tsit5 tableau: the Runge-Kutta order conditions (order 5 for the
+  propagating weights, order 4 for the embedded weights b - bt, c = A 1).
+* Fixed-step Tsit5 derivative: the gradient printed by the DiffEqGPU
+  documentation ("Enzyme reverse mode with EnsembleGPUKernel") for u' = p u,
+  20 steps of 0.05 (tests/golden/diffeqgpu_enzyme_tsit5.txt).
+* Discrete adjoint on u' = -lambda u: the closed form built from the method's
+  stability function R(z) on the mesh (GRADSOLVE's exactness definition: the
+  derivative of the fixed-step replay with the mesh held fixed), evaluated in
+  exact rational arithmetic.
+* ROS2: L-stability (R(inf) = 0 for gamma = 1 + 1/sqrt 2), second order
+  (R(z) = 1 + z + z^2/2 + O(z^3)), and the same closed-form adjoint.
+"""
+import os
+from fractions import Fraction as Fr
+from math import factorial
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+EPS = np.finfo(np.float64).eps
+
+
+def _tab():
+    c, A, bt = oracle.tsit5_tableau()
+    b = A[6].copy()                      # propagating weights (FSAL row)
+    A6 = np.zeros((7, 7))
+    A6[:, :6] = A
+    b7 = np.append(b, 0.0)
+    return c, A6, b7, bt
+
+
+def test_tsit5_row_sums():
+    c, A, b, bt = _tab()
+    assert np.max(np.abs(A.sum(1) - c)) <= 4 * EPS
+
+
+# Butcher order conditions written as (tree functional, 1/gamma(tree)).
+def _conditions(A, c, w, order):
+    e = np.ones(len(c))
+    conds = [(w @ e, 1.0)]
+    if order >= 2:
+        conds += [(w @ c, 1 / 2)]
+    if order >= 3:
+        conds += [(w @ c**2, 1 / 3), (w @ (A @ c), 1 / 6)]
+    if order >= 4:
+        conds += [(w @ c**3, 1 / 4), (w @ (c * (A @ c)), 1 / 8), (w @ (A @ c**2), 1 / 12),
+                  (w @ (A @ (A @ c)), 1 / 24)]
+    if order >= 5:
+        conds += [(w @ c**4, 1 / 5), (w @ (c**2 * (A @ c)), 1 / 10), (w @ ((A @ c) ** 2), 1 / 20),
+                  (w @ (c * (A @ c**2)), 1 / 15), (w @ (c * (A @ (A @ c))), 1 / 30),
+                  (w @ (A @ c**3), 1 / 20), (w @ (A @ (c * (A @ c))), 1 / 40),
+                  (w @ (A @ (A @ c**2)), 1 / 60), (w @ (A @ (A @ (A @ c))), 1 / 120)]
+    return conds
+
+
+def test_tsit5_order_conditions():
+    c, A, b, bt = _tab()
+    res5 = [abs(v - t) for v, t in _conditions(A, c, b, 5)]
+    assert len(res5) == 17 and max(res5) <= 8 * EPS
+    bhat = b - bt
+    res4 = [abs(v - t) for v, t in _conditions(A, c, bhat, 4)]
+    assert len(res4) == 8 and max(res4) <= 8 * EPS
+    # the pair really is 5(4): the embedded weights fail a fifth-order condition
+    assert max(abs(v - t) for v, t in _conditions(A, c, bhat, 5)[8:]) > 1e-4
+
+
+def _golden():
+    rows = []
+    with open(os.path.join(GOLD, "diffeqgpu_enzyme_tsit5.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append([float(x) for x in line.split()])
+    return np.array(rows)
+
+
+def _uniform_mesh(n, nsteps, h):
+    return oracle.Mesh(np.full((n, nsteps), h), np.full(n, nsteps, np.int32),
+                       np.full((n, 1), nsteps, np.int32), np.zeros(n, np.int32), np.zeros(n, np.int32))
+
+
+@pytest.mark.parametrize("mode", ["tape", "dual"])
+def test_worked_example_fixed_step_tsit5(mode):
+    g = _golden()
+    prob = W.scalar_linear(g[:, 0])
+    out = oracle.grad(prob, _uniform_mesh(prob.n, 20, 0.05), mode=mode, nthreads=1)
+    rel = np.abs(out["dp"][0] - g[:, 1]) / np.abs(g[:, 1])
+    # both codes round differently inside the 20 steps; the printed values
+    # differ from exp(p) by 2.6e-14 / 2.1e-13, so 2e-15 pins the DISCRETE derivative
+    assert rel.max() <= 2e-15, rel
+    assert np.abs(out["dp"][0] - np.exp(g[:, 0])).max() > 1e-14
+
+
+# ---- closed-form discrete adjoint on u' = p u (p = -lambda) ------------------
+def _tsit5_R_coeffs():
+    """R(z) = sum_k beta_k z^k: exp's Taylor coefficients up to z^5 (a
+    fifth-order method), plus beta_6 = b6 a65 a54 a43 a32 a21 (the only path
+    through the strictly lower triangular A), from the exact binary doubles."""
+    c, A, b, bt = _tab()
+    beta = [Fr(1, factorial(k)) for k in range(6)]
+    g6 = Fr(b[5])
+    for j in range(5, 0, -1):
+        g6 *= Fr(A[j, j - 1])
+    return beta + [g6]
+
+
+def _poly(coeffs, z):
+    acc = Fr(0)
+    for a in reversed(coeffs):
+        acc = acc * z + a
+    return acc
+
+
+def _dpoly(coeffs, z):
+    return _poly([k * a for k, a in enumerate(coeffs)][1:], z)
+
+
+def _ros2_R(z, g):
+    num = 1 + (1 - 2 * g) * z + (g * g - 2 * g + Fr(1, 2)) * z * z
+    den = (1 - g * z) ** 2
+    dnum = (1 - 2 * g) + 2 * (g * g - 2 * g + Fr(1, 2)) * z
+    dden = -2 * g * (1 - g * z)
+    return num / den, (dnum * den - num * dden) / (den * den)
+
+
+def _closed_form(method, p, hs, u0=Fr(1)):
+    """u_N = u0 prod R(z_n), z_n = p h_n; L = u_N^2.
+    dL/du0 = 2 u_N prod R(z_n);  dL/dp = 2 u_N^2 sum_n h_n R'(z_n)/R(z_n)."""
+    pf = Fr(p)
+    R, dR = [], []
+    if method == "tsit5":
+        co = _tsit5_R_coeffs()
+        for h in hs:
+            z = pf * Fr(h)
+            R.append(_poly(co, z))
+            dR.append(_dpoly(co, z))
+    else:
+        g = Fr(oracle.ros2_gamma())
+        for h in hs:
+            r, dr = _ros2_R(pf * Fr(h), g)
+            R.append(r)
+            dR.append(dr)
+    prod = Fr(1)
+    for r in R:
+        prod *= r
+    uN = u0 * prod
+    L = uN * uN
+    dL_du0 = 2 * uN * prod
+    dL_dp = 2 * L * sum(Fr(h) * dr / r for h, r, dr in zip(hs, R, dR))
+    return float(L), float(dL_du0), float(dL_dp)
+
+
+def _kappa(method, p, hs):
+    worst = 1.0
+    g = oracle.ros2_gamma()
+    co = [float(x) for x in _tsit5_R_coeffs()]
+    for h in hs:
+        z = p * h
+        if method == "tsit5":
+            terms = sum(abs(a) * abs(z) ** k for k, a in enumerate(co))
+            R = sum(a * z**k for k, a in enumerate(co))
+        else:
+            d = 1 - g * z
+            terms = 1 + 1.5 * abs(z / d) + 0.5 * abs(z * (z * (1 - g) - 1) / d**2)
+            R = (1 + (1 - 2 * g) * z + (g * g - 2 * g + 0.5) * z * z) / d**2
+        worst = max(worst, terms / abs(R))
+    return worst
+
+
+@pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 1e4])])
+@pytest.mark.parametrize("mode", ["tape", "dual"])
+def test_closed_form_decay_adjoint(method, lams, mode):
+    rng = np.random.default_rng(7)
+    N = 25
+    hs = rng.uniform(0.005, 0.06, N)
+    prob = W.scalar_linear([-l for l in lams], t1=float(hs.sum()), method=method)
+    prob.loss = "sumsq"
+    prob.weight = None
+    n = prob.n
+    mesh = oracle.Mesh(np.tile(hs, (n, 1)), np.full(n, N, np.int32), np.full((n, 1), N, np.int32),
+                       np.zeros(n, np.int32), np.zeros(n, np.int32))
+    out = oracle.grad(prob, mesh, mode=mode, nthreads=1)
+    for i, lam in enumerate(lams):
+        L, gu, gp = _closed_form(method, -lam, hs)
+        # Rounding bound: a step's relative rounding error is about eps times
+        # its cancellation factor kappa(z) = (sum of |terms|) / |R(z)| times the
+        # size of the method's inner weights (Tsit5: |a_6m| up to ~13, so 32;
+        # ROS2: 3/2, 1/2, 2 and gamma, so 8), summed over the N steps.  A
+        # wrong digit or a dropped term moves these numbers by 1e-8 or more.
+        tol = N * EPS * _kappa(method, -lam, hs) * (32 if method == "tsit5" else 8)
+        assert abs(out["loss"][i] - L) <= tol * abs(L)
+        assert abs(out["du0"][0, i] - gu) <= tol * abs(gu)
+        assert abs(out["dp"][0, i] - gp) <= tol * abs(gp), (method, lam, out["dp"][0, i], gp)
+
+
+def test_ros2_stability_function_facts():
+    """The ROS2 closed form itself: L-stable (R -> 0 at infinity) and second
+    order (Taylor coefficients 1, 1, 1/2), so a slip in the form used above
+    would show here."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 50
+    g = 1 + 1 / Decimal(2).sqrt()
+    gf = Fr(str(g))
+    r_big, _ = _ros2_R(Fr(-10**30), gf)
+    assert abs(float(r_big)) < 1e-25
+    eps = Fr(1, 10**6)
+    r, _ = _ros2_R(eps, gf)
+    assert abs(float((r - 1 - eps - eps * eps / 2) / eps**3)) < 10.0
+    # the oracle's gamma is 1 + 1/sqrt(2) to the double's precision
+    assert abs(Decimal(oracle.ros2_gamma()) - g) < Decimal(2e-16)
+
+
+def test_ros2_step_matches_stability_function():
+    for lam, h in [(0.7, 0.1), (1e3, 0.05), (3.0, 2.0)]:
+        un, _, ok = oracle.step("linear", "ros2", "f64", [1.0], [-lam], h)
+        r, _ = _ros2_R(Fr(-lam) * Fr(h), Fr(oracle.ros2_gamma()))
+        assert ok and abs(un[0] - float(r)) <= 8 * EPS * max(1.0, abs(float(r)))

@@ -1,0 +1,135 @@
+"""Pins of the oracle's adaptive recorder, right-hand sides and op counts.
+
+The pages print no controller, tableau or mesh, so the recorder's parity is
+pinned by self-consistency and by accuracy against independent solvers:
+steps sum to the interval and land on the save times, every accepted step
+passes its own error test, the solution meets a tight tolerance against a
+high-accuracy scipy solution, the integrators converge at their orders,
+Robertson's linear invariant is kept, the step-count spread is in the range
+the GRADSOLVE review reports (Table 5: max/mean 1.33-1.34), and the failure
+statuses fire.
+"""
+import numpy as np
+import pytest
+from scipy.integrate import solve_ivp
+
+import oracle
+import workloads as W
+
+EPS = np.finfo(float).eps
+
+
+def _err_norm(e, u, un, rtol, atol):
+    sc = atol + rtol * np.maximum(np.abs(u), np.abs(un))
+    return np.sqrt(np.mean((e / sc) ** 2))
+
+
+@pytest.mark.parametrize("name", ["lorenz_small", "lorenz_1m", "robertson"])
+def test_mesh_consistency(name):
+    prob = W.by_name(name, n=6)
+    mesh = oracle.record(prob, 20000)
+    assert (mesh.status == 0).all()
+    for i in range(prob.n):
+        S = mesh.nsteps[i]
+        h = mesh.h[i, :S]
+        assert (h > 0).all() and (mesh.h[i, S:] == 0).all()
+        t = np.cumsum(h)
+        assert abs(t[-1] - (prob.t1 - prob.t0)) <= S * EPS * prob.t1
+        for k, ts in enumerate(prob.tsave):
+            assert abs(t[mesh.save_idx[i, k] - 1] - ts) <= S * EPS * prob.t1
+        # every recorded step passes the error test it was accepted on
+        u = prob.u0[:, i].copy()
+        for s in range(S):
+            un, e, ok = oracle.step(prob.system, prob.method, "f64", u, prob.p[:, i], h[s])
+            assert ok
+            assert _err_norm(e, u, un, prob.rtol, prob.atol) <= 1.0
+            u = un
+
+
+def _lorenz(t, u, s, r, b):
+    return [s * (u[1] - u[0]), u[0] * (r - u[2]) - u[1], u[0] * u[1] - b * u[2]]
+
+
+def test_tight_tolerance_solution_matches_scipy():
+    prob = W.lorenz_small(4)
+    prob.rtol = prob.atol = 1e-10
+    mesh = oracle.record(prob, 4000)
+    _, us = oracle.replay(prob, mesh)
+    for i in range(prob.n):
+        ref = solve_ivp(_lorenz, (0.0, 1.0), prob.u0[:, i], method="DOP853", rtol=1e-13, atol=1e-13,
+                        args=tuple(prob.p[:, i]))
+        err = np.abs(us[0, :, i] - ref.y[:, -1]).max() / np.abs(ref.y[:, -1]).max()
+        assert err <= 1e-7, err
+
+
+@pytest.mark.parametrize("method,order", [("tsit5", 5), ("ros2", 2)])
+def test_convergence_order(method, order):
+    prob = W.lorenz_small(1)
+    prob.method = method
+    T = 0.4
+
+    def solve(N):
+        m = oracle.Mesh(np.full((1, N), T / N), np.array([N], np.int32), np.array([[N]], np.int32),
+                        np.zeros(1, np.int32), np.zeros(1, np.int32))
+        return oracle.replay(prob, m)[1][0, :, 0]
+
+    ref = solve(4096 if method == "ros2" else 1024)
+    e1 = np.abs(solve(32) - ref).max()
+    e2 = np.abs(solve(64) - ref).max()
+    rate = np.log2(e1 / e2)
+    assert abs(rate - order) < 0.35, rate
+
+
+def test_robertson_keeps_total_mass():
+    prob = W.robertson(8)
+    mesh = oracle.record(prob, 20000)
+    _, us = oracle.replay(prob, mesh)
+    # the rates cancel in y1' + y2' + y3' and both ROS2 stages are linear in f
+    assert np.abs(us[0].sum(0) - 1.0).max() <= 1e-12
+
+
+def test_step_count_spread_matches_review_range():
+    prob = W.lorenz_1m(256)
+    mesh = oracle.record(prob, 2048)
+    r = mesh.nsteps.max() / mesh.nsteps.mean()
+    assert 1.15 <= r <= 1.6, r
+
+
+def test_failure_statuses():
+    prob = W.lorenz_small(3)
+    assert (oracle.record(prob, 20).status == 1).all()           # capacity -> MAXSTEPS
+    bad = prob.subset(range(3))
+    bad.p = bad.p.copy()
+    bad.p[0, 1] = np.nan
+    st = oracle.record(bad, 512).status
+    assert st[1] == 3 and st[0] == 0 and st[2] == 0               # NaN input -> NONFINITE
+    tight = prob.subset(range(1))
+    tight.rtol = tight.atol = 1e-100
+    assert oracle.record(tight, 1000).status[0] in (1, 2)         # unreachable tol -> DTMIN / cap
+
+
+@pytest.mark.parametrize("system", ["lorenz", "robertson"])
+def test_jacobian_matches_differences(system):
+    rng = np.random.default_rng(5)
+    u = rng.uniform(0.1, 2.0, 3) if system == "lorenz" else np.array([0.9, 2e-5, 0.1])
+    p = np.array([10.0, 28.0, 8 / 3]) if system == "lorenz" else np.array([0.04, 3e7, 1e4])
+    _, J = oracle.rhs(system, u, p)
+    for j in range(3):
+        e = 1e-6 * max(abs(u[j]), 1e-4)
+        fp, _ = oracle.rhs(system, u + e * np.eye(3)[j], p)
+        fm, _ = oracle.rhs(system, u - e * np.eye(3)[j], p)
+        col = (fp - fm) / (2 * e)
+        assert np.abs(col - J[:, j]).max() <= 1e-6 * max(1.0, np.abs(J).max())
+
+
+def test_step_operation_counts():
+    """The per-step work the roofline counts (fma = 2 flops, the rest 1)."""
+    c = oracle.count_step("lorenz", "tsit5", 3, 3)
+    # 6 rhs evaluations x (2 add, 2 mul, 2 fma); stage sums of rows 2..7:
+    # per component sum_{j=1..6} (1 mul + j fma)
+    assert c == {"add": 12, "mul": 12 + 18, "fma": 12 + 63, "div": 0, "sqrt": 0, "tanh": 0}
+    assert c["add"] + c["mul"] + 2 * c["fma"] == 192
+    r = oracle.count_step("robertson", "ros2", 3, 3)
+    assert r == {"add": 7, "mul": 18, "fma": 38, "div": 9, "sqrt": 0, "tanh": 0}
+    nd = oracle.count_step("node64", "tsit5", 64, 64)
+    assert nd["fma"] == 6 * 64 * 64 + 64 * 21 and nd["tanh"] == 6 * 64
