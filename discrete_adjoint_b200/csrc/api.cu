@@ -1,0 +1,148 @@
+// api.cu -- the C ABI of libgradsolve: argument validation, workspace sizing
+// and dispatch to the kernels.  Nothing here allocates device memory; every
+// device buffer is the caller's (see include/gradsolve.h).
+#include <atomic>
+#include <cmath>
+
+#include "common.cuh"
+
+namespace gs {
+
+static std::atomic<int64_t> g_launches{0};
+void count_launch(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+
+// kernels (defined in the other translation units)
+gs_status count3(const gs_problem*, const gs_tol*, int32_t, int32_t*, int32_t*, cudaStream_t);
+gs_status record3(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
+size_t record_ws_bytes(int64_t n, int32_t smax);
+template <typename T>
+gs_status launch_grad_tsit5_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
+                                   cudaStream_t);
+template <typename T>
+gs_status launch_grad_ros2(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
+                           cudaStream_t);
+template <typename T>
+gs_status launch_solve3(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
+
+static size_t dsize(const gs_problem* P) { return P->dtype == GS_F64 ? 8 : 4; }
+
+static gs_status check_problem(const gs_problem* P) {
+  if (!P) return GS_EINVAL;
+  if (P->n < 0 || P->n > (int64_t)INT32_MAX) return GS_EINVAL;
+  if (P->dtype != GS_F32 && P->dtype != GS_F64) return GS_EINVAL;
+  if (P->method != GS_TSIT5 && P->method != GS_ROS2) return GS_EINVAL;
+  switch (P->system) {
+    case GS_LORENZ:
+    case GS_ROBERTSON:
+      if (P->d != 3 || P->np != 3) return GS_EINVAL;
+      break;
+    case GS_NODE64:
+      if (P->d != 64 || P->np != 64) return GS_EINVAL;
+      if (P->n > 0 && !P->shared) return GS_EINVAL;
+      return GS_EUNSUPPORTED;
+    case GS_HIRES:
+      return GS_EUNSUPPORTED;
+    default:
+      return GS_EINVAL;
+  }
+  if (P->n > 0 && (!P->p || !P->u0)) return GS_EINVAL;
+  if (!std::isfinite(P->t0) || !std::isfinite(P->t1) || !(P->t0 < P->t1)) return GS_EINVAL;
+  if (P->nsave < 1 || P->nsave > GS_MAX_SAVE || !P->tsave) return GS_EINVAL;
+  double prev = P->t0;
+  for (int k = 0; k < P->nsave; ++k) {
+    const double t = P->tsave[k];
+    if (!(t > prev) || !(t <= P->t1)) return GS_EINVAL;
+    prev = t;
+  }
+  return GS_OK;
+}
+
+static gs_status check_mesh(const gs_problem* P, const gs_mesh* M) {
+  if (!M) return GS_EINVAL;
+  if (M->smax < 1 || M->nsave != P->nsave) return GS_EINVAL;
+  if (P->n > 0 && (!M->h || !M->order || !M->nsteps || !M->save_idx || !M->status)) return GS_EINVAL;
+  return GS_OK;
+}
+
+}  // namespace gs
+
+using namespace gs;
+
+extern "C" {
+
+const char* gs_status_string(gs_status s) {
+  switch (s) {
+    case GS_OK: return "ok";
+    case GS_EINVAL: return "invalid argument";
+    case GS_ECUDA: return "CUDA error";
+    case GS_EWORKSPACE: return "workspace missing or too small";
+    case GS_EUNSUPPORTED: return "unsupported system/method/dtype combination";
+    default: return "unknown status";
+  }
+}
+
+int64_t gs_launch_count(void) { return g_launches.load(); }
+
+size_t gs_workspace_bytes(const gs_problem* P, const gs_mesh* M, int32_t op) {
+  if (check_problem(P) != GS_OK || !M || M->smax < 1) return 0;
+  if (op == GS_OP_RECORD) return record_ws_bytes(P->n, M->smax);
+  if (op == GS_OP_GRAD) return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
+  return 0;
+}
+
+gs_status gs_count(const gs_problem* P, const gs_tol* tol, int32_t smax, int32_t* nsteps, int32_t* status,
+                   void* stream) {
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0) ||
+      smax < 1)
+    return GS_EINVAL;
+  if (P->n == 0) return GS_OK;
+  if (!nsteps) return GS_EINVAL;
+  return count3(P, tol, smax, nsteps, status, (cudaStream_t)stream);
+}
+
+gs_status gs_record(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, size_t ws_bytes,
+                    void* stream) {
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if ((rc = check_mesh(P, M)) != GS_OK) return rc;
+  if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0))
+    return GS_EINVAL;
+  if (P->n == 0) return GS_OK;
+  if (!ws || ws_bytes < gs_workspace_bytes(P, M, GS_OP_RECORD)) return GS_EWORKSPACE;
+  return record3(P, tol, M, ws, (cudaStream_t)stream);
+}
+
+gs_status gs_solve(const gs_problem* P, const gs_mesh* M, void* u_save, void* stream) {
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if ((rc = check_mesh(P, M)) != GS_OK) return rc;
+  if (P->n == 0) return GS_OK;
+  if (!u_save) return GS_EINVAL;
+  return P->dtype == GS_F64 ? launch_solve3<double>(P, M, u_save, (cudaStream_t)stream)
+                            : launch_solve3<float>(P, M, u_save, (cudaStream_t)stream);
+}
+
+gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp, void* du0,
+                  void* dshared, void* ws, size_t ws_bytes, void* stream) {
+  (void)dshared;
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if ((rc = check_mesh(P, M)) != GS_OK) return rc;
+  if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
+  if (P->n == 0) return GS_OK;
+  if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;
+  if (!loss || !dp || !du0) return GS_EINVAL;
+  if (!ws || ws_bytes < gs_workspace_bytes(P, M, GS_OP_GRAD)) return GS_EWORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (P->method == GS_TSIT5 && P->system == GS_LORENZ)
+    return P->dtype == GS_F64 ? launch_grad_tsit5_lorenz<double>(P, M, Ls, loss, dp, du0, ws, st)
+                              : launch_grad_tsit5_lorenz<float>(P, M, Ls, loss, dp, du0, ws, st);
+  if (P->method == GS_ROS2)
+    return P->dtype == GS_F64 ? launch_grad_ros2<double>(P, M, Ls, loss, dp, du0, ws, st)
+                              : launch_grad_ros2<float>(P, M, Ls, loss, dp, du0, ws, st);
+  return GS_EUNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,200 @@
+// common.cuh -- device-side building blocks shared by the kernels of
+// libgradsolve: method constants, registered right-hand sides, the step
+// formulas of the forward replay, and the host-side launch bookkeeping.
+//
+// Floating-point contract.  The forward arithmetic of every step (stage
+// sums, right-hand sides, Rosenbrock LU and solves, error norm, loss) follows
+// one fixed operation order with explicit fused multiply-adds; this library
+// is compiled with -fmad=false so that no other multiply-add is fused.  A
+// replay is then bitwise reproducible by any IEEE implementation that keeps
+// the same order, which is what lets a chaotic 10-time-unit Lorenz replay be
+// checked to 1e-12.  The reverse sweep uses fused multiply-adds freely.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gradsolve.h"
+
+namespace gs {
+
+// ---------------------------------------------------------------------------
+// Tsitouras (2011) 5(4) pair.  TS_Ajm: stage j's weight on slope m; row 7 is
+// the propagating weight vector b (FSAL).  TS_Ej = b_j - bhat_j, the weights of
+// the embedded error estimate.
+// ---------------------------------------------------------------------------
+#define TS_A21 0.161
+#define TS_A31 (-0.008480655492356989)
+#define TS_A32 0.335480655492357
+#define TS_A41 2.897153057105493
+#define TS_A42 (-6.359448489975075)
+#define TS_A43 4.3622954328695815
+#define TS_A51 5.325864828439257
+#define TS_A52 (-11.748883564062828)
+#define TS_A53 7.4955393428898365
+#define TS_A54 (-0.09249506636175525)
+#define TS_A61 5.86145544294642
+#define TS_A62 (-12.92096931784711)
+#define TS_A63 8.159367898576159
+#define TS_A64 (-0.071584973281401)
+#define TS_A65 (-0.028269050394068383)
+#define TS_B1 0.09646076681806523
+#define TS_B2 0.01
+#define TS_B3 0.4798896504144996
+#define TS_B4 1.379008574103742
+#define TS_B5 (-3.290069515436081)
+#define TS_B6 2.324710524099774
+#define TS_E1 (-0.00178001105222577714)
+#define TS_E2 (-0.0008164344596567469)
+#define TS_E3 0.007880878010261995
+#define TS_E4 (-0.1447110071732629)
+#define TS_E5 0.5823571654525552
+#define TS_E6 (-0.45808210592918697)
+#define TS_E7 (1.0 / 66.0)
+
+// ROS2 (Verwer, Spee, Blom & Hundsdorfer 1999): gamma = 1 + 1/sqrt(2).
+#define ROS2_GAMMA 1.7071067811865475
+
+template <typename T>
+__device__ __forceinline__ T cst(double x) {
+  return static_cast<T>(x);
+}
+
+__device__ __forceinline__ double fmaT(double a, double b, double c) { return fma(a, b, c); }
+__device__ __forceinline__ float fmaT(float a, float b, float c) { return fmaf(a, b, c); }
+
+template <typename T> struct Eps;
+template <> struct Eps<double> { static constexpr double v = 2.220446049250313e-16; };
+template <> struct Eps<float> { static constexpr float v = 1.1920928955078125e-07f; };
+
+// ---------------------------------------------------------------------------
+// Lorenz: u' = (s (u2 - u1), u1 (r - u3) - u2, u1 u2 - b u3),
+// p = (sigma, rho, beta) -- the listing on the DiffEqGPU "ad" page.
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ void lorenz_f(T x, T y, T z, T s, T r, T b, T& fx, T& fy, T& fz) {
+  fx = s * (y - x);
+  fy = fmaT(x, r - z, -y);
+  fz = fmaT(x, y, -(b * z));
+}
+
+// ---------------------------------------------------------------------------
+// Robertson kinetics, mass action for A->B (k1), 2B->B+C (k2), B+C->A+C (k3).
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ void robertson_f(T y1, T y2, T y3, T k1, T k2, T k3, T& f1, T& f2, T& f3) {
+  T r1 = k1 * y1;
+  T r2 = k2 * (y2 * y2);
+  T r3 = k3 * (y2 * y3);
+  f1 = r3 - r1;
+  f2 = (r1 - r3) - r2;
+  f3 = r2;
+}
+
+// Robertson Jacobian, row-major 3x3.
+template <typename T>
+__device__ __forceinline__ void robertson_J(T y1, T y2, T y3, T k1, T k2, T k3, T J[9]) {
+  (void)y1;
+  T a = k3 * y3;
+  T b = k3 * y2;
+  T c = cst<T>(2.0) * (k2 * y2);
+  J[0] = -k1;
+  J[1] = a;
+  J[2] = b;
+  J[3] = k1;
+  J[4] = -(a + c);
+  J[5] = -b;
+  J[6] = cst<T>(0.0);
+  J[7] = c;
+  J[8] = cst<T>(0.0);
+}
+
+// 3x3 LU with partial pivoting (largest |entry|, ties to the lowest row),
+// right-looking; whole rows swap.  Fully unrolled so M and P stay in registers.
+// Returns false on a zero or non-finite pivot.
+template <typename T>
+__device__ __forceinline__ bool lu3(T M[9], int P[3]) {
+  P[0] = 0;
+  P[1] = 1;
+  P[2] = 2;
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    int piv = k;
+#pragma unroll
+    for (int i = k + 1; i < 3; ++i)
+      if (fabs(M[i * 3 + k]) > fabs(M[piv * 3 + k])) piv = i;
+#pragma unroll
+    for (int i = k + 1; i < 3; ++i) {
+      if (piv == i) {
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          T t = M[k * 3 + j];
+          M[k * 3 + j] = M[i * 3 + j];
+          M[i * 3 + j] = t;
+        }
+        int tp = P[k];
+        P[k] = P[i];
+        P[i] = tp;
+      }
+    }
+    T pv = M[k * 3 + k];
+    ok = ok && (pv != cst<T>(0.0)) && isfinite(pv);
+#pragma unroll
+    for (int i = k + 1; i < 3; ++i) {
+      T l = M[i * 3 + k] / M[k * 3 + k];
+      M[i * 3 + k] = l;
+#pragma unroll
+      for (int j = k + 1; j < 3; ++j) M[i * 3 + j] = fmaT(-l, M[k * 3 + j], M[i * 3 + j]);
+    }
+  }
+  return ok;
+}
+
+template <typename T>
+__device__ __forceinline__ T pick3(int i, T a, T b, T c) {
+  return i == 0 ? a : (i == 1 ? b : c);
+}
+
+// Solve (P M) x = P b with the factors of lu3: x = M^{-1} b.
+template <typename T>
+__device__ __forceinline__ void lu3_solve(const T LU[9], const int P[3], T b0, T b1, T b2, T& x0, T& x1, T& x2) {
+  x0 = pick3(P[0], b0, b1, b2);
+  x1 = pick3(P[1], b0, b1, b2);
+  x2 = pick3(P[2], b0, b1, b2);
+  x1 = fmaT(-LU[3], x0, x1);
+  x2 = fmaT(-LU[6], x0, x2);
+  x2 = fmaT(-LU[7], x1, x2);
+  x2 = x2 / LU[8];
+  x1 = fmaT(-LU[5], x2, x1);
+  x1 = x1 / LU[4];
+  x0 = fmaT(-LU[1], x1, x0);
+  x0 = fmaT(-LU[2], x2, x0);
+  x0 = x0 / LU[0];
+}
+
+// Solve M^T x = b with the factors of lu3 (P M = L U, so M^T = U^T L^T P):
+// U^T y = b (forward), L^T z = y (backward, unit diagonal), x[P[i]] = z[i].
+// Used by the reverse sweep only (not part of the bitwise contract).
+template <typename T>
+__device__ __forceinline__ void lu3_solve_T(const T LU[9], const int P[3], T b0, T b1, T b2, T& x0, T& x1, T& x2) {
+  T y0 = b0 / LU[0];
+  T y1 = fmaT(-LU[1], y0, b1) / LU[4];
+  T y2 = fmaT(-LU[5], y1, fmaT(-LU[2], y0, b2)) / LU[8];
+  T z2 = y2;
+  T z1 = fmaT(-LU[7], z2, y1);
+  T z0 = fmaT(-LU[6], z2, fmaT(-LU[3], z1, y0));
+  // scatter through the permutation
+  x0 = P[0] == 0 ? z0 : (P[1] == 0 ? z1 : z2);
+  x1 = P[0] == 1 ? z0 : (P[1] == 1 ? z1 : z2);
+  x2 = P[0] == 2 ? z0 : (P[1] == 2 ? z1 : z2);
+}
+
+// ---------------------------------------------------------------------------
+// Host-side helpers.
+// ---------------------------------------------------------------------------
+void count_launch(int k = 1);
+
+inline bool launch_ok() { return cudaGetLastError() == cudaSuccess; }
+
+}  // namespace gs

@@ -1,0 +1,104 @@
+// solve.cu -- forward-only fixed-step replay on a recorded mesh, writing the
+// state at every save point (d = 3 systems, Tsit5 or ROS2).  The forward-only
+// use of GRADSOLVE (arXiv 2609.02876, abstract); same arithmetic as the
+// forward half of the gradient kernels.
+#include "steps.cuh"
+
+namespace gs {
+
+template <typename T>
+struct SolveArgs {
+  int64_t n;
+  const T* p;
+  const T* u0;
+  const T* h;
+  const int32_t* order;
+  const int32_t* nsteps;
+  const int32_t* save_idx;
+  const int32_t* status;
+  int32_t nsave;
+  int32_t smax;
+  T* u_save;  // [nsave][3][n] by trajectory
+};
+
+template <typename T, int SYS, int METHOD>
+__global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
+  const int64_t n = a.n;
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  const int64_t i = a.order[j];
+  if (i < 0 || i >= n) return;  // not a permutation entry: nothing to write
+  const int64_t n3 = 3 * n;
+  if (a.status[j] != GS_TRAJ_OK || a.nsteps[j] < 0 || a.nsteps[j] > a.smax) {
+    const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
+    for (int k = 0; k < a.nsave; ++k)
+#pragma unroll
+      for (int c = 0; c < 3; ++c) a.u_save[k * n3 + c * n + i] = nan;
+    return;
+  }
+  T u[3], p[3], k1[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    u[c] = a.u0[c * n + i];
+    p[c] = a.p[c * n + i];
+  }
+  rhs3<T, SYS>(u, p, k1);
+  const int S = a.nsteps[j];
+  int kk = 0;
+  int next = a.save_idx[j];
+  const T* hp = a.h + j;
+  for (int st = 0; st < S; ++st) {
+    const T h = hp[(int64_t)st * n];
+    T un[3];
+    if (METHOD == GS_TSIT5) {
+      T k7[3], e[3];
+      tsit5_err_step<T, SYS>(u, p, h, k1, un, k7, e);
+#pragma unroll
+      for (int c = 0; c < 3; ++c) k1[c] = k7[c];
+    } else {
+      T LU[9], q1[3], v[3], q2[3];
+      int P[3];
+      ros2_fwd<T, SYS>(u, p, h, LU, P, q1, v, q2, un);
+    }
+#pragma unroll
+    for (int c = 0; c < 3; ++c) u[c] = un[c];
+    while (st + 1 == next) {
+#pragma unroll
+      for (int c = 0; c < 3; ++c) a.u_save[kk * n3 + c * n + i] = u[c];
+      ++kk;
+      next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
+    }
+  }
+}
+
+template <typename T>
+gs_status launch_solve3(const gs_problem* P, const gs_mesh* M, void* u_save, cudaStream_t st) {
+  SolveArgs<T> a;
+  a.n = P->n;
+  a.p = (const T*)P->p;
+  a.u0 = (const T*)P->u0;
+  a.h = (const T*)M->h;
+  a.order = M->order;
+  a.nsteps = M->nsteps;
+  a.save_idx = M->save_idx;
+  a.status = M->status;
+  a.nsave = P->nsave;
+  a.smax = M->smax;
+  a.u_save = (T*)u_save;
+  const unsigned grid = (unsigned)((P->n + 127) / 128);
+  if (P->system == GS_LORENZ && P->method == GS_TSIT5)
+    k_solve3<T, kSysLorenz, GS_TSIT5><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_LORENZ && P->method == GS_ROS2)
+    k_solve3<T, kSysLorenz, GS_ROS2><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_ROBERTSON && P->method == GS_TSIT5)
+    k_solve3<T, kSysRobertson, GS_TSIT5><<<grid, 128, 0, st>>>(a);
+  else
+    k_solve3<T, kSysRobertson, GS_ROS2><<<grid, 128, 0, st>>>(a);
+  count_launch();
+  return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
+template gs_status launch_solve3<double>(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
+template gs_status launch_solve3<float>(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
+
+}  // namespace gs

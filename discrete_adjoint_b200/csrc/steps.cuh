@@ -1,0 +1,176 @@
+// steps.cuh -- the d = 3 step formulas of the forward replay (Tsit5 and
+// ROS2 on Lorenz and Robertson), written in the floating-point contract's
+// operation order.  Shared by the recorder, the Rosenbrock gradient kernel and
+// the forward-only solve.
+#pragma once
+
+#include "common.cuh"
+
+namespace gs {
+
+constexpr int kSysLorenz = GS_LORENZ;
+constexpr int kSysRobertson = GS_ROBERTSON;
+
+// std::max / std::min semantics (the CPU reference's), NaN included.
+template <typename T> __device__ __forceinline__ T smax_(T a, T b) { return (a < b) ? b : a; }
+template <typename T> __device__ __forceinline__ T smin_(T a, T b) { return (b < a) ? b : a; }
+
+template <typename T, int SYS>
+__device__ __forceinline__ void rhs3(const T u[3], const T p[3], T f[3]) {
+  if (SYS == kSysLorenz)
+    lorenz_f(u[0], u[1], u[2], p[0], p[1], p[2], f[0], f[1], f[2]);
+  else
+    robertson_f(u[0], u[1], u[2], p[0], p[1], p[2], f[0], f[1], f[2]);
+}
+
+template <typename T, int SYS>
+__device__ __forceinline__ void jac3(const T u[3], const T p[3], T J[9]) {
+  if (SYS == kSysLorenz) {
+    J[0] = -p[0];
+    J[1] = p[0];
+    J[2] = cst<T>(0.0);
+    J[3] = p[1] - u[2];
+    J[4] = cst<T>(-1.0);
+    J[5] = -u[0];
+    J[6] = u[1];
+    J[7] = u[0];
+    J[8] = -p[2];
+  } else {
+    robertson_J(u[0], u[1], u[2], p[0], p[1], p[2], J);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ T rms3(const T x[3], const T sc[3]) {
+  T s = cst<T>(0.0);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T q = x[c] / sc[c];
+    s = fmaT(q, q, s);
+  }
+  return sqrt(s / cst<T>(3.0));
+}
+
+// One Tsit5 step with error estimate; k1 = f(u) on entry, k7 = f(u_new) out.
+template <typename T, int SYS>
+__device__ __forceinline__ void tsit5_err_step(const T u[3], const T p[3], T h, const T k1[3], T un[3], T k7[3],
+                                               T e[3]) {
+  T k2[3], k3[3], k4[3], k5[3], k6[3], U[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, cst<T>(TS_A21) * k1[c], u[c]);
+  rhs3<T, SYS>(U, p, k2);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, fmaT(cst<T>(TS_A32), k2[c], cst<T>(TS_A31) * k1[c]), u[c]);
+  rhs3<T, SYS>(U, p, k3);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(TS_A41) * k1[c];
+    acc = fmaT(cst<T>(TS_A42), k2[c], acc);
+    acc = fmaT(cst<T>(TS_A43), k3[c], acc);
+    U[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(U, p, k4);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(TS_A51) * k1[c];
+    acc = fmaT(cst<T>(TS_A52), k2[c], acc);
+    acc = fmaT(cst<T>(TS_A53), k3[c], acc);
+    acc = fmaT(cst<T>(TS_A54), k4[c], acc);
+    U[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(U, p, k5);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(TS_A61) * k1[c];
+    acc = fmaT(cst<T>(TS_A62), k2[c], acc);
+    acc = fmaT(cst<T>(TS_A63), k3[c], acc);
+    acc = fmaT(cst<T>(TS_A64), k4[c], acc);
+    acc = fmaT(cst<T>(TS_A65), k5[c], acc);
+    U[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(U, p, k6);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(TS_B1) * k1[c];
+    acc = fmaT(cst<T>(TS_B2), k2[c], acc);
+    acc = fmaT(cst<T>(TS_B3), k3[c], acc);
+    acc = fmaT(cst<T>(TS_B4), k4[c], acc);
+    acc = fmaT(cst<T>(TS_B5), k5[c], acc);
+    acc = fmaT(cst<T>(TS_B6), k6[c], acc);
+    un[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(un, p, k7);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(TS_E1) * k1[c];
+    acc = fmaT(cst<T>(TS_E2), k2[c], acc);
+    acc = fmaT(cst<T>(TS_E3), k3[c], acc);
+    acc = fmaT(cst<T>(TS_E4), k4[c], acc);
+    acc = fmaT(cst<T>(TS_E5), k5[c], acc);
+    acc = fmaT(cst<T>(TS_E6), k6[c], acc);
+    acc = fmaT(cst<T>(TS_E7), k7[c], acc);
+    e[c] = h * acc;
+  }
+}
+
+// One ROS2 step with error estimate.  Returns false on a singular matrix.
+template <typename T, int SYS>
+__device__ __forceinline__ bool ros2_err_step(const T u[3], const T p[3], T h, T un[3], T e[3]) {
+  T J[9], M[9];
+  int P[3];
+  jac3<T, SYS>(u, p, J);
+  const T gh = cst<T>(ROS2_GAMMA) * h;
+#pragma unroll
+  for (int q = 0; q < 9; ++q) M[q] = fmaT(-gh, J[q], cst<T>((q % 4) == 0 ? 1.0 : 0.0));
+  if (!lu3(M, P)) return false;
+  T f0[3], k1[3], v[3], f1[3], k2[3];
+  rhs3<T, SYS>(u, p, f0);
+  lu3_solve(M, P, f0[0], f0[1], f0[2], k1[0], k1[1], k1[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) v[c] = fmaT(h, k1[c], u[c]);
+  rhs3<T, SYS>(v, p, f1);
+  T r0 = fmaT(cst<T>(-2.0), k1[0], f1[0]);
+  T r1 = fmaT(cst<T>(-2.0), k1[1], f1[1]);
+  T r2 = fmaT(cst<T>(-2.0), k1[2], f1[2]);
+  lu3_solve(M, P, r0, r1, r2, k2[0], k2[1], k2[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(1.5) * k1[c];
+    acc = fmaT(cst<T>(0.5), k2[c], acc);
+    un[c] = fmaT(h, acc, u[c]);
+    e[c] = (h * cst<T>(0.5)) * (k1[c] + k2[c]);
+  }
+  return true;
+}
+
+// Bitwise forward step; also returns the pieces the reverse sweep needs.
+template <typename T, int SYS>
+__device__ __forceinline__ bool ros2_fwd(const T u[3], const T p[3], T h, T LU[9], int P[3], T k1[3], T v[3],
+                                         T k2[3], T un[3]) {
+  T J[9];
+  jac3<T, SYS>(u, p, J);
+  const T gh = cst<T>(ROS2_GAMMA) * h;
+#pragma unroll
+  for (int q = 0; q < 9; ++q) LU[q] = fmaT(-gh, J[q], cst<T>((q % 4) == 0 ? 1.0 : 0.0));
+  bool ok = lu3(LU, P);
+  T f0[3], f1[3];
+  rhs3<T, SYS>(u, p, f0);
+  lu3_solve(LU, P, f0[0], f0[1], f0[2], k1[0], k1[1], k1[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) v[c] = fmaT(h, k1[c], u[c]);
+  rhs3<T, SYS>(v, p, f1);
+  T r0 = fmaT(cst<T>(-2.0), k1[0], f1[0]);
+  T r1 = fmaT(cst<T>(-2.0), k1[1], f1[1]);
+  T r2 = fmaT(cst<T>(-2.0), k1[2], f1[2]);
+  lu3_solve(LU, P, r0, r1, r2, k2[0], k2[1], k2[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(1.5) * k1[c];
+    acc = fmaT(cst<T>(0.5), k2[c], acc);
+    un[c] = fmaT(h, acc, u[c]);
+  }
+  return ok;
+}
+
+
+}  // namespace gs

@@ -1,0 +1,215 @@
+/*
+ * gradsolve.h -- C ABI of the B200 record-and-replay discrete-adjoint library
+ * (libgradsolve.so).
+ *
+ * The method (GRADSOLVE, arXiv 2609.02876; abstract, and the evolve.pub
+ * review's "Summary" and "Strengths: precisely scoped exactness claim"):
+ * an adaptive solver runs once per trajectory and records the step sizes it
+ * accepts (gs_record); a fixed-step replay of that mesh, the mesh held fixed as
+ * data, defines a loss; gs_grad returns the exact derivative of that replay
+ * (the discrete adjoint) with respect to each trajectory's parameters and
+ * initial state, excluding any derivative of the step-size choices (review FAQ
+ * "Is gradsolve's gradient really exact?").  gs_solve is the forward-only
+ * replay.  One record serves any number of gs_grad / gs_solve calls: the
+ * method is aimed at ensembles whose gradient is taken many times against a
+ * single record (abstract).
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" are caller-owned device memory of the current
+ *    CUDA device; "host" pointers are read during the call only.  The library
+ *    allocates nothing: scratch memory is the caller's workspace, sized by
+ *    gs_workspace_bytes.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronize.  Results are valid once the stream reaches
+ *    the end of the call's work.
+ *  - Outputs are overwritten, never accumulated.
+ *  - Argument errors return a negative gs_status before anything is launched.
+ *    A launch failure returns GS_ECUDA.  Failures of single trajectories are
+ *    not call errors: they are reported per trajectory in mesh.status and the
+ *    call returns GS_OK.
+ *  - Layouts are structure-of-arrays over the ensemble ("SoA"): element c of
+ *    trajectory i of an array shaped [m][n] is at [c * n + i].  Floating-point
+ *    arrays have the problem's dtype (float for GS_F32, double for GS_F64).
+ *  - Not thread-safe against concurrent calls that share a mesh or workspace.
+ */
+#ifndef GRADSOLVE_H
+#define GRADSOLVE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GS_API __attribute__((visibility("default")))
+#else
+#define GS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t gs_status;
+#define GS_OK 0
+#define GS_EINVAL (-1)       /* bad argument (null pointer, size, combination) */
+#define GS_ECUDA (-2)        /* a CUDA launch or runtime call failed */
+#define GS_EWORKSPACE (-3)   /* workspace pointer null or smaller than required */
+#define GS_EUNSUPPORTED (-4) /* valid request this build does not implement */
+
+/* Per-trajectory record status (mesh.status). */
+#define GS_TRAJ_OK 0
+#define GS_TRAJ_MAXSTEPS 1  /* more than smax accepted steps or smax rejections */
+#define GS_TRAJ_DTMIN 2     /* step proposal fell below 16 eps |t| */
+#define GS_TRAJ_NONFINITE 3 /* non-finite input, f(u0) or initial step */
+#define GS_TRAJ_SINGULAR 4  /* zero or non-finite pivot in the Rosenbrock LU */
+
+/* Registered right-hand sides. */
+#define GS_LORENZ 1    /* d=3, np=3, p=(sigma, rho, beta): DiffEqGPU "ad" page, Lorenz listing */
+#define GS_ROBERTSON 2 /* d=3, np=3, p=(k1, k2, k3): mass-action kinetics A->B, 2B->B+C, B+C->A+C */
+#define GS_HIRES 3     /* reserved: not built (equations not available to this build) */
+#define GS_NODE64 4    /* d=64, np=64 (b_i), shared W [64][64]: f = tanh(W u + b) - u */
+
+/* Integrators. */
+#define GS_TSIT5 1 /* Tsitouras 5(4) pair, FSAL, PI step control */
+#define GS_ROS2 2  /* Rosenbrock ROS2, gamma = 1 + 1/sqrt(2) (Verwer et al. 1999); d = 3 only */
+
+#define GS_F32 1
+#define GS_F64 2
+
+/* Losses over the save points k = 0..nsave-1. */
+#define GS_LOSS_SUMSQ 1  /* L_i = sum_k ||u_i(t_k) - target_ik||^2  (target NULL = 0) */
+#define GS_LOSS_LINEAR 2 /* L_i = sum_k weight_ik . u_i(t_k) */
+
+#define GS_MAX_SAVE 64 /* largest nsave */
+
+/* workspace operations */
+#define GS_OP_RECORD 0
+#define GS_OP_GRAD 1
+
+/*
+ * An ensemble of n independent trajectories of one registered system.
+ *   p       device, [np][n]: per-trajectory parameters.
+ *   u0      device, [d][n]:  initial states.
+ *   shared  device, GS_NODE64 only: W, [64][64] row-major (row r, column c at
+ *           r*64 + c), shared by all trajectories; NULL otherwise.
+ *   t0, t1  time span, t0 < t1.
+ *   tsave   host, nsave (1..GS_MAX_SAVE) strictly increasing times in (t0, t1]:
+ *           the save points of gs_solve and of the loss.  Steps land on them.
+ */
+typedef struct gs_problem {
+  int32_t system, method, dtype, d, np;
+  int64_t n;
+  const void* p;
+  const void* u0;
+  const void* shared;
+  double t0, t1;
+  int32_t nsave;
+  const double* tsave;
+} gs_problem;
+
+/* Step-size control: accept iff the RMS of e_c / (atol + rtol max(|u_c|, |u'_c|))
+ * is <= 1.  h0 > 0 fixes the first proposal; h0 = 0 picks it automatically
+ * (Hairer, Norsett & Wanner I, II.4). */
+typedef struct gs_tol {
+  double rtol, atol, h0;
+} gs_tol;
+
+/*
+ * The record (the mesh), all device arrays, all indexed by SLOT, not by
+ * trajectory: slot j holds trajectory order[j].  gs_record orders slots by
+ * decreasing step count (ties by trajectory index) so that the threads of a
+ * warp replay chains of nearly equal length; any permutation is valid input to
+ * gs_grad / gs_solve (e.g. a mesh built elsewhere, with order = identity).
+ *   smax      capacity in steps (rows of h).
+ *   nsave     must equal the problem's nsave.
+ *   h         [smax][n] dtype, step-major: step s of slot j at s*n + j;
+ *             rows s >= nsteps[j] are zero.
+ *   order     [n] int32, a permutation of 0..n-1.
+ *   nsteps    [n] int32, accepted steps of slot j.
+ *   save_idx  [nsave][n] int32, number of steps taken when t reached tsave[k]
+ *             (1..nsteps[j]).
+ *   status    [n] int32, GS_TRAJ_* of slot j.
+ *   nreject   [n] int32, rejected attempts of slot j (diagnostic).
+ */
+typedef struct gs_mesh {
+  int32_t smax, nsave;
+  void* h;
+  int32_t* order;
+  int32_t* nsteps;
+  int32_t* save_idx;
+  int32_t* status;
+  int32_t* nreject;
+} gs_mesh;
+
+/* Loss description.  target / weight: device, [nsave][d][n] dtype, indexed by
+ * trajectory.  SUMSQ reads target (NULL = zero target); LINEAR reads weight. */
+typedef struct gs_loss {
+  int32_t kind;
+  const void* target;
+  const void* weight;
+} gs_loss;
+
+/*
+ * Workspace (scratch) bytes that op (GS_OP_RECORD / GS_OP_GRAD) needs for this
+ * problem and mesh capacity: record -- step counts of the sizing pass and the
+ * slot-ordering histograms; grad -- one checkpointed state per step and slot,
+ * [smax][d][n] dtype (plus the d=64 weight-gradient partials).  Returns 0 for
+ * an invalid request.  Host function; no device work.
+ */
+GS_API size_t gs_workspace_bytes(const gs_problem* prob, const gs_mesh* mesh, int32_t op);
+
+/*
+ * Sizing pass: runs the adaptive solve of every trajectory without storing a
+ * mesh and writes, indexed by TRAJECTORY, the accepted step count (nsteps) and
+ * status (both device [n] int32; status may be NULL).  smax caps the count
+ * (GS_TRAJ_MAXSTEPS beyond it).  Use it to pick the mesh capacity.
+ * (The recorder of the gptget summary, "Methodology", without its stores.)
+ */
+GS_API gs_status gs_count(const gs_problem* prob, const gs_tol* tol, int32_t smax, int32_t* nsteps, int32_t* status,
+                   void* stream);
+
+/*
+ * Record: adaptive solve of every trajectory (Tsit5 or ROS2 per prob->method)
+ * into the caller's mesh, slots ordered by decreasing step count.  Fills every
+ * mesh array.  Trajectories that fail keep a status != 0 and a truncated mesh.
+ * Runs a sizing pass, the slot ordering and the recording pass, all on stream.
+ * (Evolve.pub review, "Summary": the adaptive solve happens once and keeps each
+ * trajectory's accepted step sizes.)
+ */
+GS_API gs_status gs_record(const gs_problem* prob, const gs_tol* tol, const gs_mesh* mesh, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
+ * Forward-only replay on the mesh: u_save, device [nsave][d][n] dtype, indexed
+ * by trajectory, receives the state at each save point.  Slots with status != 0
+ * get NaN.  (The forward-only solver use of the abstract.)
+ */
+GS_API gs_status gs_solve(const gs_problem* prob, const gs_mesh* mesh, void* u_save, void* stream);
+
+/*
+ * Fused replay + reverse sweep: for every trajectory, the loss of the
+ * fixed-step replay on the mesh and its exact discrete adjoint.
+ *   loss     device [n] dtype       L_i
+ *   dp       device [np][n] dtype   dL_i/dp_i   (GS_NODE64: dL_i/db_i)
+ *   du0      device [d][n] dtype    dL_i/du0_i
+ *   dshared  device [64][64] dtype, GS_NODE64: sum_i dL_i/dW; else NULL
+ *   ws       workspace of gs_workspace_bytes(prob, mesh, GS_OP_GRAD) bytes
+ * All indexed by trajectory.  Slots with status != 0 get NaN loss/dp/du0 and
+ * do not contribute to dshared.  (Evolve.pub review, "Summary": the replay is a
+ * fixed-length chain without branches, and its backward sweep is the exact
+ * discrete adjoint.)
+ */
+GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_loss* loss_desc, void* loss, void* dp,
+                  void* du0, void* dshared, void* ws, size_t ws_bytes, void* stream);
+
+/* Static description of a status code. */
+GS_API const char* gs_status_string(gs_status status);
+
+/* Number of kernels this library has launched since it was loaded
+ * (diagnostic for launch accounting; monotone, process-wide). */
+GS_API int64_t gs_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRADSOLVE_H */

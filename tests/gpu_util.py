@@ -1,0 +1,66 @@
+"""Helpers for the GPU tests: move a workloads.Problem to the device, carry an
+oracle mesh into the library's slot layout, and read a device mesh back in
+trajectory order.  Marshalling only."""
+import numpy as np
+import torch
+
+import discrete_adjoint_b200 as gs
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def tens(a, dtype, d=None):
+    return torch.tensor(np.ascontiguousarray(a), dtype=dtype, device=d or dev())
+
+
+def ensemble(prob):
+    td = gs.gradsolve.TORCH_DTYPE[prob.dtype]
+    return gs.Ensemble(prob.system, prob.method, prob.dtype, tens(prob.p, td), tens(prob.u0, td), prob.t0,
+                       prob.t1, [float(x) for x in prob.tsave],
+                       None if prob.W is None else tens(prob.W, td))
+
+
+def loss_args(prob):
+    td = gs.gradsolve.TORCH_DTYPE[prob.dtype]
+    tgt = None if prob.target is None else tens(prob.target, td)
+    w = None if prob.weight is None else tens(prob.weight, td)
+    return dict(loss=prob.loss, target=tgt, weight=w)
+
+
+def mesh_from_oracle(om, dtype, order=None, smax=None):
+    """Slot j holds trajectory order[j] (identity by default)."""
+    n = om.h.shape[0]
+    order = np.arange(n) if order is None else np.asarray(order)
+    smax = smax or om.h.shape[1]
+    h = np.zeros((smax, n))
+    h[: om.h.shape[1]] = om.h[order].T[:smax]
+    td = gs.gradsolve.TORCH_DTYPE[dtype]
+    i32 = lambda a: tens(np.asarray(a, np.int32), torch.int32)
+    return gs.Mesh(tens(h, td), i32(order), i32(om.nsteps[order]), i32(om.save_idx[order].T),
+                   i32(om.status[order]), i32(om.nreject[order]))
+
+
+def mesh_by_trajectory(mesh):
+    """(h [n][smax], nsteps [n], save_idx [n][nsave], status [n], order) in trajectory order."""
+    order = mesh.order.cpu().numpy()
+    inv = np.empty_like(order)
+    inv[order] = np.arange(len(order))
+    h = mesh.h.double().cpu().numpy().T[inv]
+    return h, mesh.nsteps.cpu().numpy()[inv], mesh.save_idx.cpu().numpy().T[inv], mesh.status.cpu().numpy()[inv], order
+
+
+def grad_rel_err(out, ref):
+    """Per-trajectory ||g - g_ref||_inf / ||g_ref||_inf over (dp, du0)."""
+    g = np.vstack([out.dp.double().cpu().numpy(), out.du0.double().cpu().numpy()])
+    r = np.vstack([ref["dp"], ref["du0"]])
+    return np.abs(g - r).max(0) / np.abs(r).max(0)
+
+
+def mesh_rel_err(h_gpu, h_orc, ns):
+    worst = 0.0
+    for i in range(len(ns)):
+        a, b = h_gpu[i, : ns[i]], h_orc[i, : ns[i]]
+        worst = max(worst, float(np.max(np.abs(a - b) / np.abs(b))) if ns[i] else 0.0)
+    return worst

@@ -1,0 +1,120 @@
+"""The C-ABI library loads and exports every entry point the header declares;
+host-side argument validation and workspace sizing (no device work)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gradsolve.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return re.findall(r"GS_API\s+[\w\s\*]+?\b(gs_\w+)\s*\(", src)
+
+
+def test_header_declares_entry_points():
+    names = set(_declared())
+    assert {"gs_workspace_bytes", "gs_count", "gs_record", "gs_solve", "gs_grad", "gs_status_string",
+            "gs_launch_count"} <= names
+
+
+def test_library_exports_every_declared_symbol():
+    import discrete_adjoint_b200 as gs
+    lib = ctypes.CDLL(gs.gradsolve.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    import discrete_adjoint_b200 as gs
+    for code in (0, -1, -2, -3, -4):
+        assert gs.gs_status_string(code) not in ("", "unknown status")
+    assert gs.gs_status_string(17) == "unknown status"
+
+
+def _host_problem(n=1000, system=1, method=1, dtype=2, nsave=10, tsave=None):
+    from discrete_adjoint_b200.gradsolve import _Problem
+    ts = tsave if tsave is not None else [float(k) for k in range(1, nsave + 1)]
+    arr = (ctypes.c_double * len(ts))(*ts)
+    p = _Problem(system, method, dtype, 3, 3, n, 16, 16, None, 0.0, 10.0, len(ts), arr)
+    p._keep = arr
+    return p
+
+
+def test_workspace_sizes_host_only():
+    from discrete_adjoint_b200.gradsolve import _Mesh, _lib
+    p = _host_problem()
+    m = _Mesh(500, 10, None, None, None, None, None, None)
+    # one checkpointed state per step and slot
+    assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 1) == 500 * 3 * 1000 * 8
+    assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 0) >= 1000 * 4
+    assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 7) == 0
+    p32 = _host_problem(dtype=1)
+    assert _lib.gs_workspace_bytes(ctypes.byref(p32), ctypes.byref(m), 1) == 500 * 3 * 1000 * 4
+
+
+@pytest.mark.parametrize("bad", ["tsave_order", "tsave_range", "nsave0", "system", "dims", "dtype", "hires"])
+def test_invalid_problems_rejected_before_launch(bad):
+    from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol
+    kw = {}
+    if bad == "tsave_order":
+        kw["tsave"] = [1.0, 3.0, 2.0]
+    if bad == "tsave_range":
+        kw["tsave"] = [11.0]
+    if bad == "nsave0":
+        kw["tsave"] = []
+    p = _host_problem(**kw)
+    if bad == "system":
+        p.system = 9
+    if bad == "dims":
+        p.d = 4
+    if bad == "dtype":
+        p.dtype = 3
+    if bad == "hires":
+        p.system = 3
+    tol = _Tol(1e-6, 1e-6, 0.0)
+    rc = _lib.gs_count(ctypes.byref(p), ctypes.byref(tol), 100, ctypes.c_void_p(16), None, None)
+    assert rc == (-4 if bad == "hires" else -1)
+    m = _Mesh(100, p.nsave, 16, 16, 16, 16, 16, 16)
+    assert _lib.gs_record(ctypes.byref(p), ctypes.byref(tol), ctypes.byref(m), ctypes.c_void_p(16), 1 << 40,
+                          None) == (-4 if bad == "hires" else -1)
+
+
+def test_bad_tolerance_and_workspace_rejected():
+    from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
+    p = _host_problem()
+    m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+    assert _lib.gs_count(ctypes.byref(p), ctypes.byref(_Tol(-1.0, 1e-6, 0.0)), 100, ctypes.c_void_p(16), None,
+                         None) == -1
+    assert _lib.gs_count(ctypes.byref(p), ctypes.byref(_Tol(float("nan"), 1e-6, 0.0)), 100,
+                         ctypes.c_void_p(16), None, None) == -1
+    # record and grad refuse a workspace that is too small (before any launch)
+    assert _lib.gs_record(ctypes.byref(p), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), ctypes.byref(m),
+                          ctypes.c_void_p(16), 8, None) == -3
+    ls = _Loss(1, None, None)
+    assert _lib.gs_grad(ctypes.byref(p), ctypes.byref(m), ctypes.byref(ls), ctypes.c_void_p(16),
+                        ctypes.c_void_p(16), ctypes.c_void_p(16), None, ctypes.c_void_p(16), 8, None) == -3
+    # linear loss without weights
+    assert _lib.gs_grad(ctypes.byref(p), ctypes.byref(m), ctypes.byref(_Loss(2, None, None)), ctypes.c_void_p(16),
+                        ctypes.c_void_p(16), ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 40, None) == -1
+    # mesh nsave must match
+    m2 = _Mesh(100, 3, 16, 16, 16, 16, 16, 16)
+    assert _lib.gs_solve(ctypes.byref(p), ctypes.byref(m2), ctypes.c_void_p(16), None) == -1
+
+
+def test_empty_ensemble_is_a_no_op():
+    from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
+    p = _host_problem(n=0)
+    m = _Mesh(100, 10, None, None, None, None, None, None)
+    before = _lib.gs_launch_count()
+    assert _lib.gs_count(ctypes.byref(p), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, None, None, None) == 0
+    assert _lib.gs_record(ctypes.byref(p), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), ctypes.byref(m), None, 0,
+                          None) == 0
+    assert _lib.gs_grad(ctypes.byref(p), ctypes.byref(m), ctypes.byref(_Loss(1, None, None)), None, None, None,
+                        None, None, 0, None) == 0
+    assert _lib.gs_solve(ctypes.byref(p), ctypes.byref(m), None, None) == 0
+    assert _lib.gs_launch_count() == before

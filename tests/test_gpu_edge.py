@@ -1,0 +1,90 @@
+"""Edge cases of the GPU path: tiny and ragged ensembles, failing
+trajectories, invariances, call errors."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+import discrete_adjoint_b200 as gs
+from gpu_util import dev, ensemble, grad_rel_err, loss_args, mesh_by_trajectory, mesh_from_oracle, tens
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("n", [1, 31, 129])
+def test_tiny_and_ragged(n):
+    prob = W.lorenz_small(n)
+    om = oracle.record(prob, 256)
+    og = oracle.grad(prob, om)
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(n, 256, 1, "f64", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    out = gs.gs_grad(ens, mesh_from_oracle(om, "f64"), **loss_args(prob))
+    torch.cuda.synchronize()
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    assert np.array_equal(ns, om.nsteps)
+    assert grad_rel_err(out, og).max() <= 1e-12
+
+
+def test_capacity_and_nonfinite_statuses():
+    prob = W.lorenz_small(64)
+    prob.p = prob.p.copy()
+    prob.p[0, 5] = np.nan
+    om = oracle.record(prob, 140)  # some trajectories need more than 140 steps
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(prob.n, 140, 1, "f64", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    out = gs.gs_grad(ens, mesh, **loss_args(prob))
+    u = gs.gs_solve(ens, mesh)
+    torch.cuda.synchronize()
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    assert np.array_equal(st, om.status)
+    assert st[5] == gs.gradsolve.TRAJ_NONFINITE and (st == gs.gradsolve.TRAJ_MAXSTEPS).any()
+    bad = st != 0
+    assert torch.isnan(out.loss.cpu()[torch.tensor(bad)]).all()
+    assert torch.isfinite(out.dp.cpu()[:, torch.tensor(~bad)]).all()
+    assert torch.isnan(u.cpu()[:, :, torch.tensor(bad)]).all()
+
+
+def test_leading_zero_steps_are_identities():
+    prob = W.lorenz_small(100)
+    om = oracle.record(prob, 256)
+    ens = ensemble(prob)
+    ref = gs.gs_grad(ens, mesh_from_oracle(om, "f64"), **loss_args(prob))
+    z = 5
+    om2 = oracle.Mesh(np.concatenate([np.zeros((prob.n, z)), om.h], 1), om.nsteps + z, om.save_idx + z,
+                      om.status, om.nreject)
+    out = gs.gs_grad(ens, mesh_from_oracle(om2, "f64"), **loss_args(prob))
+    torch.cuda.synchronize()
+    for a, b in ((out.loss, ref.loss), (out.dp, ref.dp), (out.du0, ref.du0)):
+        assert torch.equal(a, b)
+
+
+def test_permuted_slots_give_identical_bits():
+    prob = W.lorenz_1m(300)
+    om = oracle.record(prob, 1024)
+    ens = ensemble(prob)
+    a = gs.gs_grad(ens, mesh_from_oracle(om, "f64"), **loss_args(prob))
+    b = gs.gs_grad(ens, mesh_from_oracle(om, "f64", np.random.default_rng(0).permutation(prob.n)),
+                   **loss_args(prob))
+    torch.cuda.synchronize()
+    assert torch.equal(a.dp, b.dp) and torch.equal(a.du0, b.du0) and torch.equal(a.loss, b.loss)
+
+
+def test_call_errors():
+    prob = W.lorenz_small(16)
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(16, 256, 1, "f64", dev())
+    with pytest.raises(gs.gradsolve.GradsolveError) as e:
+        gs.gs_grad(ens, mesh, ws=gs.workspace(16, dev()))
+    assert e.value.code == gs.gradsolve.GS_EWORKSPACE
+    big = gs.new_mesh(16, 256, 3, "f64", dev())
+    with pytest.raises(gs.gradsolve.GradsolveError):
+        gs.gs_solve(ens, big)
+    ens_rt = ensemble(W.robertson(16))
+    ens_rt.method = "tsit5"
+    with pytest.raises(gs.gradsolve.GradsolveError) as e:
+        gs.gs_grad(ens_rt, gs.new_mesh(16, 64, 1, "f64", dev()), loss="linear",
+                   weight=torch.ones((1, 3, 16), dtype=torch.float64, device=dev()))
+    assert e.value.code == gs.gradsolve.GS_EUNSUPPORTED
