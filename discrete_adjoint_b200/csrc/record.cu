@@ -61,7 +61,7 @@ __device__ T initial_step3(const T u0[3], const T p[3], T t0, T t1, T rtol, T at
   for (int c = 0; c < 3; ++c) df[c] = f1[c] - f0[c];
   T d2 = rms3(df, sc) / h0;
   T dm = smax_(d1, d2);
-  T h1 = dm <= cst<T>(1e-15) ? smax_(cst<T>(1e-6), h0 * cst<T>(1e-3)) : pow(cst<T>(0.01) / dm, cst<T>(1.0) / q);
+  T h1 = dm <= cst<T>(1e-15) ? smax_(cst<T>(1e-6), h0 * cst<T>(1e-3)) : ctrl_pow<T>(cst<T>(0.01) / dm, cst<T>(1.0) / q);
   return smin_(smin_(cst<T>(100.0) * h0, h1), t1 - t0);
 }
 
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
       if (err == cst<T>(0.0)) {
         fac = cst<T>(10.0);
       } else {
-        fac = (cst<T>(0.9) * pow(err, -(cst<T>(0.7) / q))) * pow(errprev, cst<T>(0.4) / q);
+        fac = (cst<T>(0.9) * ctrl_pow<T>(err, -(cst<T>(0.7) / q))) * ctrl_pow<T>(errprev, cst<T>(0.4) / q);
         fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
       }
       if (prev_rej) fac = smin_(fac, cst<T>(1.0));
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
         status = GS_TRAJ_MAXSTEPS;
         break;
       }
-      const T fac = isnan(err) ? cst<T>(0.2) : smax_(cst<T>(0.2), cst<T>(0.9) * pow(err, -(cst<T>(1.0) / q)));
+      const T fac = isnan(err) ? cst<T>(0.2) : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_pow<T>(err, -(cst<T>(1.0) / q)));
       hprop = fac * hprop;
       prev_rej = true;
     }

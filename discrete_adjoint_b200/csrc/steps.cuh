@@ -40,6 +40,71 @@ __device__ __forceinline__ void jac3(const T u[3], const T p[3], T J[9]) {
   }
 }
 
+// Powers x^y for the step-size controller.  Library pow may differ from other
+// implementations by an ulp, and the embedded error estimate (a sum with heavy
+// cancellation) turns such an ulp into ~1e-10 relative step-size differences
+// within a few steps, which chaos then amplifies.  This one uses only IEEE
+// +, -, *, /, fma and the exact frexp / ldexp / rint, in a fixed order, so its
+// bits are reproducible on any IEEE machine that keeps the order:
+//   ln x : x = m 2^e, m in [sqrt(1/2), sqrt(2)); ln m = 2 atanh(s),
+//          s = (m-1)/(m+1), series s (1 + z/3 + ... + z^12/25), z = s^2;
+//   exp w: Cody & Waite reduction w = k ln2 + r (ln2 = 21-bit head + tail),
+//          Taylor polynomial of e^r to degree 14, times 2^k.
+// Accuracy: ~1 ulp for the controller's arguments (errors 1e-4..1e3, |y| <= 1).
+__device__ __forceinline__ double frexpT(double x, int* e) { return frexp(x, e); }
+__device__ __forceinline__ float frexpT(float x, int* e) { return frexpf(x, e); }
+__device__ __forceinline__ double ldexpT(double x, int e) { return ldexp(x, e); }
+__device__ __forceinline__ float ldexpT(float x, int e) { return ldexpf(x, e); }
+__device__ __forceinline__ double rintT(double x) { return rint(x); }
+__device__ __forceinline__ float rintT(float x) { return rintf(x); }
+
+template <typename T>
+__device__ T ctrl_pow(T x, T y) {
+  if (isnan(x) || isnan(y)) return x + y;
+  if (x == cst<T>(0.0)) return y > cst<T>(0.0) ? cst<T>(0.0) : (y < cst<T>(0.0) ? cst<T>(1.0) / x : cst<T>(1.0));
+  if (isinf(x)) return y > cst<T>(0.0) ? x : (y < cst<T>(0.0) ? cst<T>(0.0) : cst<T>(1.0));
+  int e = 0;
+  T m = frexpT(x, &e);
+  if (m < cst<T>(0.7071067811865476)) {
+    m = m + m;
+    e = e - 1;
+  }
+  const T s = (m - cst<T>(1.0)) / (m + cst<T>(1.0));
+  const T z = s * s;
+  T poly = cst<T>(1.0 / 25.0);
+#pragma unroll
+  for (int k = 11; k >= 0; --k) poly = fmaT(poly, z, cst<T>(1.0 / double(2 * k + 1)));
+  const T lnm = (s + s) * poly;
+  const T ef = (T)e;
+  const T lnx = fmaT(ef, cst<T>(0.6931467056274414), fmaT(ef, cst<T>(4.7493250390316726e-07), lnm));
+  const T w = y * lnx;
+  const T kf = rintT(w * cst<T>(1.4426950408889634));
+  if (kf > cst<T>(2000.0)) return cst<T>(1.0) / cst<T>(0.0);
+  if (kf < cst<T>(-2000.0)) return cst<T>(0.0);
+  T r = fmaT(-kf, cst<T>(0.6931467056274414), w);
+  r = fmaT(-kf, cst<T>(4.7493250390316726e-07), r);
+  // Horner over 1/j!, j = 14 .. 0 (j! exact in double for j <= 14)
+  constexpr double inv_fact[15] = {1.0,
+                                   1.0,
+                                   1.0 / 2.0,
+                                   1.0 / 6.0,
+                                   1.0 / 24.0,
+                                   1.0 / 120.0,
+                                   1.0 / 720.0,
+                                   1.0 / 5040.0,
+                                   1.0 / 40320.0,
+                                   1.0 / 362880.0,
+                                   1.0 / 3628800.0,
+                                   1.0 / 39916800.0,
+                                   1.0 / 479001600.0,
+                                   1.0 / 6227020800.0,
+                                   1.0 / 87178291200.0};
+  T p = cst<T>(inv_fact[14]);
+#pragma unroll
+  for (int j = 13; j >= 0; --j) p = fmaT(p, r, cst<T>(inv_fact[j]));
+  return ldexpT(p, (int)kf);
+}
+
 template <typename T>
 __device__ __forceinline__ T rms3(const T x[3], const T sc[3]) {
   T s = cst<T>(0.0);

@@ -71,6 +71,8 @@ def lib():
         L.or_tsit5_tableau.argtypes = [dp, dp, dp]
         L.or_tsit5_tableau.restype = None
         L.or_ros2_gamma.restype = f64
+        L.or_ctrl_pow.argtypes = [i32, i64, dp, dp, dp]
+        L.or_ctrl_pow.restype = None
         _lib = L
     return _lib
 
@@ -142,7 +144,9 @@ def grad(prob, mesh: Mesh, mode: str = "tape", nthreads: int | None = None):
     """Exact gradient of the fixed-step replay loss.
 
     mode ``"tape"``: reverse-mode AD (tape).  mode ``"dual"``: forward mode,
-    one dual-number pass per input (p and u0; not node64).
+    one dual-number pass per input (p and u0; not node64).  mode
+    ``"tape_wide"``: the tape with its adjoints accumulated in a wider type
+    (long double for fp64, double for fp32).
     Returns dict(loss [n], dp [np][n], du0 [d][n], dW [64,64] or None).
     """
     L = lib()
@@ -155,7 +159,7 @@ def grad(prob, mesh: Mesh, mode: str = "tape", nthreads: int | None = None):
     dW = np.zeros((64, 64)) if prob.system == "node64" else None
     rc = L.or_grad(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, d, npar, _d(_f64(prob.p)),
                    _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si), _i(st),
-                   LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), 0 if mode == "tape" else 1,
+                   LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), {"tape": 0, "dual": 1, "tape_wide": 2}[mode],
                    _d(loss), _d(dp), _d(du0), _d(dW), nthreads or default_threads())
     _check(rc, "grad")
     return {"loss": loss, "dp": dp, "du0": du0, "dW": dW}
@@ -228,3 +232,12 @@ def tsit5_tableau():
 
 def ros2_gamma() -> float:
     return float(lib().or_ros2_gamma())
+
+
+def ctrl_pow(x, y, dtype: str = "f64"):
+    """The step-size controller's power function x**y, element-wise."""
+    x = np.ascontiguousarray(x, np.float64).ravel()
+    y = np.broadcast_to(np.asarray(y, np.float64), x.shape).copy()
+    out = np.zeros_like(x)
+    lib().or_ctrl_pow(DTYPES[dtype], len(x), _d(x), _d(y), _d(out))
+    return out

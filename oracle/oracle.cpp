@@ -372,6 +372,55 @@ bool ros2_step(int sys, int d, const S* u, const S* p, S h, S* unew, S* err) {
 }
 
 // ---------------------------------------------------------------------------
+// Powers x^y for the step-size controller, computed from IEEE +, -, *, /, fma
+// and the exact frexp / ldexp / rint only, so that any implementation keeping
+// this operation order gets the same bits (a library pow may differ by an ulp,
+// and the embedded error estimate amplifies such differences; see DESIGN).
+//   ln x : x = m 2^e with m in [sqrt(1/2), sqrt(2)); ln m = 2 atanh(s),
+//          s = (m-1)/(m+1), by the series s (1 + z/3 + ... + z^12/25), z = s^2.
+//   exp w: Cody & Waite reduction w = k ln2 + r (ln2 split in a 21-bit head and
+//          a tail), |r| <= ln2/2, Taylor polynomial to r^14, then 2^k exactly.
+// Both polynomials are evaluated by Horner's rule with fused multiply-adds.
+// ---------------------------------------------------------------------------
+static const double CP_LN2_HI = 0.6931467056274414;      // ln 2, 21 significant bits
+static const double CP_LN2_LO = 4.7493250390316726e-07;  // ln 2 - CP_LN2_HI
+static const double CP_INV_LN2 = 1.4426950408889634;
+static const double CP_SQRT_HALF = 0.7071067811865476;
+
+template <class T>
+T ctrl_pow(T x, T y) {
+  if (std::isnan(x) || std::isnan(y)) return std::numeric_limits<T>::quiet_NaN();
+  if (x == T(0)) return y > T(0) ? T(0) : (y < T(0) ? std::numeric_limits<T>::infinity() : T(1));
+  if (std::isinf(x)) return y > T(0) ? x : (y < T(0) ? T(0) : T(1));
+  int e = 0;
+  T m = std::frexp(x, &e);
+  if (m < T(CP_SQRT_HALF)) {
+    m = m + m;
+    e = e - 1;
+  }
+  T s = (m - T(1)) / (m + T(1));
+  T z = s * s;
+  T poly = T(1.0 / 25.0);
+  for (int k = 11; k >= 0; --k) poly = std::fma(poly, z, T(1.0 / double(2 * k + 1)));
+  T lnm = (s + s) * poly;
+  T lnx = std::fma(T(e), T(CP_LN2_HI), std::fma(T(e), T(CP_LN2_LO), lnm));
+  T w = y * lnx;
+  T kf = std::rint(w * T(CP_INV_LN2));
+  if (kf > T(2000)) return std::numeric_limits<T>::infinity();
+  if (kf < T(-2000)) return T(0);
+  T r = std::fma(-kf, T(CP_LN2_HI), w);
+  r = std::fma(-kf, T(CP_LN2_LO), r);
+  // 1/j!, j = 14 .. 0
+  double fact = 87178291200.0;  // 14!
+  T p = T(1.0 / fact);
+  for (int j = 13; j >= 0; --j) {
+    fact = fact / double(j + 1);  // exact: j! is an integer below 2^53
+    p = std::fma(p, r, T(1.0 / fact));
+  }
+  return std::ldexp(p, int(kf));
+}
+
+// ---------------------------------------------------------------------------
 // Adaptive recorder (plain scalar T).
 //
 // Error norm: err = sqrt( (1/d) sum_c (e_c / sc_c)^2 ), sc_c = atol + rtol *
@@ -417,7 +466,7 @@ T initial_step(int sys, int method, int d, const T* u0, const T* p, const T* W, 
   for (int c = 0; c < d; ++c) df[c] = f1[c] - f0[c];
   T d2 = rms_scaled<T>(d, df, sc) / h0;
   T dm = std::max(d1, d2);
-  T h1 = dm <= T(1e-15) ? std::max(T(1e-6), h0 * T(1e-3)) : std::pow(T(0.01) / dm, T(1) / q);
+  T h1 = dm <= T(1e-15) ? std::max(T(1e-6), h0 * T(1e-3)) : ctrl_pow<T>(T(0.01) / dm, T(1) / q);
   return std::min(std::min(T(100) * h0, h1), t1 - t0);
 }
 
@@ -476,7 +525,7 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
       if (err == T(0)) {
         fac = T(10);
       } else {
-        fac = (T(0.9) * std::pow(err, -T(0.7) / q)) * std::pow(errprev, T(0.4) / q);
+        fac = (T(0.9) * ctrl_pow<T>(err, -T(0.7) / q)) * ctrl_pow<T>(errprev, T(0.4) / q);
         fac = std::min(T(10), std::max(T(0.2), fac));
       }
       if (prev_rej) fac = std::min(fac, T(1));
@@ -490,7 +539,7 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
         out.status = TRAJ_MAXSTEPS;
         return out;
       }
-      T fac = std::isnan(err) ? T(0.2) : std::max(T(0.2), T(0.9) * std::pow(err, -T(1) / q));
+      T fac = std::isnan(err) ? T(0.2) : std::max(T(0.2), T(0.9) * ctrl_pow<T>(err, -T(1) / q));
       hprop = fac * hprop;
       prev_rej = true;
     }
@@ -586,7 +635,9 @@ inline void gather_kd(const double* src, int nsave, int d, int64_t n, int64_t i,
 
 // Reverse-mode gradient of one trajectory with the tape.  Outputs: loss, dp
 // (np), du0 (d) and, for NODE64, accumulates dW (64*64) into dW_acc.
-template <class T>
+// A = the type the reverse sweep accumulates adjoints in (T, or long double
+// for a reference with 11 more bits; the tape's partials are the same).
+template <class T, class A = T>
 void grad_one_tape(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, double* loss, double* dp,
                    double* du0, double* dW_acc) {
   using R = Rv<T>;
@@ -616,18 +667,18 @@ void grad_one_tape(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, dou
                        Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave, Mh.save_idx + i * Mh.nsave, Ls.kind,
                        Ls.target ? tg.data() : nullptr, wg.data(), nullptr);
   *loss = double(L.v);
-  std::vector<T> adj(tp.nodes.size(), T(0));
-  if (L.id >= 0) adj[L.id] = T(1);
+  std::vector<A> adj(tp.nodes.size(), A(0));
+  if (L.id >= 0) adj[L.id] = A(1);
   for (int64_t k = (int64_t)tp.nodes.size() - 1; k >= 0; --k) {
     const Node<T>& nd = tp.nodes[k];
-    T a = adj[k];
-    if (a == T(0)) continue;
-    if (nd.a >= 0) adj[nd.a] += nd.da * a;
-    if (nd.b >= 0) adj[nd.b] += nd.db * a;
-    if (nd.c >= 0) adj[nd.c] += nd.dc * a;
+    A a = adj[k];
+    if (a == A(0)) continue;
+    if (nd.a >= 0) adj[nd.a] += A(nd.da) * a;
+    if (nd.b >= 0) adj[nd.b] += A(nd.db) * a;
+    if (nd.c >= 0) adj[nd.c] += A(nd.dc) * a;
   }
-  for (int c = 0; c < d; ++c) du0[c] = double(u0[c].id >= 0 ? adj[u0[c].id] : T(0));
-  for (int c = 0; c < np; ++c) dp[c] = double(p[c].id >= 0 ? adj[p[c].id] : T(0));
+  for (int c = 0; c < d; ++c) du0[c] = double(u0[c].id >= 0 ? adj[u0[c].id] : A(0));
+  for (int c = 0; c < np; ++c) dp[c] = double(p[c].id >= 0 ? adj[p[c].id] : A(0));
   if (dW_acc)
     for (int c = 0; c < 64 * 64; ++c) dW_acc[c] += double(adj[W[c].id]);
 }
@@ -736,6 +787,9 @@ int or_record(int sys, int method, int dtype, int64_t n, int d, int np, const do
 
 // Gradient of the replay loss.  mode 0: reverse-mode tape.  mode 1: forward
 // mode, one dual-number pass per input direction (p and u0 only; not NODE64).
+// mode 2: the tape with adjoints accumulated in a wider type (long double for
+// fp64 runs, double for fp32 runs): same forward values and partials, less
+// rounding in the reverse sweep.
 // Trajectories with status != 0 get NaN outputs.  dW (NODE64) is the sum over
 // trajectories, accumulated per thread chunk and then in chunk order.
 int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
@@ -746,6 +800,7 @@ int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const doub
   int rc = check_prob(P);
   if (rc) return rc;
   if (mode == 1 && sys == SYS_NODE64) return -4;
+  if (mode < 0 || mode > 2) return -1;
   Mesh Mh{smax, nsave, h, nsteps, save_idx};
   Loss Ls{loss_kind, target, weight};
   int nt = std::max(1, nthreads);
@@ -761,12 +816,16 @@ int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const doub
         continue;
       }
       double L;
-      if (mode == 0) {
+      if (mode == 0 || mode == 2) {
         double* acc = sys == SYS_NODE64 ? dWp[tid].data() : nullptr;
-        if (dtype == DT_F64)
+        if (dtype == DT_F64 && mode == 0)
           grad_one_tape<double>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
-        else
+        else if (dtype == DT_F64)
+          grad_one_tape<double, long double>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
+        else if (mode == 0)
           grad_one_tape<float>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
+        else
+          grad_one_tape<float, double>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
       } else {
         // unit directions: the basis vectors of p, then of u0
         L = dtype == DT_F64 ? loss_one<double>(P, Mh, Ls, i, nullptr) : loss_one<float>(P, Mh, Ls, i, nullptr);
@@ -896,5 +955,11 @@ void or_tsit5_tableau(double* c, double* A, double* bt) {
 }
 
 double or_ros2_gamma(void) { return ROS2_GAMMA; }
+
+// The controller's power function, element-wise (dtype 2: double, 1: float).
+void or_ctrl_pow(int dtype, int64_t n, const double* x, const double* y, double* out) {
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = dtype == DT_F64 ? ctrl_pow<double>(x[i], y[i]) : double(ctrl_pow<float>(float(x[i]), float(y[i])));
+}
 
 }  // extern "C"

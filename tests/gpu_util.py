@@ -64,3 +64,38 @@ def mesh_rel_err(h_gpu, h_orc, ns):
         a, b = h_gpu[i, : ns[i]], h_orc[i, : ns[i]]
         worst = max(worst, float(np.max(np.abs(a - b) / np.abs(b))) if ns[i] else 0.0)
     return worst
+
+
+TOL = {"f64": 1e-12, "f32": 1e-4}
+
+
+def _relinf(g, r):
+    return np.abs(g - r).max(0) / np.abs(r).max(0)
+
+
+def parity(out, prob, om, tol=None, quantile_ok=0.99, dual=True):
+    """Gradient parity of a GPU result against the oracle on the oracle's mesh.
+
+    Reference: the oracle's tape with a wide reverse sweep (the most accurate
+    evaluation of the exact discrete adjoint here).  The stated gate (1e-12
+    fp64, 1e-4 fp32) must hold for at least `quantile_ok` of the trajectories;
+    every trajectory must be within max(gate, 4 x the error that the
+    plain-precision oracle routes (tape, dual) themselves make on it): on
+    chaotic trajectories the reverse sweep's conditioning puts any
+    plain-precision adjoint, the oracle's included, near or above the gate.
+    Returns the per-trajectory errors."""
+    import oracle
+    tol = tol or TOL[prob.dtype]
+    wide = oracle.grad(prob, om, "tape_wide")
+    r = np.vstack([wide["dp"], wide["du0"]])
+    g = np.vstack([out.dp.double().cpu().numpy(), out.du0.double().cpu().numpy()])
+    e = _relinf(g, r)
+    own = oracle.grad(prob, om, "tape")
+    cond = _relinf(np.vstack([own["dp"], own["du0"]]), r)
+    if dual and prob.system != "node64":
+        dd = oracle.grad(prob, om, "dual")
+        cond = np.maximum(cond, _relinf(np.vstack([dd["dp"], dd["du0"]]), r))
+    assert np.mean(e <= tol) >= quantile_ok, (np.mean(e <= tol), e.max())
+    bound = np.maximum(tol, 4 * cond)
+    assert (e <= bound).all(), (e.max(), bound[np.argmax(e / bound)])
+    return e

@@ -8,13 +8,10 @@ import torch
 import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
-from gpu_util import (dev, ensemble, grad_rel_err, loss_args, mesh_by_trajectory, mesh_from_oracle,
-                      mesh_rel_err, tens)
+from gpu_util import (TOL, dev, ensemble, grad_rel_err, loss_args, mesh_by_trajectory, mesh_from_oracle,
+                      mesh_rel_err, parity, tens)
 
 pytestmark = pytest.mark.gpu
-
-TOL = {"f64": 1e-12, "f32": 1e-4}
-
 
 def _record_gpu(prob, smax):
     ens = ensemble(prob)
@@ -63,6 +60,7 @@ def test_grad_on_oracle_mesh(small, perm):
     torch.cuda.synchronize()
     e = grad_rel_err(out, og)
     assert e.max() <= TOL["f64"], e.max()
+    parity(out, prob, om, quantile_ok=1.0)
     le = np.abs(out.loss.cpu().numpy() - og["loss"]) / np.abs(og["loss"])
     assert le.max() <= 1e-14, le.max()  # the forward replay follows the same contract
 
@@ -91,7 +89,6 @@ def test_lorenz_1m_shape(dtype, n):
     """Ten save points with targets, t in [0, 10]; n not a multiple of the block."""
     prob = W.lorenz_1m(n, dtype=dtype)
     om = oracle.record(prob, 1024)
-    og = oracle.grad(prob, om)
     assert (om.status == 0).all()
     ens, mesh = _record_gpu(prob, 1024)
     h, ns, si, st, order = mesh_by_trajectory(mesh)
@@ -100,12 +97,12 @@ def test_lorenz_1m_shape(dtype, n):
         assert np.array_equal(ns, om.nsteps)
         assert mesh_rel_err(h, om.h, ns) <= 1e-10
     else:
-        # fp32: libm pow may differ by an ulp; counts agree for nearly all
-        assert (ns == om.nsteps).mean() >= 0.99
+        # fp32 records follow the same contract in single precision
+        assert np.array_equal(ns, om.nsteps)
+        assert mesh_rel_err(h, om.h, ns) <= 1e-5
     out = gs.gs_grad(ens, mesh_from_oracle(om, dtype), **loss_args(prob))
     torch.cuda.synchronize()
-    e = grad_rel_err(out, og)
-    assert e.max() <= TOL[dtype], (dtype, e.max())
+    parity(out, prob, om)
 
 
 def test_full_size_sampled():
@@ -124,7 +121,6 @@ def test_full_size_sampled():
     idx = np.unique(np.concatenate([rng.choice(prob.n, 384, replace=False), np.argsort(ns_all)[-32:]]))
     sub = prob.subset(idx)
     om = oracle.record(sub, 2048)
-    og = oracle.grad(sub, om)
     # mesh parity on the sample
     order = mesh.order.cpu().numpy()
     inv = np.empty_like(order)
@@ -144,9 +140,7 @@ def test_full_size_sampled():
     mesh.save_idx[:, ts] = tens(om.save_idx.T.astype(np.int32), torch.int32)
     out = gs.gs_grad(ens, mesh, **loss_args(prob))
     torch.cuda.synchronize()
-    g = np.vstack([out.dp[:, torch.tensor(idx, device=dev())].cpu().numpy(),
-                   out.du0[:, torch.tensor(idx, device=dev())].cpu().numpy()])
-    r = np.vstack([og["dp"], og["du0"]])
-    e = np.abs(g - r).max(0) / np.abs(r).max(0)
-    assert e.max() <= TOL["f64"], e.max()
+    ti = torch.tensor(idx, device=dev())
+    sub_out = gs.GradOut(out.loss[ti], out.dp[:, ti], out.du0[:, ti], None)
+    parity(sub_out, sub, om)
     assert torch.isfinite(out.dp).all() and torch.isfinite(out.du0).all()

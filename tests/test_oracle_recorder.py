@@ -133,3 +133,26 @@ def test_step_operation_counts():
     assert r == {"add": 7, "mul": 18, "fma": 38, "div": 9, "sqrt": 0, "tanh": 0}
     nd = oracle.count_step("node64", "tsit5", 64, 64)
     assert nd["fma"] == 6 * 64 * 64 + 64 * 21 and nd["tanh"] == 6 * 64
+
+
+def test_controller_power_function():
+    """The controller's x**y (exp/log from IEEE operations only) against the
+    library power function: <= 4 ulp on the controller's arguments (errors
+    1e-4..1e3, exponents of magnitude <= 1), <= 1e-12 relative anywhere in
+    [1e-300, 1e300], exact special values."""
+    rng = np.random.default_rng(0)
+    x = 10.0 ** rng.uniform(-4, 3, 100000)
+    for y in (-0.14, 0.08, -0.2, 0.2, -0.35, 0.2, -0.5):
+        c = oracle.ctrl_pow(x, y)
+        r = np.power(x, y)
+        assert np.max(np.abs(c - r) / r) <= 4 * EPS
+    x = np.exp(rng.uniform(-690, 690, 100000))
+    y = rng.uniform(-1, 1, 100000)
+    c, r = oracle.ctrl_pow(x, y), np.power(x, y)
+    assert np.max(np.abs(c - r) / r) <= 1e-12
+    x32 = rng.uniform(1e-4, 1e3, 20000).astype(np.float32).astype(np.float64)
+    c = oracle.ctrl_pow(x32, -0.14, "f32")
+    r = np.power(x32.astype(np.float32), np.float32(-0.14)).astype(np.float64)
+    assert np.max(np.abs(c - r) / r) <= 4 * np.finfo(np.float32).eps
+    s = oracle.ctrl_pow([0.0, 0.0, np.inf, 1.0, 2.0], [0.2, -0.2, -0.2, 0.7, 0.0])
+    assert s[0] == 0 and np.isinf(s[1]) and s[2] == 0 and s[3] == 1 and s[4] == 1
