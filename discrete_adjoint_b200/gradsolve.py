@@ -74,6 +74,10 @@ _lib.gs_solve.restype = ctypes.c_int32
 _lib.gs_grad.argtypes = [_P(_Problem), _P(_Mesh), _P(_Loss), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.gs_grad.restype = ctypes.c_int32
+_lib.gs_grad_static.argtypes = [_P(_Problem), _P(_Mesh), _P(_Loss), ctypes.c_void_p, ctypes.c_void_p,
+                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+_lib.gs_grad_static.restype = ctypes.c_int32
+STATIC_SCRATCH_BYTES = 32 << 20
 _lib.gs_status_string.argtypes = [ctypes.c_int32]
 _lib.gs_status_string.restype = ctypes.c_char_p
 _lib.gs_launch_count.argtypes = []
@@ -254,4 +258,19 @@ def gs_grad(ens: Ensemble, mesh: Mesh, loss: str = "sumsq", target=None, weight=
         ws = workspace(need, ens.u0.device)
     _check(_lib.gs_grad(ctypes.byref(ps), ctypes.byref(ms), ctypes.byref(ls), _ptr(out.loss), _ptr(out.dp),
                         _ptr(out.du0), _ptr(out.dshared), _ptr(ws), ws.numel(), _stream(stream)), "gs_grad")
+    return out
+
+
+def gs_grad_static(ens: Ensemble, mesh: Mesh, loss: str = "sumsq", target=None, weight=None,
+                   out: GradOut | None = None, stream=None) -> GradOut:
+    """gs_grad for callers that cannot allocate device memory: the checkpoints
+    go to the library's own 32 MiB device array (problems that need more are
+    rejected; calls that overlap on the GPU race)."""
+    if out is None:
+        out = new_grad_out(ens)
+    ps, ms = ens._struct(), mesh._struct()
+    ls = _Loss(LOSSES[loss], None if target is None else target.data_ptr(),
+               None if weight is None else weight.data_ptr())
+    _check(_lib.gs_grad_static(ctypes.byref(ps), ctypes.byref(ms), ctypes.byref(ls), _ptr(out.loss), _ptr(out.dp),
+                               _ptr(out.du0), _ptr(out.dshared), _stream(stream)), "gs_grad_static")
     return out

@@ -201,6 +201,27 @@ GS_API gs_status gs_solve(const gs_problem* prob, const gs_mesh* mesh, void* u_s
 GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_loss* loss_desc, void* loss, void* dp,
                   void* du0, void* dshared, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * gs_grad without a caller workspace, for callers that cannot allocate device
+ * memory (a plugin whose host application owns all device memory, a real-time
+ * loop that may not call cudaMalloc, a C host without an allocator).  Same
+ * arguments, results and validation as gs_grad, minus ws / ws_bytes: the
+ * checkpoints go to a library-owned device array of GS_STATIC_SCRATCH_BYTES
+ * (32 MiB), which every GPU that loads the library holds until exit.
+ *  - Problems whose gs_grad workspace exceeds GS_STATIC_SCRATCH_BYTES return
+ *    GS_EWORKSPACE (d=3, fp64: smax * n <= 1,398,101, e.g. 1,024 trajectories
+ *    of up to 1,365 steps).
+ *  - All calls share the array: calls that overlap on the GPU race.  It keeps
+ *    the last call's contents; nothing in it needs clearing between calls.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ * No counterpart in the paper.
+ */
+#define GS_STATIC_SCRATCH_BYTES (32u << 20)
+GS_API gs_status gs_grad_static(const gs_problem* prob, const gs_mesh* mesh, const gs_loss* loss_desc, void* loss,
+                                void* dp, void* du0, void* dshared, void* stream);
+
 /* Static description of a status code. */
 GS_API const char* gs_status_string(gs_status status);
 
