@@ -31,15 +31,18 @@ def stale() -> bool:
     return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
+    """Compile every csrc/*.cu and link libgradsolve.so (skipped when fresh).
+    extra_flags: additional nvcc flags (e.g. -D tuning macros) for a forced
+    rebuild."""
+    if not force and not extra_flags and not stale():
         return LIB
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in SOURCES:
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
-        cmd = [_nvcc(), *NVCC_FLAGS, "-c", src, "-o", obj]
+        cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)
@@ -52,4 +55,5 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose=True))
+    import sys
+    print(build(force=True, verbose=True, extra_flags=sys.argv[1:]))

@@ -14,7 +14,7 @@ void count_launch(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
 // kernels (defined in the other translation units)
 gs_status count3(const gs_problem*, const gs_tol*, int32_t, int32_t*, int32_t*, cudaStream_t);
 gs_status record3(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
-size_t record_ws_bytes(int64_t n, int32_t smax);
+size_t record_ws_bytes(int64_t n, int32_t smax, int32_t nsave, size_t tsize);
 template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                                    cudaStream_t);
@@ -85,7 +85,7 @@ int64_t gs_launch_count(void) { return g_launches.load(); }
 
 size_t gs_workspace_bytes(const gs_problem* P, const gs_mesh* M, int32_t op) {
   if (check_problem(P) != GS_OK || !M || M->smax < 1) return 0;
-  if (op == GS_OP_RECORD) return record_ws_bytes(P->n, M->smax);
+  if (op == GS_OP_RECORD) return record_ws_bytes(P->n, M->smax, P->nsave, dsize(P));
   if (op == GS_OP_GRAD) return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
   return 0;
 }

@@ -190,6 +190,11 @@ __device__ __forceinline__ void lu3_solve_T(const T LU[9], const int P[3], T b0,
   x2 = P[0] == 2 ? z0 : (P[1] == 2 ? z1 : z2);
 }
 
+// Bring the line holding *p into L2 ahead of its use (no register, no wait).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ---------------------------------------------------------------------------
 // Host-side helpers.
 // ---------------------------------------------------------------------------

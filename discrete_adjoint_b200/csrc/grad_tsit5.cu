@@ -1,16 +1,16 @@
 // grad_tsit5.cu -- fused fixed-step replay + reverse sweep (the discrete
-// adjoint) for Tsit5 on the Lorenz system, one thread per trajectory slot.
+// adjoint) for Tsit5 on the Lorenz system.
 //
 // GRADSOLVE (arXiv 2609.02876), evolve.pub review "Summary" and "Strengths:
 // precisely scoped exactness claim": the gradient is the exact derivative of
 // the fixed-step replay of the recorded steps, the mesh held as data.
 //
-// Forward half: for s < S_j replay step s with h[s][j] (the forward arithmetic
+// Forward half: for s < S replay step s with h[s] (the forward arithmetic
 // follows the floating-point contract, so it is bitwise equal to any replay
 // that keeps the same operation order), store the state u_s to the checkpoint
-// workspace ck[s][c][j], and add the loss terms at the save points.
+// workspace ck[s][c][slot], and add the loss terms at the save points.
 //
-// Reverse half: for s = S_j-1 .. 0, reload u_s, recompute the stage states
+// Reverse half: for s = S-1 .. 0, reload u_s, recompute the stage states
 // U_1..U_6 of step s, and apply the transposed step.  With
 //   u_{s+1} = u_s + h sum_j b_j k_j,  k_j = f(U_j),  U_j = u_s + h sum_{m<j} a_jm k_m
 // and lambda = dL/du_{s+1}:
@@ -21,13 +21,42 @@
 // for j = 6 .. 1 (b_7 = 0, so the FSAL stage drops out).  Loss gradients enter
 // lambda at the save points.  Output: dL/dp = pbar, dL/du0 = lambda.
 //
+// Execution: the kernel is bound by the FP64 pipe, and one Lorenz trajectory
+// offers only three independent chains (x, y, z) per instruction stream, which
+// leaves the pipe idle a quarter of the time at the occupancy its registers
+// allow.  Each thread therefore carries K adjacent slots (vec<T, K>), giving 3K
+// independent chains.  gs_record orders slots by decreasing step count, so the
+// K chains of a thread (and the 32K of a warp) have nearly equal length; the
+// shorter ones run the remaining iterations as steps of size 0, which are
+// exact identities in both halves (u + 0 * acc = u; nu = 0 * (...) = 0), so the
+// results are bitwise those of one slot per thread.
+//
 // Memory layout: h [smax][n] and ck [smax][3][n] are step-major over slots, so
-// at a given step the 32 threads of a warp touch 32 consecutive elements
-// (256 B in fp64) of every array; gs_record orders slots by step count, so the
-// threads of a warp also run chains of (nearly) equal length.
-#include "common.cuh"
+// at a given step a warp touches 32K consecutive elements of every array.
+// Loads run one step ahead in registers and several steps ahead into L2.
+#include "vec.cuh"
 
 namespace gs {
+
+#ifndef GS_GRAD_K
+#define GS_GRAD_K 1
+#endif
+#ifndef GS_GRAD_BS
+#define GS_GRAD_BS 128
+#endif
+#ifndef GS_GRAD_MINB
+#define GS_GRAD_MINB (GS_GRAD_K == 1 ? 4 : 2)
+#endif
+#ifndef GS_PF_F
+#define GS_PF_F 8
+#endif
+#ifndef GS_PF_R
+#define GS_PF_R 4
+#endif
+// L2 prefetch distances in steps (a warp's forward step takes ~0.5 us and its
+// reverse step ~1 us, against a DRAM latency of ~1 us under load).
+constexpr int kPrefetchF = GS_PF_F;
+constexpr int kPrefetchR = GS_PF_R;
 
 template <typename T>
 struct TsitLorenzArgs {
@@ -51,10 +80,11 @@ struct TsitLorenzArgs {
 };
 
 // dL/dU = J(U)^T nu and pbar += f_p(U)^T nu for Lorenz.
-template <typename T>
-__device__ __forceinline__ void lorenz_vjp(T ux, T uy, T uz, T s, T r, T b, T nx, T ny, T nz, T& mx, T& my,
-                                           T& mz, T& ps, T& pr, T& pb) {
-  T m = s * nx;
+template <typename V>
+__device__ __forceinline__ void lorenz_vjp(const V& ux, const V& uy, const V& uz, const V& s, const V& r, const V& b,
+                                           const V& nx, const V& ny, const V& nz, V& mx, V& my, V& mz, V& ps, V& pr,
+                                           V& pb) {
+  V m = s * nx;
   mx = fmaT(r - uz, ny, fmaT(uy, nz, -m));
   my = fmaT(ux, nz, m - ny);
   mz = -fmaT(ux, ny, b * nz);
@@ -69,263 +99,272 @@ __device__ __forceinline__ void lorenz_vjp(T ux, T uy, T uz, T s, T r, T b, T nx
   UY = fmaT(h, AY, y);                   \
   UZ = fmaT(h, AZ, z);
 
-template <typename T>
-__global__ void __launch_bounds__(128, 4) k_grad_tsit5_lorenz(TsitLorenzArgs<T> a) {
+// acc = a1 k1 (+ a2 k2 ...) for the three components, in the contract's order.
+#define GS_ACC1(A1, K1)    \
+  ax = cst<T>(A1) * K1##x; \
+  ay = cst<T>(A1) * K1##y; \
+  az = cst<T>(A1) * K1##z;
+#define GS_ACCN(AN, KN)             \
+  ax = fmaT(cst<T>(AN), KN##x, ax); \
+  ay = fmaT(cst<T>(AN), KN##y, ay); \
+  az = fmaT(cst<T>(AN), KN##z, az);
+
+template <typename T, int K>
+__global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(TsitLorenzArgs<T> a) {
+  using V = vec<T, K>;
   const int64_t n = a.n;
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= n) return;
-  const int64_t i = a.order[j];
-  if (i < 0 || i >= n) return;  // not a permutation entry: nothing to write
-  const int S = a.nsteps[j];
-  if (a.status[j] != GS_TRAJ_OK || S < 0 || S > a.smax) {
-    const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
-    a.loss[i] = nan;
-#pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      a.dp[c * n + i] = nan;
-      a.du0[c * n + i] = nan;
-    }
-    return;
-  }
-  const T s = a.p[i], r = a.p[n + i], b = a.p[2 * n + i];
-  T x = a.u0[i], y = a.u0[n + i], z = a.u0[2 * n + i];
-  const T* __restrict__ hp = a.h + j;
-  T* __restrict__ cp = a.ck + j;
   const int64_t n3 = 3 * n;
+  const int64_t j0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * K;
+  if (j0 >= n) return;
+  const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
+
+  // per-slot set-up; inactive slots (past n, failed, malformed) run no steps
+  int64_t i[K];
+  int S[K];
+  int Smax = 0;
+  V s, r, b, x, y, z;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    const int64_t j = j0 + q;
+    i[q] = -1;
+    S[q] = 0;
+    s.e[q] = r.e[q] = b.e[q] = x.e[q] = y.e[q] = z.e[q] = cst<T>(0.0);
+    if (j < n) {
+      const int64_t ii = a.order[j];
+      if (ii >= 0 && ii < n) {
+        const int sq = a.nsteps[j];
+        if (a.status[j] != GS_TRAJ_OK || sq < 0 || sq > a.smax) {
+          a.loss[ii] = nan;
+#pragma unroll
+          for (int c = 0; c < 3; ++c) {
+            a.dp[c * n + ii] = nan;
+            a.du0[c * n + ii] = nan;
+          }
+        } else {
+          i[q] = ii;
+          S[q] = sq;
+          Smax = sq > Smax ? sq : Smax;
+          s.e[q] = a.p[ii];
+          r.e[q] = a.p[n + ii];
+          b.e[q] = a.p[2 * n + ii];
+          x.e[q] = a.u0[ii];
+          y.e[q] = a.u0[n + ii];
+          z.e[q] = a.u0[2 * n + ii];
+        }
+      }
+    }
+  }
+  const T* __restrict__ hp = a.h + j0;
+  T* __restrict__ cp = a.ck + j0;
 
   // ---------------------------------------------------------------- forward
-  T L = cst<T>(0.0);
-  int kk = 0;
-  int next = a.save_idx[j];
-  T k1x, k1y, k1z;
+  V L = vsplat<T, K>(cst<T>(0.0));
+  int kk[K], next[K];
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    kk[q] = 0;
+    next[q] = S[q] > 0 ? a.save_idx[j0 + q] : -1;
+  }
+  V k1x, k1y, k1z;
   lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);
-  T hn = S > 0 ? hp[0] : cst<T>(0.0);
-  for (int st = 0; st < S; ++st) {
-    const T h = hn;
-    if (st + 1 < S) hn = hp[(int64_t)(st + 1) * n];
-    cp[0] = x;
-    cp[n] = y;
-    cp[2 * n] = z;
+  V hn;
+#pragma unroll
+  for (int q = 0; q < K; ++q) hn.e[q] = 0 < S[q] ? hp[q] : cst<T>(0.0);
+  const T* hq = hp + n;                        // h of step st + 1
+  const T* hf = hp + (int64_t)kPrefetchF * n;  // h of step st + kPrefetchF
+  for (int st = 0; st < Smax; ++st) {
+    const V h = hn;
+    if (st + kPrefetchF < Smax) prefetch_l2(hf);
+    hf += n;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      hn.e[q] = st + 1 < S[q] ? hq[q] : cst<T>(0.0);
+      if (st < S[q]) {
+        cp[q] = x.e[q];
+        cp[n + q] = y.e[q];
+        cp[2 * n + q] = z.e[q];
+      }
+    }
+    hq += n;
     cp += n3;
-    T ax, ay, az, Ux, Uy, Uz;
-    // stage 2
-    ax = cst<T>(TS_A21) * k1x;
-    ay = cst<T>(TS_A21) * k1y;
-    az = cst<T>(TS_A21) * k1z;
+    V ax, ay, az, Ux, Uy, Uz;
+    GS_ACC1(TS_A21, k1)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
-    T k2x, k2y, k2z;
+    V k2x, k2y, k2z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k2x, k2y, k2z);
-    // stage 3
-    ax = cst<T>(TS_A31) * k1x;
-    ay = cst<T>(TS_A31) * k1y;
-    az = cst<T>(TS_A31) * k1z;
-    ax = fmaT(cst<T>(TS_A32), k2x, ax);
-    ay = fmaT(cst<T>(TS_A32), k2y, ay);
-    az = fmaT(cst<T>(TS_A32), k2z, az);
+    GS_ACC1(TS_A31, k1)
+    GS_ACCN(TS_A32, k2)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
-    T k3x, k3y, k3z;
+    V k3x, k3y, k3z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k3x, k3y, k3z);
-    // stage 4
-    ax = cst<T>(TS_A41) * k1x;
-    ay = cst<T>(TS_A41) * k1y;
-    az = cst<T>(TS_A41) * k1z;
-    ax = fmaT(cst<T>(TS_A42), k2x, ax);
-    ay = fmaT(cst<T>(TS_A42), k2y, ay);
-    az = fmaT(cst<T>(TS_A42), k2z, az);
-    ax = fmaT(cst<T>(TS_A43), k3x, ax);
-    ay = fmaT(cst<T>(TS_A43), k3y, ay);
-    az = fmaT(cst<T>(TS_A43), k3z, az);
+    GS_ACC1(TS_A41, k1)
+    GS_ACCN(TS_A42, k2)
+    GS_ACCN(TS_A43, k3)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
-    T k4x, k4y, k4z;
+    V k4x, k4y, k4z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k4x, k4y, k4z);
-    // stage 5
-    ax = cst<T>(TS_A51) * k1x;
-    ay = cst<T>(TS_A51) * k1y;
-    az = cst<T>(TS_A51) * k1z;
-    ax = fmaT(cst<T>(TS_A52), k2x, ax);
-    ay = fmaT(cst<T>(TS_A52), k2y, ay);
-    az = fmaT(cst<T>(TS_A52), k2z, az);
-    ax = fmaT(cst<T>(TS_A53), k3x, ax);
-    ay = fmaT(cst<T>(TS_A53), k3y, ay);
-    az = fmaT(cst<T>(TS_A53), k3z, az);
-    ax = fmaT(cst<T>(TS_A54), k4x, ax);
-    ay = fmaT(cst<T>(TS_A54), k4y, ay);
-    az = fmaT(cst<T>(TS_A54), k4z, az);
+    GS_ACC1(TS_A51, k1)
+    GS_ACCN(TS_A52, k2)
+    GS_ACCN(TS_A53, k3)
+    GS_ACCN(TS_A54, k4)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
-    T k5x, k5y, k5z;
+    V k5x, k5y, k5z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k5x, k5y, k5z);
-    // stage 6
-    ax = cst<T>(TS_A61) * k1x;
-    ay = cst<T>(TS_A61) * k1y;
-    az = cst<T>(TS_A61) * k1z;
-    ax = fmaT(cst<T>(TS_A62), k2x, ax);
-    ay = fmaT(cst<T>(TS_A62), k2y, ay);
-    az = fmaT(cst<T>(TS_A62), k2z, az);
-    ax = fmaT(cst<T>(TS_A63), k3x, ax);
-    ay = fmaT(cst<T>(TS_A63), k3y, ay);
-    az = fmaT(cst<T>(TS_A63), k3z, az);
-    ax = fmaT(cst<T>(TS_A64), k4x, ax);
-    ay = fmaT(cst<T>(TS_A64), k4y, ay);
-    az = fmaT(cst<T>(TS_A64), k4z, az);
-    ax = fmaT(cst<T>(TS_A65), k5x, ax);
-    ay = fmaT(cst<T>(TS_A65), k5y, ay);
-    az = fmaT(cst<T>(TS_A65), k5z, az);
+    GS_ACC1(TS_A61, k1)
+    GS_ACCN(TS_A62, k2)
+    GS_ACCN(TS_A63, k3)
+    GS_ACCN(TS_A64, k4)
+    GS_ACCN(TS_A65, k5)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
-    T k6x, k6y, k6z;
+    V k6x, k6y, k6z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k6x, k6y, k6z);
     // stage 7 = u_{s+1}
-    ax = cst<T>(TS_B1) * k1x;
-    ay = cst<T>(TS_B1) * k1y;
-    az = cst<T>(TS_B1) * k1z;
-    ax = fmaT(cst<T>(TS_B2), k2x, ax);
-    ay = fmaT(cst<T>(TS_B2), k2y, ay);
-    az = fmaT(cst<T>(TS_B2), k2z, az);
-    ax = fmaT(cst<T>(TS_B3), k3x, ax);
-    ay = fmaT(cst<T>(TS_B3), k3y, ay);
-    az = fmaT(cst<T>(TS_B3), k3z, az);
-    ax = fmaT(cst<T>(TS_B4), k4x, ax);
-    ay = fmaT(cst<T>(TS_B4), k4y, ay);
-    az = fmaT(cst<T>(TS_B4), k4z, az);
-    ax = fmaT(cst<T>(TS_B5), k5x, ax);
-    ay = fmaT(cst<T>(TS_B5), k5y, ay);
-    az = fmaT(cst<T>(TS_B5), k5z, az);
-    ax = fmaT(cst<T>(TS_B6), k6x, ax);
-    ay = fmaT(cst<T>(TS_B6), k6y, ay);
-    az = fmaT(cst<T>(TS_B6), k6z, az);
+    GS_ACC1(TS_B1, k1)
+    GS_ACCN(TS_B2, k2)
+    GS_ACCN(TS_B3, k3)
+    GS_ACCN(TS_B4, k4)
+    GS_ACCN(TS_B5, k5)
+    GS_ACCN(TS_B6, k6)
     x = fmaT(h, ax, x);
     y = fmaT(h, ay, y);
     z = fmaT(h, az, z);
     lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);  // FSAL: next step's first slope
-    if (st + 1 == next) {
-      const int64_t o = (int64_t)kk * n3 + i;
-      if (a.loss_kind == GS_LOSS_SUMSQ) {
-        T dx = a.target ? x - a.target[o] : x;
-        T dy = a.target ? y - a.target[o + n] : y;
-        T dz = a.target ? z - a.target[o + 2 * n] : z;
-        L = fmaT(dx, dx, L);
-        L = fmaT(dy, dy, L);
-        L = fmaT(dz, dz, L);
-      } else {
-        L = fmaT(a.weight[o], x, L);
-        L = fmaT(a.weight[o + n], y, L);
-        L = fmaT(a.weight[o + 2 * n], z, L);
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      if (st + 1 == next[q]) {
+        const int64_t o = (int64_t)kk[q] * n3 + i[q];
+        T Lq = L.e[q];
+        if (a.loss_kind == GS_LOSS_SUMSQ) {
+          const T dx = a.target ? x.e[q] - a.target[o] : x.e[q];
+          const T dy = a.target ? y.e[q] - a.target[o + n] : y.e[q];
+          const T dz = a.target ? z.e[q] - a.target[o + 2 * n] : z.e[q];
+          Lq = fmaT(dx, dx, Lq);
+          Lq = fmaT(dy, dy, Lq);
+          Lq = fmaT(dz, dz, Lq);
+        } else {
+          Lq = fmaT(a.weight[o], x.e[q], Lq);
+          Lq = fmaT(a.weight[o + n], y.e[q], Lq);
+          Lq = fmaT(a.weight[o + 2 * n], z.e[q], Lq);
+        }
+        L.e[q] = Lq;
+        ++kk[q];
+        next[q] = kk[q] < a.nsave ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
       }
-      ++kk;
-      next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
     }
   }
+#pragma unroll
+  for (int q = 0; q < K; ++q)
+    if (i[q] >= 0) a.loss[i[q]] = L.e[q];
 
   // ---------------------------------------------------------------- reverse
-  T lx = cst<T>(0.0), ly = cst<T>(0.0), lz = cst<T>(0.0);
-  T ps = cst<T>(0.0), pr = cst<T>(0.0), pb = cst<T>(0.0);
-  kk = a.nsave - 1;
-  next = a.save_idx[(int64_t)kk * n + j];
-  // u_{s+1} for the save-point test of step s; prefetched u_s and h_s
-  T nx = x, ny = y, nz = z;
-  T cx = cst<T>(0.0), cy = cst<T>(0.0), cz = cst<T>(0.0), hc = cst<T>(0.0);
-  if (S > 0) {
-    cp -= n3;
-    cx = cp[0];
-    cy = cp[n];
-    cz = cp[2 * n];
-    hc = hp[(int64_t)(S - 1) * n];
+  // At the top of iteration st, (x, y, z) holds u_{st+1} (the final state
+  // first, then the state loaded by the previous iteration), which is what the
+  // save-point test needs; (cx, cy, cz, hc) are the prefetched u_st and h_st.
+  V lx = vsplat<T, K>(cst<T>(0.0)), ly = lx, lz = lx;
+  V ps = lx, pr = lx, pb = lx;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    kk[q] = a.nsave - 1;
+    next[q] = S[q] > 0 ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
   }
-  for (int st = S - 1; st >= 0; --st) {
-    if (st + 1 == next) {
-      const int64_t o = (int64_t)kk * n3 + i;
-      if (a.loss_kind == GS_LOSS_SUMSQ) {
-        T dx = a.target ? nx - a.target[o] : nx;
-        T dy = a.target ? ny - a.target[o + n] : ny;
-        T dz = a.target ? nz - a.target[o + 2 * n] : nz;
-        lx = fmaT(cst<T>(2.0), dx, lx);
-        ly = fmaT(cst<T>(2.0), dy, ly);
-        lz = fmaT(cst<T>(2.0), dz, lz);
-      } else {
-        lx += a.weight[o];
-        ly += a.weight[o + n];
-        lz += a.weight[o + 2 * n];
+  V cx = x, cy = y, cz = z, hc = vsplat<T, K>(cst<T>(0.0));
+  const T* hq2 = hp + (int64_t)(Smax - 1) * n;  // h of the step being loaded
+  if (Smax > 0) {
+    cp -= n3;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      if (Smax - 1 < S[q]) {
+        cx.e[q] = cp[q];
+        cy.e[q] = cp[n + q];
+        cz.e[q] = cp[2 * n + q];
+        hc.e[q] = hq2[q];
       }
-      --kk;
-      next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
+    }
+  }
+  for (int st = Smax - 1; st >= 0; --st) {
+    if (st >= kPrefetchR) {
+      const T* c = cp - (int64_t)kPrefetchR * n3;
+      prefetch_l2(c);
+      prefetch_l2(c + n);
+      prefetch_l2(c + 2 * n);
+      prefetch_l2(hq2 - (int64_t)kPrefetchR * n);
+    }
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      if (st + 1 == next[q]) {
+        const int64_t o = (int64_t)kk[q] * n3 + i[q];
+        if (a.loss_kind == GS_LOSS_SUMSQ) {
+          const T dx = a.target ? x.e[q] - a.target[o] : x.e[q];
+          const T dy = a.target ? y.e[q] - a.target[o + n] : y.e[q];
+          const T dz = a.target ? z.e[q] - a.target[o + 2 * n] : z.e[q];
+          lx.e[q] = fmaT(cst<T>(2.0), dx, lx.e[q]);
+          ly.e[q] = fmaT(cst<T>(2.0), dy, ly.e[q]);
+          lz.e[q] = fmaT(cst<T>(2.0), dz, lz.e[q]);
+        } else {
+          lx.e[q] += a.weight[o];
+          ly.e[q] += a.weight[o + n];
+          lz.e[q] += a.weight[o + 2 * n];
+        }
+        --kk[q];
+        next[q] = kk[q] >= 0 ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
+      }
     }
     x = cx;
     y = cy;
     z = cz;
-    const T h = hc;
+    const V h = hc;
     if (st > 0) {
       cp -= n3;
-      cx = cp[0];
-      cy = cp[n];
-      cz = cp[2 * n];
-      hc = hp[(int64_t)(st - 1) * n];
+      hq2 -= n;
+#pragma unroll
+      for (int q = 0; q < K; ++q) {
+        if (st - 1 < S[q]) {
+          cx.e[q] = cp[q];
+          cy.e[q] = cp[n + q];
+          cz.e[q] = cp[2 * n + q];
+          hc.e[q] = hq2[q];
+        } else {
+          hc.e[q] = cst<T>(0.0);  // a slot past its last step: an identity step
+        }
+      }
     }
     // recompute the stage states of step st (same arithmetic as the forward)
-    T ax, ay, az;
-    T f1x, f1y, f1z;
+    V ax, ay, az;
+    V f1x, f1y, f1z;
     lorenz_f(x, y, z, s, r, b, f1x, f1y, f1z);
-    T U2x, U2y, U2z, U3x, U3y, U3z, U4x, U4y, U4z, U5x, U5y, U5z, U6x, U6y, U6z;
-    ax = cst<T>(TS_A21) * f1x;
-    ay = cst<T>(TS_A21) * f1y;
-    az = cst<T>(TS_A21) * f1z;
+    V U2x, U2y, U2z, U3x, U3y, U3z, U4x, U4y, U4z, U5x, U5y, U5z, U6x, U6y, U6z;
+    GS_ACC1(TS_A21, f1)
     GS_STAGE(U2x, U2y, U2z, ax, ay, az)
-    T f2x, f2y, f2z;
+    V f2x, f2y, f2z;
     lorenz_f(U2x, U2y, U2z, s, r, b, f2x, f2y, f2z);
-    ax = cst<T>(TS_A31) * f1x;
-    ay = cst<T>(TS_A31) * f1y;
-    az = cst<T>(TS_A31) * f1z;
-    ax = fmaT(cst<T>(TS_A32), f2x, ax);
-    ay = fmaT(cst<T>(TS_A32), f2y, ay);
-    az = fmaT(cst<T>(TS_A32), f2z, az);
+    GS_ACC1(TS_A31, f1)
+    GS_ACCN(TS_A32, f2)
     GS_STAGE(U3x, U3y, U3z, ax, ay, az)
-    T f3x, f3y, f3z;
+    V f3x, f3y, f3z;
     lorenz_f(U3x, U3y, U3z, s, r, b, f3x, f3y, f3z);
-    ax = cst<T>(TS_A41) * f1x;
-    ay = cst<T>(TS_A41) * f1y;
-    az = cst<T>(TS_A41) * f1z;
-    ax = fmaT(cst<T>(TS_A42), f2x, ax);
-    ay = fmaT(cst<T>(TS_A42), f2y, ay);
-    az = fmaT(cst<T>(TS_A42), f2z, az);
-    ax = fmaT(cst<T>(TS_A43), f3x, ax);
-    ay = fmaT(cst<T>(TS_A43), f3y, ay);
-    az = fmaT(cst<T>(TS_A43), f3z, az);
+    GS_ACC1(TS_A41, f1)
+    GS_ACCN(TS_A42, f2)
+    GS_ACCN(TS_A43, f3)
     GS_STAGE(U4x, U4y, U4z, ax, ay, az)
-    T f4x, f4y, f4z;
+    V f4x, f4y, f4z;
     lorenz_f(U4x, U4y, U4z, s, r, b, f4x, f4y, f4z);
-    ax = cst<T>(TS_A51) * f1x;
-    ay = cst<T>(TS_A51) * f1y;
-    az = cst<T>(TS_A51) * f1z;
-    ax = fmaT(cst<T>(TS_A52), f2x, ax);
-    ay = fmaT(cst<T>(TS_A52), f2y, ay);
-    az = fmaT(cst<T>(TS_A52), f2z, az);
-    ax = fmaT(cst<T>(TS_A53), f3x, ax);
-    ay = fmaT(cst<T>(TS_A53), f3y, ay);
-    az = fmaT(cst<T>(TS_A53), f3z, az);
-    ax = fmaT(cst<T>(TS_A54), f4x, ax);
-    ay = fmaT(cst<T>(TS_A54), f4y, ay);
-    az = fmaT(cst<T>(TS_A54), f4z, az);
+    GS_ACC1(TS_A51, f1)
+    GS_ACCN(TS_A52, f2)
+    GS_ACCN(TS_A53, f3)
+    GS_ACCN(TS_A54, f4)
     GS_STAGE(U5x, U5y, U5z, ax, ay, az)
-    T f5x, f5y, f5z;
+    V f5x, f5y, f5z;
     lorenz_f(U5x, U5y, U5z, s, r, b, f5x, f5y, f5z);
-    ax = cst<T>(TS_A61) * f1x;
-    ay = cst<T>(TS_A61) * f1y;
-    az = cst<T>(TS_A61) * f1z;
-    ax = fmaT(cst<T>(TS_A62), f2x, ax);
-    ay = fmaT(cst<T>(TS_A62), f2y, ay);
-    az = fmaT(cst<T>(TS_A62), f2z, az);
-    ax = fmaT(cst<T>(TS_A63), f3x, ax);
-    ay = fmaT(cst<T>(TS_A63), f3y, ay);
-    az = fmaT(cst<T>(TS_A63), f3z, az);
-    ax = fmaT(cst<T>(TS_A64), f4x, ax);
-    ay = fmaT(cst<T>(TS_A64), f4y, ay);
-    az = fmaT(cst<T>(TS_A64), f4z, az);
-    ax = fmaT(cst<T>(TS_A65), f5x, ax);
-    ay = fmaT(cst<T>(TS_A65), f5y, ay);
-    az = fmaT(cst<T>(TS_A65), f5z, az);
+    GS_ACC1(TS_A61, f1)
+    GS_ACCN(TS_A62, f2)
+    GS_ACCN(TS_A63, f3)
+    GS_ACCN(TS_A64, f4)
+    GS_ACCN(TS_A65, f5)
     GS_STAGE(U6x, U6y, U6z, ax, ay, az)
 
     // transposed step, stages 6 .. 1
-    T m6x, m6y, m6z, m5x, m5y, m5z, m4x, m4y, m4z, m3x, m3y, m3z, m2x, m2y, m2z, m1x, m1y, m1z;
-    T vx, vy, vz;
+    V m6x, m6y, m6z, m5x, m5y, m5z, m4x, m4y, m4z, m3x, m3y, m3z, m2x, m2y, m2z, m1x, m1y, m1z;
+    V vx, vy, vz;
     vx = h * (cst<T>(TS_B6) * lx);
     vy = h * (cst<T>(TS_B6) * ly);
     vz = h * (cst<T>(TS_B6) * lz);
@@ -368,21 +407,23 @@ __global__ void __launch_bounds__(128, 4) k_grad_tsit5_lorenz(TsitLorenzArgs<T> 
     lx += ((m1x + m2x) + (m3x + m4x)) + (m5x + m6x);
     ly += ((m1y + m2y) + (m3y + m4y)) + (m5y + m6y);
     lz += ((m1z + m2z) + (m3z + m4z)) + (m5z + m6z);
-    nx = x;
-    ny = y;
-    nz = z;
   }
   // save points at step 0 cannot exist (save times lie in (t0, t1])
-  a.loss[i] = L;
-  a.dp[i] = ps;
-  a.dp[n + i] = pr;
-  a.dp[2 * n + i] = pb;
-  a.du0[i] = lx;
-  a.du0[n + i] = ly;
-  a.du0[2 * n + i] = lz;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    if (i[q] < 0) continue;
+    a.dp[i[q]] = ps.e[q];
+    a.dp[n + i[q]] = pr.e[q];
+    a.dp[2 * n + i[q]] = pb.e[q];
+    a.du0[i[q]] = lx.e[q];
+    a.du0[n + i[q]] = ly.e[q];
+    a.du0[2 * n + i[q]] = lz.e[q];
+  }
 }
 
 #undef GS_STAGE
+#undef GS_ACC1
+#undef GS_ACCN
 
 template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp,
@@ -405,9 +446,11 @@ gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const 
   a.dp = (T*)dp;
   a.du0 = (T*)du0;
   a.ck = (T*)ws;
-  const int bs = 128;
-  const int64_t grid = (P->n + bs - 1) / bs;
-  k_grad_tsit5_lorenz<T><<<(unsigned)grid, bs, 0, st>>>(a);
+  constexpr int K = GS_GRAD_K;
+  const int bs = GS_GRAD_BS;
+  const int64_t threads = (P->n + K - 1) / K;
+  const int64_t grid = (threads + bs - 1) / bs;
+  k_grad_tsit5_lorenz<T, K><<<(unsigned)grid, bs, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

@@ -10,18 +10,18 @@
 //   err <= 1; PI control with error order q (Tsit5 5, ROS2 2):
 //   accept: fac = 0.9 err^(-0.7/q) errprev^(0.4/q) in [0.2, 10] (10 if
 //   err == 0), <= 1 right after a rejection, errprev = max(err, 1e-4);
-//   reject: fac = max(0.2, 0.9 err^(-1/q)) (0.2 for NaN); the proposal is
+//   reject: fac = max(0.2, 0.9 err^(-1/q)) (0.2 for NaN or inf); the proposal is
 //   multiplied by fac either way.  A step whose end would reach the next stop
 //   (save time or t1, within 4 eps) is shortened to land on it exactly.
 //   Starting step: Hairer, Norsett & Wanner I, II.4.
 // One thread per trajectory; every loop is bounded by the step capacity.
 //
-// Order of a record: gs_record runs the adaptive solve twice.  The sizing pass
-// (trajectory order) gives each trajectory's step count; a stable counting
-// sort by decreasing count gives the slot order; the recording pass runs slot
-// j on trajectory order[j], so the threads of a warp carry chains of nearly
-// equal length and write the step-major mesh h[s][j] nearly in lockstep.  The
-// two passes execute the same arithmetic, so they agree on every count.
+// Order of a record: gs_record runs the adaptive solve once, in trajectory
+// order, into workspace copies of the mesh arrays; a stable counting sort by
+// decreasing step count gives the slot order; a gather copies every array
+// into slot order (reads scattered, writes coalesced) and zero-fills the h
+// rows past each slot's last step.  The gradient kernels then find chains of
+// nearly equal length in every warp.
 #include "steps.cuh"
 
 namespace gs {
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
   const int64_t n = a.n;
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n) return;
-  const int64_t i = STORE ? (int64_t)a.order[j] : j;
+  const int64_t i = a.order ? (int64_t)a.order[j] : j;
   const T eps = Eps<T>::v;
   const T q = METHOD == GS_TSIT5 ? cst<T>(5.0) : cst<T>(2.0);
   T u[3], p[3], k1[3];
@@ -90,7 +90,9 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
     if (!(hprop > cst<T>(0.0)) || !isfinite(hprop)) finite = false;
   }
   if (!finite) status = GS_TRAJ_NONFINITE;
-  T t = a.t0, errprev = cst<T>(1.0);
+  // the controller carries ln(errprev); errprev starts at 1 and is floored at 1e-4
+  T t = a.t0, lnprev = cst<T>(0.0);
+  const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
   bool prev_rej = false;
   int kk = 0;
   T* hout = STORE ? a.h + j : nullptr;
@@ -133,15 +135,17 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
         if (STORE) a.save_idx[(int64_t)kk * n + j] = nst;
         ++kk;
       }
-      T fac;
+      // fac = 0.9 err^(-0.7/q) errprev^(0.4/q), as 0.9 exp(-(0.7/q) ln err + (0.4/q) ln errprev)
+      T fac, lnerr = ln_floor;
       if (err == cst<T>(0.0)) {
         fac = cst<T>(10.0);
       } else {
-        fac = (cst<T>(0.9) * ctrl_pow<T>(err, -(cst<T>(0.7) / q))) * ctrl_pow<T>(errprev, cst<T>(0.4) / q);
+        lnerr = ctrl_ln<T>(err);
+        fac = cst<T>(0.9) * ctrl_exp<T>(fmaT(-(cst<T>(0.7) / q), lnerr, (cst<T>(0.4) / q) * lnprev));
         fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
       }
       if (prev_rej) fac = smin_(fac, cst<T>(1.0));
-      errprev = smax_(err, cst<T>(1e-4));
+      lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
       prev_rej = false;
       hprop = fac * hprop;
       if (t >= a.t1) break;
@@ -151,14 +155,14 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
         status = GS_TRAJ_MAXSTEPS;
         break;
       }
-      const T fac = isnan(err) ? cst<T>(0.2) : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_pow<T>(err, -(cst<T>(1.0) / q)));
+      const T fac = !isfinite(err) ? cst<T>(0.2)
+                                   : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_exp<T>(-(cst<T>(1.0) / q) * ctrl_ln<T>(err)));
       hprop = fac * hprop;
       prev_rej = true;
     }
   }
   if (STORE) {
-    // zero the unused tail of the slot's column and unreached save points
-    for (int s = nst; s < a.smax; ++s) hout[(int64_t)s * n] = cst<T>(0.0);
+    // unreached save points (a failed trajectory); the h tail stays unwritten
     for (int k = kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + j] = 0;
   }
   a.nsteps[j] = nst;
@@ -284,11 +288,31 @@ gs_status count3(const gs_problem* P, const gs_tol* tol, int32_t smax, int32_t* 
   return dispatch_rec<float, false>(P->system, P->method, a, st);
 }
 
-size_t record_ws_bytes(int64_t n, int32_t smax) {
+static size_t al256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Workspace of gs_record: trajectory-order copies of nsteps, status, nreject,
+// save_idx and h, then the sort histogram.
+size_t record_ws_bytes(int64_t n, int32_t smax, int32_t nsave, size_t tsize) {
   const int64_t nchunk = (n + kChunk - 1) / kChunk;
-  const size_t cnt = ((size_t)n * 4 + 255) / 256 * 256;
-  const size_t hist = (size_t)(smax + 1) * (size_t)nchunk * 4;
-  return cnt + hist;
+  return 3 * al256((size_t)n * 4) + al256((size_t)nsave * n * 4) + al256((size_t)smax * n * tsize) +
+         (size_t)(smax + 1) * (size_t)nchunk * 4;
+}
+
+template <typename T>
+__global__ void k_gather_mesh(int64_t n, int smax, int nsave, const int32_t* __restrict__ order,
+                              const T* __restrict__ h_tmp, const int32_t* __restrict__ si_tmp,
+                              const int32_t* __restrict__ ns_tmp, const int32_t* __restrict__ st_tmp,
+                              const int32_t* __restrict__ nr_tmp, T* h, int32_t* save_idx, int32_t* nsteps,
+                              int32_t* status, int32_t* nreject) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= n) return;
+  const int64_t i = order[j];
+  const int S = ns_tmp[i];
+  nsteps[j] = S;
+  status[j] = st_tmp[i];
+  nreject[j] = nr_tmp[i];
+  for (int k = 0; k < nsave; ++k) save_idx[(int64_t)k * n + j] = si_tmp[(int64_t)k * n + i];
+  for (int s = 0; s < smax; ++s) h[(int64_t)s * n + j] = s < S ? h_tmp[(int64_t)s * n + i] : cst<T>(0.0);
 }
 
 gs_status order_slots(const int32_t* cnt, int64_t n, int32_t smax, int32_t* hist, int32_t* order, cudaStream_t st) {
@@ -302,31 +326,41 @@ gs_status order_slots(const int32_t* cnt, int64_t n, int32_t smax, int32_t* hist
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
 
+template <typename T>
+static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, cudaStream_t st) {
+  const int64_t n = P->n;
+  char* w = (char*)ws;
+  int32_t* ns_tmp = (int32_t*)w;
+  w += al256((size_t)n * 4);
+  int32_t* st_tmp = (int32_t*)w;
+  w += al256((size_t)n * 4);
+  int32_t* nr_tmp = (int32_t*)w;
+  w += al256((size_t)n * 4);
+  int32_t* si_tmp = (int32_t*)w;
+  w += al256((size_t)P->nsave * n * 4);
+  T* h_tmp = (T*)w;
+  w += al256((size_t)M->smax * n * sizeof(T));
+  int32_t* hist = (int32_t*)w;
+  RecArgs<T> a = rec_args<T>(P, tol, M->smax);
+  a.order = nullptr;  // trajectory order
+  a.h = h_tmp;
+  a.save_idx = si_tmp;
+  a.nsteps = ns_tmp;
+  a.status = st_tmp;
+  a.nreject = nr_tmp;
+  gs_status rc = dispatch_rec<T, true>(P->system, P->method, a, st);
+  if (rc != GS_OK) return rc;
+  rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
+  if (rc != GS_OK) return rc;
+  k_gather_mesh<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp,
+                                                                 st_tmp, nr_tmp, (T*)M->h, M->save_idx, M->nsteps,
+                                                                 M->status, M->nreject);
+  count_launch();
+  return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
 gs_status record3(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, cudaStream_t st) {
-  int32_t* cnt = (int32_t*)ws;
-  int32_t* hist = (int32_t*)((char*)ws + ((size_t)P->n * 4 + 255) / 256 * 256);
-  gs_status rc = count3(P, tol, M->smax, cnt, nullptr, st);
-  if (rc != GS_OK) return rc;
-  rc = order_slots(cnt, P->n, M->smax, hist, M->order, st);
-  if (rc != GS_OK) return rc;
-  if (P->dtype == GS_F64) {
-    RecArgs<double> a = rec_args<double>(P, tol, M->smax);
-    a.order = M->order;
-    a.h = (double*)M->h;
-    a.save_idx = M->save_idx;
-    a.nsteps = M->nsteps;
-    a.status = M->status;
-    a.nreject = M->nreject;
-    return dispatch_rec<double, true>(P->system, P->method, a, st);
-  }
-  RecArgs<float> a = rec_args<float>(P, tol, M->smax);
-  a.order = M->order;
-  a.h = (float*)M->h;
-  a.save_idx = M->save_idx;
-  a.nsteps = M->nsteps;
-  a.status = M->status;
-  a.nreject = M->nreject;
-  return dispatch_rec<float, true>(P->system, P->method, a, st);
+  return P->dtype == GS_F64 ? record3_t<double>(P, tol, M, ws, st) : record3_t<float>(P, tol, M, ws, st);
 }
 
 }  // namespace gs

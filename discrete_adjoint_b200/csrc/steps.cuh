@@ -40,8 +40,9 @@ __device__ __forceinline__ void jac3(const T u[3], const T p[3], T J[9]) {
   }
 }
 
-// Powers x^y for the step-size controller.  Library pow may differ from other
-// implementations by an ulp, and the embedded error estimate (a sum with heavy
+// Logarithm and exponential for the step-size controller (its powers are
+// x^y = exp(y ln x)).  Library pow may differ from other implementations by an
+// ulp, and the embedded error estimate (a sum with heavy
 // cancellation) turns such an ulp into ~1e-10 relative step-size differences
 // within a few steps, which chaos then amplifies.  This one uses only IEEE
 // +, -, *, /, fma and the exact frexp / ldexp / rint, in a fixed order, so its
@@ -59,10 +60,7 @@ __device__ __forceinline__ double rintT(double x) { return rint(x); }
 __device__ __forceinline__ float rintT(float x) { return rintf(x); }
 
 template <typename T>
-__device__ T ctrl_pow(T x, T y) {
-  if (isnan(x) || isnan(y)) return x + y;
-  if (x == cst<T>(0.0)) return y > cst<T>(0.0) ? cst<T>(0.0) : (y < cst<T>(0.0) ? cst<T>(1.0) / x : cst<T>(1.0));
-  if (isinf(x)) return y > cst<T>(0.0) ? x : (y < cst<T>(0.0) ? cst<T>(0.0) : cst<T>(1.0));
+__device__ T ctrl_ln(T x) {  // x > 0 finite
   int e = 0;
   T m = frexpT(x, &e);
   if (m < cst<T>(0.7071067811865476)) {
@@ -76,8 +74,12 @@ __device__ T ctrl_pow(T x, T y) {
   for (int k = 11; k >= 0; --k) poly = fmaT(poly, z, cst<T>(1.0 / double(2 * k + 1)));
   const T lnm = (s + s) * poly;
   const T ef = (T)e;
-  const T lnx = fmaT(ef, cst<T>(0.6931467056274414), fmaT(ef, cst<T>(4.7493250390316726e-07), lnm));
-  const T w = y * lnx;
+  return fmaT(ef, cst<T>(0.6931467056274414), fmaT(ef, cst<T>(4.7493250390316726e-07), lnm));
+}
+
+template <typename T>
+__device__ T ctrl_exp(T w) {
+  if (isnan(w)) return w;
   const T kf = rintT(w * cst<T>(1.4426950408889634));
   if (kf > cst<T>(2000.0)) return cst<T>(1.0) / cst<T>(0.0);
   if (kf < cst<T>(-2000.0)) return cst<T>(0.0);
@@ -103,6 +105,14 @@ __device__ T ctrl_pow(T x, T y) {
 #pragma unroll
   for (int j = 13; j >= 0; --j) p = fmaT(p, r, cst<T>(inv_fact[j]));
   return ldexpT(p, (int)kf);
+}
+
+template <typename T>
+__device__ T ctrl_pow(T x, T y) {
+  if (isnan(x) || isnan(y)) return x + y;
+  if (x == cst<T>(0.0)) return y > cst<T>(0.0) ? cst<T>(0.0) : (y < cst<T>(0.0) ? cst<T>(1.0) / x : cst<T>(1.0));
+  if (isinf(x)) return y > cst<T>(0.0) ? x : (y < cst<T>(0.0) ? cst<T>(0.0) : cst<T>(1.0));
+  return ctrl_exp<T>(y * ctrl_ln<T>(x));
 }
 
 template <typename T>

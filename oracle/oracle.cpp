@@ -372,10 +372,12 @@ bool ros2_step(int sys, int d, const S* u, const S* p, S h, S* unew, S* err) {
 }
 
 // ---------------------------------------------------------------------------
-// Powers x^y for the step-size controller, computed from IEEE +, -, *, /, fma
-// and the exact frexp / ldexp / rint only, so that any implementation keeping
-// this operation order gets the same bits (a library pow may differ by an ulp,
-// and the embedded error estimate amplifies such differences; see DESIGN).
+// Logarithm and exponential for the step-size controller, computed from IEEE
+// +, -, *, /, fma and the exact frexp / ldexp / rint only, so that any
+// implementation keeping this operation order gets the same bits (a library
+// pow may differ by an ulp, and the embedded error estimate amplifies such
+// differences within a few steps).  The controller's powers are
+// x^y = ctrl_exp(y ctrl_ln(x)).
 //   ln x : x = m 2^e with m in [sqrt(1/2), sqrt(2)); ln m = 2 atanh(s),
 //          s = (m-1)/(m+1), by the series s (1 + z/3 + ... + z^12/25), z = s^2.
 //   exp w: Cody & Waite reduction w = k ln2 + r (ln2 split in a 21-bit head and
@@ -388,10 +390,7 @@ static const double CP_INV_LN2 = 1.4426950408889634;
 static const double CP_SQRT_HALF = 0.7071067811865476;
 
 template <class T>
-T ctrl_pow(T x, T y) {
-  if (std::isnan(x) || std::isnan(y)) return std::numeric_limits<T>::quiet_NaN();
-  if (x == T(0)) return y > T(0) ? T(0) : (y < T(0) ? std::numeric_limits<T>::infinity() : T(1));
-  if (std::isinf(x)) return y > T(0) ? x : (y < T(0) ? T(0) : T(1));
+T ctrl_ln(T x) {  // x > 0 finite
   int e = 0;
   T m = std::frexp(x, &e);
   if (m < T(CP_SQRT_HALF)) {
@@ -403,8 +402,12 @@ T ctrl_pow(T x, T y) {
   T poly = T(1.0 / 25.0);
   for (int k = 11; k >= 0; --k) poly = std::fma(poly, z, T(1.0 / double(2 * k + 1)));
   T lnm = (s + s) * poly;
-  T lnx = std::fma(T(e), T(CP_LN2_HI), std::fma(T(e), T(CP_LN2_LO), lnm));
-  T w = y * lnx;
+  return std::fma(T(e), T(CP_LN2_HI), std::fma(T(e), T(CP_LN2_LO), lnm));
+}
+
+template <class T>
+T ctrl_exp(T w) {
+  if (std::isnan(w)) return w;
   T kf = std::rint(w * T(CP_INV_LN2));
   if (kf > T(2000)) return std::numeric_limits<T>::infinity();
   if (kf < T(-2000)) return T(0);
@@ -420,6 +423,14 @@ T ctrl_pow(T x, T y) {
   return std::ldexp(p, int(kf));
 }
 
+template <class T>
+T ctrl_pow(T x, T y) {
+  if (std::isnan(x) || std::isnan(y)) return std::numeric_limits<T>::quiet_NaN();
+  if (x == T(0)) return y > T(0) ? T(0) : (y < T(0) ? std::numeric_limits<T>::infinity() : T(1));
+  if (std::isinf(x)) return y > T(0) ? x : (y < T(0) ? T(0) : T(1));
+  return ctrl_exp<T>(y * ctrl_ln<T>(x));
+}
+
 // ---------------------------------------------------------------------------
 // Adaptive recorder (plain scalar T).
 //
@@ -428,7 +439,7 @@ T ctrl_pow(T x, T y) {
 // q (5 for Tsit5, 2 for ROS2): accepted -> fac = 0.9 err^(-0.7/q)
 // errprev^(0.4/q) clipped to [0.2, 10] (10 if err == 0), capped at 1 after a
 // rejection, errprev <- max(err, 1e-4); rejected -> fac = max(0.2, 0.9
-// err^(-1/q)) (0.2 if err is NaN).  The next proposal is fac * h_prop, where
+// err^(-1/q)) (0.2 if err is NaN or infinite).  The next proposal is fac * h_prop, where
 // h_prop is the unclipped proposal.  Steps are shortened to land exactly on
 // every save time and on t1; save_idx[k] is the number of accepted steps taken
 // when t reached tsave[k].  Starting step: Hairer, Norsett & Wanner I, II.4.
@@ -490,7 +501,9 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
     out.status = TRAJ_NONFINITE;
     return out;
   }
-  T t = t0, errprev = T(1);
+  // the controller carries ln(errprev); errprev starts at 1 and is floored at 1e-4
+  T t = t0, lnprev = T(0);
+  const T ln_floor = ctrl_ln<T>(T(1e-4));
   bool prev_rej = false;
   int kk = 0;
   while (true) {
@@ -521,15 +534,17 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
       t = clipped ? tstop : tn;
       for (int c = 0; c < d; ++c) u[c] = un[c];
       while (kk < nsave && t == tsave[kk]) out.save_idx[kk++] = out.nsteps;
-      T fac;
+      // fac = 0.9 err^(-0.7/q) errprev^(0.4/q) = 0.9 exp(-(0.7/q) ln err + (0.4/q) ln errprev)
+      T fac, lnerr = ln_floor;
       if (err == T(0)) {
         fac = T(10);
       } else {
-        fac = (T(0.9) * ctrl_pow<T>(err, -T(0.7) / q)) * ctrl_pow<T>(errprev, T(0.4) / q);
+        lnerr = ctrl_ln<T>(err);
+        fac = T(0.9) * ctrl_exp<T>(std::fma(-T(0.7) / q, lnerr, (T(0.4) / q) * lnprev));
         fac = std::min(T(10), std::max(T(0.2), fac));
       }
       if (prev_rej) fac = std::min(fac, T(1));
-      errprev = std::max(err, T(1e-4));
+      lnprev = err < T(1e-4) ? ln_floor : lnerr;
       prev_rej = false;
       hprop = fac * hprop;
       if (t >= t1) return out;  // the last step lands exactly on t1
@@ -539,7 +554,8 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
         out.status = TRAJ_MAXSTEPS;
         return out;
       }
-      T fac = std::isnan(err) ? T(0.2) : std::max(T(0.2), T(0.9) * ctrl_pow<T>(err, -T(1) / q));
+      T fac = !std::isfinite(err) ? T(0.2)
+                                  : std::max(T(0.2), T(0.9) * ctrl_exp<T>((-T(1) / q) * ctrl_ln<T>(err)));
       hprop = fac * hprop;
       prev_rej = true;
     }

