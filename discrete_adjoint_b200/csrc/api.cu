@@ -23,6 +23,13 @@ gs_status launch_grad_ros2(const gs_problem*, const gs_mesh*, const gs_loss*, vo
                            cudaStream_t);
 template <typename T>
 gs_status launch_solve3(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
+gs_status record_node64(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
+gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,
+                             int32_t*, cudaStream_t);
+gs_status node64_grad(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*, void*,
+                      cudaStream_t);
+gs_status node64_solve(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
+size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize);
 
 static size_t dsize(const gs_problem* P) { return P->dtype == GS_F64 ? 8 : 4; }
 
@@ -39,7 +46,9 @@ static gs_status check_problem(const gs_problem* P) {
     case GS_NODE64:
       if (P->d != 64 || P->np != 64) return GS_EINVAL;
       if (P->n > 0 && !P->shared) return GS_EINVAL;
-      return GS_EUNSUPPORTED;
+      // built for the single-precision Tsit5 configuration
+      if (P->method != GS_TSIT5 || P->dtype != GS_F32) return GS_EUNSUPPORTED;
+      break;
     case GS_HIRES:
       return GS_EUNSUPPORTED;
     default:
@@ -86,7 +95,10 @@ int64_t gs_launch_count(void) { return g_launches.load(); }
 size_t gs_workspace_bytes(const gs_problem* P, const gs_mesh* M, int32_t op) {
   if (check_problem(P) != GS_OK || !M || M->smax < 1) return 0;
   if (op == GS_OP_RECORD) return record_ws_bytes(P->n, M->smax, P->nsave, dsize(P));
-  if (op == GS_OP_GRAD) return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
+  if (op == GS_OP_GRAD) {
+    if (P->system == GS_NODE64) return node64_grad_ws_bytes(P->n, M->smax, dsize(P));
+    return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
+  }
   return 0;
 }
 
@@ -99,6 +111,8 @@ gs_status gs_count(const gs_problem* P, const gs_tol* tol, int32_t smax, int32_t
     return GS_EINVAL;
   if (P->n == 0) return GS_OK;
   if (!nsteps) return GS_EINVAL;
+  if (P->system == GS_NODE64)
+    return node64_record_pass(P, tol, smax, false, nullptr, nullptr, nsteps, status, nullptr, (cudaStream_t)stream);
   return count3(P, tol, smax, nsteps, status, (cudaStream_t)stream);
 }
 
@@ -111,6 +125,7 @@ gs_status gs_record(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, vo
     return GS_EINVAL;
   if (P->n == 0) return GS_OK;
   if (!ws || ws_bytes < gs_workspace_bytes(P, M, GS_OP_RECORD)) return GS_EWORKSPACE;
+  if (P->system == GS_NODE64) return record_node64(P, tol, M, ws, (cudaStream_t)stream);
   return record3(P, tol, M, ws, (cudaStream_t)stream);
 }
 
@@ -120,13 +135,13 @@ gs_status gs_solve(const gs_problem* P, const gs_mesh* M, void* u_save, void* st
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
   if (P->n == 0) return GS_OK;
   if (!u_save) return GS_EINVAL;
+  if (P->system == GS_NODE64) return node64_solve(P, M, u_save, (cudaStream_t)stream);
   return P->dtype == GS_F64 ? launch_solve3<double>(P, M, u_save, (cudaStream_t)stream)
                             : launch_solve3<float>(P, M, u_save, (cudaStream_t)stream);
 }
 
 gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp, void* du0,
                   void* dshared, void* ws, size_t ws_bytes, void* stream) {
-  (void)dshared;
   gs_status rc = check_problem(P);
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
@@ -136,6 +151,7 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (!loss || !dp || !du0) return GS_EINVAL;
   if (!ws || ws_bytes < gs_workspace_bytes(P, M, GS_OP_GRAD)) return GS_EWORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
+  if (P->system == GS_NODE64) return node64_grad(P, M, Ls, loss, dp, du0, dshared, ws, st);
   if (P->method == GS_TSIT5 && P->system == GS_LORENZ)
     return P->dtype == GS_F64 ? launch_grad_tsit5_lorenz<double>(P, M, Ls, loss, dp, du0, ws, st)
                               : launch_grad_tsit5_lorenz<float>(P, M, Ls, loss, dp, du0, ws, st);

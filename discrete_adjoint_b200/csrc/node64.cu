@@ -1,0 +1,906 @@
+// node64.cu -- the d = 64 shared-weight system  du/dt = tanh(W u + b_i) - u
+// (one W for the whole ensemble, a bias b_i per trajectory): adaptive Tsit5
+// recorder, forward-only solve, and the fused replay + reverse sweep with the
+// weight gradient summed over the ensemble.
+//
+// GRADSOLVE (arXiv 2609.02876) differentiates registered right-hand sides up to
+// state dimension 64 (evolve.pub review, "Summary"); this is the neural
+// right-hand side of its neural-ODE study, with gradients dL/db_i, dL/du0_i and
+// dL/dW = sum_i dL_i/dW.
+//
+// Layout: a CTA of 256 threads carries 32 trajectories (slots).  Every
+// per-trajectory vector of the CTA is a 64 x 32 tile [component][slot]; thread
+// (ty, tx) = (tid / 16, tid % 16) owns rows 4ty..4ty+3 of slots 2tx, 2tx+1 of
+// every tile, in registers, so all element-wise stage arithmetic is local.
+// The stage products are matrix products over the CTA's 32 trajectories, with
+// operands staged in shared memory:
+//   Z = W U      (z_r = b_r + sum_k W_rk U_k, accumulated in k = 0..63 order:
+//                 the floating-point contract's order for this right-hand side)
+//   M = W^T G    (mu = W^T g - nu, the vector-Jacobian product)
+//   dW += G U^T  (over the 32 slots; per-CTA partials, summed afterwards in
+//                 a fixed order so the weight gradient is deterministic)
+// The per-trajectory parts of the recorder (error norm as the contract's
+// sequential sum over components, the PI controller) run one thread per slot.
+#include "steps.cuh"
+
+namespace gs {
+
+namespace n64 {
+
+constexpr int D = 64;
+constexpr int TB = 32;     // trajectories (slots) per CTA
+constexpr int NT = 256;    // threads per CTA
+constexpr int LDT = D + 4;  // row stride of the [slot][component] tiles
+
+// Per-thread block of a 64 x 32 tile: 4 rows x 2 slots.
+template <typename T>
+struct Blk {
+  T v[4][2];
+};
+
+template <typename T>
+__device__ __forceinline__ Blk<T> bzero() {
+  Blk<T> r;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) r.v[a][c] = cst<T>(0.0);
+  return r;
+}
+
+template <typename T>
+struct Smem {
+  T W[D][D];    // W[r][k]
+  T Wt[D][D];   // Wt[k][r] = W[r][k]
+  T B[D][TB];   // operand [component][slot]
+  T G[D][TB];   // second operand [component][slot]
+  T Gt[TB][LDT];  // [slot][component]
+  T Ut[TB][LDT];  // [slot][component]
+  T red[D][TB];   // per-slot reductions (scaled errors, norms)
+  T hs[TB];       // per-slot step of the current attempt
+  int flag[TB];   // per-slot accept / state flags
+  int any;
+};
+
+// Z_block = W * B (contract order: start at bias, fma over k = 0..63).
+template <typename T>
+__device__ __forceinline__ Blk<T> matmul_WB(const Smem<T>& s, const Blk<T>& bias, int ty, int tx) {
+  Blk<T> z = bias;
+#pragma unroll 8
+  for (int k = 0; k < D; ++k) {
+    T w[4], u[2];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) w[a] = s.Wt[k][4 * ty + a];
+    u[0] = s.B[k][2 * tx];
+    u[1] = s.B[k][2 * tx + 1];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) z.v[a][c] = fmaT(w[a], u[c], z.v[a][c]);
+  }
+  return z;
+}
+
+// M_block = W^T * G.
+template <typename T>
+__device__ __forceinline__ Blk<T> matmul_WtG(const Smem<T>& s, int ty, int tx) {
+  Blk<T> m = bzero<T>();
+#pragma unroll 8
+  for (int k = 0; k < D; ++k) {
+    T w[4], g[2];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) w[a] = s.W[k][4 * ty + a];
+    g[0] = s.G[k][2 * tx];
+    g[1] = s.G[k][2 * tx + 1];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) m.v[a][c] = fmaT(w[a], g[c], m.v[a][c]);
+  }
+  return m;
+}
+
+template <typename T>
+__device__ __forceinline__ void store_B(Smem<T>& s, const Blk<T>& x, int ty, int tx) {
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    s.B[4 * ty + a][2 * tx] = x.v[a][0];
+    s.B[4 * ty + a][2 * tx + 1] = x.v[a][1];
+  }
+}
+
+// y = tanh(z), k = y - U  (the right-hand side on a stage state)
+template <typename T>
+__device__ __forceinline__ void rhs_tail(const Blk<T>& z, const Blk<T>& U, Blk<T>& y, Blk<T>& k) {
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      y.v[a][c] = tanh(z.v[a][c]);
+      k.v[a][c] = y.v[a][c] - U.v[a][c];
+    }
+}
+
+// f(U) for the CTA: stage U through shared memory, multiply, apply tanh.
+template <typename T>
+__device__ __forceinline__ void eval_f(Smem<T>& s, const Blk<T>& U, const Blk<T>& bias, Blk<T>& y, Blk<T>& k, int ty,
+                                       int tx) {
+  __syncthreads();  // previous readers of B are done
+  store_B(s, U, ty, tx);
+  __syncthreads();
+  Blk<T> z = matmul_WB(s, bias, ty, tx);
+  rhs_tail(z, U, y, k);
+}
+
+// U = fma(h, sum_m a_m k_m, u) with the contract's order (first term a plain
+// product, then fmas in increasing m).
+template <typename T, int NS>
+__device__ __forceinline__ Blk<T> stage(const T (&coef)[NS], const Blk<T>* const (&ks)[NS], const Blk<T>& u,
+                                        const T (&h)[2]) {
+  Blk<T> U;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      T acc = coef[0] * ks[0]->v[a][c];
+#pragma unroll
+      for (int m = 1; m < NS; ++m) acc = fmaT(coef[m], ks[m]->v[a][c], acc);
+      U.v[a][c] = fmaT(h[c], acc, u.v[a][c]);
+    }
+  return U;
+}
+
+// Tsit5 stages 2..7 from u and k1; returns u_new (stage 7) and k2..k7.
+template <typename T>
+__device__ __forceinline__ void tsit5_stages(Smem<T>& s, const Blk<T>& u, const Blk<T>& bias, const T (&h)[2],
+                                             const Blk<T>& k1, Blk<T>& k2, Blk<T>& k3, Blk<T>& k4, Blk<T>& k5,
+                                             Blk<T>& k6, Blk<T>& k7, Blk<T>& un, int ty, int tx) {
+  Blk<T> y, U;
+  {
+    const T c[1] = {cst<T>(TS_A21)};
+    const Blk<T>* const ks[1] = {&k1};
+    U = stage<T, 1>(c, ks, u, h);
+    eval_f(s, U, bias, y, k2, ty, tx);
+  }
+  {
+    const T c[2] = {cst<T>(TS_A31), cst<T>(TS_A32)};
+    const Blk<T>* const ks[2] = {&k1, &k2};
+    U = stage<T, 2>(c, ks, u, h);
+    eval_f(s, U, bias, y, k3, ty, tx);
+  }
+  {
+    const T c[3] = {cst<T>(TS_A41), cst<T>(TS_A42), cst<T>(TS_A43)};
+    const Blk<T>* const ks[3] = {&k1, &k2, &k3};
+    U = stage<T, 3>(c, ks, u, h);
+    eval_f(s, U, bias, y, k4, ty, tx);
+  }
+  {
+    const T c[4] = {cst<T>(TS_A51), cst<T>(TS_A52), cst<T>(TS_A53), cst<T>(TS_A54)};
+    const Blk<T>* const ks[4] = {&k1, &k2, &k3, &k4};
+    U = stage<T, 4>(c, ks, u, h);
+    eval_f(s, U, bias, y, k5, ty, tx);
+  }
+  {
+    const T c[5] = {cst<T>(TS_A61), cst<T>(TS_A62), cst<T>(TS_A63), cst<T>(TS_A64), cst<T>(TS_A65)};
+    const Blk<T>* const ks[5] = {&k1, &k2, &k3, &k4, &k5};
+    U = stage<T, 5>(c, ks, u, h);
+    eval_f(s, U, bias, y, k6, ty, tx);
+  }
+  {
+    const T c[6] = {cst<T>(TS_B1), cst<T>(TS_B2), cst<T>(TS_B3), cst<T>(TS_B4), cst<T>(TS_B5), cst<T>(TS_B6)};
+    const Blk<T>* const ks[6] = {&k1, &k2, &k3, &k4, &k5, &k6};
+    un = stage<T, 6>(c, ks, u, h);
+    eval_f(s, un, bias, y, k7, ty, tx);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load_W(Smem<T>& s, const T* W, int tid) {
+  for (int q = tid; q < D * D; q += NT) {
+    const int r = q / D, k = q % D;
+    const T w = W[q];
+    s.W[r][k] = w;
+    s.Wt[k][r] = w;
+  }
+}
+
+// Sequential per-slot sum over components of red[c][slot] (contract order):
+// slot t's thread returns sqrt(sum / 64) -- the RMS norm of the scaled values.
+template <typename T>
+__device__ __forceinline__ T slot_rms(const Smem<T>& s, int t) {
+  T acc = cst<T>(0.0);
+  for (int c = 0; c < D; ++c) acc = fmaT(s.red[c][t], s.red[c][t], acc);
+  return sqrt(acc / cst<T>(64.0));
+}
+
+// ---------------------------------------------------------------------------
+// Recorder: one CTA per 32 trajectories, in trajectory order (slot = index).
+// ---------------------------------------------------------------------------
+template <typename T>
+struct RecArgs64 {
+  int64_t n;
+  const T* p;   // b [64][n]
+  const T* u0;  // [64][n]
+  const T* W;   // [64][64]
+  T t0, t1, rtol, atol, h0;
+  int32_t nsave, smax;
+  T tsave[GS_MAX_SAVE];
+  bool store;
+  T* h;               // [n][smax] (trajectory-major workspace copy)
+  int32_t* save_idx;  // [nsave][n]
+  int32_t* nsteps;
+  int32_t* status;
+  int32_t* nreject;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
+  extern __shared__ unsigned char smem_raw[];
+  Smem<T>& s = *reinterpret_cast<Smem<T>*>(smem_raw);
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  const int64_t n = a.n;
+  const int64_t base = (int64_t)blockIdx.x * TB;
+  load_W(s, a.W, tid);
+  Blk<T> u, bias;
+  bool col_ok[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int64_t i = base + 2 * tx + c;
+    col_ok[c] = i < n;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = 4 * ty + q;
+      u.v[q][c] = col_ok[c] ? a.u0[(int64_t)r * n + i] : cst<T>(0.0);
+      bias.v[q][c] = col_ok[c] ? a.p[(int64_t)r * n + i] : cst<T>(0.0);
+    }
+  }
+  // per-slot controller state, held by thread t < 32 for slot t
+  const int t = tid;
+  const bool ctl = t < TB;
+  const int64_t it = base + t;
+  const bool live = ctl && it < n;
+  const T eps = Eps<T>::v;
+  const T qord = cst<T>(5.0);
+  T tcur = a.t0, hprop = cst<T>(0.0), lnprev = cst<T>(0.0);
+  const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
+  int nst = 0, nrej = 0, kk = 0, status = live ? GS_TRAJ_OK : GS_TRAJ_MAXSTEPS;
+  bool prev_rej = false, done = !live;
+
+  // k1 = f(u0) and the starting step (Hairer, Norsett & Wanner I, II.4)
+  Blk<T> y, k1;
+  eval_f(s, u, bias, y, k1, ty, tx);
+  // finiteness of u0 and f(u0): per-slot flag via shared memory
+  if (ctl) s.flag[t] = 1;
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      if (!isfinite(u.v[q][c]) || !isfinite(k1.v[q][c])) s.flag[2 * tx + c] = 0;
+  // d0 = rms(u0 / sc), sc = fma(rtol, |u0|, atol)
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) s.red[4 * ty + q][2 * tx + c] = u.v[q][c] / fmaT(a.rtol, fabs(u.v[q][c]), a.atol);
+  __syncthreads();
+  T d0 = ctl ? slot_rms(s, t) : cst<T>(0.0);
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) s.red[4 * ty + q][2 * tx + c] = k1.v[q][c] / fmaT(a.rtol, fabs(u.v[q][c]), a.atol);
+  __syncthreads();
+  T d1 = ctl ? slot_rms(s, t) : cst<T>(0.0);
+  T h0 = (d0 < cst<T>(1e-5) || d1 < cst<T>(1e-5)) ? cst<T>(1e-6) : cst<T>(0.01) * (d0 / d1);
+  h0 = smin_(h0, a.t1 - a.t0);
+  if (ctl) s.hs[t] = h0;
+  __syncthreads();
+  Blk<T> u1, k1b;
+  {
+    const T hh[2] = {s.hs[2 * tx], s.hs[2 * tx + 1]};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) u1.v[q][c] = fmaT(hh[c], k1.v[q][c], u.v[q][c]);
+  }
+  eval_f(s, u1, bias, y, k1b, ty, tx);
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      s.red[4 * ty + q][2 * tx + c] = (k1b.v[q][c] - k1.v[q][c]) / fmaT(a.rtol, fabs(u.v[q][c]), a.atol);
+  __syncthreads();
+  if (ctl) {
+    const T d2 = slot_rms(s, t) / h0;
+    const T dm = smax_(d1, d2);
+    const T h1 = dm <= cst<T>(1e-15) ? smax_(cst<T>(1e-6), h0 * cst<T>(1e-3))
+                                     : ctrl_pow<T>(cst<T>(0.01) / dm, cst<T>(1.0) / qord);
+    hprop = a.h0 > cst<T>(0.0) ? a.h0 : smin_(smin_(cst<T>(100.0) * h0, h1), a.t1 - a.t0);
+    if (live && (s.flag[t] == 0 || !(hprop > cst<T>(0.0)) || !isfinite(hprop))) {
+      status = GS_TRAJ_NONFINITE;
+      done = true;
+    }
+  }
+
+  Blk<T> k2, k3, k4, k5, k6, k7, un;
+  for (int iter = 0;; ++iter) {
+    // --- per-slot: choose the attempt
+    bool clipped = false;
+    T tstop = a.t1, tn = tcur;
+    if (ctl) {
+      if (!done && hprop < cst<T>(16.0) * eps * fabs(tcur)) {
+        status = GS_TRAJ_DTMIN;
+        done = true;
+      }
+      T hh = cst<T>(0.0);
+      if (!done) {
+        tstop = kk < a.nsave ? a.tsave[kk] : a.t1;
+        tn = tcur + hprop;
+        clipped = tn >= tstop - cst<T>(4.0) * eps * fabs(tstop);
+        hh = clipped ? tstop - tcur : hprop;
+      }
+      s.hs[t] = hh;
+      s.flag[t] = done ? 0 : 1;
+    }
+    __syncthreads();
+    if (ctl) {
+      // any slot still running?
+      if (t == 0) {
+        int any = 0;
+        for (int q = 0; q < TB; ++q) any |= s.flag[q];
+        s.any = any;
+      }
+    }
+    __syncthreads();
+    if (!s.any) break;
+    const T hh[2] = {s.hs[2 * tx], s.hs[2 * tx + 1]};
+    tsit5_stages(s, u, bias, hh, k1, k2, k3, k4, k5, k6, k7, un, ty, tx);
+    // scaled error e / sc into red
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        T acc = cst<T>(TS_E1) * k1.v[q][c];
+        acc = fmaT(cst<T>(TS_E2), k2.v[q][c], acc);
+        acc = fmaT(cst<T>(TS_E3), k3.v[q][c], acc);
+        acc = fmaT(cst<T>(TS_E4), k4.v[q][c], acc);
+        acc = fmaT(cst<T>(TS_E5), k5.v[q][c], acc);
+        acc = fmaT(cst<T>(TS_E6), k6.v[q][c], acc);
+        acc = fmaT(cst<T>(TS_E7), k7.v[q][c], acc);
+        const T e = hh[c] * acc;
+        const T sc = fmaT(a.rtol, smax_(fabs(u.v[q][c]), fabs(un.v[q][c])), a.atol);
+        s.red[4 * ty + q][2 * tx + c] = e / sc;
+      }
+    __syncthreads();
+    // --- per-slot: accept / reject, controller
+    if (ctl) {
+      int accept = 0;
+      if (!done) {
+        const T err = slot_rms(s, t);
+        const T hcur = s.hs[t];
+        if (err <= cst<T>(1.0)) {
+          if (nst >= a.smax) {
+            status = GS_TRAJ_MAXSTEPS;
+            done = true;
+          } else {
+            accept = 1;
+            if (a.store) a.h[it * a.smax + nst] = hcur;  // trajectory-major workspace copy
+            ++nst;
+            tcur = clipped ? tstop : tn;
+            while (kk < a.nsave && tcur == a.tsave[kk]) {
+              if (a.store) a.save_idx[(int64_t)kk * n + it] = nst;
+              ++kk;
+            }
+            T fac, lnerr = ln_floor;
+            if (err == cst<T>(0.0)) {
+              fac = cst<T>(10.0);
+            } else {
+              lnerr = ctrl_ln<T>(err);
+              fac = cst<T>(0.9) * ctrl_exp<T>(fmaT(-(cst<T>(0.7) / qord), lnerr, (cst<T>(0.4) / qord) * lnprev));
+              fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
+            }
+            if (prev_rej) fac = smin_(fac, cst<T>(1.0));
+            lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
+            prev_rej = false;
+            hprop = fac * hprop;
+            if (tcur >= a.t1) done = true;
+          }
+        } else {
+          ++nrej;
+          if (nrej > a.smax) {
+            status = GS_TRAJ_MAXSTEPS;
+            done = true;
+          } else {
+            const T fac = !isfinite(err) ? cst<T>(0.2)
+                                         : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_exp<T>(-(cst<T>(1.0) / qord) *
+                                                                                          ctrl_ln<T>(err)));
+            hprop = fac * hprop;
+            prev_rej = true;
+          }
+        }
+      }
+      s.flag[t] = accept;
+    }
+    __syncthreads();
+    // --- every thread: take the accepted steps
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (s.flag[2 * tx + c]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          u.v[q][c] = un.v[q][c];
+          k1.v[q][c] = k7.v[q][c];
+        }
+      }
+    }
+  }
+  if (live) {
+    if (a.store)
+      for (int k = kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + it] = 0;
+    a.nsteps[it] = nst;
+    if (a.status) a.status[it] = status;
+    if (a.nreject) a.nreject[it] = nrej;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Forward replay (solve) and fused replay + reverse sweep (grad), on slots.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct GradArgs64 {
+  int64_t n;
+  const T* p;
+  const T* u0;
+  const T* W;
+  const T* h;
+  const int32_t* order;
+  const int32_t* nsteps;
+  const int32_t* save_idx;
+  const int32_t* status;
+  int32_t nsave, smax;
+  int32_t loss_kind;
+  const T* target;
+  const T* weight;
+  T* loss;
+  T* dp;
+  T* du0;
+  T* ck;       // workspace [smax][64][n] by slot
+  T* dW_part;  // workspace [gridDim][64][64]
+  T* u_save;   // solve: [nsave][64][n] by trajectory
+};
+
+// Loss of the save point each flagged slot has reached: the terms of the
+// thread's rows go to red (and G for a linear loss), then the slot's thread
+// sums them in the contract's order (components 0..63, fma chain).
+template <typename T>
+__device__ __forceinline__ void save_point_loss(Smem<T>& s, const GradArgs64<T>& a, const Blk<T>& u,
+                                                const int64_t (&o)[2], const bool (&hit)[2], T& Lslot, int ty,
+                                                int tx, int tid) {
+  __syncthreads();
+  if (tid < TB) s.flag[tid] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    if (!hit[c]) continue;
+    if (ty == 0) s.flag[2 * tx + c] = 1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = 4 * ty + q;
+      const int64_t oo = o[c] + (int64_t)r * a.n;
+      if (a.loss_kind == GS_LOSS_SUMSQ) {
+        s.red[r][2 * tx + c] = a.target ? u.v[q][c] - a.target[oo] : u.v[q][c];
+      } else {
+        s.red[r][2 * tx + c] = a.weight[oo];
+        s.G[r][2 * tx + c] = u.v[q][c];
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < TB && s.flag[tid]) {
+    T L = Lslot;
+    for (int r = 0; r < D; ++r)
+      L = a.loss_kind == GS_LOSS_SUMSQ ? fmaT(s.red[r][tid], s.red[r][tid], L) : fmaT(s.red[r][tid], s.G[r][tid], L);
+    Lslot = L;
+  }
+}
+
+template <typename T, bool GRAD>
+__global__ void __launch_bounds__(NT, 1) k_replay_node64(GradArgs64<T> a) {
+  extern __shared__ unsigned char smem_raw[];
+  Smem<T>& s = *reinterpret_cast<Smem<T>*>(smem_raw);
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  const int64_t n = a.n;
+  const int64_t base = (int64_t)blockIdx.x * TB;
+  const int64_t n64 = (int64_t)D * n;
+  const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
+  load_W(s, a.W, tid);
+
+  // slots of this thread's two columns
+  int64_t traj[2];
+  int S[2];
+  bool act[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int64_t j = base + 2 * tx + c;
+    traj[c] = -1;
+    S[c] = 0;
+    act[c] = false;
+    if (j < n) {
+      const int64_t i = a.order[j];
+      if (i >= 0 && i < n) {
+        traj[c] = i;
+        const int sq = a.nsteps[j];
+        if (a.status[j] == GS_TRAJ_OK && sq >= 0 && sq <= a.smax) {
+          S[c] = sq;
+          act[c] = true;
+        }
+      }
+    }
+  }
+  // CTA-wide chain length
+  if (tid < TB) s.flag[tid] = 0;
+  __syncthreads();
+  if (ty == 0) {
+    s.flag[2 * tx] = S[0];
+    s.flag[2 * tx + 1] = S[1];
+  }
+  __syncthreads();
+  int Smax = 0;
+  for (int q = 0; q < TB; ++q) Smax = s.flag[q] > Smax ? s.flag[q] : Smax;
+  // the thread that owns slot tid (tid < 32) keeps that slot's loss
+  T Lslot = cst<T>(0.0);
+
+  Blk<T> u, bias;
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = 4 * ty + q;
+      u.v[q][c] = act[c] ? a.u0[(int64_t)r * n + traj[c]] : cst<T>(0.0);
+      bias.v[q][c] = act[c] ? a.p[(int64_t)r * n + traj[c]] : cst<T>(0.0);
+    }
+  int kk[2] = {0, 0}, next[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) next[c] = act[c] && S[c] > 0 ? a.save_idx[base + 2 * tx + c] : -1;
+
+  // ---------------------------------------------------------------- forward
+  {
+    Blk<T> y, k1, k2, k3, k4, k5, k6, k7, un;
+    eval_f(s, u, bias, y, k1, ty, tx);
+    for (int st = 0; st < Smax; ++st) {
+      T hh[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        hh[c] = st < S[c] ? a.h[(int64_t)st * n + base + 2 * tx + c] : cst<T>(0.0);
+        if (GRAD && st < S[c]) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            a.ck[(int64_t)st * n64 + (int64_t)(4 * ty + q) * n + base + 2 * tx + c] = u.v[q][c];
+        }
+      }
+      tsit5_stages(s, u, bias, hh, k1, k2, k3, k4, k5, k6, k7, un, ty, tx);
+      u = un;
+      k1 = k7;
+      bool hit[2];
+      int64_t o[2];
+      int anyhit = 0;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        hit[c] = st + 1 == next[c];
+        o[c] = hit[c] ? (int64_t)kk[c] * n64 + traj[c] : 0;
+        anyhit |= hit[c];
+        if (hit[c]) {
+          if (!GRAD) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a.u_save[o[c] + (int64_t)(4 * ty + q) * n] = u.v[q][c];
+          }
+          ++kk[c];
+          next[c] = kk[c] < a.nsave ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
+        }
+      }
+      if (GRAD && __syncthreads_or(anyhit)) save_point_loss(s, a, u, o, hit, Lslot, ty, tx, tid);
+    }
+  }
+  if (!GRAD) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      if (!act[c] && traj[c] >= 0)
+        for (int k = 0; k < a.nsave; ++k)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) a.u_save[(int64_t)k * n64 + (int64_t)(4 * ty + q) * n + traj[c]] = nan;
+    return;
+  }
+  // loss per slot (thread tid < 32 owns slot tid)
+  if (tid < TB) {
+    const int64_t j = base + tid;
+    if (j < n) {
+      const int64_t i = a.order[j];
+      if (i >= 0 && i < n) {
+        const bool ok = a.status[j] == GS_TRAJ_OK && a.nsteps[j] >= 0 && a.nsteps[j] <= a.smax;
+        a.loss[i] = ok ? Lslot : nan;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- reverse
+  // u holds u_{st+1} at the top of iteration st.
+  Blk<T> lam = bzero<T>(), bbar = bzero<T>();
+  T dWacc[4][4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) dWacc[q][w] = cst<T>(0.0);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    kk[c] = a.nsave - 1;
+    next[c] = act[c] && S[c] > 0 ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
+  }
+  for (int st = Smax - 1; st >= 0; --st) {
+    T hh[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (st + 1 == next[c]) {
+        const int64_t o = (int64_t)kk[c] * n64 + traj[c];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int64_t oo = o + (int64_t)(4 * ty + q) * n;
+          if (a.loss_kind == GS_LOSS_SUMSQ)
+            lam.v[q][c] = fmaT(cst<T>(2.0), a.target ? u.v[q][c] - a.target[oo] : u.v[q][c], lam.v[q][c]);
+          else
+            lam.v[q][c] += a.weight[oo];
+        }
+        --kk[c];
+        next[c] = kk[c] >= 0 ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
+      }
+      const bool run = st < S[c];
+      hh[c] = run ? a.h[(int64_t)st * n + base + 2 * tx + c] : cst<T>(0.0);
+      if (run) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          u.v[q][c] = a.ck[(int64_t)st * n64 + (int64_t)(4 * ty + q) * n + base + 2 * tx + c];
+      }
+    }
+    // recompute stage states U_j and tanh values y_j (k_j = y_j - U_j)
+    Blk<T> U1 = u, U2, U3, U4, U5, U6, y1, y2, y3, y4, y5, y6, kd;
+    eval_f(s, U1, bias, y1, kd, ty, tx);
+    Blk<T> k1 = kd;
+    {
+      const T c[1] = {cst<T>(TS_A21)};
+      const Blk<T>* const ks[1] = {&k1};
+      U2 = stage<T, 1>(c, ks, U1, hh);
+    }
+    eval_f(s, U2, bias, y2, kd, ty, tx);
+    Blk<T> k2 = kd;
+    {
+      const T c[2] = {cst<T>(TS_A31), cst<T>(TS_A32)};
+      const Blk<T>* const ks[2] = {&k1, &k2};
+      U3 = stage<T, 2>(c, ks, U1, hh);
+    }
+    eval_f(s, U3, bias, y3, kd, ty, tx);
+    Blk<T> k3 = kd;
+    {
+      const T c[3] = {cst<T>(TS_A41), cst<T>(TS_A42), cst<T>(TS_A43)};
+      const Blk<T>* const ks[3] = {&k1, &k2, &k3};
+      U4 = stage<T, 3>(c, ks, U1, hh);
+    }
+    eval_f(s, U4, bias, y4, kd, ty, tx);
+    Blk<T> k4 = kd;
+    {
+      const T c[4] = {cst<T>(TS_A51), cst<T>(TS_A52), cst<T>(TS_A53), cst<T>(TS_A54)};
+      const Blk<T>* const ks[4] = {&k1, &k2, &k3, &k4};
+      U5 = stage<T, 4>(c, ks, U1, hh);
+    }
+    eval_f(s, U5, bias, y5, kd, ty, tx);
+    Blk<T> k5 = kd;
+    {
+      const T c[5] = {cst<T>(TS_A61), cst<T>(TS_A62), cst<T>(TS_A63), cst<T>(TS_A64), cst<T>(TS_A65)};
+      const Blk<T>* const ks[5] = {&k1, &k2, &k3, &k4, &k5};
+      U6 = stage<T, 5>(c, ks, U1, hh);
+    }
+    eval_f(s, U6, bias, y6, kd, ty, tx);
+
+    // transposed step, stages 6 .. 1:
+    //   nu_j = h (b_j lambda + sum_{m>j} a_mj mu_m), g_j = nu_j (1 - y_j^2),
+    //   mu_j = W^T g_j - nu_j, bbar += g_j, dW += g_j U_j^T
+    Blk<T> mu[6];
+    const Blk<T>* Ys[6] = {&y1, &y2, &y3, &y4, &y5, &y6};
+    const Blk<T>* Us[6] = {&U1, &U2, &U3, &U4, &U5, &U6};
+    const double bw[6] = {TS_B1, TS_B2, TS_B3, TS_B4, TS_B5, TS_B6};
+    const double aw[6][6] = {{0, 0, 0, 0, 0, 0},
+                             {TS_A21, 0, 0, 0, 0, 0},
+                             {TS_A31, TS_A32, 0, 0, 0, 0},
+                             {TS_A41, TS_A42, TS_A43, 0, 0, 0},
+                             {TS_A51, TS_A52, TS_A53, TS_A54, 0, 0},
+                             {TS_A61, TS_A62, TS_A63, TS_A64, TS_A65, 0}};
+#pragma unroll
+    for (int jj = 5; jj >= 0; --jj) {
+      Blk<T> nu, g;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          T acc = cst<T>(bw[jj]) * lam.v[q][c];
+#pragma unroll
+          for (int m = 5; m > jj; --m) acc = fmaT(cst<T>(aw[m][jj]), mu[m].v[q][c], acc);
+          nu.v[q][c] = hh[c] * acc;
+          const T yv = Ys[jj]->v[q][c];
+          g.v[q][c] = nu.v[q][c] * fmaT(-yv, yv, cst<T>(1.0));
+          bbar.v[q][c] += g.v[q][c];
+        }
+      __syncthreads();  // previous readers of G / Gt / Ut are done
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int r = 4 * ty + q, t = 2 * tx + c;
+          s.G[r][t] = g.v[q][c];
+          s.Gt[t][r] = g.v[q][c];
+          s.Ut[t][r] = Us[jj]->v[q][c];
+        }
+      __syncthreads();
+      Blk<T> m = matmul_WtG(s, ty, tx);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) mu[jj].v[q][c] = m.v[q][c] - nu.v[q][c];
+      // dW block (rows 4ty.., columns 4tx..) over the CTA's slots
+#pragma unroll 4
+      for (int t = 0; t < TB; ++t) {
+        T gr[4], uc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gr[q] = s.Gt[t][4 * ty + q];
+          uc[q] = s.Ut[t][4 * tx + q];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int w = 0; w < 4; ++w) dWacc[q][w] = fmaT(gr[q], uc[w], dWacc[q][w]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        lam.v[q][c] += ((mu[0].v[q][c] + mu[1].v[q][c]) + (mu[2].v[q][c] + mu[3].v[q][c])) +
+                       (mu[4].v[q][c] + mu[5].v[q][c]);
+  }
+  // outputs: dL/db (bias), dL/du0, and this CTA's weight-gradient partial
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    if (!act[c]) {
+      if (traj[c] >= 0)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          a.dp[(int64_t)(4 * ty + q) * n + traj[c]] = nan;
+          a.du0[(int64_t)(4 * ty + q) * n + traj[c]] = nan;
+        }
+      continue;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      a.dp[(int64_t)(4 * ty + q) * n + traj[c]] = bbar.v[q][c];
+      a.du0[(int64_t)(4 * ty + q) * n + traj[c]] = lam.v[q][c];
+    }
+  }
+  T* part = a.dW_part + (int64_t)blockIdx.x * D * D;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) part[(4 * ty + q) * D + 4 * tx + w] = dWacc[q][w];
+}
+
+// dW = sum over CTAs of the partials, in CTA order (deterministic).
+template <typename T>
+__global__ void k_reduce_dW(const T* part, int nblk, T* dW) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= D * D) return;
+  T acc = cst<T>(0.0);
+  for (int b = 0; b < nblk; ++b) acc += part[(int64_t)b * D * D + e];
+  dW[e] = acc;
+}
+
+}  // namespace n64
+
+size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize) {
+  const int64_t nblk = (n + n64::TB - 1) / n64::TB;
+  const size_t ck = ((size_t)smax * 64 * n * tsize + 255) / 256 * 256;
+  return ck + (size_t)nblk * 64 * 64 * tsize;
+}
+
+template <typename T>
+static n64::GradArgs64<T> grad64_args(const gs_problem* P, const gs_mesh* M) {
+  n64::GradArgs64<T> a{};
+  a.n = P->n;
+  a.p = (const T*)P->p;
+  a.u0 = (const T*)P->u0;
+  a.W = (const T*)P->shared;
+  a.h = (const T*)M->h;
+  a.order = M->order;
+  a.nsteps = M->nsteps;
+  a.save_idx = M->save_idx;
+  a.status = M->status;
+  a.nsave = P->nsave;
+  a.smax = M->smax;
+  return a;
+}
+
+gs_status node64_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp, void* du0,
+                      void* dshared, void* ws, cudaStream_t st) {
+  using T = float;
+  n64::GradArgs64<T> a = grad64_args<T>(P, M);
+  a.loss_kind = Ls->kind;
+  a.target = (const T*)Ls->target;
+  a.weight = (const T*)Ls->weight;
+  a.loss = (T*)loss;
+  a.dp = (T*)dp;
+  a.du0 = (T*)du0;
+  a.ck = (T*)ws;
+  const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
+  a.dW_part = (T*)((char*)ws + ((size_t)M->smax * 64 * P->n * sizeof(T) + 255) / 256 * 256);
+  const size_t smem = sizeof(n64::Smem<T>);
+  if (cudaFuncSetAttribute(n64::k_replay_node64<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return GS_ECUDA;
+  n64::k_replay_node64<T, true><<<nblk, n64::NT, smem, st>>>(a);
+  count_launch();
+  if (!launch_ok()) return GS_ECUDA;
+  if (dshared) {
+    n64::k_reduce_dW<T><<<(64 * 64 + 255) / 256, 256, 0, st>>>(a.dW_part, nblk, (T*)dshared);
+    count_launch();
+  }
+  return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
+gs_status node64_solve(const gs_problem* P, const gs_mesh* M, void* u_save, cudaStream_t st) {
+  using T = float;
+  n64::GradArgs64<T> a = grad64_args<T>(P, M);
+  a.u_save = (T*)u_save;
+  const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
+  const size_t smem = sizeof(n64::Smem<T>);
+  if (cudaFuncSetAttribute(n64::k_replay_node64<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return GS_ECUDA;
+  n64::k_replay_node64<T, false><<<nblk, n64::NT, smem, st>>>(a);
+  count_launch();
+  return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
+// Adaptive record (store = true: into h / save_idx, trajectory order) or the
+// sizing pass (store = false).
+gs_status node64_record_pass(const gs_problem* P, const gs_tol* tol, int32_t smax, bool store, float* h,
+                             int32_t* save_idx, int32_t* nsteps, int32_t* status, int32_t* nreject, cudaStream_t st) {
+  using T = float;
+  n64::RecArgs64<T> a{};
+  a.n = P->n;
+  a.p = (const T*)P->p;
+  a.u0 = (const T*)P->u0;
+  a.W = (const T*)P->shared;
+  a.t0 = (T)P->t0;
+  a.t1 = (T)P->t1;
+  a.rtol = (T)tol->rtol;
+  a.atol = (T)tol->atol;
+  a.h0 = (T)tol->h0;
+  a.nsave = P->nsave;
+  a.smax = smax;
+  for (int k = 0; k < P->nsave; ++k) a.tsave[k] = (T)P->tsave[k];
+  a.store = store;
+  a.h = h;
+  a.save_idx = save_idx;
+  a.nsteps = nsteps;
+  a.status = status;
+  a.nreject = nreject;
+  const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
+  const size_t smem = sizeof(n64::Smem<T>);
+  if (cudaFuncSetAttribute(n64::k_record_node64<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return GS_ECUDA;
+  n64::k_record_node64<T><<<nblk, n64::NT, smem, st>>>(a);
+  count_launch();
+  return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
+}  // namespace gs

@@ -17,10 +17,12 @@
 // One thread per trajectory; every loop is bounded by the step capacity.
 //
 // Order of a record: gs_record runs the adaptive solve once, in trajectory
-// order, into workspace copies of the mesh arrays; a stable counting sort by
-// decreasing step count gives the slot order; a gather copies every array
-// into slot order (reads scattered, writes coalesced) and zero-fills the h
-// rows past each slot's last step.  The gradient kernels then find chains of
+// order, into workspace copies of the mesh arrays (h trajectory-major, so each
+// thread writes its own row front to back and L2 merges the partial sectors);
+// a stable counting sort by decreasing step count gives the slot order; a
+// gather copies every array into slot order (each thread reads one source row
+// in order, writes coalesced) and zero-fills the h rows past each slot's last
+// step.  The gradient kernels then find chains of
 // nearly equal length in every warp.
 #include "steps.cuh"
 
@@ -36,7 +38,8 @@ struct RecArgs {
   int32_t smax;
   T tsave[GS_MAX_SAVE];
   const int32_t* order;  // slot -> trajectory (null: identity)
-  T* h;                  // [smax][n] by slot (null: count only)
+  T* h;                  // step sizes (null: count only); step s of slot j at
+  int64_t hcol, hstep;   // h[j * hcol + s * hstep]
   int32_t* save_idx;     // [nsave][n] by slot
   int32_t* nsteps;       // [n]
   int32_t* status;       // [n] (may be null in count mode)
@@ -95,7 +98,7 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
   const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
   bool prev_rej = false;
   int kk = 0;
-  T* hout = STORE ? a.h + j : nullptr;
+  T* hout = STORE ? a.h + j * a.hcol : nullptr;
   while (status == GS_TRAJ_OK) {
     const T tstop = kk < a.nsave ? a.tsave[kk] : a.t1;
     if (hprop < cst<T>(16.0) * eps * fabs(t)) {
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
         status = GS_TRAJ_MAXSTEPS;
         break;
       }
-      if (STORE) hout[(int64_t)nst * n] = h;
+      if (STORE) hout[(int64_t)nst * a.hstep] = h;
       ++nst;
       t = clipped ? tstop : tn;
 #pragma unroll
@@ -312,7 +315,8 @@ __global__ void k_gather_mesh(int64_t n, int smax, int nsave, const int32_t* __r
   status[j] = st_tmp[i];
   nreject[j] = nr_tmp[i];
   for (int k = 0; k < nsave; ++k) save_idx[(int64_t)k * n + j] = si_tmp[(int64_t)k * n + i];
-  for (int s = 0; s < smax; ++s) h[(int64_t)s * n + j] = s < S ? h_tmp[(int64_t)s * n + i] : cst<T>(0.0);
+  const T* src = h_tmp + i * smax;  // trajectory-major: a thread reads one row in order
+  for (int s = 0; s < smax; ++s) h[(int64_t)s * n + j] = s < S ? src[s] : cst<T>(0.0);
 }
 
 gs_status order_slots(const int32_t* cnt, int64_t n, int32_t smax, int32_t* hist, int32_t* order, cudaStream_t st) {
@@ -344,6 +348,8 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
   RecArgs<T> a = rec_args<T>(P, tol, M->smax);
   a.order = nullptr;  // trajectory order
   a.h = h_tmp;
+  a.hcol = M->smax;  // trajectory-major workspace copy: each thread writes its own row
+  a.hstep = 1;
   a.save_idx = si_tmp;
   a.nsteps = ns_tmp;
   a.status = st_tmp;
@@ -361,6 +367,37 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
 
 gs_status record3(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, cudaStream_t st) {
   return P->dtype == GS_F64 ? record3_t<double>(P, tol, M, ws, st) : record3_t<float>(P, tol, M, ws, st);
+}
+
+gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,
+                             int32_t*, cudaStream_t);
+
+// The d = 64 record: the same trajectory-order pass / sort / gather sequence,
+// with the CTA-per-32-trajectories recorder of node64.cu.
+gs_status record_node64(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, cudaStream_t st) {
+  using T = float;
+  const int64_t n = P->n;
+  char* w = (char*)ws;
+  int32_t* ns_tmp = (int32_t*)w;
+  w += al256((size_t)n * 4);
+  int32_t* st_tmp = (int32_t*)w;
+  w += al256((size_t)n * 4);
+  int32_t* nr_tmp = (int32_t*)w;
+  w += al256((size_t)n * 4);
+  int32_t* si_tmp = (int32_t*)w;
+  w += al256((size_t)P->nsave * n * 4);
+  T* h_tmp = (T*)w;
+  w += al256((size_t)M->smax * n * sizeof(T));
+  int32_t* hist = (int32_t*)w;
+  gs_status rc = node64_record_pass(P, tol, M->smax, true, h_tmp, si_tmp, ns_tmp, st_tmp, nr_tmp, st);
+  if (rc != GS_OK) return rc;
+  rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
+  if (rc != GS_OK) return rc;
+  k_gather_mesh<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp,
+                                                                 st_tmp, nr_tmp, (T*)M->h, M->save_idx, M->nsteps,
+                                                                 M->status, M->nreject);
+  count_launch();
+  return launch_ok() ? GS_OK : GS_ECUDA;
 }
 
 }  // namespace gs

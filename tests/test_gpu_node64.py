@@ -1,0 +1,86 @@
+"""GPU <-> oracle parity for the d = 64 shared-weight system (workload
+node64, fp32): recorder, forward solve, per-trajectory gradients dL/db_i and
+dL/du0_i on the same mesh, and the ensemble weight gradient dL/dW."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+import discrete_adjoint_b200 as gs
+from gpu_util import TOL, dev, ensemble, loss_args, mesh_by_trajectory, mesh_from_oracle, parity, tens
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", params=[512, 100])
+def case(request):
+    prob = W.node64(request.param)
+    om = oracle.record(prob, 64)
+    assert (om.status == 0).all()
+    return prob, om
+
+
+def test_record_node64(case):
+    prob, om = case
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(prob.n, 64, 1, "f32", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    assert (st == 0).all()
+    # tanh is each side's library function (not bitwise), and in fp32 at
+    # tol 1e-5 the embedded error estimate carries ~1e-3 relative rounding
+    # noise (heavy cancellation), so accept/reject decisions within that band
+    # of err = 1 can differ: measured 96.5 % equal step counts on 512
+    # trajectories.  (No fp32 mesh gate is stated; gradient parity below runs
+    # on the oracle's mesh.)
+    # The first step (the conservative starting step) has err << 1, where the
+    # fp32 estimate is mostly cancellation noise, so its PI factor -- and the
+    # step sizes after it -- differ at the 1e-3..1e-2 level between the two
+    # sides.  Checked instead: equal counts for most, every GPU mesh spans
+    # exactly [t0, t1], and the typical step-size difference is small.
+    same = ns == om.nsteps
+    assert same.mean() >= 0.9
+    for i in range(prob.n):
+        assert abs(h[i, : ns[i]].astype(np.float32).sum(dtype=np.float64) - (prob.t1 - prob.t0)) <= 1e-5
+    rel = np.abs(h[same] - om.h[same][:, :64]) / np.maximum(np.abs(om.h[same][:, :64]), 1e-30)
+    assert np.median(rel[om.h[same][:, :64] > 0]) <= 1e-2
+    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, 64)
+    torch.cuda.synchronize()
+    assert np.array_equal(nsteps.cpu().numpy(), ns)
+
+
+def test_solve_node64(case):
+    prob, om = case
+    _, us = oracle.replay(prob, om)
+    u = gs.gs_solve(ensemble(prob), mesh_from_oracle(om, "f32")).double().cpu().numpy()
+    assert np.abs(u - us).max() <= 1e-5 * np.abs(us).max()
+
+
+def test_grad_node64(case):
+    prob, om = case
+    out = gs.gs_grad(ensemble(prob), mesh_from_oracle(om, "f32"), **loss_args(prob))
+    torch.cuda.synchronize()
+    parity(out, prob, om, dual=False)
+    wide = oracle.grad(prob, om, "tape_wide")
+    dW = out.dshared.double().cpu().numpy()
+    assert np.linalg.norm(dW - wide["dW"]) <= TOL["f32"] * np.linalg.norm(wide["dW"])
+    assert np.abs(out.loss.double().cpu().numpy() - wide["loss"]).max() <= 1e-5 * np.abs(wide["loss"]).max()
+
+
+def test_node64_weight_gradient_is_additive():
+    """dW of an ensemble equals the sum of the dW of two halves (any size)."""
+    prob = W.node64(2000)
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(prob.n, 64, 1, "f32", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    full = gs.gs_grad(ens, mesh, **loss_args(prob)).dshared.double()
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    parts = []
+    for idx in (np.arange(0, 700), np.arange(700, 2000)):
+        sub = prob.subset(idx)
+        om = oracle.Mesh(h[idx], ns[idx], si[idx], st[idx], np.zeros(len(idx), np.int32))
+        parts.append(gs.gs_grad(ensemble(sub), mesh_from_oracle(om, "f32"), **loss_args(sub)).dshared.double())
+    torch.cuda.synchronize()
+    assert torch.linalg.norm(full - parts[0] - parts[1]) <= 1e-5 * torch.linalg.norm(full)
