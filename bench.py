@@ -1,24 +1,29 @@
-"""Throughput benchmark: record + 10 gradient passes of a Lorenz ensemble.
+"""Throughput benchmark of the record-and-replay gradient path.
 
-One step = the whole hot path over one batch: gs_record (sizing pass, slot
-ordering, recording pass) followed by 10 fused replay + reverse-sweep passes
-(gs_grad) against the fixed mesh -- the workload "Lorenz (d=3), n = 2**20,
-t in [0, 10], Tsit5 rtol = atol = 1e-6, ten save points with N(0,1) targets,
-one record then ten gradient passes".  The metric is trajectory-gradients/s
-over the whole step (record included).
+One step = the whole hot path over one batch of synthetic input: gs_record
+(one adaptive pass, slot ordering, gather into the mesh) followed by the
+workload's gradient passes (fused replay + reverse sweep, gs_grad) against the
+fixed mesh.  The default workload is "Lorenz (d=3), n = 2**20 per GPU, t in
+[0, 10], Tsit5 rtol = atol = 1e-6, ten save points with N(0,1) targets, one
+record then ten gradient passes", in fp64.  The metric is
+trajectory-gradients/s over the whole step (record included); the gradient
+pass alone is reported in config.grad_only_value.
 
-  python bench.py [--gpus N --steps K --warmup W --dtype f64|f32 --impl ours|reference]
+  python bench.py [--gpus N --steps K --warmup W] [--workload lorenz_1m|lorenz_small|robertson|node64]
+                  [--dtype f64|f32] [--impl ours|reference]
 
 N > 1 runs under torchrun, one process per GPU; every rank owns its own
-2**20 trajectories (weak scaling, no data-path collective: trajectories are
-independent), timings are the max over ranks.  Inputs (mesh ~5 GB,
-checkpoints ~14 GB per rank) are far larger than L2, so no flush is needed.
-The CPU oracle appears twice: as ``cpu_baseline`` (a bounded sample timed on
-the host cores, rank 0, N = 1) and as the whole ``--impl reference`` arm.
+ensemble of the workload's size (weak scaling, no data-path collective:
+trajectories are independent); timings are the max over ranks.  Inputs of the
+default workload (mesh ~5 GB, checkpoints ~14 GB per rank) are far larger than
+L2, so no flush is needed.  The CPU oracle appears twice: as ``cpu_baseline``
+(a bounded sample timed on the host cores, rank 0, N = 1) and as the whole
+``--impl reference`` arm.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -30,14 +35,37 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-PASSES = 10
-# algorithmic flops of one Lorenz Tsit5 step: the forward replay step
-# (12 add + 30 mul + 75 fma = 192) plus its transposed step (264, see DESIGN)
-FLOP_FWD, FLOP_REV = 192, 264
-FLOP_LOSS_PER_SAVE = 18  # 3 sub + 3 fma forward, 3 sub + 3 fma reverse
-# FP64 peak derived from unit counts and clocks: 148 SMs x 64 FP64 FMA/clk x 2
+# Peaks derived from unit counts and the maximum SM clock: 148 SMs x 64 FP64
+# (128 FP32) fused multiply-adds per clock x 2 flops x 1965 MHz.
 FP64_PEAK = 148 * 64 * 2 * 1965e6
 FP32_PEAK = 148 * 128 * 2 * 1965e6
+
+# Per workload: gradient passes per recorded mesh, algorithmic flops of one
+# replay step (the forward step + its transposed step; fma = 2, division and
+# tanh = 1), flops per save point (loss term + its gradient), the gradient
+# kernel, and the configuration.
+WORKLOADS = {
+    "lorenz_1m": dict(passes=10, flop_step=192 + 264, flop_save=18, kernel="k_grad_tsit5_lorenz", n=1 << 20,
+                      dtype="f64",
+                      desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, 10 save points with N(0,1) targets, "
+                           "1 record + 10 gradient passes"),
+    "lorenz_small": dict(passes=1, flop_step=192 + 264, flop_save=12, kernel="k_grad_tsit5_lorenz", n=1024,
+                         dtype="f64",
+                         desc="Lorenz d=3, t in [0,1], Tsit5 rtol=atol=1e-8, loss sum ||u(T)||^2, "
+                              "1 record + 1 gradient pass"),
+    "robertson": dict(passes=1, flop_step=110 + 131, flop_save=9, kernel="k_grad_ros2", n=65536, dtype="f64",
+                      desc="Robertson d=3, t in [0,1e5], ROS2 gamma=1+1/sqrt2, rtol=1e-6 atol=1e-10, "
+                           "loss w . u(T), 1 record + 1 gradient pass"),
+    "node64": dict(passes=1, flop_step=52992 + 104076, flop_save=384, kernel="k_replay_node64", n=131072,
+                   dtype="f32",
+                   desc="du/dt = tanh(W u + b_i) - u, d=64, shared W, t in [0,1], Tsit5 rtol=atol=1e-5, "
+                        "loss sum ||u(T)||^2, 1 record + 1 gradient pass"),
+}
+# profile of the headline kernel (DRAM traffic per replay step), valid while
+# the kernel's sources are unchanged
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_grad_tsit5_lorenz_traffic.json")
+KERNEL_SOURCES = ["discrete_adjoint_b200/csrc/grad_tsit5.cu", "discrete_adjoint_b200/csrc/vec.cuh",
+                  "discrete_adjoint_b200/csrc/common.cuh"]
 
 
 def parse():
@@ -45,15 +73,30 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--dtype", default="f64", choices=["f64", "f32"])
+    ap.add_argument("--workload", default="lorenz_1m", choices=list(WORKLOADS))
+    ap.add_argument("--dtype", default=None, choices=["f64", "f32"], help="default: the workload's own")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--n", type=int, default=None, help="trajectories per GPU (default 2**20)")
+    ap.add_argument("--n", type=int, default=None, help="trajectories per GPU (default: the workload's size)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    a = ap.parse_args()
+    a.dtype = a.dtype or WORKLOADS[a.workload]["dtype"]
+    a.n = a.n or WORKLOADS[a.workload]["n"]
+    return a
 
 
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def metric_name(args) -> str:
+    if args.workload == "lorenz_1m":
+        return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj)"
+    return f"trajectory-gradients/s ({args.workload} {args.dtype.replace('f', 'fp')})"
+
+
+def make_problem(args, seed_offset=0, n=None):
+    import workloads
+    return workloads.by_name(args.workload, n=n or args.n, dtype=args.dtype, seed_offset=seed_offset)
 
 
 class ClockSampler:
@@ -113,88 +156,123 @@ def bus_id_of(dev) -> str | None:
         return None
 
 
-def cpu_baseline(prob_full, sample: int):
-    """The oracle as it stands: record + one gradient pass of a sample, on the
-    host cores; scaled to the step's 1 record + 10 passes."""
+def smax_cap(workload):
+    import workloads
+    return 4 * workloads.SMAX[workload]
+
+
+def oracle_step_time(prob, threads, passes):
+    """Oracle record + `passes` tape gradient passes of `prob` on the host."""
     import oracle
-    sub = prob_full.subset(np.arange(sample))
-    threads = oracle.default_threads()
     t0 = time.perf_counter()
-    om = oracle.record(sub, 2048, nthreads=threads)
+    om = oracle.record(prob, smax_cap(prob.name), nthreads=threads)
     t1 = time.perf_counter()
-    oracle.grad(sub, om, nthreads=threads)
+    oracle.grad(prob, om, nthreads=threads)
     t2 = time.perf_counter()
-    per_step = (t1 - t0) + PASSES * (t2 - t1)
-    return {"value": sample * PASSES / per_step, "unit": "trajectory-gradients/s", "cores": threads,
+    return t1 - t0, t2 - t1, (t1 - t0) + passes * (t2 - t1)
+
+
+def cpu_baseline(args, sample: int):
+    """The oracle as it stands: record + one gradient pass of a sample of the
+    workload on the host cores, scaled to the step's record + passes."""
+    import oracle
+    prob = make_problem(args).subset(np.arange(sample))
+    threads = oracle.default_threads()
+    passes = WORKLOADS[args.workload]["passes"]
+    tr, tg, per_step = oracle_step_time(prob, threads, passes)
+    return {"value": sample * passes / per_step, "unit": "trajectory-gradients/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"{sample} of the {prob_full.n} trajectories: oracle record {t1 - t0:.2f} s + one tape "
-                      f"gradient pass {t2 - t1:.2f} s, scaled to 1 record + {PASSES} passes"}
+            "sample": f"first {sample} of the {args.n} trajectories: oracle record {tr:.2f} s + one tape gradient "
+                      f"pass {tg:.2f} s, scaled to 1 record + {passes} passes"}
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle on the host cores, same metric/config."""
+    """--impl reference: the CPU oracle on the host cores, same metric/config;
+    each step is the record + gradient passes of a bounded sample."""
     import oracle
-    import workloads
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    n_full = args.n or (1 << 20)
-    sample = 256
-    prob = workloads.lorenz_1m(sample, dtype=args.dtype)
+    W = WORKLOADS[args.workload]
+    sample = {"lorenz_1m": 256, "lorenz_small": 256, "robertson": 32, "node64": 64}[args.workload]
+    prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
     times = []
     for it in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        om = oracle.record(prob, 2048, nthreads=threads)
-        for _ in range(PASSES):
+        om = oracle.record(prob, smax_cap(args.workload), nthreads=threads)
+        for _ in range(W["passes"]):
             oracle.grad(prob, om, nthreads=threads)
         dt = time.perf_counter() - t0
         if it >= args.warmup:
             times.append(dt)
     t = float(np.mean(times))
-    value = sample * PASSES / t
-    line = {"impl": "reference", "metric": "trajectory-gradients/s (Lorenz fp64, 1M traj)", "value": value,
-            "unit": "trajectory-gradients/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": args.dtype, "data": "synthetic",
-            "config": {"workload": f"lorenz_1m: Lorenz d=3, n={n_full} per GPU, t in [0,10], Tsit5 rtol=atol=1e-6, "
-                                   f"10 save points, 1 record + {PASSES} gradient passes",
+    value = sample * W["passes"] / t
+    line = {"impl": "reference", "metric": metric_name(args), "value": value, "unit": "trajectory-gradients/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype,
+            "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {W['desc']}; n={args.n} per GPU",
                        "sample_per_step": sample},
             "cpu_baseline": {"value": value, "unit": "trajectory-gradients/s", "cores": threads, "kind": "oracle",
-                             "sample": f"{sample} trajectories per step (record + {PASSES} tape gradient passes)"},
+                             "sample": f"first {sample} trajectories per step (oracle record + {W['passes']} "
+                                       f"tape gradient passes)"},
             "e2e": {"value": value, "unit": "trajectory-gradients/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def kernel_traffic(total_steps: int):
+    """DRAM bytes per gradient launch from the committed ncu capture, scaled by
+    replay steps, or None if the kernel changed since the capture."""
+    try:
+        prof = json.load(open(TRAFFIC_FILE))
+        h = hashlib.sha256()
+        for f in KERNEL_SOURCES:
+            h.update(open(os.path.join(ROOT, f), "rb").read())
+        if h.hexdigest() != prof["sources_sha256"]:
+            return None
+        return prof["dram_bytes"] / prof["replay_steps"] * total_steps
+    except Exception:
+        return None
 
 
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    import workloads
     import discrete_adjoint_b200 as gs
 
+    W = WORKLOADS[args.workload]
+    passes = W["passes"]
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    n = args.n or (1 << 20)
-    prob = workloads.lorenz_1m(n, dtype=args.dtype, seed_offset=rank)
+    n = args.n
+    prob = make_problem(args, seed_offset=rank)
     td = torch.float64 if args.dtype == "f64" else torch.float32
     esz = 8 if args.dtype == "f64" else 4
     stream = torch.cuda.current_stream()
 
     # host inputs (pinned) and their device copies
-    h_p = torch.from_numpy(np.ascontiguousarray(prob.p)).to(td).pin_memory()
-    h_u0 = torch.from_numpy(np.ascontiguousarray(prob.u0)).to(td).pin_memory()
-    h_tg = torch.from_numpy(np.ascontiguousarray(prob.target)).to(td).pin_memory()
-    d_p, d_u0, d_tg = h_p.to(dev), h_u0.to(dev), h_tg.to(dev)
-    ens = gs.Ensemble("lorenz", "tsit5", args.dtype, d_p, d_u0, prob.t0, prob.t1, [float(x) for x in prob.tsave])
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(td).pin_memory()
+    host = {"p": pin(prob.p), "u0": pin(prob.u0)}
+    if prob.target is not None:
+        host["target"] = pin(prob.target)
+    if prob.weight is not None:
+        host["weight"] = pin(prob.weight)
+    if prob.W is not None:
+        host["W"] = pin(prob.W)
+    d = {k: v.to(dev) for k, v in host.items()}
+    ens = gs.Ensemble(prob.system, prob.method, args.dtype, d["p"], d["u0"], prob.t0, prob.t1,
+                      [float(x) for x in prob.tsave], d.get("W"))
+    loss_kw = dict(loss=prob.loss, target=d.get("target"), weight=d.get("weight"))
 
     # sizing pass (setup, untimed): mesh capacity = the longest chain
-    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, 4096)
+    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload))
     smax = int(nsteps.max().item())
     mesh = gs.new_mesh(n, smax, len(prob.tsave), args.dtype, dev)
     ws_rec = gs.workspace(gs.gs_workspace_bytes(ens, mesh, gs.gradsolve.OP_RECORD), dev)
@@ -202,23 +280,22 @@ def run_ours(args):
     outs = [gs.new_grad_out(ens) for _ in range(2)]
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    grad_events = []
-    rec_events = []
+    grad_events, rec_events = [], []
 
     def step(timing):
-        e0 = ev() if timing else None
         if timing:
+            e0 = ev()
             e0.record(stream)
         gs.gs_record(ens, mesh, prob.rtol, prob.atol, ws=ws_rec, stream=stream)
         if timing:
             e1 = ev()
             e1.record(stream)
             rec_events.append((e0, e1))
-        for k in range(PASSES):
+        for k in range(passes):
             if timing:
                 a = ev()
                 a.record(stream)
-            gs.gs_grad(ens, mesh, "sumsq", target=d_tg, out=outs[k % 2], ws=ws_grad, stream=stream)
+            gs.gs_grad(ens, mesh, out=outs[k % 2], ws=ws_grad, stream=stream, **loss_kw)
             if timing:
                 b = ev()
                 b.record(stream)
@@ -252,22 +329,22 @@ def run_ours(args):
     elapsed, grad_ms, rec_ms = tmax.tolist()
 
     # end to end through the public API from host buffers: H2D of the inputs,
-    # the record, and per pass the gradient plus a D2H read of (loss, dp, du0)
-    h_loss = torch.empty(n, dtype=td).pin_memory()
-    h_dp = torch.empty((3, n), dtype=td).pin_memory()
-    h_du0 = torch.empty((3, n), dtype=td).pin_memory()
+    # the record, and per pass the gradient plus a D2H read of its results
+    o0 = outs[0]
+    h_out = [torch.empty(t.shape, dtype=td).pin_memory() for t in (o0.loss, o0.dp, o0.du0)]
+    if o0.dshared is not None:
+        h_out.append(torch.empty(o0.dshared.shape, dtype=td).pin_memory())
 
     def e2e_step():
-        d_p.copy_(h_p, non_blocking=True)
-        d_u0.copy_(h_u0, non_blocking=True)
-        d_tg.copy_(h_tg, non_blocking=True)
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
         gs.gs_record(ens, mesh, prob.rtol, prob.atol, ws=ws_rec, stream=stream)
-        for k in range(PASSES):
+        for k in range(passes):
             o = outs[k % 2]
-            gs.gs_grad(ens, mesh, "sumsq", target=d_tg, out=o, ws=ws_grad, stream=stream)
-            h_loss.copy_(o.loss, non_blocking=True)
-            h_dp.copy_(o.dp, non_blocking=True)
-            h_du0.copy_(o.du0, non_blocking=True)
+            gs.gs_grad(ens, mesh, out=o, ws=ws_grad, stream=stream, **loss_kw)
+            srcs = [o.loss, o.dp, o.du0] + ([o.dshared] if o.dshared is not None else [])
+            for hb, src in zip(h_out, srcs):
+                hb.copy_(src, non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 3))
     e2e_step()
@@ -281,44 +358,42 @@ def run_ours(args):
     e2e_t = torch.tensor([a.elapsed_time(b) / 1e3 / e2e_steps], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    h2d = (h_p.numel() + h_u0.numel() + h_tg.numel()) * esz
-    d2h = PASSES * (h_loss.numel() + h_dp.numel() + h_du0.numel()) * esz
+    h2d = sum(v.numel() for v in host.values()) * esz
+    d2h = passes * sum(t.numel() for t in h_out) * esz
 
     # algorithmic work of one gradient launch
     total_steps = int(mesh.nsteps.sum().item())
-    flops = (FLOP_FWD + FLOP_REV) * total_steps + FLOP_LOSS_PER_SAVE * len(prob.tsave) * n
+    flops = W["flop_step"] * total_steps + W["flop_save"] * len(prob.tsave) * n
     achieved = flops / (grad_ms / 1e3)
     peak = FP64_PEAK if args.dtype == "f64" else FP32_PEAK
     ns = mesh.nsteps.double()
-    value = world * n * PASSES * args.steps / elapsed
+    value = world * n * passes * args.steps / elapsed
+    traffic = kernel_traffic(total_steps) if (args.workload == "lorenz_1m" and args.dtype == "f64") else None
     line = {
-        "metric": "trajectory-gradients/s (Lorenz fp64, 1M traj)" if args.dtype == "f64"
-        else "trajectory-gradients/s (Lorenz fp32, 1M traj)",
-        "value": value, "unit": "trajectory-gradients/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
-        "config": {"workload": f"lorenz_1m: Lorenz d=3, n={n} per GPU, t in [0,10], Tsit5 rtol=atol=1e-6, "
-                               f"10 save points with N(0,1) targets, 1 record + {PASSES} gradient passes per step",
-                   "n_per_gpu": n, "passes_per_step": PASSES, "smax": smax,
+        "metric": metric_name(args), "value": value, "unit": "trajectory-gradients/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {W['desc']}; n={n} per GPU",
+                   "n_per_gpu": n, "passes_per_step": passes, "smax": smax,
                    "steps_total": total_steps, "steps_mean": float(ns.mean()),
                    "steps_max_over_mean": float(ns.max() / ns.mean()),
-                   "grad_ms": grad_ms, "record_ms": rec_ms,
-                   "grad_only_value": world * n / (grad_ms / 1e3),
-                   "l2": "inputs larger than L2 (mesh %.1f GB, checkpoints %.1f GB); no flush" % (
+                   "grad_ms": grad_ms, "record_ms": rec_ms, "grad_only_value": world * n / (grad_ms / 1e3),
+                   "l2": "inputs larger than L2 (mesh %.2f GB, gradient workspace %.2f GB); no flush" % (
                        mesh.h.numel() * esz / 1e9, ws_grad.numel() / 1e9),
                    "parallelism": f"dp{world} (independent trajectory shards)"},
         "clocks": clocks,
-        "e2e": {"value": world * n * PASSES / float(e2e_t.item()), "unit": "trajectory-gradients/s",
+        "e2e": {"value": world * n * passes / float(e2e_t.item()), "unit": "trajectory-gradients/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": peak / 1e12, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "kernel": "k_grad_tsit5_lorenz", "peak_source": "derived: 148 SMs x %d FMA/clk x 2 x 1965 MHz"
-                     % (64 if args.dtype == "f64" else 128),
+                     "frac": achieved / peak, "traffic": traffic, "kernel": W["kernel"],
+                     "peak_source": "derived: 148 SMs x %d %s FMA/clk x 2 x 1965 MHz" % (
+                         64 if args.dtype == "f64" else 128, "FP64" if args.dtype == "f64" else "FP32"),
                      "flops_per_launch": flops},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(prob, 2048)
+        sample = {"lorenz_1m": 2048, "lorenz_small": 1024, "robertson": 64, "node64": 256}[args.workload]
+        line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
