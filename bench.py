@@ -53,7 +53,7 @@ WORKLOADS = {
                          dtype="f64",
                          desc="Lorenz d=3, t in [0,1], Tsit5 rtol=atol=1e-8, loss sum ||u(T)||^2, "
                               "1 record + 1 gradient pass"),
-    "robertson": dict(passes=1, flop_step=110 + 131, flop_save=9, kernel="k_grad_ros2", n=65536, dtype="f64",
+    "robertson": dict(passes=1, flop_step=113 + 131, flop_save=9, kernel="k_grad_ros2", n=65536, dtype="f64",
                       desc="Robertson d=3, t in [0,1e5], ROS2 gamma=1+1/sqrt2, rtol=1e-6 atol=1e-10, "
                            "loss w . u(T), 1 record + 1 gradient pass"),
     "node64": dict(passes=1, flop_step=52992 + 104076, flop_save=384, kernel="k_replay_node64", n=131072,

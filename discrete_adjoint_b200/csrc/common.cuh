@@ -111,9 +111,11 @@ __device__ __forceinline__ void robertson_J(T y1, T y2, T y3, T k1, T k2, T k3, 
 
 // 3x3 LU with partial pivoting (largest |entry|, ties to the lowest row),
 // right-looking; whole rows swap.  Fully unrolled so M and P stay in registers.
-// Returns false on a zero or non-finite pivot.
+// R receives the reciprocals of the pivots (one division each); multipliers
+// and back substitution multiply by them.  Returns false on a zero or
+// non-finite pivot.
 template <typename T>
-__device__ __forceinline__ bool lu3(T M[9], int P[3]) {
+__device__ __forceinline__ bool lu3(T M[9], int P[3], T R[3]) {
   P[0] = 0;
   P[1] = 1;
   P[2] = 2;
@@ -140,9 +142,10 @@ __device__ __forceinline__ bool lu3(T M[9], int P[3]) {
     }
     T pv = M[k * 3 + k];
     ok = ok && (pv != cst<T>(0.0)) && isfinite(pv);
+    R[k] = cst<T>(1.0) / pv;
 #pragma unroll
     for (int i = k + 1; i < 3; ++i) {
-      T l = M[i * 3 + k] / M[k * 3 + k];
+      T l = M[i * 3 + k] * R[k];
       M[i * 3 + k] = l;
 #pragma unroll
       for (int j = k + 1; j < 3; ++j) M[i * 3 + j] = fmaT(-l, M[k * 3 + j], M[i * 3 + j]);
@@ -158,29 +161,31 @@ __device__ __forceinline__ T pick3(int i, T a, T b, T c) {
 
 // Solve (P M) x = P b with the factors of lu3: x = M^{-1} b.
 template <typename T>
-__device__ __forceinline__ void lu3_solve(const T LU[9], const int P[3], T b0, T b1, T b2, T& x0, T& x1, T& x2) {
+__device__ __forceinline__ void lu3_solve(const T LU[9], const int P[3], const T R[3], T b0, T b1, T b2, T& x0,
+                                          T& x1, T& x2) {
   x0 = pick3(P[0], b0, b1, b2);
   x1 = pick3(P[1], b0, b1, b2);
   x2 = pick3(P[2], b0, b1, b2);
   x1 = fmaT(-LU[3], x0, x1);
   x2 = fmaT(-LU[6], x0, x2);
   x2 = fmaT(-LU[7], x1, x2);
-  x2 = x2 / LU[8];
+  x2 = x2 * R[2];
   x1 = fmaT(-LU[5], x2, x1);
-  x1 = x1 / LU[4];
+  x1 = x1 * R[1];
   x0 = fmaT(-LU[1], x1, x0);
   x0 = fmaT(-LU[2], x2, x0);
-  x0 = x0 / LU[0];
+  x0 = x0 * R[0];
 }
 
 // Solve M^T x = b with the factors of lu3 (P M = L U, so M^T = U^T L^T P):
 // U^T y = b (forward), L^T z = y (backward, unit diagonal), x[P[i]] = z[i].
 // Used by the reverse sweep only (not part of the bitwise contract).
 template <typename T>
-__device__ __forceinline__ void lu3_solve_T(const T LU[9], const int P[3], T b0, T b1, T b2, T& x0, T& x1, T& x2) {
-  T y0 = b0 / LU[0];
-  T y1 = fmaT(-LU[1], y0, b1) / LU[4];
-  T y2 = fmaT(-LU[5], y1, fmaT(-LU[2], y0, b2)) / LU[8];
+__device__ __forceinline__ void lu3_solve_T(const T LU[9], const int P[3], const T R[3], T b0, T b1, T b2, T& x0,
+                                            T& x1, T& x2) {
+  T y0 = b0 * R[0];
+  T y1 = fmaT(-LU[1], y0, b1) * R[1];
+  T y2 = fmaT(-LU[5], y1, fmaT(-LU[2], y0, b2)) * R[2];
   T z2 = y2;
   T z1 = fmaT(-LU[7], z2, y1);
   T z0 = fmaT(-LU[6], z2, fmaT(-LU[3], z1, y0));

@@ -162,9 +162,9 @@ __global__ void __launch_bounds__(128) k_grad_ros2(Ros2Args<T> a) {
     cp[n] = u[1];
     cp[2 * n] = u[2];
     cp += n3;
-    T LU[9], k1[3], v[3], k2[3], un[3];
+    T LU[9], R[3], k1[3], v[3], k2[3], un[3];
     int P[3];
-    ok = ros2_fwd<T, SYS>(u, p, h, LU, P, k1, v, k2, un) && ok;
+    ok = ros2_fwd<T, SYS>(u, p, h, LU, P, R, k1, v, k2, un) && ok;
 #pragma unroll
     for (int c = 0; c < 3; ++c) u[c] = un[c];
     if (st + 1 == next) {
@@ -187,15 +187,15 @@ __global__ void __launch_bounds__(128) k_grad_ros2(Ros2Args<T> a) {
     cp -= n3;
     T us[3] = {cp[0], cp[n], cp[2 * n]};
     const T h = hp[(int64_t)st * n];
-    T LU[9], k1[3], v[3], k2[3], un[3];
+    T LU[9], R[3], k1[3], v[3], k2[3], un[3];
     int P[3];
-    ros2_fwd<T, SYS>(us, p, h, LU, P, k1, v, k2, un);
+    ros2_fwd<T, SYS>(us, p, h, LU, P, R, k1, v, k2, un);
     const T gh = cst<T>(ROS2_GAMMA) * h;
     T ub[3] = {lam[0], lam[1], lam[2]};
     T kb1[3], rb[3], qb[3];
 #pragma unroll
     for (int c = 0; c < 3; ++c) kb1[c] = (cst<T>(1.5) * h) * lam[c];
-    lu3_solve_T(LU, P, (cst<T>(0.5) * h) * lam[0], (cst<T>(0.5) * h) * lam[1], (cst<T>(0.5) * h) * lam[2], rb[0],
+    lu3_solve_T(LU, P, R, (cst<T>(0.5) * h) * lam[0], (cst<T>(0.5) * h) * lam[1], (cst<T>(0.5) * h) * lam[2], rb[0],
                 rb[1], rb[2]);
     T vb[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)};
     vjp3<T, SYS>(v, p, rb, vb, pb);
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(128) k_grad_ros2(Ros2Args<T> a) {
       ub[c] += vb[c];
       kb1[c] = fmaT(h, vb[c], fmaT(cst<T>(-2.0), rb[c], kb1[c]));
     }
-    lu3_solve_T(LU, P, kb1[0], kb1[1], kb1[2], qb[0], qb[1], qb[2]);
+    lu3_solve_T(LU, P, R, kb1[0], kb1[1], kb1[2], qb[0], qb[1], qb[2]);
     vjp3<T, SYS>(us, p, qb, ub, pb);
     jac_adjoint3<T, SYS>(us, p, gh, rb, qb, k1, k2, ub, pb);
 #pragma unroll

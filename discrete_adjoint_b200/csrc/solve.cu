@@ -56,9 +56,9 @@ __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
 #pragma unroll
       for (int c = 0; c < 3; ++c) k1[c] = k7[c];
     } else {
-      T LU[9], q1[3], v[3], q2[3];
+      T LU[9], R[3], q1[3], v[3], q2[3];
       int P[3];
-      ros2_fwd<T, SYS>(u, p, h, LU, P, q1, v, q2, un);
+      ros2_fwd<T, SYS>(u, p, h, LU, P, R, q1, v, q2, un);
     }
 #pragma unroll
     for (int c = 0; c < 3; ++c) u[c] = un[c];

@@ -191,23 +191,23 @@ __device__ __forceinline__ void tsit5_err_step(const T u[3], const T p[3], T h, 
 // One ROS2 step with error estimate.  Returns false on a singular matrix.
 template <typename T, int SYS>
 __device__ __forceinline__ bool ros2_err_step(const T u[3], const T p[3], T h, T un[3], T e[3]) {
-  T J[9], M[9];
+  T J[9], M[9], R[3];
   int P[3];
   jac3<T, SYS>(u, p, J);
   const T gh = cst<T>(ROS2_GAMMA) * h;
 #pragma unroll
   for (int q = 0; q < 9; ++q) M[q] = fmaT(-gh, J[q], cst<T>((q % 4) == 0 ? 1.0 : 0.0));
-  if (!lu3(M, P)) return false;
+  if (!lu3(M, P, R)) return false;
   T f0[3], k1[3], v[3], f1[3], k2[3];
   rhs3<T, SYS>(u, p, f0);
-  lu3_solve(M, P, f0[0], f0[1], f0[2], k1[0], k1[1], k1[2]);
+  lu3_solve(M, P, R, f0[0], f0[1], f0[2], k1[0], k1[1], k1[2]);
 #pragma unroll
   for (int c = 0; c < 3; ++c) v[c] = fmaT(h, k1[c], u[c]);
   rhs3<T, SYS>(v, p, f1);
   T r0 = fmaT(cst<T>(-2.0), k1[0], f1[0]);
   T r1 = fmaT(cst<T>(-2.0), k1[1], f1[1]);
   T r2 = fmaT(cst<T>(-2.0), k1[2], f1[2]);
-  lu3_solve(M, P, r0, r1, r2, k2[0], k2[1], k2[2]);
+  lu3_solve(M, P, R, r0, r1, r2, k2[0], k2[1], k2[2]);
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
     T acc = cst<T>(1.5) * k1[c];
@@ -220,24 +220,24 @@ __device__ __forceinline__ bool ros2_err_step(const T u[3], const T p[3], T h, T
 
 // Bitwise forward step; also returns the pieces the reverse sweep needs.
 template <typename T, int SYS>
-__device__ __forceinline__ bool ros2_fwd(const T u[3], const T p[3], T h, T LU[9], int P[3], T k1[3], T v[3],
-                                         T k2[3], T un[3]) {
+__device__ __forceinline__ bool ros2_fwd(const T u[3], const T p[3], T h, T LU[9], int P[3], T R[3], T k1[3],
+                                         T v[3], T k2[3], T un[3]) {
   T J[9];
   jac3<T, SYS>(u, p, J);
   const T gh = cst<T>(ROS2_GAMMA) * h;
 #pragma unroll
   for (int q = 0; q < 9; ++q) LU[q] = fmaT(-gh, J[q], cst<T>((q % 4) == 0 ? 1.0 : 0.0));
-  bool ok = lu3(LU, P);
+  bool ok = lu3(LU, P, R);
   T f0[3], f1[3];
   rhs3<T, SYS>(u, p, f0);
-  lu3_solve(LU, P, f0[0], f0[1], f0[2], k1[0], k1[1], k1[2]);
+  lu3_solve(LU, P, R, f0[0], f0[1], f0[2], k1[0], k1[1], k1[2]);
 #pragma unroll
   for (int c = 0; c < 3; ++c) v[c] = fmaT(h, k1[c], u[c]);
   rhs3<T, SYS>(v, p, f1);
   T r0 = fmaT(cst<T>(-2.0), k1[0], f1[0]);
   T r1 = fmaT(cst<T>(-2.0), k1[1], f1[1]);
   T r2 = fmaT(cst<T>(-2.0), k1[2], f1[2]);
-  lu3_solve(LU, P, r0, r1, r2, k2[0], k2[1], k2[2]);
+  lu3_solve(LU, P, R, r0, r1, r2, k2[0], k2[1], k2[2]);
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
     T acc = cst<T>(1.5) * k1[c];

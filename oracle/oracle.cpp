@@ -299,11 +299,13 @@ void tsit5_step(int sys, int d, const S* u, const S* p, const S* W, S h, S* unew
 
 // ---------------------------------------------------------------------------
 // LU with partial pivoting (largest |entry|, ties to the lowest row), Doolittle
-// right-looking order; multipliers stored below the diagonal.  Returns false on
-// an exactly zero or non-finite pivot.
+// right-looking order; multipliers stored below the diagonal.  Each pivot's
+// reciprocal is formed once (one division) and the multipliers and the back
+// substitution multiply by it.  Returns false on an exactly zero or
+// non-finite pivot.
 // ---------------------------------------------------------------------------
 template <class S>
-bool lu_factor(int d, S* M, int* P) {
+bool lu_factor(int d, S* M, int* P, S* R) {
   using T = typename base_of<S>::type;
   for (int i = 0; i < d; ++i) P[i] = i;
   for (int k = 0; k < d; ++k) {
@@ -316,8 +318,9 @@ bool lu_factor(int d, S* M, int* P) {
     }
     T pv = val(M[k * d + k]);
     if (pv == T(0) || !std::isfinite(pv)) return false;
+    R[k] = S(T(1)) / M[k * d + k];
     for (int i = k + 1; i < d; ++i) {
-      S l = M[i * d + k] / M[k * d + k];
+      S l = M[i * d + k] * R[k];
       M[i * d + k] = l;
       for (int j = k + 1; j < d; ++j) M[i * d + j] = fma_(-l, M[k * d + j], M[i * d + j]);
     }
@@ -326,13 +329,13 @@ bool lu_factor(int d, S* M, int* P) {
 }
 
 template <class S>
-void lu_solve(int d, const S* LU, const int* P, const S* b, S* x) {
+void lu_solve(int d, const S* LU, const int* P, const S* R, const S* b, S* x) {
   for (int i = 0; i < d; ++i) x[i] = b[P[i]];
   for (int i = 1; i < d; ++i)
     for (int j = 0; j < i; ++j) x[i] = fma_(-LU[i * d + j], x[j], x[i]);
   for (int i = d - 1; i >= 0; --i) {
     for (int j = i + 1; j < d; ++j) x[i] = fma_(-LU[i * d + j], x[j], x[i]);
-    x[i] = x[i] / LU[i * d + i];
+    x[i] = x[i] * R[i];
   }
 }
 
@@ -347,20 +350,20 @@ template <class S>
 bool ros2_step(int sys, int d, const S* u, const S* p, S h, S* unew, S* err) {
   using T = typename base_of<S>::type;
   S J[64];
-  S M[64];
+  S M[64], R[8];
   int P[8];
   jac<S>(sys, u, p, J);
   S gh = S(T(ROS2_GAMMA)) * h;
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) M[i * d + j] = fma_(-gh, J[i * d + j], S(T(i == j ? 1 : 0)));
-  if (!lu_factor<S>(d, M, P)) return false;
+  if (!lu_factor<S>(d, M, P, R)) return false;
   S f0[8] = {}, k1[8] = {}, v[8] = {}, f1[8] = {}, r[8] = {}, k2[8] = {};
   rhs<S>(sys, u, p, nullptr, f0);
-  lu_solve<S>(d, M, P, f0, k1);
+  lu_solve<S>(d, M, P, R, f0, k1);
   for (int c = 0; c < d; ++c) v[c] = fma_(h, k1[c], u[c]);
   rhs<S>(sys, v, p, nullptr, f1);
   for (int c = 0; c < d; ++c) r[c] = fma_(S(T(-2)), k1[c], f1[c]);
-  lu_solve<S>(d, M, P, r, k2);
+  lu_solve<S>(d, M, P, R, r, k2);
   for (int c = 0; c < d; ++c) {
     S acc = S(T(1.5)) * k1[c];
     acc = fma_(S(T(0.5)), k2[c], acc);
