@@ -328,23 +328,34 @@ def run_ours(args):
         dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
     elapsed, grad_ms, rec_ms = tmax.tolist()
 
-    # end to end through the public API from host buffers: H2D of the inputs,
-    # the record, and per pass the gradient plus a D2H read of its results
+    # End to end through the public API from host buffers: H2D of the inputs,
+    # the record, and per pass the gradient plus a D2H read of its results.
+    # Pass k's results go back on a copy stream while pass k + 1 computes into
+    # the other output buffer (the compute stream waits before reusing one).
     o0 = outs[0]
-    h_out = [torch.empty(t.shape, dtype=td).pin_memory() for t in (o0.loss, o0.dp, o0.du0)]
-    if o0.dshared is not None:
-        h_out.append(torch.empty(o0.dshared.shape, dtype=td).pin_memory())
+    shapes = [t.shape for t in (o0.loss, o0.dp, o0.du0)] + ([o0.dshared.shape] if o0.dshared is not None else [])
+    h_out = [[torch.empty(sh, dtype=td).pin_memory() for sh in shapes] for _ in range(2)]
+    copy_stream = torch.cuda.Stream(device=dev)
+    done_copy = [torch.cuda.Event(), torch.cuda.Event()]
+    done_grad = [torch.cuda.Event(), torch.cuda.Event()]
 
     def e2e_step():
         for k, v in host.items():
             d[k].copy_(v, non_blocking=True)
         gs.gs_record(ens, mesh, prob.rtol, prob.atol, ws=ws_rec, stream=stream)
         for k in range(passes):
-            o = outs[k % 2]
+            b = k % 2
+            o = outs[b]
+            stream.wait_event(done_copy[b])  # its previous contents are on the host
             gs.gs_grad(ens, mesh, out=o, ws=ws_grad, stream=stream, **loss_kw)
-            srcs = [o.loss, o.dp, o.du0] + ([o.dshared] if o.dshared is not None else [])
-            for hb, src in zip(h_out, srcs):
-                hb.copy_(src, non_blocking=True)
+            done_grad[b].record(stream)
+            copy_stream.wait_event(done_grad[b])
+            with torch.cuda.stream(copy_stream):
+                srcs = [o.loss, o.dp, o.du0] + ([o.dshared] if o.dshared is not None else [])
+                for hb, src in zip(h_out[b], srcs):
+                    hb.copy_(src, non_blocking=True)
+            done_copy[b].record(copy_stream)
+        stream.wait_stream(copy_stream)
 
     e2e_steps = max(1, min(args.steps, 3))
     e2e_step()
@@ -359,7 +370,7 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
     h2d = sum(v.numel() for v in host.values()) * esz
-    d2h = passes * sum(t.numel() for t in h_out) * esz
+    d2h = passes * sum(t.numel() for t in h_out[0]) * esz
 
     # algorithmic work of one gradient launch
     total_steps = int(mesh.nsteps.sum().item())
