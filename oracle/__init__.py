@@ -65,6 +65,8 @@ def lib():
                                   dp, dp, dp, dp, i32]
         L.or_replay.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, i32, dp, dp,
                                 dp, dp, i32]
+        L.or_solve_adaptive.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, f64, f64, i32, dp, f64, f64,
+                                        f64, i32, dp, ip, ip, i32]
         L.or_count_step.argtypes = [i32, i32, i32, i32, dp]
         L.or_step.argtypes = [i32, i32, i32, i32, dp, dp, dp, f64, dp, dp]
         L.or_rhs.argtypes = [i32, i32, dp, dp, dp, dp, dp]
@@ -131,6 +133,23 @@ def record(prob, smax: int, h0: float = 0.0, nthreads: int | None = None) -> Mes
                      _d(h), _i(nsteps), _i(save_idx), _i(status), _i(nrej), nthreads or default_threads())
     _check(rc, "record")
     return Mesh(h, nsteps, save_idx[:, :nsave], status, nrej)
+
+
+def solve_adaptive(prob, smax: int, h0: float = 0.0, nthreads: int | None = None):
+    """Adaptive forward-only solve: (u_save [nsave][d][n], nsteps [n], status [n]).
+    The recorder's iteration with its accepted states at the save times kept
+    (NaN everywhere for a trajectory whose status is not 0)."""
+    L = lib()
+    n, nsave = prob.n, len(prob.tsave)
+    us = np.zeros((nsave, prob.d, n))
+    nsteps = np.zeros(n, np.int32)
+    status = np.zeros(n, np.int32)
+    rc = L.or_solve_adaptive(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, prob.d, prob.np_,
+                             _d(_f64(prob.p)), _d(_f64(prob.u0)), _d(_f64(prob.W)), prob.t0, prob.t1, nsave,
+                             _d(_f64(prob.tsave)), prob.rtol, prob.atol, h0, smax, _d(us), _i(nsteps), _i(status),
+                             nthreads or default_threads())
+    _check(rc, "solve_adaptive")
+    return us, nsteps, status
 
 
 def _mesh_args(mesh: Mesh):

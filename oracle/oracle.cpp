@@ -452,6 +452,7 @@ struct RecordOut {
   std::vector<T> h;
   int nsteps = 0, nreject = 0, status = TRAJ_OK;
   std::vector<int> save_idx;
+  std::vector<T> usave;  // [nsave][d]: the accepted state at each save time (the forward-only solve)
 };
 
 template <class T>
@@ -489,6 +490,7 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
                         int nsave, const T* tsave, T rtol, T atol, T h0user, int smax) {
   RecordOut<T> out;
   out.save_idx.assign(nsave, 0);
+  out.usave.assign((size_t)nsave * d, std::numeric_limits<T>::quiet_NaN());
   const T eps = std::numeric_limits<T>::epsilon();
   const T q = method == M_TSIT5 ? T(5) : T(2);
   T u[DMAX], un[DMAX], e[DMAX], sc[DMAX], f0[DMAX];
@@ -536,7 +538,10 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
       out.nsteps++;
       t = clipped ? tstop : tn;
       for (int c = 0; c < d; ++c) u[c] = un[c];
-      while (kk < nsave && t == tsave[kk]) out.save_idx[kk++] = out.nsteps;
+      while (kk < nsave && t == tsave[kk]) {
+        for (int c = 0; c < d; ++c) out.usave[(size_t)kk * d + c] = u[c];
+        out.save_idx[kk++] = out.nsteps;
+      }
       // fac = 0.9 err^(-0.7/q) errprev^(0.4/q) = 0.9 exp(-(0.7/q) ln err + (0.4/q) ln errprev)
       T fac, lnerr = ln_floor;
       if (err == T(0)) {
@@ -797,6 +802,43 @@ int or_record(int sys, int method, int dtype, int64_t n, int d, int np, const do
         nreject[i] = r.nreject;
         for (int s = 0; s < smax; ++s) h[i * smax + s] = s < r.nsteps ? double(r.h[s]) : 0.0;
         for (int k = 0; k < nsave; ++k) save_idx[i * nsave + k] = r.save_idx[k];
+      }
+    };
+    if (dtype == DT_F64) run(double(0)); else run(float(0));
+  });
+  return 0;
+}
+
+// Adaptive forward-only solve (GRADSOLVE abstract: the forward-only solver):
+// the recorder's own iteration, returning the accepted state at each save time
+// instead of the mesh.  u_save [nsave][d][n] (NaN for every save point of a
+// trajectory with status != 0), nsteps and status [n].
+int or_solve_adaptive(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
+                      const double* W, double t0, double t1, int nsave, const double* tsave, double rtol,
+                      double atol, double h0, int smax, double* u_save, int* nsteps, int* status, int nthreads) {
+  Prob P{sys, method, dtype, d, np, n, p, u0, W};
+  int rc = check_prob(P);
+  if (rc) return rc;
+  parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
+    auto run = [&](auto tag) {
+      using T = decltype(tag);
+      std::vector<T> uu(d), pp(np), WW, ts(nsave);
+      for (int k = 0; k < nsave; ++k) ts[k] = T(tsave[k]);
+      if (sys == SYS_NODE64) {
+        WW.resize(4096);
+        for (int c = 0; c < 4096; ++c) WW[c] = T(W[c]);
+      }
+      for (int64_t i = a; i < b; ++i) {
+        for (int c = 0; c < d; ++c) uu[c] = T(u0[(int64_t)c * n + i]);
+        for (int c = 0; c < np; ++c) pp[c] = T(p[(int64_t)c * n + i]);
+        RecordOut<T> r = record_one<T>(sys, method, d, uu.data(), pp.data(), WW.empty() ? nullptr : WW.data(),
+                                       T(t0), T(t1), nsave, ts.data(), T(rtol), T(atol), T(h0), smax);
+        nsteps[i] = r.nsteps;
+        status[i] = r.status;
+        for (int k = 0; k < nsave; ++k)
+          for (int c = 0; c < d; ++c)
+            u_save[((int64_t)k * d + c) * n + i] =
+                r.status == TRAJ_OK ? double(r.usave[(size_t)k * d + c]) : std::numeric_limits<double>::quiet_NaN();
       }
     };
     if (dtype == DT_F64) run(double(0)); else run(float(0));
