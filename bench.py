@@ -9,8 +9,12 @@ record then ten gradient passes", in fp64.  The metric is
 trajectory-gradients/s over the whole step (record included); the gradient
 pass alone is reported in config.grad_only_value.
 
-  python bench.py [--gpus N --steps K --warmup W] [--workload lorenz_1m|lorenz_small|robertson|node64]
-                  [--dtype f64|f32] [--impl ours|reference]
+  python bench.py [--gpus N --steps K --warmup W] [--workload lorenz_1m|lorenz_small|robertson|node64|
+                  lorenz_1m_solve] [--dtype f64|f32] [--impl ours|reference]
+
+The lorenz_1m_solve workload times the adaptive forward-only solve instead
+(gs_solve_adaptive on the same ensemble, no mesh kept; metric
+trajectory-solves/s).
 
 N > 1 runs under torchrun, one process per GPU; every rank owns its own
 ensemble of the workload's size (weak scaling, no data-path collective:
@@ -60,6 +64,13 @@ WORKLOADS = {
                    dtype="f32",
                    desc="du/dt = tanh(W u + b_i) - u, d=64, shared W, t in [0,1], Tsit5 rtol=atol=1e-5, "
                         "loss sum ||u(T)||^2, 1 record + 1 gradient pass"),
+    # adaptive forward-only solve: flops per attempted step = the Tsit5 step
+    # (192) + its error estimate (7-term combination, scaling, RMS norm: 56);
+    # the step-size controller's scalar arithmetic is not counted
+    "lorenz_1m_solve": dict(kind="solve", problem="lorenz_1m", flop_attempt=192 + 56, kernel="k_record3", n=1 << 20,
+                            dtype="f64",
+                            desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, states at 10 save points, "
+                                 "one adaptive forward-only solve per step (no mesh kept)"),
 }
 # profile of the headline kernel (DRAM traffic per replay step), valid while
 # the kernel's sources are unchanged
@@ -89,6 +100,8 @@ def dist_env():
 
 
 def metric_name(args) -> str:
+    if args.workload == "lorenz_1m_solve":
+        return f"trajectory-solves/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, adaptive forward-only)"
     if args.workload == "lorenz_1m":
         return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj)"
     return f"trajectory-gradients/s ({args.workload} {args.dtype.replace('f', 'fp')})"
@@ -96,7 +109,8 @@ def metric_name(args) -> str:
 
 def make_problem(args, seed_offset=0, n=None):
     import workloads
-    return workloads.by_name(args.workload, n=n or args.n, dtype=args.dtype, seed_offset=seed_offset)
+    name = WORKLOADS[args.workload].get("problem", args.workload)
+    return workloads.by_name(name, n=n or args.n, dtype=args.dtype, seed_offset=seed_offset)
 
 
 class ClockSampler:
@@ -158,7 +172,7 @@ def bus_id_of(dev) -> str | None:
 
 def smax_cap(workload):
     import workloads
-    return 4 * workloads.SMAX[workload]
+    return 4 * workloads.SMAX[WORKLOADS[workload].get("problem", workload)]
 
 
 def oracle_step_time(prob, threads, passes):
@@ -174,10 +188,17 @@ def oracle_step_time(prob, threads, passes):
 
 def cpu_baseline(args, sample: int):
     """The oracle as it stands: record + one gradient pass of a sample of the
-    workload on the host cores, scaled to the step's record + passes."""
+    workload on the host cores, scaled to the step's record + passes (the
+    solve workload: the oracle's adaptive solve of the sample)."""
     import oracle
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
+    if WORKLOADS[args.workload].get("kind") == "solve":
+        t0 = time.perf_counter()
+        oracle.solve_adaptive(prob, smax_cap(args.workload), nthreads=threads)
+        dt = time.perf_counter() - t0
+        return {"value": sample / dt, "unit": "trajectory-solves/s", "cores": threads, "kind": "oracle",
+                "sample": f"first {sample} of the {args.n} trajectories: oracle adaptive solve {dt:.2f} s"}
     passes = WORKLOADS[args.workload]["passes"]
     tr, tg, per_step = oracle_step_time(prob, threads, passes)
     return {"value": sample * passes / per_step, "unit": "trajectory-gradients/s", "cores": threads,
@@ -194,31 +215,37 @@ def run_reference(args):
     if rank != 0:
         return
     W = WORKLOADS[args.workload]
-    sample = {"lorenz_1m": 256, "lorenz_small": 256, "robertson": 32, "node64": 64}[args.workload]
+    solve = W.get("kind") == "solve"
+    sample = {"lorenz_1m": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
+              "lorenz_1m_solve": 4096}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
     times = []
     for it in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        om = oracle.record(prob, smax_cap(args.workload), nthreads=threads)
-        for _ in range(W["passes"]):
-            oracle.grad(prob, om, nthreads=threads)
+        if solve:
+            oracle.solve_adaptive(prob, smax_cap(args.workload), nthreads=threads)
+        else:
+            om = oracle.record(prob, smax_cap(args.workload), nthreads=threads)
+            for _ in range(W["passes"]):
+                oracle.grad(prob, om, nthreads=threads)
         dt = time.perf_counter() - t0
         if it >= args.warmup:
             times.append(dt)
     t = float(np.mean(times))
-    value = sample * W["passes"] / t
-    line = {"impl": "reference", "metric": metric_name(args), "value": value, "unit": "trajectory-gradients/s",
+    passes = 1 if solve else W["passes"]
+    unit = "trajectory-solves/s" if solve else "trajectory-gradients/s"
+    what = "oracle adaptive solve" if solve else f"oracle record + {W['passes']} tape gradient passes"
+    value = sample * passes / t
+    line = {"impl": "reference", "metric": metric_name(args), "value": value, "unit": unit,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype,
             "data": "synthetic",
             "config": {"workload": f"{args.workload}: {W['desc']}; n={args.n} per GPU",
                        "sample_per_step": sample},
-            "cpu_baseline": {"value": value, "unit": "trajectory-gradients/s", "cores": threads, "kind": "oracle",
-                             "sample": f"first {sample} trajectories per step (oracle record + {W['passes']} "
-                                       f"tape gradient passes)"},
-            "e2e": {"value": value, "unit": "trajectory-gradients/s", "h2d_bytes_per_step": 0,
-                    "d2h_bytes_per_step": 0}}
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                             "sample": f"first {sample} trajectories per step ({what})"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -235,6 +262,129 @@ def kernel_traffic(total_steps: int):
         return prof["dram_bytes"] / prof["replay_steps"] * total_steps
     except Exception:
         return None
+
+
+def run_solve(args):
+    """The adaptive forward-only solve: one gs_solve_adaptive call over the
+    rank's ensemble per step."""
+    import torch
+    import torch.distributed as dist
+
+    import discrete_adjoint_b200 as gs
+
+    W = WORKLOADS[args.workload]
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    n = args.n
+    prob = make_problem(args, seed_offset=rank)
+    td = torch.float64 if args.dtype == "f64" else torch.float32
+    esz = 8 if args.dtype == "f64" else 4
+    stream = torch.cuda.current_stream()
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(td).pin_memory()
+    host = {"p": pin(prob.p), "u0": pin(prob.u0)}
+    d = {k: v.to(dev) for k, v in host.items()}
+    ens = gs.Ensemble(prob.system, prob.method, args.dtype, d["p"], d["u0"], prob.t0, prob.t1,
+                      [float(x) for x in prob.tsave])
+    smax = smax_cap(args.workload)
+    u_save = torch.empty((len(prob.tsave), prob.d, n), dtype=td, device=dev)
+    nsteps = torch.empty(n, dtype=torch.int32, device=dev)
+    status = torch.empty(n, dtype=torch.int32, device=dev)
+    # attempted steps (accepted + rejected), for the flop count: one untimed record
+    nst, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax)
+    mesh = gs.new_mesh(n, int(nst.max().item()), len(prob.tsave), args.dtype, dev)
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol, stream=stream)
+    attempts = int(mesh.nsteps.sum().item() + mesh.nreject.sum().item())
+    accepted = mesh.nsteps.double()
+    del mesh
+
+    def step():
+        gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, smax, u_save=u_save, nsteps=nsteps, status=status,
+                             stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clk = ClockSampler(bus_id_of(dev))
+    launches0 = gs.gs_launch_count()
+    barrier()
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    barrier()
+    launches = gs.gs_launch_count() - launches0
+    clocks = clk.stop()
+    tmax = torch.tensor([t_start.elapsed_time(t_end) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    elapsed = float(tmax.item())
+    assert (status == 0).all()
+
+    # end to end from host buffers: H2D of p and u0, the solve, D2H of the states
+    h_out = torch.empty(u_save.shape, dtype=td).pin_memory()
+
+    def e2e_step():
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        h_out.copy_(u_save, non_blocking=True)
+
+    e2e_step()
+    barrier()
+    e2e_steps = max(1, min(args.steps, 3))
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    barrier()
+    e2e_t = torch.tensor([a.elapsed_time(b) / 1e3 / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+
+    t_solve = elapsed / args.steps
+    flops = W["flop_attempt"] * attempts
+    achieved = flops / t_solve
+    peak = FP64_PEAK if args.dtype == "f64" else FP32_PEAK
+    line = {
+        "metric": metric_name(args), "value": world * n * args.steps / elapsed, "unit": "trajectory-solves/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_solve * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {W['desc']}; n={n} per GPU", "n_per_gpu": n,
+                   "attempted_steps": attempts, "steps_mean": float(accepted.mean()),
+                   "steps_max_over_mean": float(accepted.max() / accepted.mean()),
+                   "l2": "output states %.2f GB, larger than L2 together with the inputs; compute-bound, no flush"
+                         % (u_save.numel() * esz / 1e9),
+                   "parallelism": f"dp{world} (independent trajectory shards)"},
+        "clocks": clocks,
+        "e2e": {"value": world * n / float(e2e_t.item()), "unit": "trajectory-solves/s",
+                "h2d_bytes_per_step": sum(v.numel() for v in host.values()) * esz,
+                "d2h_bytes_per_step": h_out.numel() * esz},
+        "gpu_launches": launches,
+        "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": peak / 1e12, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": W["kernel"],
+                     "peak_source": "derived: 148 SMs x %d %s FMA/clk x 2 x 1965 MHz" % (
+                         64 if args.dtype == "f64" else 128, "FP64" if args.dtype == "f64" else "FP32"),
+                     "flops_per_launch": flops},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args, min(16384, n))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def run_ours(args):
@@ -416,6 +566,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif WORKLOADS[args.workload].get("kind") == "solve":
+        run_solve(args)
     else:
         run_ours(args)
 

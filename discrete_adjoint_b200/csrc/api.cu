@@ -14,6 +14,7 @@ void count_launch(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
 // kernels (defined in the other translation units)
 gs_status count3(const gs_problem*, const gs_tol*, int32_t, int32_t*, int32_t*, cudaStream_t);
 gs_status record3(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
+gs_status solve_adaptive3(const gs_problem*, const gs_tol*, int32_t, void*, int32_t*, int32_t*, cudaStream_t);
 size_t record_ws_bytes(int64_t n, int32_t smax, int32_t nsave, size_t tsize);
 template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
@@ -25,7 +26,7 @@ template <typename T>
 gs_status launch_solve3(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 gs_status record_node64(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
 gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,
-                             int32_t*, cudaStream_t);
+                             int32_t*, cudaStream_t, float*);
 gs_status node64_grad(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*, void*,
                       cudaStream_t);
 gs_status node64_solve(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
@@ -112,8 +113,24 @@ gs_status gs_count(const gs_problem* P, const gs_tol* tol, int32_t smax, int32_t
   if (P->n == 0) return GS_OK;
   if (!nsteps) return GS_EINVAL;
   if (P->system == GS_NODE64)
-    return node64_record_pass(P, tol, smax, false, nullptr, nullptr, nsteps, status, nullptr, (cudaStream_t)stream);
+    return node64_record_pass(P, tol, smax, false, nullptr, nullptr, nsteps, status, nullptr, (cudaStream_t)stream,
+                              nullptr);
   return count3(P, tol, smax, nsteps, status, (cudaStream_t)stream);
+}
+
+gs_status gs_solve_adaptive(const gs_problem* P, const gs_tol* tol, int32_t smax, void* u_save, int32_t* nsteps,
+                            int32_t* status, void* stream) {
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0) ||
+      smax < 1)
+    return GS_EINVAL;
+  if (P->n == 0) return GS_OK;
+  if (!u_save) return GS_EINVAL;
+  if (P->system == GS_NODE64)
+    return node64_record_pass(P, tol, smax, false, nullptr, nullptr, nsteps, status, nullptr, (cudaStream_t)stream,
+                              (float*)u_save);
+  return solve_adaptive3(P, tol, smax, u_save, nsteps, status, (cudaStream_t)stream);
 }
 
 gs_status gs_record(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, size_t ws_bytes,

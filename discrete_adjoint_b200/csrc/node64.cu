@@ -59,6 +59,7 @@ struct Smem {
   T red[D][TB];   // per-slot reductions (scaled errors, norms)
   T hs[TB];       // per-slot step of the current attempt
   int flag[TB];   // per-slot accept / state flags
+  int sv[TB];     // per-slot save point reached by the accepted step, or -1
   int any;
 };
 
@@ -231,6 +232,7 @@ struct RecArgs64 {
   int32_t* nsteps;
   int32_t* status;
   int32_t* nreject;
+  T* u_save;  // adaptive forward-only solve: [nsave][64][n] by trajectory, else null
 };
 
 template <typename T>
@@ -377,7 +379,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
     __syncthreads();
     // --- per-slot: accept / reject, controller
     if (ctl) {
-      int accept = 0;
+      int accept = 0, hit = -1;
       if (!done) {
         const T err = slot_rms(s, t);
         const T hcur = s.hs[t];
@@ -390,8 +392,9 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
             if (a.store) a.h[it * a.smax + nst] = hcur;  // trajectory-major workspace copy
             ++nst;
             tcur = clipped ? tstop : tn;
-            while (kk < a.nsave && tcur == a.tsave[kk]) {
+            while (kk < a.nsave && tcur == a.tsave[kk]) {  // save times increase: one hit at most
               if (a.store) a.save_idx[(int64_t)kk * n + it] = nst;
+              hit = kk;
               ++kk;
             }
             T fac, lnerr = ln_floor;
@@ -423,6 +426,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
         }
       }
       s.flag[t] = accept;
+      s.sv[t] = hit;
     }
     __syncthreads();
     // --- every thread: take the accepted steps
@@ -434,13 +438,24 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
           u.v[q][c] = un.v[q][c];
           k1.v[q][c] = k7.v[q][c];
         }
+        const int k = s.sv[2 * tx + c];
+        if (a.u_save && k >= 0) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) a.u_save[((int64_t)k * D + 4 * ty + q) * n + base + 2 * tx + c] = u.v[q][c];
+        }
       }
     }
+  }
+  if (live && a.u_save && status != GS_TRAJ_OK) {
+    // a failed trajectory has no solution: NaN at every save point
+    const T nan = cst<T>(__int_as_float(0x7fc00000));
+    for (int k = 0; k < a.nsave; ++k)
+      for (int r = 0; r < D; ++r) a.u_save[((int64_t)k * D + r) * n + it] = nan;
   }
   if (live) {
     if (a.store)
       for (int k = kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + it] = 0;
-    a.nsteps[it] = nst;
+    if (a.nsteps) a.nsteps[it] = nst;
     if (a.status) a.status[it] = status;
     if (a.nreject) a.nreject[it] = nrej;
   }
@@ -869,10 +884,12 @@ gs_status node64_solve(const gs_problem* P, const gs_mesh* M, void* u_save, cuda
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
 
-// Adaptive record (store = true: into h / save_idx, trajectory order) or the
-// sizing pass (store = false).
+// Adaptive record (store = true: into h / save_idx, trajectory order), the
+// sizing pass (store = false), or with u_save set the adaptive forward-only
+// solve (the state at each save time).
 gs_status node64_record_pass(const gs_problem* P, const gs_tol* tol, int32_t smax, bool store, float* h,
-                             int32_t* save_idx, int32_t* nsteps, int32_t* status, int32_t* nreject, cudaStream_t st) {
+                             int32_t* save_idx, int32_t* nsteps, int32_t* status, int32_t* nreject, cudaStream_t st,
+                             float* u_save) {
   using T = float;
   n64::RecArgs64<T> a{};
   a.n = P->n;
@@ -893,6 +910,7 @@ gs_status node64_record_pass(const gs_problem* P, const gs_tol* tol, int32_t sma
   a.nsteps = nsteps;
   a.status = status;
   a.nreject = nreject;
+  a.u_save = u_save;
   const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
   const size_t smem = sizeof(n64::Smem<T>);
   if (cudaFuncSetAttribute(n64::k_record_node64<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

@@ -14,7 +14,8 @@
 //   multiplied by fac either way.  A step whose end would reach the next stop
 //   (save time or t1, within 4 eps) is shortened to land on it exactly.
 //   Starting step: Hairer, Norsett & Wanner I, II.4.
-// One thread per trajectory; every loop is bounded by the step capacity.
+// Lanes take trajectories in turn from their warp's share (k_record3); every
+// loop is bounded by the step capacity.
 //
 // Order of a record: gs_record runs the adaptive solve once, in trajectory
 // order, into workspace copies of the mesh arrays (h trajectory-major, so each
@@ -37,14 +38,19 @@ struct RecArgs {
   int32_t nsave;
   int32_t smax;
   T tsave[GS_MAX_SAVE];
-  const int32_t* order;  // slot -> trajectory (null: identity)
-  T* h;                  // step sizes (null: count only); step s of slot j at
-  int64_t hcol, hstep;   // h[j * hcol + s * hstep]
-  int32_t* save_idx;     // [nsave][n] by slot
-  int32_t* nsteps;       // [n]
-  int32_t* status;       // [n] (may be null in count mode)
+  int64_t chunk;         // trajectories per warp (set by the launcher)
+  T* h;                  // mesh mode: step s of trajectory i at h[i * hcol + s * hstep]
+  int64_t hcol, hstep;
+  int32_t* save_idx;     // mesh mode: [nsave][n] by trajectory
+  int32_t* nsteps;       // [n] (may be null in solve mode)
+  int32_t* status;       // [n] (may be null in count and solve modes)
   int32_t* nreject;      // [n] (may be null)
+  T* u_save;             // solve mode: [nsave][3][n] by trajectory
 };
+
+// What a recorder pass writes besides the counts: nothing (the sizing pass),
+// the mesh, or the state at each save time (the adaptive forward-only solve).
+enum RecMode { kRecCount = 0, kRecMesh = 1, kRecSolve = 2 };
 
 template <typename T, int SYS, int METHOD>
 __device__ T initial_step3(const T u0[3], const T p[3], T t0, T t1, T rtol, T atol) {
@@ -68,109 +74,189 @@ __device__ T initial_step3(const T u0[3], const T p[3], T t0, T t1, T rtol, T at
   return smin_(smin_(cst<T>(100.0) * h0, h1), t1 - t0);
 }
 
-template <typename T, int SYS, int METHOD, bool STORE>
-__global__ void __launch_bounds__(128) k_record3(RecArgs<T> a) {
-  const int64_t n = a.n;
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= n) return;
-  const int64_t i = a.order ? (int64_t)a.order[j] : j;
-  const T eps = Eps<T>::v;
-  const T q = METHOD == GS_TSIT5 ? cst<T>(5.0) : cst<T>(2.0);
+// One recorder trajectory held by a lane.
+template <typename T>
+struct Traj {
+  int64_t i;  // trajectory index
   T u[3], p[3], k1[3];
+  T t, hprop, lnprev;
+  int nst, nrej, status, kk;
+  bool prev_rej;
+};
+
+// Load trajectory i and choose its first step; false if it cannot start.
+template <typename T, int SYS, int METHOD>
+__device__ __forceinline__ bool traj_start(const RecArgs<T>& a, int64_t i, Traj<T>& r) {
+  const int64_t n = a.n;
+  r.i = i;
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
-    u[c] = a.u0[c * n + i];
-    p[c] = a.p[c * n + i];
+    r.u[c] = a.u0[c * n + i];
+    r.p[c] = a.p[c * n + i];
   }
-  int nst = 0, nrej = 0, status = GS_TRAJ_OK;
-  rhs3<T, SYS>(u, p, k1);
+  r.nst = 0;
+  r.nrej = 0;
+  r.kk = 0;
+  r.status = GS_TRAJ_OK;
+  r.prev_rej = false;
+  r.t = a.t0;
+  r.lnprev = cst<T>(0.0);  // the controller carries ln(errprev); errprev starts at 1
+  rhs3<T, SYS>(r.u, r.p, r.k1);
   bool finite = true;
 #pragma unroll
-  for (int c = 0; c < 3; ++c) finite = finite && isfinite(k1[c]) && isfinite(u[c]);
-  T hprop = cst<T>(0.0);
+  for (int c = 0; c < 3; ++c) finite = finite && isfinite(r.k1[c]) && isfinite(r.u[c]);
+  r.hprop = cst<T>(0.0);
   if (finite) {
-    hprop = a.h0 > cst<T>(0.0) ? a.h0 : initial_step3<T, SYS, METHOD>(u, p, a.t0, a.t1, a.rtol, a.atol);
-    if (!(hprop > cst<T>(0.0)) || !isfinite(hprop)) finite = false;
+    r.hprop = a.h0 > cst<T>(0.0) ? a.h0 : initial_step3<T, SYS, METHOD>(r.u, r.p, a.t0, a.t1, a.rtol, a.atol);
+    if (!(r.hprop > cst<T>(0.0)) || !isfinite(r.hprop)) finite = false;
   }
-  if (!finite) status = GS_TRAJ_NONFINITE;
-  // the controller carries ln(errprev); errprev starts at 1 and is floored at 1e-4
-  T t = a.t0, lnprev = cst<T>(0.0);
-  const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
-  bool prev_rej = false;
-  int kk = 0;
-  T* hout = STORE ? a.h + j * a.hcol : nullptr;
-  while (status == GS_TRAJ_OK) {
-    const T tstop = kk < a.nsave ? a.tsave[kk] : a.t1;
-    if (hprop < cst<T>(16.0) * eps * fabs(t)) {
-      status = GS_TRAJ_DTMIN;
-      break;
-    }
-    const T tn = t + hprop;
-    const bool clipped = tn >= tstop - cst<T>(4.0) * eps * fabs(tstop);
-    const T h = clipped ? tstop - t : hprop;
-    T un[3], k7[3], e[3];
-    if (METHOD == GS_TSIT5) {
-      tsit5_err_step<T, SYS>(u, p, h, k1, un, k7, e);
-    } else {
-      if (!ros2_err_step<T, SYS>(u, p, h, un, e)) {
-        status = GS_TRAJ_SINGULAR;
-        break;
-      }
-    }
-    T sc[3];
-#pragma unroll
-    for (int c = 0; c < 3; ++c) sc[c] = fmaT(a.rtol, smax_(fabs(u[c]), fabs(un[c])), a.atol);
-    const T err = rms3(e, sc);
-    if (err <= cst<T>(1.0)) {
-      if (nst >= a.smax) {
-        status = GS_TRAJ_MAXSTEPS;
-        break;
-      }
-      if (STORE) hout[(int64_t)nst * a.hstep] = h;
-      ++nst;
-      t = clipped ? tstop : tn;
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        u[c] = un[c];
-        if (METHOD == GS_TSIT5) k1[c] = k7[c];
-      }
-      while (kk < a.nsave && t == a.tsave[kk]) {
-        if (STORE) a.save_idx[(int64_t)kk * n + j] = nst;
-        ++kk;
-      }
-      // fac = 0.9 err^(-0.7/q) errprev^(0.4/q), as 0.9 exp(-(0.7/q) ln err + (0.4/q) ln errprev)
-      T fac, lnerr = ln_floor;
-      if (err == cst<T>(0.0)) {
-        fac = cst<T>(10.0);
-      } else {
-        lnerr = ctrl_ln<T>(err);
-        fac = cst<T>(0.9) * ctrl_exp<T>(fmaT(-(cst<T>(0.7) / q), lnerr, (cst<T>(0.4) / q) * lnprev));
-        fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
-      }
-      if (prev_rej) fac = smin_(fac, cst<T>(1.0));
-      lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
-      prev_rej = false;
-      hprop = fac * hprop;
-      if (t >= a.t1) break;
-    } else {
-      ++nrej;
-      if (nrej > a.smax) {
-        status = GS_TRAJ_MAXSTEPS;
-        break;
-      }
-      const T fac = !isfinite(err) ? cst<T>(0.2)
-                                   : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_exp<T>(-(cst<T>(1.0) / q) * ctrl_ln<T>(err)));
-      hprop = fac * hprop;
-      prev_rej = true;
+  if (!finite) r.status = GS_TRAJ_NONFINITE;
+  return finite;
+}
+
+// One attempted step of a running trajectory; true when it has ended (reached
+// t1 or failed).
+template <typename T, int SYS, int METHOD, int MODE>
+__device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T ln_floor) {
+  const int64_t n = a.n;
+  const T eps = Eps<T>::v;
+  const T q = METHOD == GS_TSIT5 ? cst<T>(5.0) : cst<T>(2.0);
+  const T tstop = r.kk < a.nsave ? a.tsave[r.kk] : a.t1;
+  if (r.hprop < cst<T>(16.0) * eps * fabs(r.t)) {
+    r.status = GS_TRAJ_DTMIN;
+    return true;
+  }
+  const T tn = r.t + r.hprop;
+  const bool clipped = tn >= tstop - cst<T>(4.0) * eps * fabs(tstop);
+  const T h = clipped ? tstop - r.t : r.hprop;
+  T un[3], k7[3], e[3];
+  if (METHOD == GS_TSIT5) {
+    tsit5_err_step<T, SYS>(r.u, r.p, h, r.k1, un, k7, e);
+  } else {
+    if (!ros2_err_step<T, SYS>(r.u, r.p, h, un, e)) {
+      r.status = GS_TRAJ_SINGULAR;
+      return true;
     }
   }
-  if (STORE) {
+  T sc[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) sc[c] = fmaT(a.rtol, smax_(fabs(r.u[c]), fabs(un[c])), a.atol);
+  const T err = rms3(e, sc);
+  const bool accept = err <= cst<T>(1.0);
+  // The controller's power function, once for either outcome (each outcome's
+  // own formula, so a lane's arithmetic is that of a branch per outcome, but a
+  // warp whose lanes disagree evaluates ln and exp once, not twice):
+  //   accept: 0.9 exp(-(0.7/q) ln err + (0.4/q) ln errprev)
+  //   reject: 0.9 exp(-(1/q) ln err)
+  const bool finite_pos = err > cst<T>(0.0) && isfinite(err);
+  const T lnerr = ctrl_ln<T>(finite_pos ? err : cst<T>(1.0));
+  const T w = accept ? fmaT(-(cst<T>(0.7) / q), lnerr, (cst<T>(0.4) / q) * r.lnprev) : -(cst<T>(1.0) / q) * lnerr;
+  const T pw = cst<T>(0.9) * ctrl_exp<T>(w);
+  if (accept) {
+    if (r.nst >= a.smax) {
+      r.status = GS_TRAJ_MAXSTEPS;
+      return true;
+    }
+    if (MODE == kRecMesh) a.h[r.i * a.hcol + (int64_t)r.nst * a.hstep] = h;
+    ++r.nst;
+    r.t = clipped ? tstop : tn;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      r.u[c] = un[c];
+      if (METHOD == GS_TSIT5) r.k1[c] = k7[c];
+    }
+    while (r.kk < a.nsave && r.t == a.tsave[r.kk]) {
+      if (MODE == kRecMesh) a.save_idx[(int64_t)r.kk * n + r.i] = r.nst;
+      if (MODE == kRecSolve) {
+#pragma unroll
+        for (int c = 0; c < 3; ++c) a.u_save[((int64_t)r.kk * 3 + c) * n + r.i] = r.u[c];
+      }
+      ++r.kk;
+    }
+    // fac in [0.2, 10], 10 if err == 0, at most 1 right after a rejection
+    T fac = err == cst<T>(0.0) ? cst<T>(10.0) : smin_(cst<T>(10.0), smax_(cst<T>(0.2), pw));
+    if (r.prev_rej) fac = smin_(fac, cst<T>(1.0));
+    r.lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
+    r.prev_rej = false;
+    r.hprop = fac * r.hprop;
+    return r.t >= a.t1;
+  }
+  ++r.nrej;
+  if (r.nrej > a.smax) {
+    r.status = GS_TRAJ_MAXSTEPS;
+    return true;
+  }
+  // fac >= 0.2, 0.2 for NaN or inf
+  const T fac = finite_pos ? smax_(cst<T>(0.2), pw) : cst<T>(0.2);
+  r.hprop = fac * r.hprop;
+  r.prev_rej = true;
+  return false;
+}
+
+// Outputs of an ended trajectory.
+template <typename T, int MODE>
+__device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T>& r) {
+  const int64_t n = a.n;
+  if (MODE == kRecMesh) {
     // unreached save points (a failed trajectory); the h tail stays unwritten
-    for (int k = kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + j] = 0;
+    for (int k = r.kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + r.i] = 0;
   }
-  a.nsteps[j] = nst;
-  if (a.status) a.status[j] = status;
-  if (a.nreject) a.nreject[j] = nrej;
+  if (MODE == kRecSolve && r.status != GS_TRAJ_OK) {
+    // a failed trajectory has no solution: NaN at every save point
+    const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
+    for (int k = 0; k < a.nsave; ++k)
+#pragma unroll
+      for (int c = 0; c < 3; ++c) a.u_save[((int64_t)k * 3 + c) * n + r.i] = nan;
+  }
+  if (a.nsteps) a.nsteps[r.i] = r.nst;
+  if (a.status) a.status[r.i] = r.status;
+  if (a.nreject) a.nreject[r.i] = r.nrej;
+}
+
+// 6 resident blocks of 128 per SM (85 registers a thread): measured faster on
+// B200 than the unconstrained 90-92 registers at 5 blocks, and than 7 or 8
+// blocks (more spilling).
+#ifndef GS_REC_MINB
+#define GS_REC_MINB 6
+#endif
+
+// Each warp owns the trajectories [w * chunk, (w + 1) * chunk) and its lanes
+// take them in turn: a lane whose trajectory has ended takes the next one of
+// the chunk (handed out with a ballot), so lanes do not idle while the
+// longest trajectory of the warp finishes.  The launch gives one resident
+// wave of warps, each with an equal share.  A trajectory's arithmetic does
+// not depend on which lane runs it or when.  The loop ends: every pass either
+// hands out chunk entries or advances some trajectory's accepted or rejected
+// step count, and both are capped by smax.
+template <typename T, int SYS, int METHOD, int MODE>
+__global__ void __launch_bounds__(128, GS_REC_MINB) k_record3(RecArgs<T> a) {
+  const unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t c0 = w * a.chunk;
+  const int64_t c1 = c0 + a.chunk < a.n ? c0 + a.chunk : a.n;
+  if (c0 >= c1) return;  // whole warp
+  int64_t next = c0;
+  const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));  // errprev is floored at 1e-4
+  Traj<T> r;
+  bool run = false;
+  for (;;) {
+    const unsigned need = __ballot_sync(kFull, !run);
+    if (need) {
+      const int64_t cand = next + __popc(need & lt);
+      if (!run && cand < c1) {
+        run = traj_start<T, SYS, METHOD>(a, cand, r);
+        if (!run) traj_finish<T, MODE>(a, r);
+      }
+      next += __popc(need);
+    }
+    if (!__any_sync(kFull, run) && next >= c1) break;
+    if (run && traj_attempt<T, SYS, METHOD, MODE>(a, r, ln_floor)) {
+      traj_finish<T, MODE>(a, r);
+      run = false;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -259,21 +345,35 @@ static RecArgs<T> rec_args(const gs_problem* P, const gs_tol* tol, int32_t smax)
   return a;
 }
 
-template <typename T, int SYS, int METHOD, bool STORE>
-static gs_status launch_rec(const RecArgs<T>& a, cudaStream_t st) {
+#ifndef GS_REC_WAVES
+#define GS_REC_WAVES 1
+#endif
+
+template <typename T, int SYS, int METHOD, int MODE>
+static gs_status launch_rec(RecArgs<T> a, cudaStream_t st) {
+  // one resident wave of warps, each with an equal share of the trajectories
   const int bs = 128;
-  const int64_t grid = (a.n + bs - 1) / bs;
-  k_record3<T, SYS, METHOD, STORE><<<(unsigned)grid, bs, 0, st>>>(a);
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_record3<T, SYS, METHOD, MODE>, bs, 0) != cudaSuccess)
+    return GS_ECUDA;
+  const int64_t warps = (int64_t)(per_sm > 0 ? per_sm : 1) * sms * (bs / 32) * GS_REC_WAVES;
+  a.chunk = (a.n + warps - 1) / warps;
+  if (a.chunk < 32) a.chunk = 32;
+  const int64_t nwarps = (a.n + a.chunk - 1) / a.chunk;
+  const int64_t grid = (nwarps * 32 + bs - 1) / bs;
+  k_record3<T, SYS, METHOD, MODE><<<(unsigned)grid, bs, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
 
-template <typename T, bool STORE>
+template <typename T, int MODE>
 static gs_status dispatch_rec(int sys, int method, const RecArgs<T>& a, cudaStream_t st) {
-  if (sys == GS_LORENZ && method == GS_TSIT5) return launch_rec<T, kSysLorenz, GS_TSIT5, STORE>(a, st);
-  if (sys == GS_LORENZ && method == GS_ROS2) return launch_rec<T, kSysLorenz, GS_ROS2, STORE>(a, st);
-  if (sys == GS_ROBERTSON && method == GS_TSIT5) return launch_rec<T, kSysRobertson, GS_TSIT5, STORE>(a, st);
-  if (sys == GS_ROBERTSON && method == GS_ROS2) return launch_rec<T, kSysRobertson, GS_ROS2, STORE>(a, st);
+  if (sys == GS_LORENZ && method == GS_TSIT5) return launch_rec<T, kSysLorenz, GS_TSIT5, MODE>(a, st);
+  if (sys == GS_LORENZ && method == GS_ROS2) return launch_rec<T, kSysLorenz, GS_ROS2, MODE>(a, st);
+  if (sys == GS_ROBERTSON && method == GS_TSIT5) return launch_rec<T, kSysRobertson, GS_TSIT5, MODE>(a, st);
+  if (sys == GS_ROBERTSON && method == GS_ROS2) return launch_rec<T, kSysRobertson, GS_ROS2, MODE>(a, st);
   return GS_EUNSUPPORTED;
 }
 
@@ -283,12 +383,30 @@ gs_status count3(const gs_problem* P, const gs_tol* tol, int32_t smax, int32_t* 
     RecArgs<double> a = rec_args<double>(P, tol, smax);
     a.nsteps = nsteps;
     a.status = status;
-    return dispatch_rec<double, false>(P->system, P->method, a, st);
+    return dispatch_rec<double, kRecCount>(P->system, P->method, a, st);
   }
   RecArgs<float> a = rec_args<float>(P, tol, smax);
   a.nsteps = nsteps;
   a.status = status;
-  return dispatch_rec<float, false>(P->system, P->method, a, st);
+  return dispatch_rec<float, kRecCount>(P->system, P->method, a, st);
+}
+
+// Adaptive forward-only solve: one recorder pass in trajectory order writing
+// the state at every save time (no mesh, no workspace).
+gs_status solve_adaptive3(const gs_problem* P, const gs_tol* tol, int32_t smax, void* u_save, int32_t* nsteps,
+                          int32_t* status, cudaStream_t st) {
+  if (P->dtype == GS_F64) {
+    RecArgs<double> a = rec_args<double>(P, tol, smax);
+    a.nsteps = nsteps;
+    a.status = status;
+    a.u_save = (double*)u_save;
+    return dispatch_rec<double, kRecSolve>(P->system, P->method, a, st);
+  }
+  RecArgs<float> a = rec_args<float>(P, tol, smax);
+  a.nsteps = nsteps;
+  a.status = status;
+  a.u_save = (float*)u_save;
+  return dispatch_rec<float, kRecSolve>(P->system, P->method, a, st);
 }
 
 static size_t al256(size_t b) { return (b + 255) / 256 * 256; }
@@ -346,7 +464,6 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
   w += al256((size_t)M->smax * n * sizeof(T));
   int32_t* hist = (int32_t*)w;
   RecArgs<T> a = rec_args<T>(P, tol, M->smax);
-  a.order = nullptr;  // trajectory order
   a.h = h_tmp;
   a.hcol = M->smax;  // trajectory-major workspace copy: each thread writes its own row
   a.hstep = 1;
@@ -354,7 +471,7 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
   a.nsteps = ns_tmp;
   a.status = st_tmp;
   a.nreject = nr_tmp;
-  gs_status rc = dispatch_rec<T, true>(P->system, P->method, a, st);
+  gs_status rc = dispatch_rec<T, kRecMesh>(P->system, P->method, a, st);
   if (rc != GS_OK) return rc;
   rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
   if (rc != GS_OK) return rc;
@@ -370,7 +487,7 @@ gs_status record3(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void
 }
 
 gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,
-                             int32_t*, cudaStream_t);
+                             int32_t*, cudaStream_t, float*);
 
 // The d = 64 record: the same trajectory-order pass / sort / gather sequence,
 // with the CTA-per-32-trajectories recorder of node64.cu.
@@ -389,7 +506,7 @@ gs_status record_node64(const gs_problem* P, const gs_tol* tol, const gs_mesh* M
   T* h_tmp = (T*)w;
   w += al256((size_t)M->smax * n * sizeof(T));
   int32_t* hist = (int32_t*)w;
-  gs_status rc = node64_record_pass(P, tol, M->smax, true, h_tmp, si_tmp, ns_tmp, st_tmp, nr_tmp, st);
+  gs_status rc = node64_record_pass(P, tol, M->smax, true, h_tmp, si_tmp, ns_tmp, st_tmp, nr_tmp, st, nullptr);
   if (rc != GS_OK) return rc;
   rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
   if (rc != GS_OK) return rc;

@@ -70,6 +70,9 @@ _lib.gs_count.restype = ctypes.c_int32
 _lib.gs_record.argtypes = [_P(_Problem), _P(_Tol), _P(_Mesh), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.gs_record.restype = ctypes.c_int32
 _lib.gs_solve.argtypes = [_P(_Problem), _P(_Mesh), ctypes.c_void_p, ctypes.c_void_p]
+_lib.gs_solve_adaptive.argtypes = [_P(_Problem), _P(_Tol), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p]
+_lib.gs_solve_adaptive.restype = ctypes.c_int32
 _lib.gs_solve.restype = ctypes.c_int32
 _lib.gs_grad.argtypes = [_P(_Problem), _P(_Mesh), _P(_Loss), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
@@ -210,6 +213,23 @@ def gs_count(ens: Ensemble, rtol: float, atol: float, smax: int, h0: float = 0.0
     _check(_lib.gs_count(ctypes.byref(ps), ctypes.byref(tol), smax, _ptr(nsteps), _ptr(status), _stream(stream)),
            "gs_count")
     return nsteps, status
+
+
+def gs_solve_adaptive(ens: Ensemble, rtol: float, atol: float, smax: int, h0: float = 0.0, u_save=None,
+                      nsteps=None, status=None, stream=None):
+    """Adaptive forward-only solve: (u_save [nsave][d][n], nsteps [n], status [n]),
+    all by trajectory; no mesh is kept."""
+    dev = ens.u0.device
+    if u_save is None:
+        u_save = torch.empty((len(ens.tsave), ens.d, ens.n), dtype=TORCH_DTYPE[ens.dtype], device=dev)
+    if nsteps is None:
+        nsteps = torch.empty(ens.n, dtype=torch.int32, device=dev)
+    if status is None:
+        status = torch.empty(ens.n, dtype=torch.int32, device=dev)
+    ps, tol = ens._struct(), _Tol(rtol, atol, h0)
+    _check(_lib.gs_solve_adaptive(ctypes.byref(ps), ctypes.byref(tol), smax, _ptr(u_save), _ptr(nsteps),
+                                  _ptr(status), _stream(stream)), "gs_solve_adaptive")
+    return u_save, nsteps, status
 
 
 def gs_record(ens: Ensemble, mesh: Mesh, rtol: float, atol: float, h0: float = 0.0, ws=None, stream=None):

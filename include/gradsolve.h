@@ -186,6 +186,24 @@ GS_API gs_status gs_record(const gs_problem* prob, const gs_tol* tol, const gs_m
 GS_API gs_status gs_solve(const gs_problem* prob, const gs_mesh* mesh, void* u_save, void* stream);
 
 /*
+ * Adaptive forward-only solve: the recorder's adaptive iteration (same
+ * controller, same stops at the save times) with no mesh stored, returning
+ * the accepted state at each save time.
+ *   smax     cap on accepted steps and on rejections (GS_TRAJ_MAXSTEPS beyond)
+ *   u_save   device [nsave][d][n] dtype, by trajectory; NaN at every save point
+ *            of a trajectory whose status is not GS_TRAJ_OK
+ *   nsteps   device [n] int32 accepted steps, by trajectory; may be NULL
+ *   status   device [n] int32, by trajectory; may be NULL
+ * Needs no workspace.  The states equal, bit for bit, those that gs_record
+ * followed by gs_solve returns for the same problem and tolerances: the
+ * recorder and the replay take each step with the same operations.
+ * (GRADSOLVE abstract: the forward-only kernel, the library's second headline
+ * use besides gradients.)
+ */
+GS_API gs_status gs_solve_adaptive(const gs_problem* prob, const gs_tol* tol, int32_t smax, void* u_save,
+                                   int32_t* nsteps, int32_t* status, void* stream);
+
+/*
  * Fused replay + reverse sweep: for every trajectory, the loss of the
  * fixed-step replay on the mesh and its exact discrete adjoint.
  *   loss     device [n] dtype       L_i

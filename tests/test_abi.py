@@ -18,8 +18,8 @@ def _declared():
 
 def test_header_declares_entry_points():
     names = set(_declared())
-    assert {"gs_workspace_bytes", "gs_count", "gs_record", "gs_solve", "gs_grad", "gs_status_string",
-            "gs_launch_count"} <= names
+    assert {"gs_workspace_bytes", "gs_count", "gs_record", "gs_solve", "gs_solve_adaptive", "gs_grad",
+            "gs_status_string", "gs_launch_count"} <= names
 
 
 def test_library_exports_every_declared_symbol():
@@ -79,6 +79,8 @@ def test_invalid_problems_rejected_before_launch(bad):
     tol = _Tol(1e-6, 1e-6, 0.0)
     rc = _lib.gs_count(ctypes.byref(p), ctypes.byref(tol), 100, ctypes.c_void_p(16), None, None)
     assert rc == (-4 if bad == "hires" else -1)
+    rc = _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(tol), 100, ctypes.c_void_p(16), None, None, None)
+    assert rc == (-4 if bad == "hires" else -1)
     m = _Mesh(100, p.nsave, 16, 16, 16, 16, 16, 16)
     assert _lib.gs_record(ctypes.byref(p), ctypes.byref(tol), ctypes.byref(m), ctypes.c_void_p(16), 1 << 40,
                           None) == (-4 if bad == "hires" else -1)
@@ -101,6 +103,13 @@ def test_bad_tolerance_and_workspace_rejected():
     # linear loss without weights
     assert _lib.gs_grad(ctypes.byref(p), ctypes.byref(m), ctypes.byref(_Loss(2, None, None)), ctypes.c_void_p(16),
                         ctypes.c_void_p(16), ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 40, None) == -1
+    # the adaptive solve needs its output, a capacity and a valid tolerance
+    tol = _Tol(1e-6, 1e-6, 0.0)
+    assert _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(tol), 100, None, None, None, None) == -1
+    assert _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(tol), 0, ctypes.c_void_p(16), None, None,
+                                  None) == -1
+    assert _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(_Tol(0.0, 0.0, 0.0)), 100, ctypes.c_void_p(16),
+                                  None, None, None) == -1
     # mesh nsave must match
     m2 = _Mesh(100, 3, 16, 16, 16, 16, 16, 16)
     assert _lib.gs_solve(ctypes.byref(p), ctypes.byref(m2), ctypes.c_void_p(16), None) == -1
@@ -117,4 +126,6 @@ def test_empty_ensemble_is_a_no_op():
     assert _lib.gs_grad(ctypes.byref(p), ctypes.byref(m), ctypes.byref(_Loss(1, None, None)), None, None, None,
                         None, None, 0, None) == 0
     assert _lib.gs_solve(ctypes.byref(p), ctypes.byref(m), None, None) == 0
+    assert _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, None, None, None,
+                                  None) == 0
     assert _lib.gs_launch_count() == before

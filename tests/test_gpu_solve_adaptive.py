@@ -1,0 +1,117 @@
+"""GPU <-> oracle parity for the adaptive forward-only solve (gs_solve_adaptive):
+step counts and statuses equal to the oracle's, saved states within the mesh
+bar (1e-10 relative, fp64) or the fp32 bar (1e-4), bitwise equality with the
+GPU's own record followed by its replay, failures and ragged sizes, and the
+full 2**20-trajectory ensemble checked on a sample."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+import discrete_adjoint_b200 as gs
+from gpu_util import dev, ensemble, mesh_by_trajectory
+
+pytestmark = pytest.mark.gpu
+
+
+def _solve(prob, smax):
+    us, ns, st = gs.gs_solve_adaptive(ensemble(prob), prob.rtol, prob.atol, smax)
+    torch.cuda.synchronize()
+    return us.double().cpu().numpy(), ns.cpu().numpy(), st.cpu().numpy()
+
+
+def _rel(a, b):
+    """Largest error over the largest magnitude, per trajectory (last axis)."""
+    return (np.abs(a - b).max(axis=(0, 1)) / np.abs(b).max(axis=(0, 1))).max()
+
+
+@pytest.mark.parametrize("name,n,smax,bar", [("lorenz_small", 1024, 256, 1e-10), ("lorenz_1m", 4000, 1024, 1e-10),
+                                             ("robertson", 700, 20000, 1e-10)])
+def test_fp64_matches_oracle(name, n, smax, bar):
+    prob = W.by_name(name, n=n)
+    ref, rns, rst = oracle.solve_adaptive(prob, smax)
+    us, ns, st = _solve(prob, smax)
+    assert (rst == 0).all() and np.array_equal(st, rst)
+    assert np.array_equal(ns, rns)
+    assert _rel(us, ref) <= bar
+
+
+def test_fp32_matches_oracle():
+    prob = W.lorenz_1m(2000, dtype="f32")
+    ref, rns, rst = oracle.solve_adaptive(prob, 1024)
+    us, ns, st = _solve(prob, 1024)
+    assert (st == 0).all() and np.array_equal(ns, rns)
+    assert _rel(us, ref) <= 1e-4
+
+
+@pytest.mark.parametrize("name,dtype,n,smax", [("lorenz_1m", "f64", 3000, 1024), ("lorenz_1m", "f32", 3000, 1024),
+                                               ("robertson", "f64", 300, 20000), ("node64", "f32", 300, 64)])
+def test_equals_record_then_replay(name, dtype, n, smax):
+    """One adaptive iteration, two outputs: the states of the forward-only solve
+    are bit for bit those of gs_record followed by gs_solve."""
+    prob = W.by_name(name, n=n).as_dtype(dtype)
+    ens = ensemble(prob)
+    us, ns, st = gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, smax)
+    mesh = gs.new_mesh(prob.n, smax, len(prob.tsave), prob.dtype, dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    ur = gs.gs_solve(ens, mesh)
+    torch.cuda.synchronize()
+    h, mns, si, mst, order = mesh_by_trajectory(mesh)
+    assert np.array_equal(ns.cpu().numpy(), mns) and np.array_equal(st.cpu().numpy(), mst)
+    assert torch.equal(us, ur)
+
+
+def test_node64_matches_oracle():
+    prob = W.node64(256)
+    us, ns, st = _solve(prob, 64)
+    assert (st == 0).all()
+    # the oracle's replay of the mesh the GPU chose (the fp32 replay bar)
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(prob.n, 64, 1, "f32", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    h, mns, si, mst, order = mesh_by_trajectory(mesh)
+    _, ur = oracle.replay(prob, oracle.Mesh(h.astype(np.float64), mns, si, mst, np.zeros(prob.n, np.int32)))
+    assert np.abs(us - ur).max() <= 1e-5 * np.abs(ur).max()
+    # and the oracle's own adaptive solve: both meet the tolerance (fp32 step
+    # decisions differ near err = 1, so the meshes are not identical)
+    ref, rns, rst = oracle.solve_adaptive(prob, 64)
+    assert (rst == 0).all()
+    assert np.abs(us - ref).max() <= 1e-3 * np.abs(ref).max()
+
+
+def test_failures_and_ragged_sizes():
+    prob = W.lorenz_small(129)
+    us, ns, st = _solve(prob, 20)  # capacity -> MAXSTEPS everywhere
+    assert (st == 1).all() and np.isnan(us).all()
+    bad = W.lorenz_small(129)
+    bad.p = bad.p.copy()
+    bad.p[0, 5] = np.nan
+    us, ns, st = _solve(bad, 256)
+    ref, rns, rst = oracle.solve_adaptive(bad, 256)
+    assert np.array_equal(st, rst) and st[5] == 3 and (np.delete(st, 5) == 0).all()
+    assert np.isnan(us[:, :, 5]).all()
+    ok = np.delete(np.arange(bad.n), 5)
+    assert _rel(us[:, :, ok], ref[:, :, ok]) <= 1e-10
+    one = W.lorenz_small(1)
+    us, ns, st = _solve(one, 256)
+    ref, rns, _ = oracle.solve_adaptive(one, 256)
+    assert ns[0] == rns[0] and _rel(us, ref) <= 1e-10
+
+
+def test_full_size_sampled():
+    """2**20 trajectories, fp64, t in [0, 10], ten save points: the oracle checks
+    a sample (random + the longest chains) one by one."""
+    prob = W.lorenz_1m()
+    us, ns, st = gs.gs_solve_adaptive(ensemble(prob), prob.rtol, prob.atol, 2048)
+    torch.cuda.synchronize()
+    assert (st == 0).all()
+    ns_all = ns.cpu().numpy()
+    rng = np.random.default_rng(12)
+    idx = np.unique(np.concatenate([rng.choice(prob.n, 384, replace=False), np.argsort(ns_all)[-32:]]))
+    ref, rns, rst = oracle.solve_adaptive(prob.subset(idx), 2048)
+    assert np.array_equal(ns_all[idx], rns)
+    got = us[:, :, torch.tensor(idx, device=dev())].cpu().numpy()
+    assert _rel(got, ref) <= 1e-10
+    assert torch.isfinite(us).all()
