@@ -67,6 +67,7 @@ def lib():
                                 dp, dp, i32]
         L.or_solve_adaptive.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, f64, f64, i32, dp, f64, f64,
                                         f64, i32, dp, ip, ip, i32]
+        L.or_sens.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, i32, i32, dp, ip, ip, ip, dp, i32]
         L.or_count_step.argtypes = [i32, i32, i32, i32, dp]
         L.or_step.argtypes = [i32, i32, i32, i32, dp, dp, dp, f64, dp, dp]
         L.or_rhs.argtypes = [i32, i32, dp, dp, dp, dp, dp]
@@ -194,6 +195,21 @@ def dirderiv(prob, mesh: Mesh, dir_p=None, dir_u0=None, dir_W=None, nthreads: in
                        _i(ns), _i(si), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)),
                        _d(_f64(dir_p)), _d(_f64(dir_u0)), _d(_f64(dir_W)), _d(out), nthreads or default_threads())
     _check(rc, "dirderiv")
+    return out
+
+
+def sens(prob, mesh: Mesh, nthreads: int | None = None):
+    """Forward sensitivities of the fixed-step replay by dual numbers:
+    [nsave][d][np + d][n], column j = d u(t_k) / d (p, u0)_j; NaN rows for
+    trajectories whose mesh status is not 0."""
+    L = lib()
+    h, ns, si = _mesh_args(mesh)
+    st = np.ascontiguousarray(mesh.status, np.int32)
+    out = np.zeros((si.shape[1], prob.d, prob.np_ + prob.d, prob.n))
+    rc = L.or_sens(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], prob.n, prob.d, prob.np_,
+                   _d(_f64(prob.p)), _d(_f64(prob.u0)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si), _i(st),
+                   _d(out), nthreads or default_threads())
+    _check(rc, "sens")
     return out
 
 

@@ -731,6 +731,26 @@ double dirderiv_one(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, co
   return double(L.d);
 }
 
+// Forward sensitivities of one trajectory: the dual-number replay once per
+// input direction (the np parameters, then the d initial-state components),
+// keeping the tangent of the state at each save point.  sens [nsave][d][np+d]
+// (column j = d u / d theta_j).
+template <class T>
+void sens_one(const Prob& P, const Mesh& Mh, int64_t i, double* sens) {
+  using D = Dv<T>;
+  const int d = P.d, np = P.np, m = np + d;
+  std::vector<D> u0(d), p(np), us(Mh.nsave * d);
+  std::vector<double> wg(Mh.nsave * d, 0.0);
+  for (int j = 0; j < m; ++j) {
+    for (int c = 0; c < d; ++c) u0[c] = D(T(P.u0[(int64_t)c * P.n + i]), T(j == np + c ? 1 : 0));
+    for (int c = 0; c < np; ++c) p[c] = D(T(P.p[(int64_t)c * P.n + i]), T(j == c ? 1 : 0));
+    replay_loss<D>(P.sys, P.method, d, u0.data(), p.data(), nullptr, Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave,
+                   Mh.save_idx + i * Mh.nsave, LOSS_LINEAR, nullptr, wg.data(), us.data());
+    for (int k = 0; k < Mh.nsave; ++k)
+      for (int c = 0; c < d; ++c) sens[((int64_t)k * d + c) * m + j] = double(us[k * d + c].d);
+  }
+}
+
 template <class T>
 double loss_one(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, double* u_save) {
   int d = P.d, np = P.np;
@@ -930,6 +950,35 @@ int or_dirderiv(int sys, int method, int dtype, int64_t n, int d, int np, const 
       for (int c = 0; c < d; ++c) dui[c] = dir_u0 ? dir_u0[(int64_t)c * n + i] : 0.0;
       out[i] = dtype == DT_F64 ? dirderiv_one<double>(P, Mh, Ls, i, dpi.data(), dui.data(), dir_W)
                                : dirderiv_one<float>(P, Mh, Ls, i, dpi.data(), dui.data(), dir_W);
+    }
+  });
+  return 0;
+}
+
+// Forward sensitivities d u(t_k) / d (p, u0) of the fixed-step replay, by
+// forward-mode dual numbers (one pass per input direction).  sens
+// [nsave][d][np+d][n]; NaN for trajectories with status != 0 (status may be
+// null).  Not for NODE64 (its W directions are not inputs of this product).
+int or_sens(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0, int smax,
+            int nsave, const double* h, const int* nsteps, const int* save_idx, const int* status, double* sens,
+            int nthreads) {
+  Prob P{sys, method, dtype, d, np, n, p, u0, nullptr};
+  int rc = check_prob(P);
+  if (rc) return rc;
+  if (sys == SYS_NODE64) return -4;
+  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  const int m = np + d;
+  parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
+    std::vector<double> si((size_t)nsave * d * m);
+    for (int64_t i = a; i < b; ++i) {
+      if (status && status[i] != TRAJ_OK) {
+        std::fill(si.begin(), si.end(), std::numeric_limits<double>::quiet_NaN());
+      } else if (dtype == DT_F64) {
+        sens_one<double>(P, Mh, i, si.data());
+      } else {
+        sens_one<float>(P, Mh, i, si.data());
+      }
+      for (size_t q = 0; q < si.size(); ++q) sens[(int64_t)q * n + i] = si[q];
     }
   });
   return 0;
