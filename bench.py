@@ -14,7 +14,9 @@ pass alone is reported in config.grad_only_value.
 
 The lorenz_1m_solve workload times the adaptive forward-only solve instead
 (gs_solve_adaptive on the same ensemble, no mesh kept; metric
-trajectory-solves/s).
+trajectory-solves/s); lorenz_1m_sens times the forward sensitivities on the
+recorded mesh (gs_sens: the sensitivity matrices at the ten save points and
+the loss gradient; metric trajectory-sensitivities/s).
 
 N > 1 runs under torchrun, one process per GPU; every rank owns its own
 ensemble of the workload's size (weak scaling, no data-path collective:
@@ -71,6 +73,15 @@ WORKLOADS = {
                             dtype="f64",
                             desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, states at 10 save points, "
                                  "one adaptive forward-only solve per step (no mesh kept)"),
+    # forward sensitivities on the recorded mesh: flops per replay step = the
+    # state (192) + 6 input directions x (tangent stage combinations 144 +
+    # six Jacobian-vector products 108); the per-thread copies of the state
+    # (one per direction) are not counted
+    "lorenz_1m_sens": dict(kind="sens", problem="lorenz_1m", flop_step=192 + 6 * 252, kernel="k_sens_tsit5_lorenz",
+                           n=1 << 20, dtype="f64",
+                           desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, 10 save points with N(0,1) targets; "
+                                "one forward-sensitivity pass per step on the recorded mesh (d u(t_k)/d(p,u0) at "
+                                "every save point + the loss gradient)"),
 }
 # profile of the headline kernel (DRAM traffic per replay step), valid while
 # the kernel's sources are unchanged
@@ -100,6 +111,8 @@ def dist_env():
 
 
 def metric_name(args) -> str:
+    if args.workload == "lorenz_1m_sens":
+        return f"trajectory-sensitivities/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, forward mode)"
     if args.workload == "lorenz_1m_solve":
         return f"trajectory-solves/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, adaptive forward-only)"
     if args.workload == "lorenz_1m":
@@ -199,6 +212,14 @@ def cpu_baseline(args, sample: int):
         dt = time.perf_counter() - t0
         return {"value": sample / dt, "unit": "trajectory-solves/s", "cores": threads, "kind": "oracle",
                 "sample": f"first {sample} of the {args.n} trajectories: oracle adaptive solve {dt:.2f} s"}
+    if WORKLOADS[args.workload].get("kind") == "sens":
+        om = oracle.record(prob, smax_cap(args.workload), nthreads=threads)
+        t0 = time.perf_counter()
+        oracle.sens(prob, om, nthreads=threads)
+        dt = time.perf_counter() - t0
+        return {"value": sample / dt, "unit": "trajectory-sensitivities/s", "cores": threads, "kind": "oracle",
+                "sample": f"first {sample} of the {args.n} trajectories on the oracle's own mesh: dual-number "
+                          f"sensitivities {dt:.2f} s"}
     passes = WORKLOADS[args.workload]["passes"]
     tr, tg, per_step = oracle_step_time(prob, threads, passes)
     return {"value": sample * passes / per_step, "unit": "trajectory-gradients/s", "cores": threads,
@@ -215,16 +236,20 @@ def run_reference(args):
     if rank != 0:
         return
     W = WORKLOADS[args.workload]
-    solve = W.get("kind") == "solve"
+    kind = W.get("kind", "grad")
+    solve = kind != "grad"
     sample = {"lorenz_1m": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
-              "lorenz_1m_solve": 4096}[args.workload]
+              "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
+    om = oracle.record(prob, smax_cap(args.workload), nthreads=threads) if kind == "sens" else None
     times = []
     for it in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        if solve:
+        if kind == "solve":
             oracle.solve_adaptive(prob, smax_cap(args.workload), nthreads=threads)
+        elif kind == "sens":
+            oracle.sens(prob, om, nthreads=threads)
         else:
             om = oracle.record(prob, smax_cap(args.workload), nthreads=threads)
             for _ in range(W["passes"]):
@@ -234,8 +259,9 @@ def run_reference(args):
             times.append(dt)
     t = float(np.mean(times))
     passes = 1 if solve else W["passes"]
-    unit = "trajectory-solves/s" if solve else "trajectory-gradients/s"
-    what = "oracle adaptive solve" if solve else f"oracle record + {W['passes']} tape gradient passes"
+    unit = {"solve": "trajectory-solves/s", "sens": "trajectory-sensitivities/s"}.get(kind, "trajectory-gradients/s")
+    what = {"solve": "oracle adaptive solve", "sens": "oracle dual-number sensitivities on its own mesh"}.get(kind)
+    what = what or f"oracle record + {W['passes']} tape gradient passes"
     value = sample * passes / t
     line = {"impl": "reference", "metric": metric_name(args), "value": value, "unit": unit,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
@@ -264,15 +290,17 @@ def kernel_traffic(total_steps: int):
         return None
 
 
-def run_solve(args):
-    """The adaptive forward-only solve: one gs_solve_adaptive call over the
-    rank's ensemble per step."""
+def run_single(args):
+    """One library call per step over the rank's ensemble: the adaptive
+    forward-only solve (gs_solve_adaptive) or the forward sensitivities on the
+    recorded mesh (gs_sens)."""
     import torch
     import torch.distributed as dist
 
     import discrete_adjoint_b200 as gs
 
     W = WORKLOADS[args.workload]
+    kind = W["kind"]
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -286,24 +314,42 @@ def run_solve(args):
     stream = torch.cuda.current_stream()
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(td).pin_memory()
     host = {"p": pin(prob.p), "u0": pin(prob.u0)}
+    if kind == "sens" and prob.target is not None:
+        host["target"] = pin(prob.target)
     d = {k: v.to(dev) for k, v in host.items()}
     ens = gs.Ensemble(prob.system, prob.method, args.dtype, d["p"], d["u0"], prob.t0, prob.t1,
                       [float(x) for x in prob.tsave])
     smax = smax_cap(args.workload)
-    u_save = torch.empty((len(prob.tsave), prob.d, n), dtype=td, device=dev)
-    nsteps = torch.empty(n, dtype=torch.int32, device=dev)
-    status = torch.empty(n, dtype=torch.int32, device=dev)
-    # attempted steps (accepted + rejected), for the flop count: one untimed record
+    # setup (untimed): a record, for the attempted-step count of the solve's
+    # flop figure or as the mesh the sensitivities run on
     nst, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax)
     mesh = gs.new_mesh(n, int(nst.max().item()), len(prob.tsave), args.dtype, dev)
     gs.gs_record(ens, mesh, prob.rtol, prob.atol, stream=stream)
-    attempts = int(mesh.nsteps.sum().item() + mesh.nreject.sum().item())
     accepted = mesh.nsteps.double()
-    del mesh
+    if kind == "solve":
+        attempts = int(mesh.nsteps.sum().item() + mesh.nreject.sum().item())
+        flops = W["flop_attempt"] * attempts
+        del mesh
+        u_save = torch.empty((len(prob.tsave), prob.d, n), dtype=td, device=dev)
+        nsteps = torch.empty(n, dtype=torch.int32, device=dev)
+        status = torch.empty(n, dtype=torch.int32, device=dev)
+        outputs = [u_save]
+        work = {"attempted_steps": attempts}
 
-    def step():
-        gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, smax, u_save=u_save, nsteps=nsteps, status=status,
-                             stream=stream)
+        def step():
+            gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, smax, u_save=u_save, nsteps=nsteps, status=status,
+                                 stream=stream)
+    else:
+        total_steps = int(mesh.nsteps.sum().item())
+        flops = W["flop_step"] * total_steps
+        out = gs.new_grad_out(ens)
+        sens = torch.empty((len(prob.tsave), prob.d, prob.np_ + prob.d, n), dtype=td, device=dev)
+        outputs = [sens, out.loss, out.dp, out.du0]
+        status = mesh.status
+        work = {"replay_steps": total_steps, "sens_gb": sens.numel() * esz / 1e9}
+
+        def step():
+            gs.gs_sens(ens, mesh, loss=prob.loss, target=d.get("target"), out=out, sens=sens, stream=stream)
 
     def barrier():
         if world > 1:
@@ -331,14 +377,15 @@ def run_solve(args):
     elapsed = float(tmax.item())
     assert (status == 0).all()
 
-    # end to end from host buffers: H2D of p and u0, the solve, D2H of the states
-    h_out = torch.empty(u_save.shape, dtype=td).pin_memory()
+    # end to end from host buffers: H2D of the inputs, the call, D2H of its results
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outputs]
 
     def e2e_step():
         for k, v in host.items():
             d[k].copy_(v, non_blocking=True)
         step()
-        h_out.copy_(u_save, non_blocking=True)
+        for hb, t in zip(h_out, outputs):
+            hb.copy_(t, non_blocking=True)
 
     e2e_step()
     barrier()
@@ -353,24 +400,24 @@ def run_solve(args):
     if world > 1:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
 
-    t_solve = elapsed / args.steps
-    flops = W["flop_attempt"] * attempts
-    achieved = flops / t_solve
+    unit = "trajectory-solves/s" if kind == "solve" else "trajectory-sensitivities/s"
+    t_call = elapsed / args.steps
+    achieved = flops / t_call
     peak = FP64_PEAK if args.dtype == "f64" else FP32_PEAK
     line = {
-        "metric": metric_name(args), "value": world * n * args.steps / elapsed, "unit": "trajectory-solves/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_solve * 1e3,
+        "metric": metric_name(args), "value": world * n * args.steps / elapsed, "unit": unit,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_call * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {W['desc']}; n={n} per GPU", "n_per_gpu": n,
-                   "attempted_steps": attempts, "steps_mean": float(accepted.mean()),
-                   "steps_max_over_mean": float(accepted.max() / accepted.mean()),
-                   "l2": "output states %.2f GB, larger than L2 together with the inputs; compute-bound, no flush"
-                         % (u_save.numel() * esz / 1e9),
-                   "parallelism": f"dp{world} (independent trajectory shards)"},
+        "config": dict({"workload": f"{args.workload}: {W['desc']}; n={n} per GPU", "n_per_gpu": n,
+                        "steps_mean": float(accepted.mean()),
+                        "steps_max_over_mean": float(accepted.max() / accepted.mean()),
+                        "l2": "outputs %.2f GB, larger than L2; compute-bound, no flush"
+                              % (sum(t.numel() * t.element_size() for t in outputs) / 1e9),
+                        "parallelism": f"dp{world} (independent trajectory shards)"}, **work),
         "clocks": clocks,
-        "e2e": {"value": world * n / float(e2e_t.item()), "unit": "trajectory-solves/s",
+        "e2e": {"value": world * n / float(e2e_t.item()), "unit": unit,
                 "h2d_bytes_per_step": sum(v.numel() for v in host.values()) * esz,
-                "d2h_bytes_per_step": h_out.numel() * esz},
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_out)},
         "gpu_launches": launches,
         "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": peak / 1e12, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None, "kernel": W["kernel"],
@@ -379,7 +426,7 @@ def run_solve(args):
                      "flops_per_launch": flops},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args, min(16384, n))
+        line["cpu_baseline"] = cpu_baseline(args, min(262144 if kind == "solve" else 32768, n))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -553,7 +600,9 @@ def run_ours(args):
                      "flops_per_launch": flops},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sample = {"lorenz_1m": 2048, "lorenz_small": 1024, "robertson": 64, "node64": 256}[args.workload]
+        # samples sized for seconds of host work (and host memory for the
+        # oracle's trajectory-major meshes)
+        sample = {"lorenz_1m": 32768, "lorenz_small": 1024, "robertson": 256, "node64": 1024}[args.workload]
         line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
     if world > 1:
         dist.barrier()
@@ -566,8 +615,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
-    elif WORKLOADS[args.workload].get("kind") == "solve":
-        run_solve(args)
+    elif WORKLOADS[args.workload].get("kind") in ("solve", "sens"):
+        run_single(args)
     else:
         run_ours(args)
 

@@ -20,6 +20,9 @@ template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                                    cudaStream_t);
 template <typename T>
+gs_status launch_sens_tsit5_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
+                                   cudaStream_t);
+template <typename T>
 gs_status launch_grad_ros2(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                            cudaStream_t);
 template <typename T>
@@ -176,6 +179,21 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
     return P->dtype == GS_F64 ? launch_grad_ros2<double>(P, M, Ls, loss, dp, du0, ws, st)
                               : launch_grad_ros2<float>(P, M, Ls, loss, dp, du0, ws, st);
   return GS_EUNSUPPORTED;
+}
+
+gs_status gs_sens(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp, void* du0,
+                  void* sens, void* stream) {
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if ((rc = check_mesh(P, M)) != GS_OK) return rc;
+  if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
+  if (P->system != GS_LORENZ || P->method != GS_TSIT5) return GS_EUNSUPPORTED;
+  if (P->n == 0) return GS_OK;
+  if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;
+  if (!loss || !dp || !du0) return GS_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  return P->dtype == GS_F64 ? launch_sens_tsit5_lorenz<double>(P, M, Ls, loss, dp, du0, sens, st)
+                            : launch_sens_tsit5_lorenz<float>(P, M, Ls, loss, dp, du0, sens, st);
 }
 
 }  // extern "C"

@@ -1,0 +1,264 @@
+// sens_tsit5.cu -- forward sensitivities of the fixed-step Tsit5 replay on the
+// Lorenz system: the tangent of the replay along each input direction
+// (sigma, rho, beta, x0, y0, z0), integrated alongside the state.
+//
+// The derivative is the one the adjoint returns: the exact derivative of the
+// fixed-step replay of the recorded steps, the mesh held as data (GRADSOLVE,
+// evolve.pub review, "Strengths: precisely scoped exactness claim").  Forward
+// mode gives, besides the loss gradient, the whole sensitivity matrix
+// d u(t_k) / d (p, u0) at every save point; it is the few-parameter route the
+// gptget summary contrasts with the adjoint.
+//
+// Tangent of one Tsit5 step along a direction (v = du, w = dp):
+//   dk_j = J(U_j) dU_j + f_p(U_j) w,   dU_j = v + h sum_{m<j} a_jm dk_m,
+//   v' = v + h sum_j b_j dk_j,
+// with dk_1 carried over from the previous step (FSAL, as k_1).
+//
+// Execution: one thread per (slot, NDIR directions).  The six directions of a
+// slot run in 6 / NDIR threads, each of which replays the state itself: the
+// state costs 192 flop a step against 252 per direction, and holding all six
+// tangents (7 slopes x 3 components x 6 directions) would not fit in
+// registers.  Consecutive blocks take the direction sets of one range of 128
+// slots (block b: slots 128 (b / G) .., direction set b % G, G = 6 / NDIR), so
+// the threads of a warp share one direction set and read consecutive elements
+// of the step-major mesh, and the G blocks of a range run side by side and
+// share those lines through L2 (the mesh crosses HBM once, not G times).  No
+// workspace: nothing is stored but the save-point sensitivities.
+#include "vec.cuh"
+
+namespace gs {
+
+#ifndef GS_SENS_NDIR
+#define GS_SENS_NDIR 1
+#endif
+#ifndef GS_SENS_MINB
+#define GS_SENS_MINB 4
+#endif
+
+template <typename T>
+struct SensArgs {
+  int64_t n;
+  const T* p;   // [3][n] by trajectory
+  const T* u0;  // [3][n] by trajectory
+  const T* h;   // [smax][n] by slot
+  const int32_t* order;
+  const int32_t* nsteps;
+  const int32_t* save_idx;  // [nsave][n] by slot
+  const int32_t* status;
+  int32_t nsave, smax, loss_kind;
+  const T* target;  // [nsave][3][n] by trajectory, may be null
+  const T* weight;  // [nsave][3][n] by trajectory
+  T* loss;          // [n]
+  T* dp;            // [3][n]
+  T* du0;           // [3][n]
+  T* sens;          // [nsave][3][6][n], may be null
+};
+
+// J(u) v + f_p(u) w for f = (s (y - x), x (r - z) - y, x y - b z).
+template <typename T, typename V>
+__device__ __forceinline__ void lorenz_jvp(T x, T y, T z, T s, T r, T b, const V& vx, const V& vy, const V& vz,
+                                           const V& ws, const V& wr, const V& wb, V& gx, V& gy, V& gz) {
+  gx = fmaT(s, vy - vx, ws * (y - x));
+  gy = fmaT(r - z, vx, fmaT(x, wr - vz, -vy));
+  gz = fmaT(y, vx, fmaT(x, vy, -fmaT(b, vz, wb * z)));
+}
+
+// stage accumulators in the contract's order (state) and the same order for
+// the tangents
+#define GS_S_ACC1(A, K)          \
+  ax = cst<T>(A) * K##x;         \
+  ay = cst<T>(A) * K##y;         \
+  az = cst<T>(A) * K##z;         \
+  dax = cst<T>(A) * d##K##x;     \
+  day = cst<T>(A) * d##K##y;     \
+  daz = cst<T>(A) * d##K##z;
+#define GS_S_ACCN(A, K)                 \
+  ax = fmaT(cst<T>(A), K##x, ax);       \
+  ay = fmaT(cst<T>(A), K##y, ay);       \
+  az = fmaT(cst<T>(A), K##z, az);       \
+  dax = fmaT(cst<T>(A), d##K##x, dax);  \
+  day = fmaT(cst<T>(A), d##K##y, day);  \
+  daz = fmaT(cst<T>(A), d##K##z, daz);
+#define GS_S_STAGE(KN)                                                \
+  Ux = fmaT(h, ax, x);                                                \
+  Uy = fmaT(h, ay, y);                                                \
+  Uz = fmaT(h, az, z);                                                \
+  dUx = fmaT(h, dax, vx);                                             \
+  dUy = fmaT(h, day, vy);                                             \
+  dUz = fmaT(h, daz, vz);                                             \
+  lorenz_f(Ux, Uy, Uz, s, r, b, KN##x, KN##y, KN##z);                 \
+  lorenz_jvp(Ux, Uy, Uz, s, r, b, dUx, dUy, dUz, ws, wr, wb, d##KN##x, d##KN##y, d##KN##z);
+
+template <typename T, int NDIR>
+__global__ void __launch_bounds__(128, GS_SENS_MINB) k_sens_tsit5_lorenz(SensArgs<T> a) {
+  using V = vec<T, NDIR>;
+  const int64_t n = a.n;
+  constexpr int G = 6 / NDIR;
+  const int64_t j = (int64_t)(blockIdx.x / G) * blockDim.x + threadIdx.x;
+  const int dir0 = (int)(blockIdx.x % G) * NDIR;  // this thread's directions: dir0 .. dir0 + NDIR - 1
+  if (j >= n) return;
+  const int64_t i = a.order[j];
+  if (i < 0 || i >= n) return;
+  const int S = a.nsteps[j];
+  const int64_t n3 = 3 * n;
+  if (a.status[j] != GS_TRAJ_OK || S < 0 || S > a.smax) {
+    const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
+    if (dir0 == 0) a.loss[i] = nan;
+#pragma unroll
+    for (int q = 0; q < NDIR; ++q) {
+      const int dq = dir0 + q;
+      (dq < 3 ? a.dp : a.du0)[(dq % 3) * n + i] = nan;
+      if (a.sens)
+        for (int k = 0; k < a.nsave; ++k)
+#pragma unroll
+          for (int c = 0; c < 3; ++c) a.sens[(((int64_t)k * 3 + c) * 6 + dq) * n + i] = nan;
+    }
+    return;
+  }
+  const T s = a.p[i], r = a.p[n + i], b = a.p[2 * n + i];
+  T x = a.u0[i], y = a.u0[n + i], z = a.u0[2 * n + i];
+  V ws, wr, wb, vx, vy, vz;
+#pragma unroll
+  for (int q = 0; q < NDIR; ++q) {
+    const int dq = dir0 + q;
+    ws.e[q] = dq == 0 ? cst<T>(1.0) : cst<T>(0.0);
+    wr.e[q] = dq == 1 ? cst<T>(1.0) : cst<T>(0.0);
+    wb.e[q] = dq == 2 ? cst<T>(1.0) : cst<T>(0.0);
+    vx.e[q] = dq == 3 ? cst<T>(1.0) : cst<T>(0.0);
+    vy.e[q] = dq == 4 ? cst<T>(1.0) : cst<T>(0.0);
+    vz.e[q] = dq == 5 ? cst<T>(1.0) : cst<T>(0.0);
+  }
+  T L = cst<T>(0.0);
+  V dL = vsplat<T, NDIR>(cst<T>(0.0));
+  int kk = 0, next = S > 0 ? a.save_idx[j] : -1;
+  T k1x, k1y, k1z;
+  V dk1x, dk1y, dk1z;
+  lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);
+  lorenz_jvp(x, y, z, s, r, b, vx, vy, vz, ws, wr, wb, dk1x, dk1y, dk1z);
+  const T* hq = a.h + j;
+  T hn = S > 0 ? hq[0] : cst<T>(0.0);
+  for (int st = 0; st < S; ++st) {
+    const T h = hn;
+    hq += n;
+    if (st + 1 < S) hn = *hq;
+    if (st + 8 < S) prefetch_l2(hq + 7 * n);
+    T ax, ay, az, Ux, Uy, Uz;
+    V dax, day, daz, dUx, dUy, dUz;
+    T k2x, k2y, k2z, k3x, k3y, k3z, k4x, k4y, k4z, k5x, k5y, k5z, k6x, k6y, k6z;
+    V dk2x, dk2y, dk2z, dk3x, dk3y, dk3z, dk4x, dk4y, dk4z, dk5x, dk5y, dk5z, dk6x, dk6y, dk6z;
+    GS_S_ACC1(TS_A21, k1)
+    GS_S_STAGE(k2)
+    GS_S_ACC1(TS_A31, k1)
+    GS_S_ACCN(TS_A32, k2)
+    GS_S_STAGE(k3)
+    GS_S_ACC1(TS_A41, k1)
+    GS_S_ACCN(TS_A42, k2)
+    GS_S_ACCN(TS_A43, k3)
+    GS_S_STAGE(k4)
+    GS_S_ACC1(TS_A51, k1)
+    GS_S_ACCN(TS_A52, k2)
+    GS_S_ACCN(TS_A53, k3)
+    GS_S_ACCN(TS_A54, k4)
+    GS_S_STAGE(k5)
+    GS_S_ACC1(TS_A61, k1)
+    GS_S_ACCN(TS_A62, k2)
+    GS_S_ACCN(TS_A63, k3)
+    GS_S_ACCN(TS_A64, k4)
+    GS_S_ACCN(TS_A65, k5)
+    GS_S_STAGE(k6)
+    // u_{s+1} and its tangent
+    GS_S_ACC1(TS_B1, k1)
+    GS_S_ACCN(TS_B2, k2)
+    GS_S_ACCN(TS_B3, k3)
+    GS_S_ACCN(TS_B4, k4)
+    GS_S_ACCN(TS_B5, k5)
+    GS_S_ACCN(TS_B6, k6)
+    x = fmaT(h, ax, x);
+    y = fmaT(h, ay, y);
+    z = fmaT(h, az, z);
+    vx = fmaT(h, dax, vx);
+    vy = fmaT(h, day, vy);
+    vz = fmaT(h, daz, vz);
+    lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);  // FSAL
+    lorenz_jvp(x, y, z, s, r, b, vx, vy, vz, ws, wr, wb, dk1x, dk1y, dk1z);
+    if (st + 1 == next) {
+      const int64_t o = (int64_t)kk * n3 + i;
+      if (a.loss_kind == GS_LOSS_SUMSQ) {
+        const T ex = a.target ? x - a.target[o] : x;
+        const T ey = a.target ? y - a.target[o + n] : y;
+        const T ez = a.target ? z - a.target[o + 2 * n] : z;
+        L = fmaT(ex, ex, L);
+        L = fmaT(ey, ey, L);
+        L = fmaT(ez, ez, L);
+        dL = fmaT(cst<T>(2.0) * ex, vx, dL);
+        dL = fmaT(cst<T>(2.0) * ey, vy, dL);
+        dL = fmaT(cst<T>(2.0) * ez, vz, dL);
+      } else {
+        const T w0 = a.weight[o], w1 = a.weight[o + n], w2 = a.weight[o + 2 * n];
+        L = fmaT(w0, x, L);
+        L = fmaT(w1, y, L);
+        L = fmaT(w2, z, L);
+        dL = fmaT(w0, vx, dL);
+        dL = fmaT(w1, vy, dL);
+        dL = fmaT(w2, vz, dL);
+      }
+      if (a.sens) {
+#pragma unroll
+        for (int q = 0; q < NDIR; ++q) {
+          T* o6 = a.sens + ((int64_t)kk * 18 + dir0 + q) * n + i;
+          o6[0] = vx.e[q];
+          o6[6 * n] = vy.e[q];
+          o6[12 * n] = vz.e[q];
+        }
+      }
+      ++kk;
+      next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
+    }
+  }
+  if (dir0 == 0) a.loss[i] = L;
+#pragma unroll
+  for (int q = 0; q < NDIR; ++q) {
+    const int dq = dir0 + q;
+    (dq < 3 ? a.dp : a.du0)[(dq % 3) * n + i] = dL.e[q];
+  }
+}
+
+#undef GS_S_ACC1
+#undef GS_S_ACCN
+#undef GS_S_STAGE
+
+template <typename T>
+gs_status launch_sens_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp,
+                                   void* du0, void* sens, cudaStream_t st) {
+  SensArgs<T> a;
+  a.n = P->n;
+  a.p = (const T*)P->p;
+  a.u0 = (const T*)P->u0;
+  a.h = (const T*)M->h;
+  a.order = M->order;
+  a.nsteps = M->nsteps;
+  a.save_idx = M->save_idx;
+  a.status = M->status;
+  a.nsave = P->nsave;
+  a.smax = M->smax;
+  a.loss_kind = Ls->kind;
+  a.target = (const T*)Ls->target;
+  a.weight = (const T*)Ls->weight;
+  a.loss = (T*)loss;
+  a.dp = (T*)dp;
+  a.du0 = (T*)du0;
+  a.sens = (T*)sens;
+  constexpr int ND = GS_SENS_NDIR;
+  static_assert(6 % ND == 0, "directions per thread must divide 6");
+  const int64_t grid = (P->n + 127) / 128 * (6 / ND);
+  k_sens_tsit5_lorenz<T, ND><<<(unsigned)grid, 128, 0, st>>>(a);
+  count_launch();
+  return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
+template gs_status launch_sens_tsit5_lorenz<double>(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*,
+                                                    void*, void*, cudaStream_t);
+template gs_status launch_sens_tsit5_lorenz<float>(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*,
+                                                   void*, void*, cudaStream_t);
+
+}  // namespace gs

@@ -73,6 +73,8 @@ _lib.gs_solve.argtypes = [_P(_Problem), _P(_Mesh), ctypes.c_void_p, ctypes.c_voi
 _lib.gs_solve_adaptive.argtypes = [_P(_Problem), _P(_Tol), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p]
 _lib.gs_solve_adaptive.restype = ctypes.c_int32
+_lib.gs_sens.argtypes = [_P(_Problem), _P(_Mesh), _P(_Loss)] + [ctypes.c_void_p] * 5
+_lib.gs_sens.restype = ctypes.c_int32
 _lib.gs_solve.restype = ctypes.c_int32
 _lib.gs_grad.argtypes = [_P(_Problem), _P(_Mesh), _P(_Loss), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
@@ -279,6 +281,26 @@ def gs_grad(ens: Ensemble, mesh: Mesh, loss: str = "sumsq", target=None, weight=
     _check(_lib.gs_grad(ctypes.byref(ps), ctypes.byref(ms), ctypes.byref(ls), _ptr(out.loss), _ptr(out.dp),
                         _ptr(out.du0), _ptr(out.dshared), _ptr(ws), ws.numel(), _stream(stream)), "gs_grad")
     return out
+
+
+def gs_sens(ens: Ensemble, mesh: Mesh, loss: str = "sumsq", target=None, weight=None, out: GradOut | None = None,
+            sens=True, stream=None):
+    """Forward sensitivities of the fixed-step replay: (GradOut with the loss and
+    its gradient by forward mode, sens [nsave][d][np + d][n] or None).  Pass
+    sens=False to skip the matrices, or a tensor to write them into."""
+    if out is None:
+        out = new_grad_out(ens)
+    if sens is True:
+        sens = torch.empty((len(ens.tsave), ens.d, ens.np_ + ens.d, ens.n), dtype=TORCH_DTYPE[ens.dtype],
+                           device=ens.u0.device)
+    elif sens is False:
+        sens = None
+    ps, ms = ens._struct(), mesh._struct()
+    ls = _Loss(LOSSES[loss], None if target is None else target.data_ptr(),
+               None if weight is None else weight.data_ptr())
+    _check(_lib.gs_sens(ctypes.byref(ps), ctypes.byref(ms), ctypes.byref(ls), _ptr(out.loss), _ptr(out.dp),
+                        _ptr(out.du0), _ptr(sens), _stream(stream)), "gs_sens")
+    return out, sens
 
 
 def gs_grad_static(ens: Ensemble, mesh: Mesh, loss: str = "sumsq", target=None, weight=None,

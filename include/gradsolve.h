@@ -220,6 +220,25 @@ GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_l
                   void* du0, void* dshared, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Forward sensitivities on the mesh: the tangent of the fixed-step replay
+ * along every input direction -- the np parameters, then the d initial-state
+ * components -- integrated alongside the state (forward mode).  The same
+ * derivative as gs_grad (of the replay, the mesh held as data), and besides
+ * the loss gradient the whole sensitivity matrix at every save point:
+ *   sens     device [nsave][d][np + d][n] dtype, by trajectory:
+ *            sens[k][c][j][i] = d u_c(t_k) / d theta_j for trajectory i, with
+ *            theta = (p_0 .. p_{np-1}, u0_0 .. u0_{d-1}); may be NULL
+ *   loss, dp, du0: as gs_grad (dL/dp and dL/du0 by the chain rule through the
+ *            tangents)
+ * Needs no workspace.  Slots with status != 0 get NaN everywhere.  Built for
+ * GS_LORENZ with GS_TSIT5 (np + d = 6), fp64 and fp32; other problems return
+ * GS_EUNSUPPORTED.  (The few-parameter forward-sensitivity route that the
+ * gptget summary sets beside the adjoint.)
+ */
+GS_API gs_status gs_sens(const gs_problem* prob, const gs_mesh* mesh, const gs_loss* loss_desc, void* loss, void* dp,
+                         void* du0, void* sens, void* stream);
+
+/*
  * gs_grad without a caller workspace, for callers that cannot allocate device
  * memory (a plugin whose host application owns all device memory, a real-time
  * loop that may not call cudaMalloc, a C host without an allocator).  Same

@@ -18,7 +18,7 @@ def _declared():
 
 def test_header_declares_entry_points():
     names = set(_declared())
-    assert {"gs_workspace_bytes", "gs_count", "gs_record", "gs_solve", "gs_solve_adaptive", "gs_grad",
+    assert {"gs_workspace_bytes", "gs_count", "gs_record", "gs_solve", "gs_solve_adaptive", "gs_grad", "gs_sens",
             "gs_status_string", "gs_launch_count"} <= names
 
 
@@ -110,6 +110,13 @@ def test_bad_tolerance_and_workspace_rejected():
                                   None) == -1
     assert _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(_Tol(0.0, 0.0, 0.0)), 100, ctypes.c_void_p(16),
                                   None, None, None) == -1
+    # forward sensitivities: Lorenz with Tsit5 only, and the gradient outputs are required
+    ls = _Loss(1, None, None)
+    assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(m), ctypes.byref(ls), None, ctypes.c_void_p(16),
+                        ctypes.c_void_p(16), None, None) == -1
+    rob = _host_problem(system=2, method=2)
+    assert _lib.gs_sens(ctypes.byref(rob), ctypes.byref(m), ctypes.byref(ls), ctypes.c_void_p(16),
+                        ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == -4
     # mesh nsave must match
     m2 = _Mesh(100, 3, 16, 16, 16, 16, 16, 16)
     assert _lib.gs_solve(ctypes.byref(p), ctypes.byref(m2), ctypes.c_void_p(16), None) == -1
@@ -128,4 +135,6 @@ def test_empty_ensemble_is_a_no_op():
     assert _lib.gs_solve(ctypes.byref(p), ctypes.byref(m), None, None) == 0
     assert _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, None, None, None,
                                   None) == 0
+    assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(m), ctypes.byref(_Loss(1, None, None)), None, None, None,
+                        None, None) == 0
     assert _lib.gs_launch_count() == before
