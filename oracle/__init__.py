@@ -58,16 +58,16 @@ def lib():
         ip = ctypes.POINTER(ctypes.c_int)
         i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
         L.or_record.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, f64, f64, i32, dp, f64, f64, f64,
-                                i32, dp, ip, ip, ip, ip, i32]
-        L.or_grad.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, ip, i32, dp, dp,
+                                i32, dp, ip, ip, ip, ip, i32, dp, i32]
+        L.or_grad.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, dp, ip, i32, dp, dp,
                               i32, dp, dp, dp, dp, i32]
-        L.or_dirderiv.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, i32, dp, dp,
+        L.or_dirderiv.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, dp, i32, dp, dp,
                                   dp, dp, dp, dp, i32]
-        L.or_replay.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, i32, dp, dp,
+        L.or_replay.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, i32, dp, ip, ip, dp, i32, dp, dp,
                                 dp, dp, i32]
         L.or_solve_adaptive.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, f64, f64, i32, dp, f64, f64,
-                                        f64, i32, dp, ip, ip, i32]
-        L.or_sens.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, i32, i32, dp, ip, ip, ip, dp, i32]
+                                        f64, i32, i32, dp, ip, ip, i32]
+        L.or_sens.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, i32, i32, dp, ip, ip, dp, ip, dp, i32]
         L.or_count_step.argtypes = [i32, i32, i32, i32, dp]
         L.or_step.argtypes = [i32, i32, i32, i32, dp, dp, dp, f64, dp, dp]
         L.or_rhs.argtypes = [i32, i32, dp, dp, dp, dp, dp]
@@ -108,6 +108,7 @@ class Mesh:
     save_idx: np.ndarray  # [n][nsave] int32
     status: np.ndarray    # [n] int32
     nreject: np.ndarray   # [n] int32
+    theta: np.ndarray | None = None  # [n][nsave] dense-output positions in (0, 1]; None: save points end steps
 
     @property
     def smax(self) -> int:
@@ -119,8 +120,10 @@ def _check(rc: int, what: str):
         raise RuntimeError(f"oracle {what} failed with code {rc}")
 
 
-def record(prob, smax: int, h0: float = 0.0, nthreads: int | None = None) -> Mesh:
-    """Adaptive record of every trajectory of ``prob`` (a ``workloads.Problem``)."""
+def record(prob, smax: int, h0: float = 0.0, nthreads: int | None = None, dense: bool = False) -> Mesh:
+    """Adaptive record of every trajectory of ``prob`` (a ``workloads.Problem``).
+    dense: steps do not stop at the save times; each save time is located inside
+    its step by theta (the mesh's ``theta``) and read off the Hermite interpolant."""
     L = lib()
     n, nsave = prob.n, len(prob.tsave)
     p, u0, W, ts = _f64(prob.p), _f64(prob.u0), _f64(prob.W), _f64(prob.tsave)
@@ -129,14 +132,16 @@ def record(prob, smax: int, h0: float = 0.0, nthreads: int | None = None) -> Mes
     save_idx = np.zeros((n, max(nsave, 1)), np.int32)
     status = np.zeros(n, np.int32)
     nrej = np.zeros(n, np.int32)
+    theta = np.ones((n, max(nsave, 1)), np.float64)
     rc = L.or_record(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, prob.d, prob.np_,
                      _d(p), _d(u0), _d(W), prob.t0, prob.t1, nsave, _d(ts), prob.rtol, prob.atol, h0, smax,
-                     _d(h), _i(nsteps), _i(save_idx), _i(status), _i(nrej), nthreads or default_threads())
+                     _d(h), _i(nsteps), _i(save_idx), _i(status), _i(nrej), int(dense), _d(theta),
+                     nthreads or default_threads())
     _check(rc, "record")
-    return Mesh(h, nsteps, save_idx[:, :nsave], status, nrej)
+    return Mesh(h, nsteps, save_idx[:, :nsave], status, nrej, theta[:, :nsave] if dense else None)
 
 
-def solve_adaptive(prob, smax: int, h0: float = 0.0, nthreads: int | None = None):
+def solve_adaptive(prob, smax: int, h0: float = 0.0, nthreads: int | None = None, dense: bool = False):
     """Adaptive forward-only solve: (u_save [nsave][d][n], nsteps [n], status [n]).
     The recorder's iteration with its accepted states at the save times kept
     (NaN everywhere for a trajectory whose status is not 0)."""
@@ -147,7 +152,8 @@ def solve_adaptive(prob, smax: int, h0: float = 0.0, nthreads: int | None = None
     status = np.zeros(n, np.int32)
     rc = L.or_solve_adaptive(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, prob.d, prob.np_,
                              _d(_f64(prob.p)), _d(_f64(prob.u0)), _d(_f64(prob.W)), prob.t0, prob.t1, nsave,
-                             _d(_f64(prob.tsave)), prob.rtol, prob.atol, h0, smax, _d(us), _i(nsteps), _i(status),
+                             _d(_f64(prob.tsave)), prob.rtol, prob.atol, h0, smax, int(dense), _d(us), _i(nsteps),
+                             _i(status),
                              nthreads or default_threads())
     _check(rc, "solve_adaptive")
     return us, nsteps, status
@@ -158,6 +164,10 @@ def _mesh_args(mesh: Mesh):
     ns = np.ascontiguousarray(mesh.nsteps, np.int32)
     si = np.ascontiguousarray(mesh.save_idx, np.int32)
     return h, ns, si
+
+
+def _theta(mesh: Mesh):
+    return None if mesh.theta is None else _d(np.ascontiguousarray(mesh.theta, np.float64))
 
 
 def grad(prob, mesh: Mesh, mode: str = "tape", nthreads: int | None = None):
@@ -178,8 +188,8 @@ def grad(prob, mesh: Mesh, mode: str = "tape", nthreads: int | None = None):
     du0 = np.zeros((d, n))
     dW = np.zeros((64, 64)) if prob.system == "node64" else None
     rc = L.or_grad(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, d, npar, _d(_f64(prob.p)),
-                   _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si), _i(st),
-                   LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), {"tape": 0, "dual": 1, "tape_wide": 2}[mode],
+                   _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si),
+                   _theta(mesh), _i(st), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), {"tape": 0, "dual": 1, "tape_wide": 2}[mode],
                    _d(loss), _d(dp), _d(du0), _d(dW), nthreads or default_threads())
     _check(rc, "grad")
     return {"loss": loss, "dp": dp, "du0": du0, "dW": dW}
@@ -192,8 +202,8 @@ def dirderiv(prob, mesh: Mesh, dir_p=None, dir_u0=None, dir_W=None, nthreads: in
     out = np.zeros(prob.n)
     rc = L.or_dirderiv(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], prob.n, prob.d, prob.np_,
                        _d(_f64(prob.p)), _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h),
-                       _i(ns), _i(si), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)),
-                       _d(_f64(dir_p)), _d(_f64(dir_u0)), _d(_f64(dir_W)), _d(out), nthreads or default_threads())
+                       _i(ns), _i(si), _theta(mesh), LOSSES[prob.loss], _d(_f64(prob.target)),
+                       _d(_f64(prob.weight)), _d(_f64(dir_p)), _d(_f64(dir_u0)), _d(_f64(dir_W)), _d(out), nthreads or default_threads())
     _check(rc, "dirderiv")
     return out
 
@@ -207,8 +217,8 @@ def sens(prob, mesh: Mesh, nthreads: int | None = None):
     st = np.ascontiguousarray(mesh.status, np.int32)
     out = np.zeros((si.shape[1], prob.d, prob.np_ + prob.d, prob.n))
     rc = L.or_sens(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], prob.n, prob.d, prob.np_,
-                   _d(_f64(prob.p)), _d(_f64(prob.u0)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si), _i(st),
-                   _d(out), nthreads or default_threads())
+                   _d(_f64(prob.p)), _d(_f64(prob.u0)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si),
+                   _theta(mesh), _i(st), _d(out), nthreads or default_threads())
     _check(rc, "sens")
     return out
 
@@ -221,8 +231,8 @@ def replay(prob, mesh: Mesh, nthreads: int | None = None):
     us = np.zeros((si.shape[1], prob.d, prob.n))
     rc = L.or_replay(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], prob.n, prob.d, prob.np_,
                      _d(_f64(prob.p)), _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h),
-                     _i(ns), _i(si), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), _d(loss),
-                     _d(us), nthreads or default_threads())
+                     _i(ns), _i(si), _theta(mesh), LOSSES[prob.loss], _d(_f64(prob.target)),
+                     _d(_f64(prob.weight)), _d(loss), _d(us), nthreads or default_threads())
     _check(rc, "replay")
     return loss, us
 

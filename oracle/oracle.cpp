@@ -447,12 +447,34 @@ T ctrl_pow(T x, T y) {
 // every save time and on t1; save_idx[k] is the number of accepted steps taken
 // when t reached tsave[k].  Starting step: Hairer, Norsett & Wanner I, II.4.
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// Dense output between the ends of one step (save points that steps do not
+// land on): the cubic Hermite interpolant on [t_s, t_s + h] at theta in (0, 1],
+//   u(theta) = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
+//   H01 = theta^2 (3 - 2 theta),  H00 = 1 - H01,
+//   H10 = theta (1 - theta)^2,    H11 = -theta^2 (1 - theta),
+// the weights and the combination in this operation order.  theta is data
+// (no derivative), like h.
+// ---------------------------------------------------------------------------
+template <class S>
+void hermite(int d, const S* us, const S* un, const S* fs, const S* fn, S h, double theta, S* out) {
+  using T = typename base_of<S>::type;
+  const T th = T(theta);
+  const T t2 = th * th, om = T(1) - th;
+  const T H01 = t2 * std::fma(T(-2), th, T(3));
+  const T H00 = T(1) - H01;
+  const T H10 = (th * om) * om;
+  const T H11 = -(t2 * om);
+  for (int c = 0; c < d; ++c) out[c] = fma_(S(H00), us[c], fma_(S(H01), un[c], h * fma_(S(H10), fs[c], S(H11) * fn[c])));
+}
+
 template <class T>
 struct RecordOut {
   std::vector<T> h;
   int nsteps = 0, nreject = 0, status = TRAJ_OK;
   std::vector<int> save_idx;
   std::vector<T> usave;  // [nsave][d]: the accepted state at each save time (the forward-only solve)
+  std::vector<T> theta;  // [nsave]: dense mode, position of each save time inside its step (else 1)
 };
 
 template <class T>
@@ -487,9 +509,12 @@ T initial_step(int sys, int method, int d, const T* u0, const T* p, const T* W, 
 
 template <class T>
 RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, const T* W, T t0, T t1,
-                        int nsave, const T* tsave, T rtol, T atol, T h0user, int smax) {
+                        int nsave, const T* tsave, T rtol, T atol, T h0user, int smax, bool dense = false) {
+  // dense: steps stop only at t1; a save time inside a step is located by its
+  // position theta in (0, 1] and read off the Hermite interpolant
   RecordOut<T> out;
   out.save_idx.assign(nsave, 0);
+  out.theta.assign(nsave, T(1));
   out.usave.assign((size_t)nsave * d, std::numeric_limits<T>::quiet_NaN());
   const T eps = std::numeric_limits<T>::epsilon();
   const T q = method == M_TSIT5 ? T(5) : T(2);
@@ -512,7 +537,7 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
   bool prev_rej = false;
   int kk = 0;
   while (true) {
-    T tstop = kk < nsave ? tsave[kk] : t1;
+    T tstop = (kk < nsave && !dense) ? tsave[kk] : t1;
     if (hprop < T(16) * eps * std::fabs(t)) {
       out.status = TRAJ_DTMIN;
       return out;
@@ -536,9 +561,22 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
       }
       out.h.push_back(h);
       out.nsteps++;
+      const T tprev = t;
       t = clipped ? tstop : tn;
+      if (dense) {
+        while (kk < nsave && tsave[kk] <= t) {
+          const T th = (tsave[kk] - tprev) / h;
+          out.theta[kk] = th;
+          T fs[DMAX] = {}, fn[DMAX] = {}, ut[DMAX] = {};
+          rhs<T>(sys, u, p, W, fs);
+          rhs<T>(sys, un, p, W, fn);
+          hermite<T>(d, u, un, fs, fn, h, double(th), ut);
+          for (int c = 0; c < d; ++c) out.usave[(size_t)kk * d + c] = th == T(1) ? un[c] : ut[c];
+          out.save_idx[kk++] = out.nsteps;
+        }
+      }
       for (int c = 0; c < d; ++c) u[c] = un[c];
-      while (kk < nsave && t == tsave[kk]) {
+      while (!dense && kk < nsave && t == tsave[kk]) {
         for (int c = 0; c < d; ++c) out.usave[(size_t)kk * d + c] = u[c];
         out.save_idx[kk++] = out.nsteps;
       }
@@ -580,35 +618,49 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
 template <class S>
 S replay_loss(int sys, int method, int d, const S* u0, const S* p, const S* W, const double* h, int nsteps,
               int nsave, const int* save_idx, int loss_kind, const double* tgt /*[nsave][d] or null*/,
-              const double* wgt /*[nsave][d]*/, S* u_save /*[nsave][d] or null*/) {
+              const double* wgt /*[nsave][d]*/, S* u_save /*[nsave][d] or null*/,
+              const double* theta = nullptr /*[nsave] or null: save points at step ends*/) {
   using T = typename base_of<S>::type;
-  S u[DMAX], un[DMAX];
+  S u[DMAX], un[DMAX], up[DMAX];
   for (int c = 0; c < d; ++c) u[c] = u0[c];
   S L = S(T(0));
   int kk = 0;
-  auto visit = [&](int s) {
+  // save points reached when s steps are taken; up = u_{s-1}, hs = h[s-1]
+  auto visit = [&](int s, S hs) {
     while (kk < nsave && save_idx[kk] == s) {
+      S ut[DMAX];
+      const S* uk = u;
+      if (theta && theta[kk] != 1.0 && s > 0) {
+        S fs[DMAX], fn[DMAX];
+        rhs<S>(sys, up, p, W, fs);
+        rhs<S>(sys, u, p, W, fn);
+        hermite<S>(d, up, u, fs, fn, hs, theta[kk], ut);
+        uk = ut;
+      }
       for (int c = 0; c < d; ++c) {
-        if (u_save) u_save[kk * d + c] = u[c];
+        if (u_save) u_save[kk * d + c] = uk[c];
         if (loss_kind == LOSS_SUMSQ) {
-          S dlt = tgt ? u[c] - S(T(tgt[kk * d + c])) : u[c];
+          S dlt = tgt ? uk[c] - S(T(tgt[kk * d + c])) : uk[c];
           L = fma_(dlt, dlt, L);
         } else {
-          L = fma_(S(T(wgt[kk * d + c])), u[c], L);
+          L = fma_(S(T(wgt[kk * d + c])), uk[c], L);
         }
       }
       kk++;
     }
   };
-  visit(0);
+  visit(0, S(T(0)));
   for (int s = 0; s < nsteps; ++s) {
     S hs = S(T(h[s]));
     if (method == M_TSIT5)
       tsit5_step<S>(sys, d, u, p, W, hs, un, nullptr);
     else
       ros2_step<S>(sys, d, u, p, hs, un, nullptr);
-    for (int c = 0; c < d; ++c) u[c] = un[c];
-    visit(s + 1);
+    for (int c = 0; c < d; ++c) {
+      up[c] = u[c];
+      u[c] = un[c];
+    }
+    visit(s + 1, hs);
   }
   return L;
 }
@@ -627,6 +679,8 @@ struct Mesh {
   const double* h;      // [n][smax]
   const int* nsteps;    // [n]
   const int* save_idx;  // [n][nsave]
+  const double* theta = nullptr;  // [n][nsave] dense-output positions, or null (save points at step ends)
+  const double* theta_of(int64_t i) const { return theta ? theta + i * nsave : nullptr; }
 };
 
 struct Loss {
@@ -689,7 +743,7 @@ void grad_one_tape(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, dou
   if (Ls.weight) gather_kd(Ls.weight, Mh.nsave, d, P.n, i, wg.data());
   R L = replay_loss<R>(P.sys, P.method, d, u0.data(), p.data(), W.empty() ? nullptr : W.data(),
                        Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave, Mh.save_idx + i * Mh.nsave, Ls.kind,
-                       Ls.target ? tg.data() : nullptr, wg.data(), nullptr);
+                       Ls.target ? tg.data() : nullptr, wg.data(), nullptr, Mh.theta_of(i));
   *loss = double(L.v);
   std::vector<A> adj(tp.nodes.size(), A(0));
   if (L.id >= 0) adj[L.id] = A(1);
@@ -727,7 +781,7 @@ double dirderiv_one(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, co
   if (Ls.weight) gather_kd(Ls.weight, Mh.nsave, d, P.n, i, wg.data());
   D L = replay_loss<D>(P.sys, P.method, d, u0.data(), p.data(), W.empty() ? nullptr : W.data(),
                        Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave, Mh.save_idx + i * Mh.nsave, Ls.kind,
-                       Ls.target ? tg.data() : nullptr, wg.data(), nullptr);
+                       Ls.target ? tg.data() : nullptr, wg.data(), nullptr, Mh.theta_of(i));
   return double(L.d);
 }
 
@@ -745,7 +799,7 @@ void sens_one(const Prob& P, const Mesh& Mh, int64_t i, double* sens) {
     for (int c = 0; c < d; ++c) u0[c] = D(T(P.u0[(int64_t)c * P.n + i]), T(j == np + c ? 1 : 0));
     for (int c = 0; c < np; ++c) p[c] = D(T(P.p[(int64_t)c * P.n + i]), T(j == c ? 1 : 0));
     replay_loss<D>(P.sys, P.method, d, u0.data(), p.data(), nullptr, Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave,
-                   Mh.save_idx + i * Mh.nsave, LOSS_LINEAR, nullptr, wg.data(), us.data());
+                   Mh.save_idx + i * Mh.nsave, LOSS_LINEAR, nullptr, wg.data(), us.data(), Mh.theta_of(i));
     for (int k = 0; k < Mh.nsave; ++k)
       for (int c = 0; c < d; ++c) sens[((int64_t)k * d + c) * m + j] = double(us[k * d + c].d);
   }
@@ -766,7 +820,7 @@ double loss_one(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, double
   if (Ls.weight) gather_kd(Ls.weight, Mh.nsave, d, P.n, i, wg.data());
   T L = replay_loss<T>(P.sys, P.method, d, u0.data(), p.data(), W.empty() ? nullptr : W.data(),
                        Mh.h + i * Mh.smax, Mh.nsteps[i], Mh.nsave, Mh.save_idx + i * Mh.nsave, Ls.kind,
-                       Ls.target ? tg.data() : nullptr, wg.data(), us.data());
+                       Ls.target ? tg.data() : nullptr, wg.data(), us.data(), Mh.theta_of(i));
   if (u_save)
     for (int k = 0; k < Mh.nsave; ++k)
       for (int c = 0; c < d; ++c) u_save[((int64_t)k * d + c) * P.n + i] = double(us[k * d + c]);
@@ -799,7 +853,7 @@ extern "C" {
 int or_record(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
               const double* W, double t0, double t1, int nsave, const double* tsave, double rtol, double atol,
               double h0, int smax, double* h, int* nsteps, int* save_idx, int* status, int* nreject,
-              int nthreads) {
+              int dense, double* theta, int nthreads) {
   Prob P{sys, method, dtype, d, np, n, p, u0, W};
   int rc = check_prob(P);
   if (rc) return rc;
@@ -816,10 +870,12 @@ int or_record(int sys, int method, int dtype, int64_t n, int d, int np, const do
         for (int c = 0; c < d; ++c) uu[c] = T(u0[(int64_t)c * n + i]);
         for (int c = 0; c < np; ++c) pp[c] = T(p[(int64_t)c * n + i]);
         RecordOut<T> r = record_one<T>(sys, method, d, uu.data(), pp.data(), WW.empty() ? nullptr : WW.data(),
-                                       T(t0), T(t1), nsave, ts.data(), T(rtol), T(atol), T(h0), smax);
+                                       T(t0), T(t1), nsave, ts.data(), T(rtol), T(atol), T(h0), smax, dense != 0);
         nsteps[i] = r.nsteps;
         status[i] = r.status;
         nreject[i] = r.nreject;
+        if (theta)
+          for (int k = 0; k < nsave; ++k) theta[i * nsave + k] = double(r.theta[k]);
         for (int s = 0; s < smax; ++s) h[i * smax + s] = s < r.nsteps ? double(r.h[s]) : 0.0;
         for (int k = 0; k < nsave; ++k) save_idx[i * nsave + k] = r.save_idx[k];
       }
@@ -835,7 +891,8 @@ int or_record(int sys, int method, int dtype, int64_t n, int d, int np, const do
 // trajectory with status != 0), nsteps and status [n].
 int or_solve_adaptive(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
                       const double* W, double t0, double t1, int nsave, const double* tsave, double rtol,
-                      double atol, double h0, int smax, double* u_save, int* nsteps, int* status, int nthreads) {
+                      double atol, double h0, int smax, int dense, double* u_save, int* nsteps, int* status,
+                      int nthreads) {
   Prob P{sys, method, dtype, d, np, n, p, u0, W};
   int rc = check_prob(P);
   if (rc) return rc;
@@ -852,7 +909,7 @@ int or_solve_adaptive(int sys, int method, int dtype, int64_t n, int d, int np, 
         for (int c = 0; c < d; ++c) uu[c] = T(u0[(int64_t)c * n + i]);
         for (int c = 0; c < np; ++c) pp[c] = T(p[(int64_t)c * n + i]);
         RecordOut<T> r = record_one<T>(sys, method, d, uu.data(), pp.data(), WW.empty() ? nullptr : WW.data(),
-                                       T(t0), T(t1), nsave, ts.data(), T(rtol), T(atol), T(h0), smax);
+                                       T(t0), T(t1), nsave, ts.data(), T(rtol), T(atol), T(h0), smax, dense != 0);
         nsteps[i] = r.nsteps;
         status[i] = r.status;
         for (int k = 0; k < nsave; ++k)
@@ -875,14 +932,14 @@ int or_solve_adaptive(int sys, int method, int dtype, int64_t n, int d, int np, 
 // trajectories, accumulated per thread chunk and then in chunk order.
 int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
             const double* W, int smax, int nsave, const double* h, const int* nsteps, const int* save_idx,
-            const int* status, int loss_kind, const double* target, const double* weight, int mode,
-            double* loss, double* dp, double* du0, double* dW, int nthreads) {
+            const double* theta, const int* status, int loss_kind, const double* target, const double* weight,
+            int mode, double* loss, double* dp, double* du0, double* dW, int nthreads) {
   Prob P{sys, method, dtype, d, np, n, p, u0, W};
   int rc = check_prob(P);
   if (rc) return rc;
   if (mode == 1 && sys == SYS_NODE64) return -4;
   if (mode < 0 || mode > 2) return -1;
-  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  Mesh Mh{smax, nsave, h, nsteps, save_idx, theta};
   Loss Ls{loss_kind, target, weight};
   int nt = std::max(1, nthreads);
   std::vector<std::vector<double>> dWp(sys == SYS_NODE64 ? nt : 0, std::vector<double>(4096, 0.0));
@@ -936,12 +993,12 @@ int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const doub
 // given input directions (any may be null = zero).  out[n].
 int or_dirderiv(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
                 const double* W, int smax, int nsave, const double* h, const int* nsteps, const int* save_idx,
-                int loss_kind, const double* target, const double* weight, const double* dir_p,
+                const double* theta, int loss_kind, const double* target, const double* weight, const double* dir_p,
                 const double* dir_u0, const double* dir_W, double* out, int nthreads) {
   Prob P{sys, method, dtype, d, np, n, p, u0, W};
   int rc = check_prob(P);
   if (rc) return rc;
-  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  Mesh Mh{smax, nsave, h, nsteps, save_idx, theta};
   Loss Ls{loss_kind, target, weight};
   parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
     std::vector<double> dpi(np, 0.0), dui(d, 0.0);
@@ -960,13 +1017,13 @@ int or_dirderiv(int sys, int method, int dtype, int64_t n, int d, int np, const 
 // [nsave][d][np+d][n]; NaN for trajectories with status != 0 (status may be
 // null).  Not for NODE64 (its W directions are not inputs of this product).
 int or_sens(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0, int smax,
-            int nsave, const double* h, const int* nsteps, const int* save_idx, const int* status, double* sens,
-            int nthreads) {
+            int nsave, const double* h, const int* nsteps, const int* save_idx, const double* theta,
+            const int* status, double* sens, int nthreads) {
   Prob P{sys, method, dtype, d, np, n, p, u0, nullptr};
   int rc = check_prob(P);
   if (rc) return rc;
   if (sys == SYS_NODE64) return -4;
-  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  Mesh Mh{smax, nsave, h, nsteps, save_idx, theta};
   const int m = np + d;
   parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
     std::vector<double> si((size_t)nsave * d * m);
@@ -988,12 +1045,12 @@ int or_sens(int sys, int method, int dtype, int64_t n, int d, int np, const doub
 // points, u_save[nsave][d][n].
 int or_replay(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
               const double* W, int smax, int nsave, const double* h, const int* nsteps, const int* save_idx,
-              int loss_kind, const double* target, const double* weight, double* loss, double* u_save,
-              int nthreads) {
+              const double* theta, int loss_kind, const double* target, const double* weight, double* loss,
+              double* u_save, int nthreads) {
   Prob P{sys, method, dtype, d, np, n, p, u0, W};
   int rc = check_prob(P);
   if (rc) return rc;
-  Mesh Mh{smax, nsave, h, nsteps, save_idx};
+  Mesh Mh{smax, nsave, h, nsteps, save_idx, theta};
   Loss Ls{loss_kind, target, weight};
   parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
     for (int64_t i = a; i < b; ++i)
