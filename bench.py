@@ -55,6 +55,14 @@ WORKLOADS = {
                       dtype="f64",
                       desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, 10 save points with N(0,1) targets, "
                            "1 record + 10 gradient passes"),
+    # the headline with dense-output save points: steps stop only at t1, each
+    # save time is read off the Hermite interpolant of its step (forward 27 and
+    # reverse ~75 flop more per save point)
+    "lorenz_1m_dense": dict(passes=10, flop_step=192 + 264, flop_save=18 + 102, kernel="k_grad_tsit5_lorenz",
+                            problem="lorenz_1m", dense=True, n=1 << 20, dtype="f64",
+                            desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, dense record (steps do not stop at "
+                                 "the 10 save points; Hermite interpolant there) with N(0,1) targets, "
+                                 "1 record + 10 gradient passes"),
     "lorenz_small": dict(passes=1, flop_step=192 + 264, flop_save=12, kernel="k_grad_tsit5_lorenz", n=1024,
                          dtype="f64",
                          desc="Lorenz d=3, t in [0,1], Tsit5 rtol=atol=1e-8, loss sum ||u(T)||^2, "
@@ -87,7 +95,7 @@ WORKLOADS = {
 # the kernel's sources are unchanged
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_grad_tsit5_lorenz_traffic.json")
 KERNEL_SOURCES = ["discrete_adjoint_b200/csrc/grad_tsit5.cu", "discrete_adjoint_b200/csrc/vec.cuh",
-                  "discrete_adjoint_b200/csrc/common.cuh"]
+                  "discrete_adjoint_b200/csrc/common.cuh", "discrete_adjoint_b200/csrc/steps.cuh"]
 
 
 def parse():
@@ -111,6 +119,8 @@ def dist_env():
 
 
 def metric_name(args) -> str:
+    if args.workload == "lorenz_1m_dense":
+        return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, dense save points)"
     if args.workload == "lorenz_1m_sens":
         return f"trajectory-sensitivities/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, forward mode)"
     if args.workload == "lorenz_1m_solve":
@@ -188,11 +198,11 @@ def smax_cap(workload):
     return 4 * workloads.SMAX[WORKLOADS[workload].get("problem", workload)]
 
 
-def oracle_step_time(prob, threads, passes):
+def oracle_step_time(prob, threads, passes, dense=False):
     """Oracle record + `passes` tape gradient passes of `prob` on the host."""
     import oracle
     t0 = time.perf_counter()
-    om = oracle.record(prob, smax_cap(prob.name), nthreads=threads)
+    om = oracle.record(prob, smax_cap(prob.name), nthreads=threads, dense=dense)
     t1 = time.perf_counter()
     oracle.grad(prob, om, nthreads=threads)
     t2 = time.perf_counter()
@@ -221,7 +231,7 @@ def cpu_baseline(args, sample: int):
                 "sample": f"first {sample} of the {args.n} trajectories on the oracle's own mesh: dual-number "
                           f"sensitivities {dt:.2f} s"}
     passes = WORKLOADS[args.workload]["passes"]
-    tr, tg, per_step = oracle_step_time(prob, threads, passes)
+    tr, tg, per_step = oracle_step_time(prob, threads, passes, WORKLOADS[args.workload].get("dense", False))
     return {"value": sample * passes / per_step, "unit": "trajectory-gradients/s", "cores": threads,
             "kind": "oracle",
             "sample": f"first {sample} of the {args.n} trajectories: oracle record {tr:.2f} s + one tape gradient "
@@ -238,7 +248,7 @@ def run_reference(args):
     W = WORKLOADS[args.workload]
     kind = W.get("kind", "grad")
     solve = kind != "grad"
-    sample = {"lorenz_1m": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
+    sample = {"lorenz_1m": 256, "lorenz_1m_dense": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
               "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
@@ -251,7 +261,7 @@ def run_reference(args):
         elif kind == "sens":
             oracle.sens(prob, om, nthreads=threads)
         else:
-            om = oracle.record(prob, smax_cap(args.workload), nthreads=threads)
+            om = oracle.record(prob, smax_cap(args.workload), nthreads=threads, dense=W.get("dense", False))
             for _ in range(W["passes"]):
                 oracle.grad(prob, om, nthreads=threads)
         dt = time.perf_counter() - t0
@@ -469,9 +479,10 @@ def run_ours(args):
     loss_kw = dict(loss=prob.loss, target=d.get("target"), weight=d.get("weight"))
 
     # sizing pass (setup, untimed): mesh capacity = the longest chain
-    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload))
+    dense = W.get("dense", False)
+    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload), dense=dense)
     smax = int(nsteps.max().item())
-    mesh = gs.new_mesh(n, smax, len(prob.tsave), args.dtype, dev)
+    mesh = gs.new_mesh(n, smax, len(prob.tsave), args.dtype, dev, dense=dense)
     ws_rec = gs.workspace(gs.gs_workspace_bytes(ens, mesh, gs.gradsolve.OP_RECORD), dev)
     ws_grad = gs.workspace(gs.gs_workspace_bytes(ens, mesh, gs.gradsolve.OP_GRAD), dev)
     outs = [gs.new_grad_out(ens) for _ in range(2)]
@@ -602,7 +613,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # samples sized for seconds of host work (and host memory for the
         # oracle's trajectory-major meshes)
-        sample = {"lorenz_1m": 32768, "lorenz_small": 1024, "robertson": 256, "node64": 1024}[args.workload]
+        sample = {"lorenz_1m": 32768, "lorenz_1m_dense": 32768, "lorenz_small": 1024, "robertson": 256,
+                  "node64": 1024}[args.workload]
         line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
     if world > 1:
         dist.barrier()

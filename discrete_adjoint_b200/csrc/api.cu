@@ -77,6 +77,15 @@ static gs_status check_mesh(const gs_problem* P, const gs_mesh* M) {
   return GS_OK;
 }
 
+// Tolerances; a dense record is built for Tsit5 on the d = 3 systems.
+static gs_status check_tol(const gs_problem* P, const gs_tol* tol) {
+  if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0))
+    return GS_EINVAL;
+  if (tol->dense != 0 && tol->dense != 1) return GS_EINVAL;
+  if (tol->dense && (P->method != GS_TSIT5 || P->system == GS_NODE64)) return GS_EUNSUPPORTED;
+  return GS_OK;
+}
+
 }  // namespace gs
 
 using namespace gs;
@@ -110,9 +119,8 @@ gs_status gs_count(const gs_problem* P, const gs_tol* tol, int32_t smax, int32_t
                    void* stream) {
   gs_status rc = check_problem(P);
   if (rc != GS_OK) return rc;
-  if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0) ||
-      smax < 1)
-    return GS_EINVAL;
+  if ((rc = check_tol(P, tol)) != GS_OK) return rc;
+  if (smax < 1) return GS_EINVAL;
   if (P->n == 0) return GS_OK;
   if (!nsteps) return GS_EINVAL;
   if (P->system == GS_NODE64)
@@ -125,9 +133,8 @@ gs_status gs_solve_adaptive(const gs_problem* P, const gs_tol* tol, int32_t smax
                             int32_t* status, void* stream) {
   gs_status rc = check_problem(P);
   if (rc != GS_OK) return rc;
-  if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0) ||
-      smax < 1)
-    return GS_EINVAL;
+  if ((rc = check_tol(P, tol)) != GS_OK) return rc;
+  if (smax < 1) return GS_EINVAL;
   if (P->n == 0) return GS_OK;
   if (!u_save) return GS_EINVAL;
   if (P->system == GS_NODE64)
@@ -141,8 +148,8 @@ gs_status gs_record(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, vo
   gs_status rc = check_problem(P);
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
-  if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0))
-    return GS_EINVAL;
+  if ((rc = check_tol(P, tol)) != GS_OK) return rc;
+  if (tol->dense && P->n > 0 && !M->save_theta) return GS_EINVAL;  // a dense record writes the positions
   if (P->n == 0) return GS_OK;
   if (!ws || ws_bytes < gs_workspace_bytes(P, M, GS_OP_RECORD)) return GS_EWORKSPACE;
   if (P->system == GS_NODE64) return record_node64(P, tol, M, ws, (cudaStream_t)stream);
@@ -153,6 +160,7 @@ gs_status gs_solve(const gs_problem* P, const gs_mesh* M, void* u_save, void* st
   gs_status rc = check_problem(P);
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
+  if (M->save_theta && (P->method != GS_TSIT5 || P->system == GS_NODE64)) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (!u_save) return GS_EINVAL;
   if (P->system == GS_NODE64) return node64_solve(P, M, u_save, (cudaStream_t)stream);
@@ -166,6 +174,8 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
+  // dense save points: the Tsit5 Lorenz gradient
+  if (M->save_theta && (P->method != GS_TSIT5 || P->system != GS_LORENZ)) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;
   if (!loss || !dp || !du0) return GS_EINVAL;
@@ -187,7 +197,7 @@ gs_status gs_sens(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
-  if (P->system != GS_LORENZ || P->method != GS_TSIT5) return GS_EUNSUPPORTED;
+  if (P->system != GS_LORENZ || P->method != GS_TSIT5 || M->save_theta) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;
   if (!loss || !dp || !du0) return GS_EINVAL;

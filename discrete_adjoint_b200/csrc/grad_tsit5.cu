@@ -34,6 +34,7 @@
 // Memory layout: h [smax][n] and ck [smax][3][n] are step-major over slots, so
 // at a given step a warp touches 32K consecutive elements of every array.
 // Loads run one step ahead in registers and several steps ahead into L2.
+#include "steps.cuh"
 #include "vec.cuh"
 
 namespace gs {
@@ -77,6 +78,7 @@ struct TsitLorenzArgs {
   T* dp;            // [3][n]
   T* du0;           // [3][n]
   T* ck;            // workspace [smax][3][n] by slot
+  const T* theta;   // [nsave][n] by slot: dense save points, or null
 };
 
 // dL/dU = J(U)^T nu and pbar += f_p(U)^T nu for Lorenz.
@@ -109,7 +111,7 @@ __device__ __forceinline__ void lorenz_vjp(const V& ux, const V& uy, const V& uz
   ay = fmaT(cst<T>(AN), KN##y, ay); \
   az = fmaT(cst<T>(AN), KN##z, az);
 
-template <typename T, int K>
+template <typename T, int K, bool DENSE>
 __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(TsitLorenzArgs<T> a) {
   using V = vec<T, K>;
   const int64_t n = a.n;
@@ -225,30 +227,51 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     GS_ACCN(TS_B4, k4)
     GS_ACCN(TS_B5, k5)
     GS_ACCN(TS_B6, k6)
+    V xs, ys, zs, fsx, fsy, fsz;  // dense save points: u_s and f(u_s)
+    if (DENSE) {
+      xs = x;
+      ys = y;
+      zs = z;
+      fsx = k1x;
+      fsy = k1y;
+      fsz = k1z;
+    }
     x = fmaT(h, ax, x);
     y = fmaT(h, ay, y);
     z = fmaT(h, az, z);
     lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);  // FSAL: next step's first slope
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      if (st + 1 == next[q]) {
+      // a landing record has at most one save point per step; a dense one any number
+      while (st + 1 == next[q]) {
         const int64_t o = (int64_t)kk[q] * n3 + i[q];
+        T ux = x.e[q], uy = y.e[q], uz = z.e[q];
+        if (DENSE) {
+          const T th = a.theta[(int64_t)kk[q] * n + j0 + q];
+          if (th != cst<T>(1.0)) {
+            const HermiteW<T> w = hermite_w(th);
+            ux = hermite_c(w, xs.e[q], ux, fsx.e[q], k1x.e[q], h.e[q]);
+            uy = hermite_c(w, ys.e[q], uy, fsy.e[q], k1y.e[q], h.e[q]);
+            uz = hermite_c(w, zs.e[q], uz, fsz.e[q], k1z.e[q], h.e[q]);
+          }
+        }
         T Lq = L.e[q];
         if (a.loss_kind == GS_LOSS_SUMSQ) {
-          const T dx = a.target ? x.e[q] - a.target[o] : x.e[q];
-          const T dy = a.target ? y.e[q] - a.target[o + n] : y.e[q];
-          const T dz = a.target ? z.e[q] - a.target[o + 2 * n] : z.e[q];
+          const T dx = a.target ? ux - a.target[o] : ux;
+          const T dy = a.target ? uy - a.target[o + n] : uy;
+          const T dz = a.target ? uz - a.target[o + 2 * n] : uz;
           Lq = fmaT(dx, dx, Lq);
           Lq = fmaT(dy, dy, Lq);
           Lq = fmaT(dz, dz, Lq);
         } else {
-          Lq = fmaT(a.weight[o], x.e[q], Lq);
-          Lq = fmaT(a.weight[o + n], y.e[q], Lq);
-          Lq = fmaT(a.weight[o + 2 * n], z.e[q], Lq);
+          Lq = fmaT(a.weight[o], ux, Lq);
+          Lq = fmaT(a.weight[o + n], uy, Lq);
+          Lq = fmaT(a.weight[o + 2 * n], uz, Lq);
         }
         L.e[q] = Lq;
         ++kk[q];
         next[q] = kk[q] < a.nsave ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
+        if (!DENSE) break;
       }
     }
   }
@@ -289,24 +312,66 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
       prefetch_l2(c + 2 * n);
       prefetch_l2(hq2 - (int64_t)kPrefetchR * n);
     }
+    // dense save points inside step st: the interpolant's cotangent g reaches
+    // u_{st+1} now (H01 g + J(u_{st+1})^T (h H11 g)) and u_st after the
+    // transposed step (H00 g + J(u_st)^T (h H10 g)), with the matching
+    // parameter terms f_p^T (.)
+    V pgx, pgy, pgz, pnx, pny, pnz;
+    if (DENSE) {
+      pgx = vsplat<T, K>(cst<T>(0.0));
+      pgy = pgx, pgz = pgx, pnx = pgx, pny = pgx, pnz = pgx;
+    }
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      if (st + 1 == next[q]) {
+      while (st + 1 == next[q]) {
         const int64_t o = (int64_t)kk[q] * n3 + i[q];
+        T th = cst<T>(1.0);
+        HermiteW<T> w;
+        T ux = x.e[q], uy = y.e[q], uz = z.e[q], fsx, fsy, fsz, fnx, fny, fnz;
+        if (DENSE) {
+          th = a.theta[(int64_t)kk[q] * n + j0 + q];
+          if (th != cst<T>(1.0)) {
+            w = hermite_w(th);
+            lorenz_f(cx.e[q], cy.e[q], cz.e[q], s.e[q], r.e[q], b.e[q], fsx, fsy, fsz);
+            lorenz_f(ux, uy, uz, s.e[q], r.e[q], b.e[q], fnx, fny, fnz);
+            const T hh = hc.e[q];
+            ux = hermite_c(w, cx.e[q], x.e[q], fsx, fnx, hh);
+            uy = hermite_c(w, cy.e[q], y.e[q], fsy, fny, hh);
+            uz = hermite_c(w, cz.e[q], z.e[q], fsz, fnz, hh);
+          }
+        }
+        T gx, gy, gz;  // d loss_k / d u(t_k)
         if (a.loss_kind == GS_LOSS_SUMSQ) {
-          const T dx = a.target ? x.e[q] - a.target[o] : x.e[q];
-          const T dy = a.target ? y.e[q] - a.target[o + n] : y.e[q];
-          const T dz = a.target ? z.e[q] - a.target[o + 2 * n] : z.e[q];
-          lx.e[q] = fmaT(cst<T>(2.0), dx, lx.e[q]);
-          ly.e[q] = fmaT(cst<T>(2.0), dy, ly.e[q]);
-          lz.e[q] = fmaT(cst<T>(2.0), dz, lz.e[q]);
+          gx = cst<T>(2.0) * (a.target ? ux - a.target[o] : ux);
+          gy = cst<T>(2.0) * (a.target ? uy - a.target[o + n] : uy);
+          gz = cst<T>(2.0) * (a.target ? uz - a.target[o + 2 * n] : uz);
         } else {
-          lx.e[q] += a.weight[o];
-          ly.e[q] += a.weight[o + n];
-          lz.e[q] += a.weight[o + 2 * n];
+          gx = a.weight[o];
+          gy = a.weight[o + n];
+          gz = a.weight[o + 2 * n];
+        }
+        if (!DENSE || th == cst<T>(1.0)) {
+          lx.e[q] += gx;
+          ly.e[q] += gy;
+          lz.e[q] += gz;
+        } else {
+          const T hh = hc.e[q];
+          T mx, my, mz;
+          lorenz_vjp(x.e[q], y.e[q], z.e[q], s.e[q], r.e[q], b.e[q], (hh * w.h11) * gx, (hh * w.h11) * gy,
+                     (hh * w.h11) * gz, mx, my, mz, ps.e[q], pr.e[q], pb.e[q]);
+          lx.e[q] = fmaT(w.h01, gx, lx.e[q] + mx);
+          ly.e[q] = fmaT(w.h01, gy, ly.e[q] + my);
+          lz.e[q] = fmaT(w.h01, gz, lz.e[q] + mz);
+          pgx.e[q] = fmaT(w.h00, gx, pgx.e[q]);
+          pgy.e[q] = fmaT(w.h00, gy, pgy.e[q]);
+          pgz.e[q] = fmaT(w.h00, gz, pgz.e[q]);
+          pnx.e[q] = fmaT(hh * w.h10, gx, pnx.e[q]);
+          pny.e[q] = fmaT(hh * w.h10, gy, pny.e[q]);
+          pnz.e[q] = fmaT(hh * w.h10, gz, pnz.e[q]);
         }
         --kk[q];
         next[q] = kk[q] >= 0 ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
+        if (!DENSE) break;
       }
     }
     x = cx;
@@ -407,6 +472,13 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     lx += ((m1x + m2x) + (m3x + m4x)) + (m5x + m6x);
     ly += ((m1y + m2y) + (m3y + m4y)) + (m5y + m6y);
     lz += ((m1z + m2z) + (m3z + m4z)) + (m5z + m6z);
+    if (DENSE) {  // the interpolants' share of u_st
+      V qx, qy, qz;
+      lorenz_vjp(x, y, z, s, r, b, pnx, pny, pnz, qx, qy, qz, ps, pr, pb);
+      lx += pgx + qx;
+      ly += pgy + qy;
+      lz += pgz + qz;
+    }
   }
   // save points at step 0 cannot exist (save times lie in (t0, t1])
 #pragma unroll
@@ -446,11 +518,15 @@ gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const 
   a.dp = (T*)dp;
   a.du0 = (T*)du0;
   a.ck = (T*)ws;
+  a.theta = (const T*)M->save_theta;
   constexpr int K = GS_GRAD_K;
   const int bs = GS_GRAD_BS;
   const int64_t threads = (P->n + K - 1) / K;
   const int64_t grid = (threads + bs - 1) / bs;
-  k_grad_tsit5_lorenz<T, K><<<(unsigned)grid, bs, 0, st>>>(a);
+  if (a.theta)
+    k_grad_tsit5_lorenz<T, K, true><<<(unsigned)grid, bs, 0, st>>>(a);
+  else
+    k_grad_tsit5_lorenz<T, K, false><<<(unsigned)grid, bs, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

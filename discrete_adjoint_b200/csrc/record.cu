@@ -39,6 +39,8 @@ struct RecArgs {
   int32_t smax;
   T tsave[GS_MAX_SAVE];
   int64_t chunk;         // trajectories per warp (set by the launcher)
+  int32_t dense;         // 1: steps stop only at t1, save times located by theta (Tsit5)
+  T* theta;              // mesh mode, dense: [nsave][n] by trajectory
   T* h;                  // mesh mode: step s of trajectory i at h[i * hcol + s * hstep]
   int64_t hcol, hstep;
   int32_t* save_idx;     // mesh mode: [nsave][n] by trajectory
@@ -121,7 +123,7 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
   const int64_t n = a.n;
   const T eps = Eps<T>::v;
   const T q = METHOD == GS_TSIT5 ? cst<T>(5.0) : cst<T>(2.0);
-  const T tstop = r.kk < a.nsave ? a.tsave[r.kk] : a.t1;
+  const T tstop = (r.kk < a.nsave && !a.dense) ? a.tsave[r.kk] : a.t1;
   if (r.hprop < cst<T>(16.0) * eps * fabs(r.t)) {
     r.status = GS_TRAJ_DTMIN;
     return true;
@@ -159,13 +161,33 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
     }
     if (MODE == kRecMesh) a.h[r.i * a.hcol + (int64_t)r.nst * a.hstep] = h;
     ++r.nst;
+    const T tprev = r.t;
     r.t = clipped ? tstop : tn;
+    if (METHOD == GS_TSIT5 && a.dense) {
+      // every save time this step passed: its position inside the step, and
+      // (solve) the Hermite state there from u, f(u) = k1, u_new, f(u_new) = k7
+      while (r.kk < a.nsave && a.tsave[r.kk] <= r.t) {
+        const T th = (a.tsave[r.kk] - tprev) / h;
+        if (MODE == kRecMesh) {
+          a.save_idx[(int64_t)r.kk * n + r.i] = r.nst;
+          a.theta[(int64_t)r.kk * n + r.i] = th;
+        }
+        if (MODE == kRecSolve) {
+          const HermiteW<T> w = hermite_w(th);
+#pragma unroll
+          for (int c = 0; c < 3; ++c)
+            a.u_save[((int64_t)r.kk * 3 + c) * n + r.i] =
+                th == cst<T>(1.0) ? un[c] : hermite_c(w, r.u[c], un[c], r.k1[c], k7[c], h);
+        }
+        ++r.kk;
+      }
+    }
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
       r.u[c] = un[c];
       if (METHOD == GS_TSIT5) r.k1[c] = k7[c];
     }
-    while (r.kk < a.nsave && r.t == a.tsave[r.kk]) {
+    while (!a.dense && r.kk < a.nsave && r.t == a.tsave[r.kk]) {
       if (MODE == kRecMesh) a.save_idx[(int64_t)r.kk * n + r.i] = r.nst;
       if (MODE == kRecSolve) {
 #pragma unroll
@@ -199,7 +221,10 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T>& 
   const int64_t n = a.n;
   if (MODE == kRecMesh) {
     // unreached save points (a failed trajectory); the h tail stays unwritten
-    for (int k = r.kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + r.i] = 0;
+    for (int k = r.kk; k < a.nsave; ++k) {
+      a.save_idx[(int64_t)k * n + r.i] = 0;
+      if (a.dense) a.theta[(int64_t)k * n + r.i] = cst<T>(1.0);
+    }
   }
   if (MODE == kRecSolve && r.status != GS_TRAJ_OK) {
     // a failed trajectory has no solution: NaN at every save point
@@ -341,6 +366,7 @@ static RecArgs<T> rec_args(const gs_problem* P, const gs_tol* tol, int32_t smax)
   a.h0 = (T)tol->h0;
   a.nsave = P->nsave;
   a.smax = smax;
+  a.dense = tol->dense;
   for (int k = 0; k < P->nsave; ++k) a.tsave[k] = (T)P->tsave[k];
   return a;
 }
@@ -412,19 +438,20 @@ gs_status solve_adaptive3(const gs_problem* P, const gs_tol* tol, int32_t smax, 
 static size_t al256(size_t b) { return (b + 255) / 256 * 256; }
 
 // Workspace of gs_record: trajectory-order copies of nsteps, status, nreject,
-// save_idx and h, then the sort histogram.
+// save_idx, h and (dense records) the save-point positions, then the sort
+// histogram.
 size_t record_ws_bytes(int64_t n, int32_t smax, int32_t nsave, size_t tsize) {
   const int64_t nchunk = (n + kChunk - 1) / kChunk;
   return 3 * al256((size_t)n * 4) + al256((size_t)nsave * n * 4) + al256((size_t)smax * n * tsize) +
-         (size_t)(smax + 1) * (size_t)nchunk * 4;
+         al256((size_t)nsave * n * tsize) + (size_t)(smax + 1) * (size_t)nchunk * 4;
 }
 
 template <typename T>
 __global__ void k_gather_mesh(int64_t n, int smax, int nsave, const int32_t* __restrict__ order,
                               const T* __restrict__ h_tmp, const int32_t* __restrict__ si_tmp,
                               const int32_t* __restrict__ ns_tmp, const int32_t* __restrict__ st_tmp,
-                              const int32_t* __restrict__ nr_tmp, T* h, int32_t* save_idx, int32_t* nsteps,
-                              int32_t* status, int32_t* nreject) {
+                              const int32_t* __restrict__ nr_tmp, const T* __restrict__ th_tmp, T* h,
+                              int32_t* save_idx, int32_t* nsteps, int32_t* status, int32_t* nreject, T* theta) {
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n) return;
   const int64_t i = order[j];
@@ -433,6 +460,8 @@ __global__ void k_gather_mesh(int64_t n, int smax, int nsave, const int32_t* __r
   status[j] = st_tmp[i];
   nreject[j] = nr_tmp[i];
   for (int k = 0; k < nsave; ++k) save_idx[(int64_t)k * n + j] = si_tmp[(int64_t)k * n + i];
+  if (theta)
+    for (int k = 0; k < nsave; ++k) theta[(int64_t)k * n + j] = th_tmp[(int64_t)k * n + i];
   const T* src = h_tmp + i * smax;  // trajectory-major: a thread reads one row in order
   for (int s = 0; s < smax; ++s) h[(int64_t)s * n + j] = s < S ? src[s] : cst<T>(0.0);
 }
@@ -462,8 +491,11 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
   w += al256((size_t)P->nsave * n * 4);
   T* h_tmp = (T*)w;
   w += al256((size_t)M->smax * n * sizeof(T));
+  T* th_tmp = (T*)w;
+  w += al256((size_t)P->nsave * n * sizeof(T));
   int32_t* hist = (int32_t*)w;
   RecArgs<T> a = rec_args<T>(P, tol, M->smax);
+  a.theta = th_tmp;
   a.h = h_tmp;
   a.hcol = M->smax;  // trajectory-major workspace copy: each thread writes its own row
   a.hstep = 1;
@@ -475,9 +507,9 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
   if (rc != GS_OK) return rc;
   rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
   if (rc != GS_OK) return rc;
-  k_gather_mesh<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp,
-                                                                 st_tmp, nr_tmp, (T*)M->h, M->save_idx, M->nsteps,
-                                                                 M->status, M->nreject);
+  k_gather_mesh<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+      n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp, st_tmp, nr_tmp, th_tmp, (T*)M->h, M->save_idx,
+      M->nsteps, M->status, M->nreject, tol->dense ? (T*)M->save_theta : nullptr);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
@@ -511,8 +543,8 @@ gs_status record_node64(const gs_problem* P, const gs_tol* tol, const gs_mesh* M
   rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
   if (rc != GS_OK) return rc;
   k_gather_mesh<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp,
-                                                                 st_tmp, nr_tmp, (T*)M->h, M->save_idx, M->nsteps,
-                                                                 M->status, M->nreject);
+                                                                 st_tmp, nr_tmp, nullptr, (T*)M->h, M->save_idx,
+                                                                 M->nsteps, M->status, M->nreject, nullptr);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

@@ -18,7 +18,8 @@ struct SolveArgs {
   const int32_t* status;
   int32_t nsave;
   int32_t smax;
-  T* u_save;  // [nsave][3][n] by trajectory
+  const T* theta;  // [nsave][n] by slot: dense save points (Tsit5), or null
+  T* u_save;       // [nsave][3][n] by trajectory
 };
 
 template <typename T, int SYS, int METHOD>
@@ -53,6 +54,19 @@ __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
     if (METHOD == GS_TSIT5) {
       T k7[3], e[3];
       tsit5_err_step<T, SYS>(u, p, h, k1, un, k7, e);
+      if (a.theta) {
+        // dense save points inside this step: the Hermite state on u, f(u),
+        // u_new, f(u_new)
+        while (st + 1 == next) {
+          const T th = a.theta[(int64_t)kk * n + j];
+          const HermiteW<T> w = hermite_w(th);
+#pragma unroll
+          for (int c = 0; c < 3; ++c)
+            a.u_save[kk * n3 + c * n + i] = th == cst<T>(1.0) ? un[c] : hermite_c(w, u[c], un[c], k1[c], k7[c], h);
+          ++kk;
+          next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
+        }
+      }
 #pragma unroll
       for (int c = 0; c < 3; ++c) k1[c] = k7[c];
     } else {
@@ -84,6 +98,7 @@ gs_status launch_solve3(const gs_problem* P, const gs_mesh* M, void* u_save, cud
   a.status = M->status;
   a.nsave = P->nsave;
   a.smax = M->smax;
+  a.theta = P->method == GS_TSIT5 ? (const T*)M->save_theta : nullptr;
   a.u_save = (T*)u_save;
   const unsigned grid = (unsigned)((P->n + 127) / 128);
   if (P->system == GS_LORENZ && P->method == GS_TSIT5)

@@ -115,6 +115,32 @@ __device__ T ctrl_pow(T x, T y) {
   return ctrl_exp<T>(y * ctrl_ln<T>(x));
 }
 
+// Dense output inside one step [t_s, t_s + h] at theta in (0, 1]: the cubic
+// Hermite interpolant on the end states and slopes,
+//   u = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
+// weights and combination in the floating-point contract's order (the same
+// operations as the CPU reference, so the values agree bit for bit).
+template <typename T>
+struct HermiteW {
+  T h00, h01, h10, h11;
+};
+
+template <typename T>
+__device__ __forceinline__ HermiteW<T> hermite_w(T th) {
+  const T t2 = th * th, om = cst<T>(1.0) - th;
+  HermiteW<T> w;
+  w.h01 = t2 * fmaT(cst<T>(-2.0), th, cst<T>(3.0));
+  w.h00 = cst<T>(1.0) - w.h01;
+  w.h10 = (th * om) * om;
+  w.h11 = -(t2 * om);
+  return w;
+}
+
+template <typename T>
+__device__ __forceinline__ T hermite_c(const HermiteW<T>& w, T us, T un, T fs, T fn, T h) {
+  return fmaT(w.h00, us, fmaT(w.h01, un, h * fmaT(w.h10, fs, w.h11 * fn)));
+}
+
 template <typename T>
 __device__ __forceinline__ T rms3(const T x[3], const T sc[3]) {
   T s = cst<T>(0.0);

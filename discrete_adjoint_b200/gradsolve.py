@@ -49,13 +49,14 @@ class _Problem(ctypes.Structure):
 
 
 class _Tol(ctypes.Structure):
-    _fields_ = [("rtol", ctypes.c_double), ("atol", ctypes.c_double), ("h0", ctypes.c_double)]
+    _fields_ = [("rtol", ctypes.c_double), ("atol", ctypes.c_double), ("h0", ctypes.c_double),
+                ("dense", ctypes.c_int32)]
 
 
 class _Mesh(ctypes.Structure):
     _fields_ = [("smax", ctypes.c_int32), ("nsave", ctypes.c_int32), ("h", ctypes.c_void_p),
                 ("order", ctypes.c_void_p), ("nsteps", ctypes.c_void_p), ("save_idx", ctypes.c_void_p),
-                ("status", ctypes.c_void_p), ("nreject", ctypes.c_void_p)]
+                ("status", ctypes.c_void_p), ("nreject", ctypes.c_void_p), ("save_theta", ctypes.c_void_p)]
 
 
 class _Loss(ctypes.Structure):
@@ -163,6 +164,7 @@ class Mesh:
     save_idx: torch.Tensor  # [nsave][n] int32
     status: torch.Tensor    # [n] int32
     nreject: torch.Tensor   # [n] int32
+    save_theta: torch.Tensor | None = None  # [nsave][n] dtype: dense record (position inside the step)
 
     @property
     def smax(self) -> int:
@@ -174,14 +176,18 @@ class Mesh:
 
     def _struct(self):
         return _Mesh(self.smax, self.nsave, self.h.data_ptr(), self.order.data_ptr(), self.nsteps.data_ptr(),
-                     self.save_idx.data_ptr(), self.status.data_ptr(), self.nreject.data_ptr())
+                     self.save_idx.data_ptr(), self.status.data_ptr(), self.nreject.data_ptr(),
+                     None if self.save_theta is None else self.save_theta.data_ptr())
 
 
-def new_mesh(n: int, smax: int, nsave: int, dtype: str, device="cuda") -> Mesh:
-    """Allocate (caller-side, via torch) an empty mesh of capacity smax."""
+def new_mesh(n: int, smax: int, nsave: int, dtype: str, device="cuda", dense: bool = False) -> Mesh:
+    """Allocate (caller-side, via torch) an empty mesh of capacity smax; dense
+    adds the save-point positions a dense record writes."""
     i32 = dict(dtype=torch.int32, device=device)
-    return Mesh(torch.zeros((smax, n), dtype=TORCH_DTYPE[dtype], device=device), torch.zeros(n, **i32),
-                torch.zeros(n, **i32), torch.zeros((nsave, n), **i32), torch.zeros(n, **i32), torch.zeros(n, **i32))
+    td = TORCH_DTYPE[dtype]
+    return Mesh(torch.zeros((smax, n), dtype=td, device=device), torch.zeros(n, **i32),
+                torch.zeros(n, **i32), torch.zeros((nsave, n), **i32), torch.zeros(n, **i32), torch.zeros(n, **i32),
+                torch.ones((nsave, n), dtype=td, device=device) if dense else None)
 
 
 def gs_workspace_bytes(ens: Ensemble, mesh: Mesh | None, op: int, smax: int | None = None) -> int:
@@ -189,7 +195,7 @@ def gs_workspace_bytes(ens: Ensemble, mesh: Mesh | None, op: int, smax: int | No
     if mesh is not None:
         ms = mesh._struct()
     else:
-        ms = _Mesh(smax, len(ens.tsave), None, None, None, None, None, None)
+        ms = _Mesh(smax, len(ens.tsave), None, None, None, None, None, None, None)
     return int(_lib.gs_workspace_bytes(ctypes.byref(ps), ctypes.byref(ms), op))
 
 
@@ -204,21 +210,21 @@ def _check(rc: int, what: str):
 
 
 def gs_count(ens: Ensemble, rtol: float, atol: float, smax: int, h0: float = 0.0, nsteps=None, status=None,
-             stream=None):
+             stream=None, dense: bool = False):
     """Step counts and statuses per TRAJECTORY (sizing pass)."""
     dev = ens.u0.device
     if nsteps is None:
         nsteps = torch.empty(ens.n, dtype=torch.int32, device=dev)
     if status is None:
         status = torch.empty(ens.n, dtype=torch.int32, device=dev)
-    ps, tol = ens._struct(), _Tol(rtol, atol, h0)
+    ps, tol = ens._struct(), _Tol(rtol, atol, h0, int(dense))
     _check(_lib.gs_count(ctypes.byref(ps), ctypes.byref(tol), smax, _ptr(nsteps), _ptr(status), _stream(stream)),
            "gs_count")
     return nsteps, status
 
 
 def gs_solve_adaptive(ens: Ensemble, rtol: float, atol: float, smax: int, h0: float = 0.0, u_save=None,
-                      nsteps=None, status=None, stream=None):
+                      nsteps=None, status=None, stream=None, dense: bool = False):
     """Adaptive forward-only solve: (u_save [nsave][d][n], nsteps [n], status [n]),
     all by trajectory; no mesh is kept."""
     dev = ens.u0.device
@@ -228,14 +234,18 @@ def gs_solve_adaptive(ens: Ensemble, rtol: float, atol: float, smax: int, h0: fl
         nsteps = torch.empty(ens.n, dtype=torch.int32, device=dev)
     if status is None:
         status = torch.empty(ens.n, dtype=torch.int32, device=dev)
-    ps, tol = ens._struct(), _Tol(rtol, atol, h0)
+    ps, tol = ens._struct(), _Tol(rtol, atol, h0, int(dense))
     _check(_lib.gs_solve_adaptive(ctypes.byref(ps), ctypes.byref(tol), smax, _ptr(u_save), _ptr(nsteps),
                                   _ptr(status), _stream(stream)), "gs_solve_adaptive")
     return u_save, nsteps, status
 
 
-def gs_record(ens: Ensemble, mesh: Mesh, rtol: float, atol: float, h0: float = 0.0, ws=None, stream=None):
-    ps, ms, tol = ens._struct(), mesh._struct(), _Tol(rtol, atol, h0)
+def gs_record(ens: Ensemble, mesh: Mesh, rtol: float, atol: float, h0: float = 0.0, ws=None, stream=None,
+              dense: bool | None = None):
+    """Adaptive record into mesh; dense (default: whether the mesh carries
+    save_theta) records steps that do not stop at the save times."""
+    dense = mesh.save_theta is not None if dense is None else dense
+    ps, ms, tol = ens._struct(), mesh._struct(), _Tol(rtol, atol, h0, int(dense))
     need = int(_lib.gs_workspace_bytes(ctypes.byref(ps), ctypes.byref(ms), OP_RECORD))
     if ws is None:
         ws = workspace(need, ens.u0.device)

@@ -93,7 +93,8 @@ typedef int32_t gs_status;
  *           r*64 + c), shared by all trajectories; NULL otherwise.
  *   t0, t1  time span, t0 < t1.
  *   tsave   host, nsave (1..GS_MAX_SAVE) strictly increasing times in (t0, t1]:
- *           the save points of gs_solve and of the loss.  Steps land on them.
+ *           the save points of gs_solve and of the loss.  Steps land on them,
+ *           unless the record is dense (gs_tol.dense).
  */
 typedef struct gs_problem {
   int32_t system, method, dtype, d, np;
@@ -108,9 +109,20 @@ typedef struct gs_problem {
 
 /* Step-size control: accept iff the RMS of e_c / (atol + rtol max(|u_c|, |u'_c|))
  * is <= 1.  h0 > 0 fixes the first proposal; h0 = 0 picks it automatically
- * (Hairer, Norsett & Wanner I, II.4). */
+ * (Hairer, Norsett & Wanner I, II.4).
+ * dense = 0: steps are shortened to land on every save time.  dense = 1 (Tsit5,
+ * d = 3 only): steps stop only at t1; a save time inside a step is located by
+ * its position theta in (0, 1] (gs_mesh.save_theta) and the state there is the
+ * cubic Hermite interpolant of the step on its end states and slopes,
+ *   u = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
+ *   H01 = theta^2 (3 - 2 theta), H00 = 1 - H01, H10 = theta (1 - theta)^2,
+ *   H11 = -theta^2 (1 - theta).
+ * The loss and its derivative then pass through that interpolant (theta, like
+ * h, is data).  The survey's dense-output save points; the pages print no
+ * interpolant, so this one is this library's reading. */
 typedef struct gs_tol {
   double rtol, atol, h0;
+  int32_t dense;
 } gs_tol;
 
 /*
@@ -129,6 +141,10 @@ typedef struct gs_tol {
  *             (1..nsteps[j]).
  *   status    [n] int32, GS_TRAJ_* of slot j.
  *   nreject   [n] int32, rejected attempts of slot j (diagnostic).
+ *   save_theta [nsave][n] dtype, or NULL: for a dense record, the position of
+ *             save time k inside step save_idx - 1, in (0, 1]; NULL means the
+ *             save points are step ends (theta = 1).  gs_record writes it when
+ *             gs_tol.dense is set (and then requires it).
  */
 typedef struct gs_mesh {
   int32_t smax, nsave;
@@ -138,6 +154,7 @@ typedef struct gs_mesh {
   int32_t* save_idx;
   int32_t* status;
   int32_t* nreject;
+  void* save_theta;
 } gs_mesh;
 
 /* Loss description.  target / weight: device, [nsave][d][n] dtype, indexed by

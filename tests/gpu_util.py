@@ -38,8 +38,9 @@ def mesh_from_oracle(om, dtype, order=None, smax=None):
     h[: om.h.shape[1]] = om.h[order].T[:smax]
     td = gs.gradsolve.TORCH_DTYPE[dtype]
     i32 = lambda a: tens(np.asarray(a, np.int32), torch.int32)
+    theta = None if om.theta is None else tens(om.theta[order].T, td)
     return gs.Mesh(tens(h, td), i32(order), i32(om.nsteps[order]), i32(om.save_idx[order].T),
-                   i32(om.status[order]), i32(om.nreject[order]))
+                   i32(om.status[order]), i32(om.nreject[order]), theta)
 
 
 def mesh_by_trajectory(mesh):
@@ -49,6 +50,14 @@ def mesh_by_trajectory(mesh):
     inv[order] = np.arange(len(order))
     h = mesh.h.double().cpu().numpy().T[inv]
     return h, mesh.nsteps.cpu().numpy()[inv], mesh.save_idx.cpu().numpy().T[inv], mesh.status.cpu().numpy()[inv], order
+
+
+def theta_by_trajectory(mesh):
+    """save_theta [n][nsave] in trajectory order (a dense record)."""
+    order = mesh.order.cpu().numpy()
+    inv = np.empty_like(order)
+    inv[order] = np.arange(len(order))
+    return mesh.save_theta.double().cpu().numpy().T[inv]
 
 
 def grad_rel_err(out, ref):
