@@ -33,6 +33,7 @@ gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, fl
 gs_status node64_grad(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*, void*,
                       cudaStream_t);
 gs_status node64_solve(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
+void node64_set_tensor(int on);
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize);
 
 static size_t dsize(const gs_problem* P) { return P->dtype == GS_F64 ? 8 : 4; }
@@ -91,6 +92,14 @@ static gs_status check_tol(const gs_problem* P, const gs_tol* tol) {
 using namespace gs;
 
 extern "C" {
+
+gs_status gs_set_option(int32_t option, int32_t value) {
+  if (option == GS_OPT_NODE64_TENSOR_CORES && (value == 0 || value == 1)) {
+    node64_set_tensor(value);
+    return GS_OK;
+  }
+  return GS_EINVAL;
+}
 
 const char* gs_status_string(gs_status s) {
   switch (s) {

@@ -21,6 +21,8 @@
 //                 a fixed order so the weight gradient is deterministic)
 // The per-trajectory parts of the recorder (error norm as the contract's
 // sequential sum over components, the PI controller) run one thread per slot.
+#include <atomic>
+
 #include "steps.cuh"
 
 namespace gs {
@@ -483,15 +485,15 @@ struct GradArgs64 {
   T* dp;
   T* du0;
   T* ck;       // workspace [smax][64][n] by slot
-  T* dW_part;  // workspace [gridDim][64][64]
+  T* dW_part;  // workspace [parts][64][64]: one per CTA (two with the tensor-core products)
   T* u_save;   // solve: [nsave][64][n] by trajectory
 };
 
 // Loss of the save point each flagged slot has reached: the terms of the
 // thread's rows go to red (and G for a linear loss), then the slot's thread
 // sums them in the contract's order (components 0..63, fma chain).
-template <typename T>
-__device__ __forceinline__ void save_point_loss(Smem<T>& s, const GradArgs64<T>& a, const Blk<T>& u,
+template <typename T, typename SM>
+__device__ __forceinline__ void save_point_loss(SM& s, const GradArgs64<T>& a, const Blk<T>& u,
                                                 const int64_t (&o)[2], const bool (&hit)[2], T& Lslot, int ty,
                                                 int tx, int tid) {
   __syncthreads();
@@ -818,12 +820,635 @@ __global__ void k_reduce_dW(const T* part, int nblk, T* dW) {
   dW[e] = acc;
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core products for the d = 64 replay and gradient (tcgen05, sm_100a).
+//
+// The three products of a stage -- Z = W U, W^T G and dW += G U^T over the
+// CTA's 32 slots -- run as tcgen05 MMAs of kind tf32 with a 3xTF32 split
+// (x = hi + lo, both rounded to TF32; A B ~ hi hi + hi lo + lo hi), which keeps
+// fp32 accuracy (measured: 5.6e-7 relative against a float64 product).
+//   Z, W^T G : M = 64 (components), N = 16 (a group's slots), K = 64, fp32
+//              accumulator in TMEM
+//   dW       : M = 64, N = 64, K = 16 (slots), accumulated in TMEM over the
+//              whole reverse sweep, read out once per group
+// Operands sit in shared memory as K-major tiles of 8-row x 16-byte core
+// matrices (row groups 128 B apart, 4-column chunks one tile-height of groups
+// apart), no swizzle.  TF32 operands cannot be MN-major here, so G and U are
+// written twice: by slot (the N operand of W^T G and of Z) and by component
+// (the operands of dW).  An M = 64 accumulator holds row m in TMEM lane
+// (m / 16) * 32 + m % 16; warps 0..3 read their lane quadrant and stage the
+// product through shared memory into the threads' 4 x 2 register blocks.
+// One thread issues the MMAs and commits them to an mbarrier; every wait is
+// bounded, and a CTA whose MMAs do not complete marks itself failed, skips
+// the remaining products, writes NaN results and still frees its TMEM.
+// ---------------------------------------------------------------------------
+namespace tc {
+
+constexpr int kSpin = 1 << 22;  // mbarrier polls before a CTA gives up
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ float tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// byte offset of element (row r, column k) in a tile of R rows
+__device__ __forceinline__ uint32_t off(int r, int k, int R) {
+  return (uint32_t)(((k >> 2) * (R >> 3) + (r >> 3)) * 128 + (r & 7) * 16 + (k & 3) * 4);
+}
+
+__device__ __forceinline__ void put(float* hi, float* lo, uint32_t o, float x) {
+  const float h = tf32_rna(x);
+  *(float*)((char*)hi + o) = h;
+  *(float*)((char*)lo + o) = tf32_rna(x - h);
+}
+
+// shared-memory matrix descriptor: start, leading (K chunk) and stride (row
+// group) byte offsets, descriptor version 1, no swizzle
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46);
+}
+
+// instruction descriptor: fp32 accumulate, tf32 A and B, both K-major
+__host__ __device__ constexpr uint32_t idesc(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
+      :
+      : "r"(d), "l"(a), "l"(b), "r"(id), "r"(acc));
+}
+
+// 3xTF32 product over nk K-steps of 8: D (+)= A B^T with A, B K-major tiles of
+// chunk strides ca, cb (bytes); acc0 = 0 overwrites D with the first MMA.
+__device__ __forceinline__ void mma3(uint32_t d, uint32_t ahi, uint32_t alo, uint32_t ca, uint32_t bhi, uint32_t blo,
+                                     uint32_t cb, int nk, uint32_t id, uint32_t acc0) {
+  for (int st = 0; st < nk; ++st) {
+    const uint32_t oa = 2 * st * ca, ob = 2 * st * cb;
+    mma(d, sdesc(ahi + oa, ca, 128), sdesc(blo + ob, cb, 128), id, st > 0 ? 1u : acc0);
+    mma(d, sdesc(alo + oa, ca, 128), sdesc(bhi + ob, cb, 128), id, 1u);
+    mma(d, sdesc(ahi + oa, ca, 128), sdesc(bhi + ob, cb, 128), id, 1u);
+  }
+}
+
+__device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(r[c]);
+}
+
+}  // namespace tc
+
+// The CTA's 32 slots form two groups of 16, one per half of the CTA (warps
+// 0..3 and 4..7), each with its own operand tiles, accumulators, mbarrier and
+// named barrier: the groups step independently, so one group's element-wise
+// work overlaps the other's MMAs and waits.
+constexpr int GS = 16;        // slots per group
+constexpr int GT = NT / 2;    // threads per group
+
+struct GroupTC {
+  float Thi[GS * D], Tlo[GS * D];    // U or G by slot: rows t, K = component
+  float GChi[D * GS], GClo[D * GS];  // G by component: rows c, K = slot
+  float UEhi[D * GS], UElo[D * GS];  // U by component: rows e, K = slot
+  float Z[D][GS];    // product staging [component][slot]
+  float red[D][GS];  // per-slot loss terms
+  float G[D][GS];    // second loss operand (linear loss)
+  unsigned long long bar;  // MMA completion
+  int failed;              // an MMA wait ran out
+  int flag[GS];
+  int pad[13];
+};
+
+struct SmemTC {
+  float Whi[D * D], Wlo[D * D];    // W, rows n, K = k
+  float WThi[D * D], WTlo[D * D];  // W^T, rows c, K = k (element (c, k) = W[k][c])
+  GroupTC grp[2];
+  uint32_t tmem;  // TMEM base (256 columns): group g uses [16g, 16g + 16) and [32 + 64g, 96 + 64g)
+};
+
+__device__ __forceinline__ void gbar(int g) { asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(GT) : "memory"); }
+
+// Wait for the group's last commit (bounded); the phase bit alternates per commit.
+__device__ __forceinline__ void tc_wait(GroupTC& q, uint32_t& phase) {
+  if (!q.failed) {
+    uint32_t done = 0;
+    for (int it = 0; it < tc::kSpin && !done; ++it)
+      asm volatile(
+          "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+          "selp.b32 %0, 1, 0, P1;\n\t}\n"
+          : "=r"(done)
+          : "r"(tc::smem_u32(&q.bar)), "r"(phase)
+          : "memory");
+    if (!done) q.failed = 1;
+  }
+  phase ^= 1u;
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(GroupTC& q) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   tc::smem_u32(&q.bar))
+               : "memory");
+}
+
+// Operands written by the group's threads are visible to its MMAs.
+__device__ __forceinline__ void tc_publish(int g) {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  gbar(g);
+}
+
+__device__ __forceinline__ void ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]);
+}
+
+// The group's M = 64, N = 16 accumulator into q.Z: warp 4g + w reads lane
+// quadrant w, whose lanes 0..15 hold rows 16w..16w+15.
+__device__ __forceinline__ void tc_stage_out(const SmemTC& s, GroupTC& q, int g, int tg) {
+  const int w = tg >> 5, lane = tg & 31;
+  if (!q.failed) {
+    float v[16];
+    ld16(s.tmem + ((uint32_t)(32 * w) << 16) + (uint32_t)(16 * g), v);
+    if (lane < 16)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) q.Z[16 * w + lane][c] = v[c];
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  gbar(g);
+}
+
+// f(U) for the group on the tensor cores: y = tanh(b + W U), k = y - U.
+__device__ __forceinline__ void eval_f_tc(SmemTC& s, GroupTC& q, uint32_t& phase, const Blk<float>& U,
+                                          const Blk<float>& bias, Blk<float>& y, Blk<float>& k, int ty, int tx, int g,
+                                          int tg) {
+  gbar(g);  // previous readers of T and Z are done
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) tc::put(q.Thi, q.Tlo, tc::off(2 * tx + c, 4 * ty + a, GS), U.v[a][c]);
+  tc_publish(g);
+  if (tg == 0 && !q.failed) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    tc::mma3(s.tmem + 16 * g, tc::smem_u32(s.Whi), tc::smem_u32(s.Wlo), 1024, tc::smem_u32(q.Thi),
+             tc::smem_u32(q.Tlo), 256, 8, tc::idesc(64, 16), 0u);
+    tc_commit(q);
+  }
+  tc_wait(q, phase);
+  tc_stage_out(s, q, g, tg);
+  Blk<float> z;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) z.v[a][c] = bias.v[a][c] + q.Z[4 * ty + a][2 * tx + c];
+  rhs_tail(z, U, y, k);
+}
+
+__device__ __forceinline__ void tsit5_stages_tc(SmemTC& s, GroupTC& q, uint32_t& phase, const Blk<float>& u,
+                                                const Blk<float>& bias, const float (&h)[2], const Blk<float>& k1,
+                                                Blk<float>& k2, Blk<float>& k3, Blk<float>& k4, Blk<float>& k5,
+                                                Blk<float>& k6, Blk<float>& k7, Blk<float>& un, int ty, int tx, int g,
+                                                int tg) {
+  using T = float;
+  Blk<T> y, U;
+  {
+    const T c[1] = {cst<T>(TS_A21)};
+    const Blk<T>* const ks[1] = {&k1};
+    U = stage<T, 1>(c, ks, u, h);
+    eval_f_tc(s, q, phase, U, bias, y, k2, ty, tx, g, tg);
+  }
+  {
+    const T c[2] = {cst<T>(TS_A31), cst<T>(TS_A32)};
+    const Blk<T>* const ks[2] = {&k1, &k2};
+    U = stage<T, 2>(c, ks, u, h);
+    eval_f_tc(s, q, phase, U, bias, y, k3, ty, tx, g, tg);
+  }
+  {
+    const T c[3] = {cst<T>(TS_A41), cst<T>(TS_A42), cst<T>(TS_A43)};
+    const Blk<T>* const ks[3] = {&k1, &k2, &k3};
+    U = stage<T, 3>(c, ks, u, h);
+    eval_f_tc(s, q, phase, U, bias, y, k4, ty, tx, g, tg);
+  }
+  {
+    const T c[4] = {cst<T>(TS_A51), cst<T>(TS_A52), cst<T>(TS_A53), cst<T>(TS_A54)};
+    const Blk<T>* const ks[4] = {&k1, &k2, &k3, &k4};
+    U = stage<T, 4>(c, ks, u, h);
+    eval_f_tc(s, q, phase, U, bias, y, k5, ty, tx, g, tg);
+  }
+  {
+    const T c[5] = {cst<T>(TS_A61), cst<T>(TS_A62), cst<T>(TS_A63), cst<T>(TS_A64), cst<T>(TS_A65)};
+    const Blk<T>* const ks[5] = {&k1, &k2, &k3, &k4, &k5};
+    U = stage<T, 5>(c, ks, u, h);
+    eval_f_tc(s, q, phase, U, bias, y, k6, ty, tx, g, tg);
+  }
+  {
+    const T c[6] = {cst<T>(TS_B1), cst<T>(TS_B2), cst<T>(TS_B3), cst<T>(TS_B4), cst<T>(TS_B5), cst<T>(TS_B6)};
+    const Blk<T>* const ks[6] = {&k1, &k2, &k3, &k4, &k5, &k6};
+    un = stage<T, 6>(c, ks, u, h);
+    eval_f_tc(s, q, phase, un, bias, y, k7, ty, tx, g, tg);
+  }
+}
+
+// Loss terms of the save points the group's flagged slots reached (the
+// contract's order: components 0..63, an fma chain by the slot's thread).
+__device__ __forceinline__ void save_point_loss_tc(GroupTC& q, const GradArgs64<float>& a, const Blk<float>& u,
+                                                   const int64_t (&o)[2], const bool (&hit)[2], float& Lslot, int ty,
+                                                   int tx, int g, int tg) {
+  gbar(g);
+  if (tg < GS) q.flag[tg] = 0;
+  gbar(g);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    if (!hit[c]) continue;
+    if (ty == 0) q.flag[2 * tx + c] = 1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = 4 * ty + k;
+      const int64_t oo = o[c] + (int64_t)r * a.n;
+      if (a.loss_kind == GS_LOSS_SUMSQ) {
+        q.red[r][2 * tx + c] = a.target ? u.v[k][c] - a.target[oo] : u.v[k][c];
+      } else {
+        q.red[r][2 * tx + c] = a.weight[oo];
+        q.G[r][2 * tx + c] = u.v[k][c];
+      }
+    }
+  }
+  gbar(g);
+  if (tg < GS && q.flag[tg]) {
+    float L = Lslot;
+    for (int r = 0; r < D; ++r)
+      L = a.loss_kind == GS_LOSS_SUMSQ ? fmaT(q.red[r][tg], q.red[r][tg], L) : fmaT(q.red[r][tg], q.G[r][tg], L);
+    Lslot = L;
+  }
+}
+
+// The replay (solve) and the fused replay + reverse sweep with the products on
+// the tensor cores; same slots, save points, loss and outputs as
+// k_replay_node64 (dW partials: one per group, two per CTA).
+template <bool GRAD>
+__global__ void __launch_bounds__(NT, 1) k_replay_node64_tc(GradArgs64<float> a) {
+  using T = float;
+  extern __shared__ __align__(128) unsigned char smem_raw_tc[];
+  SmemTC& s = *reinterpret_cast<SmemTC*>(smem_raw_tc);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int g = tid / GT, tg = tid % GT, ty = tg / 8, tx = tg % 8;
+  GroupTC& q = s.grp[g];
+  const int64_t n = a.n;
+  const int64_t base = (int64_t)blockIdx.x * TB + GS * g;  // the group's first slot
+  const int64_t n64 = (int64_t)D * n;
+  const T nan = cst<T>(__int_as_float(0x7fc00000));
+  for (int e = tid; e < D * D; e += NT) {
+    const int r = e / D, c = e % D;
+    const T w = a.W[e];  // W[r][c]
+    tc::put(s.Whi, s.Wlo, tc::off(r, c, D), w);
+    tc::put(s.WThi, s.WTlo, tc::off(c, r, D), w);
+  }
+  if (tg == 0) {
+    q.failed = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc::smem_u32(&q.bar)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(tc::smem_u32(&s.tmem)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  uint32_t phase = 0;
+
+  int64_t traj[2];
+  int S[2];
+  bool act[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int64_t j = base + 2 * tx + c;
+    traj[c] = -1;
+    S[c] = 0;
+    act[c] = false;
+    if (j < n) {
+      const int64_t i = a.order[j];
+      if (i >= 0 && i < n) {
+        traj[c] = i;
+        const int sq = a.nsteps[j];
+        if (a.status[j] == GS_TRAJ_OK && sq >= 0 && sq <= a.smax) {
+          S[c] = sq;
+          act[c] = true;
+        }
+      }
+    }
+  }
+  if (tg < GS) q.flag[tg] = 0;
+  gbar(g);
+  if (ty == 0) {
+    q.flag[2 * tx] = S[0];
+    q.flag[2 * tx + 1] = S[1];
+  }
+  gbar(g);
+  int Smax = 0;
+  for (int k = 0; k < GS; ++k) Smax = q.flag[k] > Smax ? q.flag[k] : Smax;
+  T Lslot = cst<T>(0.0);
+
+  Blk<T> u, bias;
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = 4 * ty + k;
+      u.v[k][c] = act[c] ? a.u0[(int64_t)r * n + traj[c]] : cst<T>(0.0);
+      bias.v[k][c] = act[c] ? a.p[(int64_t)r * n + traj[c]] : cst<T>(0.0);
+    }
+  int kk[2] = {0, 0}, next[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) next[c] = act[c] && S[c] > 0 ? a.save_idx[base + 2 * tx + c] : -1;
+
+  // ---------------------------------------------------------------- forward
+  {
+    Blk<T> y, k1, k2, k3, k4, k5, k6, k7, un;
+    eval_f_tc(s, q, phase, u, bias, y, k1, ty, tx, g, tg);
+    for (int st = 0; st < Smax; ++st) {
+      T hh[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        hh[c] = st < S[c] ? a.h[(int64_t)st * n + base + 2 * tx + c] : cst<T>(0.0);
+        if (GRAD && st < S[c]) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            a.ck[(int64_t)st * n64 + (int64_t)(4 * ty + k) * n + base + 2 * tx + c] = u.v[k][c];
+        }
+      }
+      tsit5_stages_tc(s, q, phase, u, bias, hh, k1, k2, k3, k4, k5, k6, k7, un, ty, tx, g, tg);
+      u = un;
+      k1 = k7;
+      bool hit[2];
+      int64_t o[2];
+      int anyhit = 0;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        hit[c] = st + 1 == next[c];
+        o[c] = hit[c] ? (int64_t)kk[c] * n64 + traj[c] : 0;
+        anyhit |= hit[c];
+        if (hit[c]) {
+          if (!GRAD) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) a.u_save[o[c] + (int64_t)(4 * ty + k) * n] = u.v[k][c];
+          }
+          ++kk[c];
+          next[c] = kk[c] < a.nsave ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
+        }
+      }
+      if (GRAD) {
+        // the group's threads agree on whether any of its slots hit a save point
+        gbar(g);
+        if (tg < GS) q.flag[tg] = 0;
+        gbar(g);
+        if (anyhit) q.flag[0] = 1;
+        gbar(g);
+        if (q.flag[0]) save_point_loss_tc(q, a, u, o, hit, Lslot, ty, tx, g, tg);
+      }
+    }
+  }
+  bool dw_started = false;
+  Blk<T> lam = bzero<T>(), bbar = bzero<T>();
+  if (GRAD) {
+    if (tg < GS) {
+      const int64_t j = base + tg;
+      if (j < n) {
+        const int64_t i = a.order[j];
+        if (i >= 0 && i < n) {
+          const bool ok = a.status[j] == GS_TRAJ_OK && a.nsteps[j] >= 0 && a.nsteps[j] <= a.smax;
+          a.loss[i] = ok ? Lslot : nan;
+        }
+      }
+    }
+    // ---------------------------------------------------------------- reverse
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      kk[c] = a.nsave - 1;
+      next[c] = act[c] && S[c] > 0 ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
+    }
+    for (int st = Smax - 1; st >= 0; --st) {
+      T hh[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (st + 1 == next[c]) {
+          const int64_t o = (int64_t)kk[c] * n64 + traj[c];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int64_t oo = o + (int64_t)(4 * ty + k) * n;
+            if (a.loss_kind == GS_LOSS_SUMSQ)
+              lam.v[k][c] = fmaT(cst<T>(2.0), a.target ? u.v[k][c] - a.target[oo] : u.v[k][c], lam.v[k][c]);
+            else
+              lam.v[k][c] += a.weight[oo];
+          }
+          --kk[c];
+          next[c] = kk[c] >= 0 ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
+        }
+        const bool run = st < S[c];
+        hh[c] = run ? a.h[(int64_t)st * n + base + 2 * tx + c] : cst<T>(0.0);
+        if (run) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            u.v[k][c] = a.ck[(int64_t)st * n64 + (int64_t)(4 * ty + k) * n + base + 2 * tx + c];
+        }
+      }
+      Blk<T> U1 = u, U2, U3, U4, U5, U6, y1, y2, y3, y4, y5, y6, kd;
+      eval_f_tc(s, q, phase, U1, bias, y1, kd, ty, tx, g, tg);
+      Blk<T> k1 = kd;
+      {
+        const T c[1] = {cst<T>(TS_A21)};
+        const Blk<T>* const ks[1] = {&k1};
+        U2 = stage<T, 1>(c, ks, U1, hh);
+      }
+      eval_f_tc(s, q, phase, U2, bias, y2, kd, ty, tx, g, tg);
+      Blk<T> k2 = kd;
+      {
+        const T c[2] = {cst<T>(TS_A31), cst<T>(TS_A32)};
+        const Blk<T>* const ks[2] = {&k1, &k2};
+        U3 = stage<T, 2>(c, ks, U1, hh);
+      }
+      eval_f_tc(s, q, phase, U3, bias, y3, kd, ty, tx, g, tg);
+      Blk<T> k3 = kd;
+      {
+        const T c[3] = {cst<T>(TS_A41), cst<T>(TS_A42), cst<T>(TS_A43)};
+        const Blk<T>* const ks[3] = {&k1, &k2, &k3};
+        U4 = stage<T, 3>(c, ks, U1, hh);
+      }
+      eval_f_tc(s, q, phase, U4, bias, y4, kd, ty, tx, g, tg);
+      Blk<T> k4 = kd;
+      {
+        const T c[4] = {cst<T>(TS_A51), cst<T>(TS_A52), cst<T>(TS_A53), cst<T>(TS_A54)};
+        const Blk<T>* const ks[4] = {&k1, &k2, &k3, &k4};
+        U5 = stage<T, 4>(c, ks, U1, hh);
+      }
+      eval_f_tc(s, q, phase, U5, bias, y5, kd, ty, tx, g, tg);
+      Blk<T> k5 = kd;
+      {
+        const T c[5] = {cst<T>(TS_A61), cst<T>(TS_A62), cst<T>(TS_A63), cst<T>(TS_A64), cst<T>(TS_A65)};
+        const Blk<T>* const ks[5] = {&k1, &k2, &k3, &k4, &k5};
+        U6 = stage<T, 5>(c, ks, U1, hh);
+      }
+      eval_f_tc(s, q, phase, U6, bias, y6, kd, ty, tx, g, tg);
+
+      Blk<T> mu[6];
+      const Blk<T>* Ys[6] = {&y1, &y2, &y3, &y4, &y5, &y6};
+      const Blk<T>* Us[6] = {&U1, &U2, &U3, &U4, &U5, &U6};
+      const double bw[6] = {TS_B1, TS_B2, TS_B3, TS_B4, TS_B5, TS_B6};
+      const double aw[6][6] = {{0, 0, 0, 0, 0, 0},
+                               {TS_A21, 0, 0, 0, 0, 0},
+                               {TS_A31, TS_A32, 0, 0, 0, 0},
+                               {TS_A41, TS_A42, TS_A43, 0, 0, 0},
+                               {TS_A51, TS_A52, TS_A53, TS_A54, 0, 0},
+                               {TS_A61, TS_A62, TS_A63, TS_A64, TS_A65, 0}};
+#pragma unroll
+      for (int jj = 5; jj >= 0; --jj) {
+        Blk<T> nu, gg;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            T acc = cst<T>(bw[jj]) * lam.v[k][c];
+#pragma unroll
+            for (int m = 5; m > jj; --m) acc = fmaT(cst<T>(aw[m][jj]), mu[m].v[k][c], acc);
+            nu.v[k][c] = hh[c] * acc;
+            const T yv = Ys[jj]->v[k][c];
+            gg.v[k][c] = nu.v[k][c] * fmaT(-yv, yv, cst<T>(1.0));
+            bbar.v[k][c] += gg.v[k][c];
+          }
+        gbar(g);  // previous readers of the operand tiles and of Z are done
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int r = 4 * ty + k, t = 2 * tx + c;
+            tc::put(q.Thi, q.Tlo, tc::off(t, r, GS), gg.v[k][c]);
+            tc::put(q.GChi, q.GClo, tc::off(r, t, D), gg.v[k][c]);
+            tc::put(q.UEhi, q.UElo, tc::off(r, t, D), Us[jj]->v[k][c]);
+          }
+        tc_publish(g);
+        if (tg == 0 && !q.failed) {
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          // W^T g (M = 64, N = 16) and dW += G U^T (M = 64, N = 64, K = 16 slots)
+          tc::mma3(s.tmem + 16 * g, tc::smem_u32(s.WThi), tc::smem_u32(s.WTlo), 1024, tc::smem_u32(q.Thi),
+                   tc::smem_u32(q.Tlo), 256, 8, tc::idesc(64, 16), 0u);
+          tc::mma3(s.tmem + 32 + 64 * g, tc::smem_u32(q.GChi), tc::smem_u32(q.GClo), 1024, tc::smem_u32(q.UEhi),
+                   tc::smem_u32(q.UElo), 1024, 2, tc::idesc(64, 64), dw_started ? 1u : 0u);
+          tc_commit(q);
+        }
+        dw_started = true;
+        tc_wait(q, phase);
+        tc_stage_out(s, q, g, tg);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) mu[jj].v[k][c] = q.Z[4 * ty + k][2 * tx + c] - nu.v[k][c];
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          lam.v[k][c] += ((mu[0].v[k][c] + mu[1].v[k][c]) + (mu[2].v[k][c] + mu[3].v[k][c])) +
+                         (mu[4].v[k][c] + mu[5].v[k][c]);
+    }
+  }
+  // a group whose MMAs did not complete has no valid results
+  const bool bad = q.failed != 0;
+  if (!GRAD) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      if ((!act[c] || bad) && traj[c] >= 0)
+        for (int k = 0; k < a.nsave; ++k)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) a.u_save[(int64_t)k * n64 + (int64_t)(4 * ty + r) * n + traj[c]] = nan;
+  } else {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (traj[c] < 0) continue;
+      const bool ok = act[c] && !bad;
+      if (bad && ty == 0) a.loss[traj[c]] = nan;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        a.dp[(int64_t)(4 * ty + r) * n + traj[c]] = ok ? bbar.v[r][c] : nan;
+        a.du0[(int64_t)(4 * ty + r) * n + traj[c]] = ok ? lam.v[r][c] : nan;
+      }
+    }
+    // the group's weight-gradient partial: warp 4g + w reads rows 16w..16w+15
+    T* part = a.dW_part + ((int64_t)blockIdx.x * 2 + g) * D * D;
+    const int w = tg >> 5, lane = tg & 31;
+    float v0[16], v1[16], v2[16], v3[16];
+    const uint32_t ta = s.tmem + ((uint32_t)(32 * w) << 16) + (uint32_t)(32 + 64 * g);
+    if (dw_started && !bad) {
+      ld16(ta, v0);
+      ld16(ta + 16, v1);
+      ld16(ta + 32, v2);
+      ld16(ta + 48, v3);
+    }
+    if (lane < 16) {
+      const int row = 16 * w + lane;
+      const bool z = !dw_started;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        part[row * D + c] = bad ? nan : (z ? cst<T>(0.0) : v0[c]);
+        part[row * D + 16 + c] = bad ? nan : (z ? cst<T>(0.0) : v1[c]);
+        part[row * D + 32 + c] = bad ? nan : (z ? cst<T>(0.0) : v2[c]);
+        part[row * D + 48 + c] = bad ? nan : (z ? cst<T>(0.0) : v3[c]);
+      }
+    }
+  }
+  // no MMA in flight and every TMEM read done before the columns are freed
+  if (bad && tg == 0) {
+    uint32_t done = 0;
+    for (int it = 0; it < tc::kSpin && !done; ++it)
+      asm volatile(
+          "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+          "selp.b32 %0, 1, 0, P1;\n\t}\n"
+          : "=r"(done)
+          : "r"(tc::smem_u32(&q.bar)), "r"(phase ^ 1u)
+          : "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(s.tmem));
+  }
+}
+
 }  // namespace n64
+
+// Which products the d = 64 replay and gradient use (process-wide, set by
+// gs_set_option): the SIMT FP32 products (default, faster at 32 slots per CTA)
+// or the tcgen05 3xTF32 products.
+static std::atomic<int> g_node64_tensor{0};
+void node64_set_tensor(int on) { g_node64_tensor.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize) {
   const int64_t nblk = (n + n64::TB - 1) / n64::TB;
   const size_t ck = ((size_t)smax * 64 * n * tsize + 255) / 256 * 256;
-  return ck + (size_t)nblk * 64 * 64 * tsize;
+  return ck + (size_t)nblk * 2 * 64 * 64 * tsize;  // up to two weight-gradient partials per CTA
 }
 
 template <typename T>
@@ -856,15 +1481,25 @@ gs_status node64_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, 
   a.ck = (T*)ws;
   const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
   a.dW_part = (T*)((char*)ws + ((size_t)M->smax * 64 * P->n * sizeof(T) + 255) / 256 * 256);
-  const size_t smem = sizeof(n64::Smem<T>);
-  if (cudaFuncSetAttribute(n64::k_replay_node64<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return GS_ECUDA;
-  n64::k_replay_node64<T, true><<<nblk, n64::NT, smem, st>>>(a);
+  const bool tensor = g_node64_tensor.load(std::memory_order_relaxed) != 0;
+  if (tensor) {
+    const size_t smem = sizeof(n64::SmemTC) + 128;
+    if (cudaFuncSetAttribute(n64::k_replay_node64_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return GS_ECUDA;
+    n64::k_replay_node64_tc<true><<<nblk, n64::NT, smem, st>>>(a);
+  } else {
+    const size_t smem = sizeof(n64::Smem<T>);
+    if (cudaFuncSetAttribute(n64::k_replay_node64<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return GS_ECUDA;
+    n64::k_replay_node64<T, true><<<nblk, n64::NT, smem, st>>>(a);
+  }
   count_launch();
   if (!launch_ok()) return GS_ECUDA;
   if (dshared) {
-    n64::k_reduce_dW<T><<<(64 * 64 + 255) / 256, 256, 0, st>>>(a.dW_part, nblk, (T*)dshared);
+    n64::k_reduce_dW<T><<<(64 * 64 + 255) / 256, 256, 0, st>>>(a.dW_part, tensor ? 2 * nblk : nblk,
+                                                                (T*)dshared);
     count_launch();
   }
   return launch_ok() ? GS_OK : GS_ECUDA;
@@ -875,11 +1510,19 @@ gs_status node64_solve(const gs_problem* P, const gs_mesh* M, void* u_save, cuda
   n64::GradArgs64<T> a = grad64_args<T>(P, M);
   a.u_save = (T*)u_save;
   const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
-  const size_t smem = sizeof(n64::Smem<T>);
-  if (cudaFuncSetAttribute(n64::k_replay_node64<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return GS_ECUDA;
-  n64::k_replay_node64<T, false><<<nblk, n64::NT, smem, st>>>(a);
+  if (g_node64_tensor.load(std::memory_order_relaxed) != 0) {
+    const size_t smem = sizeof(n64::SmemTC) + 128;
+    if (cudaFuncSetAttribute(n64::k_replay_node64_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return GS_ECUDA;
+    n64::k_replay_node64_tc<false><<<nblk, n64::NT, smem, st>>>(a);
+  } else {
+    const size_t smem = sizeof(n64::Smem<T>);
+    if (cudaFuncSetAttribute(n64::k_replay_node64<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return GS_ECUDA;
+    n64::k_replay_node64<T, false><<<nblk, n64::NT, smem, st>>>(a);
+  }
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

@@ -74,6 +74,8 @@ _lib.gs_solve.argtypes = [_P(_Problem), _P(_Mesh), ctypes.c_void_p, ctypes.c_voi
 _lib.gs_solve_adaptive.argtypes = [_P(_Problem), _P(_Tol), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p]
 _lib.gs_solve_adaptive.restype = ctypes.c_int32
+_lib.gs_set_option.argtypes = [ctypes.c_int32, ctypes.c_int32]
+_lib.gs_set_option.restype = ctypes.c_int32
 _lib.gs_sens.argtypes = [_P(_Problem), _P(_Mesh), _P(_Loss)] + [ctypes.c_void_p] * 5
 _lib.gs_sens.restype = ctypes.c_int32
 _lib.gs_solve.restype = ctypes.c_int32
@@ -291,6 +293,15 @@ def gs_grad(ens: Ensemble, mesh: Mesh, loss: str = "sumsq", target=None, weight=
     _check(_lib.gs_grad(ctypes.byref(ps), ctypes.byref(ms), ctypes.byref(ls), _ptr(out.loss), _ptr(out.dp),
                         _ptr(out.du0), _ptr(out.dshared), _ptr(ws), ws.numel(), _stream(stream)), "gs_grad")
     return out
+
+
+OPT_NODE64_TENSOR_CORES = 1
+
+
+def gs_set_option(option: int, value: int) -> None:
+    """Process-wide option (OPT_NODE64_TENSOR_CORES: 1 = the d = 64 products on
+    the tensor cores, 0 = SIMT, the default)."""
+    _check(_lib.gs_set_option(option, value), "gs_set_option")
 
 
 def gs_sens(ens: Ensemble, mesh: Mesh, loss: str = "sumsq", target=None, weight=None, out: GradOut | None = None,

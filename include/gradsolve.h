@@ -276,6 +276,18 @@ GS_API gs_status gs_sens(const gs_problem* prob, const gs_mesh* mesh, const gs_l
 GS_API gs_status gs_grad_static(const gs_problem* prob, const gs_mesh* mesh, const gs_loss* loss_desc, void* loss,
                                 void* dp, void* du0, void* dshared, void* stream);
 
+/*
+ * Process-wide options (not thread-safe against concurrent calls).
+ *   GS_OPT_NODE64_TENSOR_CORES  0 (default): the d = 64 replay and gradient
+ *       compute W U, W^T g and g U^T with FP32 SIMT products; 1: on the
+ *       tensor cores (tcgen05, tf32 with a 3xTF32 split: fp32 accuracy).
+ *       Same results to fp32 rounding; at 32 slots per CTA the tensor-core
+ *       form is slower on B200, so it is off by default.
+ * Returns GS_EINVAL for an unknown option or value.
+ */
+#define GS_OPT_NODE64_TENSOR_CORES 1
+GS_API gs_status gs_set_option(int32_t option, int32_t value);
+
 /* Static description of a status code. */
 GS_API const char* gs_status_string(gs_status status);
 

@@ -138,3 +138,9 @@ def test_empty_ensemble_is_a_no_op():
     assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(m), ctypes.byref(_Loss(1, None, None)), None, None, None,
                         None, None) == 0
     assert _lib.gs_launch_count() == before
+
+
+def test_set_option_host_only():
+    from discrete_adjoint_b200.gradsolve import _lib
+    assert _lib.gs_set_option(1, 1) == 0 and _lib.gs_set_option(1, 0) == 0
+    assert _lib.gs_set_option(1, 2) == -1 and _lib.gs_set_option(99, 0) == -1

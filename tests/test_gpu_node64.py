@@ -1,6 +1,8 @@
 """GPU <-> oracle parity for the d = 64 shared-weight system (workload
 node64, fp32): recorder, forward solve, per-trajectory gradients dL/db_i and
-dL/du0_i on the same mesh, and the ensemble weight gradient dL/dW."""
+dL/du0_i on the same mesh, and the ensemble weight gradient dL/dW -- with the
+stage products in FP32 SIMT (the default) and on the tensor cores (tcgen05,
+3xTF32)."""
 import numpy as np
 import pytest
 import torch
@@ -11,6 +13,13 @@ import discrete_adjoint_b200 as gs
 from gpu_util import TOL, dev, ensemble, loss_args, mesh_by_trajectory, mesh_from_oracle, parity, tens
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=["simt", "tensor"])
+def products(request):
+    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, int(request.param == "tensor"))
+    yield request.param
+    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, 0)
 
 
 @pytest.fixture(scope="module", params=[512, 100])
@@ -51,14 +60,14 @@ def test_record_node64(case):
     assert np.array_equal(nsteps.cpu().numpy(), ns)
 
 
-def test_solve_node64(case):
+def test_solve_node64(case, products):
     prob, om = case
     _, us = oracle.replay(prob, om)
     u = gs.gs_solve(ensemble(prob), mesh_from_oracle(om, "f32")).double().cpu().numpy()
     assert np.abs(u - us).max() <= 1e-5 * np.abs(us).max()
 
 
-def test_grad_node64(case):
+def test_grad_node64(case, products):
     prob, om = case
     out = gs.gs_grad(ensemble(prob), mesh_from_oracle(om, "f32"), **loss_args(prob))
     torch.cuda.synchronize()
@@ -69,7 +78,7 @@ def test_grad_node64(case):
     assert np.abs(out.loss.double().cpu().numpy() - wide["loss"]).max() <= 1e-5 * np.abs(wide["loss"]).max()
 
 
-def test_node64_weight_gradient_is_additive():
+def test_node64_weight_gradient_is_additive(products):
     """dW of an ensemble equals the sum of the dW of two halves (any size)."""
     prob = W.node64(2000)
     ens = ensemble(prob)
@@ -84,3 +93,22 @@ def test_node64_weight_gradient_is_additive():
         parts.append(gs.gs_grad(ensemble(sub), mesh_from_oracle(om, "f32"), **loss_args(sub)).dshared.double())
     torch.cuda.synchronize()
     assert torch.linalg.norm(full - parts[0] - parts[1]) <= 1e-5 * torch.linalg.norm(full)
+
+
+def test_tensor_core_products_match_simt():
+    """The two product forms give the same gradients to fp32 rounding (the
+    3xTF32 split keeps fp32 accuracy), on a ragged ensemble."""
+    prob = W.node64(1000)
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(prob.n, 64, 1, "f32", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    outs = []
+    for on in (0, 1):
+        gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, on)
+        o = gs.gs_grad(ens, mesh, **loss_args(prob))
+        torch.cuda.synchronize()
+        outs.append([t.double().cpu().numpy() for t in (o.loss, o.dp, o.du0, o.dshared)])
+    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, 0)
+    for a, b in zip(*outs):
+        assert np.isfinite(b).all()
+        assert np.abs(a - b).max() <= 1e-4 * np.abs(a).max()
