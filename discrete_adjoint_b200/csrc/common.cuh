@@ -60,6 +60,32 @@ __device__ __forceinline__ T cst(double x) {
   return static_cast<T>(x);
 }
 
+// The same Tsit5 coefficients by index.  A double literal inside a loop is
+// rebuilt from two 32-bit halves at every use (two issue slots, ~55 uses per
+// replay step); read from this constant-bank table it enters its DFMA as an
+// operand and holds no register.  float coefficients stay immediates.  The
+// values are the #defines above, so results are bitwise unchanged.
+enum TsIdx : int {
+  kTsA21, kTsA31, kTsA32, kTsA41, kTsA42, kTsA43, kTsA51, kTsA52, kTsA53, kTsA54,
+  kTsA61, kTsA62, kTsA63, kTsA64, kTsA65, kTsB1, kTsB2, kTsB3, kTsB4, kTsB5, kTsB6,
+  kTsE1, kTsE2, kTsE3, kTsE4, kTsE5, kTsE6, kTsE7, kTsCount
+};
+#define GS_TS_LIST                                                                                      \
+  TS_A21, TS_A31, TS_A32, TS_A41, TS_A42, TS_A43, TS_A51, TS_A52, TS_A53, TS_A54, TS_A61, TS_A62, TS_A63, \
+      TS_A64, TS_A65, TS_B1, TS_B2, TS_B3, TS_B4, TS_B5, TS_B6, TS_E1, TS_E2, TS_E3, TS_E4, TS_E5, TS_E6, TS_E7
+static __constant__ double kTsTab[kTsCount] = {GS_TS_LIST};
+__host__ __device__ constexpr double ts_lit(int i) {
+  constexpr double v[kTsCount] = {GS_TS_LIST};
+  return v[i];
+}
+#undef GS_TS_LIST
+template <typename T, int I>
+__device__ __forceinline__ T tsc() {
+  static_assert(I >= 0 && I < kTsCount, "Tsit5 coefficient index");
+  if constexpr (sizeof(T) == 8) return kTsTab[I];
+  else return static_cast<T>(ts_lit(I));
+}
+
 __device__ __forceinline__ double fmaT(double a, double b, double c) { return fma(a, b, c); }
 __device__ __forceinline__ float fmaT(float a, float b, float c) { return fmaf(a, b, c); }
 

@@ -103,13 +103,13 @@ __device__ __forceinline__ void lorenz_vjp(const V& ux, const V& uy, const V& uz
 
 // acc = a1 k1 (+ a2 k2 ...) for the three components, in the contract's order.
 #define GS_ACC1(A1, K1)    \
-  ax = cst<T>(A1) * K1##x; \
-  ay = cst<T>(A1) * K1##y; \
-  az = cst<T>(A1) * K1##z;
+  ax = tsc<T, A1>() * K1##x; \
+  ay = tsc<T, A1>() * K1##y; \
+  az = tsc<T, A1>() * K1##z;
 #define GS_ACCN(AN, KN)             \
-  ax = fmaT(cst<T>(AN), KN##x, ax); \
-  ay = fmaT(cst<T>(AN), KN##y, ay); \
-  az = fmaT(cst<T>(AN), KN##z, az);
+  ax = fmaT(tsc<T, AN>(), KN##x, ax); \
+  ay = fmaT(tsc<T, AN>(), KN##y, ay); \
+  az = fmaT(tsc<T, AN>(), KN##z, az);
 
 template <typename T, int K, bool DENSE>
 __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(TsitLorenzArgs<T> a) {
@@ -190,43 +190,43 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     hq += n;
     cp += n3;
     V ax, ay, az, Ux, Uy, Uz;
-    GS_ACC1(TS_A21, k1)
+    GS_ACC1(kTsA21, k1)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
     V k2x, k2y, k2z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k2x, k2y, k2z);
-    GS_ACC1(TS_A31, k1)
-    GS_ACCN(TS_A32, k2)
+    GS_ACC1(kTsA31, k1)
+    GS_ACCN(kTsA32, k2)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
     V k3x, k3y, k3z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k3x, k3y, k3z);
-    GS_ACC1(TS_A41, k1)
-    GS_ACCN(TS_A42, k2)
-    GS_ACCN(TS_A43, k3)
+    GS_ACC1(kTsA41, k1)
+    GS_ACCN(kTsA42, k2)
+    GS_ACCN(kTsA43, k3)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
     V k4x, k4y, k4z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k4x, k4y, k4z);
-    GS_ACC1(TS_A51, k1)
-    GS_ACCN(TS_A52, k2)
-    GS_ACCN(TS_A53, k3)
-    GS_ACCN(TS_A54, k4)
+    GS_ACC1(kTsA51, k1)
+    GS_ACCN(kTsA52, k2)
+    GS_ACCN(kTsA53, k3)
+    GS_ACCN(kTsA54, k4)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
     V k5x, k5y, k5z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k5x, k5y, k5z);
-    GS_ACC1(TS_A61, k1)
-    GS_ACCN(TS_A62, k2)
-    GS_ACCN(TS_A63, k3)
-    GS_ACCN(TS_A64, k4)
-    GS_ACCN(TS_A65, k5)
+    GS_ACC1(kTsA61, k1)
+    GS_ACCN(kTsA62, k2)
+    GS_ACCN(kTsA63, k3)
+    GS_ACCN(kTsA64, k4)
+    GS_ACCN(kTsA65, k5)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
     V k6x, k6y, k6z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k6x, k6y, k6z);
     // stage 7 = u_{s+1}
-    GS_ACC1(TS_B1, k1)
-    GS_ACCN(TS_B2, k2)
-    GS_ACCN(TS_B3, k3)
-    GS_ACCN(TS_B4, k4)
-    GS_ACCN(TS_B5, k5)
-    GS_ACCN(TS_B6, k6)
+    GS_ACC1(kTsB1, k1)
+    GS_ACCN(kTsB2, k2)
+    GS_ACCN(kTsB3, k3)
+    GS_ACCN(kTsB4, k4)
+    GS_ACCN(kTsB5, k5)
+    GS_ACCN(kTsB6, k6)
     V xs, ys, zs, fsx, fsy, fsz;  // dense save points: u_s and f(u_s)
     if (DENSE) {
       xs = x;
@@ -398,75 +398,75 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     V f1x, f1y, f1z;
     lorenz_f(x, y, z, s, r, b, f1x, f1y, f1z);
     V U2x, U2y, U2z, U3x, U3y, U3z, U4x, U4y, U4z, U5x, U5y, U5z, U6x, U6y, U6z;
-    GS_ACC1(TS_A21, f1)
+    GS_ACC1(kTsA21, f1)
     GS_STAGE(U2x, U2y, U2z, ax, ay, az)
     V f2x, f2y, f2z;
     lorenz_f(U2x, U2y, U2z, s, r, b, f2x, f2y, f2z);
-    GS_ACC1(TS_A31, f1)
-    GS_ACCN(TS_A32, f2)
+    GS_ACC1(kTsA31, f1)
+    GS_ACCN(kTsA32, f2)
     GS_STAGE(U3x, U3y, U3z, ax, ay, az)
     V f3x, f3y, f3z;
     lorenz_f(U3x, U3y, U3z, s, r, b, f3x, f3y, f3z);
-    GS_ACC1(TS_A41, f1)
-    GS_ACCN(TS_A42, f2)
-    GS_ACCN(TS_A43, f3)
+    GS_ACC1(kTsA41, f1)
+    GS_ACCN(kTsA42, f2)
+    GS_ACCN(kTsA43, f3)
     GS_STAGE(U4x, U4y, U4z, ax, ay, az)
     V f4x, f4y, f4z;
     lorenz_f(U4x, U4y, U4z, s, r, b, f4x, f4y, f4z);
-    GS_ACC1(TS_A51, f1)
-    GS_ACCN(TS_A52, f2)
-    GS_ACCN(TS_A53, f3)
-    GS_ACCN(TS_A54, f4)
+    GS_ACC1(kTsA51, f1)
+    GS_ACCN(kTsA52, f2)
+    GS_ACCN(kTsA53, f3)
+    GS_ACCN(kTsA54, f4)
     GS_STAGE(U5x, U5y, U5z, ax, ay, az)
     V f5x, f5y, f5z;
     lorenz_f(U5x, U5y, U5z, s, r, b, f5x, f5y, f5z);
-    GS_ACC1(TS_A61, f1)
-    GS_ACCN(TS_A62, f2)
-    GS_ACCN(TS_A63, f3)
-    GS_ACCN(TS_A64, f4)
-    GS_ACCN(TS_A65, f5)
+    GS_ACC1(kTsA61, f1)
+    GS_ACCN(kTsA62, f2)
+    GS_ACCN(kTsA63, f3)
+    GS_ACCN(kTsA64, f4)
+    GS_ACCN(kTsA65, f5)
     GS_STAGE(U6x, U6y, U6z, ax, ay, az)
 
     // transposed step, stages 6 .. 1
     V m6x, m6y, m6z, m5x, m5y, m5z, m4x, m4y, m4z, m3x, m3y, m3z, m2x, m2y, m2z, m1x, m1y, m1z;
     V vx, vy, vz;
-    vx = h * (cst<T>(TS_B6) * lx);
-    vy = h * (cst<T>(TS_B6) * ly);
-    vz = h * (cst<T>(TS_B6) * lz);
+    vx = h * (tsc<T, kTsB6>() * lx);
+    vy = h * (tsc<T, kTsB6>() * ly);
+    vz = h * (tsc<T, kTsB6>() * lz);
     lorenz_vjp(U6x, U6y, U6z, s, r, b, vx, vy, vz, m6x, m6y, m6z, ps, pr, pb);
 
-    vx = h * fmaT(cst<T>(TS_A65), m6x, cst<T>(TS_B5) * lx);
-    vy = h * fmaT(cst<T>(TS_A65), m6y, cst<T>(TS_B5) * ly);
-    vz = h * fmaT(cst<T>(TS_A65), m6z, cst<T>(TS_B5) * lz);
+    vx = h * fmaT(tsc<T, kTsA65>(), m6x, tsc<T, kTsB5>() * lx);
+    vy = h * fmaT(tsc<T, kTsA65>(), m6y, tsc<T, kTsB5>() * ly);
+    vz = h * fmaT(tsc<T, kTsA65>(), m6z, tsc<T, kTsB5>() * lz);
     lorenz_vjp(U5x, U5y, U5z, s, r, b, vx, vy, vz, m5x, m5y, m5z, ps, pr, pb);
 
-    vx = h * fmaT(cst<T>(TS_A54), m5x, fmaT(cst<T>(TS_A64), m6x, cst<T>(TS_B4) * lx));
-    vy = h * fmaT(cst<T>(TS_A54), m5y, fmaT(cst<T>(TS_A64), m6y, cst<T>(TS_B4) * ly));
-    vz = h * fmaT(cst<T>(TS_A54), m5z, fmaT(cst<T>(TS_A64), m6z, cst<T>(TS_B4) * lz));
+    vx = h * fmaT(tsc<T, kTsA54>(), m5x, fmaT(tsc<T, kTsA64>(), m6x, tsc<T, kTsB4>() * lx));
+    vy = h * fmaT(tsc<T, kTsA54>(), m5y, fmaT(tsc<T, kTsA64>(), m6y, tsc<T, kTsB4>() * ly));
+    vz = h * fmaT(tsc<T, kTsA54>(), m5z, fmaT(tsc<T, kTsA64>(), m6z, tsc<T, kTsB4>() * lz));
     lorenz_vjp(U4x, U4y, U4z, s, r, b, vx, vy, vz, m4x, m4y, m4z, ps, pr, pb);
 
-    vx = h * fmaT(cst<T>(TS_A43), m4x, fmaT(cst<T>(TS_A53), m5x, fmaT(cst<T>(TS_A63), m6x, cst<T>(TS_B3) * lx)));
-    vy = h * fmaT(cst<T>(TS_A43), m4y, fmaT(cst<T>(TS_A53), m5y, fmaT(cst<T>(TS_A63), m6y, cst<T>(TS_B3) * ly)));
-    vz = h * fmaT(cst<T>(TS_A43), m4z, fmaT(cst<T>(TS_A53), m5z, fmaT(cst<T>(TS_A63), m6z, cst<T>(TS_B3) * lz)));
+    vx = h * fmaT(tsc<T, kTsA43>(), m4x, fmaT(tsc<T, kTsA53>(), m5x, fmaT(tsc<T, kTsA63>(), m6x, tsc<T, kTsB3>() * lx)));
+    vy = h * fmaT(tsc<T, kTsA43>(), m4y, fmaT(tsc<T, kTsA53>(), m5y, fmaT(tsc<T, kTsA63>(), m6y, tsc<T, kTsB3>() * ly)));
+    vz = h * fmaT(tsc<T, kTsA43>(), m4z, fmaT(tsc<T, kTsA53>(), m5z, fmaT(tsc<T, kTsA63>(), m6z, tsc<T, kTsB3>() * lz)));
     lorenz_vjp(U3x, U3y, U3z, s, r, b, vx, vy, vz, m3x, m3y, m3z, ps, pr, pb);
 
-    vx = h * fmaT(cst<T>(TS_A32), m3x,
-                  fmaT(cst<T>(TS_A42), m4x, fmaT(cst<T>(TS_A52), m5x, fmaT(cst<T>(TS_A62), m6x, cst<T>(TS_B2) * lx))));
-    vy = h * fmaT(cst<T>(TS_A32), m3y,
-                  fmaT(cst<T>(TS_A42), m4y, fmaT(cst<T>(TS_A52), m5y, fmaT(cst<T>(TS_A62), m6y, cst<T>(TS_B2) * ly))));
-    vz = h * fmaT(cst<T>(TS_A32), m3z,
-                  fmaT(cst<T>(TS_A42), m4z, fmaT(cst<T>(TS_A52), m5z, fmaT(cst<T>(TS_A62), m6z, cst<T>(TS_B2) * lz))));
+    vx = h * fmaT(tsc<T, kTsA32>(), m3x,
+                  fmaT(tsc<T, kTsA42>(), m4x, fmaT(tsc<T, kTsA52>(), m5x, fmaT(tsc<T, kTsA62>(), m6x, tsc<T, kTsB2>() * lx))));
+    vy = h * fmaT(tsc<T, kTsA32>(), m3y,
+                  fmaT(tsc<T, kTsA42>(), m4y, fmaT(tsc<T, kTsA52>(), m5y, fmaT(tsc<T, kTsA62>(), m6y, tsc<T, kTsB2>() * ly))));
+    vz = h * fmaT(tsc<T, kTsA32>(), m3z,
+                  fmaT(tsc<T, kTsA42>(), m4z, fmaT(tsc<T, kTsA52>(), m5z, fmaT(tsc<T, kTsA62>(), m6z, tsc<T, kTsB2>() * lz))));
     lorenz_vjp(U2x, U2y, U2z, s, r, b, vx, vy, vz, m2x, m2y, m2z, ps, pr, pb);
 
-    vx = h * fmaT(cst<T>(TS_A21), m2x,
-                  fmaT(cst<T>(TS_A31), m3x,
-                       fmaT(cst<T>(TS_A41), m4x, fmaT(cst<T>(TS_A51), m5x, fmaT(cst<T>(TS_A61), m6x, cst<T>(TS_B1) * lx)))));
-    vy = h * fmaT(cst<T>(TS_A21), m2y,
-                  fmaT(cst<T>(TS_A31), m3y,
-                       fmaT(cst<T>(TS_A41), m4y, fmaT(cst<T>(TS_A51), m5y, fmaT(cst<T>(TS_A61), m6y, cst<T>(TS_B1) * ly)))));
-    vz = h * fmaT(cst<T>(TS_A21), m2z,
-                  fmaT(cst<T>(TS_A31), m3z,
-                       fmaT(cst<T>(TS_A41), m4z, fmaT(cst<T>(TS_A51), m5z, fmaT(cst<T>(TS_A61), m6z, cst<T>(TS_B1) * lz)))));
+    vx = h * fmaT(tsc<T, kTsA21>(), m2x,
+                  fmaT(tsc<T, kTsA31>(), m3x,
+                       fmaT(tsc<T, kTsA41>(), m4x, fmaT(tsc<T, kTsA51>(), m5x, fmaT(tsc<T, kTsA61>(), m6x, tsc<T, kTsB1>() * lx)))));
+    vy = h * fmaT(tsc<T, kTsA21>(), m2y,
+                  fmaT(tsc<T, kTsA31>(), m3y,
+                       fmaT(tsc<T, kTsA41>(), m4y, fmaT(tsc<T, kTsA51>(), m5y, fmaT(tsc<T, kTsA61>(), m6y, tsc<T, kTsB1>() * ly)))));
+    vz = h * fmaT(tsc<T, kTsA21>(), m2z,
+                  fmaT(tsc<T, kTsA31>(), m3z,
+                       fmaT(tsc<T, kTsA41>(), m4z, fmaT(tsc<T, kTsA51>(), m5z, fmaT(tsc<T, kTsA61>(), m6z, tsc<T, kTsB1>() * lz)))));
     lorenz_vjp(x, y, z, s, r, b, vx, vy, vz, m1x, m1y, m1z, ps, pr, pb);
 
     lx += ((m1x + m2x) + (m3x + m4x)) + (m5x + m6x);

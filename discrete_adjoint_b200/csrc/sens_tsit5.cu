@@ -66,19 +66,19 @@ __device__ __forceinline__ void lorenz_jvp(T x, T y, T z, T s, T r, T b, const V
 // stage accumulators in the contract's order (state) and the same order for
 // the tangents
 #define GS_S_ACC1(A, K)          \
-  ax = cst<T>(A) * K##x;         \
-  ay = cst<T>(A) * K##y;         \
-  az = cst<T>(A) * K##z;         \
-  dax = cst<T>(A) * d##K##x;     \
-  day = cst<T>(A) * d##K##y;     \
-  daz = cst<T>(A) * d##K##z;
+  ax = tsc<T, A>() * K##x;         \
+  ay = tsc<T, A>() * K##y;         \
+  az = tsc<T, A>() * K##z;         \
+  dax = tsc<T, A>() * d##K##x;     \
+  day = tsc<T, A>() * d##K##y;     \
+  daz = tsc<T, A>() * d##K##z;
 #define GS_S_ACCN(A, K)                 \
-  ax = fmaT(cst<T>(A), K##x, ax);       \
-  ay = fmaT(cst<T>(A), K##y, ay);       \
-  az = fmaT(cst<T>(A), K##z, az);       \
-  dax = fmaT(cst<T>(A), d##K##x, dax);  \
-  day = fmaT(cst<T>(A), d##K##y, day);  \
-  daz = fmaT(cst<T>(A), d##K##z, daz);
+  ax = fmaT(tsc<T, A>(), K##x, ax);       \
+  ay = fmaT(tsc<T, A>(), K##y, ay);       \
+  az = fmaT(tsc<T, A>(), K##z, az);       \
+  dax = fmaT(tsc<T, A>(), d##K##x, dax);  \
+  day = fmaT(tsc<T, A>(), d##K##y, day);  \
+  daz = fmaT(tsc<T, A>(), d##K##z, daz);
 #define GS_S_STAGE(KN)                                                \
   Ux = fmaT(h, ax, x);                                                \
   Uy = fmaT(h, ay, y);                                                \
@@ -146,33 +146,33 @@ __global__ void __launch_bounds__(128, GS_SENS_MINB) k_sens_tsit5_lorenz(SensArg
     V dax, day, daz, dUx, dUy, dUz;
     T k2x, k2y, k2z, k3x, k3y, k3z, k4x, k4y, k4z, k5x, k5y, k5z, k6x, k6y, k6z;
     V dk2x, dk2y, dk2z, dk3x, dk3y, dk3z, dk4x, dk4y, dk4z, dk5x, dk5y, dk5z, dk6x, dk6y, dk6z;
-    GS_S_ACC1(TS_A21, k1)
+    GS_S_ACC1(kTsA21, k1)
     GS_S_STAGE(k2)
-    GS_S_ACC1(TS_A31, k1)
-    GS_S_ACCN(TS_A32, k2)
+    GS_S_ACC1(kTsA31, k1)
+    GS_S_ACCN(kTsA32, k2)
     GS_S_STAGE(k3)
-    GS_S_ACC1(TS_A41, k1)
-    GS_S_ACCN(TS_A42, k2)
-    GS_S_ACCN(TS_A43, k3)
+    GS_S_ACC1(kTsA41, k1)
+    GS_S_ACCN(kTsA42, k2)
+    GS_S_ACCN(kTsA43, k3)
     GS_S_STAGE(k4)
-    GS_S_ACC1(TS_A51, k1)
-    GS_S_ACCN(TS_A52, k2)
-    GS_S_ACCN(TS_A53, k3)
-    GS_S_ACCN(TS_A54, k4)
+    GS_S_ACC1(kTsA51, k1)
+    GS_S_ACCN(kTsA52, k2)
+    GS_S_ACCN(kTsA53, k3)
+    GS_S_ACCN(kTsA54, k4)
     GS_S_STAGE(k5)
-    GS_S_ACC1(TS_A61, k1)
-    GS_S_ACCN(TS_A62, k2)
-    GS_S_ACCN(TS_A63, k3)
-    GS_S_ACCN(TS_A64, k4)
-    GS_S_ACCN(TS_A65, k5)
+    GS_S_ACC1(kTsA61, k1)
+    GS_S_ACCN(kTsA62, k2)
+    GS_S_ACCN(kTsA63, k3)
+    GS_S_ACCN(kTsA64, k4)
+    GS_S_ACCN(kTsA65, k5)
     GS_S_STAGE(k6)
     // u_{s+1} and its tangent
-    GS_S_ACC1(TS_B1, k1)
-    GS_S_ACCN(TS_B2, k2)
-    GS_S_ACCN(TS_B3, k3)
-    GS_S_ACCN(TS_B4, k4)
-    GS_S_ACCN(TS_B5, k5)
-    GS_S_ACCN(TS_B6, k6)
+    GS_S_ACC1(kTsB1, k1)
+    GS_S_ACCN(kTsB2, k2)
+    GS_S_ACCN(kTsB3, k3)
+    GS_S_ACCN(kTsB4, k4)
+    GS_S_ACCN(kTsB5, k5)
+    GS_S_ACCN(kTsB6, k6)
     x = fmaT(h, ax, x);
     y = fmaT(h, ay, y);
     z = fmaT(h, az, z);

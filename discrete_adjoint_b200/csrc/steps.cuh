@@ -158,58 +158,58 @@ __device__ __forceinline__ void tsit5_err_step(const T u[3], const T p[3], T h, 
                                                T e[3]) {
   T k2[3], k3[3], k4[3], k5[3], k6[3], U[3];
 #pragma unroll
-  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, cst<T>(TS_A21) * k1[c], u[c]);
+  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, tsc<T, kTsA21>() * k1[c], u[c]);
   rhs3<T, SYS>(U, p, k2);
 #pragma unroll
-  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, fmaT(cst<T>(TS_A32), k2[c], cst<T>(TS_A31) * k1[c]), u[c]);
+  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, fmaT(tsc<T, kTsA32>(), k2[c], tsc<T, kTsA31>() * k1[c]), u[c]);
   rhs3<T, SYS>(U, p, k3);
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
-    T acc = cst<T>(TS_A41) * k1[c];
-    acc = fmaT(cst<T>(TS_A42), k2[c], acc);
-    acc = fmaT(cst<T>(TS_A43), k3[c], acc);
+    T acc = tsc<T, kTsA41>() * k1[c];
+    acc = fmaT(tsc<T, kTsA42>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsA43>(), k3[c], acc);
     U[c] = fmaT(h, acc, u[c]);
   }
   rhs3<T, SYS>(U, p, k4);
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
-    T acc = cst<T>(TS_A51) * k1[c];
-    acc = fmaT(cst<T>(TS_A52), k2[c], acc);
-    acc = fmaT(cst<T>(TS_A53), k3[c], acc);
-    acc = fmaT(cst<T>(TS_A54), k4[c], acc);
+    T acc = tsc<T, kTsA51>() * k1[c];
+    acc = fmaT(tsc<T, kTsA52>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsA53>(), k3[c], acc);
+    acc = fmaT(tsc<T, kTsA54>(), k4[c], acc);
     U[c] = fmaT(h, acc, u[c]);
   }
   rhs3<T, SYS>(U, p, k5);
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
-    T acc = cst<T>(TS_A61) * k1[c];
-    acc = fmaT(cst<T>(TS_A62), k2[c], acc);
-    acc = fmaT(cst<T>(TS_A63), k3[c], acc);
-    acc = fmaT(cst<T>(TS_A64), k4[c], acc);
-    acc = fmaT(cst<T>(TS_A65), k5[c], acc);
+    T acc = tsc<T, kTsA61>() * k1[c];
+    acc = fmaT(tsc<T, kTsA62>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsA63>(), k3[c], acc);
+    acc = fmaT(tsc<T, kTsA64>(), k4[c], acc);
+    acc = fmaT(tsc<T, kTsA65>(), k5[c], acc);
     U[c] = fmaT(h, acc, u[c]);
   }
   rhs3<T, SYS>(U, p, k6);
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
-    T acc = cst<T>(TS_B1) * k1[c];
-    acc = fmaT(cst<T>(TS_B2), k2[c], acc);
-    acc = fmaT(cst<T>(TS_B3), k3[c], acc);
-    acc = fmaT(cst<T>(TS_B4), k4[c], acc);
-    acc = fmaT(cst<T>(TS_B5), k5[c], acc);
-    acc = fmaT(cst<T>(TS_B6), k6[c], acc);
+    T acc = tsc<T, kTsB1>() * k1[c];
+    acc = fmaT(tsc<T, kTsB2>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsB3>(), k3[c], acc);
+    acc = fmaT(tsc<T, kTsB4>(), k4[c], acc);
+    acc = fmaT(tsc<T, kTsB5>(), k5[c], acc);
+    acc = fmaT(tsc<T, kTsB6>(), k6[c], acc);
     un[c] = fmaT(h, acc, u[c]);
   }
   rhs3<T, SYS>(un, p, k7);
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
-    T acc = cst<T>(TS_E1) * k1[c];
-    acc = fmaT(cst<T>(TS_E2), k2[c], acc);
-    acc = fmaT(cst<T>(TS_E3), k3[c], acc);
-    acc = fmaT(cst<T>(TS_E4), k4[c], acc);
-    acc = fmaT(cst<T>(TS_E5), k5[c], acc);
-    acc = fmaT(cst<T>(TS_E6), k6[c], acc);
-    acc = fmaT(cst<T>(TS_E7), k7[c], acc);
+    T acc = tsc<T, kTsE1>() * k1[c];
+    acc = fmaT(tsc<T, kTsE2>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsE3>(), k3[c], acc);
+    acc = fmaT(tsc<T, kTsE4>(), k4[c], acc);
+    acc = fmaT(tsc<T, kTsE5>(), k5[c], acc);
+    acc = fmaT(tsc<T, kTsE6>(), k6[c], acc);
+    acc = fmaT(tsc<T, kTsE7>(), k7[c], acc);
     e[c] = h * acc;
   }
 }
