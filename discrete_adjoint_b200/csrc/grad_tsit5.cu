@@ -33,7 +33,10 @@
 //
 // Memory layout: h [smax][n] and ck [smax][3][n] are step-major over slots, so
 // at a given step a warp touches 32K consecutive elements of every array.
-// Loads run one step ahead in registers and several steps ahead into L2.
+// With one slot per thread, h and the checkpoints stream into per-thread
+// shared-memory rings (cp.async, kRingF / kRingR steps ahead) and are read
+// from there one step ahead; with K > 1 they are loaded one step ahead into
+// registers and prefetched several steps ahead into L2.
 #include "steps.cuh"
 #include "vec.cuh"
 
@@ -54,6 +57,22 @@ namespace gs {
 #ifndef GS_PF_R
 #define GS_PF_R 4
 #endif
+#ifndef GS_GRAD_ASYNC
+#define GS_GRAD_ASYNC 1
+#endif
+// Copy rings (one trajectory per thread): the forward streams h kRingF steps
+// ahead, the reverse streams (u_s, h_s) kRingR steps ahead, each thread into
+// its own shared-memory slots with cp.async, so that no register waits on DRAM.
+#ifndef GS_RING_F
+#define GS_RING_F 8
+#endif
+#ifndef GS_RING_R
+#define GS_RING_R 8
+#endif
+constexpr int kRingF = GS_RING_F;
+constexpr int kRingR = GS_RING_R;
+static_assert((kRingF & (kRingF - 1)) == 0 && kRingF >= 2 && (kRingR & (kRingR - 1)) == 0 && kRingR >= 2,
+              "ring depths: powers of two, at least 2");
 // L2 prefetch distances in steps (a warp's forward step takes ~0.5 us and its
 // reverse step ~1 us, against a DRAM latency of ~1 us under load).
 constexpr int kPrefetchF = GS_PF_F;
@@ -158,6 +177,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   }
   const T* __restrict__ hp = a.h + j0;
   T* __restrict__ cp = a.ck + j0;
+  constexpr bool kAsync = GS_GRAD_ASYNC != 0 && K == 1;
+  __shared__ T ring[kAsync ? 4 * kRingR * GS_GRAD_BS : 1];
+  T* const rg = ring + threadIdx.x;  // this thread's element of slot row w: rg[w * GS_GRAD_BS]
 
   // ---------------------------------------------------------------- forward
   V L = vsplat<T, K>(cst<T>(0.0));
@@ -170,17 +192,32 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   V k1x, k1y, k1z;
   lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);
   V hn;
+  if constexpr (kAsync) {  // h of step s in slot s % kRingF
 #pragma unroll
-  for (int q = 0; q < K; ++q) hn.e[q] = 0 < S[q] ? hp[q] : cst<T>(0.0);
+    for (int s = 0; s < kRingF; ++s) {
+      if (s < S[0]) cp_async_el(rg + s * GS_GRAD_BS, hp + (int64_t)s * n);
+      cp_async_commit();
+    }
+    cp_async_wait<kRingF - 1>();
+    hn.e[0] = 0 < S[0] ? rg[0] : cst<T>(0.0);
+  } else {
+#pragma unroll
+    for (int q = 0; q < K; ++q) hn.e[q] = 0 < S[q] ? hp[q] : cst<T>(0.0);
+  }
   const T* hq = hp + n;                        // h of step st + 1
   const T* hf = hp + (int64_t)kPrefetchF * n;  // h of step st + kPrefetchF
   for (int st = 0; st < Smax; ++st) {
     const V h = hn;
-    if (st + kPrefetchF < Smax) prefetch_l2(hf);
-    hf += n;
+    if constexpr (kAsync) {
+      cp_async_wait<kRingF - 2>();  // the group of step st + 1
+      hn.e[0] = st + 1 < S[0] ? rg[((st + 1) & (kRingF - 1)) * GS_GRAD_BS] : cst<T>(0.0);
+    } else {
+      if (st + kPrefetchF < Smax) prefetch_l2(hf);
+      hf += n;
+    }
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      hn.e[q] = st + 1 < S[q] ? hq[q] : cst<T>(0.0);
+      if constexpr (!kAsync) hn.e[q] = st + 1 < S[q] ? hq[q] : cst<T>(0.0);
       if (st < S[q]) {
         cp[q] = x.e[q];
         cp[n + q] = y.e[q];
@@ -274,7 +311,13 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
         if (!DENSE) break;
       }
     }
+    if constexpr (kAsync) {  // step st + kRingF into the slot that step st has left
+      const int sn = st + kRingF;
+      if (sn < S[0]) cp_async_el(rg + (sn & (kRingF - 1)) * GS_GRAD_BS, hp + (int64_t)sn * n);
+      cp_async_commit();
+    }
   }
+  if constexpr (kAsync) cp_async_wait<0>();  // the reverse reuses the slots
 #pragma unroll
   for (int q = 0; q < K; ++q)
     if (i[q] >= 0) a.loss[i[q]] = L.e[q];
@@ -292,7 +335,32 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   }
   V cx = x, cy = y, cz = z, hc = vsplat<T, K>(cst<T>(0.0));
   const T* hq2 = hp + (int64_t)(Smax - 1) * n;  // h of the step being loaded
-  if (Smax > 0) {
+  // reverse ring: (u_s, h_s) of step s in slot s % kRingR, components in rows
+  // 4 (s % kRingR) + c; the copies of one step form one group
+  auto issue_r = [&](int sr) {
+    if (sr >= 0 && sr < S[0]) {
+      T* d = rg + (sr & (kRingR - 1)) * 4 * GS_GRAD_BS;
+      const T* c = a.ck + (int64_t)sr * n3 + j0;
+      cp_async_el(d, c);
+      cp_async_el(d + GS_GRAD_BS, c + n);
+      cp_async_el(d + 2 * GS_GRAD_BS, c + 2 * n);
+      cp_async_el(d + 3 * GS_GRAD_BS, hp + (int64_t)sr * n);
+    }
+    cp_async_commit();
+  };
+  auto take_r = [&](int sr) {  // step sr's values, its group complete
+    const T* d = rg + (sr & (kRingR - 1)) * 4 * GS_GRAD_BS;
+    cx.e[0] = d[0];
+    cy.e[0] = d[GS_GRAD_BS];
+    cz.e[0] = d[2 * GS_GRAD_BS];
+    hc.e[0] = d[3 * GS_GRAD_BS];
+  };
+  if constexpr (kAsync) {
+#pragma unroll
+    for (int i2 = 0; i2 < kRingR; ++i2) issue_r(Smax - 1 - i2);
+    cp_async_wait<kRingR - 1>();
+    if (Smax > 0 && Smax - 1 < S[0]) take_r(Smax - 1);
+  } else if (Smax > 0) {
     cp -= n3;
 #pragma unroll
     for (int q = 0; q < K; ++q) {
@@ -305,7 +373,7 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     }
   }
   for (int st = Smax - 1; st >= 0; --st) {
-    if (st >= kPrefetchR) {
+    if (!kAsync && st >= kPrefetchR) {
       const T* c = cp - (int64_t)kPrefetchR * n3;
       prefetch_l2(c);
       prefetch_l2(c + n);
@@ -378,7 +446,13 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     y = cy;
     z = cz;
     const V h = hc;
-    if (st > 0) {
+    if (kAsync && st > 0) {
+      cp_async_wait<kRingR - 2>();  // the group of step st - 1
+      if (st - 1 < S[0])
+        take_r(st - 1);
+      else
+        hc.e[0] = cst<T>(0.0);
+    } else if (st > 0) {
       cp -= n3;
       hq2 -= n;
 #pragma unroll
@@ -479,7 +553,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
       ly += pgy + qy;
       lz += pgz + qz;
     }
+    if constexpr (kAsync) issue_r(st - kRingR);  // into the slot that step st has left
   }
+  if constexpr (kAsync) cp_async_wait<0>();
   // save points at step 0 cannot exist (save times lie in (t0, t1])
 #pragma unroll
   for (int q = 0; q < K; ++q) {
