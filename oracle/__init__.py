@@ -30,7 +30,7 @@ _SRC = os.path.join(_HERE, "oracle.cpp")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 SYSTEMS = {"lorenz": 1, "robertson": 2, "hires": 3, "node64": 4, "linear": 5}
-METHODS = {"tsit5": 1, "ros2": 2}
+METHODS = {"tsit5": 1, "ros2": 2, "ros3": 3}
 DTYPES = {"f32": 1, "f64": 2}
 LOSSES = {"sumsq": 1, "linear": 2}
 
@@ -74,6 +74,8 @@ def lib():
         L.or_tsit5_tableau.argtypes = [dp, dp, dp]
         L.or_tsit5_tableau.restype = None
         L.or_ros2_gamma.restype = f64
+        L.or_ros3_coeffs.argtypes = [dp]
+        L.or_ros3_coeffs.restype = None
         L.or_ctrl_pow.argtypes = [i32, i64, dp, dp, dp]
         L.or_ctrl_pow.restype = None
         _lib = L
@@ -277,6 +279,15 @@ def tsit5_tableau():
 
 def ros2_gamma() -> float:
     return float(lib().or_ros2_gamma())
+
+
+def ros3_coeffs() -> dict:
+    """The oracle's ROS3 coefficients: gamma, inv_gamma, c21, c31, c32, m2, m3,
+    e1, e2, e3 (m1 = 1, a21 = a31 = 1, a32 = 0)."""
+    v = np.zeros(10)
+    lib().or_ros3_coeffs(_d(v))
+    keys = ["gamma", "inv_gamma", "c21", "c31", "c32", "m2", "m3", "e1", "e2", "e3"]
+    return dict(zip(keys, (float(x) for x in v)))
 
 
 def ctrl_pow(x, y, dtype: str = "f64"):

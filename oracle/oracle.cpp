@@ -23,9 +23,10 @@
 //              an independent second route to the same derivative.
 //   flops      a counting scalar (S = Cn) to count the replay's operations.
 //
-// Integrators: Tsitouras' 5(4) pair (Tsit5, Tsitouras 2011) and the
+// Integrators: Tsitouras' 5(4) pair (Tsit5, Tsitouras 2011), the
 // second-order Rosenbrock method ROS2 of Verwer, Spee, Blom & Hundsdorfer
-// (1999) with gamma = 1 + 1/sqrt(2).  Systems: Lorenz (DiffEqGPU "ad" example,
+// (1999) with gamma = 1 + 1/sqrt(2), and the third-order Rosenbrock method
+// ROS3 of Sandu, Verwer, Blom, Spee, Carmichael & Potra (1997).  Systems: Lorenz (DiffEqGPU "ad" example,
 // "Forward-mode automatic differentiation" listing), Robertson kinetics
 // (mass-action form of the reaction scheme A->B (k1), 2B->B+C (k2),
 // B+C->A+C (k3)), and the d=64 shared-weight system tanh(W u + b) - u.
@@ -179,7 +180,7 @@ template <> struct base_of<Cn> { using type = double; };
 // Method constants.
 // ---------------------------------------------------------------------------
 enum { SYS_LORENZ = 1, SYS_ROBERTSON = 2, SYS_HIRES = 3, SYS_NODE64 = 4, SYS_LINEAR = 5 };
-enum { M_TSIT5 = 1, M_ROS2 = 2 };
+enum { M_TSIT5 = 1, M_ROS2 = 2, M_ROS3 = 3 };
 enum { DT_F32 = 1, DT_F64 = 2 };
 enum { LOSS_SUMSQ = 1, LOSS_LINEAR = 2 };
 enum { TRAJ_OK = 0, TRAJ_MAXSTEPS = 1, TRAJ_DTMIN = 2, TRAJ_NONFINITE = 3, TRAJ_SINGULAR = 4 };
@@ -202,6 +203,28 @@ static const double TS_BT[7] = {-0.00178001105222577714, -0.0008164344596567469,
 
 // ROS2 (Verwer et al. 1999): gamma = 1 + 1/sqrt(2), L-stable choice.
 static const double ROS2_GAMMA = 1.7071067811865475;  // 1 + 1/sqrt(2) rounded to double
+
+// ROS3 (Sandu et al. 1997, "Benchmarking stiff ODE solvers for atmospheric
+// chemistry problems II: Rosenbrock solvers", method ROS3): three stages,
+// order 3, L-stable, with an embedded second-order solution.  gamma is the
+// root in (1/6, 1/2) of x^3 - 3x^2 + 3/2 x - 1/6.  The coefficients are those
+// of the transformed stage form (a_ij, c_ij / h, m_i, e_i); a21 = a31 = 1,
+// a32 = 0 and m1 = 1.  Each is the published value rounded to double; 1/gamma
+// is rounded once from the exact quotient.
+static const double ROS3_GAMMA = 0.435866521508459;
+static const double ROS3_INV_GAMMA = 2.294280360279042;
+static const double ROS3_C21 = -1.0156171083877703;
+static const double ROS3_C31 = 4.07599564525377;
+static const double ROS3_C32 = 9.20767942983308;
+static const double ROS3_M2 = 6.1697947043828245;
+static const double ROS3_M3 = -0.42772256543218573;
+static const double ROS3_E1 = 0.5;
+static const double ROS3_E2 = -2.907955871680547;
+static const double ROS3_E3 = 0.2235406989781157;
+
+// Error order q of the step-size controller: the local error estimate of
+// Tsit5 is O(h^5), of ROS2 O(h^2), of ROS3 O(h^3).
+inline int method_order(int method) { return method == M_TSIT5 ? 5 : (method == M_ROS3 ? 3 : 2); }
 
 constexpr int DMAX = 64;
 
@@ -375,6 +398,56 @@ bool ros2_step(int sys, int d, const S* u, const S* p, S h, S* unew, S* err) {
 }
 
 // ---------------------------------------------------------------------------
+// One ROS3 step (Sandu et al. 1997), with k_i = K_i / h of the paper's
+// transformed form (K_i are the paper's stage increments):
+//   M = I/gamma - h J(u);  M k1 = f(u);  v = u + h k1;
+//   M k2 = f(v) + c21 k1;  M k3 = f(v) + c31 k1 + c32 k2
+//   (a31 = a21 = 1 and a32 = 0, so stage 3 evaluates f at the same point as
+//   stage 2);  u_new = u + h (k1 + m2 k2 + m3 k3);
+//   error e = h (e1 k1 + e2 k2 + e3 k3)  (u_new minus the embedded solution).
+// Returns false when M is singular.
+// ---------------------------------------------------------------------------
+template <class S>
+bool ros3_step(int sys, int d, const S* u, const S* p, S h, S* unew, S* err) {
+  using T = typename base_of<S>::type;
+  S J[64];
+  S M[64], R[8];
+  int P[8];
+  jac<S>(sys, u, p, J);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) M[i * d + j] = fma_(-h, J[i * d + j], S(T(i == j ? ROS3_INV_GAMMA : 0.0)));
+  if (!lu_factor<S>(d, M, P, R)) return false;
+  S f0[8] = {}, k1[8] = {}, v[8] = {}, f1[8] = {}, r[8] = {}, k2[8] = {}, k3[8] = {};
+  rhs<S>(sys, u, p, nullptr, f0);
+  lu_solve<S>(d, M, P, R, f0, k1);
+  for (int c = 0; c < d; ++c) v[c] = fma_(h, k1[c], u[c]);
+  rhs<S>(sys, v, p, nullptr, f1);
+  for (int c = 0; c < d; ++c) r[c] = fma_(S(T(ROS3_C21)), k1[c], f1[c]);
+  lu_solve<S>(d, M, P, R, r, k2);
+  for (int c = 0; c < d; ++c) r[c] = fma_(S(T(ROS3_C32)), k2[c], fma_(S(T(ROS3_C31)), k1[c], f1[c]));
+  lu_solve<S>(d, M, P, R, r, k3);
+  for (int c = 0; c < d; ++c) {
+    S acc = fma_(S(T(ROS3_M3)), k3[c], fma_(S(T(ROS3_M2)), k2[c], k1[c]));
+    unew[c] = fma_(h, acc, u[c]);
+  }
+  if (err)
+    for (int c = 0; c < d; ++c)
+      err[c] = h * fma_(S(T(ROS3_E3)), k3[c], fma_(S(T(ROS3_E2)), k2[c], S(T(ROS3_E1)) * k1[c]));
+  return true;
+}
+
+// One step of the given method (Tsit5 never fails).
+template <class S>
+bool method_step(int sys, int method, int d, const S* u, const S* p, const S* W, S h, S* unew, S* err) {
+  if (method == M_TSIT5) {
+    tsit5_step<S>(sys, d, u, p, W, h, unew, err);
+    return true;
+  }
+  if (method == M_ROS3) return ros3_step<S>(sys, d, u, p, h, unew, err);
+  return ros2_step<S>(sys, d, u, p, h, unew, err);
+}
+
+// ---------------------------------------------------------------------------
 // Logarithm and exponential for the step-size controller, computed from IEEE
 // +, -, *, /, fma and the exact frexp / ldexp / rint only, so that any
 // implementation keeping this operation order gets the same bits (a library
@@ -439,7 +512,7 @@ T ctrl_pow(T x, T y) {
 //
 // Error norm: err = sqrt( (1/d) sum_c (e_c / sc_c)^2 ), sc_c = atol + rtol *
 // max(|u_c|, |u_new_c|), accept iff err <= 1.  PI controller with error order
-// q (5 for Tsit5, 2 for ROS2): accepted -> fac = 0.9 err^(-0.7/q)
+// q (5 for Tsit5, 2 for ROS2, 3 for ROS3): accepted -> fac = 0.9 err^(-0.7/q)
 // errprev^(0.4/q) clipped to [0.2, 10] (10 if err == 0), capped at 1 after a
 // rejection, errprev <- max(err, 1e-4); rejected -> fac = max(0.2, 0.9
 // err^(-1/q)) (0.2 if err is NaN or infinite).  The next proposal is fac * h_prop, where
@@ -490,7 +563,7 @@ T rms_scaled(int d, const T* x, const T* sc) {
 template <class T>
 T initial_step(int sys, int method, int d, const T* u0, const T* p, const T* W, T t0, T t1, T rtol,
                T atol) {
-  T q = method == M_TSIT5 ? T(5) : T(2);
+  T q = T(method_order(method));
   T sc[DMAX] = {}, f0[DMAX] = {}, u1[DMAX] = {}, f1[DMAX] = {}, df[DMAX] = {};
   for (int c = 0; c < d; ++c) sc[c] = std::fma(rtol, std::fabs(u0[c]), atol);
   rhs<T>(sys, u0, p, W, f0);
@@ -517,7 +590,7 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
   out.theta.assign(nsave, T(1));
   out.usave.assign((size_t)nsave * d, std::numeric_limits<T>::quiet_NaN());
   const T eps = std::numeric_limits<T>::epsilon();
-  const T q = method == M_TSIT5 ? T(5) : T(2);
+  const T q = T(method_order(method));
   T u[DMAX], un[DMAX], e[DMAX], sc[DMAX], f0[DMAX];
   for (int c = 0; c < d; ++c) u[c] = u0[c];
   rhs<T>(sys, u, p, W, f0);
@@ -546,8 +619,7 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
     T tn = t + hprop;
     bool clipped = tn >= tstop - T(4) * eps * std::fabs(tstop);
     T h = clipped ? tstop - t : hprop;
-    bool ok = method == M_TSIT5 ? (tsit5_step<T>(sys, d, u, p, W, h, un, e), true)
-                                : ros2_step<T>(sys, d, u, p, h, un, e);
+    bool ok = method_step<T>(sys, method, d, u, p, W, h, un, e);
     if (!ok) {
       out.status = TRAJ_SINGULAR;
       return out;
@@ -652,10 +724,7 @@ S replay_loss(int sys, int method, int d, const S* u0, const S* p, const S* W, c
   visit(0, S(T(0)));
   for (int s = 0; s < nsteps; ++s) {
     S hs = S(T(h[s]));
-    if (method == M_TSIT5)
-      tsit5_step<S>(sys, d, u, p, W, hs, un, nullptr);
-    else
-      ros2_step<S>(sys, d, u, p, hs, un, nullptr);
+    method_step<S>(sys, method, d, u, p, W, hs, un, nullptr);
     for (int c = 0; c < d; ++c) {
       up[c] = u[c];
       u[c] = un[c];
@@ -835,9 +904,9 @@ int check_prob(const Prob& P) {
   if (P.sys == SYS_HIRES) return -4;  // not built: equations not available here
   if (P.sys == SYS_LINEAR && (P.d != 1 || P.np != 1)) return -1;
   if (P.sys < 1 || P.sys > 5) return -1;
-  if (P.method != M_TSIT5 && P.method != M_ROS2) return -1;
-  if (P.method == M_ROS2 && P.d > 8) return -4;
-  if (P.method == M_ROS2 && P.sys == SYS_NODE64) return -4;
+  if (P.method != M_TSIT5 && P.method != M_ROS2 && P.method != M_ROS3) return -1;
+  if (P.method != M_TSIT5 && P.d > 8) return -4;
+  if (P.method != M_TSIT5 && P.sys == SYS_NODE64) return -4;
   if (P.dtype != DT_F32 && P.dtype != DT_F64) return -1;
   return 0;
 }
@@ -1066,10 +1135,7 @@ int or_count_step(int sys, int method, int d, int np, double* out6) {
   if (sys == SYS_NODE64) W.assign(4096, Cn(0.01));
   opcount() = OpCount();
   Cn h(0.01);
-  if (method == M_TSIT5)
-    tsit5_step<Cn>(sys, d, u.data(), p.data(), W.empty() ? nullptr : W.data(), h, un.data(), nullptr);
-  else
-    ros2_step<Cn>(sys, d, u.data(), p.data(), h, un.data(), nullptr);
+  method_step<Cn>(sys, method, d, u.data(), p.data(), W.empty() ? nullptr : W.data(), h, un.data(), nullptr);
   OpCount c = opcount();
   out6[0] = double(c.add);
   out6[1] = double(c.mul);
@@ -1092,9 +1158,8 @@ int or_step(int sys, int method, int dtype, int d, const double* u, const double
       WW.resize(4096);
       for (int c = 0; c < 4096; ++c) WW[c] = T(W[c]);
     }
-    bool ok = method == M_TSIT5
-                  ? (tsit5_step<T>(sys, d, uu.data(), pp.data(), WW.empty() ? nullptr : WW.data(), T(h), un.data(), e.data()), true)
-                  : ros2_step<T>(sys, d, uu.data(), pp.data(), T(h), un.data(), e.data());
+    bool ok = method_step<T>(sys, method, d, uu.data(), pp.data(), WW.empty() ? nullptr : WW.data(), T(h), un.data(),
+                             e.data());
     for (int c = 0; c < d; ++c) {
       unew[c] = double(un[c]);
       if (err) err[c] = double(e[c]);
@@ -1122,6 +1187,14 @@ void or_tsit5_tableau(double* c, double* A, double* bt) {
 }
 
 double or_ros2_gamma(void) { return ROS2_GAMMA; }
+
+// ROS3 coefficients for the order-condition pins: {gamma, 1/gamma, c21, c31,
+// c32, m2, m3, e1, e2, e3}.
+void or_ros3_coeffs(double* out10) {
+  const double v[10] = {ROS3_GAMMA, ROS3_INV_GAMMA, ROS3_C21, ROS3_C31, ROS3_C32,
+                        ROS3_M2,    ROS3_M3,        ROS3_E1,  ROS3_E2,  ROS3_E3};
+  for (int i = 0; i < 10; ++i) out10[i] = v[i];
+}
 
 // The controller's power function, element-wise (dtype 2: double, 1: float).
 void or_ctrl_pow(int dtype, int64_t n, const double* x, const double* y, double* out) {

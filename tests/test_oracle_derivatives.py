@@ -28,10 +28,17 @@ def _relinf(a, b):
     return np.abs(a - b).max(0) / np.abs(b).max(0)
 
 
+def _ros3(prob):
+    prob.method = "ros3"
+    return prob
+
+
 CASES = {
     "lorenz_small": lambda: W.lorenz_small(48),
     "lorenz_1m": lambda: W.lorenz_1m(24),
     "robertson": lambda: W.robertson(8),
+    "robertson_ros3": lambda: _ros3(W.robertson(8)),
+    "lorenz_ros3": lambda: _ros3(W.lorenz_small(16)),
 }
 
 
@@ -40,7 +47,8 @@ def recorded():
     out = {}
     for k, f in CASES.items():
         prob = f()
-        mesh = oracle.record(prob, W.SMAX[prob.name] * (2 if k == "robertson" else 1))
+        mesh = oracle.record(prob, W.SMAX[prob.name] * (2 if k.startswith("robertson") else 1)
+                             * (32 if k == "lorenz_ros3" else 1))
         assert (mesh.status == 0).all()
         out[k] = (prob, mesh)
     return out
@@ -59,12 +67,12 @@ def test_tape_matches_dual(recorded, case):
     assert e.max() <= tol, (e.max(), tol)
 
 
-@pytest.mark.parametrize("case", ["lorenz_small", "robertson"])
+@pytest.mark.parametrize("case", ["lorenz_small", "robertson", "robertson_ros3"])
 def test_tape_matches_fixed_mesh_fd(recorded, case):
     prob, mesh = recorded[case]
     prob = prob.subset(range(4))
     ns = mesh.nsteps[:4].copy()
-    if case == "robertson":
+    if case.startswith("robertson"):
         # the first 600 steps (t ~ 1e-3, through the stiff transient): the
         # 13,000-step chain's rounding noise would swamp a difference quotient
         ns = np.minimum(ns, 600).astype(np.int32)
@@ -74,13 +82,13 @@ def test_tape_matches_fixed_mesh_fd(recorded, case):
     # difference steps: relative for the rate constants, absolute for states;
     # Robertson's y2 lives near 1e-5, so its step is 1e-6
     scale = np.ones(base.shape[0])
-    if case == "robertson":
+    if case.startswith("robertson"):
         scale[4] = 1e-2
     fd = np.zeros_like(base)
     for r in range(base.shape[0]):
         for i in range(prob.n):
             x = base[r, i]
-            e = 1e-4 * (abs(x) if (case == "robertson" and r < 3) else max(scale[r], abs(x)))
+            e = 1e-4 * (abs(x) if (case.startswith("robertson") and r < 3) else max(scale[r], abs(x)))
 
             def Lat(delta):
                 pp = base.copy()
@@ -97,7 +105,7 @@ def test_tape_matches_fixed_mesh_fd(recorded, case):
     # stiff Robertson chain the loss carries rounding noise that a difference
     # quotient divides by the step, so its floor is ~1e-8..1e-7 (the exact
     # check for ROS2 is the decimal brute force below)
-    assert e.max() <= (1e-8 if case != "robertson" else 1e-7), e
+    assert e.max() <= (1e-8 if not case.startswith("robertson") else 1e-7), e
 
 
 def test_dot_product_node64():

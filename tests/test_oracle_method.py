@@ -11,6 +11,9 @@
   exact rational arithmetic.
 * ROS2: L-stability (R(inf) = 0 for gamma = 1 + 1/sqrt 2), second order
   (R(z) = 1 + z + z^2/2 + O(z^3)), and the same closed-form adjoint.
+* ROS3: the same closed-form adjoint, with R(z) = 1 + z b^T (I - z beta)^{-1} 1
+  of the standard Rosenbrock form recovered from the oracle's transformed-form
+  coefficients (the coefficient pins themselves are in test_oracle_ros3.py).
 """
 import os
 from fractions import Fraction as Fr
@@ -128,6 +131,66 @@ def _ros2_R(z, g):
     return num / den, (dnum * den - num * dden) / (den * den)
 
 
+def _lower_solve(Lm, rhs):
+    """Forward substitution with a lower-triangular matrix, exact."""
+    x = []
+    for i in range(len(rhs)):
+        acc = rhs[i] - sum(Lm[i][j] * x[j] for j in range(i))
+        x.append(acc / Lm[i][i])
+    return x
+
+
+def _ros3_std():
+    """ROS3 in the standard Rosenbrock form (alpha, Gamma, b, bhat), exact
+    rationals of the oracle's doubles.  The transformed form's relations
+    (Hairer & Wanner, Solving ODEs II, Sec. IV.7): Gamma^{-1} = diag(1/gamma) - C,
+    a = alpha Gamma^{-1}, m^T = b^T Gamma^{-1}; the error weights e give the
+    embedded solution with weights m - e.  1/gamma is the oracle's rounded
+    reciprocal, the value its arithmetic uses."""
+    co = oracle.ros3_coeffs()
+    ig = Fr(co["inv_gamma"])
+    C = [[Fr(0)] * 3, [Fr(co["c21"]), Fr(0), Fr(0)], [Fr(co["c31"]), Fr(co["c32"]), Fr(0)]]
+    Ginv = [[(ig if i == j else Fr(0)) - C[i][j] for j in range(3)] for i in range(3)]
+    cols = [_lower_solve(Ginv, [Fr(int(i == j)) for i in range(3)]) for j in range(3)]
+    G = [[cols[j][i] for j in range(3)] for i in range(3)]
+    A = [[Fr(0)] * 3, [Fr(1), Fr(0), Fr(0)], [Fr(1), Fr(0), Fr(0)]]
+    alpha = [[sum(A[i][k] * G[k][j] for k in range(3)) for j in range(3)] for i in range(3)]
+    m = [Fr(1), Fr(co["m2"]), Fr(co["m3"])]
+    e = [Fr(co["e1"]), Fr(co["e2"]), Fr(co["e3"])]
+    b = [sum(m[k] * G[k][j] for k in range(3)) for j in range(3)]
+    bh = [sum((m[k] - e[k]) * G[k][j] for k in range(3)) for j in range(3)]
+    beta = [[alpha[i][j] + G[i][j] for j in range(3)] for i in range(3)]
+    return alpha, G, beta, b, bh
+
+
+_ROS3 = None
+
+
+def _ros3_R(z):
+    """R(z) = 1 + z b^T w and R'(z) = b^T w + z b^T (I - z beta)^{-1} beta w,
+    w = (I - z beta)^{-1} 1: the stability function of the standard form."""
+    global _ROS3
+    if _ROS3 is None:
+        _ROS3 = _ros3_std()
+    _, _, beta, b, _ = _ROS3
+    Mz = [[Fr(int(i == j)) - z * beta[i][j] for j in range(3)] for i in range(3)]
+    w = _lower_solve(Mz, [Fr(1)] * 3)
+    bw = [sum(beta[i][j] * w[j] for j in range(3)) for i in range(3)]
+    y = _lower_solve(Mz, bw)
+    bt_w = sum(b[i] * w[i] for i in range(3))
+    return 1 + z * bt_w, bt_w + z * sum(b[i] * y[i] for i in range(3))
+
+
+def _R_any(method, z):
+    """(R, R') of Tsit5, ROS2 or ROS3 at z, exact."""
+    if method == "tsit5":
+        co = _tsit5_R_coeffs()
+        return _poly(co, z), _dpoly(co, z)
+    if method == "ros3":
+        return _ros3_R(z)
+    return _ros2_R(z, Fr(oracle.ros2_gamma()))
+
+
 def _closed_form(method, p, hs, u0=Fr(1)):
     """u_N = u0 prod R(z_n), z_n = p h_n; L = u_N^2.
     dL/du0 = 2 u_N prod R(z_n);  dL/dp = 2 u_N^2 sum_n h_n R'(z_n)/R(z_n)."""
@@ -140,9 +203,8 @@ def _closed_form(method, p, hs, u0=Fr(1)):
             R.append(_poly(co, z))
             dR.append(_dpoly(co, z))
     else:
-        g = Fr(oracle.ros2_gamma())
         for h in hs:
-            r, dr = _ros2_R(pf * Fr(h), g)
+            r, dr = _R_any(method, pf * Fr(h))
             R.append(r)
             dR.append(dr)
     prod = Fr(1)
@@ -164,6 +226,16 @@ def _kappa(method, p, hs):
         if method == "tsit5":
             terms = sum(abs(a) * abs(z) ** k for k, a in enumerate(co))
             R = sum(a * z**k for k, a in enumerate(co))
+        elif method == "ros3":
+            # |terms| of R = 1 + z b^T w, with |b_i w_i| summed
+            if _ROS3 is None:
+                _ros3_R(Fr(0))
+            beta, b = _ROS3[2], _ROS3[3]
+            zf = Fr(z)
+            Mz = [[Fr(int(i == j)) - zf * beta[i][j] for j in range(3)] for i in range(3)]
+            w = _lower_solve(Mz, [Fr(1)] * 3)
+            terms = 1 + abs(z) * sum(abs(float(b[i] * w[i])) for i in range(3))
+            R = float(1 + zf * sum(b[i] * w[i] for i in range(3)))
         else:
             d = 1 - g * z
             terms = 1 + 1.5 * abs(z / d) + 0.5 * abs(z * (z * (1 - g) - 1) / d**2)
@@ -172,7 +244,8 @@ def _kappa(method, p, hs):
     return worst
 
 
-@pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 1e4])])
+@pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 1e4]),
+                                         ("ros3", [0.5, 50.0, 1e4])])
 @pytest.mark.parametrize("mode", ["tape", "dual"])
 def test_closed_form_decay_adjoint(method, lams, mode):
     rng = np.random.default_rng(7)

@@ -46,6 +46,44 @@ def test_mesh_consistency(name):
             u = un
 
 
+@pytest.mark.parametrize("name,method,q", [("lorenz_small", "tsit5", 5), ("lorenz_small", "ros3", 3),
+                                           ("robertson", "ros2", 2), ("robertson", "ros3", 3)])
+def test_controller_reproduces_recorded_steps(name, method, q):
+    """The ratio of consecutive recorded steps is the PI controller's factor
+    clip(0.9 err_s^(-0.7/q) max(err_{s-1}, 1e-4)^(0.4/q), 0.2, 10), with err_s
+    recomputed from each recorded step: this pins the error order q the
+    controller uses for each method.  Steps clipped onto a save time or t1
+    and the pairs around a rejection (positions not recorded) are skipped;
+    a rejection disturbs at most two pairs."""
+    prob = W.by_name(name, n=4)
+    prob.method = method
+    mesh = oracle.record(prob, 20000)
+    assert (mesh.status == 0).all()
+    checked = 0
+    for i in range(prob.n):
+        S = mesh.nsteps[i]
+        h = mesh.h[i, :S]
+        clipped = np.zeros(S, bool)
+        clipped[mesh.save_idx[i] - 1] = True
+        u = prob.u0[:, i].copy()
+        errs = []
+        for s in range(S):
+            un, e, ok = oracle.step(prob.system, method, "f64", u, prob.p[:, i], h[s])
+            errs.append(_err_norm(e, u, un, prob.rtol, prob.atol))
+            u = un
+        bad = 0
+        for s in range(S - 1):
+            if clipped[s] or clipped[s + 1]:
+                continue
+            prev = 1.0 if s == 0 else max(errs[s - 1], 1e-4)
+            fac = 10.0 if errs[s] == 0 else min(10.0, max(0.2, 0.9 * errs[s] ** (-0.7 / q) * prev ** (0.4 / q)))
+            checked += 1
+            if abs(h[s + 1] / h[s] - fac) > 1e-11 * fac:
+                bad += 1
+        assert bad <= 2 * mesh.nreject[i], (i, bad, mesh.nreject[i])
+    assert checked > 100
+
+
 def _lorenz(t, u, s, r, b):
     return [s * (u[1] - u[0]), u[0] * (r - u[2]) - u[1], u[0] * u[1] - b * u[2]]
 
@@ -62,7 +100,7 @@ def test_tight_tolerance_solution_matches_scipy():
         assert err <= 1e-7, err
 
 
-@pytest.mark.parametrize("method,order", [("tsit5", 5), ("ros2", 2)])
+@pytest.mark.parametrize("method,order", [("tsit5", 5), ("ros2", 2), ("ros3", 3)])
 def test_convergence_order(method, order):
     prob = W.lorenz_small(1)
     prob.method = method
@@ -73,18 +111,21 @@ def test_convergence_order(method, order):
                         np.zeros(1, np.int32), np.zeros(1, np.int32))
         return oracle.replay(prob, m)[1][0, :, 0]
 
-    ref = solve(4096 if method == "ros2" else 1024)
+    ref = solve({"ros2": 4096, "ros3": 2048}.get(method, 1024))
     e1 = np.abs(solve(32) - ref).max()
     e2 = np.abs(solve(64) - ref).max()
     rate = np.log2(e1 / e2)
     assert abs(rate - order) < 0.35, rate
 
 
-def test_robertson_keeps_total_mass():
+@pytest.mark.parametrize("method", ["ros2", "ros3"])
+def test_robertson_keeps_total_mass(method):
     prob = W.robertson(8)
+    prob.method = method
     mesh = oracle.record(prob, 20000)
     _, us = oracle.replay(prob, mesh)
-    # the rates cancel in y1' + y2' + y3' and both ROS2 stages are linear in f
+    # the rates cancel in y1' + y2' + y3' (the rows of J sum to zero too), and
+    # every Rosenbrock stage is linear in f and J
     assert np.abs(us[0].sum(0) - 1.0).max() <= 1e-12
 
 

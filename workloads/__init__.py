@@ -47,7 +47,7 @@ SMAX = {"lorenz_small": 256, "lorenz_1m": 1024, "robertson": 8192, "node64": 256
 @dataclass
 class Problem:
     system: str            # "lorenz" | "robertson" | "node64" | "linear"
-    method: str            # "tsit5" | "ros2"
+    method: str            # "tsit5" | "ros2" | "ros3"
     dtype: str             # "f64" | "f32"
     n: int
     d: int
