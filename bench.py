@@ -70,6 +70,13 @@ WORKLOADS = {
     "robertson": dict(passes=1, flop_step=113 + 131, flop_save=9, kernel="k_grad_ros2", n=65536, dtype="f64",
                       desc="Robertson d=3, t in [0,1e5], ROS2 gamma=1+1/sqrt2, rtol=1e-6 atol=1e-10, "
                            "loss w . u(T), 1 record + 1 gradient pass"),
+    # third-order Rosenbrock: the forward step 142 (7 add, 26 mul, 53 fma, 3
+    # divisions, oracle count) + the transposed step 177 (hand count: three
+    # transposed LU solves, two Robertson VJPs, the second-derivative term)
+    "robertson_ros3": dict(passes=1, flop_step=142 + 177, flop_save=9, kernel="k_grad_ros3", problem="robertson",
+                           method="ros3", n=65536, dtype="f64",
+                           desc="Robertson d=3, t in [0,1e5], ROS3 (Sandu et al. 1997, order 3), rtol=1e-6 "
+                                "atol=1e-10, loss w . u(T), 1 record + 1 gradient pass"),
     "node64": dict(passes=1, flop_step=52992 + 104076, flop_save=384, kernel="k_replay_node64", n=131072,
                    dtype="f32",
                    desc="du/dt = tanh(W u + b_i) - u, d=64, shared W, t in [0,1], Tsit5 rtol=atol=1e-5, "
@@ -133,7 +140,10 @@ def metric_name(args) -> str:
 def make_problem(args, seed_offset=0, n=None):
     import workloads
     name = WORKLOADS[args.workload].get("problem", args.workload)
-    return workloads.by_name(name, n=n or args.n, dtype=args.dtype, seed_offset=seed_offset)
+    prob = workloads.by_name(name, n=n or args.n, dtype=args.dtype, seed_offset=seed_offset)
+    if "method" in WORKLOADS[args.workload]:
+        prob.method = WORKLOADS[args.workload]["method"]
+    return prob
 
 
 class ClockSampler:
@@ -249,7 +259,7 @@ def run_reference(args):
     kind = W.get("kind", "grad")
     solve = kind != "grad"
     sample = {"lorenz_1m": 256, "lorenz_1m_dense": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
-              "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512}[args.workload]
+              "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512, "robertson_ros3": 256}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
     om = oracle.record(prob, smax_cap(args.workload), nthreads=threads) if kind == "sens" else None
@@ -614,7 +624,7 @@ def run_ours(args):
         # samples sized for seconds of host work (and host memory for the
         # oracle's trajectory-major meshes)
         sample = {"lorenz_1m": 32768, "lorenz_1m_dense": 32768, "lorenz_small": 1024, "robertson": 256,
-                  "node64": 1024}[args.workload]
+                  "robertson_ros3": 2048, "node64": 1024}[args.workload]
         line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
     if world > 1:
         dist.barrier()

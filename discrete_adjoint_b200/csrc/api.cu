@@ -26,6 +26,9 @@ template <typename T>
 gs_status launch_grad_ros2(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                            cudaStream_t);
 template <typename T>
+gs_status launch_grad_ros3(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
+                           cudaStream_t);
+template <typename T>
 gs_status launch_solve3(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 gs_status record_node64(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
 gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,
@@ -42,7 +45,7 @@ static gs_status check_problem(const gs_problem* P) {
   if (!P) return GS_EINVAL;
   if (P->n < 0 || P->n > (int64_t)INT32_MAX) return GS_EINVAL;
   if (P->dtype != GS_F32 && P->dtype != GS_F64) return GS_EINVAL;
-  if (P->method != GS_TSIT5 && P->method != GS_ROS2) return GS_EINVAL;
+  if (P->method != GS_TSIT5 && P->method != GS_ROS2 && P->method != GS_ROS3) return GS_EINVAL;
   switch (P->system) {
     case GS_LORENZ:
     case GS_ROBERTSON:
@@ -197,6 +200,9 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (P->method == GS_ROS2)
     return P->dtype == GS_F64 ? launch_grad_ros2<double>(P, M, Ls, loss, dp, du0, ws, st)
                               : launch_grad_ros2<float>(P, M, Ls, loss, dp, du0, ws, st);
+  if (P->method == GS_ROS3)
+    return P->dtype == GS_F64 ? launch_grad_ros3<double>(P, M, Ls, loss, dp, du0, ws, st)
+                              : launch_grad_ros3<float>(P, M, Ls, loss, dp, du0, ws, st);
   return GS_EUNSUPPORTED;
 }
 

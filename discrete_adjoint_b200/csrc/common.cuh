@@ -55,6 +55,27 @@ namespace gs {
 // ROS2 (Verwer, Spee, Blom & Hundsdorfer 1999): gamma = 1 + 1/sqrt(2).
 #define ROS2_GAMMA 1.7071067811865475
 
+// ROS3 (Sandu, Verwer, Blom, Spee, Carmichael & Potra 1997): three stages,
+// order 3, L-stable, embedded order 2.  Coefficients of the transformed stage
+// form (a21 = a31 = 1, a32 = 0, m1 = 1) rounded to double; gamma is the root
+// in (1/6, 1/2) of x^3 - 3x^2 + 3/2 x - 1/6, ROS3_INV_GAMMA its reciprocal
+// rounded once.
+#define ROS3_INV_GAMMA 2.294280360279042
+#define ROS3_C21 (-1.0156171083877703)
+#define ROS3_C31 4.07599564525377
+#define ROS3_C32 9.20767942983308
+#define ROS3_M2 6.1697947043828245
+#define ROS3_M3 (-0.42772256543218573)
+#define ROS3_E1 0.5
+#define ROS3_E2 (-2.907955871680547)
+#define ROS3_E3 0.2235406989781157
+
+// Error order q of the step-size controller for each method: the local error
+// estimate of Tsit5 is O(h^5), of ROS2 O(h^2), of ROS3 O(h^3).
+__host__ __device__ constexpr double method_order(int method) {
+  return method == GS_TSIT5 ? 5.0 : (method == GS_ROS3 ? 3.0 : 2.0);
+}
+
 template <typename T>
 __device__ __forceinline__ T cst(double x) {
   return static_cast<T>(x);

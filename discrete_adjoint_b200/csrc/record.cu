@@ -56,7 +56,7 @@ enum RecMode { kRecCount = 0, kRecMesh = 1, kRecSolve = 2 };
 
 template <typename T, int SYS, int METHOD>
 __device__ T initial_step3(const T u0[3], const T p[3], T t0, T t1, T rtol, T atol) {
-  const T q = METHOD == GS_TSIT5 ? cst<T>(5.0) : cst<T>(2.0);
+  const T q = cst<T>(method_order(METHOD));
   T sc[3], f0[3], u1[3], f1[3], df[3];
 #pragma unroll
   for (int c = 0; c < 3; ++c) sc[c] = fmaT(rtol, fabs(u0[c]), atol);
@@ -122,7 +122,7 @@ template <typename T, int SYS, int METHOD, int MODE>
 __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T ln_floor) {
   const int64_t n = a.n;
   const T eps = Eps<T>::v;
-  const T q = METHOD == GS_TSIT5 ? cst<T>(5.0) : cst<T>(2.0);
+  const T q = cst<T>(method_order(METHOD));
   const T tstop = (r.kk < a.nsave && !a.dense) ? a.tsave[r.kk] : a.t1;
   if (r.hprop < cst<T>(16.0) * eps * fabs(r.t)) {
     r.status = GS_TRAJ_DTMIN;
@@ -135,7 +135,9 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
   if (METHOD == GS_TSIT5) {
     tsit5_err_step<T, SYS>(r.u, r.p, h, r.k1, un, k7, e);
   } else {
-    if (!ros2_err_step<T, SYS>(r.u, r.p, h, un, e)) {
+    const bool ok = METHOD == GS_ROS3 ? ros3_err_step<T, SYS>(r.u, r.p, h, un, e)
+                                      : ros2_err_step<T, SYS>(r.u, r.p, h, un, e);
+    if (!ok) {
       r.status = GS_TRAJ_SINGULAR;
       return true;
     }
@@ -400,6 +402,8 @@ static gs_status dispatch_rec(int sys, int method, const RecArgs<T>& a, cudaStre
   if (sys == GS_LORENZ && method == GS_ROS2) return launch_rec<T, kSysLorenz, GS_ROS2, MODE>(a, st);
   if (sys == GS_ROBERTSON && method == GS_TSIT5) return launch_rec<T, kSysRobertson, GS_TSIT5, MODE>(a, st);
   if (sys == GS_ROBERTSON && method == GS_ROS2) return launch_rec<T, kSysRobertson, GS_ROS2, MODE>(a, st);
+  if (sys == GS_LORENZ && method == GS_ROS3) return launch_rec<T, kSysLorenz, GS_ROS3, MODE>(a, st);
+  if (sys == GS_ROBERTSON && method == GS_ROS3) return launch_rec<T, kSysRobertson, GS_ROS3, MODE>(a, st);
   return GS_EUNSUPPORTED;
 }
 

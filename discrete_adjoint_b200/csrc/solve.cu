@@ -69,6 +69,10 @@ __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
       }
 #pragma unroll
       for (int c = 0; c < 3; ++c) k1[c] = k7[c];
+    } else if (METHOD == GS_ROS3) {
+      T LU[9], R[3], q1[3], v[3], q2[3], q3[3];
+      int P[3];
+      ros3_fwd<T, SYS>(u, p, h, LU, P, R, q1, v, q2, q3, un);
     } else {
       T LU[9], R[3], q1[3], v[3], q2[3];
       int P[3];
@@ -105,8 +109,12 @@ gs_status launch_solve3(const gs_problem* P, const gs_mesh* M, void* u_save, cud
     k_solve3<T, kSysLorenz, GS_TSIT5><<<grid, 128, 0, st>>>(a);
   else if (P->system == GS_LORENZ && P->method == GS_ROS2)
     k_solve3<T, kSysLorenz, GS_ROS2><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_LORENZ && P->method == GS_ROS3)
+    k_solve3<T, kSysLorenz, GS_ROS3><<<grid, 128, 0, st>>>(a);
   else if (P->system == GS_ROBERTSON && P->method == GS_TSIT5)
     k_solve3<T, kSysRobertson, GS_TSIT5><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_ROBERTSON && P->method == GS_ROS3)
+    k_solve3<T, kSysRobertson, GS_ROS3><<<grid, 128, 0, st>>>(a);
   else
     k_solve3<T, kSysRobertson, GS_ROS2><<<grid, 128, 0, st>>>(a);
   count_launch();

@@ -273,5 +273,49 @@ __device__ __forceinline__ bool ros2_fwd(const T u[3], const T p[3], T h, T LU[9
   return ok;
 }
 
+// ROS3 (Sandu et al. 1997) in the transformed stage form with k_i = K_i / h:
+//   M = I/gamma - h J(u);  M k1 = f(u);  v = u + h k1;
+//   M k2 = f(v) + c21 k1;  M k3 = f(v) + c31 k1 + c32 k2;
+//   u_new = u + h (k1 + m2 k2 + m3 k3);  e = h (e1 k1 + e2 k2 + e3 k3).
+// The operation order below is the floating-point contract of the method.
+template <typename T, int SYS>
+__device__ __forceinline__ bool ros3_fwd(const T u[3], const T p[3], T h, T LU[9], int P[3], T R[3], T k1[3],
+                                         T v[3], T k2[3], T k3[3], T un[3]) {
+  T J[9];
+  jac3<T, SYS>(u, p, J);
+#pragma unroll
+  for (int q = 0; q < 9; ++q) LU[q] = fmaT(-h, J[q], cst<T>((q % 4) == 0 ? ROS3_INV_GAMMA : 0.0));
+  bool ok = lu3(LU, P, R);
+  T f0[3], f1[3];
+  rhs3<T, SYS>(u, p, f0);
+  lu3_solve(LU, P, R, f0[0], f0[1], f0[2], k1[0], k1[1], k1[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) v[c] = fmaT(h, k1[c], u[c]);
+  rhs3<T, SYS>(v, p, f1);
+  lu3_solve(LU, P, R, fmaT(cst<T>(ROS3_C21), k1[0], f1[0]), fmaT(cst<T>(ROS3_C21), k1[1], f1[1]),
+            fmaT(cst<T>(ROS3_C21), k1[2], f1[2]), k2[0], k2[1], k2[2]);
+  T r[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) r[c] = fmaT(cst<T>(ROS3_C32), k2[c], fmaT(cst<T>(ROS3_C31), k1[c], f1[c]));
+  lu3_solve(LU, P, R, r[0], r[1], r[2], k3[0], k3[1], k3[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    const T acc = fmaT(cst<T>(ROS3_M3), k3[c], fmaT(cst<T>(ROS3_M2), k2[c], k1[c]));
+    un[c] = fmaT(h, acc, u[c]);
+  }
+  return ok;
+}
+
+// One ROS3 step with error estimate.  Returns false on a singular matrix.
+template <typename T, int SYS>
+__device__ __forceinline__ bool ros3_err_step(const T u[3], const T p[3], T h, T un[3], T e[3]) {
+  T LU[9], R[3], k1[3], v[3], k2[3], k3[3];
+  int P[3];
+  if (!ros3_fwd<T, SYS>(u, p, h, LU, P, R, k1, v, k2, k3, un)) return false;
+#pragma unroll
+  for (int c = 0; c < 3; ++c)
+    e[c] = h * fmaT(cst<T>(ROS3_E3), k3[c], fmaT(cst<T>(ROS3_E2), k2[c], cst<T>(ROS3_E1) * k1[c]));
+  return true;
+}
 
 }  // namespace gs

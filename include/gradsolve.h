@@ -71,6 +71,14 @@ typedef int32_t gs_status;
 /* Integrators. */
 #define GS_TSIT5 1 /* Tsitouras 5(4) pair, FSAL, PI step control */
 #define GS_ROS2 2  /* Rosenbrock ROS2, gamma = 1 + 1/sqrt(2) (Verwer et al. 1999); d = 3 only */
+/* Rosenbrock ROS3 (Sandu, Verwer, Blom, Spee, Carmichael & Potra 1997): three
+ * stages, order 3, L-stable, embedded order 2, controller order q = 3; d = 3
+ * only.  Stage form, with J = J(u) and gamma = 0.435866521508459:
+ *   M = I/gamma - h J;  M k1 = f(u);  v = u + h k1;  M k2 = f(v) + c21 k1;
+ *   M k3 = f(v) + c31 k1 + c32 k2;  u_new = u + h (k1 + m2 k2 + m3 k3);
+ *   error estimate h (e1 k1 + e2 k2 + e3 k3).  Higher-order stiff option of
+ * the pages' "explicit and Rosenbrock integrators" (GRADSOLVE abstract). */
+#define GS_ROS3 3
 
 #define GS_F32 1
 #define GS_F64 2
@@ -185,7 +193,7 @@ GS_API gs_status gs_count(const gs_problem* prob, const gs_tol* tol, int32_t sma
                    void* stream);
 
 /*
- * Record: adaptive solve of every trajectory (Tsit5 or ROS2 per prob->method)
+ * Record: adaptive solve of every trajectory (Tsit5, ROS2 or ROS3 per prob->method)
  * into the caller's mesh, slots ordered by decreasing step count.  Fills every
  * mesh array.  Trajectories that fail keep a status != 0 and a truncated mesh.
  * Runs a sizing pass, the slot ordering and the recording pass, all on stream.

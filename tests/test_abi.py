@@ -144,3 +144,25 @@ def test_set_option_host_only():
     from discrete_adjoint_b200.gradsolve import _lib
     assert _lib.gs_set_option(1, 1) == 0 and _lib.gs_set_option(1, 0) == 0
     assert _lib.gs_set_option(1, 2) == -1 and _lib.gs_set_option(99, 0) == -1
+
+
+def test_ros3_method_validation_host_only():
+    """ROS3 (method 3) is accepted for the d = 3 systems and refused where it is
+    not built: forward sensitivities, dense save points, the d = 64 system; an
+    unknown method is an invalid argument.  No call here reaches a launch."""
+    from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
+    m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+    ls = _Loss(1, None, None)
+    for system in (1, 2):
+        p = _host_problem(system=system, method=3)
+        assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 1) == 100 * 3 * 1000 * 8
+        assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(m), ctypes.byref(ls), ctypes.c_void_p(16),
+                            ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == -4
+        dense = _Tol(1e-6, 1e-6, 0.0)
+        dense.dense = 1
+        assert _lib.gs_count(ctypes.byref(p), ctypes.byref(dense), 100, ctypes.c_void_p(16), None, None) == -4
+        e = _host_problem(n=0, system=system, method=3)
+        assert _lib.gs_count(ctypes.byref(e), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, None, None, None) == 0
+    bad = _host_problem(method=4)
+    assert _lib.gs_count(ctypes.byref(bad), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, ctypes.c_void_p(16), None,
+                         None) == -1
