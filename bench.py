@@ -115,6 +115,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--n", type=int, default=None, help="trajectories per GPU (default: the workload's size)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--products", default="tensor", choices=["simt", "tensor"],
+                    help="d = 64 stage products: FP32 SIMT or tcgen05 3xTF32 (node64 only)")
     a = ap.parse_args()
     a.dtype = a.dtype or WORKLOADS[a.workload]["dtype"]
     a.n = a.n or WORKLOADS[a.workload]["n"]
@@ -464,6 +466,7 @@ def run_ours(args):
     passes = W["passes"]
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
+    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, int(args.products == "tensor"))
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
@@ -609,7 +612,8 @@ def run_ours(args):
                    "grad_ms": grad_ms, "record_ms": rec_ms, "grad_only_value": world * n / (grad_ms / 1e3),
                    "l2": "inputs larger than L2 (mesh %.2f GB, gradient workspace %.2f GB); no flush" % (
                        mesh.h.numel() * esz / 1e9, ws_grad.numel() / 1e9),
-                   "parallelism": f"dp{world} (independent trajectory shards)"},
+                   "parallelism": f"dp{world} (independent trajectory shards)",
+                   **({"products": args.products} if args.workload == "node64" else {})},
         "clocks": clocks,
         "e2e": {"value": world * n * passes / float(e2e_t.item()), "unit": "trajectory-gradients/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

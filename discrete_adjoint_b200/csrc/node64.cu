@@ -821,26 +821,15 @@ __global__ void k_reduce_dW(const T* part, int nblk, T* dW) {
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core products for the d = 64 replay and gradient (tcgen05, sm_100a).
-//
-// The three products of a stage -- Z = W U, W^T G and dW += G U^T over the
-// CTA's 32 slots -- run as tcgen05 MMAs of kind tf32 with a 3xTF32 split
-// (x = hi + lo, both rounded to TF32; A B ~ hi hi + hi lo + lo hi), which keeps
-// fp32 accuracy (measured: 5.6e-7 relative against a float64 product).
-//   Z, W^T G : M = 64 (components), N = 16 (a group's slots), K = 64, fp32
-//              accumulator in TMEM
-//   dW       : M = 64, N = 64, K = 16 (slots), accumulated in TMEM over the
-//              whole reverse sweep, read out once per group
-// Operands sit in shared memory as K-major tiles of 8-row x 16-byte core
-// matrices (row groups 128 B apart, 4-column chunks one tile-height of groups
-// apart), no swizzle.  TF32 operands cannot be MN-major here, so G and U are
-// written twice: by slot (the N operand of W^T G and of Z) and by component
-// (the operands of dW).  An M = 64 accumulator holds row m in TMEM lane
-// (m / 16) * 32 + m % 16; warps 0..3 read their lane quadrant and stage the
-// product through shared memory into the threads' 4 x 2 register blocks.
-// One thread issues the MMAs and commits them to an mbarrier; every wait is
-// bounded, and a CTA whose MMAs do not complete marks itself failed, skips
-// the remaining products, writes NaN results and still frees its TMEM.
+// tcgen05 building blocks for the d = 64 products (sm_100a): TF32 rounding and
+// the 3xTF32 split (x = hi + lo, both rounded to TF32; A B ~ hi lo + lo hi +
+// hi hi keeps fp32 accuracy: measured 5.6e-7 relative against a float64
+// product), byte offsets of K-major no-swizzle operand tiles (8-row x 16-byte
+// core matrices, row groups 128 B apart, 4-column K chunks one chunk stride
+// apart), shared-memory and instruction descriptors, the MMA issue and TMEM
+// loads.  TF32 operands cannot be MN-major here, so an operand needed with
+// either dimension as K is written twice.  An M = 128 accumulator holds row
+// m in TMEM lane m; an M = 64 one holds row m in lane (m / 16) * 32 + m % 16.
 // ---------------------------------------------------------------------------
 namespace tc {
 
@@ -914,65 +903,6 @@ __device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
 
 }  // namespace tc
 
-// The CTA's 32 slots form two groups of 16, one per half of the CTA (warps
-// 0..3 and 4..7), each with its own operand tiles, accumulators, mbarrier and
-// named barrier: the groups step independently, so one group's element-wise
-// work overlaps the other's MMAs and waits.
-constexpr int GS = 16;        // slots per group
-constexpr int GT = NT / 2;    // threads per group
-
-struct GroupTC {
-  float Thi[GS * D], Tlo[GS * D];    // U or G by slot: rows t, K = component
-  float GChi[D * GS], GClo[D * GS];  // G by component: rows c, K = slot
-  float UEhi[D * GS], UElo[D * GS];  // U by component: rows e, K = slot
-  float Z[D][GS];    // product staging [component][slot]
-  float red[D][GS];  // per-slot loss terms
-  float G[D][GS];    // second loss operand (linear loss)
-  unsigned long long bar;  // MMA completion
-  int failed;              // an MMA wait ran out
-  int flag[GS];
-  int pad[13];
-};
-
-struct SmemTC {
-  float Whi[D * D], Wlo[D * D];    // W, rows n, K = k
-  float WThi[D * D], WTlo[D * D];  // W^T, rows c, K = k (element (c, k) = W[k][c])
-  GroupTC grp[2];
-  uint32_t tmem;  // TMEM base (256 columns): group g uses [16g, 16g + 16) and [32 + 64g, 96 + 64g)
-};
-
-__device__ __forceinline__ void gbar(int g) { asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(GT) : "memory"); }
-
-// Wait for the group's last commit (bounded); the phase bit alternates per commit.
-__device__ __forceinline__ void tc_wait(GroupTC& q, uint32_t& phase) {
-  if (!q.failed) {
-    uint32_t done = 0;
-    for (int it = 0; it < tc::kSpin && !done; ++it)
-      asm volatile(
-          "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
-          "selp.b32 %0, 1, 0, P1;\n\t}\n"
-          : "=r"(done)
-          : "r"(tc::smem_u32(&q.bar)), "r"(phase)
-          : "memory");
-    if (!done) q.failed = 1;
-  }
-  phase ^= 1u;
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_commit(GroupTC& q) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   tc::smem_u32(&q.bar))
-               : "memory");
-}
-
-// Operands written by the group's threads are visible to its MMAs.
-__device__ __forceinline__ void tc_publish(int g) {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  gbar(g);
-}
-
 __device__ __forceinline__ void ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(
@@ -985,138 +915,271 @@ __device__ __forceinline__ void ld16(uint32_t taddr, float (&v)[16]) {
   for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]);
 }
 
-// The group's M = 64, N = 16 accumulator into q.Z: warp 4g + w reads lane
-// quadrant w, whose lanes 0..15 hold rows 16w..16w+15.
-__device__ __forceinline__ void tc_stage_out(const SmemTC& s, GroupTC& q, int g, int tg) {
-  const int w = tg >> 5, lane = tg & 31;
-  if (!q.failed) {
-    float v[16];
-    ld16(s.tmem + ((uint32_t)(32 * w) << 16) + (uint32_t)(16 * g), v);
-    if (lane < 16)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) q.Z[16 * w + lane][c] = v[c];
-  }
+// ---------------------------------------------------------------------------
+// Tensor-core replay with 128 trajectories per CTA (k_node64_t128).
+//
+// One TMEM lane per trajectory: the products are M = 128 MMAs whose
+// accumulator row t is trajectory t's vector, so every element-wise step runs
+// on the thread that owns the lane, without shuffles or shared-memory round
+// trips.  A CTA has 256 threads; trajectory t = 32 (w mod 4) + lane is owned by
+// warps w and w + 4, which hold its components [0, 32) and [32, 64).
+//   Z   = U W^T      M = 128 (t) x N = 64 (r) x K = 64 (k): A = U (rows t,
+//                    K = component), B = W (rows r, K = k)
+//   VJP = G W        M = 128 (t) x N = 64 (c) x K = 64 (r): A = G, B = W^T
+//   dW += G^T U      M = 64 (c) x N = 64 (e) x K = 128 (t), in two halves of
+//                    64 trajectories: A = G^T, B = U^T (rows component,
+//                    K = trajectory)
+// each as 3xTF32 (hi lo + lo hi + hi hi, hi = tf32(x), lo = tf32(x - hi)).
+// TMEM (512 columns): [0, 64) the M = 128 accumulator (Z, then W^T g);
+// [64 + 64 (j - 1), 64 + 64 j) stage slot j = 1..6, holding k_j during the
+// forward step and the stage recompute and mu_j once the transposed sweep has
+// passed stage j; [448, 512) the dW accumulator (M = 64: row c in lane
+// 32 (c / 16) + c mod 16).  The slots hold each trajectory's stage slopes, so
+// a stage sum reads them back lane by lane.  The arithmetic of the stage
+// sums, the transposed step and the outputs is that of k_replay_node64; the
+// products round differently (3xTF32 against an fp32 fma chain).
+// ---------------------------------------------------------------------------
+namespace t128 {
+
+constexpr int TT = 128;                              // trajectories per CTA
+constexpr int NT = 256;                              // threads per CTA
+constexpr int HC = D / 2;                            // components per thread
+constexpr uint32_t kChunkT = (TT / 8) * 128;         // K-chunk stride, trajectory-row tile (B)
+constexpr uint32_t kChunkW = (D / 8) * 128;          // K-chunk stride, 64-row weight tiles (B)
+constexpr uint32_t kChunkC = (D / 8) * 128 + 16;     // K-chunk stride, component-row tiles, padded (B)
+constexpr int kTileC = (TT / 2 / 4) * kChunkC / 4;   // floats per component-row tile (64 trajectories)
+constexpr uint32_t kColAcc = 0, kColSlot = 64, kColDW = 448;
+// Tsit5 weights in float for the transposed sweep (row m: a_{m+1, j+1}; b_j)
+__constant__ float kA[6][6] = {{0.f, 0.f, 0.f, 0.f, 0.f, 0.f},
+                               {(float)TS_A21, 0.f, 0.f, 0.f, 0.f, 0.f},
+                               {(float)TS_A31, (float)TS_A32, 0.f, 0.f, 0.f, 0.f},
+                               {(float)TS_A41, (float)TS_A42, (float)TS_A43, 0.f, 0.f, 0.f},
+                               {(float)TS_A51, (float)TS_A52, (float)TS_A53, (float)TS_A54, 0.f, 0.f},
+                               {(float)TS_A61, (float)TS_A62, (float)TS_A63, (float)TS_A64, (float)TS_A65, 0.f}};
+__constant__ float kB[6] = {(float)TS_B1, (float)TS_B2, (float)TS_B3, (float)TS_B4, (float)TS_B5, (float)TS_B6};
+
+struct Smem {
+  float Whi[D * D], Wlo[D * D];      // W: rows r, K = k
+  float WThi[D * D], WTlo[D * D];    // W^T: rows c, K = r (element (c, r) = W[r][c])
+  float Thi[TT * D], Tlo[TT * D];    // A operand of Z and the VJP: rows t, K = component
+  float GChi[kTileC], GClo[kTileC];  // G^T of one half: rows c, K = trajectory
+  float UEhi[kTileC], UElo[kTileC];  // U^T of one half: rows e, K = trajectory
+  float lpart[TT];                   // loss partials of the upper component halves
+  unsigned long long bar;            // MMA completion
+  uint32_t tmem;                     // TMEM base (512 columns)
+  int failed;                        // an MMA wait ran out
+  int smax;                          // CTA-wide chain length
+};
+
+// byte offset of (row c, trajectory t) in a component-row tile
+__device__ __forceinline__ uint32_t offC(int c, int t) {
+  return (uint32_t)(t >> 2) * kChunkC + (uint32_t)((c >> 3) * 128 + (c & 7) * 16 + (t & 3) * 4);
+}
+
+// Operands written by the CTA's threads become visible to its MMAs; earlier
+// TMEM reads are ordered before the MMAs that follow the barrier.
+__device__ __forceinline__ void publish() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  gbar(g);
+  __syncthreads();
 }
 
-// f(U) for the group on the tensor cores: y = tanh(b + W U), k = y - U.
-__device__ __forceinline__ void eval_f_tc(SmemTC& s, GroupTC& q, uint32_t& phase, const Blk<float>& U,
-                                          const Blk<float>& bias, Blk<float>& y, Blk<float>& k, int ty, int tx, int g,
-                                          int tg) {
-  gbar(g);  // previous readers of T and Z are done
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 2; ++c) tc::put(q.Thi, q.Tlo, tc::off(2 * tx + c, 4 * ty + a, GS), U.v[a][c]);
-  tc_publish(g);
-  if (tg == 0 && !q.failed) {
+__device__ __forceinline__ void commit(Smem& s) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   tc::smem_u32(&s.bar))
+               : "memory");
+}
+
+// Wait for the next completion of the CTA's mbarrier (bounded; a timeout
+// marks the CTA failed, after which no MMA is issued and no wait spins).
+__device__ __forceinline__ void wait(Smem& s, uint32_t& phase) {
+  if (!s.failed) {
+    uint32_t done = 0;
+    for (int it = 0; it < tc::kSpin && !done; ++it)
+      asm volatile(
+          "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+          "selp.b32 %0, 1, 0, P1;\n\t}\n"
+          : "=r"(done)
+          : "r"(tc::smem_u32(&s.bar)), "r"(phase)
+          : "memory");
+    if (!done) s.failed = 1;
+  }
+  phase ^= 1u;
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Z (or the VJP) for the CTA: ACC = T B^T with B = W (vjp = false) or W^T.
+__device__ __forceinline__ void product(Smem& s, int tid, uint32_t& phase, bool vjp) {
+  publish();
+  if (tid == 0 && !s.failed) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    tc::mma3(s.tmem + 16 * g, tc::smem_u32(s.Whi), tc::smem_u32(s.Wlo), 1024, tc::smem_u32(q.Thi),
-             tc::smem_u32(q.Tlo), 256, 8, tc::idesc(64, 16), 0u);
-    tc_commit(q);
+    tc::mma3(s.tmem + kColAcc, tc::smem_u32(s.Thi), tc::smem_u32(s.Tlo), kChunkT,
+             tc::smem_u32(vjp ? s.WThi : s.Whi), tc::smem_u32(vjp ? s.WTlo : s.Wlo), kChunkW, D / 8,
+             tc::idesc(TT, D), 0u);
+    commit(s);
   }
-  tc_wait(q, phase);
-  tc_stage_out(s, q, g, tg);
-  Blk<float> z;
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 2; ++c) z.v[a][c] = bias.v[a][c] + q.Z[4 * ty + a][2 * tx + c];
-  rhs_tail(z, U, y, k);
+  wait(s, phase);
 }
 
-__device__ __forceinline__ void tsit5_stages_tc(SmemTC& s, GroupTC& q, uint32_t& phase, const Blk<float>& u,
-                                                const Blk<float>& bias, const float (&h)[2], const Blk<float>& k1,
-                                                Blk<float>& k2, Blk<float>& k3, Blk<float>& k4, Blk<float>& k5,
-                                                Blk<float>& k6, Blk<float>& k7, Blk<float>& un, int ty, int tx, int g,
-                                                int tg) {
-  using T = float;
-  Blk<T> y, U;
-  {
-    const T c[1] = {cst<T>(TS_A21)};
-    const Blk<T>* const ks[1] = {&k1};
-    U = stage<T, 1>(c, ks, u, h);
-    eval_f_tc(s, q, phase, U, bias, y, k2, ty, tx, g, tg);
-  }
-  {
-    const T c[2] = {cst<T>(TS_A31), cst<T>(TS_A32)};
-    const Blk<T>* const ks[2] = {&k1, &k2};
-    U = stage<T, 2>(c, ks, u, h);
-    eval_f_tc(s, q, phase, U, bias, y, k3, ty, tx, g, tg);
-  }
-  {
-    const T c[3] = {cst<T>(TS_A41), cst<T>(TS_A42), cst<T>(TS_A43)};
-    const Blk<T>* const ks[3] = {&k1, &k2, &k3};
-    U = stage<T, 3>(c, ks, u, h);
-    eval_f_tc(s, q, phase, U, bias, y, k4, ty, tx, g, tg);
-  }
-  {
-    const T c[4] = {cst<T>(TS_A51), cst<T>(TS_A52), cst<T>(TS_A53), cst<T>(TS_A54)};
-    const Blk<T>* const ks[4] = {&k1, &k2, &k3, &k4};
-    U = stage<T, 4>(c, ks, u, h);
-    eval_f_tc(s, q, phase, U, bias, y, k5, ty, tx, g, tg);
-  }
-  {
-    const T c[5] = {cst<T>(TS_A61), cst<T>(TS_A62), cst<T>(TS_A63), cst<T>(TS_A64), cst<T>(TS_A65)};
-    const Blk<T>* const ks[5] = {&k1, &k2, &k3, &k4, &k5};
-    U = stage<T, 5>(c, ks, u, h);
-    eval_f_tc(s, q, phase, U, bias, y, k6, ty, tx, g, tg);
-  }
-  {
-    const T c[6] = {cst<T>(TS_B1), cst<T>(TS_B2), cst<T>(TS_B3), cst<T>(TS_B4), cst<T>(TS_B5), cst<T>(TS_B6)};
-    const Blk<T>* const ks[6] = {&k1, &k2, &k3, &k4, &k5, &k6};
-    un = stage<T, 6>(c, ks, u, h);
-    eval_f_tc(s, q, phase, un, bias, y, k7, ty, tx, g, tg);
+__device__ __forceinline__ void load32(uint32_t taddr, float (&v)[HC]) { tc::ld32(taddr, v); }
+
+__device__ __forceinline__ void st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      :
+      : "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 16 components [k0, k0 + 16) of a trajectory-row operand (hi / lo).
+__device__ __forceinline__ void put_rows16(Smem& s, int t, int k0, const float (&x)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float4 h, l;
+    h.x = tc::tf32_rna(x[4 * q]);
+    h.y = tc::tf32_rna(x[4 * q + 1]);
+    h.z = tc::tf32_rna(x[4 * q + 2]);
+    h.w = tc::tf32_rna(x[4 * q + 3]);
+    l.x = tc::tf32_rna(x[4 * q] - h.x);
+    l.y = tc::tf32_rna(x[4 * q + 1] - h.y);
+    l.z = tc::tf32_rna(x[4 * q + 2] - h.z);
+    l.w = tc::tf32_rna(x[4 * q + 3] - h.w);
+    const uint32_t o = tc::off(t, k0 + 4 * q, TT);
+    *(float4*)((char*)s.Thi + o) = h;
+    *(float4*)((char*)s.Tlo + o) = l;
   }
 }
 
-// Loss terms of the save points the group's flagged slots reached (the
-// contract's order: components 0..63, an fma chain by the slot's thread).
-__device__ __forceinline__ void save_point_loss_tc(GroupTC& q, const GradArgs64<float>& a, const Blk<float>& u,
-                                                   const int64_t (&o)[2], const bool (&hit)[2], float& Lslot, int ty,
-                                                   int tx, int g, int tg) {
-  gbar(g);
-  if (tg < GS) q.flag[tg] = 0;
-  gbar(g);
+// Stage J's state U = fma(h, sum_{m<J} a_Jm k_m, u) (the contract's order;
+// J = 1: U = u, J = 7: u_{s+1}) into the A operand and, to wait out the
+// product, into its slot (J = 7: slot 1, whose k_1 this pass has read);
+// 16 columns per pass.  For J = 7, u becomes u_{s+1}.
+template <int J>
+__device__ __forceinline__ void stage_in(Smem& s, uint32_t tl, int t, int c0, float h, float (&u)[HC]) {
+  constexpr double A[8][7] = {{0, 0, 0, 0, 0, 0, 0},
+                              {0, 0, 0, 0, 0, 0, 0},
+                              {TS_A21, 0, 0, 0, 0, 0, 0},
+                              {TS_A31, TS_A32, 0, 0, 0, 0, 0},
+                              {TS_A41, TS_A42, TS_A43, 0, 0, 0, 0},
+                              {TS_A51, TS_A52, TS_A53, TS_A54, 0, 0, 0},
+                              {TS_A61, TS_A62, TS_A63, TS_A64, TS_A65, 0, 0},
+                              {TS_B1, TS_B2, TS_B3, TS_B4, TS_B5, TS_B6, 0}};
+  constexpr int slot = J <= 6 ? J : 1;
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    if (!hit[c]) continue;
-    if (ty == 0) q.flag[2 * tx + c] = 1;
+  for (int qh = 0; qh < 2; ++qh) {
+    float U[16], v[16];
+    if (J == 1) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int r = 4 * ty + k;
-      const int64_t oo = o[c] + (int64_t)r * a.n;
-      if (a.loss_kind == GS_LOSS_SUMSQ) {
-        q.red[r][2 * tx + c] = a.target ? u.v[k][c] - a.target[oo] : u.v[k][c];
-      } else {
-        q.red[r][2 * tx + c] = a.weight[oo];
-        q.G[r][2 * tx + c] = u.v[k][c];
+      for (int c = 0; c < 16; ++c) U[c] = u[16 * qh + c];
+    } else {
+      ld16(tl + kColSlot + 16 * qh, v);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) U[c] = cst<float>(A[J][0]) * v[c];
+#pragma unroll
+      for (int m = 2; m < J; ++m) {
+        ld16(tl + kColSlot + 64 * (m - 1) + 16 * qh, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) U[c] = fmaT(cst<float>(A[J][m - 1]), v[c], U[c]);
       }
+#pragma unroll
+      for (int c = 0; c < 16; ++c) U[c] = fmaT(h, U[c], u[16 * qh + c]);
+    }
+    put_rows16(s, t, c0 + 16 * qh, U);
+    st16(tl + kColSlot + 64 * (slot - 1) + 16 * qh, U);
+    if (J == 7) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) u[16 * qh + c] = U[c];
     }
   }
-  gbar(g);
-  if (tg < GS && q.flag[tg]) {
-    float L = Lslot;
-    for (int r = 0; r < D; ++r)
-      L = a.loss_kind == GS_LOSS_SUMSQ ? fmaT(q.red[r][tg], q.red[r][tg], L) : fmaT(q.red[r][tg], q.G[r][tg], L);
-    Lslot = L;
+}
+
+// After the product: k = tanh(Z + b) - U, U from the slot, k into the slot.
+__device__ __forceinline__ void stage_out(uint32_t tl, const float (&bias)[HC], int slot) {
+#pragma unroll
+  for (int qh = 0; qh < 2; ++qh) {
+    float z[16], U[16];
+    ld16(tl + kColAcc + 16 * qh, z);
+    ld16(tl + kColSlot + 64 * (slot - 1) + 16 * qh, U);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) z[c] = tanh(bias[16 * qh + c] + z[c]) - U[c];
+    st16(tl + kColSlot + 64 * (slot - 1) + 16 * qh, z);
   }
 }
 
-// The replay (solve) and the fused replay + reverse sweep with the products on
-// the tensor cores; same slots, save points, loss and outputs as
-// k_replay_node64 (dW partials: one per group, two per CTA).
+template <int J>
+__device__ __forceinline__ void fwd_stage(Smem& s, int tid, int t, int c0, uint32_t& phase, uint32_t tl, float h,
+                                          float (&u)[HC], const float (&bias)[HC]) {
+  stage_in<J>(s, tl, t, c0, h, u);
+  product(s, tid, phase, false);
+  stage_out(tl, bias, J <= 6 ? J : 1);
+}
+
+// 16 components of trajectory tk (0..63 within its half) into G^T and U^T.
+__device__ __forceinline__ void put_cols16(Smem& s, int tk, int c0, const float (&g)[16], const float (&U)[16]) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t o = offC(c0 + c, tk);
+    tc::put(s.GChi, s.GClo, o, g[c]);
+    tc::put(s.UEhi, s.UElo, o, U[c]);
+  }
+}
+
+// nu_j on 16 columns: h (b_j lambda + sum_{m>j} a_mj mu_m), mu_m from slots m > j.
+__device__ __forceinline__ void sweep_nu(uint32_t tl, int jj, int qh, float h, const float (&lam)[HC],
+                                         float (&nu)[16]) {
+  float v[16];
+  const float bj = kB[jj];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) nu[c] = bj * lam[16 * qh + c];
+#pragma unroll 1
+  for (int m = 5; m > jj; --m) {
+    ld16(tl + kColSlot + 64 * m + 16 * qh, v);
+    const float am = kA[m][jj];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) nu[c] = fmaT(am, v[c], nu[c]);
+  }
+#pragma unroll
+  for (int c = 0; c < 16; ++c) nu[c] = h * nu[c];
+}
+
+// U_j on 16 columns: fma(h, sum_{m<j} a_jm k_m, u) from slots m < j (u for j = 1).
+__device__ __forceinline__ void sweep_U(uint32_t tl, int jj, int qh, float h, const float (&u)[HC], float (&U)[16]) {
+  if (jj == 0) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) U[c] = u[16 * qh + c];
+    return;
+  }
+  float v[16];
+  ld16(tl + kColSlot + 16 * qh, v);
+  const float a0 = kA[jj][0];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) U[c] = a0 * v[c];
+#pragma unroll 1
+  for (int m = 1; m < jj; ++m) {
+    ld16(tl + kColSlot + 64 * m + 16 * qh, v);
+    const float am = kA[jj][m];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) U[c] = fmaT(am, v[c], U[c]);
+  }
+#pragma unroll
+  for (int c = 0; c < 16; ++c) U[c] = fmaT(h, U[c], u[16 * qh + c]);
+}
+
 template <bool GRAD>
-__global__ void __launch_bounds__(NT, 1) k_replay_node64_tc(GradArgs64<float> a) {
+__global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
   using T = float;
-  extern __shared__ __align__(128) unsigned char smem_raw_tc[];
-  SmemTC& s = *reinterpret_cast<SmemTC*>(smem_raw_tc);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int g = tid / GT, tg = tid % GT, ty = tg / 8, tx = tg % 8;
-  GroupTC& q = s.grp[g];
+  extern __shared__ __align__(1024) unsigned char smem_raw_t128[];
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw_t128);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = 32 * (warp & 3) + lane, hf = warp >> 2, c0 = HC * hf;
   const int64_t n = a.n;
-  const int64_t base = (int64_t)blockIdx.x * TB + GS * g;  // the group's first slot
+  const int64_t base = (int64_t)blockIdx.x * TT;
   const int64_t n64 = (int64_t)D * n;
   const T nan = cst<T>(__int_as_float(0x7fc00000));
   for (int e = tid; e < D * D; e += NT) {
@@ -1125,13 +1188,14 @@ __global__ void __launch_bounds__(NT, 1) k_replay_node64_tc(GradArgs64<float> a)
     tc::put(s.Whi, s.Wlo, tc::off(r, c, D), w);
     tc::put(s.WThi, s.WTlo, tc::off(c, r, D), w);
   }
-  if (tg == 0) {
-    q.failed = 0;
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc::smem_u32(&q.bar)));
+  if (tid == 0) {
+    s.failed = 0;
+    s.smax = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc::smem_u32(&s.bar)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(tc::smem_u32(&s.tmem)));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(tc::smem_u32(&s.tmem)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1139,316 +1203,255 @@ __global__ void __launch_bounds__(NT, 1) k_replay_node64_tc(GradArgs64<float> a)
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   uint32_t phase = 0;
+  const uint32_t tl = s.tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0;  // lane t, this half
 
-  int64_t traj[2];
-  int S[2];
-  bool act[2];
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const int64_t j = base + 2 * tx + c;
-    traj[c] = -1;
-    S[c] = 0;
-    act[c] = false;
-    if (j < n) {
-      const int64_t i = a.order[j];
-      if (i >= 0 && i < n) {
-        traj[c] = i;
-        const int sq = a.nsteps[j];
-        if (a.status[j] == GS_TRAJ_OK && sq >= 0 && sq <= a.smax) {
-          S[c] = sq;
-          act[c] = true;
-        }
+  // this thread's slot
+  const int64_t j = base + t;
+  int64_t traj = -1;
+  int S = 0;
+  bool act = false;
+  if (j < n) {
+    const int64_t i = a.order[j];
+    if (i >= 0 && i < n) {
+      traj = i;
+      const int sq = a.nsteps[j];
+      if (a.status[j] == GS_TRAJ_OK && sq >= 0 && sq <= a.smax) {
+        S = sq;
+        act = true;
       }
     }
   }
-  if (tg < GS) q.flag[tg] = 0;
-  gbar(g);
-  if (ty == 0) {
-    q.flag[2 * tx] = S[0];
-    q.flag[2 * tx + 1] = S[1];
-  }
-  gbar(g);
-  int Smax = 0;
-  for (int k = 0; k < GS; ++k) Smax = q.flag[k] > Smax ? q.flag[k] : Smax;
-  T Lslot = cst<T>(0.0);
+  atomicMax(&s.smax, S);
+  __syncthreads();
+  const int Smax = s.smax;
 
-  Blk<T> u, bias;
+  T u[HC], bias[HC];
 #pragma unroll
-  for (int c = 0; c < 2; ++c)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int r = 4 * ty + k;
-      u.v[k][c] = act[c] ? a.u0[(int64_t)r * n + traj[c]] : cst<T>(0.0);
-      bias.v[k][c] = act[c] ? a.p[(int64_t)r * n + traj[c]] : cst<T>(0.0);
-    }
-  int kk[2] = {0, 0}, next[2];
-#pragma unroll
-  for (int c = 0; c < 2; ++c) next[c] = act[c] && S[c] > 0 ? a.save_idx[base + 2 * tx + c] : -1;
+  for (int c = 0; c < HC; ++c) {
+    u[c] = act ? a.u0[(int64_t)(c0 + c) * n + traj] : cst<T>(0.0);
+    bias[c] = act ? a.p[(int64_t)(c0 + c) * n + traj] : cst<T>(0.0);
+  }
+  T Lh = cst<T>(0.0);  // loss terms of this thread's components
+  int kk = 0, next = act && S > 0 ? a.save_idx[j] : -1;
 
   // ---------------------------------------------------------------- forward
-  {
-    Blk<T> y, k1, k2, k3, k4, k5, k6, k7, un;
-    eval_f_tc(s, q, phase, u, bias, y, k1, ty, tx, g, tg);
-    for (int st = 0; st < Smax; ++st) {
-      T hh[2];
+  fwd_stage<1>(s, tid, t, c0, phase, tl, cst<T>(0.0), u, bias);  // k1 = f(u0)
+  for (int st = 0; st < Smax; ++st) {
+    const T h = st < S ? a.h[(int64_t)st * n + j] : cst<T>(0.0);
+    if (GRAD && st < S) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        hh[c] = st < S[c] ? a.h[(int64_t)st * n + base + 2 * tx + c] : cst<T>(0.0);
-        if (GRAD && st < S[c]) {
+      for (int c = 0; c < HC; ++c) a.ck[(int64_t)st * n64 + (int64_t)(c0 + c) * n + j] = u[c];
+    }
+    fwd_stage<2>(s, tid, t, c0, phase, tl, h, u, bias);
+    fwd_stage<3>(s, tid, t, c0, phase, tl, h, u, bias);
+    fwd_stage<4>(s, tid, t, c0, phase, tl, h, u, bias);
+    fwd_stage<5>(s, tid, t, c0, phase, tl, h, u, bias);
+    fwd_stage<6>(s, tid, t, c0, phase, tl, h, u, bias);
+    fwd_stage<7>(s, tid, t, c0, phase, tl, h, u, bias);  // u <- u_{st+1}; k7 -> slot 1 (FSAL)
+    if (st + 1 == next) {
+      const int64_t o = (int64_t)kk * n64 + traj;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            a.ck[(int64_t)st * n64 + (int64_t)(4 * ty + k) * n + base + 2 * tx + c] = u.v[k][c];
+      for (int c = 0; c < HC; ++c) {
+        const int64_t oo = o + (int64_t)(c0 + c) * n;
+        if (!GRAD) {
+          a.u_save[oo] = u[c];
+        } else if (a.loss_kind == GS_LOSS_SUMSQ) {
+          const T d = a.target ? u[c] - a.target[oo] : u[c];
+          Lh = fmaT(d, d, Lh);
+        } else {
+          Lh = fmaT(a.weight[oo], u[c], Lh);
         }
       }
-      tsit5_stages_tc(s, q, phase, u, bias, hh, k1, k2, k3, k4, k5, k6, k7, un, ty, tx, g, tg);
-      u = un;
-      k1 = k7;
-      bool hit[2];
-      int64_t o[2];
-      int anyhit = 0;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        hit[c] = st + 1 == next[c];
-        o[c] = hit[c] ? (int64_t)kk[c] * n64 + traj[c] : 0;
-        anyhit |= hit[c];
-        if (hit[c]) {
-          if (!GRAD) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) a.u_save[o[c] + (int64_t)(4 * ty + k) * n] = u.v[k][c];
-          }
-          ++kk[c];
-          next[c] = kk[c] < a.nsave ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
-        }
-      }
-      if (GRAD) {
-        // the group's threads agree on whether any of its slots hit a save point
-        gbar(g);
-        if (tg < GS) q.flag[tg] = 0;
-        gbar(g);
-        if (anyhit) q.flag[0] = 1;
-        gbar(g);
-        if (q.flag[0]) save_point_loss_tc(q, a, u, o, hit, Lslot, ty, tx, g, tg);
-      }
+      ++kk;
+      next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
     }
   }
-  bool dw_started = false;
-  Blk<T> lam = bzero<T>(), bbar = bzero<T>();
-  if (GRAD) {
-    if (tg < GS) {
-      const int64_t j = base + tg;
-      if (j < n) {
-        const int64_t i = a.order[j];
-        if (i >= 0 && i < n) {
-          const bool ok = a.status[j] == GS_TRAJ_OK && a.nsteps[j] >= 0 && a.nsteps[j] <= a.smax;
-          a.loss[i] = ok ? Lslot : nan;
-        }
-      }
-    }
-    // ---------------------------------------------------------------- reverse
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      kk[c] = a.nsave - 1;
-      next[c] = act[c] && S[c] > 0 ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
-    }
-    for (int st = Smax - 1; st >= 0; --st) {
-      T hh[2];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        if (st + 1 == next[c]) {
-          const int64_t o = (int64_t)kk[c] * n64 + traj[c];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int64_t oo = o + (int64_t)(4 * ty + k) * n;
-            if (a.loss_kind == GS_LOSS_SUMSQ)
-              lam.v[k][c] = fmaT(cst<T>(2.0), a.target ? u.v[k][c] - a.target[oo] : u.v[k][c], lam.v[k][c]);
-            else
-              lam.v[k][c] += a.weight[oo];
-          }
-          --kk[c];
-          next[c] = kk[c] >= 0 ? a.save_idx[(int64_t)kk[c] * n + base + 2 * tx + c] : -1;
-        }
-        const bool run = st < S[c];
-        hh[c] = run ? a.h[(int64_t)st * n + base + 2 * tx + c] : cst<T>(0.0);
-        if (run) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            u.v[k][c] = a.ck[(int64_t)st * n64 + (int64_t)(4 * ty + k) * n + base + 2 * tx + c];
-        }
-      }
-      Blk<T> U1 = u, U2, U3, U4, U5, U6, y1, y2, y3, y4, y5, y6, kd;
-      eval_f_tc(s, q, phase, U1, bias, y1, kd, ty, tx, g, tg);
-      Blk<T> k1 = kd;
-      {
-        const T c[1] = {cst<T>(TS_A21)};
-        const Blk<T>* const ks[1] = {&k1};
-        U2 = stage<T, 1>(c, ks, U1, hh);
-      }
-      eval_f_tc(s, q, phase, U2, bias, y2, kd, ty, tx, g, tg);
-      Blk<T> k2 = kd;
-      {
-        const T c[2] = {cst<T>(TS_A31), cst<T>(TS_A32)};
-        const Blk<T>* const ks[2] = {&k1, &k2};
-        U3 = stage<T, 2>(c, ks, U1, hh);
-      }
-      eval_f_tc(s, q, phase, U3, bias, y3, kd, ty, tx, g, tg);
-      Blk<T> k3 = kd;
-      {
-        const T c[3] = {cst<T>(TS_A41), cst<T>(TS_A42), cst<T>(TS_A43)};
-        const Blk<T>* const ks[3] = {&k1, &k2, &k3};
-        U4 = stage<T, 3>(c, ks, U1, hh);
-      }
-      eval_f_tc(s, q, phase, U4, bias, y4, kd, ty, tx, g, tg);
-      Blk<T> k4 = kd;
-      {
-        const T c[4] = {cst<T>(TS_A51), cst<T>(TS_A52), cst<T>(TS_A53), cst<T>(TS_A54)};
-        const Blk<T>* const ks[4] = {&k1, &k2, &k3, &k4};
-        U5 = stage<T, 4>(c, ks, U1, hh);
-      }
-      eval_f_tc(s, q, phase, U5, bias, y5, kd, ty, tx, g, tg);
-      Blk<T> k5 = kd;
-      {
-        const T c[5] = {cst<T>(TS_A61), cst<T>(TS_A62), cst<T>(TS_A63), cst<T>(TS_A64), cst<T>(TS_A65)};
-        const Blk<T>* const ks[5] = {&k1, &k2, &k3, &k4, &k5};
-        U6 = stage<T, 5>(c, ks, U1, hh);
-      }
-      eval_f_tc(s, q, phase, U6, bias, y6, kd, ty, tx, g, tg);
-
-      Blk<T> mu[6];
-      const Blk<T>* Ys[6] = {&y1, &y2, &y3, &y4, &y5, &y6};
-      const Blk<T>* Us[6] = {&U1, &U2, &U3, &U4, &U5, &U6};
-      const double bw[6] = {TS_B1, TS_B2, TS_B3, TS_B4, TS_B5, TS_B6};
-      const double aw[6][6] = {{0, 0, 0, 0, 0, 0},
-                               {TS_A21, 0, 0, 0, 0, 0},
-                               {TS_A31, TS_A32, 0, 0, 0, 0},
-                               {TS_A41, TS_A42, TS_A43, 0, 0, 0},
-                               {TS_A51, TS_A52, TS_A53, TS_A54, 0, 0},
-                               {TS_A61, TS_A62, TS_A63, TS_A64, TS_A65, 0}};
-#pragma unroll
-      for (int jj = 5; jj >= 0; --jj) {
-        Blk<T> nu, gg;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            T acc = cst<T>(bw[jj]) * lam.v[k][c];
-#pragma unroll
-            for (int m = 5; m > jj; --m) acc = fmaT(cst<T>(aw[m][jj]), mu[m].v[k][c], acc);
-            nu.v[k][c] = hh[c] * acc;
-            const T yv = Ys[jj]->v[k][c];
-            gg.v[k][c] = nu.v[k][c] * fmaT(-yv, yv, cst<T>(1.0));
-            bbar.v[k][c] += gg.v[k][c];
-          }
-        gbar(g);  // previous readers of the operand tiles and of Z are done
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int r = 4 * ty + k, t = 2 * tx + c;
-            tc::put(q.Thi, q.Tlo, tc::off(t, r, GS), gg.v[k][c]);
-            tc::put(q.GChi, q.GClo, tc::off(r, t, D), gg.v[k][c]);
-            tc::put(q.UEhi, q.UElo, tc::off(r, t, D), Us[jj]->v[k][c]);
-          }
-        tc_publish(g);
-        if (tg == 0 && !q.failed) {
-          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          // W^T g (M = 64, N = 16) and dW += G U^T (M = 64, N = 64, K = 16 slots)
-          tc::mma3(s.tmem + 16 * g, tc::smem_u32(s.WThi), tc::smem_u32(s.WTlo), 1024, tc::smem_u32(q.Thi),
-                   tc::smem_u32(q.Tlo), 256, 8, tc::idesc(64, 16), 0u);
-          tc::mma3(s.tmem + 32 + 64 * g, tc::smem_u32(q.GChi), tc::smem_u32(q.GClo), 1024, tc::smem_u32(q.UEhi),
-                   tc::smem_u32(q.UElo), 1024, 2, tc::idesc(64, 64), dw_started ? 1u : 0u);
-          tc_commit(q);
-        }
-        dw_started = true;
-        tc_wait(q, phase);
-        tc_stage_out(s, q, g, tg);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) mu[jj].v[k][c] = q.Z[4 * ty + k][2 * tx + c] - nu.v[k][c];
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          lam.v[k][c] += ((mu[0].v[k][c] + mu[1].v[k][c]) + (mu[2].v[k][c] + mu[3].v[k][c])) +
-                         (mu[4].v[k][c] + mu[5].v[k][c]);
-    }
-  }
-  // a group whose MMAs did not complete has no valid results
-  const bool bad = q.failed != 0;
+  const bool bad0 = s.failed != 0;
   if (!GRAD) {
+    if ((!act || bad0) && traj >= 0)
+      for (int k = 0; k < a.nsave; ++k)
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
-      if ((!act[c] || bad) && traj[c] >= 0)
-        for (int k = 0; k < a.nsave; ++k)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) a.u_save[(int64_t)k * n64 + (int64_t)(4 * ty + r) * n + traj[c]] = nan;
+        for (int c = 0; c < HC; ++c) a.u_save[(int64_t)k * n64 + (int64_t)(c0 + c) * n + traj] = nan;
   } else {
+    if (hf == 1) s.lpart[t] = Lh;
+    __syncthreads();
+    if (hf == 0 && traj >= 0) a.loss[traj] = (act && !bad0) ? Lh + s.lpart[t] : nan;
+
+    // -------------------------------------------------------------- reverse
+    // u holds u_{st+1} at the top of iteration st
+    T lam[HC], bbar[HC];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      if (traj[c] < 0) continue;
-      const bool ok = act[c] && !bad;
-      if (bad && ty == 0) a.loss[traj[c]] = nan;
+    for (int c = 0; c < HC; ++c) lam[c] = bbar[c] = cst<T>(0.0);
+    uint32_t dw_acc = 0;  // 1 once the dW accumulator holds a product
+    kk = a.nsave - 1;
+    next = act && S > 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
+    for (int st = Smax - 1; st >= 0; --st) {
+      if (st + 1 == next) {
+        const int64_t o = (int64_t)kk * n64 + traj;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        a.dp[(int64_t)(4 * ty + r) * n + traj[c]] = ok ? bbar.v[r][c] : nan;
-        a.du0[(int64_t)(4 * ty + r) * n + traj[c]] = ok ? lam.v[r][c] : nan;
+        for (int c = 0; c < HC; ++c) {
+          const int64_t oo = o + (int64_t)(c0 + c) * n;
+          if (a.loss_kind == GS_LOSS_SUMSQ)
+            lam[c] = fmaT(cst<T>(2.0), a.target ? u[c] - a.target[oo] : u[c], lam[c]);
+          else
+            lam[c] += a.weight[oo];
+        }
+        --kk;
+        next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
+      }
+      const bool run = st < S;
+      const T h = run ? a.h[(int64_t)st * n + j] : cst<T>(0.0);
+      if (run) {
+#pragma unroll
+        for (int c = 0; c < HC; ++c) u[c] = a.ck[(int64_t)st * n64 + (int64_t)(c0 + c) * n + j];
+      }
+      // recompute the stage slopes k_1..k_6 of step st into the slots
+      fwd_stage<1>(s, tid, t, c0, phase, tl, h, u, bias);
+      fwd_stage<2>(s, tid, t, c0, phase, tl, h, u, bias);
+      fwd_stage<3>(s, tid, t, c0, phase, tl, h, u, bias);
+      fwd_stage<4>(s, tid, t, c0, phase, tl, h, u, bias);
+      fwd_stage<5>(s, tid, t, c0, phase, tl, h, u, bias);
+      fwd_stage<6>(s, tid, t, c0, phase, tl, h, u, bias);
+
+      // transposed step, stages 6 .. 1:
+      //   nu_j = h (b_j lambda + sum_{m>j} a_mj mu_m), g_j = nu_j (1 - y_j^2),
+      //   y_j = k_j + U_j, mu_j = W^T g_j - nu_j, bbar += g_j, dW += g_j U_j^T.
+      // Element-wise work runs in two passes of 16 columns; slot j takes g_j
+      // once k_j is spent, and mu_j after the VJP (nu_j and U_j are recomputed
+      // from the slots where they are needed again, which keeps them out of
+      // registers across the waits).
+#pragma unroll 1
+      for (int jj = 5; jj >= 0; --jj) {
+#pragma unroll
+        for (int qh = 0; qh < 2; ++qh) {
+          T nu[16], Uq[16], v[16];
+          sweep_nu(tl, jj, qh, h, lam, nu);
+          sweep_U(tl, jj, qh, h, u, Uq);
+          ld16(tl + kColSlot + 64 * jj + 16 * qh, v);  // k_j
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const T y = v[c] + Uq[c];
+            v[c] = nu[c] * fmaT(-y, y, cst<T>(1.0));  // g_j
+            bbar[16 * qh + c] += v[c];
+          }
+          st16(tl + kColSlot + 64 * jj + 16 * qh, v);
+          put_rows16(s, t, c0 + 16 * qh, v);
+          if (t < TT / 2) put_cols16(s, t, c0 + 16 * qh, v, Uq);
+        }
+        publish();
+        if (tid == 0 && !s.failed) {
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          tc::mma3(s.tmem + kColAcc, tc::smem_u32(s.Thi), tc::smem_u32(s.Tlo), kChunkT, tc::smem_u32(s.WThi),
+                   tc::smem_u32(s.WTlo), kChunkW, D / 8, tc::idesc(TT, D), 0u);
+          tc::mma3(s.tmem + kColDW, tc::smem_u32(s.GChi), tc::smem_u32(s.GClo), kChunkC, tc::smem_u32(s.UEhi),
+                   tc::smem_u32(s.UElo), kChunkC, TT / 2 / 8, tc::idesc(D, D), dw_acc);
+          commit(s);
+        }
+        dw_acc = 1u;
+        wait(s, phase);
+        // the upper half of dW (its trajectories' g_j from slot j, U_j again)
+        if (t >= TT / 2) {
+#pragma unroll
+          for (int qh = 0; qh < 2; ++qh) {
+            T g[16], Uq[16];
+            ld16(tl + kColSlot + 64 * jj + 16 * qh, g);
+            sweep_U(tl, jj, qh, h, u, Uq);
+            put_cols16(s, t - TT / 2, c0 + 16 * qh, g, Uq);
+          }
+        }
+        publish();
+        if (tid == 0 && !s.failed) {
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          tc::mma3(s.tmem + kColDW, tc::smem_u32(s.GChi), tc::smem_u32(s.GClo), kChunkC, tc::smem_u32(s.UEhi),
+                   tc::smem_u32(s.UElo), kChunkC, TT / 2 / 8, tc::idesc(D, D), 1u);
+          commit(s);
+        }
+        // mu_j = W^T g_j - nu_j (the VJP completed at the previous wait)
+#pragma unroll
+        for (int qh = 0; qh < 2; ++qh) {
+          T nu[16], v[16];
+          sweep_nu(tl, jj, qh, h, lam, nu);
+          ld16(tl + kColAcc + 16 * qh, v);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) v[c] = v[c] - nu[c];
+          st16(tl + kColSlot + 64 * jj + 16 * qh, v);
+        }
+        wait(s, phase);  // the upper-half dW products have read G^T / U^T
+      }
+      // lambda += ((mu_1 + mu_2) + (mu_3 + mu_4)) + (mu_5 + mu_6)
+#pragma unroll
+      for (int qh = 0; qh < 2; ++qh) {
+        T m1[16], m3[16], v[16];
+        ld16(tl + kColSlot + 16 * qh, m1);
+        ld16(tl + kColSlot + 64 + 16 * qh, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) m1[c] = m1[c] + v[c];
+        ld16(tl + kColSlot + 128 + 16 * qh, m3);
+        ld16(tl + kColSlot + 192 + 16 * qh, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) m3[c] = m3[c] + v[c];
+        ld16(tl + kColSlot + 256 + 16 * qh, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) m1[c] = m1[c] + m3[c], m3[c] = v[c];
+        ld16(tl + kColSlot + 320 + 16 * qh, v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) lam[16 * qh + c] += m1[c] + (m3[c] + v[c]);
       }
     }
-    // the group's weight-gradient partial: warp 4g + w reads rows 16w..16w+15
-    T* part = a.dW_part + ((int64_t)blockIdx.x * 2 + g) * D * D;
-    const int w = tg >> 5, lane = tg & 31;
-    float v0[16], v1[16], v2[16], v3[16];
-    const uint32_t ta = s.tmem + ((uint32_t)(32 * w) << 16) + (uint32_t)(32 + 64 * g);
-    if (dw_started && !bad) {
-      ld16(ta, v0);
-      ld16(ta + 16, v1);
-      ld16(ta + 32, v2);
-      ld16(ta + 48, v3);
+    const bool bad = s.failed != 0;
+    if (traj >= 0) {
+#pragma unroll
+      for (int c = 0; c < HC; ++c) {
+        a.dp[(int64_t)(c0 + c) * n + traj] = act && !bad ? bbar[c] : nan;
+        a.du0[(int64_t)(c0 + c) * n + traj] = act && !bad ? lam[c] : nan;
+      }
     }
+    // the CTA's weight-gradient partial: warp w reads rows 16 (w mod 4) .. + 15,
+    // columns [32 (w / 4), + 32)
+    T* part = a.dW_part + (int64_t)blockIdx.x * D * D;
+    T v[HC];
+#pragma unroll
+    for (int c = 0; c < HC; ++c) v[c] = cst<T>(0.0);
+    if (dw_acc && !bad) load32(s.tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kColDW + (uint32_t)c0, v);
     if (lane < 16) {
-      const int row = 16 * w + lane;
-      const bool z = !dw_started;
+      const int row = 16 * (warp & 3) + lane;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        part[row * D + c] = bad ? nan : (z ? cst<T>(0.0) : v0[c]);
-        part[row * D + 16 + c] = bad ? nan : (z ? cst<T>(0.0) : v1[c]);
-        part[row * D + 32 + c] = bad ? nan : (z ? cst<T>(0.0) : v2[c]);
-        part[row * D + 48 + c] = bad ? nan : (z ? cst<T>(0.0) : v3[c]);
-      }
+      for (int c = 0; c < HC; ++c) part[row * D + c0 + c] = bad ? nan : v[c];
     }
   }
-  // no MMA in flight and every TMEM read done before the columns are freed
-  if (bad && tg == 0) {
+  // no MMA in flight and every TMEM access done before the columns are freed
+  if (s.failed && tid == 0) {
     uint32_t done = 0;
     for (int it = 0; it < tc::kSpin && !done; ++it)
       asm volatile(
           "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
           "selp.b32 %0, 1, 0, P1;\n\t}\n"
           : "=r"(done)
-          : "r"(tc::smem_u32(&q.bar)), "r"(phase ^ 1u)
+          : "r"(tc::smem_u32(&s.bar)), "r"(phase ^ 1u)
           : "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(s.tmem));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(s.tmem));
   }
 }
+
+}  // namespace t128
 
 }  // namespace n64
 
 // Which products the d = 64 replay and gradient use (process-wide, set by
-// gs_set_option): the SIMT FP32 products (default, faster at 32 slots per CTA)
-// or the tcgen05 3xTF32 products.
-static std::atomic<int> g_node64_tensor{0};
+// gs_set_option): the tcgen05 3xTF32 products with 128 trajectories per CTA
+// (default) or the SIMT FP32 products, the recorder's own arithmetic.
+static std::atomic<int> g_node64_tensor{1};
 void node64_set_tensor(int on) { g_node64_tensor.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize) {
   const int64_t nblk = (n + n64::TB - 1) / n64::TB;
   const size_t ck = ((size_t)smax * 64 * n * tsize + 255) / 256 * 256;
-  return ck + (size_t)nblk * 2 * 64 * 64 * tsize;  // up to two weight-gradient partials per CTA
+  return ck + (size_t)nblk * 64 * 64 * tsize;  // one weight-gradient partial per CTA (fewer CTAs with tensor cores)
 }
 
 template <typename T>
@@ -1482,12 +1485,13 @@ gs_status node64_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, 
   const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
   a.dW_part = (T*)((char*)ws + ((size_t)M->smax * 64 * P->n * sizeof(T) + 255) / 256 * 256);
   const bool tensor = g_node64_tensor.load(std::memory_order_relaxed) != 0;
+  const int nblk128 = (int)((P->n + n64::t128::TT - 1) / n64::t128::TT);
   if (tensor) {
-    const size_t smem = sizeof(n64::SmemTC) + 128;
-    if (cudaFuncSetAttribute(n64::k_replay_node64_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = sizeof(n64::t128::Smem);
+    if (cudaFuncSetAttribute(n64::t128::k_node64_t128<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return GS_ECUDA;
-    n64::k_replay_node64_tc<true><<<nblk, n64::NT, smem, st>>>(a);
+    n64::t128::k_node64_t128<true><<<nblk128, n64::t128::NT, smem, st>>>(a);
   } else {
     const size_t smem = sizeof(n64::Smem<T>);
     if (cudaFuncSetAttribute(n64::k_replay_node64<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1498,7 +1502,7 @@ gs_status node64_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, 
   count_launch();
   if (!launch_ok()) return GS_ECUDA;
   if (dshared) {
-    n64::k_reduce_dW<T><<<(64 * 64 + 255) / 256, 256, 0, st>>>(a.dW_part, tensor ? 2 * nblk : nblk,
+    n64::k_reduce_dW<T><<<(64 * 64 + 255) / 256, 256, 0, st>>>(a.dW_part, tensor ? nblk128 : nblk,
                                                                 (T*)dshared);
     count_launch();
   }
@@ -1511,11 +1515,12 @@ gs_status node64_solve(const gs_problem* P, const gs_mesh* M, void* u_save, cuda
   a.u_save = (T*)u_save;
   const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
   if (g_node64_tensor.load(std::memory_order_relaxed) != 0) {
-    const size_t smem = sizeof(n64::SmemTC) + 128;
-    if (cudaFuncSetAttribute(n64::k_replay_node64_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = sizeof(n64::t128::Smem);
+    if (cudaFuncSetAttribute(n64::t128::k_node64_t128<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return GS_ECUDA;
-    n64::k_replay_node64_tc<false><<<nblk, n64::NT, smem, st>>>(a);
+    n64::t128::k_node64_t128<false><<<(unsigned)((P->n + n64::t128::TT - 1) / n64::t128::TT), n64::t128::NT,
+                                       smem, st>>>(a);
   } else {
     const size_t smem = sizeof(n64::Smem<T>);
     if (cudaFuncSetAttribute(n64::k_replay_node64<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,

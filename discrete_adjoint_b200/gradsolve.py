@@ -300,7 +300,7 @@ OPT_NODE64_TENSOR_CORES = 1
 
 def gs_set_option(option: int, value: int) -> None:
     """Process-wide option (OPT_NODE64_TENSOR_CORES: 1 = the d = 64 products on
-    the tensor cores, 0 = SIMT, the default)."""
+    the tensor cores, the default; 0 = SIMT, the recorder's arithmetic)."""
     _check(_lib.gs_set_option(option, value), "gs_set_option")
 
 

@@ -1,8 +1,8 @@
 """GPU <-> oracle parity for the d = 64 shared-weight system (workload
 node64, fp32): recorder, forward solve, per-trajectory gradients dL/db_i and
 dL/du0_i on the same mesh, and the ensemble weight gradient dL/dW -- with the
-stage products in FP32 SIMT (the default) and on the tensor cores (tcgen05,
-3xTF32)."""
+stage products on the tensor cores (tcgen05, 3xTF32, 128 trajectories per
+CTA: the default) and in FP32 SIMT."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 def products(request):
     gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, int(request.param == "tensor"))
     yield request.param
-    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, 0)
+    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, 1)
 
 
 @pytest.fixture(scope="module", params=[512, 100])
@@ -108,7 +108,7 @@ def test_tensor_core_products_match_simt():
         o = gs.gs_grad(ens, mesh, **loss_args(prob))
         torch.cuda.synchronize()
         outs.append([t.double().cpu().numpy() for t in (o.loss, o.dp, o.du0, o.dshared)])
-    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, 0)
+    gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, 1)
     for a, b in zip(*outs):
         assert np.isfinite(b).all()
         assert np.abs(a - b).max() <= 1e-4 * np.abs(a).max()
