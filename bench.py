@@ -456,6 +456,29 @@ def run_single(args):
         print(json.dumps(line), flush=True)
 
 
+def tensor_roofline(alu, total_steps, grad_ms):
+    """Roofline of the d = 64 gradient with its products on the tensor cores:
+    the algorithmic product work (forward W U: 6, transposed step W^T g and
+    g U^T: 12 products of 64 x 64 per replay step, 2 flops per multiply-add,
+    fp32 accuracy) against the TF32 dense peak, taken as the measured bf16
+    GEMM peak (MEASURED_PEAKS.json, burst) times the nominal TF32 / bf16 ratio
+    1.1 / 2.25.  The 3xTF32 split issues three TF32 products per fp32 one;
+    those are implementation, not algorithmic work.  The ALU form (all
+    algorithmic flops against the FP32 peak) is kept beside it."""
+    gemm = 18 * 64 * 64 * 2 * total_steps
+    try:
+        bf16 = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] * 1e12
+        src = "measured bf16 %.1f TF/s x 1.1/2.25 (nominal TF32/bf16)" % (bf16 / 1e12)
+    except Exception:
+        bf16 = 1.59e15
+        src = "fallback bf16 1590 TF/s x 1.1/2.25 (nominal TF32/bf16)"
+    peak = bf16 * 1.1 / 2.25
+    achieved = gemm / (grad_ms / 1e3)
+    return {"bound": "tensor", "achieved": achieved / 1e12, "peak": peak / 1e12, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None, "kernel": "k_node64_t128", "peak_source": src,
+            "flops_per_launch": gemm, "alu": {k: alu[k] for k in ("achieved", "peak", "frac", "flops_per_launch")}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -624,6 +647,8 @@ def run_ours(args):
                          64 if args.dtype == "f64" else 128, "FP64" if args.dtype == "f64" else "FP32"),
                      "flops_per_launch": flops},
     }
+    if args.workload == "node64" and args.products == "tensor":
+        line["roofline"] = tensor_roofline(line["roofline"], total_steps, grad_ms)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # samples sized for seconds of host work (and host memory for the
         # oracle's trajectory-major meshes)
