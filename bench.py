@@ -92,6 +92,15 @@ WORKLOADS = {
     # state (192) + 6 input directions x (tangent stage combinations 144 +
     # six Jacobian-vector products 108); the per-thread copies of the state
     # (one per direction) are not counted
+    # forward sensitivities of the ROS3 replay on the robertson ensemble: the
+    # state (142) + 6 directions x the tangent step (207: two JVPs, three
+    # directional Jacobian products dJ k, three solves, the combinations; hand
+    # count); the per-direction copies of the state are not counted
+    "robertson_ros3_sens": dict(kind="sens", problem="robertson", method="ros3", flop_step=142 + 6 * 207,
+                                kernel="k_sens_ros", n=65536, dtype="f64",
+                                desc="Robertson d=3, t in [0,1e5], ROS3, rtol=1e-6 atol=1e-10, loss w . u(T); one "
+                                     "forward-sensitivity pass per step on the recorded mesh (d u(T)/d(p,u0) + the "
+                                     "loss gradient)"),
     "lorenz_1m_sens": dict(kind="sens", problem="lorenz_1m", flop_step=192 + 6 * 252, kernel="k_sens_tsit5_lorenz",
                            n=1 << 20, dtype="f64",
                            desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, 10 save points with N(0,1) targets; "
@@ -132,6 +141,8 @@ def metric_name(args) -> str:
         return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, dense save points)"
     if args.workload == "lorenz_1m_sens":
         return f"trajectory-sensitivities/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, forward mode)"
+    if args.workload == "robertson_ros3_sens":
+        return f"trajectory-sensitivities/s (Robertson ROS3 {args.dtype.replace('f', 'fp')}, forward mode)"
     if args.workload == "lorenz_1m_solve":
         return f"trajectory-solves/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, adaptive forward-only)"
     if args.workload == "lorenz_1m":
@@ -261,7 +272,8 @@ def run_reference(args):
     kind = W.get("kind", "grad")
     solve = kind != "grad"
     sample = {"lorenz_1m": 256, "lorenz_1m_dense": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
-              "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512, "robertson_ros3": 256}[args.workload]
+              "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512, "robertson_ros3": 256,
+              "robertson_ros3_sens": 256}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
     om = oracle.record(prob, smax_cap(args.workload), nthreads=threads) if kind == "sens" else None
@@ -338,6 +350,8 @@ def run_single(args):
     host = {"p": pin(prob.p), "u0": pin(prob.u0)}
     if kind == "sens" and prob.target is not None:
         host["target"] = pin(prob.target)
+    if kind == "sens" and prob.weight is not None:
+        host["weight"] = pin(prob.weight)
     d = {k: v.to(dev) for k, v in host.items()}
     ens = gs.Ensemble(prob.system, prob.method, args.dtype, d["p"], d["u0"], prob.t0, prob.t1,
                       [float(x) for x in prob.tsave])
@@ -371,7 +385,8 @@ def run_single(args):
         work = {"replay_steps": total_steps, "sens_gb": sens.numel() * esz / 1e9}
 
         def step():
-            gs.gs_sens(ens, mesh, loss=prob.loss, target=d.get("target"), out=out, sens=sens, stream=stream)
+            gs.gs_sens(ens, mesh, loss=prob.loss, target=d.get("target"), weight=d.get("weight"), out=out, sens=sens,
+                       stream=stream)
 
     def barrier():
         if world > 1:

@@ -255,10 +255,12 @@ GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_l
  *            theta = (p_0 .. p_{np-1}, u0_0 .. u0_{d-1}); may be NULL
  *   loss, dp, du0: as gs_grad (dL/dp and dL/du0 by the chain rule through the
  *            tangents)
- * Needs no workspace.  Slots with status != 0 get NaN everywhere.  Built for
- * GS_LORENZ with GS_TSIT5 (np + d = 6), fp64 and fp32; other problems return
- * GS_EUNSUPPORTED.  (The few-parameter forward-sensitivity route that the
- * gptget summary sets beside the adjoint.)
+ * Needs no workspace.  Slots with status != 0 (or whose Rosenbrock matrix
+ * turns singular) get NaN everywhere.  Built for GS_LORENZ with GS_TSIT5, and
+ * for GS_LORENZ and GS_ROBERTSON with GS_ROS2 or GS_ROS3 (np + d = 6), fp64
+ * and fp32, on landing meshes; other problems, and meshes with dense save
+ * points, return GS_EUNSUPPORTED.  (The few-parameter forward-sensitivity
+ * route that the gptget summary sets beside the adjoint.)
  */
 GS_API gs_status gs_sens(const gs_problem* prob, const gs_mesh* mesh, const gs_loss* loss_desc, void* loss, void* dp,
                          void* du0, void* sens, void* stream);

@@ -110,11 +110,12 @@ def test_bad_tolerance_and_workspace_rejected():
                                   None) == -1
     assert _lib.gs_solve_adaptive(ctypes.byref(p), ctypes.byref(_Tol(0.0, 0.0, 0.0)), 100, ctypes.c_void_p(16),
                                   None, None, None) == -1
-    # forward sensitivities: Lorenz with Tsit5 only, and the gradient outputs are required
+    # forward sensitivities: Tsit5 on Lorenz, ROS2 / ROS3 on both d = 3 systems;
+    # the gradient outputs are required
     ls = _Loss(1, None, None)
     assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(m), ctypes.byref(ls), None, ctypes.c_void_p(16),
                         ctypes.c_void_p(16), None, None) == -1
-    rob = _host_problem(system=2, method=2)
+    rob = _host_problem(system=2, method=1)
     assert _lib.gs_sens(ctypes.byref(rob), ctypes.byref(m), ctypes.byref(ls), ctypes.c_void_p(16),
                         ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == -4
     # mesh nsave must match
@@ -148,15 +149,17 @@ def test_set_option_host_only():
 
 def test_ros3_method_validation_host_only():
     """ROS3 (method 3) is accepted for the d = 3 systems and refused where it is
-    not built: forward sensitivities, dense save points, the d = 64 system; an
-    unknown method is an invalid argument.  No call here reaches a launch."""
+    not built: dense save points (records and sensitivities); an unknown method
+    is an invalid argument.  No call here reaches a launch."""
     from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
     m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
     ls = _Loss(1, None, None)
     for system in (1, 2):
         p = _host_problem(system=system, method=3)
         assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 1) == 100 * 3 * 1000 * 8
-        assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(m), ctypes.byref(ls), ctypes.c_void_p(16),
+        md = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+        md.save_theta = 16
+        assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(md), ctypes.byref(ls), ctypes.c_void_p(16),
                             ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == -4
         dense = _Tol(1e-6, 1e-6, 0.0)
         dense.dense = 1

@@ -18,19 +18,16 @@ import pytest
 
 import oracle
 import workloads as W
-from test_oracle_method import _dpoly, _kappa, _poly, _ros2_R, _tsit5_R_coeffs
+from test_oracle_method import _R_any, _kappa
 
 EPS = np.finfo(np.float64).eps
 
 
-def _R_dR(method, z):
-    if method == "tsit5":
-        co = _tsit5_R_coeffs()
-        return _poly(co, z), _dpoly(co, z)
-    return _ros2_R(z, Fr(oracle.ros2_gamma()))
+_R_dR = _R_any
 
 
-@pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 400.0])])
+@pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 400.0]),
+                                         ("ros3", [0.5, 50.0, 400.0])])
 def test_closed_form_on_the_test_equation(method, lams):
     prob = W.scalar_linear([-l for l in lams], t1=2.0, method=method)
     prob.tsave = np.array([0.25, 1.0, 2.0])
