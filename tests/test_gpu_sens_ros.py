@@ -84,3 +84,27 @@ def test_failed_and_ragged():
     assert np.isnan(out.dp.cpu().numpy()[:, 7]).all() and np.isnan(out.du0.cpu().numpy()[:, 7]).all()
     keep = np.arange(prob.n) != 7
     assert np.array_equal(S[..., keep], S0[..., keep])
+
+
+def test_full_size_sampled():
+    """The 65,536-trajectory robertson ensemble with ROS3 in the benchmark's
+    launch configuration; the oracle's dual numbers check a sample."""
+    from gpu_util import dev
+    prob = _prob("robertson", "ros3", None)
+    ens = ensemble(prob)
+    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, 20000)
+    mesh = gs.new_mesh(prob.n, int(nsteps.max().item()), 1, "f64", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    out, S = gs.gs_sens(ens, mesh, **loss_args(prob))
+    torch.cuda.synchronize()
+    assert (mesh.status == 0).all()
+    from gpu_util import mesh_by_trajectory
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    rng = np.random.default_rng(10)
+    idx = np.unique(np.concatenate([rng.choice(prob.n, 64, replace=False), np.argsort(ns)[-8:]]))
+    sub = prob.subset(idx)
+    om = oracle.Mesh(h[idx].astype(np.float64), ns[idx], si[idx], st[idx], np.zeros(len(idx), np.int32))
+    ref = oracle.sens(sub, om)
+    got = S[..., torch.tensor(idx, device=dev())].double().cpu().numpy()
+    e = np.abs(got - ref).max(axis=(0, 1, 2)) / np.abs(ref).max(axis=(0, 1, 2))
+    assert e.max() <= max(1e-12, 8 * EPS * ns.max()), e.max()
