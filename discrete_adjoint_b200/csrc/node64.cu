@@ -984,7 +984,8 @@ __device__ __forceinline__ void publish() {
   __syncthreads();
 }
 
-__device__ __forceinline__ void commit(Smem& s) {
+template <typename SM>
+__device__ __forceinline__ void commit(SM& s) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    tc::smem_u32(&s.bar))
                : "memory");
@@ -992,7 +993,8 @@ __device__ __forceinline__ void commit(Smem& s) {
 
 // Wait for the next completion of the CTA's mbarrier (bounded; a timeout
 // marks the CTA failed, after which no MMA is issued and no wait spins).
-__device__ __forceinline__ void wait(Smem& s, uint32_t& phase) {
+template <typename SM>
+__device__ __forceinline__ void wait(SM& s, uint32_t& phase) {
   if (!s.failed) {
     uint32_t done = 0;
     for (int it = 0; it < tc::kSpin && !done; ++it)
@@ -1008,14 +1010,14 @@ __device__ __forceinline__ void wait(Smem& s, uint32_t& phase) {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Z (or the VJP) for the CTA: ACC = T B^T with B = W (vjp = false) or W^T.
-__device__ __forceinline__ void product(Smem& s, int tid, uint32_t& phase, bool vjp) {
+// Z for the CTA: ACC = T W^T (Z[t][r] = sum_k U[t][k] W[r][k]).
+template <typename SM>
+__device__ __forceinline__ void product(SM& s, int tid, uint32_t& phase) {
   publish();
   if (tid == 0 && !s.failed) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    tc::mma3(s.tmem + kColAcc, tc::smem_u32(s.Thi), tc::smem_u32(s.Tlo), kChunkT,
-             tc::smem_u32(vjp ? s.WThi : s.Whi), tc::smem_u32(vjp ? s.WTlo : s.Wlo), kChunkW, D / 8,
-             tc::idesc(TT, D), 0u);
+    tc::mma3(s.tmem + kColAcc, tc::smem_u32(s.Thi), tc::smem_u32(s.Tlo), kChunkT, tc::smem_u32(s.Whi),
+             tc::smem_u32(s.Wlo), kChunkW, D / 8, tc::idesc(TT, D), 0u);
     commit(s);
   }
   wait(s, phase);
@@ -1038,7 +1040,8 @@ __device__ __forceinline__ void st16(uint32_t taddr, const float (&v)[16]) {
 }
 
 // 16 components [k0, k0 + 16) of a trajectory-row operand (hi / lo).
-__device__ __forceinline__ void put_rows16(Smem& s, int t, int k0, const float (&x)[16]) {
+template <typename SM>
+__device__ __forceinline__ void put_rows16(SM& s, int t, int k0, const float (&x)[16]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     float4 h, l;
@@ -1058,10 +1061,12 @@ __device__ __forceinline__ void put_rows16(Smem& s, int t, int k0, const float (
 
 // Stage J's state U = fma(h, sum_{m<J} a_Jm k_m, u) (the contract's order;
 // J = 1: U = u, J = 7: u_{s+1}) into the A operand and, to wait out the
-// product, into its slot (J = 7: slot 1, whose k_1 this pass has read);
-// 16 columns per pass.  For J = 7, u becomes u_{s+1}.
-template <int J>
-__device__ __forceinline__ void stage_in(Smem& s, uint32_t tl, int t, int c0, float h, float (&u)[HC]) {
+// product, into slot `dst`; k_1 is read from slot s1, k_2..k_6 from slots
+// 2..6; 16 columns per pass (a pass reads only its own columns, so dst may
+// be s1).  For J = 7, un receives u_{s+1} (un may be u).
+template <int J, typename SM>
+__device__ __forceinline__ void stage_in(SM& s, uint32_t tl, int t, int c0, float h, const float (&u)[HC],
+                                         float (&un)[HC], int s1, int dst) {
   constexpr double A[8][7] = {{0, 0, 0, 0, 0, 0, 0},
                               {0, 0, 0, 0, 0, 0, 0},
                               {TS_A21, 0, 0, 0, 0, 0, 0},
@@ -1070,7 +1075,6 @@ __device__ __forceinline__ void stage_in(Smem& s, uint32_t tl, int t, int c0, fl
                               {TS_A51, TS_A52, TS_A53, TS_A54, 0, 0, 0},
                               {TS_A61, TS_A62, TS_A63, TS_A64, TS_A65, 0, 0},
                               {TS_B1, TS_B2, TS_B3, TS_B4, TS_B5, TS_B6, 0}};
-  constexpr int slot = J <= 6 ? J : 1;
 #pragma unroll
   for (int qh = 0; qh < 2; ++qh) {
     float U[16], v[16];
@@ -1078,7 +1082,7 @@ __device__ __forceinline__ void stage_in(Smem& s, uint32_t tl, int t, int c0, fl
 #pragma unroll
       for (int c = 0; c < 16; ++c) U[c] = u[16 * qh + c];
     } else {
-      ld16(tl + kColSlot + 16 * qh, v);
+      ld16(tl + kColSlot + 64 * (s1 - 1) + 16 * qh, v);
 #pragma unroll
       for (int c = 0; c < 16; ++c) U[c] = cst<float>(A[J][0]) * v[c];
 #pragma unroll
@@ -1091,10 +1095,10 @@ __device__ __forceinline__ void stage_in(Smem& s, uint32_t tl, int t, int c0, fl
       for (int c = 0; c < 16; ++c) U[c] = fmaT(h, U[c], u[16 * qh + c]);
     }
     put_rows16(s, t, c0 + 16 * qh, U);
-    st16(tl + kColSlot + 64 * (slot - 1) + 16 * qh, U);
+    st16(tl + kColSlot + 64 * (dst - 1) + 16 * qh, U);
     if (J == 7) {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) u[16 * qh + c] = U[c];
+      for (int c = 0; c < 16; ++c) un[16 * qh + c] = U[c];
     }
   }
 }
@@ -1112,12 +1116,14 @@ __device__ __forceinline__ void stage_out(uint32_t tl, const float (&bias)[HC], 
   }
 }
 
+// One stage of the replay: k_1 in slot 1, k_7 into slot 1 (FSAL), u <- u_{s+1}.
 template <int J>
 __device__ __forceinline__ void fwd_stage(Smem& s, int tid, int t, int c0, uint32_t& phase, uint32_t tl, float h,
                                           float (&u)[HC], const float (&bias)[HC]) {
-  stage_in<J>(s, tl, t, c0, h, u);
-  product(s, tid, phase, false);
-  stage_out(tl, bias, J <= 6 ? J : 1);
+  constexpr int slot = J <= 6 ? J : 1;
+  stage_in<J>(s, tl, t, c0, h, u, u, 1, slot);
+  product(s, tid, phase);
+  stage_out(tl, bias, slot);
 }
 
 // 16 components of trajectory tk (0..63 within its half) into G^T and U^T.
@@ -1438,13 +1444,347 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core recorder (k_record_node64_t128): the adaptive Tsit5 iteration of
+// k_record_node64 in the layout of k_node64_t128 -- 128 trajectories per CTA
+// (in trajectory order), one TMEM lane each, the stage products Z = U W^T as
+// M = 128 3xTF32 MMAs -- so that the recorded states are bit for bit those of
+// the tensor-core replay.  TMEM: the accumulator and seven stage slots (k_1 in
+// slot 1, k_j in slot j, k_7 in slot 7; an accepted step copies k_7 into slot
+// 1, FSAL).  Each trajectory's controller (starting step, error norm, PI
+// control, save points, statuses) runs on its lower-half thread with the
+// arithmetic of k_record_node64; the RMS norms keep the contract's sequential
+// sum over components 0..63 (the upper half's 32 scaled values pass through
+// shared memory).
+// ---------------------------------------------------------------------------
+struct RecSmem {
+  float Whi[D * D], Wlo[D * D];    // W: rows r, K = k
+  float Thi[TT * D], Tlo[TT * D];  // stage operand: rows t, K = component
+  float red[HC][TT];               // upper halves' scaled values, for the norms
+  float hs[TT];                    // the attempt's step per trajectory
+  int flag[TT];                    // per trajectory: finite start / accepted
+  int sv[TT];                      // save point the accepted step reached, or -1
+  unsigned long long bar;          // MMA completion
+  uint32_t tmem;                   // TMEM base (512 columns)
+  int failed;                      // an MMA wait ran out
+};
+
+// RMS of a trajectory's 64 scaled values in the contract's order: acc holds
+// the squares of components 0..31 (summed in order by the caller), red the
+// values of components 32..63.
+__device__ __forceinline__ float rms_finish(const RecSmem& s, int t, float acc) {
+  for (int c = 0; c < HC; ++c) acc = fmaT(s.red[c][t], s.red[c][t], acc);
+  return sqrt(acc / cst<float>(64.0));
+}
+
+// Scaled values x_c / sc_c of this thread's components into the norm: the
+// lower half accumulates squares in order, the upper half stores its values.
+__device__ __forceinline__ void norm_part(RecSmem& s, int t, int hf, int c, float r, float& acc) {
+  if (hf == 0)
+    acc = fmaT(r, r, acc);
+  else
+    s.red[c][t] = r;
+}
+
+// One stage of the recorder: state of stage J into the A operand and slot J,
+// the product, k_J = tanh(Z + b) - U into slot J (J = 7: un <- u_{s+1}).
+template <int J>
+__device__ __forceinline__ void rec_stage(RecSmem& s, int tid, int t, int c0, uint32_t& phase, uint32_t tl, float h,
+                                          const float (&u)[HC], float (&un)[HC], const float (&bias)[HC]) {
+  stage_in<J>(s, tl, t, c0, h, u, un, 1, J);
+  product(s, tid, phase);
+  stage_out(tl, bias, J);
+}
+
+__global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a) {
+  using T = float;
+  extern __shared__ __align__(1024) unsigned char smem_raw_rec128[];
+  RecSmem& s = *reinterpret_cast<RecSmem*>(smem_raw_rec128);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = 32 * (warp & 3) + lane, hf = warp >> 2, c0 = HC * hf;
+  const bool ctl = hf == 0;  // the trajectory's controller thread
+  const int64_t n = a.n;
+  const int64_t it = (int64_t)blockIdx.x * TT + t;
+  const bool live = it < n;
+  for (int e = tid; e < D * D; e += NT) {
+    const int r = e / D, c = e % D;
+    tc::put(s.Whi, s.Wlo, tc::off(r, c, D), a.W[e]);
+  }
+  if (tid == 0) {
+    s.failed = 0;
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc::smem_u32(&s.bar)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(tc::smem_u32(&s.tmem)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  uint32_t phase = 0;
+  const uint32_t tl = s.tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0;
+  const uint32_t slot1 = tl + kColSlot, slot2 = tl + kColSlot + 64, slot7 = tl + kColSlot + 6 * 64;
+
+  T u[HC], bias[HC], un[HC];
+#pragma unroll
+  for (int c = 0; c < HC; ++c) {
+    u[c] = live ? a.u0[(int64_t)(c0 + c) * n + it] : cst<T>(0.0);
+    bias[c] = live ? a.p[(int64_t)(c0 + c) * n + it] : cst<T>(0.0);
+  }
+  const T eps = Eps<T>::v;
+  const T qord = cst<T>(5.0);
+  T tcur = a.t0, hprop = cst<T>(0.0), lnprev = cst<T>(0.0);
+  const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
+  int nst = 0, nrej = 0, kk = 0, status = live ? GS_TRAJ_OK : GS_TRAJ_MAXSTEPS;
+  bool prev_rej = false, done = !live;
+
+  // k1 = f(u0) and the starting step (Hairer, Norsett & Wanner I, II.4)
+  rec_stage<1>(s, tid, t, c0, phase, tl, cst<T>(0.0), u, un, bias);
+  if (ctl) s.flag[t] = 1;
+  __syncthreads();
+  T acc0 = cst<T>(0.0), acc1 = cst<T>(0.0);
+#pragma unroll
+  for (int qh = 0; qh < 2; ++qh) {
+    T k[16];
+    ld16(slot1 + 16 * qh, k);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int cc = 16 * qh + c;
+      if (!isfinite(u[cc]) || !isfinite(k[c])) s.flag[t] = 0;
+      norm_part(s, t, hf, cc, u[cc] / fmaT(a.rtol, fabs(u[cc]), a.atol), acc0);
+    }
+  }
+  __syncthreads();
+  const T d0 = ctl ? rms_finish(s, t, acc0) : cst<T>(0.0);
+  __syncthreads();
+#pragma unroll
+  for (int qh = 0; qh < 2; ++qh) {
+    T k[16];
+    ld16(slot1 + 16 * qh, k);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int cc = 16 * qh + c;
+      norm_part(s, t, hf, cc, k[c] / fmaT(a.rtol, fabs(u[cc]), a.atol), acc1);
+    }
+  }
+  __syncthreads();
+  T d1 = cst<T>(0.0), h0 = cst<T>(0.0);
+  if (ctl) {
+    d1 = rms_finish(s, t, acc1);
+    h0 = (d0 < cst<T>(1e-5) || d1 < cst<T>(1e-5)) ? cst<T>(1e-6) : cst<T>(0.01) * (d0 / d1);
+    h0 = smin_(h0, a.t1 - a.t0);
+    s.hs[t] = h0;
+  }
+  __syncthreads();
+  h0 = s.hs[t];
+  // f(u0 + h0 f(u0)) into slot 2
+#pragma unroll
+  for (int qh = 0; qh < 2; ++qh) {
+    T k[16], U[16];
+    ld16(slot1 + 16 * qh, k);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) U[c] = fmaT(h0, k[c], u[16 * qh + c]);
+    put_rows16(s, t, c0 + 16 * qh, U);
+    st16(slot2 + 16 * qh, U);
+  }
+  product(s, tid, phase);
+  stage_out(tl, bias, 2);
+  T acc2 = cst<T>(0.0);
+#pragma unroll
+  for (int qh = 0; qh < 2; ++qh) {
+    T k[16], kb[16];
+    ld16(slot1 + 16 * qh, k);
+    ld16(slot2 + 16 * qh, kb);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int cc = 16 * qh + c;
+      norm_part(s, t, hf, cc, (kb[c] - k[c]) / fmaT(a.rtol, fabs(u[cc]), a.atol), acc2);
+    }
+  }
+  __syncthreads();
+  if (ctl) {
+    const T d2 = rms_finish(s, t, acc2) / h0;
+    const T dm = smax_(d1, d2);
+    const T h1 = dm <= cst<T>(1e-15) ? smax_(cst<T>(1e-6), h0 * cst<T>(1e-3))
+                                     : ctrl_pow<T>(cst<T>(0.01) / dm, cst<T>(1.0) / qord);
+    hprop = a.h0 > cst<T>(0.0) ? a.h0 : smin_(smin_(cst<T>(100.0) * h0, h1), a.t1 - a.t0);
+    if (live && (s.flag[t] == 0 || !(hprop > cst<T>(0.0)) || !isfinite(hprop))) {
+      status = GS_TRAJ_NONFINITE;
+      done = true;
+    }
+  }
+
+  for (;;) {
+    // --- controller: choose the attempt
+    bool clipped = false;
+    T tstop = a.t1, tn = tcur;
+    if (ctl) {
+      if (!done && hprop < cst<T>(16.0) * eps * fabs(tcur)) {
+        status = GS_TRAJ_DTMIN;
+        done = true;
+      }
+      T hh = cst<T>(0.0);
+      if (!done) {
+        tstop = kk < a.nsave ? a.tsave[kk] : a.t1;
+        tn = tcur + hprop;
+        clipped = tn >= tstop - cst<T>(4.0) * eps * fabs(tstop);
+        hh = clipped ? tstop - tcur : hprop;
+      }
+      s.hs[t] = hh;
+    }
+    if (!__syncthreads_or(ctl && !done)) break;
+    const T hh = s.hs[t];
+    rec_stage<2>(s, tid, t, c0, phase, tl, hh, u, un, bias);
+    rec_stage<3>(s, tid, t, c0, phase, tl, hh, u, un, bias);
+    rec_stage<4>(s, tid, t, c0, phase, tl, hh, u, un, bias);
+    rec_stage<5>(s, tid, t, c0, phase, tl, hh, u, un, bias);
+    rec_stage<6>(s, tid, t, c0, phase, tl, hh, u, un, bias);
+    rec_stage<7>(s, tid, t, c0, phase, tl, hh, u, un, bias);  // un = u_{s+1}, k7 in slot 7
+    // scaled error e / sc, e = h sum_j E_j k_j (the contract's order)
+    T acc = cst<T>(0.0);
+    {
+      constexpr double E[7] = {TS_E1, TS_E2, TS_E3, TS_E4, TS_E5, TS_E6, TS_E7};
+#pragma unroll
+      for (int qh = 0; qh < 2; ++qh) {
+        T e[16], k[16];
+        ld16(slot1 + 16 * qh, k);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) e[c] = cst<T>(E[0]) * k[c];
+#pragma unroll
+        for (int m = 1; m < 7; ++m) {
+          ld16(tl + kColSlot + 64 * m + 16 * qh, k);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) e[c] = fmaT(cst<T>(E[m]), k[c], e[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int cc = 16 * qh + c;
+          const T sc = fmaT(a.rtol, smax_(fabs(u[cc]), fabs(un[cc])), a.atol);
+          norm_part(s, t, hf, cc, (hh * e[c]) / sc, acc);
+        }
+      }
+    }
+    __syncthreads();
+    // --- controller: accept / reject
+    if (ctl) {
+      int accept = 0, hit = -1;
+      if (!done) {
+        const T err = rms_finish(s, t, acc);
+        const T hcur = s.hs[t];
+        if (err <= cst<T>(1.0)) {
+          if (nst >= a.smax) {
+            status = GS_TRAJ_MAXSTEPS;
+            done = true;
+          } else {
+            accept = 1;
+            if (a.store) a.h[it * a.smax + nst] = hcur;  // trajectory-major workspace copy
+            ++nst;
+            tcur = clipped ? tstop : tn;
+            while (kk < a.nsave && tcur == a.tsave[kk]) {  // save times increase: one hit at most
+              if (a.store) a.save_idx[(int64_t)kk * n + it] = nst;
+              hit = kk;
+              ++kk;
+            }
+            T fac, lnerr = ln_floor;
+            if (err == cst<T>(0.0)) {
+              fac = cst<T>(10.0);
+            } else {
+              lnerr = ctrl_ln<T>(err);
+              fac = cst<T>(0.9) * ctrl_exp<T>(fmaT(-(cst<T>(0.7) / qord), lnerr, (cst<T>(0.4) / qord) * lnprev));
+              fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
+            }
+            if (prev_rej) fac = smin_(fac, cst<T>(1.0));
+            lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
+            prev_rej = false;
+            hprop = fac * hprop;
+            if (tcur >= a.t1) done = true;
+          }
+        } else {
+          ++nrej;
+          if (nrej > a.smax) {
+            status = GS_TRAJ_MAXSTEPS;
+            done = true;
+          } else {
+            const T fac = !isfinite(err) ? cst<T>(0.2)
+                                         : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_exp<T>(-(cst<T>(1.0) / qord) *
+                                                                                          ctrl_ln<T>(err)));
+            hprop = fac * hprop;
+            prev_rej = true;
+          }
+        }
+      }
+      s.flag[t] = accept;
+      s.sv[t] = hit;
+    }
+    __syncthreads();
+    // --- the accepted steps: u <- u_{s+1}, k1 <- k7 (every thread rewrites
+    // slot 1 with its own choice: the TMEM address is the warp's)
+    const bool acc_t = s.flag[t] != 0;
+#pragma unroll
+    for (int qh = 0; qh < 2; ++qh) {
+      T k1[16], k7[16];
+      ld16(slot1 + 16 * qh, k1);
+      ld16(slot7 + 16 * qh, k7);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) k1[c] = acc_t ? k7[c] : k1[c];
+      st16(slot1 + 16 * qh, k1);
+    }
+    if (acc_t) {
+#pragma unroll
+      for (int c = 0; c < HC; ++c) u[c] = un[c];
+      const int k = s.sv[t];
+      if (a.u_save && k >= 0) {
+#pragma unroll
+        for (int c = 0; c < HC; ++c) a.u_save[((int64_t)k * D + c0 + c) * n + it] = u[c];
+      }
+    }
+  }
+  // outcome: statuses and counts from the controller threads; a failed
+  // trajectory of the solve has NaN at every save point
+  if (ctl && s.failed && live) status = GS_TRAJ_NONFINITE;
+  if (ctl) s.flag[t] = status;
+  __syncthreads();
+  if (live && a.u_save && s.flag[t] != GS_TRAJ_OK) {
+    const T nan = cst<T>(__int_as_float(0x7fc00000));
+    for (int k = 0; k < a.nsave; ++k)
+#pragma unroll
+      for (int c = 0; c < HC; ++c) a.u_save[((int64_t)k * D + c0 + c) * n + it] = nan;
+  }
+  if (ctl && live) {
+    if (a.store)
+      for (int k = kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + it] = 0;
+    if (a.nsteps) a.nsteps[it] = nst;
+    if (a.status) a.status[it] = status;
+    if (a.nreject) a.nreject[it] = nrej;
+  }
+  // no MMA in flight and every TMEM access done before the columns are freed
+  if (s.failed && tid == 0) {
+    uint32_t done_w = 0;
+    for (int itw = 0; itw < tc::kSpin && !done_w; ++itw)
+      asm volatile(
+          "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+          "selp.b32 %0, 1, 0, P1;\n\t}\n"
+          : "=r"(done_w)
+          : "r"(tc::smem_u32(&s.bar)), "r"(phase ^ 1u)
+          : "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(s.tmem));
+  }
+}
+
 }  // namespace t128
 
 }  // namespace n64
 
-// Which products the d = 64 replay and gradient use (process-wide, set by
-// gs_set_option): the tcgen05 3xTF32 products with 128 trajectories per CTA
-// (default) or the SIMT FP32 products, the recorder's own arithmetic.
+// Which products the d = 64 recorder, replay and gradient use (process-wide,
+// set by gs_set_option): the tcgen05 3xTF32 products with 128 trajectories
+// per CTA (default) or the SIMT FP32 products.
 static std::atomic<int> g_node64_tensor{1};
 void node64_set_tensor(int on) { g_node64_tensor.store(on ? 1 : 0, std::memory_order_relaxed); }
 
@@ -1559,12 +1899,22 @@ gs_status node64_record_pass(const gs_problem* P, const gs_tol* tol, int32_t sma
   a.status = status;
   a.nreject = nreject;
   a.u_save = u_save;
-  const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
-  const size_t smem = sizeof(n64::Smem<T>);
-  if (cudaFuncSetAttribute(n64::k_record_node64<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return GS_ECUDA;
-  n64::k_record_node64<T><<<nblk, n64::NT, smem, st>>>(a);
+  if (g_node64_tensor.load(std::memory_order_relaxed) != 0) {
+    // the recorder of the tensor-core replay (the same stage arithmetic)
+    const size_t smem = sizeof(n64::t128::RecSmem);
+    if (cudaFuncSetAttribute(n64::t128::k_record_node64_t128, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return GS_ECUDA;
+    n64::t128::k_record_node64_t128<<<(unsigned)((P->n + n64::t128::TT - 1) / n64::t128::TT), n64::t128::NT, smem,
+                                       st>>>(a);
+  } else {
+    const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
+    const size_t smem = sizeof(n64::Smem<T>);
+    if (cudaFuncSetAttribute(n64::k_record_node64<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return GS_ECUDA;
+    n64::k_record_node64<T><<<nblk, n64::NT, smem, st>>>(a);
+  }
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

@@ -288,12 +288,14 @@ GS_API gs_status gs_grad_static(const gs_problem* prob, const gs_mesh* mesh, con
 
 /*
  * Process-wide options (not thread-safe against concurrent calls).
- *   GS_OPT_NODE64_TENSOR_CORES  1 (default): the d = 64 replay and gradient
- *       compute W U, W^T g and g U^T on the tensor cores (tcgen05, tf32 with
- *       a 3xTF32 split: fp32 accuracy; 128 trajectories per CTA, one TMEM
- *       lane each); 0: with FP32 SIMT products, whose arithmetic is the
- *       recorder's, so a replay then repeats the recorded states bit for bit.
- *       The two agree to fp32 rounding.
+ *   GS_OPT_NODE64_TENSOR_CORES  1 (default): the d = 64 recorder, replay and
+ *       gradient compute W U, W^T g and g U^T on the tensor cores (tcgen05,
+ *       tf32 with a 3xTF32 split: fp32 accuracy; 128 trajectories per CTA,
+ *       one TMEM lane each); 0: with FP32 SIMT products.  Within either form
+ *       the recorder and the replay share their arithmetic, so a replay
+ *       repeats the recorded states bit for bit; the two forms agree to fp32
+ *       rounding (a mesh recorded with one and replayed with the other is
+ *       still a valid mesh: the replay is what is differentiated).
  * Returns GS_EINVAL for an unknown option or value.
  */
 #define GS_OPT_NODE64_TENSOR_CORES 1
