@@ -485,7 +485,8 @@ struct GradArgs64 {
   T* dp;
   T* du0;
   T* ck;       // workspace [smax][64][n] by slot
-  T* dW_part;  // workspace [parts][64][64]: one per CTA (two with the tensor-core products)
+  T* dW_part;  // workspace [parts][64][64]: one per CTA
+  T* kst;      // tensor-core gradient: stage slopes k_1..k_6 [smax][6][64][n] by slot
   T* u_save;   // solve: [nsave][64][n] by trajectory
 };
 
@@ -1104,7 +1105,9 @@ __device__ __forceinline__ void stage_in(SM& s, uint32_t tl, int t, int c0, floa
 }
 
 // After the product: k = tanh(Z + b) - U, U from the slot, k into the slot.
-__device__ __forceinline__ void stage_out(uint32_t tl, const float (&bias)[HC], int slot) {
+// gk (may be null): this thread's 32 components of k, component stride n.
+__device__ __forceinline__ void stage_out(uint32_t tl, const float (&bias)[HC], int slot, float* gk = nullptr,
+                                          int64_t n = 0) {
 #pragma unroll
   for (int qh = 0; qh < 2; ++qh) {
     float z[16], U[16];
@@ -1113,17 +1116,23 @@ __device__ __forceinline__ void stage_out(uint32_t tl, const float (&bias)[HC], 
 #pragma unroll
     for (int c = 0; c < 16; ++c) z[c] = tanh(bias[16 * qh + c] + z[c]) - U[c];
     st16(tl + kColSlot + 64 * (slot - 1) + 16 * qh, z);
+    if (gk) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) gk[(int64_t)(16 * qh + c) * n] = z[c];
+    }
   }
 }
 
-// One stage of the replay: k_1 in slot 1, k_7 into slot 1 (FSAL), u <- u_{s+1}.
+// One stage of the replay: k_1 in slot 1, k_7 into slot 1 (FSAL), u <- u_{s+1};
+// gk (may be null) receives k_J.
 template <int J>
 __device__ __forceinline__ void fwd_stage(Smem& s, int tid, int t, int c0, uint32_t& phase, uint32_t tl, float h,
-                                          float (&u)[HC], const float (&bias)[HC]) {
+                                          float (&u)[HC], const float (&bias)[HC], float* gk = nullptr,
+                                          int64_t n = 0) {
   constexpr int slot = J <= 6 ? J : 1;
   stage_in<J>(s, tl, t, c0, h, u, u, 1, slot);
   product(s, tid, phase);
-  stage_out(tl, bias, slot);
+  stage_out(tl, bias, slot, gk, n);
 }
 
 // 16 components of trajectory tk (0..63 within its half) into G^T and U^T.
@@ -1241,19 +1250,26 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
   int kk = 0, next = act && S > 0 ? a.save_idx[j] : -1;
 
   // ---------------------------------------------------------------- forward
-  fwd_stage<1>(s, tid, t, c0, phase, tl, cst<T>(0.0), u, bias);  // k1 = f(u0)
+  // the stage slopes of step st go to kst[st][j - 1][c][slot] for the reverse sweep
+  const int64_t kstep = (int64_t)6 * n64;
+  T* const kj = GRAD ? a.kst + (int64_t)c0 * n + j : nullptr;
+  auto kdst = [&](int st, int jslot) -> T* {
+    return (GRAD && st < S) ? kj + (int64_t)st * kstep + (int64_t)(jslot - 1) * n64 : nullptr;
+  };
+  fwd_stage<1>(s, tid, t, c0, phase, tl, cst<T>(0.0), u, bias, kdst(0, 1), n);  // k1 = f(u0)
   for (int st = 0; st < Smax; ++st) {
     const T h = st < S ? a.h[(int64_t)st * n + j] : cst<T>(0.0);
     if (GRAD && st < S) {
 #pragma unroll
       for (int c = 0; c < HC; ++c) a.ck[(int64_t)st * n64 + (int64_t)(c0 + c) * n + j] = u[c];
     }
-    fwd_stage<2>(s, tid, t, c0, phase, tl, h, u, bias);
-    fwd_stage<3>(s, tid, t, c0, phase, tl, h, u, bias);
-    fwd_stage<4>(s, tid, t, c0, phase, tl, h, u, bias);
-    fwd_stage<5>(s, tid, t, c0, phase, tl, h, u, bias);
-    fwd_stage<6>(s, tid, t, c0, phase, tl, h, u, bias);
-    fwd_stage<7>(s, tid, t, c0, phase, tl, h, u, bias);  // u <- u_{st+1}; k7 -> slot 1 (FSAL)
+    fwd_stage<2>(s, tid, t, c0, phase, tl, h, u, bias, kdst(st, 2), n);
+    fwd_stage<3>(s, tid, t, c0, phase, tl, h, u, bias, kdst(st, 3), n);
+    fwd_stage<4>(s, tid, t, c0, phase, tl, h, u, bias, kdst(st, 4), n);
+    fwd_stage<5>(s, tid, t, c0, phase, tl, h, u, bias, kdst(st, 5), n);
+    fwd_stage<6>(s, tid, t, c0, phase, tl, h, u, bias, kdst(st, 6), n);
+    // u <- u_{st+1}; k7 -> slot 1 (FSAL) and, as the next step's k_1, to kst
+    fwd_stage<7>(s, tid, t, c0, phase, tl, h, u, bias, kdst(st + 1, 1), n);
     if (st + 1 == next) {
       const int64_t o = (int64_t)kk * n64 + traj;
 #pragma unroll
@@ -1311,13 +1327,19 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
 #pragma unroll
         for (int c = 0; c < HC; ++c) u[c] = a.ck[(int64_t)st * n64 + (int64_t)(c0 + c) * n + j];
       }
-      // recompute the stage slopes k_1..k_6 of step st into the slots
-      fwd_stage<1>(s, tid, t, c0, phase, tl, h, u, bias);
-      fwd_stage<2>(s, tid, t, c0, phase, tl, h, u, bias);
-      fwd_stage<3>(s, tid, t, c0, phase, tl, h, u, bias);
-      fwd_stage<4>(s, tid, t, c0, phase, tl, h, u, bias);
-      fwd_stage<5>(s, tid, t, c0, phase, tl, h, u, bias);
-      fwd_stage<6>(s, tid, t, c0, phase, tl, h, u, bias);
+      // the stage slopes k_1..k_6 of step st from the forward pass into the
+      // slots (zero for a slot past its last step, whose step is 0)
+#pragma unroll
+      for (int jj = 0; jj < 6; ++jj) {
+        const T* src = kj + (int64_t)st * kstep + (int64_t)jj * n64;
+#pragma unroll
+        for (int qh = 0; qh < 2; ++qh) {
+          T v[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) v[c] = run ? src[(int64_t)(16 * qh + c) * n] : cst<T>(0.0);
+          st16(tl + kColSlot + 64 * jj + 16 * qh, v);
+        }
+      }
 
       // transposed step, stages 6 .. 1:
       //   nu_j = h (b_j lambda + sum_{m>j} a_mj mu_m), g_j = nu_j (1 - y_j^2),
@@ -1788,10 +1810,17 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
 static std::atomic<int> g_node64_tensor{1};
 void node64_set_tensor(int on) { g_node64_tensor.store(on ? 1 : 0, std::memory_order_relaxed); }
 
+// Gradient workspace: the checkpoints [smax][64][n], one weight-gradient
+// partial per CTA (fewer CTAs with tensor cores) and, with the tensor-core
+// products, the stage slopes [smax][6][64][n] that the reverse sweep reads
+// instead of recomputing them.  The size follows the product option in force.
+static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize) {
   const int64_t nblk = (n + n64::TB - 1) / n64::TB;
-  const size_t ck = ((size_t)smax * 64 * n * tsize + 255) / 256 * 256;
-  return ck + (size_t)nblk * 64 * 64 * tsize;  // one weight-gradient partial per CTA (fewer CTAs with tensor cores)
+  const size_t ck = align256((size_t)smax * 64 * n * tsize);
+  const size_t dw = align256((size_t)nblk * 64 * 64 * tsize);
+  const size_t kst = g_node64_tensor.load(std::memory_order_relaxed) != 0 ? (size_t)smax * 6 * 64 * n * tsize : 0;
+  return ck + dw + kst;
 }
 
 template <typename T>
@@ -1823,7 +1852,9 @@ gs_status node64_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, 
   a.du0 = (T*)du0;
   a.ck = (T*)ws;
   const int nblk = (int)((P->n + n64::TB - 1) / n64::TB);
-  a.dW_part = (T*)((char*)ws + ((size_t)M->smax * 64 * P->n * sizeof(T) + 255) / 256 * 256);
+  const size_t ck_bytes = align256((size_t)M->smax * 64 * P->n * sizeof(T));
+  a.dW_part = (T*)((char*)ws + ck_bytes);
+  a.kst = (T*)((char*)ws + ck_bytes + align256((size_t)nblk * 64 * 64 * sizeof(T)));
   const bool tensor = g_node64_tensor.load(std::memory_order_relaxed) != 0;
   const int nblk128 = (int)((P->n + n64::t128::TT - 1) / n64::t128::TT);
   if (tensor) {
