@@ -502,45 +502,43 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     GS_STAGE(U6x, U6y, U6z, ax, ay, az)
 
     // transposed step, stages 6 .. 1
+#define GS_C(N) tsc<T, kTs##N>()
     V m6x, m6y, m6z, m5x, m5y, m5z, m4x, m4y, m4z, m3x, m3y, m3z, m2x, m2y, m2z, m1x, m1y, m1z;
     V vx, vy, vz;
-    vx = h * (tsc<T, kTsB6>() * lx);
-    vy = h * (tsc<T, kTsB6>() * ly);
-    vz = h * (tsc<T, kTsB6>() * lz);
+    vx = h * (GS_C(B6) * lx);
+    vy = h * (GS_C(B6) * ly);
+    vz = h * (GS_C(B6) * lz);
     lorenz_vjp(U6x, U6y, U6z, s, r, b, vx, vy, vz, m6x, m6y, m6z, ps, pr, pb);
 
-    vx = h * fmaT(tsc<T, kTsA65>(), m6x, tsc<T, kTsB5>() * lx);
-    vy = h * fmaT(tsc<T, kTsA65>(), m6y, tsc<T, kTsB5>() * ly);
-    vz = h * fmaT(tsc<T, kTsA65>(), m6z, tsc<T, kTsB5>() * lz);
+    vx = h * fmaT(GS_C(A65), m6x, GS_C(B5) * lx);
+    vy = h * fmaT(GS_C(A65), m6y, GS_C(B5) * ly);
+    vz = h * fmaT(GS_C(A65), m6z, GS_C(B5) * lz);
     lorenz_vjp(U5x, U5y, U5z, s, r, b, vx, vy, vz, m5x, m5y, m5z, ps, pr, pb);
 
-    vx = h * fmaT(tsc<T, kTsA54>(), m5x, fmaT(tsc<T, kTsA64>(), m6x, tsc<T, kTsB4>() * lx));
-    vy = h * fmaT(tsc<T, kTsA54>(), m5y, fmaT(tsc<T, kTsA64>(), m6y, tsc<T, kTsB4>() * ly));
-    vz = h * fmaT(tsc<T, kTsA54>(), m5z, fmaT(tsc<T, kTsA64>(), m6z, tsc<T, kTsB4>() * lz));
+    vx = h * fmaT(GS_C(A54), m5x, fmaT(GS_C(A64), m6x, GS_C(B4) * lx));
+    vy = h * fmaT(GS_C(A54), m5y, fmaT(GS_C(A64), m6y, GS_C(B4) * ly));
+    vz = h * fmaT(GS_C(A54), m5z, fmaT(GS_C(A64), m6z, GS_C(B4) * lz));
     lorenz_vjp(U4x, U4y, U4z, s, r, b, vx, vy, vz, m4x, m4y, m4z, ps, pr, pb);
 
-    vx = h * fmaT(tsc<T, kTsA43>(), m4x, fmaT(tsc<T, kTsA53>(), m5x, fmaT(tsc<T, kTsA63>(), m6x, tsc<T, kTsB3>() * lx)));
-    vy = h * fmaT(tsc<T, kTsA43>(), m4y, fmaT(tsc<T, kTsA53>(), m5y, fmaT(tsc<T, kTsA63>(), m6y, tsc<T, kTsB3>() * ly)));
-    vz = h * fmaT(tsc<T, kTsA43>(), m4z, fmaT(tsc<T, kTsA53>(), m5z, fmaT(tsc<T, kTsA63>(), m6z, tsc<T, kTsB3>() * lz)));
+    vx = h * fmaT(GS_C(A43), m4x, fmaT(GS_C(A53), m5x, fmaT(GS_C(A63), m6x, GS_C(B3) * lx)));
+    vy = h * fmaT(GS_C(A43), m4y, fmaT(GS_C(A53), m5y, fmaT(GS_C(A63), m6y, GS_C(B3) * ly)));
+    vz = h * fmaT(GS_C(A43), m4z, fmaT(GS_C(A53), m5z, fmaT(GS_C(A63), m6z, GS_C(B3) * lz)));
     lorenz_vjp(U3x, U3y, U3z, s, r, b, vx, vy, vz, m3x, m3y, m3z, ps, pr, pb);
 
-    vx = h * fmaT(tsc<T, kTsA32>(), m3x,
-                  fmaT(tsc<T, kTsA42>(), m4x, fmaT(tsc<T, kTsA52>(), m5x, fmaT(tsc<T, kTsA62>(), m6x, tsc<T, kTsB2>() * lx))));
-    vy = h * fmaT(tsc<T, kTsA32>(), m3y,
-                  fmaT(tsc<T, kTsA42>(), m4y, fmaT(tsc<T, kTsA52>(), m5y, fmaT(tsc<T, kTsA62>(), m6y, tsc<T, kTsB2>() * ly))));
-    vz = h * fmaT(tsc<T, kTsA32>(), m3z,
-                  fmaT(tsc<T, kTsA42>(), m4z, fmaT(tsc<T, kTsA52>(), m5z, fmaT(tsc<T, kTsA62>(), m6z, tsc<T, kTsB2>() * lz))));
+    vx = h * fmaT(GS_C(A32), m3x, fmaT(GS_C(A42), m4x, fmaT(GS_C(A52), m5x, fmaT(GS_C(A62), m6x, GS_C(B2) * lx))));
+    vy = h * fmaT(GS_C(A32), m3y, fmaT(GS_C(A42), m4y, fmaT(GS_C(A52), m5y, fmaT(GS_C(A62), m6y, GS_C(B2) * ly))));
+    vz = h * fmaT(GS_C(A32), m3z, fmaT(GS_C(A42), m4z, fmaT(GS_C(A52), m5z, fmaT(GS_C(A62), m6z, GS_C(B2) * lz))));
     lorenz_vjp(U2x, U2y, U2z, s, r, b, vx, vy, vz, m2x, m2y, m2z, ps, pr, pb);
 
-    vx = h * fmaT(tsc<T, kTsA21>(), m2x,
-                  fmaT(tsc<T, kTsA31>(), m3x,
-                       fmaT(tsc<T, kTsA41>(), m4x, fmaT(tsc<T, kTsA51>(), m5x, fmaT(tsc<T, kTsA61>(), m6x, tsc<T, kTsB1>() * lx)))));
-    vy = h * fmaT(tsc<T, kTsA21>(), m2y,
-                  fmaT(tsc<T, kTsA31>(), m3y,
-                       fmaT(tsc<T, kTsA41>(), m4y, fmaT(tsc<T, kTsA51>(), m5y, fmaT(tsc<T, kTsA61>(), m6y, tsc<T, kTsB1>() * ly)))));
-    vz = h * fmaT(tsc<T, kTsA21>(), m2z,
-                  fmaT(tsc<T, kTsA31>(), m3z,
-                       fmaT(tsc<T, kTsA41>(), m4z, fmaT(tsc<T, kTsA51>(), m5z, fmaT(tsc<T, kTsA61>(), m6z, tsc<T, kTsB1>() * lz)))));
+    vx = h * fmaT(GS_C(A21), m2x,
+                  fmaT(GS_C(A31), m3x,
+                       fmaT(GS_C(A41), m4x, fmaT(GS_C(A51), m5x, fmaT(GS_C(A61), m6x, GS_C(B1) * lx)))));
+    vy = h * fmaT(GS_C(A21), m2y,
+                  fmaT(GS_C(A31), m3y,
+                       fmaT(GS_C(A41), m4y, fmaT(GS_C(A51), m5y, fmaT(GS_C(A61), m6y, GS_C(B1) * ly)))));
+    vz = h * fmaT(GS_C(A21), m2z,
+                  fmaT(GS_C(A31), m3z,
+                       fmaT(GS_C(A41), m4z, fmaT(GS_C(A51), m5z, fmaT(GS_C(A61), m6z, GS_C(B1) * lz)))));
     lorenz_vjp(x, y, z, s, r, b, vx, vy, vz, m1x, m1y, m1z, ps, pr, pb);
 
     lx += ((m1x + m2x) + (m3x + m4x)) + (m5x + m6x);
@@ -572,6 +570,7 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #undef GS_STAGE
 #undef GS_ACC1
 #undef GS_ACCN
+#undef GS_C
 
 template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp,

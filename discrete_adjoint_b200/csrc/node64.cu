@@ -237,6 +237,74 @@ struct RecArgs64 {
   T* u_save;  // adaptive forward-only solve: [nsave][64][n] by trajectory, else null
 };
 
+// Per-trajectory state of the d = 64 recorders: time, proposal, the
+// controller's ln(errprev), counts, next save point, status.
+template <typename T>
+struct Ctl64 {
+  T tcur, hprop, lnprev;
+  int nst, nrej, kk, status;
+  bool prev_rej, done;
+};
+
+// The outcome of trajectory it's attempt with scaled error err and step hcur
+// (clipped onto tstop, or ending at tn): accepted -> the step is stored (a
+// trajectory-major workspace copy), t advances, the save point reached is
+// returned in hit, and the PI factor 0.9 err^(-0.7/q) errprev^(0.4/q)
+// (clipped to [0.2, 10], at most 1 right after a rejection) scales the
+// proposal; rejected -> the proposal shrinks by max(0.2, 0.9 err^(-1/q)).
+// Exceeding smax accepted or rejected attempts ends the trajectory with
+// MAXSTEPS.  Returns 1 when the step is accepted.
+template <typename T>
+__device__ __forceinline__ int ctl_decide(Ctl64<T>& rec, const RecArgs64<T>& a, int64_t it, T err, T hcur,
+                                          bool clipped, T tstop, T tn, T ln_floor, int& hit) {
+  const int64_t n = a.n;
+  const T qord = cst<T>(5.0);
+  int accept = 0;
+  hit = -1;
+  if (err <= cst<T>(1.0)) {
+    if (rec.nst >= a.smax) {
+      rec.status = GS_TRAJ_MAXSTEPS;
+      rec.done = true;
+    } else {
+      accept = 1;
+      if (a.store) a.h[it * a.smax + rec.nst] = hcur;  // trajectory-major workspace copy
+      ++rec.nst;
+      rec.tcur = clipped ? tstop : tn;
+      while (rec.kk < a.nsave && rec.tcur == a.tsave[rec.kk]) {  // save times increase: one hit at most
+        if (a.store) a.save_idx[(int64_t)rec.kk * n + it] = rec.nst;
+        hit = rec.kk;
+        ++rec.kk;
+      }
+      T fac, lnerr = ln_floor;
+      if (err == cst<T>(0.0)) {
+        fac = cst<T>(10.0);
+      } else {
+        lnerr = ctrl_ln<T>(err);
+        fac = cst<T>(0.9) * ctrl_exp<T>(fmaT(-(cst<T>(0.7) / qord), lnerr, (cst<T>(0.4) / qord) * rec.lnprev));
+        fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
+      }
+      if (rec.prev_rej) fac = smin_(fac, cst<T>(1.0));
+      rec.lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
+      rec.prev_rej = false;
+      rec.hprop = fac * rec.hprop;
+      if (rec.tcur >= a.t1) rec.done = true;
+    }
+  } else {
+    ++rec.nrej;
+    if (rec.nrej > a.smax) {
+      rec.status = GS_TRAJ_MAXSTEPS;
+      rec.done = true;
+    } else {
+      const T fac = !isfinite(err) ? cst<T>(0.2)
+                                   : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_exp<T>(-(cst<T>(1.0) / qord) *
+                                                                                    ctrl_ln<T>(err)));
+      rec.hprop = fac * rec.hprop;
+      rec.prev_rej = true;
+    }
+  }
+  return accept;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
   extern __shared__ unsigned char smem_raw[];
@@ -265,10 +333,8 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
   const bool live = ctl && it < n;
   const T eps = Eps<T>::v;
   const T qord = cst<T>(5.0);
-  T tcur = a.t0, hprop = cst<T>(0.0), lnprev = cst<T>(0.0);
+  Ctl64<T> rec{a.t0, cst<T>(0.0), cst<T>(0.0), 0, 0, 0, live ? GS_TRAJ_OK : GS_TRAJ_MAXSTEPS, false, !live};
   const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
-  int nst = 0, nrej = 0, kk = 0, status = live ? GS_TRAJ_OK : GS_TRAJ_MAXSTEPS;
-  bool prev_rej = false, done = !live;
 
   // k1 = f(u0) and the starting step (Hairer, Norsett & Wanner I, II.4)
   Blk<T> y, k1;
@@ -321,10 +387,10 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
     const T dm = smax_(d1, d2);
     const T h1 = dm <= cst<T>(1e-15) ? smax_(cst<T>(1e-6), h0 * cst<T>(1e-3))
                                      : ctrl_pow<T>(cst<T>(0.01) / dm, cst<T>(1.0) / qord);
-    hprop = a.h0 > cst<T>(0.0) ? a.h0 : smin_(smin_(cst<T>(100.0) * h0, h1), a.t1 - a.t0);
-    if (live && (s.flag[t] == 0 || !(hprop > cst<T>(0.0)) || !isfinite(hprop))) {
-      status = GS_TRAJ_NONFINITE;
-      done = true;
+    rec.hprop = a.h0 > cst<T>(0.0) ? a.h0 : smin_(smin_(cst<T>(100.0) * h0, h1), a.t1 - a.t0);
+    if (live && (s.flag[t] == 0 || !(rec.hprop > cst<T>(0.0)) || !isfinite(rec.hprop))) {
+      rec.status = GS_TRAJ_NONFINITE;
+      rec.done = true;
     }
   }
 
@@ -332,21 +398,21 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
   for (int iter = 0;; ++iter) {
     // --- per-slot: choose the attempt
     bool clipped = false;
-    T tstop = a.t1, tn = tcur;
+    T tstop = a.t1, tn = rec.tcur;
     if (ctl) {
-      if (!done && hprop < cst<T>(16.0) * eps * fabs(tcur)) {
-        status = GS_TRAJ_DTMIN;
-        done = true;
+      if (!rec.done && rec.hprop < cst<T>(16.0) * eps * fabs(rec.tcur)) {
+        rec.status = GS_TRAJ_DTMIN;
+        rec.done = true;
       }
       T hh = cst<T>(0.0);
-      if (!done) {
-        tstop = kk < a.nsave ? a.tsave[kk] : a.t1;
-        tn = tcur + hprop;
+      if (!rec.done) {
+        tstop = rec.kk < a.nsave ? a.tsave[rec.kk] : a.t1;
+        tn = rec.tcur + rec.hprop;
         clipped = tn >= tstop - cst<T>(4.0) * eps * fabs(tstop);
-        hh = clipped ? tstop - tcur : hprop;
+        hh = clipped ? tstop - rec.tcur : rec.hprop;
       }
       s.hs[t] = hh;
-      s.flag[t] = done ? 0 : 1;
+      s.flag[t] = rec.done ? 0 : 1;
     }
     __syncthreads();
     if (ctl) {
@@ -382,51 +448,8 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
     // --- per-slot: accept / reject, controller
     if (ctl) {
       int accept = 0, hit = -1;
-      if (!done) {
-        const T err = slot_rms(s, t);
-        const T hcur = s.hs[t];
-        if (err <= cst<T>(1.0)) {
-          if (nst >= a.smax) {
-            status = GS_TRAJ_MAXSTEPS;
-            done = true;
-          } else {
-            accept = 1;
-            if (a.store) a.h[it * a.smax + nst] = hcur;  // trajectory-major workspace copy
-            ++nst;
-            tcur = clipped ? tstop : tn;
-            while (kk < a.nsave && tcur == a.tsave[kk]) {  // save times increase: one hit at most
-              if (a.store) a.save_idx[(int64_t)kk * n + it] = nst;
-              hit = kk;
-              ++kk;
-            }
-            T fac, lnerr = ln_floor;
-            if (err == cst<T>(0.0)) {
-              fac = cst<T>(10.0);
-            } else {
-              lnerr = ctrl_ln<T>(err);
-              fac = cst<T>(0.9) * ctrl_exp<T>(fmaT(-(cst<T>(0.7) / qord), lnerr, (cst<T>(0.4) / qord) * lnprev));
-              fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
-            }
-            if (prev_rej) fac = smin_(fac, cst<T>(1.0));
-            lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
-            prev_rej = false;
-            hprop = fac * hprop;
-            if (tcur >= a.t1) done = true;
-          }
-        } else {
-          ++nrej;
-          if (nrej > a.smax) {
-            status = GS_TRAJ_MAXSTEPS;
-            done = true;
-          } else {
-            const T fac = !isfinite(err) ? cst<T>(0.2)
-                                         : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_exp<T>(-(cst<T>(1.0) / qord) *
-                                                                                          ctrl_ln<T>(err)));
-            hprop = fac * hprop;
-            prev_rej = true;
-          }
-        }
-      }
+      if (!rec.done)
+        accept = ctl_decide(rec, a, it, slot_rms(s, t), s.hs[t], clipped, tstop, tn, ln_floor, hit);
       s.flag[t] = accept;
       s.sv[t] = hit;
     }
@@ -448,7 +471,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
       }
     }
   }
-  if (live && a.u_save && status != GS_TRAJ_OK) {
+  if (live && a.u_save && rec.status != GS_TRAJ_OK) {
     // a failed trajectory has no solution: NaN at every save point
     const T nan = cst<T>(__int_as_float(0x7fc00000));
     for (int k = 0; k < a.nsave; ++k)
@@ -456,10 +479,10 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64(RecArgs64<T> a) {
   }
   if (live) {
     if (a.store)
-      for (int k = kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + it] = 0;
-    if (a.nsteps) a.nsteps[it] = nst;
-    if (a.status) a.status[it] = status;
-    if (a.nreject) a.nreject[it] = nrej;
+      for (int k = rec.kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + it] = 0;
+    if (a.nsteps) a.nsteps[it] = rec.nst;
+    if (a.status) a.status[it] = rec.status;
+    if (a.nreject) a.nreject[it] = rec.nrej;
   }
 }
 
@@ -1557,10 +1580,8 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
   }
   const T eps = Eps<T>::v;
   const T qord = cst<T>(5.0);
-  T tcur = a.t0, hprop = cst<T>(0.0), lnprev = cst<T>(0.0);
+  Ctl64<T> rec{a.t0, cst<T>(0.0), cst<T>(0.0), 0, 0, 0, live ? GS_TRAJ_OK : GS_TRAJ_MAXSTEPS, false, !live};
   const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
-  int nst = 0, nrej = 0, kk = 0, status = live ? GS_TRAJ_OK : GS_TRAJ_MAXSTEPS;
-  bool prev_rej = false, done = !live;
 
   // k1 = f(u0) and the starting step (Hairer, Norsett & Wanner I, II.4)
   rec_stage<1>(s, tid, t, c0, phase, tl, cst<T>(0.0), u, un, bias);
@@ -1631,32 +1652,32 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
     const T dm = smax_(d1, d2);
     const T h1 = dm <= cst<T>(1e-15) ? smax_(cst<T>(1e-6), h0 * cst<T>(1e-3))
                                      : ctrl_pow<T>(cst<T>(0.01) / dm, cst<T>(1.0) / qord);
-    hprop = a.h0 > cst<T>(0.0) ? a.h0 : smin_(smin_(cst<T>(100.0) * h0, h1), a.t1 - a.t0);
-    if (live && (s.flag[t] == 0 || !(hprop > cst<T>(0.0)) || !isfinite(hprop))) {
-      status = GS_TRAJ_NONFINITE;
-      done = true;
+    rec.hprop = a.h0 > cst<T>(0.0) ? a.h0 : smin_(smin_(cst<T>(100.0) * h0, h1), a.t1 - a.t0);
+    if (live && (s.flag[t] == 0 || !(rec.hprop > cst<T>(0.0)) || !isfinite(rec.hprop))) {
+      rec.status = GS_TRAJ_NONFINITE;
+      rec.done = true;
     }
   }
 
   for (;;) {
     // --- controller: choose the attempt
     bool clipped = false;
-    T tstop = a.t1, tn = tcur;
+    T tstop = a.t1, tn = rec.tcur;
     if (ctl) {
-      if (!done && hprop < cst<T>(16.0) * eps * fabs(tcur)) {
-        status = GS_TRAJ_DTMIN;
-        done = true;
+      if (!rec.done && rec.hprop < cst<T>(16.0) * eps * fabs(rec.tcur)) {
+        rec.status = GS_TRAJ_DTMIN;
+        rec.done = true;
       }
       T hh = cst<T>(0.0);
-      if (!done) {
-        tstop = kk < a.nsave ? a.tsave[kk] : a.t1;
-        tn = tcur + hprop;
+      if (!rec.done) {
+        tstop = rec.kk < a.nsave ? a.tsave[rec.kk] : a.t1;
+        tn = rec.tcur + rec.hprop;
         clipped = tn >= tstop - cst<T>(4.0) * eps * fabs(tstop);
-        hh = clipped ? tstop - tcur : hprop;
+        hh = clipped ? tstop - rec.tcur : rec.hprop;
       }
       s.hs[t] = hh;
     }
-    if (!__syncthreads_or(ctl && !done)) break;
+    if (!__syncthreads_or(ctl && !rec.done)) break;
     const T hh = s.hs[t];
     rec_stage<2>(s, tid, t, c0, phase, tl, hh, u, un, bias);
     rec_stage<3>(s, tid, t, c0, phase, tl, hh, u, un, bias);
@@ -1692,51 +1713,8 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
     // --- controller: accept / reject
     if (ctl) {
       int accept = 0, hit = -1;
-      if (!done) {
-        const T err = rms_finish(s, t, acc);
-        const T hcur = s.hs[t];
-        if (err <= cst<T>(1.0)) {
-          if (nst >= a.smax) {
-            status = GS_TRAJ_MAXSTEPS;
-            done = true;
-          } else {
-            accept = 1;
-            if (a.store) a.h[it * a.smax + nst] = hcur;  // trajectory-major workspace copy
-            ++nst;
-            tcur = clipped ? tstop : tn;
-            while (kk < a.nsave && tcur == a.tsave[kk]) {  // save times increase: one hit at most
-              if (a.store) a.save_idx[(int64_t)kk * n + it] = nst;
-              hit = kk;
-              ++kk;
-            }
-            T fac, lnerr = ln_floor;
-            if (err == cst<T>(0.0)) {
-              fac = cst<T>(10.0);
-            } else {
-              lnerr = ctrl_ln<T>(err);
-              fac = cst<T>(0.9) * ctrl_exp<T>(fmaT(-(cst<T>(0.7) / qord), lnerr, (cst<T>(0.4) / qord) * lnprev));
-              fac = smin_(cst<T>(10.0), smax_(cst<T>(0.2), fac));
-            }
-            if (prev_rej) fac = smin_(fac, cst<T>(1.0));
-            lnprev = err < cst<T>(1e-4) ? ln_floor : lnerr;
-            prev_rej = false;
-            hprop = fac * hprop;
-            if (tcur >= a.t1) done = true;
-          }
-        } else {
-          ++nrej;
-          if (nrej > a.smax) {
-            status = GS_TRAJ_MAXSTEPS;
-            done = true;
-          } else {
-            const T fac = !isfinite(err) ? cst<T>(0.2)
-                                         : smax_(cst<T>(0.2), cst<T>(0.9) * ctrl_exp<T>(-(cst<T>(1.0) / qord) *
-                                                                                          ctrl_ln<T>(err)));
-            hprop = fac * hprop;
-            prev_rej = true;
-          }
-        }
-      }
+      if (!rec.done)
+        accept = ctl_decide(rec, a, it, rms_finish(s, t, acc), s.hs[t], clipped, tstop, tn, ln_floor, hit);
       s.flag[t] = accept;
       s.sv[t] = hit;
     }
@@ -1765,8 +1743,8 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
   }
   // outcome: statuses and counts from the controller threads; a failed
   // trajectory of the solve has NaN at every save point
-  if (ctl && s.failed && live) status = GS_TRAJ_NONFINITE;
-  if (ctl) s.flag[t] = status;
+  if (ctl && s.failed && live) rec.status = GS_TRAJ_NONFINITE;
+  if (ctl) s.flag[t] = rec.status;
   __syncthreads();
   if (live && a.u_save && s.flag[t] != GS_TRAJ_OK) {
     const T nan = cst<T>(__int_as_float(0x7fc00000));
@@ -1776,12 +1754,12 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
   }
   if (ctl && live) {
     if (a.store)
-      for (int k = kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + it] = 0;
-    if (a.nsteps) a.nsteps[it] = nst;
-    if (a.status) a.status[it] = status;
-    if (a.nreject) a.nreject[it] = nrej;
+      for (int k = rec.kk; k < a.nsave; ++k) a.save_idx[(int64_t)k * n + it] = 0;
+    if (a.nsteps) a.nsteps[it] = rec.nst;
+    if (a.status) a.status[it] = rec.status;
+    if (a.nreject) a.nreject[it] = rec.nrej;
   }
-  // no MMA in flight and every TMEM access done before the columns are freed
+  // no MMA in flight and every TMEM access rec.done before the columns are freed
   if (s.failed && tid == 0) {
     uint32_t done_w = 0;
     for (int itw = 0; itw < tc::kSpin && !done_w; ++itw)
