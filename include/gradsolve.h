@@ -53,7 +53,7 @@ typedef int32_t gs_status;
 #define GS_EINVAL (-1)       /* bad argument (null pointer, size, combination) */
 #define GS_ECUDA (-2)        /* a CUDA launch or runtime call failed */
 #define GS_EWORKSPACE (-3)   /* workspace pointer null or smaller than required */
-#define GS_EUNSUPPORTED (-4) /* valid request this build does not implement */
+#define GS_EUNSUPPORTED (-4) /* valid request this library does not implement */
 
 /* Per-trajectory record status (mesh.status). */
 #define GS_TRAJ_OK 0
@@ -65,7 +65,7 @@ typedef int32_t gs_status;
 /* Registered right-hand sides. */
 #define GS_LORENZ 1    /* d=3, np=3, p=(sigma, rho, beta): DiffEqGPU "ad" page, Lorenz listing */
 #define GS_ROBERTSON 2 /* d=3, np=3, p=(k1, k2, k3): mass-action kinetics A->B, 2B->B+C, B+C->A+C */
-#define GS_HIRES 3     /* reserved: not built (equations not available to this build) */
+#define GS_HIRES 3     /* reserved: not implemented (equations not given by the sources followed) */
 #define GS_NODE64 4    /* d=64, np=64 (b_i), shared W [64][64]: f = tanh(W u + b) - u */
 
 /* Integrators. */
@@ -77,7 +77,8 @@ typedef int32_t gs_status;
  *   M = I/gamma - h J;  M k1 = f(u);  v = u + h k1;  M k2 = f(v) + c21 k1;
  *   M k3 = f(v) + c31 k1 + c32 k2;  u_new = u + h (k1 + m2 k2 + m3 k3);
  *   error estimate h (e1 k1 + e2 k2 + e3 k3).  Higher-order stiff option of
- * the pages' "explicit and Rosenbrock integrators" (GRADSOLVE abstract). */
+ * GRADSOLVE's explicit and Rosenbrock integrators (abstract), with the
+ * higher-order integrators it names as a next step ("Future directions"). */
 #define GS_ROS3 3
 
 #define GS_F32 1
@@ -126,8 +127,9 @@ typedef struct gs_problem {
  *   H01 = theta^2 (3 - 2 theta), H00 = 1 - H01, H10 = theta (1 - theta)^2,
  *   H11 = -theta^2 (1 - theta).
  * The loss and its derivative then pass through that interpolant (theta, like
- * h, is data).  The survey's dense-output save points; the pages print no
- * interpolant, so this one is this library's reading. */
+ * h, is data).  Dense output (interpolated save times, as in the H200
+ * forward-sensitivity study) prints no interpolant, so this cubic Hermite one
+ * is this library's choice. */
 typedef struct gs_tol {
   double rtol, atol, h0;
   int32_t dense;

@@ -1,5 +1,5 @@
 """Pins of the oracle's forward sensitivities d u(t_k) / d (p, u0) of the
-fixed-step replay (the survey's in-kernel forward-sensitivity row; GRADSOLVE
+fixed-step replay (the in-kernel forward-sensitivity route; GRADSOLVE
 review: the derivative is that of the replay with the mesh held fixed).
 
 * Closed form: on u' = p u a step multiplies the state by R(p h), so

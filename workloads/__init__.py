@@ -6,7 +6,7 @@ the CPU oracle can take their inputs from it without sharing any of the method.
 
 Workloads (GRADSOLVE, arXiv 2609.02876: the Lorenz and Robertson studies of
 the evolve.pub review "Summary", the neural right-hand side named there as
-well; the distributions are the benchmark configurations of this build):
+well; the distributions are those of the benchmark configurations):
 
   lorenz_small  n=1,024   Lorenz, fp64, t in [0,1], rtol=atol=1e-8,
                 loss = sum ||u(T)||^2.
@@ -15,8 +15,8 @@ well; the distributions are the benchmark configurations of this build):
                 ||u(t_k) - target_k||^2 with target ~ N(0,1).
   robertson     n=65,536  Robertson kinetics, ROS2, fp64, t in [0,1e5],
                 rtol=1e-6, atol=1e-10, loss = w . u(T), w ~ U[0,1]^3.
-  hires         (not built: the HIRES equations and constants are neither on
-                the pages nor available in this environment)
+  hires         (not built: the HIRES equations and rate constants are not
+                given by the sources this library follows)
   node64        n=131,072 du/dt = tanh(W u + b_i) - u, d=64, fp32, t in [0,1],
                 rtol=atol=1e-5, loss = sum ||u(T)||^2.
 
