@@ -29,7 +29,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.cpp")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-SYSTEMS = {"lorenz": 1, "robertson": 2, "hires": 3, "node64": 4, "linear": 5}
+SYSTEMS = {"lorenz": 1, "robertson": 2, "hires": 3, "node64": 4, "linear": 5, "kin8": 6}
 METHODS = {"tsit5": 1, "ros2": 2, "ros3": 3}
 DTYPES = {"f32": 1, "f64": 2}
 LOSSES = {"sumsq": 1, "linear": 2}

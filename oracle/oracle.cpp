@@ -29,7 +29,9 @@
 // ROS3 of Sandu, Verwer, Blom, Spee, Carmichael & Potra (1997).  Systems: Lorenz (DiffEqGPU "ad" example,
 // "Forward-mode automatic differentiation" listing), Robertson kinetics
 // (mass-action form of the reaction scheme A->B (k1), 2B->B+C (k2),
-// B+C->A+C (k3)), and the d=64 shared-weight system tanh(W u + b) - u.
+// B+C->A+C (k3)), the d=64 shared-weight system tanh(W u + b) - u, and kin8,
+// an 8-species stiff mass-action network defined in this library (below; not a
+// published test problem) that exercises the Rosenbrock path at d = 8.
 //
 // Parity pins for every function here live in tests/test_oracle_*.py.
 #include <algorithm>
@@ -179,7 +181,7 @@ template <> struct base_of<Cn> { using type = double; };
 // ---------------------------------------------------------------------------
 // Method constants.
 // ---------------------------------------------------------------------------
-enum { SYS_LORENZ = 1, SYS_ROBERTSON = 2, SYS_HIRES = 3, SYS_NODE64 = 4, SYS_LINEAR = 5 };
+enum { SYS_LORENZ = 1, SYS_ROBERTSON = 2, SYS_HIRES = 3, SYS_NODE64 = 4, SYS_LINEAR = 5, SYS_KIN8 = 6 };
 enum { M_TSIT5 = 1, M_ROS2 = 2, M_ROS3 = 3 };
 enum { DT_F32 = 1, DT_F64 = 2 };
 enum { LOSS_SUMSQ = 1, LOSS_LINEAR = 2 };
@@ -250,6 +252,28 @@ void rhs(int sys, const S* u, const S* p, const S* W, S* out) {
   } else if (sys == SYS_LINEAR) {
     // scalar test equation u' = p u (pins only: closed forms exist)
     out[0] = p[0] * u[0];
+  } else if (sys == SYS_KIN8) {
+    // kin8: species A1..A8 (u[0..7]), rate constants p[0..7], mass action for
+    //   A1 -> A2, A2 -> A1, A2 + A3 -> A4, A4 -> A3 + A5,
+    //   A5 -> A6, A6 -> A5, A6 + A7 -> A8, A8 -> A7 + A1,
+    // i.e. f = N r(u) with the stoichiometric matrix N of these eight
+    // reactions.  u1+u2+u4+u5+u6+u8, u3+u4 and u7+u8 are conserved.
+    S r1 = p[0] * u[0];
+    S r2 = p[1] * u[1];
+    S r3 = p[2] * (u[1] * u[2]);
+    S r4 = p[3] * u[3];
+    S r5 = p[4] * u[4];
+    S r6 = p[5] * u[5];
+    S r7 = p[6] * (u[5] * u[6]);
+    S r8 = p[7] * u[7];
+    out[0] = (r2 - r1) + r8;
+    out[1] = (r1 - r2) - r3;
+    out[2] = r4 - r3;
+    out[3] = r3 - r4;
+    out[4] = (r4 - r5) + r6;
+    out[5] = (r5 - r6) - r7;
+    out[6] = r8 - r7;
+    out[7] = r7 - r8;
   } else if (sys == SYS_NODE64) {
     for (int r = 0; r < 64; ++r) {
       S acc = p[r];
@@ -277,6 +301,36 @@ void jac(int sys, const S* u, const S* p, S* J) {
     J[8] = S(0);
   } else if (sys == SYS_LINEAR) {
     J[0] = p[0];
+  } else if (sys == SYS_KIN8) {
+    for (int q = 0; q < 64; ++q) J[q] = S(0);
+    S a = p[2] * u[2];  // k3 y3
+    S b = p[2] * u[1];  // k3 y2
+    S c = p[6] * u[6];  // k7 y7
+    S e = p[6] * u[5];  // k7 y6
+    J[0 * 8 + 0] = -p[0];
+    J[0 * 8 + 1] = p[1];
+    J[0 * 8 + 7] = p[7];
+    J[1 * 8 + 0] = p[0];
+    J[1 * 8 + 1] = -(p[1] + a);
+    J[1 * 8 + 2] = -b;
+    J[2 * 8 + 1] = -a;
+    J[2 * 8 + 2] = -b;
+    J[2 * 8 + 3] = p[3];
+    J[3 * 8 + 1] = a;
+    J[3 * 8 + 2] = b;
+    J[3 * 8 + 3] = -p[3];
+    J[4 * 8 + 3] = p[3];
+    J[4 * 8 + 4] = -p[4];
+    J[4 * 8 + 5] = p[5];
+    J[5 * 8 + 4] = p[4];
+    J[5 * 8 + 5] = -(p[5] + c);
+    J[5 * 8 + 6] = -e;
+    J[6 * 8 + 5] = -c;
+    J[6 * 8 + 6] = -e;
+    J[6 * 8 + 7] = p[7];
+    J[7 * 8 + 5] = c;
+    J[7 * 8 + 6] = e;
+    J[7 * 8 + 7] = -p[7];
   } else if (sys == SYS_LORENZ) {
     J[0] = -p[0];
     J[1] = p[0];
@@ -903,7 +957,8 @@ int check_prob(const Prob& P) {
   if (P.sys == SYS_NODE64 && (P.d != 64 || P.np != 64 || !P.W)) return -1;
   if (P.sys == SYS_HIRES) return -4;  // not built: equations not available here
   if (P.sys == SYS_LINEAR && (P.d != 1 || P.np != 1)) return -1;
-  if (P.sys < 1 || P.sys > 5) return -1;
+  if (P.sys == SYS_KIN8 && (P.d != 8 || P.np != 8)) return -1;
+  if (P.sys < 1 || P.sys > 6) return -1;
   if (P.method != M_TSIT5 && P.method != M_ROS2 && P.method != M_ROS3) return -1;
   if (P.method != M_TSIT5 && P.d > 8) return -4;
   if (P.method != M_TSIT5 && P.sys == SYS_NODE64) return -4;

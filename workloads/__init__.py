@@ -19,6 +19,14 @@ well; the distributions are those of the benchmark configurations):
                 given by the sources this library follows)
   node64        n=131,072 du/dt = tanh(W u + b_i) - u, d=64, fp32, t in [0,1],
                 rtol=atol=1e-5, loss = sum ||u(T)||^2.
+  kin8          n=262,144 (the HIRES configuration's size, tolerances, loss
+                and parameter spread) an 8-species stiff mass-action network
+                defined by this library, d=8, np=8, ROS3, fp64,
+                t in [0, 100], rtol=atol=1e-7, loss = sum ||u(T)||^2: it
+                stands in for HIRES to exercise the Rosenbrock path at d=8
+                (8x8 LU).  Nominal rate constants
+                k = (800, 400, 2, 0.2, 0.05, 0.025, 6, 0.004), each scaled by
+                lognormal(0, 0.05); u0 = (1, 0, 0.5, 0, 0, 0, 0.3, 0).
 
 Distribution notation: N(m, v) has VARIANCE v; lognormal(0, s) is exp(N(0, s^2))
 (s is the standard deviation of the log); u0 = (1,0,0) + eps * (1,1,1) draws ONE
@@ -35,9 +43,10 @@ import numpy as np
 
 SEED_BASE = 20261201
 
-CONFIG_INDEX = {"lorenz_small": 0, "lorenz_1m": 1, "robertson": 2, "hires": 3, "node64": 4}
+CONFIG_INDEX = {"lorenz_small": 0, "lorenz_1m": 1, "robertson": 2, "hires": 3, "node64": 4, "kin8": 5}
 
-FULL_N = {"lorenz_small": 1024, "lorenz_1m": 1 << 20, "robertson": 65536, "hires": 262144, "node64": 131072}
+FULL_N = {"lorenz_small": 1024, "lorenz_1m": 1 << 20, "robertson": 65536, "hires": 262144, "node64": 131072,
+          "kin8": 262144}
 
 # Recorded-step capacity each workload is sized for (the recorder reports
 # MAXSTEPS beyond it); generous relative to the observed maxima.
@@ -46,7 +55,7 @@ SMAX = {"lorenz_small": 256, "lorenz_1m": 1024, "robertson": 8192, "node64": 256
 
 @dataclass
 class Problem:
-    system: str            # "lorenz" | "robertson" | "node64" | "linear"
+    system: str            # "lorenz" | "robertson" | "node64" | "kin8" | "linear"
     method: str            # "tsit5" | "ros2" | "ros3"
     dtype: str             # "f64" | "f32"
     n: int
@@ -134,6 +143,19 @@ def node64(n: int | None = None, seed_offset: int = 0, dtype: str = "f32") -> Pr
     return prob.as_dtype(dtype)
 
 
+KIN8_RATES = np.array([800.0, 400.0, 2.0, 0.2, 0.05, 0.025, 6.0, 0.004])
+KIN8_U0 = np.array([1.0, 0.0, 0.5, 0.0, 0.0, 0.0, 0.3, 0.0])
+
+
+def kin8(n: int | None = None, seed_offset: int = 0) -> Problem:
+    n = FULL_N["kin8"] if n is None else n
+    g = _rng("kin8", seed_offset)
+    k = KIN8_RATES[:, None] * np.exp(g.normal(0.0, 0.05, (8, n)))
+    u0 = np.repeat(KIN8_U0[:, None], n, axis=1)
+    return Problem("kin8", "ros3", "f64", n, 8, 8, k, u0, 0.0, 100.0, np.array([100.0]), 1e-7, 1e-7, "sumsq",
+                   name="kin8")
+
+
 def by_name(name: str, n: int | None = None, dtype: str | None = None, seed_offset: int = 0) -> Problem:
     if name == "lorenz_small":
         return lorenz_small(n, seed_offset)
@@ -143,6 +165,8 @@ def by_name(name: str, n: int | None = None, dtype: str | None = None, seed_offs
         return robertson(n, seed_offset)
     if name == "node64":
         return node64(n, seed_offset, dtype or "f32")
+    if name == "kin8":
+        return kin8(n, seed_offset)
     if name == "hires":
         raise NotImplementedError("hires: the HIRES equations and constants are not available here")
     raise KeyError(name)
