@@ -78,6 +78,24 @@ WORKLOADS = {
                            method="ros3", n=65536, dtype="f64",
                            desc="Robertson d=3, t in [0,1e5], ROS3 (Sandu et al. 1997, order 3), rtol=1e-6 "
                                 "atol=1e-10, loss w . u(T), 1 record + 1 gradient pass"),
+    # the Rosenbrock path at d = 8 (kin8, 8 x 8 LU per step): the forward ROS3
+    # step 966 (26 add, 76 mul, 428 fma, 8 divisions: oracle count of the dense
+    # LU, its solves and the stages) + the transposed step 702 (hand count:
+    # three transposed LU solves 360, two kin8 VJPs 108, the second-derivative
+    # term 128, the stage combinations 106)
+    "kin8": dict(passes=1, flop_step=966 + 702, flop_save=32, kernel="k_grad_kin8", n=262144, dtype="f64",
+                 desc="kin8 d=8 stiff mass-action network (stands in for HIRES at its size), t in [0,100], ROS3 "
+                      "rtol=atol=1e-7, loss sum ||u(T)||^2, 1 record + 1 gradient pass"),
+    # the same with ROS2 (the configuration's second-order method): ~16,000
+    # steps per trajectory at this tolerance, so a sixteenth of the ensemble
+    # (checkpoints ~17 GB); forward step 807 (26 add, 77 mul, 348 fma, 8
+    # divisions, oracle count) + transposed step 503 (hand count: two
+    # transposed LU solves 240, two VJPs 108, second-derivative term 97,
+    # combinations 58)
+    "kin8_ros2": dict(passes=1, flop_step=807 + 503, flop_save=32, kernel="k_grad_kin8", problem="kin8",
+                      method="ros2", n=16384, dtype="f64", smax=20000,
+                      desc="kin8 d=8 stiff mass-action network, t in [0,100], ROS2 gamma=1+1/sqrt2 "
+                           "rtol=atol=1e-7, loss sum ||u(T)||^2, 1 record + 1 gradient pass"),
     "node64": dict(passes=1, flop_step=52992 + 104076, flop_save=384, kernel="k_replay_node64", n=131072,
                    dtype="f32",
                    desc="du/dt = tanh(W u + b_i) - u, d=64, shared W, t in [0,1], Tsit5 rtol=atol=1e-5, "
@@ -219,14 +237,16 @@ def bus_id_of(dev) -> str | None:
 
 def smax_cap(workload):
     import workloads
-    return 4 * workloads.SMAX[WORKLOADS[workload].get("problem", workload)]
+    W = WORKLOADS[workload]
+    return W.get("smax") or 4 * workloads.SMAX[W.get("problem", workload)]
 
 
-def oracle_step_time(prob, threads, passes, dense=False):
-    """Oracle record + `passes` tape gradient passes of `prob` on the host."""
+def oracle_step_time(prob, threads, passes, cap, dense=False):
+    """Oracle record (step capacity `cap`) + `passes` tape gradient passes of
+    `prob` on the host."""
     import oracle
     t0 = time.perf_counter()
-    om = oracle.record(prob, smax_cap(prob.name), nthreads=threads, dense=dense)
+    om = oracle.record(prob, cap, nthreads=threads, dense=dense)
     t1 = time.perf_counter()
     oracle.grad(prob, om, nthreads=threads)
     t2 = time.perf_counter()
@@ -255,7 +275,8 @@ def cpu_baseline(args, sample: int):
                 "sample": f"first {sample} of the {args.n} trajectories on the oracle's own mesh: dual-number "
                           f"sensitivities {dt:.2f} s"}
     passes = WORKLOADS[args.workload]["passes"]
-    tr, tg, per_step = oracle_step_time(prob, threads, passes, WORKLOADS[args.workload].get("dense", False))
+    tr, tg, per_step = oracle_step_time(prob, threads, passes, smax_cap(args.workload),
+                                        WORKLOADS[args.workload].get("dense", False))
     return {"value": sample * passes / per_step, "unit": "trajectory-gradients/s", "cores": threads,
             "kind": "oracle",
             "sample": f"first {sample} of the {args.n} trajectories: oracle record {tr:.2f} s + one tape gradient "
@@ -274,7 +295,7 @@ def run_reference(args):
     solve = kind != "grad"
     sample = {"lorenz_1m": 256, "lorenz_1m_dense": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
               "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512, "robertson_ros3": 256,
-              "robertson_ros3_sens": 256}[args.workload]
+              "robertson_ros3_sens": 256, "kin8": 256, "kin8_ros2": 16}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
     om = oracle.record(prob, smax_cap(args.workload), nthreads=threads) if kind == "sens" else None
@@ -676,7 +697,7 @@ def run_ours(args):
         # samples sized for seconds of host work (and host memory for the
         # oracle's trajectory-major meshes)
         sample = {"lorenz_1m": 32768, "lorenz_1m_dense": 32768, "lorenz_small": 1024, "robertson": 256,
-                  "robertson_ros3": 2048, "node64": 1024}[args.workload]
+                  "robertson_ros3": 2048, "node64": 1024, "kin8": 2048, "kin8_ros2": 128}[args.workload]
         line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
     if world > 1:
         dist.barrier()

@@ -32,6 +32,9 @@ template <typename T>
 gs_status launch_grad_ros3(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                            cudaStream_t);
 template <typename T>
+gs_status launch_grad_kin8(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
+                           cudaStream_t);
+template <typename T>
 gs_status launch_solve3(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 gs_status record_node64(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
 gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,
@@ -59,6 +62,11 @@ static gs_status check_problem(const gs_problem* P) {
       if (P->n > 0 && !P->shared) return GS_EINVAL;
       // built for the single-precision Tsit5 configuration
       if (P->method != GS_TSIT5 || P->dtype != GS_F32) return GS_EUNSUPPORTED;
+      break;
+    case GS_KIN8:
+      if (P->d != 8 || P->np != 8) return GS_EINVAL;
+      // a stiff system: built for the Rosenbrock methods
+      if (P->method == GS_TSIT5) return GS_EUNSUPPORTED;
       break;
     case GS_HIRES:
       return GS_EUNSUPPORTED;
@@ -200,6 +208,9 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (P->method == GS_TSIT5 && P->system == GS_LORENZ)
     return P->dtype == GS_F64 ? launch_grad_tsit5_lorenz<double>(P, M, Ls, loss, dp, du0, ws, st)
                               : launch_grad_tsit5_lorenz<float>(P, M, Ls, loss, dp, du0, ws, st);
+  if (P->system == GS_KIN8)
+    return P->dtype == GS_F64 ? launch_grad_kin8<double>(P, M, Ls, loss, dp, du0, ws, st)
+                              : launch_grad_kin8<float>(P, M, Ls, loss, dp, du0, ws, st);
   if (P->method == GS_ROS2)
     return P->dtype == GS_F64 ? launch_grad_ros2<double>(P, M, Ls, loss, dp, du0, ws, st)
                               : launch_grad_ros2<float>(P, M, Ls, loss, dp, du0, ws, st);
@@ -216,7 +227,7 @@ gs_status gs_sens(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
   // Tsit5: Lorenz; ROS2 / ROS3: Lorenz and Robertson; no dense save points
-  if (M->save_theta || P->system == GS_NODE64) return GS_EUNSUPPORTED;
+  if (M->save_theta || P->system == GS_NODE64 || P->system == GS_KIN8) return GS_EUNSUPPORTED;
   if (P->method == GS_TSIT5 && P->system != GS_LORENZ) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;

@@ -1,5 +1,6 @@
-// record.cu -- adaptive recorder (Tsit5 / ROS2, d = 3 systems), the sizing
-// pass and the ordering of mesh slots by step count.
+// record.cu -- adaptive recorder (Tsit5 / ROS2 / ROS3 on the d = 3 systems,
+// ROS2 / ROS3 on the d = 8 one), the sizing pass and the ordering of mesh
+// slots by step count.
 //
 // GRADSOLVE (arXiv 2609.02876), gptget summary "Methodology" and evolve.pub
 // review "Summary": one adaptive solve per trajectory records the accepted
@@ -25,15 +26,15 @@
 // in order, writes coalesced) and zero-fills the h rows past each slot's last
 // step.  The gradient kernels then find chains of
 // nearly equal length in every warp.
-#include "steps.cuh"
+#include "kin8.cuh"
 
 namespace gs {
 
 template <typename T>
 struct RecArgs {
   int64_t n;
-  const T* p;   // [3][n] by trajectory
-  const T* u0;  // [3][n] by trajectory
+  const T* p;   // [d][n] by trajectory
+  const T* u0;  // [d][n] by trajectory
   T t0, t1, rtol, atol, h0;
   int32_t nsave;
   int32_t smax;
@@ -47,7 +48,7 @@ struct RecArgs {
   int32_t* nsteps;       // [n] (may be null in solve mode)
   int32_t* status;       // [n] (may be null in count and solve modes)
   int32_t* nreject;      // [n] (may be null)
-  T* u_save;             // solve mode: [nsave][3][n] by trajectory
+  T* u_save;             // solve mode: [nsave][d][n] by trajectory
 };
 
 // What a recorder pass writes besides the counts: nothing (the sizing pass),
@@ -55,32 +56,33 @@ struct RecArgs {
 enum RecMode { kRecCount = 0, kRecMesh = 1, kRecSolve = 2 };
 
 template <typename T, int SYS, int METHOD>
-__device__ T initial_step3(const T u0[3], const T p[3], T t0, T t1, T rtol, T atol) {
+__device__ T initial_step_d(const T* u0, const T* p, T t0, T t1, T rtol, T atol) {
+  constexpr int D = SysDim<SYS>::D;
   const T q = cst<T>(method_order(METHOD));
-  T sc[3], f0[3], u1[3], f1[3], df[3];
+  T sc[D], f0[D], u1[D], f1[D], df[D];
 #pragma unroll
-  for (int c = 0; c < 3; ++c) sc[c] = fmaT(rtol, fabs(u0[c]), atol);
-  rhs3<T, SYS>(u0, p, f0);
-  T d0 = rms3(u0, sc);
-  T d1 = rms3(f0, sc);
+  for (int c = 0; c < D; ++c) sc[c] = fmaT(rtol, fabs(u0[c]), atol);
+  rhs_s<T, SYS>(u0, p, f0);
+  T d0 = rms_d<T, D>(u0, sc);
+  T d1 = rms_d<T, D>(f0, sc);
   T h0 = (d0 < cst<T>(1e-5) || d1 < cst<T>(1e-5)) ? cst<T>(1e-6) : cst<T>(0.01) * (d0 / d1);
   h0 = smin_(h0, t1 - t0);
 #pragma unroll
-  for (int c = 0; c < 3; ++c) u1[c] = fmaT(h0, f0[c], u0[c]);
-  rhs3<T, SYS>(u1, p, f1);
+  for (int c = 0; c < D; ++c) u1[c] = fmaT(h0, f0[c], u0[c]);
+  rhs_s<T, SYS>(u1, p, f1);
 #pragma unroll
-  for (int c = 0; c < 3; ++c) df[c] = f1[c] - f0[c];
-  T d2 = rms3(df, sc) / h0;
+  for (int c = 0; c < D; ++c) df[c] = f1[c] - f0[c];
+  T d2 = rms_d<T, D>(df, sc) / h0;
   T dm = smax_(d1, d2);
   T h1 = dm <= cst<T>(1e-15) ? smax_(cst<T>(1e-6), h0 * cst<T>(1e-3)) : ctrl_pow<T>(cst<T>(0.01) / dm, cst<T>(1.0) / q);
   return smin_(smin_(cst<T>(100.0) * h0, h1), t1 - t0);
 }
 
-// One recorder trajectory held by a lane.
-template <typename T>
+// One recorder trajectory held by a lane (D components).
+template <typename T, int D>
 struct Traj {
   int64_t i;  // trajectory index
-  T u[3], p[3], k1[3];
+  T u[D], p[D], k1[D];
   T t, hprop, lnprev;
   int nst, nrej, status, kk;
   bool prev_rej;
@@ -88,11 +90,12 @@ struct Traj {
 
 // Load trajectory i and choose its first step; false if it cannot start.
 template <typename T, int SYS, int METHOD>
-__device__ __forceinline__ bool traj_start(const RecArgs<T>& a, int64_t i, Traj<T>& r) {
+__device__ __forceinline__ bool traj_start(const RecArgs<T>& a, int64_t i, Traj<T, SysDim<SYS>::D>& r) {
+  constexpr int D = SysDim<SYS>::D;
   const int64_t n = a.n;
   r.i = i;
 #pragma unroll
-  for (int c = 0; c < 3; ++c) {
+  for (int c = 0; c < D; ++c) {
     r.u[c] = a.u0[c * n + i];
     r.p[c] = a.p[c * n + i];
   }
@@ -103,13 +106,13 @@ __device__ __forceinline__ bool traj_start(const RecArgs<T>& a, int64_t i, Traj<
   r.prev_rej = false;
   r.t = a.t0;
   r.lnprev = cst<T>(0.0);  // the controller carries ln(errprev); errprev starts at 1
-  rhs3<T, SYS>(r.u, r.p, r.k1);
+  rhs_s<T, SYS>(r.u, r.p, r.k1);
   bool finite = true;
 #pragma unroll
-  for (int c = 0; c < 3; ++c) finite = finite && isfinite(r.k1[c]) && isfinite(r.u[c]);
+  for (int c = 0; c < D; ++c) finite = finite && isfinite(r.k1[c]) && isfinite(r.u[c]);
   r.hprop = cst<T>(0.0);
   if (finite) {
-    r.hprop = a.h0 > cst<T>(0.0) ? a.h0 : initial_step3<T, SYS, METHOD>(r.u, r.p, a.t0, a.t1, a.rtol, a.atol);
+    r.hprop = a.h0 > cst<T>(0.0) ? a.h0 : initial_step_d<T, SYS, METHOD>(r.u, r.p, a.t0, a.t1, a.rtol, a.atol);
     if (!(r.hprop > cst<T>(0.0)) || !isfinite(r.hprop)) finite = false;
   }
   if (!finite) r.status = GS_TRAJ_NONFINITE;
@@ -119,7 +122,8 @@ __device__ __forceinline__ bool traj_start(const RecArgs<T>& a, int64_t i, Traj<
 // One attempted step of a running trajectory; true when it has ended (reached
 // t1 or failed).
 template <typename T, int SYS, int METHOD, int MODE>
-__device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T ln_floor) {
+__device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim<SYS>::D>& r, T ln_floor) {
+  constexpr int D = SysDim<SYS>::D;
   const int64_t n = a.n;
   const T eps = Eps<T>::v;
   const T q = cst<T>(method_order(METHOD));
@@ -131,21 +135,25 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
   const T tn = r.t + r.hprop;
   const bool clipped = tn >= tstop - cst<T>(4.0) * eps * fabs(tstop);
   const T h = clipped ? tstop - r.t : r.hprop;
-  T un[3], k7[3], e[3];
-  if (METHOD == GS_TSIT5) {
+  T un[D], k7[D], e[D];
+  if constexpr (METHOD == GS_TSIT5) {
+    static_assert(D == 3, "Tsit5 recorder: d = 3 systems");
     tsit5_err_step<T, SYS>(r.u, r.p, h, r.k1, un, k7, e);
   } else {
-    const bool ok = METHOD == GS_ROS3 ? ros3_err_step<T, SYS>(r.u, r.p, h, un, e)
-                                      : ros2_err_step<T, SYS>(r.u, r.p, h, un, e);
+    bool ok;
+    if constexpr (SYS == GS_KIN8)
+      ok = METHOD == GS_ROS3 ? kin8_ros3_err_step<T>(r.u, r.p, h, un, e) : kin8_ros2_err_step<T>(r.u, r.p, h, un, e);
+    else
+      ok = METHOD == GS_ROS3 ? ros3_err_step<T, SYS>(r.u, r.p, h, un, e) : ros2_err_step<T, SYS>(r.u, r.p, h, un, e);
     if (!ok) {
       r.status = GS_TRAJ_SINGULAR;
       return true;
     }
   }
-  T sc[3];
+  T sc[D];
 #pragma unroll
-  for (int c = 0; c < 3; ++c) sc[c] = fmaT(a.rtol, smax_(fabs(r.u[c]), fabs(un[c])), a.atol);
-  const T err = rms3(e, sc);
+  for (int c = 0; c < D; ++c) sc[c] = fmaT(a.rtol, smax_(fabs(r.u[c]), fabs(un[c])), a.atol);
+  const T err = rms_d<T, D>(e, sc);
   const bool accept = err <= cst<T>(1.0);
   // The controller's power function, once for either outcome (each outcome's
   // own formula, so a lane's arithmetic is that of a branch per outcome, but a
@@ -165,7 +173,7 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
     ++r.nst;
     const T tprev = r.t;
     r.t = clipped ? tstop : tn;
-    if (METHOD == GS_TSIT5 && a.dense) {
+    if (METHOD == GS_TSIT5 && D == 3 && a.dense) {
       // every save time this step passed: its position inside the step, and
       // (solve) the Hermite state there from u, f(u) = k1, u_new, f(u_new) = k7
       while (r.kk < a.nsave && a.tsave[r.kk] <= r.t) {
@@ -177,15 +185,15 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
         if (MODE == kRecSolve) {
           const HermiteW<T> w = hermite_w(th);
 #pragma unroll
-          for (int c = 0; c < 3; ++c)
-            a.u_save[((int64_t)r.kk * 3 + c) * n + r.i] =
+          for (int c = 0; c < D; ++c)
+            a.u_save[((int64_t)r.kk * D + c) * n + r.i] =
                 th == cst<T>(1.0) ? un[c] : hermite_c(w, r.u[c], un[c], r.k1[c], k7[c], h);
         }
         ++r.kk;
       }
     }
 #pragma unroll
-    for (int c = 0; c < 3; ++c) {
+    for (int c = 0; c < D; ++c) {
       r.u[c] = un[c];
       if (METHOD == GS_TSIT5) r.k1[c] = k7[c];
     }
@@ -193,7 +201,7 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
       if (MODE == kRecMesh) a.save_idx[(int64_t)r.kk * n + r.i] = r.nst;
       if (MODE == kRecSolve) {
 #pragma unroll
-        for (int c = 0; c < 3; ++c) a.u_save[((int64_t)r.kk * 3 + c) * n + r.i] = r.u[c];
+        for (int c = 0; c < D; ++c) a.u_save[((int64_t)r.kk * D + c) * n + r.i] = r.u[c];
       }
       ++r.kk;
     }
@@ -218,8 +226,8 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T>& r, T 
 }
 
 // Outputs of an ended trajectory.
-template <typename T, int MODE>
-__device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T>& r) {
+template <typename T, int MODE, int D>
+__device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T, D>& r) {
   const int64_t n = a.n;
   if (MODE == kRecMesh) {
     // unreached save points (a failed trajectory); the h tail stays unwritten
@@ -233,7 +241,7 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T>& 
     const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
     for (int k = 0; k < a.nsave; ++k)
 #pragma unroll
-      for (int c = 0; c < 3; ++c) a.u_save[((int64_t)k * 3 + c) * n + r.i] = nan;
+      for (int c = 0; c < D; ++c) a.u_save[((int64_t)k * D + c) * n + r.i] = nan;
   }
   if (a.nsteps) a.nsteps[r.i] = r.nst;
   if (a.status) a.status[r.i] = r.status;
@@ -242,10 +250,12 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T>& 
 
 // 6 resident blocks of 128 per SM (85 registers a thread): measured faster on
 // B200 than the unconstrained 90-92 registers at 5 blocks, and than 7 or 8
-// blocks (more spilling).
+// blocks (more spilling).  The d = 8 system (an 8 x 8 LU per step) takes the
+// registers it needs.
 #ifndef GS_REC_MINB
 #define GS_REC_MINB 6
 #endif
+template <int SYS> constexpr int rec_minb() { return SYS == GS_KIN8 ? 1 : GS_REC_MINB; }
 
 // Each warp owns the trajectories [w * chunk, (w + 1) * chunk) and its lanes
 // take them in turn: a lane whose trajectory has ended takes the next one of
@@ -256,7 +266,7 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T>& 
 // hands out chunk entries or advances some trajectory's accepted or rejected
 // step count, and both are capped by smax.
 template <typename T, int SYS, int METHOD, int MODE>
-__global__ void __launch_bounds__(128, GS_REC_MINB) k_record3(RecArgs<T> a) {
+__global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3(RecArgs<T> a) {
   const unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
@@ -266,7 +276,7 @@ __global__ void __launch_bounds__(128, GS_REC_MINB) k_record3(RecArgs<T> a) {
   if (c0 >= c1) return;  // whole warp
   int64_t next = c0;
   const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));  // errprev is floored at 1e-4
-  Traj<T> r;
+  Traj<T, SysDim<SYS>::D> r;
   bool run = false;
   for (;;) {
     const unsigned need = __ballot_sync(kFull, !run);
@@ -404,6 +414,8 @@ static gs_status dispatch_rec(int sys, int method, const RecArgs<T>& a, cudaStre
   if (sys == GS_ROBERTSON && method == GS_ROS2) return launch_rec<T, kSysRobertson, GS_ROS2, MODE>(a, st);
   if (sys == GS_LORENZ && method == GS_ROS3) return launch_rec<T, kSysLorenz, GS_ROS3, MODE>(a, st);
   if (sys == GS_ROBERTSON && method == GS_ROS3) return launch_rec<T, kSysRobertson, GS_ROS3, MODE>(a, st);
+  if (sys == GS_KIN8 && method == GS_ROS2) return launch_rec<T, kSysKin8, GS_ROS2, MODE>(a, st);
+  if (sys == GS_KIN8 && method == GS_ROS3) return launch_rec<T, kSysKin8, GS_ROS3, MODE>(a, st);
   return GS_EUNSUPPORTED;
 }
 

@@ -1,5 +1,5 @@
 // rosenbrock.cuh -- pieces shared by the fused replay + reverse sweep kernels
-// of the Rosenbrock methods (grad_ros2.cu, grad_ros3.cu), d = 3 systems: the
+// of the Rosenbrock methods (grad_ros2.cu, grad_ros3.cu, grad_kin8.cu): the
 // kernels' arguments, the right-hand sides' vector-Jacobian products, and the
 // loss terms and their gradients at the save points.
 #pragma once
@@ -52,11 +52,12 @@ __device__ __forceinline__ void vjp3(const T u[3], const T p[3], const T w[3], T
   }
 }
 
-template <typename T>
+// Loss terms of one save point (D components at o + c n of target / weight).
+template <typename T, int D = 3>
 __device__ __forceinline__ void loss_terms3(int kind, const T* target, const T* weight, int64_t o, int64_t n,
-                                            const T u[3], T& L) {
+                                            const T* u, T& L) {
 #pragma unroll
-  for (int c = 0; c < 3; ++c) {
+  for (int c = 0; c < D; ++c) {
     if (kind == GS_LOSS_SUMSQ) {
       T dl = target ? u[c] - target[o + c * n] : u[c];
       L = fmaT(dl, dl, L);
@@ -66,11 +67,11 @@ __device__ __forceinline__ void loss_terms3(int kind, const T* target, const T* 
   }
 }
 
-template <typename T>
+template <typename T, int D = 3>
 __device__ __forceinline__ void loss_grad3(int kind, const T* target, const T* weight, int64_t o, int64_t n,
-                                           const T u[3], T lam[3]) {
+                                           const T* u, T* lam) {
 #pragma unroll
-  for (int c = 0; c < 3; ++c) {
+  for (int c = 0; c < D; ++c) {
     if (kind == GS_LOSS_SUMSQ)
       lam[c] = fmaT(cst<T>(2.0), target ? u[c] - target[o + c * n] : u[c], lam[c]);
     else

@@ -1,8 +1,9 @@
 // solve.cu -- forward-only fixed-step replay on a recorded mesh, writing the
-// state at every save point (d = 3 systems, Tsit5 or ROS2).  The forward-only
+// state at every save point (d = 3 systems with Tsit5, ROS2 or ROS3; the
+// d = 8 system with ROS2 or ROS3).  The forward-only
 // use of GRADSOLVE (arXiv 2609.02876, abstract); same arithmetic as the
 // forward half of the gradient kernels.
-#include "steps.cuh"
+#include "kin8.cuh"
 
 namespace gs {
 
@@ -19,39 +20,47 @@ struct SolveArgs {
   int32_t nsave;
   int32_t smax;
   const T* theta;  // [nsave][n] by slot: dense save points (Tsit5), or null
-  T* u_save;       // [nsave][3][n] by trajectory
+  T* u_save;       // [nsave][d][n] by trajectory
 };
 
 template <typename T, int SYS, int METHOD>
 __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
+  constexpr int D = SysDim<SYS>::D;
   const int64_t n = a.n;
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n) return;
   const int64_t i = a.order[j];
   if (i < 0 || i >= n) return;  // not a permutation entry: nothing to write
-  const int64_t n3 = 3 * n;
+  const int64_t n3 = D * n;
   if (a.status[j] != GS_TRAJ_OK || a.nsteps[j] < 0 || a.nsteps[j] > a.smax) {
     const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
     for (int k = 0; k < a.nsave; ++k)
 #pragma unroll
-      for (int c = 0; c < 3; ++c) a.u_save[k * n3 + c * n + i] = nan;
+      for (int c = 0; c < D; ++c) a.u_save[k * n3 + c * n + i] = nan;
     return;
   }
-  T u[3], p[3], k1[3];
+  T u[D], p[D], k1[D];
 #pragma unroll
-  for (int c = 0; c < 3; ++c) {
+  for (int c = 0; c < D; ++c) {
     u[c] = a.u0[c * n + i];
     p[c] = a.p[c * n + i];
   }
-  rhs3<T, SYS>(u, p, k1);
+  rhs_s<T, SYS>(u, p, k1);
   const int S = a.nsteps[j];
   int kk = 0;
   int next = a.save_idx[j];
   const T* hp = a.h + j;
   for (int st = 0; st < S; ++st) {
     const T h = hp[(int64_t)st * n];
-    T un[3];
-    if (METHOD == GS_TSIT5) {
+    T un[D];
+    if constexpr (SYS == GS_KIN8) {
+      T LU[64], R[8], q1[8], v[8], q2[8], q3[8];
+      int P[8];
+      if constexpr (METHOD == GS_ROS3)
+        kin8_ros3_fwd<T>(u, p, h, LU, P, R, q1, v, q2, q3, un);
+      else
+        kin8_ros2_fwd<T>(u, p, h, LU, P, R, q1, v, q2, un);
+    } else if constexpr (METHOD == GS_TSIT5) {
       T k7[3], e[3];
       tsit5_err_step<T, SYS>(u, p, h, k1, un, k7, e);
       if (a.theta) {
@@ -79,10 +88,10 @@ __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
       ros2_fwd<T, SYS>(u, p, h, LU, P, R, q1, v, q2, un);
     }
 #pragma unroll
-    for (int c = 0; c < 3; ++c) u[c] = un[c];
+    for (int c = 0; c < D; ++c) u[c] = un[c];
     while (st + 1 == next) {
 #pragma unroll
-      for (int c = 0; c < 3; ++c) a.u_save[kk * n3 + c * n + i] = u[c];
+      for (int c = 0; c < D; ++c) a.u_save[kk * n3 + c * n + i] = u[c];
       ++kk;
       next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
     }
@@ -115,6 +124,10 @@ gs_status launch_solve3(const gs_problem* P, const gs_mesh* M, void* u_save, cud
     k_solve3<T, kSysRobertson, GS_TSIT5><<<grid, 128, 0, st>>>(a);
   else if (P->system == GS_ROBERTSON && P->method == GS_ROS3)
     k_solve3<T, kSysRobertson, GS_ROS3><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_KIN8 && P->method == GS_ROS3)
+    k_solve3<T, kSysKin8, GS_ROS3><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_KIN8 && P->method == GS_ROS2)
+    k_solve3<T, kSysKin8, GS_ROS2><<<grid, 128, 0, st>>>(a);
   else
     k_solve3<T, kSysRobertson, GS_ROS2><<<grid, 128, 0, st>>>(a);
   count_launch();

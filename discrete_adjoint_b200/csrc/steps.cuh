@@ -1,7 +1,7 @@
-// steps.cuh -- the d = 3 step formulas of the forward replay (Tsit5 and
-// ROS2 on Lorenz and Robertson), written in the floating-point contract's
-// operation order.  Shared by the recorder, the Rosenbrock gradient kernel and
-// the forward-only solve.
+// steps.cuh -- the d = 3 step formulas of the forward replay (Tsit5, ROS2
+// and ROS3 on Lorenz and Robertson), written in the floating-point contract's
+// operation order.  Shared by the recorder, the Rosenbrock gradient kernels
+// and the forward-only solve (kin8.cuh adds the d = 8 system on top).
 #pragma once
 
 #include "common.cuh"
@@ -141,15 +141,16 @@ __device__ __forceinline__ T hermite_c(const HermiteW<T>& w, T us, T un, T fs, T
   return fmaT(w.h00, us, fmaT(w.h01, un, h * fmaT(w.h10, fs, w.h11 * fn)));
 }
 
-template <typename T>
-__device__ __forceinline__ T rms3(const T x[3], const T sc[3]) {
+// RMS of x / sc over D components (the error norm), in the contract's order.
+template <typename T, int D>
+__device__ __forceinline__ T rms_d(const T* x, const T* sc) {
   T s = cst<T>(0.0);
 #pragma unroll
-  for (int c = 0; c < 3; ++c) {
+  for (int c = 0; c < D; ++c) {
     T q = x[c] / sc[c];
     s = fmaT(q, q, s);
   }
-  return sqrt(s / cst<T>(3.0));
+  return sqrt(s / cst<T>((double)D));
 }
 
 // One Tsit5 step with error estimate; k1 = f(u) on entry, k7 = f(u_new) out.

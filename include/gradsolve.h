@@ -67,13 +67,21 @@ typedef int32_t gs_status;
 #define GS_ROBERTSON 2 /* d=3, np=3, p=(k1, k2, k3): mass-action kinetics A->B, 2B->B+C, B+C->A+C */
 #define GS_HIRES 3     /* reserved: not implemented (equations not given by the sources followed) */
 #define GS_NODE64 4    /* d=64, np=64 (b_i), shared W [64][64]: f = tanh(W u + b) - u */
+/* d=8, np=8 (k1..k8), GS_ROS2 / GS_ROS3 only: kin8, an 8-species stiff
+ * mass-action network defined by this library (not a published test problem)
+ * that runs the Rosenbrock path at d = 8 (8 x 8 LU in registers):
+ *   A1 -> A2 (k1), A2 -> A1 (k2), A2 + A3 -> A4 (k3), A4 -> A3 + A5 (k4),
+ *   A5 -> A6 (k5), A6 -> A5 (k6), A6 + A7 -> A8 (k7), A8 -> A7 + A1 (k8);
+ * f = N r(u), r = (k1 u1, k2 u2, k3 u2 u3, k4 u4, k5 u5, k6 u6, k7 u6 u7,
+ * k8 u8) with N the reactions' stoichiometric matrix. */
+#define GS_KIN8 5
 
 /* Integrators. */
 #define GS_TSIT5 1 /* Tsitouras 5(4) pair, FSAL, PI step control */
-#define GS_ROS2 2  /* Rosenbrock ROS2, gamma = 1 + 1/sqrt(2) (Verwer et al. 1999); d = 3 only */
+#define GS_ROS2 2  /* Rosenbrock ROS2, gamma = 1 + 1/sqrt(2) (Verwer et al. 1999); d = 3 and kin8 */
 /* Rosenbrock ROS3 (Sandu, Verwer, Blom, Spee, Carmichael & Potra 1997): three
  * stages, order 3, L-stable, embedded order 2, controller order q = 3; d = 3
- * only.  Stage form, with J = J(u) and gamma = 0.435866521508459:
+ * and kin8.  Stage form, with J = J(u) and gamma = 0.435866521508459:
  *   M = I/gamma - h J;  M k1 = f(u);  v = u + h k1;  M k2 = f(v) + c21 k1;
  *   M k3 = f(v) + c31 k1 + c32 k2;  u_new = u + h (k1 + m2 k2 + m3 k3);
  *   error estimate h (e1 k1 + e2 k2 + e3 k3).  Higher-order stiff option of

@@ -50,7 +50,7 @@ FULL_N = {"lorenz_small": 1024, "lorenz_1m": 1 << 20, "robertson": 65536, "hires
 
 # Recorded-step capacity each workload is sized for (the recorder reports
 # MAXSTEPS beyond it); generous relative to the observed maxima.
-SMAX = {"lorenz_small": 256, "lorenz_1m": 1024, "robertson": 8192, "node64": 256}
+SMAX = {"lorenz_small": 256, "lorenz_1m": 1024, "robertson": 8192, "node64": 256, "kin8": 2048}
 
 
 @dataclass
