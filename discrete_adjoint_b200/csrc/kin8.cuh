@@ -174,7 +174,7 @@ struct Kin8JacAdj {
 
 // ---------------------------------------------------------------------------
 // Compile-time loops.  sfor<B, E>(f) calls f(Ix<B>{}) .. f(Ix<E-1>{}); the body
-// reads its index as a constant (IX(i)).  The triangular loop nests of an 8 x 8
+// reads its index as a constant (GS_IX(i)).  The triangular loop nests of an 8 x 8
 // LU written with #pragma unroll are not fully unrolled by the compiler, which
 // then keeps the matrix in local memory; with constant indices it stays in
 // registers.
@@ -190,7 +190,7 @@ __device__ __forceinline__ void sfor(F&& f) {
     sfor<B + 1, E>(f);
   }
 }
-#define IX(x) decltype(x)::v
+#define GS_IX(x) decltype(x)::v
 
 // ---------------------------------------------------------------------------
 // D x D LU with partial pivoting (largest |entry|, ties to the lowest row),
@@ -200,24 +200,24 @@ __device__ __forceinline__ void sfor(F&& f) {
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __device__ __forceinline__ bool lu_d(T M[D * D], int P[D], T R[D]) {
-  sfor<0, D>([&](auto q_) { P[IX(q_)] = IX(q_); });
+  sfor<0, D>([&](auto q_) { P[GS_IX(q_)] = GS_IX(q_); });
   bool ok = true;
   sfor<0, D>([&](auto k_) {
-    constexpr int k = IX(k_);
+    constexpr int k = GS_IX(k_);
     int piv = k;
     T best = fabs(M[k * D + k]);
     sfor<k + 1, D>([&](auto i_) {
-      constexpr int i = IX(i_);
+      constexpr int i = GS_IX(i_);
       const T a = fabs(M[i * D + k]);
       const bool gt = a > best;
       best = gt ? a : best;
       piv = gt ? i : piv;
     });
     sfor<k + 1, D>([&](auto i_) {
-      constexpr int i = IX(i_);
+      constexpr int i = GS_IX(i_);
       const bool sw = piv == i;
       sfor<0, D>([&](auto j_) {
-        constexpr int j = IX(j_);
+        constexpr int j = GS_IX(j_);
         const T x = M[k * D + j], y = M[i * D + j];
         M[k * D + j] = sw ? y : x;
         M[i * D + j] = sw ? x : y;
@@ -230,11 +230,11 @@ __device__ __forceinline__ bool lu_d(T M[D * D], int P[D], T R[D]) {
     ok = ok && (pv != cst<T>(0.0)) && isfinite(pv);
     R[k] = cst<T>(1.0) / pv;
     sfor<k + 1, D>([&](auto i_) {
-      constexpr int i = IX(i_);
+      constexpr int i = GS_IX(i_);
       const T l = M[i * D + k] * R[k];
       M[i * D + k] = l;
       sfor<k + 1, D>([&](auto j_) {
-        constexpr int j = IX(j_);
+        constexpr int j = GS_IX(j_);
         M[i * D + j] = fmaT(-l, M[k * D + j], M[i * D + j]);
       });
     });
@@ -248,18 +248,18 @@ __device__ __forceinline__ bool lu_d(T M[D * D], int P[D], T R[D]) {
 template <typename T, int D>
 __device__ __forceinline__ void lu_d_solve(const T LU[D * D], const int P[D], const T R[D], const T b[D], T x[D]) {
   sfor<0, D>([&](auto i_) {
-    constexpr int i = IX(i_);
+    constexpr int i = GS_IX(i_);
     T v = b[0];
-    sfor<1, D>([&](auto q_) { v = P[i] == IX(q_) ? b[IX(q_)] : v; });
+    sfor<1, D>([&](auto q_) { v = P[i] == GS_IX(q_) ? b[GS_IX(q_)] : v; });
     x[i] = v;
   });
   sfor<1, D>([&](auto i_) {
-    constexpr int i = IX(i_);
-    sfor<0, i>([&](auto j_) { x[i] = fmaT(-LU[i * D + IX(j_)], x[IX(j_)], x[i]); });
+    constexpr int i = GS_IX(i_);
+    sfor<0, i>([&](auto j_) { x[i] = fmaT(-LU[i * D + GS_IX(j_)], x[GS_IX(j_)], x[i]); });
   });
   sfor<0, D>([&](auto r_) {
-    constexpr int i = D - 1 - IX(r_);
-    sfor<i + 1, D>([&](auto j_) { x[i] = fmaT(-LU[i * D + IX(j_)], x[IX(j_)], x[i]); });
+    constexpr int i = D - 1 - GS_IX(r_);
+    sfor<i + 1, D>([&](auto j_) { x[i] = fmaT(-LU[i * D + GS_IX(j_)], x[GS_IX(j_)], x[i]); });
     x[i] = x[i] * R[i];
   });
 }
@@ -272,19 +272,19 @@ template <typename T, int D, typename LUA, typename RA>
 __device__ __forceinline__ void lu_d_solve_T(LUA lu, RA rc, const int P[D], const T b[D], T x[D]) {
   T y[D];
   sfor<0, D>([&](auto i_) {
-    constexpr int i = IX(i_);
+    constexpr int i = GS_IX(i_);
     T acc = b[i];
-    sfor<0, i>([&](auto j_) { acc = fmaT(-lu(IX(j_) * D + i), y[IX(j_)], acc); });
+    sfor<0, i>([&](auto j_) { acc = fmaT(-lu(GS_IX(j_) * D + i), y[GS_IX(j_)], acc); });
     y[i] = acc * rc(i);
   });
   sfor<1, D>([&](auto r_) {
-    constexpr int i = D - 1 - IX(r_);
-    sfor<i + 1, D>([&](auto j_) { y[i] = fmaT(-lu(IX(j_) * D + i), y[IX(j_)], y[i]); });
+    constexpr int i = D - 1 - GS_IX(r_);
+    sfor<i + 1, D>([&](auto j_) { y[i] = fmaT(-lu(GS_IX(j_) * D + i), y[GS_IX(j_)], y[i]); });
   });
   sfor<0, D>([&](auto q_) {
-    constexpr int q = IX(q_);
+    constexpr int q = GS_IX(q_);
     T v = y[0];
-    sfor<1, D>([&](auto i_) { v = P[IX(i_)] == q ? y[IX(i_)] : v; });
+    sfor<1, D>([&](auto i_) { v = P[GS_IX(i_)] == q ? y[GS_IX(i_)] : v; });
     x[q] = v;
   });
 }
