@@ -87,13 +87,13 @@ WORKLOADS = {
                  desc="kin8 d=8 stiff mass-action network (stands in for HIRES at its size), t in [0,100], ROS3 "
                       "rtol=atol=1e-7, loss sum ||u(T)||^2, 1 record + 1 gradient pass"),
     # the same with ROS2 (the configuration's second-order method): ~16,000
-    # steps per trajectory at this tolerance, so a sixteenth of the ensemble
-    # (checkpoints ~17 GB); forward step 807 (26 add, 77 mul, 348 fma, 8
+    # steps per trajectory at this tolerance, so a quarter of the ensemble
+    # (checkpoints ~67 GB); forward step 807 (26 add, 77 mul, 348 fma, 8
     # divisions, oracle count) + transposed step 503 (hand count: two
     # transposed LU solves 240, two VJPs 108, second-derivative term 97,
     # combinations 58)
     "kin8_ros2": dict(passes=1, flop_step=807 + 503, flop_save=32, kernel="k_grad_kin8", problem="kin8",
-                      method="ros2", n=16384, dtype="f64", smax=20000,
+                      method="ros2", n=65536, dtype="f64", smax=20000,
                       desc="kin8 d=8 stiff mass-action network, t in [0,100], ROS2 gamma=1+1/sqrt2 "
                            "rtol=atol=1e-7, loss sum ||u(T)||^2, 1 record + 1 gradient pass"),
     "node64": dict(passes=1, flop_step=52992 + 104076, flop_save=384, kernel="k_replay_node64", n=131072,
@@ -697,7 +697,7 @@ def run_ours(args):
         # samples sized for seconds of host work (and host memory for the
         # oracle's trajectory-major meshes)
         sample = {"lorenz_1m": 32768, "lorenz_1m_dense": 32768, "lorenz_small": 1024, "robertson": 256,
-                  "robertson_ros3": 2048, "node64": 1024, "kin8": 2048, "kin8_ros2": 128}[args.workload]
+                  "robertson_ros3": 2048, "node64": 1024, "kin8": 2048, "kin8_ros2": 64}[args.workload]
         line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
     if world > 1:
         dist.barrier()
