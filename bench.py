@@ -676,6 +676,7 @@ def run_ours(args):
                    "n_per_gpu": n, "passes_per_step": passes, "smax": smax,
                    "steps_total": total_steps, "steps_mean": float(ns.mean()),
                    "steps_max_over_mean": float(ns.max() / ns.mean()),
+                   "rejects_total": int(mesh.nreject.sum().item()),
                    "grad_ms": grad_ms, "record_ms": rec_ms, "grad_only_value": world * n / (grad_ms / 1e3),
                    "l2": "inputs larger than L2 (mesh %.2f GB, gradient workspace %.2f GB); no flush" % (
                        mesh.h.numel() * esz / 1e9, ws_grad.numel() / 1e9),
