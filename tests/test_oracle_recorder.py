@@ -179,6 +179,30 @@ def test_step_operation_counts():
     assert nd["fma"] == 6 * 64 * 64 + 64 * 21 and nd["tanh"] == 6 * 64
 
 
+def test_kin8_step_operation_counts():
+    """The d = 8 Rosenbrock steps on kin8, counted from the method's
+    structure: the Jacobian (4 rate products, 2 sums), M = fma over all 64
+    entries, the dense 8 x 8 LU (8 pivot reciprocals, 28 multipliers, 140
+    updates), two right-hand sides (10 products and 12 sums each), and per
+    solve 56 fma + 8 products by the pivot reciprocals.  The bench's per-step
+    work carries these forward counts."""
+    lu_mul, lu_fma, solve_fma, solve_mul = 28, 140, 56, 8
+    f_add, f_mul = 12, 10
+    r3 = oracle.count_step("kin8", "ros3", 8, 8)
+    # stages: v = u + h k1 (8), two stage right sides (8 + 16), u_new (24)
+    assert r3 == {"add": 2 + 2 * f_add, "mul": 4 + lu_mul + 2 * f_mul + 3 * solve_mul,
+                  "fma": 64 + lu_fma + 3 * solve_fma + 8 + 8 + 16 + 24, "div": 8, "sqrt": 0, "tanh": 0}
+    r2 = oracle.count_step("kin8", "ros2", 8, 8)
+    # gamma h (1 mul), v (8 fma), f(v) - 2 k1 (8 fma), 3/2 k1 (8 mul) + 1/2 k2 and u_new (16 fma)
+    assert r2 == {"add": 2 + 2 * f_add, "mul": 4 + 1 + lu_mul + 2 * f_mul + 2 * solve_mul + 8,
+                  "fma": 64 + lu_fma + 2 * solve_fma + 8 + 8 + 16, "div": 8, "sqrt": 0, "tanh": 0}
+    flop = lambda c: c["add"] + c["mul"] + 2 * c["fma"] + c["div"]
+    assert (flop(r3), flop(r2)) == (966, 807)
+    import bench
+    assert bench.WORKLOADS["kin8"]["flop_step"] == 966 + 702
+    assert bench.WORKLOADS["kin8_ros2"]["flop_step"] == 807 + 503
+
+
 def test_controller_power_function():
     """The controller's x**y (exp/log from IEEE operations only) against the
     library power function: <= 4 ulp on the controller's arguments (errors
