@@ -212,3 +212,117 @@ def test_gradient_matches_fixed_mesh_differences():
     a, b = np.vstack([g["dp"], g["du0"]]), fd
     e = np.abs(a - b).max(0) / np.abs(b).max(0)
     assert e.max() <= 1e-8, e
+
+
+# ---- brute force in 50-digit decimal ------------------------------------------
+def _dec_kin8_replay(method, u, p, hs):
+    """The ROS2 / ROS3 replay of kin8 in 50-digit decimal arithmetic, written
+    from the methods' stage equations with the coefficients as the exact
+    binary values the oracle uses; linear systems by Gaussian elimination."""
+    from decimal import Decimal as D
+
+    def f(y):
+        return [D(x) for x in mass_action_dec(y, p)]
+
+    def J(y):
+        return mass_action_jac_dec(y, p)
+
+    def solve(M, rhs):
+        A = [row[:] + [v] for row, v in zip(M, rhs)]
+        for k in range(8):
+            piv = max(range(k, 8), key=lambda i: abs(A[i][k]))
+            A[k], A[piv] = A[piv], A[k]
+            for i in range(k + 1, 8):
+                l = A[i][k] / A[k][k]
+                for j in range(k, 9):
+                    A[i][j] -= l * A[k][j]
+        x = [D(0)] * 8
+        for i in range(7, -1, -1):
+            x[i] = (A[i][8] - sum(A[i][j] * x[j] for j in range(i + 1, 8))) / A[i][i]
+        return x
+
+    for h in hs:
+        Jm = J(u)
+        if method == "ros2":
+            g = D(oracle.ros2_gamma())
+            M = [[(D(1) if i == j else D(0)) - g * h * Jm[i][j] for j in range(8)] for i in range(8)]
+            k1 = solve(M, f(u))
+            v = [u[q] + h * k1[q] for q in range(8)]
+            fv = f(v)
+            k2 = solve(M, [fv[q] - 2 * k1[q] for q in range(8)])
+            u = [u[q] + h * (D(3) / 2 * k1[q] + D(1) / 2 * k2[q]) for q in range(8)]
+        else:
+            c = {k: D(v) for k, v in oracle.ros3_coeffs().items()}
+            M = [[(c["inv_gamma"] if i == j else D(0)) - h * Jm[i][j] for j in range(8)] for i in range(8)]
+            k1 = solve(M, f(u))
+            v = [u[q] + h * k1[q] for q in range(8)]
+            fv = f(v)
+            k2 = solve(M, [fv[q] + c["c21"] * k1[q] for q in range(8)])
+            k3 = solve(M, [fv[q] + c["c31"] * k1[q] + c["c32"] * k2[q] for q in range(8)])
+            u = [u[q] + h * (k1[q] + c["m2"] * k2[q] + c["m3"] * k3[q]) for q in range(8)]
+    return u
+
+
+def mass_action_dec(u, k):
+    """mass_action in Decimal arithmetic (u, k lists of Decimal)."""
+    N = _stoich()
+    rates = []
+    for r, (re, _) in enumerate(REACTIONS):
+        v = k[r]
+        for s, a in re.items():
+            for _ in range(a):
+                v = v * u[s]
+        rates.append(v)
+    return [sum(int(N[s, r]) * rates[r] for r in range(len(REACTIONS))) for s in range(8)]
+
+
+def mass_action_jac_dec(u, k):
+    N = _stoich()
+    from decimal import Decimal as D
+    dr = [[D(0)] * 8 for _ in REACTIONS]
+    for r, (re, _) in enumerate(REACTIONS):
+        for s, a in re.items():
+            other = k[r]
+            for q, b in re.items():
+                if q != s:
+                    for _ in range(b):
+                        other = other * u[q]
+            dr[r][s] = a * other * (u[s] ** (a - 1) if a > 1 else D(1))
+    return [[sum(int(N[i, r]) * dr[r][j] for r in range(len(REACTIONS))) for j in range(8)] for i in range(8)]
+
+
+@pytest.mark.parametrize("method", ["ros2", "ros3"])
+def test_bruteforce_decimal_tiny(method):
+    """Two trajectories of 3-4 steps up to h = 0.5 (h |lambda_fast| ~ 600, the
+    stiff regime): the oracle's tape gradient and loss against the replay in
+    50-digit decimal differentiated by 1e-20 central differences."""
+    from decimal import Decimal as D, getcontext
+    getcontext().prec = 50
+    prob = W.kin8(2)
+    prob.method = method
+    hs_all = [[0.01, 0.1, 0.5, 0.25], [0.002, 0.3, 0.05]]
+    S = max(len(x) for x in hs_all)
+    h = np.zeros((2, S))
+    for i, hs in enumerate(hs_all):
+        h[i, : len(hs)] = hs
+    ns = np.array([len(x) for x in hs_all], np.int32)
+    mesh = oracle.Mesh(h, ns, ns[:, None].copy(), np.zeros(2, np.int32), np.zeros(2, np.int32))
+    g = oracle.grad(prob, mesh, "tape", nthreads=1)
+    step = D("1e-20")
+    loss = lambda u: sum(x * x for x in u)
+    for i in range(2):
+        hs = [D(float(x)) for x in hs_all[i]]
+        x0 = [D(float(v)) for v in np.concatenate([prob.p[:, i], prob.u0[:, i]])]
+        ref = []
+        for r in range(16):
+            xp, xm = list(x0), list(x0)
+            xp[r] += step
+            xm[r] -= step
+            Lp = loss(_dec_kin8_replay(method, xp[8:], xp[:8], hs))
+            Lm = loss(_dec_kin8_replay(method, xm[8:], xm[:8], hs))
+            ref.append(float((Lp - Lm) / (2 * step)))
+        ref = np.array(ref)
+        got = np.concatenate([g["dp"][:, i], g["du0"][:, i]])
+        assert np.abs(got - ref).max() <= 1e-14 * np.abs(ref).max(), (i, np.abs(got - ref).max())
+        L = float(loss(_dec_kin8_replay(method, x0[8:], x0[:8], hs)))
+        assert abs(g["loss"][i] - L) <= 1e-14 * abs(L)
