@@ -177,3 +177,41 @@ def test_full_size_sampled():
     ti = torch.tensor(idx, device=dev())
     e = grad_rel_err(gs.GradOut(out.loss[ti], out.dp[:, ti], out.du0[:, ti], None), og)
     assert e.max() <= 1e-12, e.max()
+
+
+def test_linear_loss_and_leading_zero_steps():
+    """The weighted-linear loss at three save points, and leading zero steps
+    (exact identities of both Rosenbrock steps) leave loss and gradient
+    bitwise unchanged."""
+    prob = _multi(_kin8(64))
+    prob.loss = "linear"
+    prob.weight = np.random.default_rng(11).uniform(0.0, 1.0, (3, 8, prob.n))
+    om = oracle.record(prob, SMAX3)
+    og = oracle.grad(prob, om)
+    ens = ensemble(prob)
+    out = gs.gs_grad(ens, mesh_from_oracle(om, "f64"), **loss_args(prob))
+    torch.cuda.synchronize()
+    assert grad_rel_err(out, og).max() <= 1e-12
+    z = 2
+    om2 = oracle.Mesh(np.concatenate([np.zeros((prob.n, z)), om.h], 1), om.nsteps + z, om.save_idx + z,
+                      om.status, om.nreject)
+    out2 = gs.gs_grad(ens, mesh_from_oracle(om2, "f64"), **loss_args(prob))
+    torch.cuda.synchronize()
+    for a, b in ((out.loss, out2.loss), (out.dp, out2.dp), (out.du0, out2.du0)):
+        assert torch.equal(a, b)
+
+
+def test_ros2_fp32():
+    prob = _kin8(100, "ros2").as_dtype("f32")
+    prob.rtol = prob.atol = 1e-5
+    om = oracle.record(prob, SMAX2)
+    assert (om.status == 0).all()
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(prob.n, 2048, 1, "f32", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    assert np.array_equal(ns, om.nsteps)
+    out = gs.gs_grad(ens, mesh_from_oracle(om, "f32"), **loss_args(prob))
+    torch.cuda.synchronize()
+    parity(out, prob, om, tol=TOL["f32"])
