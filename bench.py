@@ -84,7 +84,7 @@ WORKLOADS = {
     # three transposed LU solves 360, two kin8 VJPs 108, the second-derivative
     # term 128, the stage combinations 106)
     "kin8": dict(passes=1, flop_step=966 + 702, flop_save=32, kernel="k_grad_kin8", n=262144, dtype="f64",
-                 desc="kin8 d=8 stiff mass-action network (stands in for HIRES at its size), t in [0,100], ROS3 "
+                 desc="kin8 d=8 stiff mass-action network (HIRES-sized ensemble), t in [0,100], ROS3 "
                       "rtol=atol=1e-7, loss sum ||u(T)||^2, 1 record + 1 gradient pass"),
     # the same with ROS2 (the configuration's second-order method): ~16,000
     # steps per trajectory at this tolerance, so a quarter of the ensemble

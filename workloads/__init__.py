@@ -19,12 +19,12 @@ well; the distributions are those of the benchmark configurations):
                 given by the sources this library follows)
   node64        n=131,072 du/dt = tanh(W u + b_i) - u, d=64, fp32, t in [0,1],
                 rtol=atol=1e-5, loss = sum ||u(T)||^2.
-  kin8          n=262,144 (the HIRES configuration's size, tolerances, loss
-                and parameter spread) an 8-species stiff mass-action network
-                defined by this library, d=8, np=8, ROS3, fp64,
-                t in [0, 100], rtol=atol=1e-7, loss = sum ||u(T)||^2: it
-                stands in for HIRES to exercise the Rosenbrock path at d=8
-                (8x8 LU).  Nominal rate constants
+  kin8          n=262,144, an 8-species stiff mass-action network defined
+                by this library, d=8, np=8, ROS3, fp64, t in [0, 100],
+                rtol=atol=1e-7, loss = sum ||u(T)||^2, rate constants spread
+                by lognormal(0, 0.05): the Rosenbrock path at d=8 (8x8 LU),
+                with HIRES's ensemble size, tolerances and loss (HIRES itself
+                is not built).  Nominal rate constants
                 k = (800, 400, 2, 0.2, 0.05, 0.025, 6, 0.004), each scaled by
                 lognormal(0, 0.05); u0 = (1, 0, 0.5, 0, 0, 0, 0.3, 0).
 
