@@ -7,14 +7,17 @@ import os
 import subprocess
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
         "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"}
 
 
-def test_reference_arm_json_line():
+@pytest.mark.parametrize("workload", ["lorenz_small", "kin8"])
+def test_reference_arm_json_line(workload):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
-                        "lorenz_small", "--steps", "1", "--warmup", "1"], capture_output=True, text=True, cwd=ROOT,
+                        workload, "--steps", "1", "--warmup", "1"], capture_output=True, text=True, cwd=ROOT,
                        timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.strip().splitlines() if l.startswith("{")]
