@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kKin8Block) k_grad_kin8(RosArgs<T> a) {
 #pragma unroll
     for (int c = 0; c < D; ++c) u[c] = un[c];
     if (st + 1 == next) {
-      loss_terms3<T, D>(a.loss_kind, a.target, a.weight, (int64_t)kk * nD + i, n, u, L);
+      loss_terms<T, D>(a.loss_kind, a.target, a.weight, (int64_t)kk * nD + i, n, u, L);
       ++kk;
       next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
     }
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kKin8Block) k_grad_kin8(RosArgs<T> a) {
   next = a.save_idx[(int64_t)kk * n + j];
   for (int st = S - 1; st >= 0; --st) {
     if (st + 1 == next) {
-      loss_grad3<T, D>(a.loss_kind, a.target, a.weight, (int64_t)kk * nD + i, n, unx, lam);
+      loss_grad<T, D>(a.loss_kind, a.target, a.weight, (int64_t)kk * nD + i, n, unx, lam);
       --kk;
       next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
     }

@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(128) k_grad_ros2(RosArgs<T> a) {
 #pragma unroll
     for (int c = 0; c < 3; ++c) u[c] = un[c];
     if (st + 1 == next) {
-      loss_terms3(a.loss_kind, a.target, a.weight, (int64_t)kk * n3 + i, n, u, L);
+      loss_terms(a.loss_kind, a.target, a.weight, (int64_t)kk * n3 + i, n, u, L);
       ++kk;
       next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
     }
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(128) k_grad_ros2(RosArgs<T> a) {
   T unx[3] = {u[0], u[1], u[2]};
   for (int st = S - 1; st >= 0; --st) {
     if (st + 1 == next) {
-      loss_grad3(a.loss_kind, a.target, a.weight, (int64_t)kk * n3 + i, n, unx, lam);
+      loss_grad(a.loss_kind, a.target, a.weight, (int64_t)kk * n3 + i, n, unx, lam);
       --kk;
       next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
     }

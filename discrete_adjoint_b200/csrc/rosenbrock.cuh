@@ -54,7 +54,7 @@ __device__ __forceinline__ void vjp3(const T u[3], const T p[3], const T w[3], T
 
 // Loss terms of one save point (D components at o + c n of target / weight).
 template <typename T, int D = 3>
-__device__ __forceinline__ void loss_terms3(int kind, const T* target, const T* weight, int64_t o, int64_t n,
+__device__ __forceinline__ void loss_terms(int kind, const T* target, const T* weight, int64_t o, int64_t n,
                                             const T* u, T& L) {
 #pragma unroll
   for (int c = 0; c < D; ++c) {
@@ -68,7 +68,7 @@ __device__ __forceinline__ void loss_terms3(int kind, const T* target, const T* 
 }
 
 template <typename T, int D = 3>
-__device__ __forceinline__ void loss_grad3(int kind, const T* target, const T* weight, int64_t o, int64_t n,
+__device__ __forceinline__ void loss_grad(int kind, const T* target, const T* weight, int64_t o, int64_t n,
                                            const T* u, T* lam) {
 #pragma unroll
   for (int c = 0; c < D; ++c) {
