@@ -247,9 +247,12 @@ GS_API gs_status gs_solve_adaptive(const gs_problem* prob, const gs_tol* tol, in
  *   dshared  device [64][64] dtype, GS_NODE64: sum_i dL_i/dW; else NULL
  *   ws       workspace of gs_workspace_bytes(prob, mesh, GS_OP_GRAD) bytes
  * All indexed by trajectory.  Slots with status != 0 get NaN loss/dp/du0 and
- * do not contribute to dshared.  (Evolve.pub review, "Summary": the replay is a
- * fixed-length chain without branches, and its backward sweep is the exact
- * discrete adjoint.)
+ * do not contribute to dshared.  Built for GS_LORENZ with GS_TSIT5 (dense
+ * save points included), GS_ROS2 or GS_ROS3; GS_ROBERTSON and GS_KIN8 with
+ * GS_ROS2 or GS_ROS3 (fp64 and fp32 for all of these); GS_NODE64 with GS_TSIT5
+ * in fp32.  Other combinations return GS_EUNSUPPORTED.  (Evolve.pub review,
+ * "Summary": the replay is a fixed-length chain without branches, and its
+ * backward sweep is the exact discrete adjoint.)
  */
 GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_loss* loss_desc, void* loss, void* dp,
                   void* du0, void* dshared, void* ws, size_t ws_bytes, void* stream);
