@@ -206,9 +206,13 @@ GS_API gs_status gs_count(const gs_problem* prob, const gs_tol* tol, int32_t sma
  * Record: adaptive solve of every trajectory (Tsit5, ROS2 or ROS3 per prob->method)
  * into the caller's mesh, slots ordered by decreasing step count.  Fills every
  * mesh array.  Trajectories that fail keep a status != 0 and a truncated mesh.
- * Runs a sizing pass, the slot ordering and the recording pass, all on stream.
- * (Evolve.pub review, "Summary": the adaptive solve happens once and keeps each
- * trajectory's accepted step sizes.)
+ * Runs the adaptive pass into the workspace (trajectory order), the slot
+ * ordering and a gather into slot order, all on stream.  Built for GS_LORENZ
+ * and GS_ROBERTSON with GS_TSIT5, GS_ROS2 or GS_ROS3, GS_KIN8 with GS_ROS2 or
+ * GS_ROS3 (fp64 and fp32), and GS_NODE64 with GS_TSIT5 in fp32; dense records
+ * for GS_TSIT5 on the d = 3 systems.  gs_count, gs_solve and gs_solve_adaptive
+ * take the same combinations.  (Evolve.pub review, "Summary": the adaptive
+ * solve happens once and keeps each trajectory's accepted step sizes.)
  */
 GS_API gs_status gs_record(const gs_problem* prob, const gs_tol* tol, const gs_mesh* mesh, void* ws, size_t ws_bytes,
                     void* stream);
