@@ -131,9 +131,9 @@ __device__ __forceinline__ void kin8_vjp(const T u[8], const T p[8], const T w[8
 // ubar += d<Jbar, J(u,p)>/du,  pbar += d<Jbar, J(u,p)>/dp for
 // Jbar = s sum_i w_i k_i^T.  With J = N dr/du, <Jbar, J> = sum_r G_r . grad_u r_r,
 // G_r = Jbar^T N[:, r] = s sum_i g_r(w_i) k_i; only the components of G_r that
-// meet a nonzero rate derivative are kept.  add() takes one stage pair as soon
-// as w_i is known (so k_i need not stay live); finish() applies the sums.  The
-// linear rates contribute only to pbar; the two bilinear ones (r3, r7) to both.
+// meet a nonzero rate derivative are kept.  add() takes one stage pair
+// (w_i, k_i); finish() applies the sums.  The linear rates contribute only to
+// pbar; the two bilinear ones (r3, r7) to both.
 template <typename T>
 struct Kin8JacAdj {
   T G0, G1, G2a, G2b, G3, G4, G5, G6a, G6b, G7;
@@ -267,7 +267,7 @@ __device__ __forceinline__ void lu_d_solve(const T LU[D * D], const int P[D], co
 // Solve M^T x = b with the factors of lu_d (M^T = U^T L^T P): U^T y = b
 // (forward), L^T z = y (backward, unit diagonal), x[P[i]] = z[i].  Reverse
 // sweep only (not part of the bitwise contract).  lu(e) / rc(i) read the
-// factors (registers or shared memory) at compile-time indices.
+// caller's factors at compile-time indices.
 template <typename T, int D, typename LUA, typename RA>
 __device__ __forceinline__ void lu_d_solve_T(LUA lu, RA rc, const int P[D], const T b[D], T x[D]) {
   T y[D];
