@@ -7,7 +7,7 @@ import torch
 import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
-from gpu_util import dev, ensemble, grad_rel_err, loss_args, mesh_by_trajectory, mesh_from_oracle, tens
+from gpu_util import dev, ensemble, grad_rel_err, loss_args, mesh_by_trajectory, mesh_from_oracle
 
 pytestmark = pytest.mark.gpu
 

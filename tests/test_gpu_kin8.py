@@ -11,7 +11,7 @@ import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
 from gpu_util import (TOL, dev, ensemble, grad_rel_err, loss_args, mesh_by_trajectory, mesh_from_oracle,
-                      mesh_rel_err, parity, tens)
+                      mesh_rel_err, parity)
 
 pytestmark = pytest.mark.gpu
 
