@@ -37,16 +37,21 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
     rebuild."""
     if not force and not extra_flags and not stale():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    cmds, objs = [], []
     for src in SOURCES:
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
-        cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-c", src, "-o", obj]
-        if verbose:
-            print(" ".join(cmd))
-        subprocess.run(cmd, check=True)
+        cmds.append([_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-c", src, "-o", obj])
         objs.append(obj)
+        if verbose:
+            print(" ".join(cmds[-1]))
+    # one nvcc per translation unit, in parallel; any failure raises
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for fut in [pool.submit(subprocess.run, c, check=True) for c in cmds]:
+            fut.result()
     tmp = LIB + ".tmp"
     subprocess.run([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
                     "-o", tmp, *objs], check=True)

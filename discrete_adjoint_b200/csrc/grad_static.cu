@@ -18,8 +18,6 @@
 // cleared between calls.
 //
 // The paper has no counterpart for this entry point.
-#include <mutex>
-
 #include "common.cuh"
 
 // Checkpoint scratch shared by all gs_grad_static calls on a device.
@@ -27,23 +25,16 @@ static __device__ __align__(256) unsigned char g_static_scratch[GS_STATIC_SCRATC
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_ptr[kMaxDevices] = {};
-
-// The device address of g_static_scratch on the current device.  In host code
-// the array's name is only a host-side stand-in, so its address must be looked
-// up, once per device, with that device current.
+// The device address of g_static_scratch in the current device's context.  In
+// host code the array's name is only a host-side stand-in, so the address is
+// looked up with the device current.  It is looked up on every call, not kept:
+// a context torn down and created again (cudaDeviceReset) loads the module
+// anew, possibly at another address, and a kept pointer would then be stale.
+// After the first call on a device the lookup costs no device work.
 gs_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GS_ECUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return GS_ECUDA;
-    g_ptr[dev] = p;
-  }
-  *out = g_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return GS_ECUDA;
+  *out = p;
   return GS_OK;
 }
 

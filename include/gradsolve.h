@@ -294,9 +294,10 @@ GS_API gs_status gs_sens(const gs_problem* prob, const gs_mesh* mesh, const gs_l
  *    of up to 1,365 steps).
  *  - All calls share the array: calls that overlap on the GPU race.  It keeps
  *    the last call's contents; nothing in it needs clearing between calls.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *    with the caller's device current, so a context reset between calls is
+ *    safe.  The first call on a device also loads the library's module there;
+ *    make that first call before any stream capture.
  * No counterpart in the paper.
  */
 #define GS_STATIC_SCRATCH_BYTES (32u << 20)

@@ -1,14 +1,43 @@
 """The C-ABI library loads and exports every entry point the header declares;
-host-side argument validation and workspace sizing (no device work)."""
+host-side argument validation and workspace sizing (no device work).
+
+The validation tests hand the library placeholder device pointers (address
+16) and oversized workspace sizes that only its argument checks stand
+between and a launch.  They run in a child process with the GPU hidden
+(CUDA_VISIBLE_DEVICES empty), so that a check that regressed would make a
+launch fail with a CUDA error instead of touching a real device; each also
+checks that the library's launch counter did not move."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
-import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "gradsolve.h")
+GPU_HIDDEN = os.environ.get("CUDA_VISIBLE_DEVICES") == ""
+hidden_only = pytest.mark.skipif(not GPU_HIDDEN, reason="runs in the GPU-hidden child process "
+                                                          "(test_host_checks_with_gpu_hidden)")
+
+
+@pytest.fixture
+def no_launch():
+    from discrete_adjoint_b200.gradsolve import _lib
+    before = _lib.gs_launch_count()
+    yield
+    assert _lib.gs_launch_count() == before, "a host-side check reached a kernel launch"
+
+
+@pytest.mark.skipif(GPU_HIDDEN, reason="this is the child process")
+def test_host_checks_with_gpu_hidden():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.abspath(__file__), "-q", "-m", "not gpu",
+                        "-p", "no:cacheprovider"], env=env, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+    passed = re.search(r"(\d+) passed", r.stdout.splitlines()[-1])
+    assert passed and int(passed.group(1)) >= 12, r.stdout[-2000:]
 
 
 def _declared():
@@ -45,7 +74,8 @@ def _host_problem(n=1000, system=1, method=1, dtype=2, nsave=10, tsave=None):
     return p
 
 
-def test_workspace_sizes_host_only():
+@hidden_only
+def test_workspace_sizes_host_only(no_launch):
     from discrete_adjoint_b200.gradsolve import _Mesh, _lib
     p = _host_problem()
     m = _Mesh(500, 10, None, None, None, None, None, None)
@@ -57,8 +87,9 @@ def test_workspace_sizes_host_only():
     assert _lib.gs_workspace_bytes(ctypes.byref(p32), ctypes.byref(m), 1) == 500 * 3 * 1000 * 4
 
 
+@hidden_only
 @pytest.mark.parametrize("bad", ["tsave_order", "tsave_range", "nsave0", "system", "dims", "dtype", "hires"])
-def test_invalid_problems_rejected_before_launch(bad):
+def test_invalid_problems_rejected_before_launch(bad, no_launch):
     from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol
     kw = {}
     if bad == "tsave_order":
@@ -86,7 +117,8 @@ def test_invalid_problems_rejected_before_launch(bad):
                           None) == (-4 if bad == "hires" else -1)
 
 
-def test_bad_tolerance_and_workspace_rejected():
+@hidden_only
+def test_bad_tolerance_and_workspace_rejected(no_launch):
     from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
     p = _host_problem()
     m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
@@ -123,7 +155,8 @@ def test_bad_tolerance_and_workspace_rejected():
     assert _lib.gs_solve(ctypes.byref(p), ctypes.byref(m2), ctypes.c_void_p(16), None) == -1
 
 
-def test_empty_ensemble_is_a_no_op():
+@hidden_only
+def test_empty_ensemble_is_a_no_op(no_launch):
     from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
     p = _host_problem(n=0)
     m = _Mesh(100, 10, None, None, None, None, None, None)
@@ -147,7 +180,8 @@ def test_set_option_host_only():
     assert _lib.gs_set_option(1, 2) == -1 and _lib.gs_set_option(99, 0) == -1
 
 
-def test_ros3_method_validation_host_only():
+@hidden_only
+def test_ros3_method_validation_host_only(no_launch):
     """ROS3 (method 3) is accepted for the d = 3 systems and refused where it is
     not built: dense save points (records and sensitivities); an unknown method
     is an invalid argument.  No call here reaches a launch."""
@@ -171,7 +205,8 @@ def test_ros3_method_validation_host_only():
                          None) == -1
 
 
-def test_kin8_validation_host_only():
+@hidden_only
+def test_kin8_validation_host_only(no_launch):
     """kin8 (system 5, d = np = 8) takes ROS2 / ROS3; Tsit5, forward
     sensitivities and dense records are not built for it; wrong sizes are
     invalid.  The gradient workspace is one checkpointed 8-state per step and
