@@ -283,6 +283,50 @@ def cpu_baseline(args, sample: int):
                       f"pass {tg:.2f} s, scaled to 1 record + {passes} passes"}
 
 
+def parity_sample(args, sample: int):
+    """Gradient parity of the GPU kernel on a sample of the workload, in the
+    step's launch configuration: the oracle records the sample, the library's
+    gs_grad runs on that mesh (slot j = trajectory j), and each trajectory's
+    error is ||g - g_ref||_inf / ||g_ref||_inf over (dp, du0) against the
+    oracle's tape with its reverse sweep accumulated in extended precision.
+    The oracle's own plain-precision tape error on the same sample is reported
+    beside it: on chaotic trajectories the reverse sweep's conditioning puts
+    both near the gate."""
+    import torch
+
+    import oracle
+    import discrete_adjoint_b200 as gs
+    W = WORKLOADS[args.workload]
+    prob = make_problem(args).subset(np.arange(sample))
+    threads = oracle.default_threads()
+    om = oracle.record(prob, smax_cap(args.workload), nthreads=threads, dense=W.get("dense", False))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    td = torch.float64 if args.dtype == "f64" else torch.float32
+    f = lambda a: torch.tensor(np.ascontiguousarray(a), dtype=td, device=dev)
+    i32 = lambda a: torch.tensor(np.ascontiguousarray(a, dtype=np.int32), device=dev)
+    ens = gs.Ensemble(prob.system, prob.method, args.dtype, f(prob.p), f(prob.u0), prob.t0, prob.t1,
+                      [float(x) for x in prob.tsave], None if prob.W is None else f(prob.W))
+    mesh = gs.Mesh(f(om.h.T), i32(np.arange(sample)), i32(om.nsteps), i32(om.save_idx.T), i32(om.status),
+                   i32(om.nreject), None if om.theta is None else f(om.theta.T))
+    out = gs.gs_grad(ens, mesh, loss=prob.loss, target=None if prob.target is None else f(prob.target),
+                     weight=None if prob.weight is None else f(prob.weight))
+    torch.cuda.synchronize()
+    g = np.vstack([out.dp.double().cpu().numpy(), out.du0.double().cpu().numpy()])
+    wide = oracle.grad(prob, om, "tape_wide", nthreads=threads)
+    tape = oracle.grad(prob, om, "tape", nthreads=threads)
+    r = np.vstack([wide["dp"], wide["du0"]])
+    ok = om.status == 0
+    rel = lambda a: (np.abs(a - r).max(0) / np.abs(r).max(0))[ok]
+    e, k = rel(g), rel(np.vstack([tape["dp"], tape["du0"]]))
+    gate = 1e-12 if args.dtype == "f64" else 1e-4
+    q = lambda a, x: float(np.quantile(a, x)) if len(a) else None
+    return {"sample": f"first {sample} trajectories, oracle mesh", "reference": "oracle tape, extended-precision "
+            "reverse sweep", "metric": "per-trajectory ||g - g_ref||_inf / ||g_ref||_inf over (dp, du0)",
+            "p50": q(e, 0.5), "p99": q(e, 0.99), "max": q(e, 1.0), "gate": gate,
+            "frac_within_gate": float(np.mean(e <= gate)) if len(e) else None,
+            "oracle_tape": {"p50": q(k, 0.5), "p99": q(k, 0.99), "max": q(k, 1.0)}}
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle on the host cores, same metric/config;
     each step is the record + gradient passes of a bounded sample."""
@@ -560,8 +604,12 @@ def run_ours(args):
 
     # sizing pass (setup, untimed): mesh capacity = the longest chain
     dense = W.get("dense", False)
-    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload), dense=dense)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload), dense=dense, stream=stream)
+    c1.record(stream)
     smax = int(nsteps.max().item())
+    count_ms = c0.elapsed_time(c1)
     mesh = gs.new_mesh(n, smax, len(prob.tsave), args.dtype, dev, dense=dense)
     ws_rec = gs.workspace(gs.gs_workspace_bytes(ens, mesh, gs.gradsolve.OP_RECORD), dev)
     ws_grad = gs.workspace(gs.gs_workspace_bytes(ens, mesh, gs.gradsolve.OP_GRAD), dev)
@@ -678,6 +726,9 @@ def run_ours(args):
                    "steps_max_over_mean": float(ns.max() / ns.mean()),
                    "rejects_total": int(mesh.nreject.sum().item()),
                    "grad_ms": grad_ms, "record_ms": rec_ms, "grad_only_value": world * n / (grad_ms / 1e3),
+                   "count_ms": count_ms,
+                   "count_note": "sizing pass (gs_count) run once as untimed setup; the timed records reuse the "
+                                 "capacity it found",
                    "l2": "inputs larger than L2 (mesh %.2f GB, gradient workspace %.2f GB); no flush" % (
                        mesh.h.numel() * esz / 1e9, ws_grad.numel() / 1e9),
                    "parallelism": f"dp{world} (independent trajectory shards)",
@@ -700,6 +751,9 @@ def run_ours(args):
         sample = {"lorenz_1m": 32768, "lorenz_1m_dense": 32768, "lorenz_small": 1024, "robertson": 256,
                   "robertson_ros3": 2048, "node64": 1024, "kin8": 2048, "kin8_ros2": 64}[args.workload]
         line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
+        psample = {"lorenz_1m": 8192, "lorenz_1m_dense": 8192, "lorenz_small": 1024, "robertson": 256,
+                   "robertson_ros3": 2048, "node64": 256, "kin8": 1024, "kin8_ros2": 32}[args.workload]
+        line["parity"] = parity_sample(args, min(psample, n))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

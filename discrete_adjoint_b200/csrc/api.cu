@@ -44,6 +44,7 @@ gs_status node64_grad(const gs_problem*, const gs_mesh*, const gs_loss*, void*, 
 gs_status node64_solve(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 void node64_set_tensor(int on);
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize);
+int grad_tsit5_lorenz_ck_rows(int32_t dtype);
 
 static size_t dsize(const gs_problem* P) { return P->dtype == GS_F64 ? 8 : 4; }
 
@@ -92,12 +93,12 @@ static gs_status check_mesh(const gs_problem* P, const gs_mesh* M) {
   return GS_OK;
 }
 
-// Tolerances; a dense record is built for Tsit5 on the d = 3 systems.
+// Tolerances; a dense record is built for the d = 3 systems (every method).
 static gs_status check_tol(const gs_problem* P, const gs_tol* tol) {
   if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0))
     return GS_EINVAL;
   if (tol->dense != 0 && tol->dense != 1) return GS_EINVAL;
-  if (tol->dense && (P->method != GS_TSIT5 || P->system == GS_NODE64)) return GS_EUNSUPPORTED;
+  if (tol->dense && (P->system == GS_NODE64 || P->system == GS_KIN8)) return GS_EUNSUPPORTED;
   return GS_OK;
 }
 
@@ -133,7 +134,11 @@ size_t gs_workspace_bytes(const gs_problem* P, const gs_mesh* M, int32_t op) {
   if (op == GS_OP_RECORD) return record_ws_bytes(P->n, M->smax, P->nsave, dsize(P));
   if (op == GS_OP_GRAD) {
     if (P->system == GS_NODE64) return node64_grad_ws_bytes(P->n, M->smax, dsize(P));
-    return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
+    // one checkpointed state per step and slot (the Tsit5 Lorenz kernel may
+    // keep a stage state beside it)
+    const size_t rows = (P->method == GS_TSIT5 && P->system == GS_LORENZ) ? (size_t)grad_tsit5_lorenz_ck_rows(P->dtype)
+                                                                           : (size_t)P->d;
+    return (size_t)M->smax * rows * (size_t)P->n * dsize(P);
   }
   return 0;
 }
@@ -183,7 +188,7 @@ gs_status gs_solve(const gs_problem* P, const gs_mesh* M, void* u_save, void* st
   gs_status rc = check_problem(P);
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
-  if (M->save_theta && (P->method != GS_TSIT5 || P->system == GS_NODE64)) return GS_EUNSUPPORTED;
+  if (M->save_theta && (P->system == GS_NODE64 || P->system == GS_KIN8)) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (!u_save) return GS_EINVAL;
   if (P->system == GS_NODE64) return node64_solve(P, M, u_save, (cudaStream_t)stream);
@@ -197,8 +202,8 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
-  // dense save points: the Tsit5 Lorenz gradient
-  if (M->save_theta && (P->method != GS_TSIT5 || P->system != GS_LORENZ)) return GS_EUNSUPPORTED;
+  // dense save points: the d = 3 gradients (Tsit5 on Lorenz, ROS2 / ROS3 on Lorenz and Robertson)
+  if (M->save_theta && (P->system == GS_NODE64 || P->system == GS_KIN8)) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;
   if (!loss || !dp || !du0) return GS_EINVAL;

@@ -63,8 +63,64 @@ __device__ __forceinline__ void jac_adjoint3_ros3(const T u[3], const T p[3], T 
   }
 }
 
+// Copy rings: the forward streams h, the reverse (u_s, h_s), kRos3Ring steps
+// ahead (DRAM latency is most of a step at the few warps per SM that these
+// ensembles fill).
+constexpr int kRos3Ring = 8;
+
+// One recomputed forward step, as its transposed step needs it.
+template <typename T>
+struct Ros3Step {
+  T us[3], h, LU[9], R[3], k1[3], v[3], k2[3], k3[3];
+  int P[3];
+};
+
+template <typename T, int SYS>
+__device__ __forceinline__ void ros3_recompute(Ros3Step<T>& q, const T p[3]) {
+  T un[3];
+  ros3_fwd<T, SYS>(q.us, p, q.h, q.LU, q.P, q.R, q.k1, q.v, q.k2, q.k3, un);
+}
+
+// The transposed step of q: lam <- dL/du_s from lam = dL/du_{s+1}; pb += dL/dp.
+template <typename T, int SYS>
+__device__ __forceinline__ void ros3_transpose(const Ros3Step<T>& q, const T p[3], T lam[3], T pb[3]) {
+  const T h = q.h;
+  T ub[3] = {lam[0], lam[1], lam[2]};
+  T kb1[3], kb2[3], r1[3], r2[3], r3[3], fb[3];
+  const T hm2 = cst<T>(ROS3_M2) * h, hm3 = cst<T>(ROS3_M3) * h;
+  lu3_solve_T(q.LU, q.P, q.R, hm3 * lam[0], hm3 * lam[1], hm3 * lam[2], r3[0], r3[1], r3[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    kb1[c] = fmaT(cst<T>(ROS3_C31), r3[c], h * lam[c]);
+    kb2[c] = fmaT(cst<T>(ROS3_C32), r3[c], hm2 * lam[c]);
+  }
+  lu3_solve_T(q.LU, q.P, q.R, kb2[0], kb2[1], kb2[2], r2[0], r2[1], r2[2]);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    fb[c] = r3[c] + r2[c];
+    kb1[c] = fmaT(cst<T>(ROS3_C21), r2[c], kb1[c]);
+  }
+  T vb[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)};
+  vjp3<T, SYS>(q.v, p, fb, vb, pb);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    ub[c] += vb[c];
+    kb1[c] = fmaT(h, vb[c], kb1[c]);
+  }
+  lu3_solve_T(q.LU, q.P, q.R, kb1[0], kb1[1], kb1[2], r1[0], r1[1], r1[2]);
+  vjp3<T, SYS>(q.us, p, r1, ub, pb);
+  jac_adjoint3_ros3<T, SYS>(q.us, p, h, r1, r2, r3, q.k1, q.k2, q.k3, ub, pb);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) lam[c] = ub[c];
+}
+
+// Reverse loop, software-pipelined: iteration st recomputes step st - 1 from
+// its checkpoint while it runs the transposed step of st (recomputed by the
+// iteration before).  The recompute does not depend on lambda, so the two are
+// independent chains in one instruction stream.
 template <typename T, int SYS>
 __global__ void __launch_bounds__(128) k_grad_ros3(RosArgs<T> a) {
+  extern __shared__ __align__(16) unsigned char ring_raw[];
   const int64_t n = a.n;
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n) return;
@@ -95,8 +151,16 @@ __global__ void __launch_bounds__(128) k_grad_ros3(RosArgs<T> a) {
   int next = a.save_idx[j];
   bool ok = true;
   // ---------------------------------------------------------------- forward
+  const ThreadRing<T, 1, kRos3Ring> rf(ring_raw);
+  auto issue_f = [&](int sf) {
+    if (sf < S) cp_async_el(rf.at(sf, 0), hp + (int64_t)sf * n);
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int sf = 0; sf < kRos3Ring; ++sf) issue_f(sf);
   for (int st = 0; st < S; ++st) {
-    const T h = hp[(int64_t)st * n];
+    cp_async_wait<kRos3Ring - 1>();  // the group of step st
+    const T h = *rf.at(st, 0);
     cp[0] = u[0];
     cp[n] = u[1];
     cp[2 * n] = u[2];
@@ -104,63 +168,60 @@ __global__ void __launch_bounds__(128) k_grad_ros3(RosArgs<T> a) {
     T LU[9], R[3], k1[3], v[3], k2[3], k3[3], un[3];
     int P[3];
     ok = ros3_fwd<T, SYS>(u, p, h, LU, P, R, k1, v, k2, k3, un) && ok;
+    save_points_fwd<T, SYS>(a, i, j, st, p, u, un, h, kk, next, L);
 #pragma unroll
     for (int c = 0; c < 3; ++c) u[c] = un[c];
-    if (st + 1 == next) {
-      loss_terms(a.loss_kind, a.target, a.weight, (int64_t)kk * n3 + i, n, u, L);
-      ++kk;
-      next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
-    }
+    issue_f(st + kRos3Ring);  // into the slot step st has left
   }
+  cp_async_wait<0>();  // the reverse reuses the ring
   // ---------------------------------------------------------------- reverse
+  const ThreadRing<T, 4, kRos3Ring> rr(ring_raw);
+  auto issue_r = [&](int sr) {
+    if (sr >= 0 && sr < S) {
+      const T* c = a.ck + (int64_t)sr * n3 + j;
+      cp_async_el(rr.at(sr, 0), c);
+      cp_async_el(rr.at(sr, 1), c + n);
+      cp_async_el(rr.at(sr, 2), c + 2 * n);
+      cp_async_el(rr.at(sr, 3), hp + (int64_t)sr * n);
+    }
+    cp_async_commit();
+  };
+  auto take_r = [&](int sr, Ros3Step<T>& q) {
+    q.us[0] = *rr.at(sr, 0);
+    q.us[1] = *rr.at(sr, 1);
+    q.us[2] = *rr.at(sr, 2);
+    q.h = *rr.at(sr, 3);
+  };
   T lam[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)};
   T pb[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)};
   kk = a.nsave - 1;
-  next = a.save_idx[(int64_t)kk * n + j];
+  next = S > 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
   T unx[3] = {u[0], u[1], u[2]};  // u_{st+1}
-  for (int st = S - 1; st >= 0; --st) {
-    if (st + 1 == next) {
-      loss_grad(a.loss_kind, a.target, a.weight, (int64_t)kk * n3 + i, n, unx, lam);
-      --kk;
-      next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
-    }
-    cp -= n3;
-    const T us[3] = {cp[0], cp[n], cp[2 * n]};
-    const T h = hp[(int64_t)st * n];
-    T LU[9], R[3], k1[3], v[3], k2[3], k3[3], un[3];
-    int P[3];
-    ros3_fwd<T, SYS>(us, p, h, LU, P, R, k1, v, k2, k3, un);
-    T ub[3] = {lam[0], lam[1], lam[2]};
-    T kb1[3], kb2[3], r1[3], r2[3], r3[3], fb[3];
-    const T hm2 = cst<T>(ROS3_M2) * h, hm3 = cst<T>(ROS3_M3) * h;
-    lu3_solve_T(LU, P, R, hm3 * lam[0], hm3 * lam[1], hm3 * lam[2], r3[0], r3[1], r3[2]);
 #pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      kb1[c] = fmaT(cst<T>(ROS3_C31), r3[c], h * lam[c]);
-      kb2[c] = fmaT(cst<T>(ROS3_C32), r3[c], hm2 * lam[c]);
-    }
-    lu3_solve_T(LU, P, R, kb2[0], kb2[1], kb2[2], r2[0], r2[1], r2[2]);
-#pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      fb[c] = r3[c] + r2[c];
-      kb1[c] = fmaT(cst<T>(ROS3_C21), r2[c], kb1[c]);
-    }
-    T vb[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)};
-    vjp3<T, SYS>(v, p, fb, vb, pb);
-#pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      ub[c] += vb[c];
-      kb1[c] = fmaT(h, vb[c], kb1[c]);
-    }
-    lu3_solve_T(LU, P, R, kb1[0], kb1[1], kb1[2], r1[0], r1[1], r1[2]);
-    vjp3<T, SYS>(us, p, r1, ub, pb);
-    jac_adjoint3_ros3<T, SYS>(us, p, h, r1, r2, r3, k1, k2, k3, ub, pb);
-#pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      lam[c] = ub[c];
-      unx[c] = us[c];
-    }
+  for (int i2 = 0; i2 < kRos3Ring; ++i2) issue_r(S - 1 - i2);
+  Ros3Step<T> cur;
+  if (S > 0) {
+    cp_async_wait<kRos3Ring - 1>();
+    take_r(S - 1, cur);
+    ros3_recompute<T, SYS>(cur, p);
   }
+  for (int st = S - 1; st >= 0; --st) {
+    T pg[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)}, pn[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)};
+    const bool interior = save_points_rev<T, SYS>(a, i, j, st, p, cur.us, unx, cur.h, kk, next, lam, pb, pg, pn);
+    // step st - 1 (step 0 again on the last iteration, whose result is unused:
+    // its ring slot still holds step 0, since no later copy targets it)
+    cp_async_wait<kRos3Ring - 2>();
+    Ros3Step<T> nxt;
+    take_r(st > 0 ? st - 1 : 0, nxt);
+    ros3_recompute<T, SYS>(nxt, p);
+    ros3_transpose<T, SYS>(cur, p, lam, pb);
+    if (interior) save_points_rev_finish<T, SYS>(p, cur.us, pg, pn, lam, pb);
+#pragma unroll
+    for (int c = 0; c < 3; ++c) unx[c] = cur.us[c];
+    cur = nxt;
+    issue_r(st - kRos3Ring);  // into the slot step st has left
+  }
+  cp_async_wait<0>();
   if (!ok) {
     L = nan;
 #pragma unroll
@@ -180,10 +241,11 @@ gs_status launch_grad_ros3(const gs_problem* P, const gs_mesh* M, const gs_loss*
   const RosArgs<T> a = ros_args<T>(P, M, Ls, loss, dp, du0, ws);
   const int bs = 128;
   const unsigned grid = (unsigned)((P->n + bs - 1) / bs);
-  if (P->system == GS_ROBERTSON)
-    k_grad_ros3<T, GS_ROBERTSON><<<grid, bs, 0, st>>>(a);
-  else
-    k_grad_ros3<T, GS_LORENZ><<<grid, bs, 0, st>>>(a);
+  const size_t smem = (size_t)ThreadRing<T, 4, kRos3Ring>::kElems * bs * sizeof(T);
+  auto kern = P->system == GS_ROBERTSON ? k_grad_ros3<T, GS_ROBERTSON> : k_grad_ros3<T, GS_LORENZ>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return GS_ECUDA;
+  kern<<<grid, bs, smem, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

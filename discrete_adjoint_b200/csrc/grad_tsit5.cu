@@ -22,21 +22,28 @@
 // lambda at the save points.  Output: dL/dp = pbar, dL/du0 = lambda.
 //
 // Execution: the kernel is bound by the FP64 pipe, and one Lorenz trajectory
-// offers only three independent chains (x, y, z) per instruction stream, which
-// leaves the pipe idle a quarter of the time at the occupancy its registers
-// allow.  Each thread therefore carries K adjacent slots (vec<T, K>), giving 3K
-// independent chains.  gs_record orders slots by decreasing step count, so the
-// K chains of a thread (and the 32K of a warp) have nearly equal length; the
-// shorter ones run the remaining iterations as steps of size 0, which are
-// exact identities in both halves (u + 0 * acc = u; nu = 0 * (...) = 0), so the
-// results are bitwise those of one slot per thread.
+// offers only three independent chains (x, y, z) per instruction stream.  Each
+// thread may carry K adjacent slots (vec<T, K>), giving 3K independent chains.
+// gs_record orders slots by decreasing step count, so the K chains of a thread
+// (and the 32K of a warp) have nearly equal length; the shorter ones run the
+// remaining iterations as steps of size 0, which are exact identities in both
+// halves (u + 0 * acc = u; nu = 0 * (...) = 0), so the results are bitwise
+// those of one slot per thread.
 //
-// Memory layout: h [smax][n] and ck [smax][3][n] are step-major over slots, so
-// at a given step a warp touches 32K consecutive elements of every array.
-// With one slot per thread, h and the checkpoints stream into per-thread
-// shared-memory rings (cp.async, kRingF / kRingR steps ahead) and are read
-// from there one step ahead; with K > 1 they are loaded one step ahead into
-// registers and prefetched several steps ahead into L2.
+// Store or recompute: the reverse step needs the stage states U_2..U_6 of its
+// step.  It recomputes U_2..U_5 from the checkpointed u_s; with KEEP6 the
+// forward also keeps U_6 (the costliest to rebuild: a five-term combination
+// and the right-hand side at U_5, ~22 FP64 instructions per step) beside u_s,
+// for 48 more bytes per step (fp64) of HBM traffic.  The kept U_6 is the value
+// the forward computed, so a recompute would give the same bits.
+//
+// Memory layout: h [smax][n] and the checkpoints ck [smax][R][n] (R = 3 rows
+// u_s, or 6 with U_6) are step-major over slots, so at a given step a warp
+// touches 32K consecutive elements of every array.  They stream into
+// per-thread shared-memory rings with cp.async, kRingF (forward: h) and kRingR
+// (reverse: checkpoint rows and h) steps ahead, and are read from there one
+// step ahead, so no register waits on DRAM and no barrier is involved: each
+// thread waits only on its own copies.
 #include "steps.cuh"
 #include "vec.cuh"
 
@@ -51,18 +58,13 @@ namespace gs {
 #ifndef GS_GRAD_MINB
 #define GS_GRAD_MINB (GS_GRAD_K == 1 ? 4 : 2)
 #endif
-#ifndef GS_PF_F
-#define GS_PF_F 8
+// keep U_6 in the checkpoint workspace (1) or recompute it (0), per dtype
+#ifndef GS_GRAD_KEEP6_F64
+#define GS_GRAD_KEEP6_F64 0
 #endif
-#ifndef GS_PF_R
-#define GS_PF_R 4
+#ifndef GS_GRAD_KEEP6_F32
+#define GS_GRAD_KEEP6_F32 0
 #endif
-#ifndef GS_GRAD_ASYNC
-#define GS_GRAD_ASYNC 1
-#endif
-// Copy rings (one trajectory per thread): the forward streams h kRingF steps
-// ahead, the reverse streams (u_s, h_s) kRingR steps ahead, each thread into
-// its own shared-memory slots with cp.async, so that no register waits on DRAM.
 #ifndef GS_RING_F
 #define GS_RING_F 8
 #endif
@@ -73,10 +75,21 @@ constexpr int kRingF = GS_RING_F;
 constexpr int kRingR = GS_RING_R;
 static_assert((kRingF & (kRingF - 1)) == 0 && kRingF >= 2 && (kRingR & (kRingR - 1)) == 0 && kRingR >= 2,
               "ring depths: powers of two, at least 2");
-// L2 prefetch distances in steps (a warp's forward step takes ~0.5 us and its
-// reverse step ~1 us, against a DRAM latency of ~1 us under load).
-constexpr int kPrefetchF = GS_PF_F;
-constexpr int kPrefetchR = GS_PF_R;
+
+template <typename T>
+__host__ __device__ constexpr bool keep6() {
+  return sizeof(T) == 8 ? GS_GRAD_KEEP6_F64 != 0 : GS_GRAD_KEEP6_F32 != 0;
+}
+// checkpoint rows per step and slot
+template <typename T>
+__host__ __device__ constexpr int ck_rows() {
+  return keep6<T>() ? 6 : 3;
+}
+// shared-memory ring elements per thread: the larger of the two rings
+template <typename T, int K>
+__host__ __device__ constexpr int ring_elems() {
+  return (kRingF * K > kRingR * (ck_rows<T>() + 1) * K) ? kRingF * K : kRingR * (ck_rows<T>() + 1) * K;
+}
 
 template <typename T>
 struct TsitLorenzArgs {
@@ -96,7 +109,7 @@ struct TsitLorenzArgs {
   T* loss;          // [n] by trajectory
   T* dp;            // [3][n]
   T* du0;           // [3][n]
-  T* ck;            // workspace [smax][3][n] by slot
+  T* ck;            // workspace [smax][ck_rows][n] by slot
   const T* theta;   // [nsave][n] by slot: dense save points, or null
 };
 
@@ -133,8 +146,12 @@ __device__ __forceinline__ void lorenz_vjp(const V& ux, const V& uy, const V& uz
 template <typename T, int K, bool DENSE>
 __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(TsitLorenzArgs<T> a) {
   using V = vec<T, K>;
+  constexpr bool kKeep6 = keep6<T>();
+  constexpr int kCk = ck_rows<T>();   // checkpoint rows per step
+  constexpr int kRowsR = kCk + 1;     // reverse ring rows per step: checkpoint + h
+  constexpr int BS = GS_GRAD_BS;
   const int64_t n = a.n;
-  const int64_t n3 = 3 * n;
+  const int64_t nck = kCk * n;        // checkpoint elements per step
   const int64_t j0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * K;
   if (j0 >= n) return;
   const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
@@ -177,11 +194,25 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   }
   const T* __restrict__ hp = a.h + j0;
   T* __restrict__ cp = a.ck + j0;
-  constexpr bool kAsync = GS_GRAD_ASYNC != 0 && K == 1;
-  __shared__ T ring[kAsync ? 4 * kRingR * GS_GRAD_BS : 1];
-  T* const rg = ring + threadIdx.x;  // this thread's element of slot row w: rg[w * GS_GRAD_BS]
+  // Per-thread copy rings.  Element (row w, slot q) of a thread lives at
+  // rg[(w * K + q) * BS]: consecutive threads touch consecutive words.
+  // Forward: row w = s % kRingF holds h of step s.  Reverse: rows
+  // kRowsR (s % kRingR) + c hold checkpoint row c (c < kCk) and h (c = kCk) of
+  // step s.  One commit group per step; a thread waits on its own groups only.
+  extern __shared__ __align__(16) unsigned char ring_raw[];  // ring_elems<T, K>() * BS elements
+  T* const rg = reinterpret_cast<T*>(ring_raw) + threadIdx.x;
 
   // ---------------------------------------------------------------- forward
+  auto issue_f = [&](int sf) {  // h of step sf into its ring row
+#pragma unroll
+    for (int q = 0; q < K; ++q)
+      if (sf < S[q]) cp_async_el(rg + ((sf & (kRingF - 1)) * K + q) * BS, hp + (int64_t)sf * n + q);
+    cp_async_commit();
+  };
+  auto take_f = [&](int sf, V& hv) {  // its group complete; 0 past a slot's last step
+#pragma unroll
+    for (int q = 0; q < K; ++q) hv.e[q] = sf < S[q] ? rg[((sf & (kRingF - 1)) * K + q) * BS] : cst<T>(0.0);
+  };
   V L = vsplat<T, K>(cst<T>(0.0));
   int kk[K], next[K];
 #pragma unroll
@@ -192,40 +223,22 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   V k1x, k1y, k1z;
   lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);
   V hn;
-  if constexpr (kAsync) {  // h of step s in slot s % kRingF
 #pragma unroll
-    for (int s = 0; s < kRingF; ++s) {
-      if (s < S[0]) cp_async_el(rg + s * GS_GRAD_BS, hp + (int64_t)s * n);
-      cp_async_commit();
-    }
-    cp_async_wait<kRingF - 1>();
-    hn.e[0] = 0 < S[0] ? rg[0] : cst<T>(0.0);
-  } else {
-#pragma unroll
-    for (int q = 0; q < K; ++q) hn.e[q] = 0 < S[q] ? hp[q] : cst<T>(0.0);
-  }
-  const T* hq = hp + n;                        // h of step st + 1
-  const T* hf = hp + (int64_t)kPrefetchF * n;  // h of step st + kPrefetchF
+  for (int sf = 0; sf < kRingF; ++sf) issue_f(sf);
+  cp_async_wait<kRingF - 1>();
+  take_f(0, hn);
   for (int st = 0; st < Smax; ++st) {
     const V h = hn;
-    if constexpr (kAsync) {
-      cp_async_wait<kRingF - 2>();  // the group of step st + 1
-      hn.e[0] = st + 1 < S[0] ? rg[((st + 1) & (kRingF - 1)) * GS_GRAD_BS] : cst<T>(0.0);
-    } else {
-      if (st + kPrefetchF < Smax) prefetch_l2(hf);
-      hf += n;
-    }
+    cp_async_wait<kRingF - 2>();  // the group of step st + 1
+    take_f(st + 1, hn);
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      if constexpr (!kAsync) hn.e[q] = st + 1 < S[q] ? hq[q] : cst<T>(0.0);
       if (st < S[q]) {
         cp[q] = x.e[q];
         cp[n + q] = y.e[q];
         cp[2 * n + q] = z.e[q];
       }
     }
-    hq += n;
-    cp += n3;
     V ax, ay, az, Ux, Uy, Uz;
     GS_ACC1(kTsA21, k1)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
@@ -255,6 +268,17 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     GS_ACCN(kTsA64, k4)
     GS_ACCN(kTsA65, k5)
     GS_STAGE(Ux, Uy, Uz, ax, ay, az)
+    if constexpr (kKeep6) {  // U_6 beside u_s
+#pragma unroll
+      for (int q = 0; q < K; ++q) {
+        if (st < S[q]) {
+          cp[3 * n + q] = Ux.e[q];
+          cp[4 * n + q] = Uy.e[q];
+          cp[5 * n + q] = Uz.e[q];
+        }
+      }
+    }
+    cp += nck;
     V k6x, k6y, k6z;
     lorenz_f(Ux, Uy, Uz, s, r, b, k6x, k6y, k6z);
     // stage 7 = u_{s+1}
@@ -281,7 +305,7 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     for (int q = 0; q < K; ++q) {
       // a landing record has at most one save point per step; a dense one any number
       while (st + 1 == next[q]) {
-        const int64_t o = (int64_t)kk[q] * n3 + i[q];
+        const int64_t o = (int64_t)kk[q] * 3 * n + i[q];
         T ux = x.e[q], uy = y.e[q], uz = z.e[q];
         if (DENSE) {
           const T th = a.theta[(int64_t)kk[q] * n + j0 + q];
@@ -311,13 +335,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
         if (!DENSE) break;
       }
     }
-    if constexpr (kAsync) {  // step st + kRingF into the slot that step st has left
-      const int sn = st + kRingF;
-      if (sn < S[0]) cp_async_el(rg + (sn & (kRingF - 1)) * GS_GRAD_BS, hp + (int64_t)sn * n);
-      cp_async_commit();
-    }
+    issue_f(st + kRingF);  // into the row that step st has left
   }
-  if constexpr (kAsync) cp_async_wait<0>();  // the reverse reuses the slots
+  cp_async_wait<0>();  // the reverse reuses the rows
 #pragma unroll
   for (int q = 0; q < K; ++q)
     if (i[q] >= 0) a.loss[i[q]] = L.e[q];
@@ -325,7 +345,8 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   // ---------------------------------------------------------------- reverse
   // At the top of iteration st, (x, y, z) holds u_{st+1} (the final state
   // first, then the state loaded by the previous iteration), which is what the
-  // save-point test needs; (cx, cy, cz, hc) are the prefetched u_st and h_st.
+  // save-point test needs; (cx, cy, cz, hc) and, with KEEP6, (gx6, gy6, gz6)
+  // are the prefetched u_st, h_st and U_6 of step st.
   V lx = vsplat<T, K>(cst<T>(0.0)), ly = lx, lz = lx;
   V ps = lx, pr = lx, pb = lx;
 #pragma unroll
@@ -334,52 +355,46 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     next[q] = S[q] > 0 ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
   }
   V cx = x, cy = y, cz = z, hc = vsplat<T, K>(cst<T>(0.0));
-  const T* hq2 = hp + (int64_t)(Smax - 1) * n;  // h of the step being loaded
-  // reverse ring: (u_s, h_s) of step s in slot s % kRingR, components in rows
-  // 4 (s % kRingR) + c; the copies of one step form one group
-  auto issue_r = [&](int sr) {
-    if (sr >= 0 && sr < S[0]) {
-      T* d = rg + (sr & (kRingR - 1)) * 4 * GS_GRAD_BS;
-      const T* c = a.ck + (int64_t)sr * n3 + j0;
-      cp_async_el(d, c);
-      cp_async_el(d + GS_GRAD_BS, c + n);
-      cp_async_el(d + 2 * GS_GRAD_BS, c + 2 * n);
-      cp_async_el(d + 3 * GS_GRAD_BS, hp + (int64_t)sr * n);
+  V gx6 = x, gy6 = y, gz6 = z;
+  auto issue_r = [&](int sr) {  // step sr's checkpoint rows and h
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      if (sr >= 0 && sr < S[q]) {
+        T* d = rg + ((sr & (kRingR - 1)) * kRowsR * K + q) * BS;
+        const T* c = a.ck + (int64_t)sr * nck + j0 + q;
+#pragma unroll
+        for (int w = 0; w < kCk; ++w) cp_async_el(d + w * K * BS, c + w * n);
+        cp_async_el(d + kCk * K * BS, hp + (int64_t)sr * n + q);
+      }
     }
     cp_async_commit();
   };
-  auto take_r = [&](int sr) {  // step sr's values, its group complete
-    const T* d = rg + (sr & (kRingR - 1)) * 4 * GS_GRAD_BS;
-    cx.e[0] = d[0];
-    cy.e[0] = d[GS_GRAD_BS];
-    cz.e[0] = d[2 * GS_GRAD_BS];
-    hc.e[0] = d[3 * GS_GRAD_BS];
-  };
-  if constexpr (kAsync) {
-#pragma unroll
-    for (int i2 = 0; i2 < kRingR; ++i2) issue_r(Smax - 1 - i2);
-    cp_async_wait<kRingR - 1>();
-    if (Smax > 0 && Smax - 1 < S[0]) take_r(Smax - 1);
-  } else if (Smax > 0) {
-    cp -= n3;
+  // step sr's values, its group complete; a slot past its last step runs an
+  // identity step (h = 0) at its final state
+  auto take_r = [&](int sr) {
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      if (Smax - 1 < S[q]) {
-        cx.e[q] = cp[q];
-        cy.e[q] = cp[n + q];
-        cz.e[q] = cp[2 * n + q];
-        hc.e[q] = hq2[q];
+      const T* d = rg + ((sr & (kRingR - 1)) * kRowsR * K + q) * BS;
+      if (sr < S[q]) {
+        cx.e[q] = d[0];
+        cy.e[q] = d[K * BS];
+        cz.e[q] = d[2 * K * BS];
+        if constexpr (kKeep6) {
+          gx6.e[q] = d[3 * K * BS];
+          gy6.e[q] = d[4 * K * BS];
+          gz6.e[q] = d[5 * K * BS];
+        }
+        hc.e[q] = d[kCk * K * BS];
+      } else {
+        hc.e[q] = cst<T>(0.0);
       }
     }
-  }
+  };
+#pragma unroll
+  for (int i2 = 0; i2 < kRingR; ++i2) issue_r(Smax - 1 - i2);
+  cp_async_wait<kRingR - 1>();
+  if (Smax > 0) take_r(Smax - 1);
   for (int st = Smax - 1; st >= 0; --st) {
-    if (!kAsync && st >= kPrefetchR) {
-      const T* c = cp - (int64_t)kPrefetchR * n3;
-      prefetch_l2(c);
-      prefetch_l2(c + n);
-      prefetch_l2(c + 2 * n);
-      prefetch_l2(hq2 - (int64_t)kPrefetchR * n);
-    }
     // dense save points inside step st: the interpolant's cotangent g reaches
     // u_{st+1} now (H01 g + J(u_{st+1})^T (h H11 g)) and u_st after the
     // transposed step (H00 g + J(u_st)^T (h H10 g)), with the matching
@@ -392,7 +407,7 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #pragma unroll
     for (int q = 0; q < K; ++q) {
       while (st + 1 == next[q]) {
-        const int64_t o = (int64_t)kk[q] * n3 + i[q];
+        const int64_t o = (int64_t)kk[q] * 3 * n + i[q];
         T th = cst<T>(1.0);
         HermiteW<T> w;
         T ux = x.e[q], uy = y.e[q], uz = z.e[q], fsx, fsy, fsz, fnx, fny, fnz;
@@ -446,32 +461,21 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     y = cy;
     z = cz;
     const V h = hc;
-    if (kAsync && st > 0) {
+    V U6x, U6y, U6z;
+    if constexpr (kKeep6) {
+      U6x = gx6;
+      U6y = gy6;
+      U6z = gz6;
+    }
+    if (st > 0) {
       cp_async_wait<kRingR - 2>();  // the group of step st - 1
-      if (st - 1 < S[0])
-        take_r(st - 1);
-      else
-        hc.e[0] = cst<T>(0.0);
-    } else if (st > 0) {
-      cp -= n3;
-      hq2 -= n;
-#pragma unroll
-      for (int q = 0; q < K; ++q) {
-        if (st - 1 < S[q]) {
-          cx.e[q] = cp[q];
-          cy.e[q] = cp[n + q];
-          cz.e[q] = cp[2 * n + q];
-          hc.e[q] = hq2[q];
-        } else {
-          hc.e[q] = cst<T>(0.0);  // a slot past its last step: an identity step
-        }
-      }
+      take_r(st - 1);
     }
     // recompute the stage states of step st (same arithmetic as the forward)
     V ax, ay, az;
     V f1x, f1y, f1z;
     lorenz_f(x, y, z, s, r, b, f1x, f1y, f1z);
-    V U2x, U2y, U2z, U3x, U3y, U3z, U4x, U4y, U4z, U5x, U5y, U5z, U6x, U6y, U6z;
+    V U2x, U2y, U2z, U3x, U3y, U3z, U4x, U4y, U4z, U5x, U5y, U5z;
     GS_ACC1(kTsA21, f1)
     GS_STAGE(U2x, U2y, U2z, ax, ay, az)
     V f2x, f2y, f2z;
@@ -492,14 +496,16 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     GS_ACCN(kTsA53, f3)
     GS_ACCN(kTsA54, f4)
     GS_STAGE(U5x, U5y, U5z, ax, ay, az)
-    V f5x, f5y, f5z;
-    lorenz_f(U5x, U5y, U5z, s, r, b, f5x, f5y, f5z);
-    GS_ACC1(kTsA61, f1)
-    GS_ACCN(kTsA62, f2)
-    GS_ACCN(kTsA63, f3)
-    GS_ACCN(kTsA64, f4)
-    GS_ACCN(kTsA65, f5)
-    GS_STAGE(U6x, U6y, U6z, ax, ay, az)
+    if constexpr (!kKeep6) {
+      V f5x, f5y, f5z;
+      lorenz_f(U5x, U5y, U5z, s, r, b, f5x, f5y, f5z);
+      GS_ACC1(kTsA61, f1)
+      GS_ACCN(kTsA62, f2)
+      GS_ACCN(kTsA63, f3)
+      GS_ACCN(kTsA64, f4)
+      GS_ACCN(kTsA65, f5)
+      GS_STAGE(U6x, U6y, U6z, ax, ay, az)
+    }
 
     // transposed step, stages 6 .. 1
 #define GS_C(N) tsc<T, kTs##N>()
@@ -551,9 +557,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
       ly += pgy + qy;
       lz += pgz + qz;
     }
-    if constexpr (kAsync) issue_r(st - kRingR);  // into the slot that step st has left
+    issue_r(st - kRingR);  // into the rows that step st has left
   }
-  if constexpr (kAsync) cp_async_wait<0>();
+  cp_async_wait<0>();
   // save points at step 0 cannot exist (save times lie in (t0, t1])
 #pragma unroll
   for (int q = 0; q < K; ++q) {
@@ -571,6 +577,10 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #undef GS_ACC1
 #undef GS_ACCN
 #undef GS_C
+
+// Checkpoint rows per step and slot of the gradient workspace (3, or 6 when
+// U_6 is kept), for gs_workspace_bytes.
+int grad_tsit5_lorenz_ck_rows(int32_t dtype) { return dtype == GS_F64 ? ck_rows<double>() : ck_rows<float>(); }
 
 template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp,
@@ -598,10 +608,12 @@ gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const 
   const int bs = GS_GRAD_BS;
   const int64_t threads = (P->n + K - 1) / K;
   const int64_t grid = (threads + bs - 1) / bs;
-  if (a.theta)
-    k_grad_tsit5_lorenz<T, K, true><<<(unsigned)grid, bs, 0, st>>>(a);
-  else
-    k_grad_tsit5_lorenz<T, K, false><<<(unsigned)grid, bs, 0, st>>>(a);
+  const size_t smem = (size_t)ring_elems<T, K>() * bs * sizeof(T);
+  auto kern = a.theta ? k_grad_tsit5_lorenz<T, K, true> : k_grad_tsit5_lorenz<T, K, false>;
+  // the rings may exceed the 48 KB a launch gets without asking
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return GS_ECUDA;
+  kern<<<(unsigned)grid, bs, smem, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

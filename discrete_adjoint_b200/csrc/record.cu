@@ -22,9 +22,9 @@
 // order, into workspace copies of the mesh arrays (h trajectory-major, so each
 // thread writes its own row front to back and L2 merges the partial sectors);
 // a stable counting sort by decreasing step count gives the slot order; a
-// gather copies every array into slot order (each thread reads one source row
-// in order, writes coalesced) and zero-fills the h rows past each slot's last
-// step.  The gradient kernels then find chains of
+// gather copies every array into slot order (tiles of 32 slots x 32 steps
+// turned in shared memory, so reads and writes are both coalesced) and
+// zero-fills the h rows past each slot's last step.  The gradient kernels then find chains of
 // nearly equal length in every warp.
 #include "kin8.cuh"
 
@@ -173,9 +173,11 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
     ++r.nst;
     const T tprev = r.t;
     r.t = clipped ? tstop : tn;
-    if (METHOD == GS_TSIT5 && D == 3 && a.dense) {
+    if (D == 3 && a.dense) {
       // every save time this step passed: its position inside the step, and
-      // (solve) the Hermite state there from u, f(u) = k1, u_new, f(u_new) = k7
+      // (solve) the Hermite state there from u, f(u), u_new, f(u_new) -- for
+      // Tsit5 the slopes k1 and k7 it already holds, for the Rosenbrock
+      // methods two evaluations of f
       while (r.kk < a.nsave && a.tsave[r.kk] <= r.t) {
         const T th = (a.tsave[r.kk] - tprev) / h;
         if (MODE == kRecMesh) {
@@ -184,10 +186,21 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
         }
         if (MODE == kRecSolve) {
           const HermiteW<T> w = hermite_w(th);
+          T fs[D], fn[D];
+          if constexpr (METHOD == GS_TSIT5) {
+#pragma unroll
+            for (int c = 0; c < D; ++c) {
+              fs[c] = r.k1[c];
+              fn[c] = k7[c];
+            }
+          } else {
+            rhs_s<T, SYS>(r.u, r.p, fs);
+            rhs_s<T, SYS>(un, r.p, fn);
+          }
 #pragma unroll
           for (int c = 0; c < D; ++c)
             a.u_save[((int64_t)r.kk * D + c) * n + r.i] =
-                th == cst<T>(1.0) ? un[c] : hermite_c(w, r.u[c], un[c], r.k1[c], k7[c], h);
+                th == cst<T>(1.0) ? un[c] : hermite_c(w, r.u[c], un[c], fs[c], fn[c], h);
         }
         ++r.kk;
       }
@@ -462,24 +475,60 @@ size_t record_ws_bytes(int64_t n, int32_t smax, int32_t nsave, size_t tsize) {
          al256((size_t)nsave * n * tsize) + (size_t)(smax + 1) * (size_t)nchunk * 4;
 }
 
+// Gather into slot order.  A block owns 32 slots and walks their steps in
+// tiles of 32: each warp reads whole 32-step pieces of the trajectory-major
+// rows (256 contiguous bytes per row in fp64), the tile turns in shared
+// memory, and each warp writes 32 consecutive slots of one step.  Steps past
+// a slot's count are written as zeros (the mesh is zero padded); rows of
+// inactive slots (past n) are neither read nor written.
+constexpr int kGatherWarps = 8;
+
 template <typename T>
-__global__ void k_gather_mesh(int64_t n, int smax, int nsave, const int32_t* __restrict__ order,
-                              const T* __restrict__ h_tmp, const int32_t* __restrict__ si_tmp,
-                              const int32_t* __restrict__ ns_tmp, const int32_t* __restrict__ st_tmp,
-                              const int32_t* __restrict__ nr_tmp, const T* __restrict__ th_tmp, T* h,
-                              int32_t* save_idx, int32_t* nsteps, int32_t* status, int32_t* nreject, T* theta) {
-  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= n) return;
-  const int64_t i = order[j];
-  const int S = ns_tmp[i];
-  nsteps[j] = S;
-  status[j] = st_tmp[i];
-  nreject[j] = nr_tmp[i];
-  for (int k = 0; k < nsave; ++k) save_idx[(int64_t)k * n + j] = si_tmp[(int64_t)k * n + i];
-  if (theta)
-    for (int k = 0; k < nsave; ++k) theta[(int64_t)k * n + j] = th_tmp[(int64_t)k * n + i];
-  const T* src = h_tmp + i * smax;  // trajectory-major: a thread reads one row in order
-  for (int s = 0; s < smax; ++s) h[(int64_t)s * n + j] = s < S ? src[s] : cst<T>(0.0);
+__global__ void __launch_bounds__(32 * kGatherWarps) k_gather_mesh(
+    int64_t n, int smax, int nsave, const int32_t* __restrict__ order, const T* __restrict__ h_tmp,
+    const int32_t* __restrict__ si_tmp, const int32_t* __restrict__ ns_tmp, const int32_t* __restrict__ st_tmp,
+    const int32_t* __restrict__ nr_tmp, const T* __restrict__ th_tmp, T* h, int32_t* save_idx, int32_t* nsteps,
+    int32_t* status, int32_t* nreject, T* theta) {
+  __shared__ T tile[32][33];
+  __shared__ int64_t row[32];
+  __shared__ int cnt[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t j0 = (int64_t)blockIdx.x * 32;
+  if (warp == 0) {
+    const int64_t j = j0 + lane;
+    int S = 0;
+    int64_t i = -1;
+    if (j < n) {
+      i = order[j];
+      S = ns_tmp[i];
+      nsteps[j] = S;
+      status[j] = st_tmp[i];
+      nreject[j] = nr_tmp[i];
+      for (int k = 0; k < nsave; ++k) save_idx[(int64_t)k * n + j] = si_tmp[(int64_t)k * n + i];
+      if (theta)
+        for (int k = 0; k < nsave; ++k) theta[(int64_t)k * n + j] = th_tmp[(int64_t)k * n + i];
+    }
+    row[lane] = i;
+    cnt[lane] = S < 0 ? 0 : (S > smax ? smax : S);
+  }
+  __syncthreads();
+  for (int s0 = 0; s0 < smax; s0 += 32) {
+    // read: warp w takes slots w, w + 8, ...; lane = step within the tile
+    for (int r = warp; r < 32; r += kGatherWarps) {
+      const int s = s0 + lane;
+      T v = cst<T>(0.0);
+      if (row[r] >= 0 && s < cnt[r]) v = h_tmp[row[r] * smax + s];
+      tile[r][lane] = v;
+    }
+    __syncthreads();
+    // write: warp w takes steps w, w + 8, ...; lane = slot
+    const int64_t j = j0 + lane;
+    for (int c = warp; c < 32; c += kGatherWarps) {
+      const int s = s0 + c;
+      if (s < smax && j < n) h[(int64_t)s * n + j] = tile[lane][c];
+    }
+    __syncthreads();
+  }
 }
 
 gs_status order_slots(const int32_t* cnt, int64_t n, int32_t smax, int32_t* hist, int32_t* order, cudaStream_t st) {
@@ -523,7 +572,7 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
   if (rc != GS_OK) return rc;
   rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
   if (rc != GS_OK) return rc;
-  k_gather_mesh<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+  k_gather_mesh<T><<<(unsigned)((n + 31) / 32), 32 * kGatherWarps, 0, st>>>(
       n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp, st_tmp, nr_tmp, th_tmp, (T*)M->h, M->save_idx,
       M->nsteps, M->status, M->nreject, tol->dense ? (T*)M->save_theta : nullptr);
   count_launch();
@@ -558,7 +607,7 @@ gs_status record_node64(const gs_problem* P, const gs_tol* tol, const gs_mesh* M
   if (rc != GS_OK) return rc;
   rc = order_slots(ns_tmp, n, M->smax, hist, M->order, st);
   if (rc != GS_OK) return rc;
-  k_gather_mesh<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp,
+  k_gather_mesh<T><<<(unsigned)((n + 31) / 32), 32 * kGatherWarps, 0, st>>>(n, M->smax, P->nsave, M->order, h_tmp, si_tmp, ns_tmp,
                                                                  st_tmp, nr_tmp, nullptr, (T*)M->h, M->save_idx,
                                                                  M->nsteps, M->status, M->nreject, nullptr);
   count_launch();

@@ -19,7 +19,7 @@ struct SolveArgs {
   const int32_t* status;
   int32_t nsave;
   int32_t smax;
-  const T* theta;  // [nsave][n] by slot: dense save points (Tsit5), or null
+  const T* theta;  // [nsave][n] by slot: dense save points (d = 3 systems), or null
   T* u_save;       // [nsave][d][n] by trajectory
 };
 
@@ -78,14 +78,31 @@ __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
       }
 #pragma unroll
       for (int c = 0; c < 3; ++c) k1[c] = k7[c];
-    } else if (METHOD == GS_ROS3) {
-      T LU[9], R[3], q1[3], v[3], q2[3], q3[3];
-      int P[3];
-      ros3_fwd<T, SYS>(u, p, h, LU, P, R, q1, v, q2, q3, un);
     } else {
       T LU[9], R[3], q1[3], v[3], q2[3];
       int P[3];
-      ros2_fwd<T, SYS>(u, p, h, LU, P, R, q1, v, q2, un);
+      if constexpr (METHOD == GS_ROS3) {
+        T q3[3];
+        ros3_fwd<T, SYS>(u, p, h, LU, P, R, q1, v, q2, q3, un);
+      } else {
+        ros2_fwd<T, SYS>(u, p, h, LU, P, R, q1, v, q2, un);
+      }
+      if (a.theta && st + 1 == next) {
+        // dense save points inside this step: the Hermite state on u, f(u),
+        // u_new, f(u_new), the slopes evaluated here
+        T fs[3], fn[3];
+        rhs3<T, SYS>(u, p, fs);
+        rhs3<T, SYS>(un, p, fn);
+        while (st + 1 == next) {
+          const T th = a.theta[(int64_t)kk * n + j];
+          const HermiteW<T> w = hermite_w(th);
+#pragma unroll
+          for (int c = 0; c < 3; ++c)
+            a.u_save[kk * n3 + c * n + i] = th == cst<T>(1.0) ? un[c] : hermite_c(w, u[c], un[c], fs[c], fn[c], h);
+          ++kk;
+          next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
+        }
+      }
     }
 #pragma unroll
     for (int c = 0; c < D; ++c) u[c] = un[c];
@@ -111,7 +128,7 @@ gs_status launch_solve3(const gs_problem* P, const gs_mesh* M, void* u_save, cud
   a.status = M->status;
   a.nsave = P->nsave;
   a.smax = M->smax;
-  a.theta = P->method == GS_TSIT5 ? (const T*)M->save_theta : nullptr;
+  a.theta = P->system != GS_KIN8 ? (const T*)M->save_theta : nullptr;
   a.u_save = (T*)u_save;
   const unsigned grid = (unsigned)((P->n + 127) / 128);
   if (P->system == GS_LORENZ && P->method == GS_TSIT5)

@@ -127,15 +127,17 @@ typedef struct gs_problem {
 /* Step-size control: accept iff the RMS of e_c / (atol + rtol max(|u_c|, |u'_c|))
  * is <= 1.  h0 > 0 fixes the first proposal; h0 = 0 picks it automatically
  * (Hairer, Norsett & Wanner I, II.4).
- * dense = 0: steps are shortened to land on every save time.  dense = 1 (Tsit5,
- * d = 3 only): steps stop only at t1; a save time inside a step is located by
+ * dense = 0: steps are shortened to land on every save time.  dense = 1 (the
+ * d = 3 systems, every method): steps stop only at t1; a save time inside a step is located by
  * its position theta in (0, 1] (gs_mesh.save_theta) and the state there is the
  * cubic Hermite interpolant of the step on its end states and slopes,
  *   u = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
  *   H01 = theta^2 (3 - 2 theta), H00 = 1 - H01, H10 = theta (1 - theta)^2,
  *   H11 = -theta^2 (1 - theta).
  * The loss and its derivative then pass through that interpolant (theta, like
- * h, is data).  Dense output (interpolated save times, as in the H200
+ * h, is data).  Tsit5 holds both slopes already (its first and FSAL stages);
+ * the Rosenbrock methods evaluate f twice more on a step that holds an
+ * interior save point.  Dense output (interpolated save times, as in the H200
  * forward-sensitivity study) prints no interpolant, so this cubic Hermite one
  * is this library's choice. */
 typedef struct gs_tol {
@@ -210,7 +212,7 @@ GS_API gs_status gs_count(const gs_problem* prob, const gs_tol* tol, int32_t sma
  * ordering and a gather into slot order, all on stream.  Built for GS_LORENZ
  * and GS_ROBERTSON with GS_TSIT5, GS_ROS2 or GS_ROS3, GS_KIN8 with GS_ROS2 or
  * GS_ROS3 (fp64 and fp32), and GS_NODE64 with GS_TSIT5 in fp32; dense records
- * for GS_TSIT5 on the d = 3 systems.  gs_count, gs_solve and gs_solve_adaptive
+ * for every method on the d = 3 systems.  gs_count, gs_solve and gs_solve_adaptive
  * take the same combinations.  (Evolve.pub review, "Summary": the adaptive
  * solve happens once and keeps each trajectory's accepted step sizes.)
  */
@@ -251,9 +253,10 @@ GS_API gs_status gs_solve_adaptive(const gs_problem* prob, const gs_tol* tol, in
  *   dshared  device [64][64] dtype, GS_NODE64: sum_i dL_i/dW; else NULL
  *   ws       workspace of gs_workspace_bytes(prob, mesh, GS_OP_GRAD) bytes
  * All indexed by trajectory.  Slots with status != 0 get NaN loss/dp/du0 and
- * do not contribute to dshared.  Built for GS_LORENZ with GS_TSIT5 (dense
- * save points included), GS_ROS2 or GS_ROS3; GS_ROBERTSON and GS_KIN8 with
- * GS_ROS2 or GS_ROS3 (fp64 and fp32 for all of these); GS_NODE64 with GS_TSIT5
+ * do not contribute to dshared.  Built for GS_LORENZ with GS_TSIT5, GS_ROS2
+ * or GS_ROS3; GS_ROBERTSON with GS_ROS2 or GS_ROS3 (dense save points
+ * included for all of these); GS_KIN8 with GS_ROS2 or GS_ROS3 (fp64 and fp32
+ * for all of these); GS_NODE64 with GS_TSIT5
  * in fp32.  Other combinations return GS_EUNSUPPORTED.  (Evolve.pub review,
  * "Summary": the replay is a fixed-length chain without branches, and its
  * backward sweep is the exact discrete adjoint.)

@@ -82,33 +82,47 @@ def _relinf(g, r):
     return np.abs(g - r).max(0) / np.abs(r).max(0)
 
 
-def parity(out, prob, om, tol=None, quantile_ok=0.99, dual=True):
+# Per-trajectory allowance over the oracle's own plain-precision error.
+ROUTE_FACTOR = 4.0
+
+
+def route_error(prob, om, ref, dual=True):
+    """kappa_i: the larger per-trajectory error, against `ref`, of the
+    oracle's own plain-precision routes on the same mesh (its tape, and its
+    dual numbers where built).  It measures how much rounding in this
+    precision costs on trajectory i: the conditioning of its reverse sweep."""
+    import oracle
+    own = oracle.grad(prob, om, "tape")
+    k = _relinf(np.vstack([own["dp"], own["du0"]]), ref)
+    if dual and prob.system != "node64":
+        dd = oracle.grad(prob, om, "dual")
+        k = np.maximum(k, _relinf(np.vstack([dd["dp"], dd["du0"]]), ref))
+    return k
+
+
+def parity(out, prob, om, tol=None, c=ROUTE_FACTOR, dual=True):
     """Gradient parity of a GPU result against the oracle on the oracle's mesh.
 
     Reference: the oracle's tape with a wide reverse sweep (the most accurate
     evaluation of the exact discrete adjoint here).  Error: per trajectory,
-    ||g - g_ref||_inf / ||g_ref||_inf over (dp, du0).  On chaotic trajectories
-    the reverse sweep's conditioning puts any plain-precision adjoint -- the
-    oracle's own tape and dual routes included -- near or above the stated
-    gate (1e-12 fp64, 1e-4 fp32), with heavy-tailed errors.  So:
-      - at least `quantile_ok` of the trajectories meet the stated gate;
-      - the worst GPU error is within 4x the worst error of the oracle's own
-        plain-precision routes on the same sample (or the gate);
-      - no trajectory exceeds max(gate, 64 x the oracle routes' error on it).
-    Returns the per-trajectory errors."""
+    e_i = ||g - g_ref||_inf / ||g_ref||_inf over (dp, du0).  Gate, for every
+    trajectory i: e_i <= max(tol, c kappa_i), tol the stated gate (1e-12
+    fp64, 1e-4 fp32) and kappa_i the oracle's own plain-precision error on
+    that trajectory (route_error).  So the GPU may miss the stated gate only
+    on a trajectory where the oracle's own evaluation in the same precision
+    misses it too, and then by at most the factor c.  Returns e."""
     import oracle
     tol = tol or TOL[prob.dtype]
     wide = oracle.grad(prob, om, "tape_wide")
     r = np.vstack([wide["dp"], wide["du0"]])
     g = np.vstack([out.dp.double().cpu().numpy(), out.du0.double().cpu().numpy()])
     e = _relinf(g, r)
-    own = oracle.grad(prob, om, "tape")
-    cond = _relinf(np.vstack([own["dp"], own["du0"]]), r)
-    if dual and prob.system != "node64":
-        dd = oracle.grad(prob, om, "dual")
-        cond = np.maximum(cond, _relinf(np.vstack([dd["dp"], dd["du0"]]), r))
-    assert np.mean(e <= tol) >= quantile_ok, (np.mean(e <= tol), e.max())
-    assert e.max() <= max(tol, 4 * cond.max()), (e.max(), cond.max())
-    bound = np.maximum(tol, 64 * cond)
-    assert (e <= bound).all(), (e.max(), bound[np.argmax(e / bound)])
+    over = e > tol
+    if over.any():
+        kappa = np.zeros_like(e)
+        kappa[:] = route_error(prob, om, r, dual)
+        bound = np.maximum(tol, c * kappa)
+        w = int(np.argmax(e / bound))
+        assert (e <= bound).all(), (f"{int((e > bound).sum())} of {len(e)} trajectories over the gate; worst {w}: "
+                                    f"error {e[w]:.3e}, oracle routes {kappa[w]:.3e}, bound {bound[w]:.3e}")
     return e

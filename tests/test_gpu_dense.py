@@ -102,9 +102,9 @@ def test_dense_unsupported_paths(case):
     mesh = mesh_from_oracle(om, "f64")
     with pytest.raises(gs.gradsolve.GradsolveError):
         gs.gs_sens(ensemble(prob), mesh, **loss_args(prob))
-    rob = W.robertson(4)
+    k8 = W.kin8(4)  # dense records are built for the d = 3 systems
     with pytest.raises(gs.gradsolve.GradsolveError):
-        gs.gs_count(ensemble(rob), rob.rtol, rob.atol, 100, dense=True)
+        gs.gs_count(ensemble(k8), k8.rtol, k8.atol, 100, dense=True)
 
 
 def test_full_size_sampled():

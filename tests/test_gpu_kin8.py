@@ -76,7 +76,7 @@ def test_ros2_grad():
     assert (om.status == 0).all()
     out = gs.gs_grad(ensemble(prob), mesh_from_oracle(om, "f64"), **loss_args(prob))
     torch.cuda.synchronize()
-    parity(out, prob, om, quantile_ok=1.0)
+    parity(out, prob, om)
 
 
 def test_solve_and_adaptive_solve(k3):

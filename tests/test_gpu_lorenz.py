@@ -60,7 +60,7 @@ def test_grad_on_oracle_mesh(small, perm):
     torch.cuda.synchronize()
     e = grad_rel_err(out, og)
     assert e.max() <= TOL["f64"], e.max()
-    parity(out, prob, om, quantile_ok=1.0)
+    parity(out, prob, om)
     le = np.abs(out.loss.cpu().numpy() - og["loss"]) / np.abs(og["loss"])
     assert le.max() <= 1e-14, le.max()  # the forward replay follows the same contract
 
@@ -105,37 +105,48 @@ def test_lorenz_1m_shape(dtype, n):
     parity(out, prob, om)
 
 
-def test_full_size_sampled():
+@pytest.mark.parametrize("dtype", ["f64", "f32"])
+def test_full_size_sampled(dtype):
     """2**20 trajectories in the launch configuration the benchmark times; the
-    oracle checks a sample (random + the longest chains) one by one."""
-    prob = W.lorenz_1m()
+    oracle checks a sample (random + the longest chains) one by one.  fp64
+    meshes equal the oracle's to 1e-10 (bitwise in practice); fp32 ones, of the
+    fp32 instantiation of the oracle, have equal step counts on almost every
+    trajectory and step sizes within fp32 rounding where they do."""
+    prob = W.lorenz_1m(dtype=dtype)
+    td = torch.float64 if dtype == "f64" else torch.float32
     ens = ensemble(prob)
     nsteps, status = gs.gs_count(ens, prob.rtol, prob.atol, 2048)
-    smax = int(nsteps.max().item())
-    mesh = gs.new_mesh(prob.n, smax, 10, "f64", dev())
-    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
-    torch.cuda.synchronize()
-    assert (mesh.status == 0).all()
     ns_all = nsteps.cpu().numpy()
     rng = np.random.default_rng(11)
     idx = np.unique(np.concatenate([rng.choice(prob.n, 384, replace=False), np.argsort(ns_all)[-32:]]))
     sub = prob.subset(idx)
     om = oracle.record(sub, 2048)
+    assert (om.status == 0).all()
+    smax = max(int(nsteps.max().item()), int(om.nsteps.max()))
+    mesh = gs.new_mesh(prob.n, smax, 10, dtype, dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    assert (mesh.status == 0).all()
     # mesh parity on the sample
     order = mesh.order.cpu().numpy()
     inv = np.empty_like(order)
     inv[order] = np.arange(prob.n)
     slots = inv[idx]
-    hs = mesh.h[:, torch.tensor(slots, device=dev())].cpu().numpy().T
+    hs = mesh.h[:, torch.tensor(slots, device=dev())].double().cpu().numpy().T
     ns = mesh.nsteps.cpu().numpy()[slots]
-    assert np.array_equal(ns, om.nsteps)
-    assert mesh_rel_err(hs, om.h[:, :smax], ns) <= 1e-10
+    if dtype == "f64":
+        assert np.array_equal(ns, om.nsteps)
+        assert mesh_rel_err(hs, om.h[:, :smax], ns) <= 1e-10
+    else:
+        same = ns == om.nsteps
+        assert same.mean() >= 0.97, same.mean()
+        assert mesh_rel_err(hs[same], om.h[same, :smax], ns[same]) <= 1e-5
     # gradient parity on the oracle's mesh, injected into the sampled slots of
     # the full-size mesh (trajectories are independent)
     ts = torch.tensor(slots, device=dev())
     hi = np.zeros((smax, len(idx)))
     hi[:] = om.h[:, :smax].T
-    mesh.h[:, ts] = tens(hi, torch.float64)
+    mesh.h[:, ts] = tens(hi, td)
     mesh.nsteps[ts] = tens(om.nsteps.astype(np.int32), torch.int32)
     mesh.save_idx[:, ts] = tens(om.save_idx.T.astype(np.int32), torch.int32)
     out = gs.gs_grad(ens, mesh, **loss_args(prob))

@@ -12,7 +12,7 @@ import torch
 import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
-from gpu_util import TOL, dev, ensemble, loss_args, mesh_from_oracle, parity
+from gpu_util import ROUTE_FACTOR, TOL, dev, ensemble, loss_args, mesh_from_oracle, parity
 
 pytestmark = pytest.mark.gpu
 
@@ -38,14 +38,16 @@ def _rel(a, ref):
 
 
 def _sens_parity(S, prob, om, tol):
-    """The gradient criterion applied to the matrices: most trajectories within
-    the gate, the worst within 4x the oracle's own plain-precision route (dual
-    numbers) against the wide reference."""
+    """The gradient criterion applied to the matrices, per trajectory: every
+    trajectory within max(tol, c kappa_i), kappa_i the error of the oracle's
+    own plain-precision route (dual numbers) on it against the wide
+    reference."""
     ref = _sens_wide(prob, om)
     e = _rel(S, ref)
-    cond = _rel(oracle.sens(prob, om), ref)
-    assert np.mean(e <= tol) >= 0.99, (np.mean(e <= tol), e.max())
-    assert e.max() <= max(tol, 4 * cond.max()), (e.max(), cond.max())
+    kappa = _rel(oracle.sens(prob, om), ref)
+    bound = np.maximum(tol, ROUTE_FACTOR * kappa)
+    w = int(np.argmax(e / bound))
+    assert (e <= bound).all(), (int((e > bound).sum()), w, e[w], kappa[w])
     return e
 
 
@@ -65,7 +67,7 @@ def test_small_fp64():
     _sens_parity(S[..., :64], sub, oracle.record(sub, 256), 1e-12)
     loss, _ = oracle.replay(prob, om)
     assert np.abs(out.loss.cpu().numpy() - loss).max() <= 1e-14 * np.abs(loss).max()
-    parity(out, prob, om, quantile_ok=1.0)
+    parity(out, prob, om)
 
 
 @pytest.mark.parametrize("dtype", ["f64", "f32"])

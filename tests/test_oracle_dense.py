@@ -21,16 +21,13 @@ from scipy.integrate import solve_ivp
 
 import oracle
 import workloads as W
-from test_oracle_method import _dpoly, _kappa, _poly, _ros2_R, _tsit5_R_coeffs
+from test_oracle_method import _R_any, _kappa
 
 EPS = np.finfo(np.float64).eps
 
 
 def _R_dR(method, z):
-    if method == "tsit5":
-        co = _tsit5_R_coeffs()
-        return _poly(co, z), _dpoly(co, z)
-    return _ros2_R(z, Fr(oracle.ros2_gamma()))
+    return _R_any(method, z)
 
 
 def _weights(th):
@@ -39,7 +36,8 @@ def _weights(th):
     return 1 - th * th * (3 - 2 * th), th * th * (3 - 2 * th), th * (1 - th) ** 2, -th * th * (1 - th)
 
 
-@pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 400.0])])
+@pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 400.0]),
+                                         ("ros3", [0.5, 50.0, 400.0])])
 def test_closed_form_on_the_test_equation(method, lams):
     prob = W.scalar_linear([-l for l in lams], t1=2.0, method=method)
     prob.tsave = np.array([0.2345, 0.777, 1.3, 2.0])
