@@ -213,12 +213,34 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #pragma unroll
     for (int q = 0; q < K; ++q) hv.e[q] = sf < S[q] ? rg[((sf & (kRingF - 1)) * K + q) * BS] : cst<T>(0.0);
   };
+  // Save points, read one save point ahead: next[q] is the step count at
+  // which slot q's current save point kk[q] falls, (tv0, tv1, tv2)[q] its loss
+  // vector (the target for SUMSQ, zero without one; the weights for LINEAR)
+  // and next2[q] the step count of the save point after it.  Each load is
+  // issued a whole save interval before its value is used, so the divergent
+  // save-point branch never waits on DRAM.
+  auto sp_idx = [&](int q, int k) -> int {
+    return (k >= 0 && k < a.nsave && S[q] > 0) ? a.save_idx[(int64_t)k * n + j0 + q] : -1;
+  };
+  const T* const lvec = a.loss_kind == GS_LOSS_SUMSQ ? a.target : a.weight;
+  auto sp_vec = [&](int q, int k, T& v0, T& v1, T& v2) {
+    v0 = v1 = v2 = cst<T>(0.0);
+    if (lvec && k >= 0 && k < a.nsave && i[q] >= 0) {
+      const int64_t o = (int64_t)k * 3 * n + i[q];
+      v0 = lvec[o];
+      v1 = lvec[o + n];
+      v2 = lvec[o + 2 * n];
+    }
+  };
   V L = vsplat<T, K>(cst<T>(0.0));
-  int kk[K], next[K];
+  int kk[K], next[K], next2[K];
+  T tv0[K], tv1[K], tv2[K];
 #pragma unroll
   for (int q = 0; q < K; ++q) {
     kk[q] = 0;
-    next[q] = S[q] > 0 ? a.save_idx[j0 + q] : -1;
+    next[q] = sp_idx(q, 0);
+    next2[q] = sp_idx(q, 1);
+    sp_vec(q, 0, tv0[q], tv1[q], tv2[q]);
   }
   V k1x, k1y, k1z;
   lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);
@@ -305,7 +327,6 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     for (int q = 0; q < K; ++q) {
       // a landing record has at most one save point per step; a dense one any number
       while (st + 1 == next[q]) {
-        const int64_t o = (int64_t)kk[q] * 3 * n + i[q];
         T ux = x.e[q], uy = y.e[q], uz = z.e[q];
         if (DENSE) {
           const T th = a.theta[(int64_t)kk[q] * n + j0 + q];
@@ -317,21 +338,23 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
           }
         }
         T Lq = L.e[q];
-        if (a.loss_kind == GS_LOSS_SUMSQ) {
-          const T dx = a.target ? ux - a.target[o] : ux;
-          const T dy = a.target ? uy - a.target[o + n] : uy;
-          const T dz = a.target ? uz - a.target[o + 2 * n] : uz;
+        if (a.loss_kind == GS_LOSS_SUMSQ) {  // u - 0 = u bitwise when there is no target
+          const T dx = ux - tv0[q];
+          const T dy = uy - tv1[q];
+          const T dz = uz - tv2[q];
           Lq = fmaT(dx, dx, Lq);
           Lq = fmaT(dy, dy, Lq);
           Lq = fmaT(dz, dz, Lq);
         } else {
-          Lq = fmaT(a.weight[o], ux, Lq);
-          Lq = fmaT(a.weight[o + n], uy, Lq);
-          Lq = fmaT(a.weight[o + 2 * n], uz, Lq);
+          Lq = fmaT(tv0[q], ux, Lq);
+          Lq = fmaT(tv1[q], uy, Lq);
+          Lq = fmaT(tv2[q], uz, Lq);
         }
         L.e[q] = Lq;
         ++kk[q];
-        next[q] = kk[q] < a.nsave ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
+        next[q] = next2[q];
+        next2[q] = sp_idx(q, kk[q] + 1);
+        sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
         if (!DENSE) break;
       }
     }
@@ -350,9 +373,11 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   V lx = vsplat<T, K>(cst<T>(0.0)), ly = lx, lz = lx;
   V ps = lx, pr = lx, pb = lx;
 #pragma unroll
-  for (int q = 0; q < K; ++q) {
+  for (int q = 0; q < K; ++q) {  // save points in reverse, read one ahead as in the forward
     kk[q] = a.nsave - 1;
-    next[q] = S[q] > 0 ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
+    next[q] = sp_idx(q, kk[q]);
+    next2[q] = sp_idx(q, kk[q] - 1);
+    sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
   }
   V cx = x, cy = y, cz = z, hc = vsplat<T, K>(cst<T>(0.0));
   V gx6 = x, gy6 = y, gz6 = z;
@@ -407,7 +432,6 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #pragma unroll
     for (int q = 0; q < K; ++q) {
       while (st + 1 == next[q]) {
-        const int64_t o = (int64_t)kk[q] * 3 * n + i[q];
         T th = cst<T>(1.0);
         HermiteW<T> w;
         T ux = x.e[q], uy = y.e[q], uz = z.e[q], fsx, fsy, fsz, fnx, fny, fnz;
@@ -425,13 +449,13 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
         }
         T gx, gy, gz;  // d loss_k / d u(t_k)
         if (a.loss_kind == GS_LOSS_SUMSQ) {
-          gx = cst<T>(2.0) * (a.target ? ux - a.target[o] : ux);
-          gy = cst<T>(2.0) * (a.target ? uy - a.target[o + n] : uy);
-          gz = cst<T>(2.0) * (a.target ? uz - a.target[o + 2 * n] : uz);
+          gx = cst<T>(2.0) * (ux - tv0[q]);
+          gy = cst<T>(2.0) * (uy - tv1[q]);
+          gz = cst<T>(2.0) * (uz - tv2[q]);
         } else {
-          gx = a.weight[o];
-          gy = a.weight[o + n];
-          gz = a.weight[o + 2 * n];
+          gx = tv0[q];
+          gy = tv1[q];
+          gz = tv2[q];
         }
         if (!DENSE || th == cst<T>(1.0)) {
           lx.e[q] += gx;
@@ -453,7 +477,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
           pnz.e[q] = fmaT(hh * w.h10, gz, pnz.e[q]);
         }
         --kk[q];
-        next[q] = kk[q] >= 0 ? a.save_idx[(int64_t)kk[q] * n + j0 + q] : -1;
+        next[q] = next2[q];
+        next2[q] = sp_idx(q, kk[q] - 1);
+        sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
         if (!DENSE) break;
       }
     }

@@ -178,7 +178,9 @@ def grad(prob, mesh: Mesh, mode: str = "tape", nthreads: int | None = None):
     mode ``"tape"``: reverse-mode AD (tape).  mode ``"dual"``: forward mode,
     one dual-number pass per input (p and u0; not node64).  mode
     ``"tape_wide"``: the tape with its adjoints accumulated in a wider type
-    (long double for fp64, double for fp32).
+    (long double for fp64, double for fp32).  mode ``"tape_fused"``: the tape
+    with every adjoint update as one fused multiply-add (plain precision,
+    rounded differently from ``"tape"``).
     Returns dict(loss [n], dp [np][n], du0 [d][n], dW [64,64] or None).
     """
     L = lib()
@@ -191,7 +193,7 @@ def grad(prob, mesh: Mesh, mode: str = "tape", nthreads: int | None = None):
     dW = np.zeros((64, 64)) if prob.system == "node64" else None
     rc = L.or_grad(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[prob.dtype], n, d, npar, _d(_f64(prob.p)),
                    _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, si.shape[1], _d(h), _i(ns), _i(si),
-                   _theta(mesh), _i(st), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), {"tape": 0, "dual": 1, "tape_wide": 2}[mode],
+                   _theta(mesh), _i(st), LOSSES[prob.loss], _d(_f64(prob.target)), _d(_f64(prob.weight)), {"tape": 0, "dual": 1, "tape_wide": 2, "tape_fused": 3}[mode],
                    _d(loss), _d(dp), _d(du0), _d(dW), nthreads or default_threads())
     _check(rc, "grad")
     return {"loss": loss, "dp": dp, "du0": du0, "dW": dW}

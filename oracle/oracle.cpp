@@ -838,7 +838,11 @@ inline void gather_kd(const double* src, int nsave, int d, int64_t n, int64_t i,
 // (np), du0 (d) and, for NODE64, accumulates dW (64*64) into dW_acc.
 // A = the type the reverse sweep accumulates adjoints in (T, or long double
 // for a reference with 11 more bits; the tape's partials are the same).
-template <class T, class A = T>
+// FUSED: each adjoint update adj[parent] += partial * adj[node] as one fused
+// multiply-add (one rounding instead of two): the same derivative evaluated
+// with different rounding, a third plain-precision route beside the tape and
+// the dual numbers (used to gauge how much rounding costs on a trajectory).
+template <class T, class A = T, bool FUSED = false>
 void grad_one_tape(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, double* loss, double* dp,
                    double* du0, double* dW_acc) {
   using R = Rv<T>;
@@ -874,9 +878,15 @@ void grad_one_tape(const Prob& P, const Mesh& Mh, const Loss& Ls, int64_t i, dou
     const Node<T>& nd = tp.nodes[k];
     A a = adj[k];
     if (a == A(0)) continue;
-    if (nd.a >= 0) adj[nd.a] += A(nd.da) * a;
-    if (nd.b >= 0) adj[nd.b] += A(nd.db) * a;
-    if (nd.c >= 0) adj[nd.c] += A(nd.dc) * a;
+    if (FUSED) {
+      if (nd.a >= 0) adj[nd.a] = std::fma(A(nd.da), a, adj[nd.a]);
+      if (nd.b >= 0) adj[nd.b] = std::fma(A(nd.db), a, adj[nd.b]);
+      if (nd.c >= 0) adj[nd.c] = std::fma(A(nd.dc), a, adj[nd.c]);
+    } else {
+      if (nd.a >= 0) adj[nd.a] += A(nd.da) * a;
+      if (nd.b >= 0) adj[nd.b] += A(nd.db) * a;
+      if (nd.c >= 0) adj[nd.c] += A(nd.dc) * a;
+    }
   }
   for (int c = 0; c < d; ++c) du0[c] = double(u0[c].id >= 0 ? adj[u0[c].id] : A(0));
   for (int c = 0; c < np; ++c) dp[c] = double(p[c].id >= 0 ? adj[p[c].id] : A(0));
@@ -1051,7 +1061,8 @@ int or_solve_adaptive(int sys, int method, int dtype, int64_t n, int d, int np, 
 // mode, one dual-number pass per input direction (p and u0 only; not NODE64).
 // mode 2: the tape with adjoints accumulated in a wider type (long double for
 // fp64 runs, double for fp32 runs): same forward values and partials, less
-// rounding in the reverse sweep.
+// rounding in the reverse sweep.  mode 3: the tape with fused adjoint updates
+// (plain precision, rounded differently from mode 0).
 // Trajectories with status != 0 get NaN outputs.  dW (NODE64) is the sum over
 // trajectories, accumulated per thread chunk and then in chunk order.
 int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
@@ -1062,7 +1073,7 @@ int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const doub
   int rc = check_prob(P);
   if (rc) return rc;
   if (mode == 1 && sys == SYS_NODE64) return -4;
-  if (mode < 0 || mode > 2) return -1;
+  if (mode < 0 || mode > 3) return -1;
   Mesh Mh{smax, nsave, h, nsteps, save_idx, theta};
   Loss Ls{loss_kind, target, weight};
   int nt = std::max(1, nthreads);
@@ -1078,7 +1089,13 @@ int or_grad(int sys, int method, int dtype, int64_t n, int d, int np, const doub
         continue;
       }
       double L;
-      if (mode == 0 || mode == 2) {
+      if (mode == 3) {
+        double* acc = sys == SYS_NODE64 ? dWp[tid].data() : nullptr;
+        if (dtype == DT_F64)
+          grad_one_tape<double, double, true>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
+        else
+          grad_one_tape<float, float, true>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);
+      } else if (mode == 0 || mode == 2) {
         double* acc = sys == SYS_NODE64 ? dWp[tid].data() : nullptr;
         if (dtype == DT_F64 && mode == 0)
           grad_one_tape<double>(P, Mh, Ls, i, &L, gp.data(), gu.data(), acc);

@@ -87,16 +87,18 @@ ROUTE_FACTOR = 4.0
 
 
 def route_error(prob, om, ref, dual=True):
-    """kappa_i: the larger per-trajectory error, against `ref`, of the
-    oracle's own plain-precision routes on the same mesh (its tape, and its
-    dual numbers where built).  It measures how much rounding in this
-    precision costs on trajectory i: the conditioning of its reverse sweep."""
+    """kappa_i: the largest per-trajectory error, against `ref`, of the
+    oracle's own plain-precision routes on the same mesh: its tape, the tape
+    with fused adjoint updates, and its dual numbers where built.  Each is
+    one draw of what rounding in this precision costs on trajectory i (on a
+    chaotic trajectory a few amplified roundings dominate, so single draws
+    differ by up to ~20x); the largest of three is a steadier gauge."""
     import oracle
-    own = oracle.grad(prob, om, "tape")
-    k = _relinf(np.vstack([own["dp"], own["du0"]]), ref)
-    if dual and prob.system != "node64":
-        dd = oracle.grad(prob, om, "dual")
-        k = np.maximum(k, _relinf(np.vstack([dd["dp"], dd["du0"]]), ref))
+    k = None
+    for mode in ("tape", "tape_fused") + (("dual",) if dual and prob.system != "node64" else ()):
+        g = oracle.grad(prob, om, mode)
+        e = _relinf(np.vstack([g["dp"], g["du0"]]), ref)
+        k = e if k is None else np.maximum(k, e)
     return k
 
 

@@ -17,9 +17,10 @@ from gpu_util import ROUTE_FACTOR, TOL, dev, ensemble, loss_args, mesh_from_orac
 pytestmark = pytest.mark.gpu
 
 
-def _sens_wide(prob, om):
-    """Rows of S from the oracle's tape with a wide reverse sweep: one linear
-    loss per (save point, component) whose weight selects that entry."""
+def _sens_wide(prob, om, mode="tape_wide"):
+    """Rows of S from the oracle's tape (by default with a wide reverse
+    sweep): one linear loss per (save point, component) whose weight selects
+    that entry."""
     K = len(prob.tsave)
     S = np.zeros((K, 3, 6, prob.n))
     for k in range(K):
@@ -27,7 +28,7 @@ def _sens_wide(prob, om):
             w = np.zeros((K, 3, prob.n))
             w[k, c] = 1.0
             q = dataclasses.replace(prob, loss="linear", weight=w, target=None)
-            g = oracle.grad(q, om, mode="tape_wide")
+            g = oracle.grad(q, om, mode=mode)
             S[k, c, :3], S[k, c, 3:] = g["dp"], g["du0"]
     return S
 
@@ -39,12 +40,13 @@ def _rel(a, ref):
 
 def _sens_parity(S, prob, om, tol):
     """The gradient criterion applied to the matrices, per trajectory: every
-    trajectory within max(tol, c kappa_i), kappa_i the error of the oracle's
-    own plain-precision route (dual numbers) on it against the wide
-    reference."""
+    trajectory within max(tol, c kappa_i), kappa_i the largest error of the
+    oracle's own plain-precision routes (dual numbers, the tape, the tape
+    with fused updates) on it against the wide reference."""
     ref = _sens_wide(prob, om)
     e = _rel(S, ref)
-    kappa = _rel(oracle.sens(prob, om), ref)
+    kappa = np.maximum.reduce([_rel(oracle.sens(prob, om), ref), _rel(_sens_wide(prob, om, "tape"), ref),
+                               _rel(_sens_wide(prob, om, "tape_fused"), ref)])
     bound = np.maximum(tol, ROUTE_FACTOR * kappa)
     w = int(np.argmax(e / bound))
     assert (e <= bound).all(), (int((e > bound).sum()), w, e[w], kappa[w])

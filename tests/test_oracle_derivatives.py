@@ -67,6 +67,25 @@ def test_tape_matches_dual(recorded, case):
     assert e.max() <= tol, (e.max(), tol)
 
 
+@pytest.mark.parametrize("case", list(CASES))
+def test_fused_tape_matches_dual(recorded, case):
+    """The tape with fused adjoint updates (a third plain-precision route,
+    which the GPU parity gate uses to gauge what rounding costs on each
+    trajectory) computes the same derivative: within eps per step of the
+    dual numbers, like the tape, with the same forward values.  Its rounding
+    differs from the tape's on the chaotic ensemble."""
+    prob, mesh = recorded[case]
+    gf = oracle.grad(prob, mesh, "tape_fused")
+    gd = oracle.grad(prob, mesh, "dual")
+    assert np.array_equal(gf["loss"], gd["loss"])
+    e = _relinf([gf["dp"], gf["du0"]], [gd["dp"], gd["du0"]])
+    tol = max(1e-13, np.finfo(float).eps * mesh.nsteps.max())
+    assert e.max() <= tol, (e.max(), tol)
+    if case == "lorenz_1m":
+        gt = oracle.grad(prob, mesh, "tape")
+        assert not np.array_equal(gf["du0"], gt["du0"])
+
+
 @pytest.mark.parametrize("case", ["lorenz_small", "robertson", "robertson_ros3"])
 def test_tape_matches_fixed_mesh_fd(recorded, case):
     prob, mesh = recorded[case]
