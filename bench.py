@@ -604,11 +604,14 @@ def run_ours(args):
 
     # sizing pass (setup, untimed): mesh capacity = the longest chain
     dense = W.get("dense", False)
+    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload), dense=dense, stream=stream)
+    smax = int(nsteps.max().item())
+    # its time, on a second call (the first also loads the library's kernels)
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     c0.record(stream)
-    nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload), dense=dense, stream=stream)
+    gs.gs_count(ens, prob.rtol, prob.atol, smax_cap(args.workload), nsteps=nsteps, dense=dense, stream=stream)
     c1.record(stream)
-    smax = int(nsteps.max().item())
+    c1.synchronize()
     count_ms = c0.elapsed_time(c1)
     mesh = gs.new_mesh(n, smax, len(prob.tsave), args.dtype, dev, dense=dense)
     ws_rec = gs.workspace(gs.gs_workspace_bytes(ens, mesh, gs.gradsolve.OP_RECORD), dev)

@@ -231,8 +231,8 @@ gs_status gs_sens(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
-  // Tsit5: Lorenz; ROS2 / ROS3: Lorenz and Robertson; no dense save points
-  if (M->save_theta || P->system == GS_NODE64 || P->system == GS_KIN8) return GS_EUNSUPPORTED;
+  // Tsit5: Lorenz; ROS2 / ROS3: Lorenz and Robertson; landing or dense save points
+  if (P->system == GS_NODE64 || P->system == GS_KIN8) return GS_EUNSUPPORTED;
   if (P->method == GS_TSIT5 && P->system != GS_LORENZ) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;

@@ -28,13 +28,9 @@ namespace gs {
 // 128 (8 warps per SM) and twice the blocks to spread a small ensemble over
 // the SMs.
 constexpr int kKin8Block = 64;
-// Copy rings: the forward streams h, the reverse (u_s, h_s), kKin8Ring steps
-// ahead, so the step's first instructions do not wait on DRAM.
-constexpr int kKin8Ring = 4;
 
 template <typename T, int METHOD>
 __global__ void __launch_bounds__(kKin8Block) k_grad_kin8(RosArgs<T> a) {
-  extern __shared__ __align__(16) unsigned char ring_raw[];
   constexpr int D = 8;
   const int64_t n = a.n;
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -66,17 +62,8 @@ __global__ void __launch_bounds__(kKin8Block) k_grad_kin8(RosArgs<T> a) {
   int next = a.save_idx[j];
   bool ok = true;
   // ---------------------------------------------------------------- forward
-  const ThreadRing<T, 1, kKin8Ring> rf(ring_raw);
-  auto issue_f = [&](int sf) {
-    if (sf < S) cp_async_el(rf.at(sf, 0), hp + (int64_t)sf * n);
-    cp_async_commit();
-  };
-#pragma unroll
-  for (int sf = 0; sf < kKin8Ring; ++sf) issue_f(sf);
   for (int st = 0; st < S; ++st) {
-    cp_async_wait<kKin8Ring - 1>();  // the group of step st
-    const T h = *rf.at(st, 0);
-    issue_f(st + kKin8Ring);  // its slot is free once h is in a register
+    const T h = hp[(int64_t)st * n];
 #pragma unroll
     for (int c = 0; c < D; ++c) cp[c * n] = u[c];
     cp += nD;
@@ -96,20 +83,7 @@ __global__ void __launch_bounds__(kKin8Block) k_grad_kin8(RosArgs<T> a) {
       next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
     }
   }
-  cp_async_wait<0>();  // the reverse reuses the ring
   // ---------------------------------------------------------------- reverse
-  const ThreadRing<T, D + 1, kKin8Ring> rr(ring_raw);
-  auto issue_r = [&](int sr) {
-    if (sr >= 0 && sr < S) {
-      const T* c = a.ck + (int64_t)sr * nD + j;
-#pragma unroll
-      for (int w = 0; w < D; ++w) cp_async_el(rr.at(sr, w), c + w * n);
-      cp_async_el(rr.at(sr, D), hp + (int64_t)sr * n);
-    }
-    cp_async_commit();
-  };
-#pragma unroll
-  for (int i2 = 0; i2 < kKin8Ring; ++i2) issue_r(S - 1 - i2);
   T lam[D], pb[D], unx[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) {
@@ -125,12 +99,11 @@ __global__ void __launch_bounds__(kKin8Block) k_grad_kin8(RosArgs<T> a) {
       --kk;
       next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
     }
-    cp_async_wait<kKin8Ring - 1>();  // the group of step st
+    cp -= nD;
     T us[D];
 #pragma unroll
-    for (int c = 0; c < D; ++c) us[c] = *rr.at(st, c);
-    const T h = *rr.at(st, D);
-    issue_r(st - kKin8Ring);  // its slot is free once its values are in registers
+    for (int c = 0; c < D; ++c) us[c] = cp[c * n];
+    const T h = hp[(int64_t)st * n];
     T LU[D * D], R[D], kv[3][D], v[D], un[D], ub[D], vb[D], kb1[D], w[3][D], t[D];
     int P[D];
     if constexpr (METHOD == GS_ROS3)
@@ -199,7 +172,6 @@ __global__ void __launch_bounds__(kKin8Block) k_grad_kin8(RosArgs<T> a) {
       unx[c] = us[c];
     }
   }
-  cp_async_wait<0>();
   if (!ok) {
     L = nan;
 #pragma unroll
@@ -219,11 +191,10 @@ gs_status launch_grad_kin8(const gs_problem* P, const gs_mesh* M, const gs_loss*
   const RosArgs<T> a = ros_args<T>(P, M, Ls, loss, dp, du0, ws);
   const int bs = kKin8Block;
   const unsigned grid = (unsigned)((P->n + bs - 1) / bs);
-  const size_t smem = (size_t)ThreadRing<T, 9, kKin8Ring>::kElems * bs * sizeof(T);
-  auto kern = P->method == GS_ROS3 ? k_grad_kin8<T, GS_ROS3> : k_grad_kin8<T, GS_ROS2>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return GS_ECUDA;
-  kern<<<grid, bs, smem, st>>>(a);
+  if (P->method == GS_ROS3)
+    k_grad_kin8<T, GS_ROS3><<<grid, bs, 0, st>>>(a);
+  else
+    k_grad_kin8<T, GS_ROS2><<<grid, bs, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

@@ -103,7 +103,7 @@ __device__ __forceinline__ void ros2_transpose(const Ros2Step<T>& q, const T p[3
 // iteration before).  The recompute does not depend on lambda, so the two are
 // independent chains in one instruction stream.
 template <typename T, int SYS>
-__global__ void __launch_bounds__(128) k_grad_ros2(RosArgs<T> a) {
+__global__ void __launch_bounds__(GS_ROS_BS, GS_ROS_MINB) k_grad_ros2(RosArgs<T> a) {
   extern __shared__ __align__(16) unsigned char ring_raw[];
   const int64_t n = a.n;
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -194,11 +194,18 @@ __global__ void __launch_bounds__(128) k_grad_ros2(RosArgs<T> a) {
     const bool interior = save_points_rev<T, SYS>(a, i, j, st, p, cur.us, unx, cur.h, kk, next, lam, pb, pg, pn);
     // step st - 1 (step 0 again on the last iteration, whose result is unused:
     // its ring slot still holds step 0, since no later copy targets it)
-    cp_async_wait<kRosRing - 2>();
     Ros2Step<T> nxt;
-    take_r(st > 0 ? st - 1 : 0, nxt);
-    ros2_recompute<T, SYS>(nxt, p);
-    ros2_transpose<T, SYS>(cur, p, lam, pb);
+    if constexpr (GS_ROS_PIPE != 0) {
+      cp_async_wait<kRosRing - 2>();
+      take_r(st > 0 ? st - 1 : 0, nxt);
+      ros2_recompute<T, SYS>(nxt, p);
+      ros2_transpose<T, SYS>(cur, p, lam, pb);
+    } else {  // one step at a time: transpose st, then load and recompute st - 1
+      ros2_transpose<T, SYS>(cur, p, lam, pb);
+      cp_async_wait<kRosRing - 2>();
+      take_r(st > 0 ? st - 1 : 0, nxt);
+      ros2_recompute<T, SYS>(nxt, p);
+    }
     if (interior) save_points_rev_finish<T, SYS>(p, cur.us, pg, pn, lam, pb);
 #pragma unroll
     for (int c = 0; c < 3; ++c) unx[c] = cur.us[c];
@@ -223,7 +230,7 @@ template <typename T>
 gs_status launch_grad_ros2(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp, void* du0,
                            void* ws, cudaStream_t st) {
   const RosArgs<T> a = ros_args<T>(P, M, Ls, loss, dp, du0, ws);
-  const int bs = 128;
+  const int bs = GS_ROS_BS;
   const unsigned grid = (unsigned)((P->n + bs - 1) / bs);
   const size_t smem = (size_t)ThreadRing<T, 4, kRosRing>::kElems * bs * sizeof(T);
   auto kern = P->system == GS_ROBERTSON ? k_grad_ros2<T, GS_ROBERTSON> : k_grad_ros2<T, GS_LORENZ>;

@@ -177,6 +177,21 @@ __device__ __forceinline__ void save_points_rev_finish(const T p[3], const T us[
   for (int c = 0; c < 3; ++c) lam[c] += pg[c];
 }
 
+// Launch shape of the d = 3 Rosenbrock gradient kernels: the pipelined
+// reverse step keeps two recomputed steps live (~150 fp64 registers), and the
+// resident threads per SM must cover an ensemble of 65,536 in one wave
+// (>= 443 per SM): 64-thread blocks, 7 per SM, at most 144 registers.
+#ifndef GS_ROS_BS
+#define GS_ROS_BS 64
+#endif
+#ifndef GS_ROS_MINB
+#define GS_ROS_MINB 7
+#endif
+// 1: the reverse step of s overlaps the recompute of s - 1 (software pipeline)
+#ifndef GS_ROS_PIPE
+#define GS_ROS_PIPE 1
+#endif
+
 // Per-thread copy ring in dynamic shared memory: ROWS values per step for
 // DEPTH steps (a power of two).  Value r of step s of a thread lives at
 // base[((s % DEPTH) * ROWS + r) * blockDim.x], so consecutive threads touch

@@ -21,6 +21,12 @@
 // (ros2_fwd / ros3_fwd), so the loss is bitwise that of gs_solve / gs_grad,
 // and the tangent solves reuse its LU factors.
 //
+// Dense save points (theta in (0, 1) inside a step): the state there is the
+// cubic Hermite interpolant of the step on u_s, u_{s+1} and f at both ends,
+// theta and h data; its tangent is the same combination of the end tangents
+// and of df = J(u) du + f_p(u) w at both ends, evaluated on the steps that
+// hold such a save point.
+//
 // Execution: one thread per (slot, direction); the six directions of a slot
 // run in the six blocks of one range of 128 slots (block b: slots
 // 128 (b / 6) .., direction b % 6), which read the same mesh lines through
@@ -47,6 +53,7 @@ struct RosSensArgs {
   T* dp;            // [3][n]
   T* du0;           // [3][n]
   T* sens;          // [nsave][3][6][n], may be null
+  const T* theta;   // [nsave][n] by slot: dense save points, or null
 };
 
 // df = J(x) dx + f_p(x) w.
@@ -86,7 +93,7 @@ __device__ __forceinline__ void djk3(const T u[3], const T p[3], const T v[3], c
   }
 }
 
-template <typename T, int SYS, int METHOD>
+template <typename T, int SYS, int METHOD, bool DENSE>
 __global__ void __launch_bounds__(128) k_sens_ros(RosSensArgs<T> a) {
   const int64_t n = a.n;
   const int64_t j = (int64_t)(blockIdx.x / 6) * blockDim.x + threadIdx.x;
@@ -168,28 +175,51 @@ __global__ void __launch_bounds__(128) k_sens_ros(RosSensArgs<T> a) {
 #pragma unroll
       for (int c = 0; c < 3; ++c) dun[c] = fmaT(h, fmaT(cst<T>(0.5), dk2[c], cst<T>(1.5) * dk1[c]), v[c]);
     }
+    // save points of this step (a landing record: at most one, at its end)
+    bool slopes = false;
+    T fs[3], fn[3], dfs[3], dfn[3];
+    while (st + 1 == next) {
+      T ut[3] = {un[0], un[1], un[2]}, vt[3] = {dun[0], dun[1], dun[2]};
+      if (DENSE) {
+        const T th = a.theta[(int64_t)kk * n + j];
+        if (th != cst<T>(1.0)) {
+          if (!slopes) {
+            rhs3<T, SYS>(u, p, fs);
+            rhs3<T, SYS>(un, p, fn);
+            jvp3<T, SYS>(u, p, v, w, dfs);
+            jvp3<T, SYS>(un, p, dun, w, dfn);
+            slopes = true;
+          }
+          const HermiteW<T> hw = hermite_w(th);
 #pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      u[c] = un[c];
-      v[c] = dun[c];
-    }
-    if (st + 1 == next) {
+          for (int c = 0; c < 3; ++c) {
+            ut[c] = hermite_c(hw, u[c], un[c], fs[c], fn[c], h);
+            vt[c] = hermite_c(hw, v[c], dun[c], dfs[c], dfn[c], h);
+          }
+        }
+      }
       const int64_t o = (int64_t)kk * n3 + i;
 #pragma unroll
       for (int c = 0; c < 3; ++c) {
         if (a.loss_kind == GS_LOSS_SUMSQ) {
-          const T e = a.target ? u[c] - a.target[o + c * n] : u[c];
+          const T e = a.target ? ut[c] - a.target[o + c * n] : ut[c];
           L = fmaT(e, e, L);
-          dL = fmaT(cst<T>(2.0) * e, v[c], dL);
+          dL = fmaT(cst<T>(2.0) * e, vt[c], dL);
         } else {
           const T wc = a.weight[o + c * n];
-          L = fmaT(wc, u[c], L);
-          dL = fmaT(wc, v[c], dL);
+          L = fmaT(wc, ut[c], L);
+          dL = fmaT(wc, vt[c], dL);
         }
-        if (a.sens) a.sens[(((int64_t)kk * 3 + c) * 6 + dq) * n + i] = v[c];
+        if (a.sens) a.sens[(((int64_t)kk * 3 + c) * 6 + dq) * n + i] = vt[c];
       }
       ++kk;
       next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
+      if (!DENSE) break;
+    }
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      u[c] = un[c];
+      v[c] = dun[c];
     }
   }
   if (!ok) {
@@ -221,19 +251,14 @@ gs_status launch_sens_ros(const gs_problem* P, const gs_mesh* M, const gs_loss* 
   a.dp = (T*)dp;
   a.du0 = (T*)du0;
   a.sens = (T*)sens;
+  a.theta = (const T*)M->save_theta;
   const unsigned grid = (unsigned)((P->n + 127) / 128 * 6);
-  const bool rob = P->system == GS_ROBERTSON;
-  if (P->method == GS_ROS3) {
-    if (rob)
-      k_sens_ros<T, GS_ROBERTSON, GS_ROS3><<<grid, 128, 0, st>>>(a);
-    else
-      k_sens_ros<T, GS_LORENZ, GS_ROS3><<<grid, 128, 0, st>>>(a);
-  } else {
-    if (rob)
-      k_sens_ros<T, GS_ROBERTSON, GS_ROS2><<<grid, 128, 0, st>>>(a);
-    else
-      k_sens_ros<T, GS_LORENZ, GS_ROS2><<<grid, 128, 0, st>>>(a);
-  }
+  const bool rob = P->system == GS_ROBERTSON, ros3 = P->method == GS_ROS3, dense = a.theta != nullptr;
+  auto kern = rob ? (ros3 ? (dense ? k_sens_ros<T, GS_ROBERTSON, GS_ROS3, true> : k_sens_ros<T, GS_ROBERTSON, GS_ROS3, false>)
+                          : (dense ? k_sens_ros<T, GS_ROBERTSON, GS_ROS2, true> : k_sens_ros<T, GS_ROBERTSON, GS_ROS2, false>))
+                  : (ros3 ? (dense ? k_sens_ros<T, GS_LORENZ, GS_ROS3, true> : k_sens_ros<T, GS_LORENZ, GS_ROS3, false>)
+                          : (dense ? k_sens_ros<T, GS_LORENZ, GS_ROS2, true> : k_sens_ros<T, GS_LORENZ, GS_ROS2, false>));
+  kern<<<grid, 128, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

@@ -14,6 +14,13 @@
 //   v' = v + h sum_j b_j dk_j,
 // with dk_1 carried over from the previous step (FSAL, as k_1).
 //
+// Dense save points (a dense record: theta in (0, 1) inside a step): the
+// state there is the cubic Hermite interpolant of the step,
+//   u(theta) = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
+// theta and h data, so its tangent is the same combination of the end
+// tangents and the tangent slopes dk_1 of both ends, all of which the replay
+// holds (FSAL).
+//
 // Execution: one thread per (slot, NDIR directions).  The six directions of a
 // slot run in 6 / NDIR threads, each of which replays the state itself: the
 // state costs 192 flop a step against 252 per direction, and holding all six
@@ -24,6 +31,7 @@
 // of the step-major mesh, and the G blocks of a range run side by side and
 // share those lines through L2 (the mesh crosses HBM once, not G times).  No
 // workspace: nothing is stored but the save-point sensitivities.
+#include "steps.cuh"
 #include "vec.cuh"
 
 namespace gs {
@@ -52,6 +60,7 @@ struct SensArgs {
   T* dp;            // [3][n]
   T* du0;           // [3][n]
   T* sens;          // [nsave][3][6][n], may be null
+  const T* theta;   // [nsave][n] by slot: dense save points, or null
 };
 
 // J(u) v + f_p(u) w for f = (s (y - x), x (r - z) - y, x y - b z).
@@ -89,7 +98,7 @@ __device__ __forceinline__ void lorenz_jvp(T x, T y, T z, T s, T r, T b, const V
   lorenz_f(Ux, Uy, Uz, s, r, b, KN##x, KN##y, KN##z);                 \
   lorenz_jvp(Ux, Uy, Uz, s, r, b, dUx, dUy, dUz, ws, wr, wb, d##KN##x, d##KN##y, d##KN##z);
 
-template <typename T, int NDIR>
+template <typename T, int NDIR, bool DENSE>
 __global__ void __launch_bounds__(128, GS_SENS_MINB) k_sens_tsit5_lorenz(SensArgs<T> a) {
   using V = vec<T, NDIR>;
   const int64_t n = a.n;
@@ -166,6 +175,13 @@ __global__ void __launch_bounds__(128, GS_SENS_MINB) k_sens_tsit5_lorenz(SensArg
     GS_S_ACCN(kTsA64, k4)
     GS_S_ACCN(kTsA65, k5)
     GS_S_STAGE(k6)
+    // dense save points: u_s, f(u_s) and their tangents
+    T xs, ys, zs, fsx, fsy, fsz;
+    V vsx, vsy, vsz, dfsx, dfsy, dfsz;
+    if (DENSE) {
+      xs = x, ys = y, zs = z, fsx = k1x, fsy = k1y, fsz = k1z;
+      vsx = vx, vsy = vy, vsz = vz, dfsx = dk1x, dfsy = dk1y, dfsz = dk1z;
+    }
     // u_{s+1} and its tangent
     GS_S_ACC1(kTsB1, k1)
     GS_S_ACCN(kTsB2, k2)
@@ -181,38 +197,57 @@ __global__ void __launch_bounds__(128, GS_SENS_MINB) k_sens_tsit5_lorenz(SensArg
     vz = fmaT(h, daz, vz);
     lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);  // FSAL
     lorenz_jvp(x, y, z, s, r, b, vx, vy, vz, ws, wr, wb, dk1x, dk1y, dk1z);
-    if (st + 1 == next) {
+    // a landing record has at most one save point per step; a dense one any number
+    while (st + 1 == next) {
+      T ux = x, uy = y, uz = z;
+      V tx = vx, ty = vy, tz = vz;
+      if (DENSE) {
+        const T th = a.theta[(int64_t)kk * n + j];
+        if (th != cst<T>(1.0)) {
+          const HermiteW<T> w = hermite_w(th);
+          ux = hermite_c(w, xs, x, fsx, k1x, h);
+          uy = hermite_c(w, ys, y, fsy, k1y, h);
+          uz = hermite_c(w, zs, z, fsz, k1z, h);
+#pragma unroll
+          for (int q = 0; q < NDIR; ++q) {
+            tx.e[q] = hermite_c(w, vsx.e[q], vx.e[q], dfsx.e[q], dk1x.e[q], h);
+            ty.e[q] = hermite_c(w, vsy.e[q], vy.e[q], dfsy.e[q], dk1y.e[q], h);
+            tz.e[q] = hermite_c(w, vsz.e[q], vz.e[q], dfsz.e[q], dk1z.e[q], h);
+          }
+        }
+      }
       const int64_t o = (int64_t)kk * n3 + i;
       if (a.loss_kind == GS_LOSS_SUMSQ) {
-        const T ex = a.target ? x - a.target[o] : x;
-        const T ey = a.target ? y - a.target[o + n] : y;
-        const T ez = a.target ? z - a.target[o + 2 * n] : z;
+        const T ex = a.target ? ux - a.target[o] : ux;
+        const T ey = a.target ? uy - a.target[o + n] : uy;
+        const T ez = a.target ? uz - a.target[o + 2 * n] : uz;
         L = fmaT(ex, ex, L);
         L = fmaT(ey, ey, L);
         L = fmaT(ez, ez, L);
-        dL = fmaT(cst<T>(2.0) * ex, vx, dL);
-        dL = fmaT(cst<T>(2.0) * ey, vy, dL);
-        dL = fmaT(cst<T>(2.0) * ez, vz, dL);
+        dL = fmaT(cst<T>(2.0) * ex, tx, dL);
+        dL = fmaT(cst<T>(2.0) * ey, ty, dL);
+        dL = fmaT(cst<T>(2.0) * ez, tz, dL);
       } else {
         const T w0 = a.weight[o], w1 = a.weight[o + n], w2 = a.weight[o + 2 * n];
-        L = fmaT(w0, x, L);
-        L = fmaT(w1, y, L);
-        L = fmaT(w2, z, L);
-        dL = fmaT(w0, vx, dL);
-        dL = fmaT(w1, vy, dL);
-        dL = fmaT(w2, vz, dL);
+        L = fmaT(w0, ux, L);
+        L = fmaT(w1, uy, L);
+        L = fmaT(w2, uz, L);
+        dL = fmaT(w0, tx, dL);
+        dL = fmaT(w1, ty, dL);
+        dL = fmaT(w2, tz, dL);
       }
       if (a.sens) {
 #pragma unroll
         for (int q = 0; q < NDIR; ++q) {
           T* o6 = a.sens + ((int64_t)kk * 18 + dir0 + q) * n + i;
-          o6[0] = vx.e[q];
-          o6[6 * n] = vy.e[q];
-          o6[12 * n] = vz.e[q];
+          o6[0] = tx.e[q];
+          o6[6 * n] = ty.e[q];
+          o6[12 * n] = tz.e[q];
         }
       }
       ++kk;
       next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
+      if (!DENSE) break;
     }
   }
   if (dir0 == 0) a.loss[i] = L;
@@ -248,10 +283,14 @@ gs_status launch_sens_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const 
   a.dp = (T*)dp;
   a.du0 = (T*)du0;
   a.sens = (T*)sens;
+  a.theta = (const T*)M->save_theta;
   constexpr int ND = GS_SENS_NDIR;
   static_assert(6 % ND == 0, "directions per thread must divide 6");
   const int64_t grid = (P->n + 127) / 128 * (6 / ND);
-  k_sens_tsit5_lorenz<T, ND><<<(unsigned)grid, 128, 0, st>>>(a);
+  if (a.theta)
+    k_sens_tsit5_lorenz<T, ND, true><<<(unsigned)grid, 128, 0, st>>>(a);
+  else
+    k_sens_tsit5_lorenz<T, ND, false><<<(unsigned)grid, 128, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

@@ -1,6 +1,8 @@
 """Helpers for the GPU tests: move a workloads.Problem to the device, carry an
 oracle mesh into the library's slot layout, and read a device mesh back in
 trajectory order.  Marshalling only."""
+import dataclasses
+
 import numpy as np
 import torch
 
@@ -127,4 +129,42 @@ def parity(out, prob, om, tol=None, c=ROUTE_FACTOR, dual=True):
         w = int(np.argmax(e / bound))
         assert (e <= bound).all(), (f"{int((e > bound).sum())} of {len(e)} trajectories over the gate; worst {w}: "
                                     f"error {e[w]:.3e}, oracle routes {kappa[w]:.3e}, bound {bound[w]:.3e}")
+    return e
+
+
+def sens_wide(prob, om, mode="tape_wide"):
+    """The sensitivity matrices [nsave][d][np + d][n] from the oracle's tape
+    (by default with a wide reverse sweep): one linear loss per (save point,
+    component) whose weight selects that entry (d = 3 systems)."""
+    K = len(prob.tsave)
+    S = np.zeros((K, 3, 6, prob.n))
+    import oracle
+    for k in range(K):
+        for c in range(3):
+            w = np.zeros((K, 3, prob.n))
+            w[k, c] = 1.0
+            q = dataclasses.replace(prob, loss="linear", weight=w, target=None)
+            g = oracle.grad(q, om, mode=mode)
+            S[k, c, :3], S[k, c, 3:] = g["dp"], g["du0"]
+    return S
+
+
+def sens_rel(a, ref):
+    """Per trajectory: the largest entry error over the largest entry."""
+    return np.abs(a - ref).max(axis=(0, 1, 2)) / np.abs(ref).max(axis=(0, 1, 2))
+
+
+def sens_parity(S, prob, om, tol, c=ROUTE_FACTOR):
+    """The gradient criterion applied to the matrices, per trajectory: every
+    trajectory within max(tol, c kappa_i), kappa_i the largest error of the
+    oracle's own plain-precision routes (dual numbers, the tape, the tape
+    with fused updates) on it against the wide reference."""
+    import oracle
+    ref = sens_wide(prob, om)
+    e = sens_rel(S, ref)
+    kappa = np.maximum.reduce([sens_rel(oracle.sens(prob, om), ref), sens_rel(sens_wide(prob, om, "tape"), ref),
+                               sens_rel(sens_wide(prob, om, "tape_fused"), ref)])
+    bound = np.maximum(tol, c * kappa)
+    w = int(np.argmax(e / bound))
+    assert (e <= bound).all(), (int((e > bound).sum()), w, e[w], kappa[w])
     return e

@@ -182,10 +182,10 @@ def test_set_option_host_only():
 
 @hidden_only
 def test_ros3_method_validation_host_only(no_launch):
-    """ROS3 (method 3) is accepted for the d = 3 systems, dense records
-    included, and refused where it is not built: sensitivities on dense
-    meshes; an unknown method is an invalid argument.  No call here reaches a
-    launch (the dense record is checked on an empty ensemble)."""
+    """ROS3 (method 3) is accepted for the d = 3 systems, dense records and
+    sensitivities on dense meshes included; an unknown method is an invalid
+    argument.  No call here reaches a launch (the dense paths are checked on
+    an empty ensemble)."""
     from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
     m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
     ls = _Loss(1, None, None)
@@ -194,12 +194,11 @@ def test_ros3_method_validation_host_only(no_launch):
         assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 1) == 100 * 3 * 1000 * 8
         md = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
         md.save_theta = 16
-        assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(md), ctypes.byref(ls), ctypes.c_void_p(16),
-                            ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == -4
         dense = _Tol(1e-6, 1e-6, 0.0)
         dense.dense = 1
         e = _host_problem(n=0, system=system, method=3)
         assert _lib.gs_count(ctypes.byref(e), ctypes.byref(dense), 100, None, None, None) == 0
+        assert _lib.gs_sens(ctypes.byref(e), ctypes.byref(md), ctypes.byref(ls), None, None, None, None, None) == 0
         assert _lib.gs_count(ctypes.byref(e), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, None, None, None) == 0
     bad = _host_problem(method=4)
     assert _lib.gs_count(ctypes.byref(bad), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, ctypes.c_void_p(16), None,

@@ -11,7 +11,7 @@ import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
 from gpu_util import (TOL, dev, ensemble, loss_args, mesh_by_trajectory, mesh_from_oracle, mesh_rel_err, parity,
-                      theta_by_trajectory)
+                      sens_parity, theta_by_trajectory)
 
 pytestmark = pytest.mark.gpu
 
@@ -97,11 +97,23 @@ def test_dense_linear_loss_and_own_mesh(case):
     parity(out, prob, om)
 
 
-def test_dense_unsupported_paths(case):
+def test_dense_sensitivities(case):
+    """Forward sensitivities on the dense mesh: at each save point the tangent
+    of the Hermite interpolant, against the oracle's dual numbers on the same
+    mesh, and the loss gradient equal to the adjoint's."""
     prob, om = case
-    mesh = mesh_from_oracle(om, "f64")
-    with pytest.raises(gs.gradsolve.GradsolveError):
-        gs.gs_sens(ensemble(prob), mesh, **loss_args(prob))
+    sub = prob.subset(np.arange(256))
+    osub = oracle.Mesh(om.h[:256], om.nsteps[:256], om.save_idx[:256], om.status[:256], om.nreject[:256],
+                       om.theta[:256])
+    out, S = gs.gs_sens(ensemble(sub), mesh_from_oracle(osub, "f64"), **loss_args(sub))
+    torch.cuda.synchronize()
+    sens_parity(S.double().cpu().numpy(), sub, osub, TOL["f64"])
+    parity(out, sub, osub)
+    loss, _ = oracle.replay(sub, osub)
+    assert np.abs(out.loss.cpu().numpy() - loss).max() <= 1e-14 * np.abs(loss).max()
+
+
+def test_dense_unsupported_paths(case):
     k8 = W.kin8(4)  # dense records are built for the d = 3 systems
     with pytest.raises(gs.gradsolve.GradsolveError):
         gs.gs_count(ensemble(k8), k8.rtol, k8.atol, 100, dense=True)

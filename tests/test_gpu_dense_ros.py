@@ -12,7 +12,7 @@ import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
 from gpu_util import (TOL, dev, ensemble, loss_args, mesh_by_trajectory, mesh_from_oracle, mesh_rel_err, parity,
-                      theta_by_trajectory)
+                      sens_parity, theta_by_trajectory)
 
 pytestmark = pytest.mark.gpu
 
@@ -107,6 +107,22 @@ def test_dense_gradient_fp32(system, method):
     sub = np.flatnonzero(ok)
     parity(gs.GradOut(out.loss[sub], out.dp[:, sub], out.du0[:, sub], None), prob.subset(sub),
            _sub_mesh(om, sub), tol=TOL["f32"])
+
+
+def test_dense_sensitivities(case):
+    """Forward sensitivities on the dense mesh: at each save point the tangent
+    of the Hermite interpolant (f and its Jacobian-vector product at both
+    step ends), against the oracle's wide-tape matrices, and the loss
+    gradient by forward mode against the adjoint's parity."""
+    prob, om, _ = case
+    idx = np.arange(40)
+    sub, osub = prob.subset(idx), _sub_mesh(om, idx)
+    out, S = gs.gs_sens(ensemble(sub), mesh_from_oracle(osub, "f64"), **loss_args(sub))
+    torch.cuda.synchronize()
+    sens_parity(S.double().cpu().numpy(), sub, osub, TOL["f64"])
+    parity(out, sub, osub)
+    loss, _ = oracle.replay(sub, osub)
+    assert np.abs(out.loss.cpu().numpy() - loss).max() <= 1e-14 * np.abs(loss).max()
 
 
 def _sub_mesh(om, idx):

@@ -3,8 +3,6 @@ the sensitivity matrices d u(t_k) / d (p, u0) against the oracle, the loss
 gradient against the adjoint (the same derivative by the other mode), fp64 and
 fp32, failures, ragged sizes and the full 2**20-trajectory ensemble on a
 sample."""
-import dataclasses
-
 import numpy as np
 import pytest
 import torch
@@ -12,45 +10,9 @@ import torch
 import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
-from gpu_util import ROUTE_FACTOR, TOL, dev, ensemble, loss_args, mesh_from_oracle, parity
+from gpu_util import TOL, dev, ensemble, loss_args, mesh_from_oracle, parity, sens_parity, sens_rel
 
 pytestmark = pytest.mark.gpu
-
-
-def _sens_wide(prob, om, mode="tape_wide"):
-    """Rows of S from the oracle's tape (by default with a wide reverse
-    sweep): one linear loss per (save point, component) whose weight selects
-    that entry."""
-    K = len(prob.tsave)
-    S = np.zeros((K, 3, 6, prob.n))
-    for k in range(K):
-        for c in range(3):
-            w = np.zeros((K, 3, prob.n))
-            w[k, c] = 1.0
-            q = dataclasses.replace(prob, loss="linear", weight=w, target=None)
-            g = oracle.grad(q, om, mode=mode)
-            S[k, c, :3], S[k, c, 3:] = g["dp"], g["du0"]
-    return S
-
-
-def _rel(a, ref):
-    """Per trajectory: largest entry error over the largest entry."""
-    return np.abs(a - ref).max(axis=(0, 1, 2)) / np.abs(ref).max(axis=(0, 1, 2))
-
-
-def _sens_parity(S, prob, om, tol):
-    """The gradient criterion applied to the matrices, per trajectory: every
-    trajectory within max(tol, c kappa_i), kappa_i the largest error of the
-    oracle's own plain-precision routes (dual numbers, the tape, the tape
-    with fused updates) on it against the wide reference."""
-    ref = _sens_wide(prob, om)
-    e = _rel(S, ref)
-    kappa = np.maximum.reduce([_rel(oracle.sens(prob, om), ref), _rel(_sens_wide(prob, om, "tape"), ref),
-                               _rel(_sens_wide(prob, om, "tape_fused"), ref)])
-    bound = np.maximum(tol, ROUTE_FACTOR * kappa)
-    w = int(np.argmax(e / bound))
-    assert (e <= bound).all(), (int((e > bound).sum()), w, e[w], kappa[w])
-    return e
 
 
 def _run(prob, om, sens=True):
@@ -63,10 +25,10 @@ def test_small_fp64():
     prob = W.lorenz_small(1024)
     om = oracle.record(prob, 256)
     out, S = _run(prob, om)
-    e = _rel(S, oracle.sens(prob, om))
+    e = sens_rel(S, oracle.sens(prob, om))
     assert e.max() <= 1e-12, e.max()
     sub = prob.subset(np.arange(64))
-    _sens_parity(S[..., :64], sub, oracle.record(sub, 256), 1e-12)
+    sens_parity(S[..., :64], sub, oracle.record(sub, 256), 1e-12)
     loss, _ = oracle.replay(prob, om)
     assert np.abs(out.loss.cpu().numpy() - loss).max() <= 1e-14 * np.abs(loss).max()
     parity(out, prob, om)
@@ -78,7 +40,7 @@ def test_ten_save_points(dtype):
     prob = W.lorenz_1m(300, dtype=dtype)
     om = oracle.record(prob, 1024)
     out, S = _run(prob, om)
-    _sens_parity(S, prob, om, TOL[dtype])
+    sens_parity(S, prob, om, TOL[dtype])
     parity(out, prob, om)
 
 
@@ -108,7 +70,7 @@ def test_failures_ragged_and_unsupported():
     assert np.isnan(S[..., [0, 77]]).all() and np.isfinite(np.delete(S, [0, 77], axis=3)).all()
     assert torch.isnan(out.loss[[0, 77]]).all() and torch.isnan(out.dp[:, [0, 77]]).all()
     ok = np.delete(np.arange(prob.n), [0, 77])
-    assert _rel(np.delete(S, [0, 77], axis=3), oracle.sens(prob, om)[..., ok]).max() <= 1e-12
+    assert sens_rel(np.delete(S, [0, 77], axis=3), oracle.sens(prob, om)[..., ok]).max() <= 1e-12
     out2, none = _run(prob, om, sens=False)
     assert none is None and torch.equal(out2.dp[:, 1:77], out.dp[:, 1:77])
     rob = W.robertson(4)  # Tsit5 forward sensitivities are built for Lorenz only
@@ -135,5 +97,5 @@ def test_full_size_sampled():
     sub = prob.subset(idx)
     om = oracle.record(sub, 2048)  # equal to the GPU's mesh for these trajectories
     got = S[..., torch.tensor(idx, device=dev())].cpu().numpy()
-    _sens_parity(got, sub, om, 1e-12)
+    sens_parity(got, sub, om, 1e-12)
     assert torch.isfinite(S).all()
