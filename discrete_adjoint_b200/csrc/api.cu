@@ -44,7 +44,7 @@ gs_status node64_grad(const gs_problem*, const gs_mesh*, const gs_loss*, void*, 
 gs_status node64_solve(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 void node64_set_tensor(int on);
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize);
-int grad_tsit5_lorenz_ck_rows(int32_t dtype);
+size_t grad_tsit5_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave);
 
 static size_t dsize(const gs_problem* P) { return P->dtype == GS_F64 ? 8 : 4; }
 
@@ -134,11 +134,11 @@ size_t gs_workspace_bytes(const gs_problem* P, const gs_mesh* M, int32_t op) {
   if (op == GS_OP_RECORD) return record_ws_bytes(P->n, M->smax, P->nsave, dsize(P));
   if (op == GS_OP_GRAD) {
     if (P->system == GS_NODE64) return node64_grad_ws_bytes(P->n, M->smax, dsize(P));
-    // one checkpointed state per step and slot (the Tsit5 Lorenz kernel may
-    // keep a stage state beside it)
-    const size_t rows = (P->method == GS_TSIT5 && P->system == GS_LORENZ) ? (size_t)grad_tsit5_lorenz_ck_rows(P->dtype)
-                                                                           : (size_t)P->d;
-    return (size_t)M->smax * rows * (size_t)P->n * dsize(P);
+    // one checkpointed state per step and slot (the Tsit5 Lorenz kernel adds
+    // the save points' loss gradients)
+    if (P->method == GS_TSIT5 && P->system == GS_LORENZ)
+      return grad_tsit5_lorenz_ws_bytes(P->dtype, P->n, M->smax, P->nsave);
+    return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
   }
   return 0;
 }

@@ -110,6 +110,7 @@ struct TsitLorenzArgs {
   T* dp;            // [3][n]
   T* du0;           // [3][n]
   T* ck;            // workspace [smax][ck_rows][n] by slot
+  T* gsave;         // workspace tail [nsave][3][n] by slot: landing save points' loss gradients
   const T* theta;   // [nsave][n] by slot: dense save points, or null
 };
 
@@ -324,8 +325,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     z = fmaT(h, az, z);
     lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);  // FSAL: next step's first slope
 #pragma unroll
-    for (int q = 0; q < K; ++q) {
-      // a landing record has at most one save point per step; a dense one any number
+    for (int q = 0; q < K && DENSE; ++q) {
+      // dense save points (any number per step); a landing record's are
+      // summed after the forward half
       while (st + 1 == next[q]) {
         T ux = x.e[q], uy = y.e[q], uz = z.e[q];
         if (DENSE) {
@@ -355,12 +357,76 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
         next[q] = next2[q];
         next2[q] = sp_idx(q, kk[q] + 1);
         sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
-        if (!DENSE) break;
       }
     }
     issue_f(st + kRingF);  // into the row that step st has left
   }
   cp_async_wait<0>();  // the reverse reuses the rows
+  // Landing save points: u(t_k) is the checkpoint of step save_idx[k] (or the
+  // final state), so every lane sums its loss here at once, in the contract's
+  // order (save points, then components), instead of one lane at a time
+  // inside the step loop.  The loss gradient at each save point (2 (u - target)
+  // or the weights) goes to the workspace for the reverse half.  Save points
+  // are taken while their step counts increase within [1, S]; nvalid[q] counts
+  // them (all of them for a well-formed mesh).
+  int nvalid[K];
+#pragma unroll
+  for (int q = 0; q < K; ++q) nvalid[q] = 0;
+  if constexpr (!DENSE) {
+    int prev[K];
+    bool alive[K];
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      prev[q] = 0;
+      alive[q] = S[q] > 0;
+    }
+    for (int k = 0; k < a.nsave; ++k) {
+#pragma unroll
+      for (int q = 0; q < K; ++q) {
+        if (!alive[q]) continue;
+        const int sk = a.save_idx[(int64_t)k * n + j0 + q];
+        if (!(sk > prev[q] && sk <= S[q])) {
+          alive[q] = false;
+          continue;
+        }
+        prev[q] = sk;
+        T ux = x.e[q], uy = y.e[q], uz = z.e[q];
+        if (sk < S[q]) {
+          const T* c = a.ck + (int64_t)sk * nck + j0 + q;
+          ux = c[0];
+          uy = c[n];
+          uz = c[2 * n];
+        }
+        T v0, v1, v2, g0, g1, g2;
+        sp_vec(q, k, v0, v1, v2);
+        T Lq = L.e[q];
+        if (a.loss_kind == GS_LOSS_SUMSQ) {  // u - 0 = u bitwise when there is no target
+          const T dx = ux - v0;
+          const T dy = uy - v1;
+          const T dz = uz - v2;
+          Lq = fmaT(dx, dx, Lq);
+          Lq = fmaT(dy, dy, Lq);
+          Lq = fmaT(dz, dz, Lq);
+          g0 = cst<T>(2.0) * dx;
+          g1 = cst<T>(2.0) * dy;
+          g2 = cst<T>(2.0) * dz;
+        } else {
+          Lq = fmaT(v0, ux, Lq);
+          Lq = fmaT(v1, uy, Lq);
+          Lq = fmaT(v2, uz, Lq);
+          g0 = v0;
+          g1 = v1;
+          g2 = v2;
+        }
+        L.e[q] = Lq;
+        T* G = a.gsave + (int64_t)k * 3 * n + j0 + q;
+        G[0] = g0;
+        G[n] = g1;
+        G[2 * n] = g2;
+        nvalid[q] = k + 1;
+      }
+    }
+  }
 #pragma unroll
   for (int q = 0; q < K; ++q)
     if (i[q] >= 0) a.loss[i[q]] = L.e[q];
@@ -372,12 +438,25 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   // are the prefetched u_st, h_st and U_6 of step st.
   V lx = vsplat<T, K>(cst<T>(0.0)), ly = lx, lz = lx;
   V ps = lx, pr = lx, pb = lx;
+  // a landing save point's loss gradient, from the workspace
+  auto sp_g = [&](int q, int k, T& v0, T& v1, T& v2) {
+    v0 = v1 = v2 = cst<T>(0.0);
+    if (k >= 0 && k < nvalid[q]) {
+      const T* G = a.gsave + (int64_t)k * 3 * n + j0 + q;
+      v0 = G[0];
+      v1 = G[n];
+      v2 = G[2 * n];
+    }
+  };
 #pragma unroll
   for (int q = 0; q < K; ++q) {  // save points in reverse, read one ahead as in the forward
-    kk[q] = a.nsave - 1;
+    kk[q] = DENSE ? a.nsave - 1 : nvalid[q] - 1;
     next[q] = sp_idx(q, kk[q]);
     next2[q] = sp_idx(q, kk[q] - 1);
-    sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
+    if (DENSE)
+      sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
+    else
+      sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
   }
   V cx = x, cy = y, cz = z, hc = vsplat<T, K>(cst<T>(0.0));
   V gx6 = x, gy6 = y, gz6 = z;
@@ -447,8 +526,8 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
             uz = hermite_c(w, cz.e[q], z.e[q], fsz, fnz, hh);
           }
         }
-        T gx, gy, gz;  // d loss_k / d u(t_k)
-        if (a.loss_kind == GS_LOSS_SUMSQ) {
+        T gx, gy, gz;  // d loss_k / d u(t_k): computed here (dense) or by the forward half (landing)
+        if (DENSE && a.loss_kind == GS_LOSS_SUMSQ) {
           gx = cst<T>(2.0) * (ux - tv0[q]);
           gy = cst<T>(2.0) * (uy - tv1[q]);
           gz = cst<T>(2.0) * (uz - tv2[q]);
@@ -479,7 +558,10 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
         --kk[q];
         next[q] = next2[q];
         next2[q] = sp_idx(q, kk[q] - 1);
-        sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
+        if (DENSE)
+          sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
+        else
+          sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
         if (!DENSE) break;
       }
     }
@@ -604,9 +686,13 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #undef GS_ACCN
 #undef GS_C
 
-// Checkpoint rows per step and slot of the gradient workspace (3, or 6 when
-// U_6 is kept), for gs_workspace_bytes.
-int grad_tsit5_lorenz_ck_rows(int32_t dtype) { return dtype == GS_F64 ? ck_rows<double>() : ck_rows<float>(); }
+// Gradient workspace: checkpoint rows per step and slot (3, or 6 when U_6 is
+// kept), then [nsave][3][n] loss gradients of the landing save points.
+size_t grad_tsit5_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave) {
+  const size_t rows = dtype == GS_F64 ? ck_rows<double>() : ck_rows<float>();
+  const size_t tsize = dtype == GS_F64 ? 8 : 4;
+  return ((size_t)smax * rows + (size_t)nsave * 3) * (size_t)n * tsize;
+}
 
 template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void* loss, void* dp,
@@ -629,6 +715,7 @@ gs_status launch_grad_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const 
   a.dp = (T*)dp;
   a.du0 = (T*)du0;
   a.ck = (T*)ws;
+  a.gsave = (T*)ws + (size_t)M->smax * ck_rows<T>() * (size_t)P->n;
   a.theta = (const T*)M->save_theta;
   constexpr int K = GS_GRAD_K;
   const int bs = GS_GRAD_BS;

@@ -182,14 +182,14 @@ __device__ __forceinline__ void save_points_rev_finish(const T p[3], const T us[
 // resident threads per SM must cover an ensemble of 65,536 in one wave
 // (>= 443 per SM): 64-thread blocks, 7 per SM, at most 144 registers.
 #ifndef GS_ROS_BS
-#define GS_ROS_BS 64
+#define GS_ROS_BS 128
 #endif
 #ifndef GS_ROS_MINB
-#define GS_ROS_MINB 7
+#define GS_ROS_MINB 4
 #endif
 // 1: the reverse step of s overlaps the recompute of s - 1 (software pipeline)
 #ifndef GS_ROS_PIPE
-#define GS_ROS_PIPE 1
+#define GS_ROS_PIPE 0
 #endif
 
 // Per-thread copy ring in dynamic shared memory: ROWS values per step for

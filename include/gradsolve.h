@@ -294,8 +294,9 @@ GS_API gs_status gs_sens(const gs_problem* prob, const gs_mesh* mesh, const gs_l
  * checkpoints go to a library-owned device array of GS_STATIC_SCRATCH_BYTES
  * (32 MiB), which every GPU that loads the library holds until exit.
  *  - Problems whose gs_grad workspace exceeds GS_STATIC_SCRATCH_BYTES return
- *    GS_EWORKSPACE (d=3, fp64: smax * n <= 1,398,101, e.g. 1,024 trajectories
- *    of up to 1,365 steps).
+ *    GS_EWORKSPACE (d=3, fp64: (smax + nsave) * n <= 1,398,101 for Tsit5 on
+ *    Lorenz, smax * n <= 1,398,101 for the Rosenbrock methods; e.g. 1,024
+ *    trajectories of up to 1,355 steps with 10 save points).
  *  - All calls share the array: calls that overlap on the GPU race.  It keeps
  *    the last call's contents; nothing in it needs clearing between calls.
  *  - Every call looks up the array's device address (cudaGetSymbolAddress)

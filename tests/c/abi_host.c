@@ -43,10 +43,11 @@ int main(void) {
   /* status strings */
   CHECK(1, strcmp(gs_status_string(GS_OK), "ok") == 0);
   CHECK(2, strlen(gs_status_string(GS_EUNSUPPORTED)) > 0);
-  /* workspace: one checkpointed state per step and slot */
-  CHECK(3, gs_workspace_bytes(&p, &m, GS_OP_GRAD) == (size_t)500 * 3 * 1000 * 8);
+  /* workspace: one checkpointed state per step and slot, then (Tsit5 on
+     Lorenz) the loss gradient of each save point */
+  CHECK(3, gs_workspace_bytes(&p, &m, GS_OP_GRAD) == (size_t)(500 * 3 + 2 * 3) * 1000 * 8);
   p.dtype = GS_F32;
-  CHECK(4, gs_workspace_bytes(&p, &m, GS_OP_GRAD) == (size_t)500 * 3 * 1000 * 4);
+  CHECK(4, gs_workspace_bytes(&p, &m, GS_OP_GRAD) == (size_t)(500 * 3 + 2 * 3) * 1000 * 4);
   p.dtype = GS_F64;
   CHECK(5, gs_workspace_bytes(&p, &m, GS_OP_RECORD) >= (size_t)1000 * 4);
   /* kin8: d = np = 8, Rosenbrock only */

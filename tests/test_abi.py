@@ -79,12 +79,13 @@ def test_workspace_sizes_host_only(no_launch):
     from discrete_adjoint_b200.gradsolve import _Mesh, _lib
     p = _host_problem()
     m = _Mesh(500, 10, None, None, None, None, None, None)
-    # one checkpointed state per step and slot
-    assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 1) == 500 * 3 * 1000 * 8
+    # one checkpointed state per step and slot, then (Tsit5 on Lorenz) the
+    # loss gradient of each save point
+    assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 1) == (500 * 3 + 10 * 3) * 1000 * 8
     assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 0) >= 1000 * 4
     assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 7) == 0
     p32 = _host_problem(dtype=1)
-    assert _lib.gs_workspace_bytes(ctypes.byref(p32), ctypes.byref(m), 1) == 500 * 3 * 1000 * 4
+    assert _lib.gs_workspace_bytes(ctypes.byref(p32), ctypes.byref(m), 1) == (500 * 3 + 10 * 3) * 1000 * 4
 
 
 @hidden_only
