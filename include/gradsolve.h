@@ -279,7 +279,8 @@ GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_l
  * turns singular) get NaN everywhere.  Built for GS_LORENZ with GS_TSIT5, and
  * for GS_LORENZ and GS_ROBERTSON with GS_ROS2 or GS_ROS3 (np + d = 6), fp64
  * and fp32, on landing and dense meshes (at a dense save point the matrix is
- * the tangent of the Hermite interpolant); other problems return
+ * the tangent of the Hermite interpolant); for GS_KIN8 with GS_ROS2 or
+ * GS_ROS3 (np + d = 16) on landing meshes; other problems return
  * GS_EUNSUPPORTED.  (The few-parameter forward-sensitivity
  * route that the gptget summary sets beside the adjoint.)
  */

@@ -135,17 +135,17 @@ def parity(out, prob, om, tol=None, c=ROUTE_FACTOR, dual=True):
 def sens_wide(prob, om, mode="tape_wide"):
     """The sensitivity matrices [nsave][d][np + d][n] from the oracle's tape
     (by default with a wide reverse sweep): one linear loss per (save point,
-    component) whose weight selects that entry (d = 3 systems)."""
-    K = len(prob.tsave)
-    S = np.zeros((K, 3, 6, prob.n))
+    component) whose weight selects that entry."""
+    K, d, npar = len(prob.tsave), prob.d, prob.np_
+    S = np.zeros((K, d, npar + d, prob.n))
     import oracle
     for k in range(K):
-        for c in range(3):
-            w = np.zeros((K, 3, prob.n))
+        for c in range(d):
+            w = np.zeros((K, d, prob.n))
             w[k, c] = 1.0
             q = dataclasses.replace(prob, loss="linear", weight=w, target=None)
             g = oracle.grad(q, om, mode=mode)
-            S[k, c, :3], S[k, c, 3:] = g["dp"], g["du0"]
+            S[k, c, :npar], S[k, c, npar:] = g["dp"], g["du0"]
     return S
 
 

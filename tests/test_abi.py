@@ -208,10 +208,11 @@ def test_ros3_method_validation_host_only(no_launch):
 
 @hidden_only
 def test_kin8_validation_host_only(no_launch):
-    """kin8 (system 5, d = np = 8) takes ROS2 / ROS3; Tsit5, forward
-    sensitivities and dense records are not built for it; wrong sizes are
-    invalid.  The gradient workspace is one checkpointed 8-state per step and
-    slot.  No call here reaches a launch."""
+    """kin8 (system 5, d = np = 8) takes ROS2 / ROS3, forward sensitivities
+    included (on landing meshes); Tsit5 and dense records are not built for
+    it; wrong sizes are invalid.  The gradient workspace is one checkpointed
+    8-state per step and slot.  No call here reaches a launch (the accepted
+    sensitivities are checked on an empty ensemble)."""
     from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
     m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
     ls = _Loss(1, None, None)
@@ -220,7 +221,9 @@ def test_kin8_validation_host_only(no_launch):
         p = _host_problem(system=5, method=method)
         p.d = p.np = 8
         assert _lib.gs_workspace_bytes(ctypes.byref(p), ctypes.byref(m), 1) == 100 * 8 * 1000 * 8
-        assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(m), ctypes.byref(ls), ctypes.c_void_p(16),
+        md = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+        md.save_theta = 16
+        assert _lib.gs_sens(ctypes.byref(p), ctypes.byref(md), ctypes.byref(ls), ctypes.c_void_p(16),
                             ctypes.c_void_p(16), ctypes.c_void_p(16), None, None) == -4
         dense = _Tol(1e-7, 1e-7, 0.0)
         dense.dense = 1
@@ -228,6 +231,7 @@ def test_kin8_validation_host_only(no_launch):
         e = _host_problem(n=0, system=5, method=method)
         e.d = e.np = 8
         assert _lib.gs_count(ctypes.byref(e), ctypes.byref(tol), 100, None, None, None) == 0
+        assert _lib.gs_sens(ctypes.byref(e), ctypes.byref(m), ctypes.byref(ls), None, None, None, None, None) == 0
         wrong = _host_problem(system=5, method=method)  # d = np = 3
         assert _lib.gs_count(ctypes.byref(wrong), ctypes.byref(tol), 100, ctypes.c_void_p(16), None, None) == -1
     t5 = _host_problem(system=5, method=1)

@@ -1,8 +1,8 @@
 """GPU <-> oracle parity for the Rosenbrock path at d = 8 (kin8, 8 x 8 LU in
 registers): the recorder (ROS3 and ROS2), the fused replay + reverse sweep,
-the replay and the adaptive solve, fp32, failure statuses, and the full
-262,144-trajectory ensemble in the benchmark's launch configuration on a
-sample."""
+the replay and the adaptive solve, the forward sensitivities (16 directions),
+fp32, failure statuses, and the full 262,144-trajectory ensemble in the
+benchmark's launch configuration on a sample."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +11,7 @@ import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
 from gpu_util import (TOL, dev, ensemble, grad_rel_err, loss_args, mesh_by_trajectory, mesh_from_oracle,
-                      mesh_rel_err, parity)
+                      mesh_rel_err, parity, sens_parity, sens_rel)
 
 pytestmark = pytest.mark.gpu
 
@@ -68,9 +68,8 @@ def test_ros3_grad(k3, perm):
 
 
 def test_ros2_grad():
-    """ROS2 takes ~16,000 steps per trajectory at this tolerance: the gate of
-    the parity helper (the stated 1e-12 for the bulk, the worst within the
-    oracle's own plain-precision routes)."""
+    """ROS2 takes ~16,000 steps per trajectory at this tolerance: the
+    per-trajectory gate of the parity helper."""
     prob = _multi(_kin8(12, "ros2"))
     om = oracle.record(prob, SMAX2)
     assert (om.status == 0).all()
@@ -215,3 +214,36 @@ def test_ros2_fp32():
     out = gs.gs_grad(ens, mesh_from_oracle(om, "f32"), **loss_args(prob))
     torch.cuda.synchronize()
     parity(out, prob, om, tol=TOL["f32"])
+
+
+def test_ros3_sensitivities():
+    """Forward sensitivities along the 16 input directions (eight rate
+    constants, eight initial states) on the oracle's mesh: per trajectory
+    against the wide-tape matrices (the gradient's rule), the loss bitwise
+    that of the replay, and the forward-mode gradient at the adjoint's
+    parity."""
+    prob = _multi(_kin8(40, "ros3"))
+    om = oracle.record(prob, SMAX3)
+    assert (om.status == 0).all()
+    out, S = gs.gs_sens(ensemble(prob), mesh_from_oracle(om, "f64"), **loss_args(prob))
+    torch.cuda.synchronize()
+    assert S.shape == (3, 8, 16, prob.n)
+    sens_parity(S.double().cpu().numpy(), prob, om, TOL["f64"])
+    parity(out, prob, om)
+    loss, _ = oracle.replay(prob, om)
+    assert np.abs(out.loss.cpu().numpy() - loss).max() <= 1e-14 * np.abs(loss).max()
+
+
+def test_ros2_sensitivities():
+    """ROS2 (~16,000 steps per trajectory): the matrices against the oracle's
+    dual numbers on the same mesh within eps per step, the forward-mode
+    gradient at the adjoint's parity."""
+    prob = _multi(_kin8(6, "ros2"))
+    om = oracle.record(prob, SMAX2)
+    assert (om.status == 0).all()
+    out, S = gs.gs_sens(ensemble(prob), mesh_from_oracle(om, "f64"), **loss_args(prob))
+    torch.cuda.synchronize()
+    tol = max(1e-12, 4 * np.finfo(float).eps * int(om.nsteps.max()))
+    e = sens_rel(S.double().cpu().numpy(), oracle.sens(prob, om))
+    assert e.max() <= tol, (e.max(), tol)
+    parity(out, prob, om)
