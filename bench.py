@@ -678,10 +678,25 @@ def run_ours(args):
     done_copy = [torch.cuda.Event(), torch.cuda.Event()]
     done_grad = [torch.cuda.Event(), torch.cuda.Event()]
 
+    # the record needs p, u0 (and W); the targets and weights are needed from
+    # the first gradient pass on, so they cross on the copy stream while the
+    # record runs (after the previous step's passes are done with them)
+    side = [k for k in host if k in ("target", "weight")]
+    side_ready = torch.cuda.Event()
+
     def e2e_step():
         for k, v in host.items():
-            d[k].copy_(v, non_blocking=True)
+            if k not in side:
+                d[k].copy_(v, non_blocking=True)
+        if side:
+            copy_stream.wait_stream(stream)
+            with torch.cuda.stream(copy_stream):
+                for k in side:
+                    d[k].copy_(host[k], non_blocking=True)
+            side_ready.record(copy_stream)
         gs.gs_record(ens, mesh, prob.rtol, prob.atol, ws=ws_rec, stream=stream)
+        if side:
+            stream.wait_event(side_ready)
         for k in range(passes):
             b = k % 2
             o = outs[b]
