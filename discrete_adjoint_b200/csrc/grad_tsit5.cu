@@ -214,12 +214,8 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #pragma unroll
     for (int q = 0; q < K; ++q) hv.e[q] = sf < S[q] ? rg[((sf & (kRingF - 1)) * K + q) * BS] : cst<T>(0.0);
   };
-  // Save points, read one save point ahead: next[q] is the step count at
-  // which slot q's current save point kk[q] falls, (tv0, tv1, tv2)[q] its loss
-  // vector (the target for SUMSQ, zero without one; the weights for LINEAR)
-  // and next2[q] the step count of the save point after it.  Each load is
-  // issued a whole save interval before its value is used, so the divergent
-  // save-point branch never waits on DRAM.
+  // A save point's step count, and its loss vector (the target for SUMSQ,
+  // zero without one; the weights for LINEAR).
   auto sp_idx = [&](int q, int k) -> int {
     return (k >= 0 && k < a.nsave && S[q] > 0) ? a.save_idx[(int64_t)k * n + j0 + q] : -1;
   };
@@ -234,15 +230,6 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     }
   };
   V L = vsplat<T, K>(cst<T>(0.0));
-  int kk[K], next[K], next2[K];
-  T tv0[K], tv1[K], tv2[K];
-#pragma unroll
-  for (int q = 0; q < K; ++q) {
-    kk[q] = 0;
-    next[q] = sp_idx(q, 0);
-    next2[q] = sp_idx(q, 1);
-    sp_vec(q, 0, tv0[q], tv1[q], tv2[q]);
-  }
   V k1x, k1y, k1z;
   lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);
   V hn;
@@ -311,73 +298,32 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     GS_ACCN(kTsB4, k4)
     GS_ACCN(kTsB5, k5)
     GS_ACCN(kTsB6, k6)
-    V xs, ys, zs, fsx, fsy, fsz;  // dense save points: u_s and f(u_s)
-    if (DENSE) {
-      xs = x;
-      ys = y;
-      zs = z;
-      fsx = k1x;
-      fsy = k1y;
-      fsz = k1z;
-    }
     x = fmaT(h, ax, x);
     y = fmaT(h, ay, y);
     z = fmaT(h, az, z);
     lorenz_f(x, y, z, s, r, b, k1x, k1y, k1z);  // FSAL: next step's first slope
-#pragma unroll
-    for (int q = 0; q < K && DENSE; ++q) {
-      // dense save points (any number per step); a landing record's are
-      // summed after the forward half
-      while (st + 1 == next[q]) {
-        T ux = x.e[q], uy = y.e[q], uz = z.e[q];
-        if (DENSE) {
-          const T th = a.theta[(int64_t)kk[q] * n + j0 + q];
-          if (th != cst<T>(1.0)) {
-            const HermiteW<T> w = hermite_w(th);
-            ux = hermite_c(w, xs.e[q], ux, fsx.e[q], k1x.e[q], h.e[q]);
-            uy = hermite_c(w, ys.e[q], uy, fsy.e[q], k1y.e[q], h.e[q]);
-            uz = hermite_c(w, zs.e[q], uz, fsz.e[q], k1z.e[q], h.e[q]);
-          }
-        }
-        T Lq = L.e[q];
-        if (a.loss_kind == GS_LOSS_SUMSQ) {  // u - 0 = u bitwise when there is no target
-          const T dx = ux - tv0[q];
-          const T dy = uy - tv1[q];
-          const T dz = uz - tv2[q];
-          Lq = fmaT(dx, dx, Lq);
-          Lq = fmaT(dy, dy, Lq);
-          Lq = fmaT(dz, dz, Lq);
-        } else {
-          Lq = fmaT(tv0[q], ux, Lq);
-          Lq = fmaT(tv1[q], uy, Lq);
-          Lq = fmaT(tv2[q], uz, Lq);
-        }
-        L.e[q] = Lq;
-        ++kk[q];
-        next[q] = next2[q];
-        next2[q] = sp_idx(q, kk[q] + 1);
-        sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
-      }
-    }
     issue_f(st + kRingF);  // into the row that step st has left
   }
   cp_async_wait<0>();  // the reverse reuses the rows
-  // Landing save points: u(t_k) is the checkpoint of step save_idx[k] (or the
-  // final state), so every lane sums its loss here at once, in the contract's
-  // order (save points, then components), instead of one lane at a time
-  // inside the step loop.  The loss gradient at each save point (2 (u - target)
-  // or the weights) goes to the workspace for the reverse half.  Save points
-  // are taken while their step counts increase within [1, S]; nvalid[q] counts
+  // Save points: u(t_k) is read off the checkpoints -- the state after step
+  // save_idx[k] (the checkpoint of that step, or the final state) for a
+  // landing record, the Hermite interpolant of step save_idx[k] - 1 at theta_k
+  // on its checkpointed ends and their slopes for a dense one -- so every lane
+  // sums its loss here at once, in the contract's order (save points, then
+  // components), instead of one lane at a time inside the step loop; the
+  // values are bitwise those of the step loop.  The loss gradient at each
+  // save point (2 (u - target) or the weights) goes to the workspace for the
+  // reverse half.  Save points are taken while their step counts stay in
+  // [1, S] and increase (landing) or do not decrease (dense); nvalid[q] counts
   // them (all of them for a well-formed mesh).
   int nvalid[K];
-#pragma unroll
-  for (int q = 0; q < K; ++q) nvalid[q] = 0;
-  if constexpr (!DENSE) {
+  {
     int prev[K];
     bool alive[K];
 #pragma unroll
     for (int q = 0; q < K; ++q) {
-      prev[q] = 0;
+      nvalid[q] = 0;
+      prev[q] = DENSE ? 1 : 0;
       alive[q] = S[q] > 0;
     }
     for (int k = 0; k < a.nsave; ++k) {
@@ -385,17 +331,32 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
       for (int q = 0; q < K; ++q) {
         if (!alive[q]) continue;
         const int sk = a.save_idx[(int64_t)k * n + j0 + q];
-        if (!(sk > prev[q] && sk <= S[q])) {
+        if (!((DENSE ? sk >= prev[q] : sk > prev[q]) && sk <= S[q])) {
           alive[q] = false;
           continue;
         }
         prev[q] = sk;
-        T ux = x.e[q], uy = y.e[q], uz = z.e[q];
+        T ux = x.e[q], uy = y.e[q], uz = z.e[q];  // the state after step sk (final: registers)
         if (sk < S[q]) {
           const T* c = a.ck + (int64_t)sk * nck + j0 + q;
           ux = c[0];
           uy = c[n];
           uz = c[2 * n];
+        }
+        if (DENSE) {
+          const T th = a.theta[(int64_t)k * n + j0 + q];
+          if (th != cst<T>(1.0)) {  // inside step sk - 1
+            const T* c = a.ck + (int64_t)(sk - 1) * nck + j0 + q;
+            const T xs = c[0], ys = c[n], zs = c[2 * n];
+            const T hs = hp[(int64_t)(sk - 1) * n + q];
+            T fsx, fsy, fsz, fnx, fny, fnz;
+            lorenz_f(xs, ys, zs, s.e[q], r.e[q], b.e[q], fsx, fsy, fsz);
+            lorenz_f(ux, uy, uz, s.e[q], r.e[q], b.e[q], fnx, fny, fnz);
+            const HermiteW<T> w = hermite_w(th);
+            ux = hermite_c(w, xs, ux, fsx, fnx, hs);
+            uy = hermite_c(w, ys, uy, fsy, fny, hs);
+            uz = hermite_c(w, zs, uz, fsz, fnz, hs);
+          }
         }
         T v0, v1, v2, g0, g1, g2;
         sp_vec(q, k, v0, v1, v2);
@@ -438,7 +399,14 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   // are the prefetched u_st, h_st and U_6 of step st.
   V lx = vsplat<T, K>(cst<T>(0.0)), ly = lx, lz = lx;
   V ps = lx, pr = lx, pb = lx;
-  // a landing save point's loss gradient, from the workspace
+  // Save points in reverse, read one save point ahead: next[q] is the step
+  // count at which slot q's current save point kk[q] falls, (tv0, tv1,
+  // tv2)[q] its loss gradient (from the workspace) and next2[q] the step count
+  // of the save point before it.  Each load is issued a whole save interval
+  // before its value is used, so the divergent save-point branch never waits
+  // on DRAM.
+  int kk[K], next[K], next2[K];
+  T tv0[K], tv1[K], tv2[K];
   auto sp_g = [&](int q, int k, T& v0, T& v1, T& v2) {
     v0 = v1 = v2 = cst<T>(0.0);
     if (k >= 0 && k < nvalid[q]) {
@@ -449,14 +417,11 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     }
   };
 #pragma unroll
-  for (int q = 0; q < K; ++q) {  // save points in reverse, read one ahead as in the forward
-    kk[q] = DENSE ? a.nsave - 1 : nvalid[q] - 1;
+  for (int q = 0; q < K; ++q) {
+    kk[q] = nvalid[q] - 1;
     next[q] = sp_idx(q, kk[q]);
     next2[q] = sp_idx(q, kk[q] - 1);
-    if (DENSE)
-      sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
-    else
-      sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
+    sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
   }
   V cx = x, cy = y, cz = z, hc = vsplat<T, K>(cst<T>(0.0));
   V gx6 = x, gy6 = y, gz6 = z;
@@ -513,29 +478,11 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
       while (st + 1 == next[q]) {
         T th = cst<T>(1.0);
         HermiteW<T> w;
-        T ux = x.e[q], uy = y.e[q], uz = z.e[q], fsx, fsy, fsz, fnx, fny, fnz;
         if (DENSE) {
           th = a.theta[(int64_t)kk[q] * n + j0 + q];
-          if (th != cst<T>(1.0)) {
-            w = hermite_w(th);
-            lorenz_f(cx.e[q], cy.e[q], cz.e[q], s.e[q], r.e[q], b.e[q], fsx, fsy, fsz);
-            lorenz_f(ux, uy, uz, s.e[q], r.e[q], b.e[q], fnx, fny, fnz);
-            const T hh = hc.e[q];
-            ux = hermite_c(w, cx.e[q], x.e[q], fsx, fnx, hh);
-            uy = hermite_c(w, cy.e[q], y.e[q], fsy, fny, hh);
-            uz = hermite_c(w, cz.e[q], z.e[q], fsz, fnz, hh);
-          }
+          if (th != cst<T>(1.0)) w = hermite_w(th);
         }
-        T gx, gy, gz;  // d loss_k / d u(t_k): computed here (dense) or by the forward half (landing)
-        if (DENSE && a.loss_kind == GS_LOSS_SUMSQ) {
-          gx = cst<T>(2.0) * (ux - tv0[q]);
-          gy = cst<T>(2.0) * (uy - tv1[q]);
-          gz = cst<T>(2.0) * (uz - tv2[q]);
-        } else {
-          gx = tv0[q];
-          gy = tv1[q];
-          gz = tv2[q];
-        }
+        const T gx = tv0[q], gy = tv1[q], gz = tv2[q];  // d loss_k / d u(t_k), from the forward half
         if (!DENSE || th == cst<T>(1.0)) {
           lx.e[q] += gx;
           ly.e[q] += gy;
@@ -558,10 +505,7 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
         --kk[q];
         next[q] = next2[q];
         next2[q] = sp_idx(q, kk[q] - 1);
-        if (DENSE)
-          sp_vec(q, kk[q], tv0[q], tv1[q], tv2[q]);
-        else
-          sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
+        sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
         if (!DENSE) break;
       }
     }
