@@ -155,6 +155,12 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+def distributed() -> bool:
+    """Launched by torchrun (any world size, one included): the NCCL process
+    group, its barriers and the max-over-ranks reductions run."""
+    return "TORCHELASTIC_RUN_ID" in os.environ or int(os.environ.get("WORLD_SIZE", 1)) > 1
+
+
 def metric_name(args) -> str:
     if args.workload == "lorenz_1m_dense":
         return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, dense save points)"
@@ -402,9 +408,10 @@ def run_single(args):
     W = WORKLOADS[args.workload]
     kind = W["kind"]
     rank, world, local = dist_env()
+    dist_on = distributed()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
+    if dist_on:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     n = args.n
@@ -463,7 +470,7 @@ def run_single(args):
         mesh_gb, out_gb, "larger than L2, no flush" if big else "fits in L2 (compute-bound kernel), no flush")
 
     def barrier():
-        if world > 1:
+        if dist_on:
             dist.barrier()
         torch.cuda.synchronize()
 
@@ -483,7 +490,7 @@ def run_single(args):
     launches = gs.gs_launch_count() - launches0
     clocks = clk.stop()
     tmax = torch.tensor([t_start.elapsed_time(t_end) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
+    if dist_on:
         dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
     elapsed = float(tmax.item())
     assert (status == 0).all()
@@ -508,7 +515,7 @@ def run_single(args):
     b.record(stream)
     barrier()
     e2e_t = torch.tensor([a.elapsed_time(b) / 1e3 / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
+    if dist_on:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
 
     unit = "trajectory-solves/s" if kind == "solve" else "trajectory-sensitivities/s"
@@ -537,7 +544,7 @@ def run_single(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args, min(262144 if kind == "solve" else 32768, n))
-    if world > 1:
+    if dist_on:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
@@ -576,10 +583,11 @@ def run_ours(args):
     W = WORKLOADS[args.workload]
     passes = W["passes"]
     rank, world, local = dist_env()
+    dist_on = distributed()
     torch.cuda.set_device(local)
     gs.gs_set_option(gs.gradsolve.OPT_NODE64_TENSOR_CORES, int(args.products == "tensor"))
     dev = torch.device("cuda", local)
-    if world > 1:
+    if dist_on:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     n = args.n
@@ -641,7 +649,7 @@ def run_ours(args):
                 grad_events.append((a, b))
 
     def barrier():
-        if world > 1:
+        if dist_on:
             dist.barrier()
         torch.cuda.synchronize()
 
@@ -663,7 +671,7 @@ def run_ours(args):
     grad_ms = float(np.mean([a.elapsed_time(b) for a, b in grad_events]))
     rec_ms = float(np.mean([a.elapsed_time(b) for a, b in rec_events]))
     tmax = torch.tensor([elapsed, grad_ms, rec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
+    if dist_on:
         dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
     elapsed, grad_ms, rec_ms = tmax.tolist()
 
@@ -721,7 +729,7 @@ def run_ours(args):
     b.record(stream)
     barrier()
     e2e_t = torch.tensor([a.elapsed_time(b) / 1e3 / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
+    if dist_on:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
     h2d = sum(v.numel() for v in host.values()) * esz
     d2h = passes * sum(t.numel() for t in h_out[0]) * esz
@@ -777,7 +785,7 @@ def run_ours(args):
         psample = {"lorenz_1m": 8192, "lorenz_1m_dense": 8192, "lorenz_small": 1024, "robertson": 256,
                    "robertson_ros3": 2048, "node64": 256, "kin8": 1024, "kin8_ros2": 32}[args.workload]
         line["parity"] = parity_sample(args, min(psample, n))
-    if world > 1:
+    if dist_on:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
