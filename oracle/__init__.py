@@ -68,6 +68,8 @@ def lib():
         L.or_solve_adaptive.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, f64, f64, i32, dp, f64, f64,
                                         f64, i32, i32, dp, ip, ip, i32]
         L.or_sens.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, i32, i32, dp, ip, ip, dp, ip, dp, i32]
+        L.or_step_errors.argtypes = [i32, i32, i32, i64, i32, i32, dp, dp, dp, i32, dp, ip, ip, f64, f64, dp, dp,
+                                     i32, dp, i32]
         L.or_count_step.argtypes = [i32, i32, i32, i32, dp]
         L.or_step.argtypes = [i32, i32, i32, i32, dp, dp, dp, f64, dp, dp]
         L.or_rhs.argtypes = [i32, i32, dp, dp, dp, dp, dp]
@@ -239,6 +241,28 @@ def replay(prob, mesh: Mesh, nthreads: int | None = None):
                      _d(_f64(prob.weight)), _d(loss), _d(us), nthreads or default_threads())
     _check(rc, "replay")
     return loss, us
+
+
+def step_errors(prob, mesh: Mesh, dtype: str | None = None, nperturb: int = 0, nthreads: int | None = None):
+    """The recorder's view of a given mesh (in `dtype`, default the problem's):
+    (err [n][smax], fac [n][smax]) -- each step's scaled error on the replay
+    of that mesh and the PI factor accepting it gives (no cap after a
+    rejection).  Zeros past nsteps and on trajectories with status != 0.
+    nperturb > 0 adds draws [nperturb][n][smax]: the factors again with each
+    step's start state perturbed at the precision's epsilon (one draw of
+    rounding per evaluation)."""
+    L = lib()
+    h, ns, _ = _mesh_args(mesh)
+    st = np.ascontiguousarray(mesh.status, np.int32)
+    err = np.zeros((prob.n, mesh.smax))
+    fac = np.zeros((prob.n, mesh.smax))
+    draws = np.zeros((nperturb, prob.n, mesh.smax)) if nperturb else None
+    rc = L.or_step_errors(SYSTEMS[prob.system], METHODS[prob.method], DTYPES[dtype or prob.dtype], prob.n, prob.d,
+                          prob.np_, _d(_f64(prob.p)), _d(_f64(prob.u0)), _d(_f64(prob.W)), mesh.smax, _d(h), _i(ns),
+                          _i(st), prob.rtol, prob.atol, _d(err), _d(fac), nperturb, _d(draws),
+                          nthreads or default_threads())
+    _check(rc, "step_errors")
+    return (err, fac, draws) if nperturb else (err, fac)
 
 
 def count_step(system: str, method: str, d: int, npar: int) -> dict:

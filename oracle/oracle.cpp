@@ -634,6 +634,25 @@ T initial_step(int sys, int method, int d, const T* u0, const T* p, const T* W, 
   return std::min(std::min(T(100) * h0, h1), t1 - t0);
 }
 
+// The PI factor after an accepted step with scaled error err (error order q):
+// 0.9 exp(-(0.7/q) ln err + (0.4/q) ln errprev) clipped to [0.2, 10], 10 if
+// err == 0; lnprev carries ln(errprev) (errprev floored at 1e-4) and is
+// updated here.  The cap at 1 after a rejection is the caller's.
+template <class T>
+T accept_factor(T err, T q, T& lnprev) {
+  const T ln_floor = ctrl_ln<T>(T(1e-4));
+  T fac, lnerr = ln_floor;
+  if (err == T(0)) {
+    fac = T(10);
+  } else {
+    lnerr = ctrl_ln<T>(err);
+    fac = T(0.9) * ctrl_exp<T>(std::fma(-T(0.7) / q, lnerr, (T(0.4) / q) * lnprev));
+    fac = std::min(T(10), std::max(T(0.2), fac));
+  }
+  lnprev = err < T(1e-4) ? ln_floor : lnerr;
+  return fac;
+}
+
 template <class T>
 RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, const T* W, T t0, T t1,
                         int nsave, const T* tsave, T rtol, T atol, T h0user, int smax, bool dense = false) {
@@ -660,7 +679,6 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
   }
   // the controller carries ln(errprev); errprev starts at 1 and is floored at 1e-4
   T t = t0, lnprev = T(0);
-  const T ln_floor = ctrl_ln<T>(T(1e-4));
   bool prev_rej = false;
   int kk = 0;
   while (true) {
@@ -707,16 +725,8 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
         out.save_idx[kk++] = out.nsteps;
       }
       // fac = 0.9 err^(-0.7/q) errprev^(0.4/q) = 0.9 exp(-(0.7/q) ln err + (0.4/q) ln errprev)
-      T fac, lnerr = ln_floor;
-      if (err == T(0)) {
-        fac = T(10);
-      } else {
-        lnerr = ctrl_ln<T>(err);
-        fac = T(0.9) * ctrl_exp<T>(std::fma(-T(0.7) / q, lnerr, (T(0.4) / q) * lnprev));
-        fac = std::min(T(10), std::max(T(0.2), fac));
-      }
+      T fac = accept_factor<T>(err, q, lnprev);
       if (prev_rej) fac = std::min(fac, T(1));
-      lnprev = err < T(1e-4) ? ln_floor : lnerr;
       prev_rej = false;
       hprop = fac * hprop;
       if (t >= t1) return out;  // the last step lands exactly on t1
@@ -1239,6 +1249,84 @@ int or_step(int sys, int method, int dtype, int d, const double* u, const double
     return ok ? 0 : 4;
   };
   return dtype == DT_F64 ? run(double(0)) : run(float(0));
+}
+
+// splitmix64 (Steele, Lea & Flood 2014): a counter-based 64-bit mixer, used
+// only to draw the perturbations of or_step_errors.
+static inline uint64_t splitmix64(uint64_t x) {
+  x += 0x9E3779B97F4A7C15ull;
+  x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+  x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+  return x ^ (x >> 31);
+}
+
+// The recorder's view of a given mesh: trajectory i replayed over h[i][0..
+// nsteps[i]) (no landing logic: the steps are data), and for every step s its
+// scaled error err[i][s] (the recorder's error norm on that step's embedded
+// estimate) and the PI factor fac[i][s] that accepting it gives (the cap after
+// a rejection not applied: the mesh does not show rejections).  On a mesh the
+// recorder wrote in the same precision, the proposal chain fac * h_prop
+// reproduces its steps.  Outputs [n][smax], zero past nsteps; a trajectory
+// whose status is not 0 is skipped (zeros).
+// nperturb > 0: fac_draws[k][n][smax] receives the same factors evaluated
+// again with every step's start state multiplied by 1 + r eps (r uniform in
+// [-1, 1) per component, draw, step and trajectory; eps of the precision),
+// each draw carrying its own errprev: the spread of the draws shows how far
+// rounding at the precision's level moves each factor (the embedded estimate
+// is a sum with cancellation, so a small error carries a large relative
+// rounding noise).
+int or_step_errors(int sys, int method, int dtype, int64_t n, int d, int np, const double* p, const double* u0,
+                   const double* W, int smax, const double* h, const int* nsteps, const int* status, double rtol,
+                   double atol, double* err, double* fac, int nperturb, double* fac_draws, int nthreads) {
+  Prob P{sys, method, dtype, d, np, n, p, u0, W};
+  int rc = check_prob(P);
+  if (rc) return rc;
+  parallel_for(n, nthreads, [&](int, int64_t a, int64_t b) {
+    auto run = [&](auto tag) {
+      using T = decltype(tag);
+      const T q = T(method_order(method));
+      std::vector<T> u(d), un(d), e(d), sc(d), pp(np), WW;
+      if (sys == SYS_NODE64) {
+        WW.resize(4096);
+        for (int c = 0; c < 4096; ++c) WW[c] = T(W[c]);
+      }
+      for (int64_t i = a; i < b; ++i) {
+        for (int s = 0; s < smax; ++s) err[i * smax + s] = fac[i * smax + s] = 0.0;
+        if (status && status[i] != TRAJ_OK) continue;
+        for (int c = 0; c < d; ++c) u[c] = T(u0[(int64_t)c * n + i]);
+        for (int c = 0; c < np; ++c) pp[c] = T(p[(int64_t)c * n + i]);
+        for (int k = 0; k < nperturb; ++k)
+          for (int s = 0; s < smax; ++s) fac_draws[((int64_t)k * n + i) * smax + s] = 0.0;
+        const int S = std::min(nsteps[i], smax);
+        T lnprev = T(0);
+        std::vector<T> lnprev_k(nperturb, T(0)), up(d), unp(d), ep(d), scp(d);
+        for (int s = 0; s < S; ++s) {
+          const T hs = T(h[i * smax + s]);
+          const T* Wp = WW.empty() ? nullptr : WW.data();
+          method_step<T>(sys, method, d, u.data(), pp.data(), Wp, hs, un.data(), e.data());
+          for (int c = 0; c < d; ++c) sc[c] = std::fma(T(rtol), std::max(std::fabs(u[c]), std::fabs(un[c])), T(atol));
+          const T er = rms_scaled<T>(d, e.data(), sc.data());
+          err[i * smax + s] = double(er);
+          fac[i * smax + s] = double(accept_factor<T>(er, q, lnprev));
+          for (int k = 0; k < nperturb; ++k) {
+            for (int c = 0; c < d; ++c) {
+              const uint64_t r = splitmix64(((((uint64_t)i * 4096 + (uint64_t)s) * 64 + (uint64_t)k) << 8) + c);
+              const T rho = T(double(r >> 11) * 0x1.0p-52 - 1.0);  // uniform in [-1, 1)
+              up[c] = u[c] * (T(1) + rho * std::numeric_limits<T>::epsilon());
+            }
+            method_step<T>(sys, method, d, up.data(), pp.data(), Wp, hs, unp.data(), ep.data());
+            for (int c = 0; c < d; ++c)
+              scp[c] = std::fma(T(rtol), std::max(std::fabs(up[c]), std::fabs(unp[c])), T(atol));
+            const T erk = rms_scaled<T>(d, ep.data(), scp.data());
+            fac_draws[((int64_t)k * n + i) * smax + s] = double(accept_factor<T>(erk, q, lnprev_k[k]));
+          }
+          for (int c = 0; c < d; ++c) u[c] = un[c];
+        }
+      }
+    };
+    if (dtype == DT_F64) run(double(0)); else run(float(0));
+  });
+  return 0;
 }
 
 // The right-hand side and its analytic Jacobian at one point (double).

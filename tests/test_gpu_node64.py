@@ -11,6 +11,7 @@ import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
 from gpu_util import TOL, dev, ensemble, loss_args, mesh_by_trajectory, mesh_from_oracle, parity, tens
+from mesh_check import controller_chain
 
 pytestmark = pytest.mark.gpu
 
@@ -38,17 +39,14 @@ def test_record_node64(case):
     torch.cuda.synchronize()
     h, ns, si, st, order = mesh_by_trajectory(mesh)
     assert (st == 0).all()
-    # tanh is each side's library function (not bitwise), and in fp32 at
-    # tol 1e-5 the embedded error estimate carries ~1e-3 relative rounding
-    # noise (heavy cancellation), so accept/reject decisions within that band
-    # of err = 1 can differ: measured 96.5 % equal step counts on 512
-    # trajectories.  (No fp32 mesh gate is stated; gradient parity below runs
-    # on the oracle's mesh.)
-    # The first step (the conservative starting step) has err << 1, where the
-    # fp32 estimate is mostly cancellation noise, so its PI factor -- and the
-    # step sizes after it -- differ at the 1e-3..1e-2 level between the two
-    # sides.  Checked instead: equal counts for most, every GPU mesh spans
-    # exactly [t0, t1], and the typical step-size difference is small.
+    # tanh is each side's library function (not bitwise), and the first step
+    # (the conservative starting step) has err << 1, where the fp32 estimate
+    # is mostly cancellation noise, so its PI factor -- and the step sizes
+    # after it -- differ between the GPU's fp32 record and the oracle's: about
+    # 3 % of step counts differ.  The mesh's gate is the controller chain
+    # (test_record_node64_follows_the_controller); here: equal counts for
+    # most, every GPU mesh spans exactly [t0, t1], and the typical step-size
+    # difference from the oracle's own record is small.
     same = ns == om.nsteps
     assert same.mean() >= 0.9
     for i in range(prob.n):
@@ -58,6 +56,69 @@ def test_record_node64(case):
     nsteps, _ = gs.gs_count(ens, prob.rtol, prob.atol, 64)
     torch.cuda.synchronize()
     assert np.array_equal(nsteps.cpu().numpy(), ns)
+
+
+def _chain_stats(prob, mesh, idx=None):
+    """The GPU mesh (trajectories idx, default all) against the recorder's
+    rules as the oracle evaluates them in fp64 on that mesh; each factor's
+    tolerance is CHAIN_C times the spread of the oracle's fp32 evaluations of
+    it under rounding-level perturbations (at least CHAIN_FLOOR)."""
+    h, ns, si, st, order = mesh_by_trajectory(mesh)
+    inv = np.empty_like(order)
+    inv[order] = np.arange(len(order))
+    nrej = mesh.nreject.cpu().numpy()[inv]
+    if idx is not None:
+        prob, h, ns, si, st, nrej = prob.subset(idx), h[idx], ns[idx], si[idx], st[idx], nrej[idx]
+    gm = oracle.Mesh(h, ns, si, st, nrej)
+    err, fac = oracle.step_errors(prob.as_dtype("f64"), gm)
+    _, _, draws = oracle.step_errors(prob, gm, dtype="f32", nperturb=CHAIN_DRAWS)
+    spread = np.max(np.abs(draws / np.where(fac > 0, fac, 1.0) - 1.0), axis=0)
+    devs = []
+    dev, short, bad = controller_chain(h, ns, si, nrej, fac, np.maximum(CHAIN_FLOOR, CHAIN_C * spread), devs)
+    devs = np.array(devs)
+    stats = dict(steps=int(ns.sum()), predicted=len(devs), median=float(np.median(devs)),
+                 p99_abs=float(np.quantile(np.abs(devs), 0.99)), max_abs=float(np.abs(devs).max()),
+                 max_over_tol=float(dev.max()),
+                 short=int(short.sum()), rejections=int(nrej.sum()), bad=int(bad.sum()),
+                 err_max=float(err[h > 0].max()), spread_median=float(np.median(spread[h > 0])))
+    print("node64 fp32 record vs the controller (fp64 view):", stats)
+    return stats, short, nrej
+
+
+# Tolerance of one controller factor on an fp32 record.  The GPU's scaled error
+# carries fp32 rounding, and the embedded estimate is a sum with cancellation:
+# the conservative first step's err (~2e-5 here) is mostly rounding noise, so
+# the factor after it moves by ~30 %, later ones by ~0.5 %.  The oracle
+# evaluates every factor again in fp32 with the step's start state perturbed
+# at fp32's epsilon (CHAIN_DRAWS draws); the GPU's factor must lie within
+# CHAIN_C times the largest deviation among them.  The oracle's own fp32 record
+# lies within 2.1 times it on these ensembles.  The signed deviations are
+# centred on 0 (median within 1e-3); a controller constant 0.5 % off moves
+# their median by 5e-3.
+CHAIN_DRAWS, CHAIN_C, CHAIN_FLOOR = 16, 4.0, 1e-5
+
+
+def _check_chain(stats, short, nrej):
+    assert stats["bad"] == 0
+    assert (short <= nrej).all()
+    assert abs(stats["median"]) <= 1e-3  # rounding is centred on 0; a biased controller is not
+    assert stats["err_max"] <= 1.0 + 1e-3
+
+
+def test_record_node64_follows_the_controller(case):
+    """The fp32 tensor-core recorder's mesh holds to the recorder's own rules
+    (mesh_check.controller_chain): every step that does not end on a stop is
+    the proposal fac * h_prop that the oracle's fp64 view of the same mesh
+    predicts, within fp32 rounding of the error estimate; steps shorter than
+    predicted number at most the trajectory's rejections; and every accepted
+    step passes the error test.  A wrong stage, error weight, norm or
+    controller constant moves the factors on every step."""
+    prob, _ = case
+    mesh = gs.new_mesh(prob.n, 64, 1, "f32", dev())
+    gs.gs_record(ensemble(prob), mesh, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    assert (mesh.status == 0).all()
+    _check_chain(*_chain_stats(prob, mesh))
 
 
 def test_solve_node64(case, products):
@@ -135,3 +196,5 @@ def test_full_size_sampled():
     om = oracle.Mesh(h[idx].astype(np.float64), ns[idx], si[idx], st[idx], np.zeros(len(idx), np.int32))
     ti = torch.tensor(idx, device=dev())
     parity(gs.GradOut(out.loss[ti], out.dp[:, ti], out.du0[:, ti], None), sub, om, dual=False)
+    # the full-size record holds to the controller on a sample of 512
+    _check_chain(*_chain_stats(prob, mesh, np.sort(rng.choice(prob.n, 512, replace=False))))

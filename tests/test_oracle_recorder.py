@@ -224,3 +224,69 @@ def test_controller_power_function():
     assert np.max(np.abs(c - r) / r) <= 4 * np.finfo(np.float32).eps
     s = oracle.ctrl_pow([0.0, 0.0, np.inf, 1.0, 2.0], [0.2, -0.2, -0.2, 0.7, 0.0])
     assert s[0] == 0 and np.isinf(s[1]) and s[2] == 0 and s[3] == 1 and s[4] == 1
+
+
+@pytest.mark.parametrize("name,method", [("lorenz_1m", "tsit5"), ("robertson", "ros2"), ("robertson", "ros3"),
+                                         ("node64", "tsit5")])
+def test_step_errors_reproduce_the_recorders_chain(name, method):
+    """oracle.step_errors on the oracle's own fp64 mesh: every step's error is
+    the norm of oracle.step's estimate (numpy), every factor the PI formula
+    (numpy pow), and the proposal chain fac * h_prop rebuilds every step
+    bitwise wherever no rejection intervened (mesh_check.controller_chain at
+    tolerance 0).  This is what the GPU recorders' fp32 meshes are held to,
+    within their rounding."""
+    from mesh_check import controller_chain
+    prob = W.node64(6, dtype="f64") if name == "node64" else W.by_name(name, n=6)
+    prob.method = method
+    mesh = oracle.record(prob, 20000)
+    assert (mesh.status == 0).all()
+    err, fac = oracle.step_errors(prob, mesh)
+    q = {"tsit5": 5, "ros2": 2, "ros3": 3}[method]
+    for i in range(2):
+        u = prob.u0[:, i].copy()
+        prev = 1.0
+        for s in range(mesh.nsteps[i]):
+            un, e, ok = oracle.step(prob.system, method, "f64", u, prob.p[:, i], mesh.h[i, s], prob.W)
+            en = _err_norm(e, u, un, prob.rtol, prob.atol)
+            assert abs(err[i, s] - en) <= 1e-13 * en
+            f = 10.0 if en == 0 else min(10.0, max(0.2, 0.9 * en ** (-0.7 / q) * prev ** (0.4 / q)))
+            assert abs(fac[i, s] - f) <= 1e-11 * f
+            prev = max(en, 1e-4)
+            u = un
+    assert (err[:, :][mesh.h == 0] == 0).all()
+    dev, short, bad = controller_chain(mesh.h, mesh.nsteps, mesh.save_idx, mesh.nreject, fac, 0.0)
+    assert (bad == 0).all() and (dev == 0).all(), (bad, dev)  # every prediction exact
+    assert (short <= mesh.nreject).all() and (short[mesh.nreject == 0] == 0).all()
+    # a controller with another safety factor fails the same check
+    dev2, short2, bad2 = controller_chain(mesh.h, mesh.nsteps, mesh.save_idx, mesh.nreject, fac * 0.95, 0.01)
+    assert (bad2 > 0).any()
+
+
+def test_step_errors_rounding_draws_bound_an_fp32_record():
+    """The perturbed fp32 draws of oracle.step_errors bound the rounding of
+    an fp32 record's controller: the oracle's own fp32 record of the d = 64
+    system follows the fp64 view's chain within 4x the draws' spread (its
+    own evaluation is one more draw), with the signed deviations centred on
+    0 (median within 1e-3); a safety factor 0.5 % off shifts that median to
+    5e-3, and one 3 % off also fails the per-step tolerance on most steps.
+    In fp64 the draws barely move (spread far below the fp32 one)."""
+    from mesh_check import controller_chain
+    prob = W.node64(100)
+    mesh = oracle.record(prob, 64)
+    assert (mesh.status == 0).all()
+    err, fac = oracle.step_errors(prob.as_dtype("f64"), mesh)
+    _, f32, draws = oracle.step_errors(prob, mesh, dtype="f32", nperturb=16)
+    spread = np.max(np.abs(draws / np.where(fac > 0, fac, 1.0) - 1.0), axis=0)
+    tol = np.maximum(1e-5, 4.0 * spread)
+    devs = []
+    dev, short, bad = controller_chain(mesh.h, mesh.nsteps, mesh.save_idx, mesh.nreject, fac, tol, devs)
+    assert (bad == 0).all() and (short == 0).all() and dev.max() <= 0.75
+    assert abs(np.median(devs)) <= 1e-3
+    d2 = []
+    controller_chain(mesh.h, mesh.nsteps, mesh.save_idx, mesh.nreject, fac * (0.8955 / 0.9), tol, d2)
+    assert np.median(d2) >= 4e-3
+    _, short3, bad3 = controller_chain(mesh.h, mesh.nsteps, mesh.save_idx, mesh.nreject, fac * (0.87 / 0.9), tol)
+    assert bad3.sum() + short3.sum() > 0.5 * len(devs)
+    _, _, d64 = oracle.step_errors(prob.as_dtype("f64"), mesh, nperturb=4)
+    s64 = np.max(np.abs(d64 / np.where(fac > 0, fac, 1.0) - 1.0), axis=0)
+    assert np.median(s64[mesh.h > 0]) <= 1e-6 * np.median(spread[mesh.h > 0])
