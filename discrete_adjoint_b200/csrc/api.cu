@@ -14,6 +14,7 @@ void count_launch(int k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
 // kernels (defined in the other translation units)
 gs_status count3(const gs_problem*, const gs_tol*, int32_t, int32_t*, int32_t*, cudaStream_t);
 gs_status record3(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
+gs_status record3_inplace(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
 gs_status solve_adaptive3(const gs_problem*, const gs_tol*, int32_t, void*, int32_t*, int32_t*, cudaStream_t);
 size_t record_ws_bytes(int64_t n, int32_t smax, int32_t nsave, size_t tsize);
 template <typename T>
@@ -185,6 +186,20 @@ gs_status gs_record(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, vo
   if (!ws || ws_bytes < gs_workspace_bytes(P, M, GS_OP_RECORD)) return GS_EWORKSPACE;
   if (P->system == GS_NODE64) return record_node64(P, tol, M, ws, (cudaStream_t)stream);
   return record3(P, tol, M, ws, (cudaStream_t)stream);
+}
+
+gs_status gs_record_inplace(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, size_t ws_bytes,
+                            void* stream) {
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if ((rc = check_mesh(P, M)) != GS_OK) return rc;
+  if ((rc = check_tol(P, tol)) != GS_OK) return rc;
+  if (P->system == GS_NODE64) return GS_EUNSUPPORTED;
+  if (tol->dense && P->n > 0 && !M->save_theta) return GS_EINVAL;  // a dense record writes the positions
+  if (P->n == 0) return GS_OK;
+  if (!ws || ws_bytes < GS_RECORD_INPLACE_WS) return GS_EWORKSPACE;
+  if ((uintptr_t)ws % 8 != 0) return GS_EINVAL;
+  return record3_inplace(P, tol, M, ws, (cudaStream_t)stream);
 }
 
 gs_status gs_solve(const gs_problem* P, const gs_mesh* M, void* u_save, void* stream) {

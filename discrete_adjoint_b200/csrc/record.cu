@@ -81,7 +81,8 @@ __device__ T initial_step_d(const T* u0, const T* p, T t0, T t1, T rtol, T atol)
 // One recorder trajectory held by a lane (D components).
 template <typename T, int D>
 struct Traj {
-  int64_t i;  // trajectory index
+  int64_t i;  // trajectory index (inputs)
+  int64_t o;  // where its outputs go: the trajectory index, or its slot (in-place re-record)
   T u[D], p[D], k1[D];
   T t, hprop, lnprev;
   int nst, nrej, status, kk;
@@ -94,6 +95,7 @@ __device__ __forceinline__ bool traj_start(const RecArgs<T>& a, int64_t i, Traj<
   constexpr int D = SysDim<SYS>::D;
   const int64_t n = a.n;
   r.i = i;
+  r.o = i;
 #pragma unroll
   for (int c = 0; c < D; ++c) {
     r.u[c] = a.u0[c * n + i];
@@ -169,7 +171,7 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
       r.status = GS_TRAJ_MAXSTEPS;
       return true;
     }
-    if (MODE == kRecMesh) a.h[r.i * a.hcol + (int64_t)r.nst * a.hstep] = h;
+    if (MODE == kRecMesh) a.h[r.o * a.hcol + (int64_t)r.nst * a.hstep] = h;
     ++r.nst;
     const T tprev = r.t;
     r.t = clipped ? tstop : tn;
@@ -181,8 +183,8 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
       while (r.kk < a.nsave && a.tsave[r.kk] <= r.t) {
         const T th = (a.tsave[r.kk] - tprev) / h;
         if (MODE == kRecMesh) {
-          a.save_idx[(int64_t)r.kk * n + r.i] = r.nst;
-          a.theta[(int64_t)r.kk * n + r.i] = th;
+          a.save_idx[(int64_t)r.kk * n + r.o] = r.nst;
+          a.theta[(int64_t)r.kk * n + r.o] = th;
         }
         if (MODE == kRecSolve) {
           const HermiteW<T> w = hermite_w(th);
@@ -211,7 +213,7 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
       if (METHOD == GS_TSIT5) r.k1[c] = k7[c];
     }
     while (!a.dense && r.kk < a.nsave && r.t == a.tsave[r.kk]) {
-      if (MODE == kRecMesh) a.save_idx[(int64_t)r.kk * n + r.i] = r.nst;
+      if (MODE == kRecMesh) a.save_idx[(int64_t)r.kk * n + r.o] = r.nst;
       if (MODE == kRecSolve) {
 #pragma unroll
         for (int c = 0; c < D; ++c) a.u_save[((int64_t)r.kk * D + c) * n + r.i] = r.u[c];
@@ -245,8 +247,8 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T, D
   if (MODE == kRecMesh) {
     // unreached save points (a failed trajectory); the h tail stays unwritten
     for (int k = r.kk; k < a.nsave; ++k) {
-      a.save_idx[(int64_t)k * n + r.i] = 0;
-      if (a.dense) a.theta[(int64_t)k * n + r.i] = cst<T>(1.0);
+      a.save_idx[(int64_t)k * n + r.o] = 0;
+      if (a.dense) a.theta[(int64_t)k * n + r.o] = cst<T>(1.0);
     }
   }
   if (MODE == kRecSolve && r.status != GS_TRAJ_OK) {
@@ -256,9 +258,9 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T, D
 #pragma unroll
       for (int c = 0; c < D; ++c) a.u_save[((int64_t)k * D + c) * n + r.i] = nan;
   }
-  if (a.nsteps) a.nsteps[r.i] = r.nst;
-  if (a.status) a.status[r.i] = r.status;
-  if (a.nreject) a.nreject[r.i] = r.nrej;
+  if (a.nsteps) a.nsteps[r.o] = r.nst;
+  if (a.status) a.status[r.o] = r.status;
+  if (a.nreject) a.nreject[r.o] = r.nrej;
 }
 
 // 6 resident blocks of 128 per SM (85 registers a thread): measured faster on
@@ -306,6 +308,62 @@ __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3(RecArgs<T> a) 
       traj_finish<T, MODE>(a, r);
       run = false;
     }
+  }
+}
+
+// In-place re-record: the slots keep the order an earlier record gave them
+// (slot j runs trajectory order[j]) and every output goes straight to its
+// slot (h step-major at s * n + j).  Slots are handed out in groups of 32, one
+// group per warp at a time from a global counter, in slot order: an earlier
+// record sorted them by decreasing step count, so the 32 lanes of a group run
+// chains of about equal length side by side, and the longest groups go first.
+// A lane whose chain ends waits for its group (the chains differ only by
+// their rejections when the ensemble is unchanged).  Rows from the new count
+// up to the slot's previous count are zeroed, so the mesh stays zero padded.
+// An order entry outside [0, n) leaves its slot with GS_TRAJ_BADORDER, no
+// steps, and its rows zeroed up to the previous count.  The loop ends: every
+// pass takes a group from a counter that only grows, and a group's inner loop
+// advances some chain's accepted or rejected count, both capped by smax.
+template <typename T, int SYS, int METHOD>
+__global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3_inplace(RecArgs<T> a, const int32_t* order,
+                                                                         unsigned long long* next_group) {
+  const unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const int64_t n = a.n;
+  const unsigned long long ngroups = (unsigned long long)((n + 31) / 32);
+  const T ln_floor = ctrl_ln<T>(cst<T>(1e-4));
+  Traj<T, SysDim<SYS>::D> r;
+  for (;;) {
+    unsigned long long g = 0;
+    if (lane == 0) g = atomicAdd(next_group, 1ull);
+    g = __shfl_sync(kFull, g, 0);
+    if (g >= ngroups) break;  // whole warp
+    const int64_t j = (int64_t)g * 32 + lane;
+    bool run = false;
+    int old = 0;
+    if (j < n) {
+      old = a.nsteps[j];
+      old = old < 0 ? 0 : (old > a.smax ? a.smax : old);
+      const int32_t i = order[j];
+      if (i >= 0 && i < n) {
+        run = traj_start<T, SYS, METHOD>(a, i, r);
+        r.o = j;
+        if (!run) traj_finish<T, kRecMesh>(a, r);
+      } else {
+        r.o = j;
+        r.nst = r.nrej = r.kk = 0;
+        r.status = GS_TRAJ_BADORDER;
+        traj_finish<T, kRecMesh>(a, r);
+      }
+    }
+    while (__any_sync(kFull, run)) {
+      if (run && traj_attempt<T, SYS, METHOD, kRecMesh>(a, r, ln_floor)) {
+        traj_finish<T, kRecMesh>(a, r);
+        run = false;
+      }
+    }
+    if (j < n)
+      for (int s = r.nst < 0 ? 0 : r.nst; s < old; ++s) a.h[j * a.hcol + (int64_t)s * a.hstep] = cst<T>(0.0);
   }
 }
 
@@ -417,6 +475,42 @@ static gs_status launch_rec(RecArgs<T> a, cudaStream_t st) {
   k_record3<T, SYS, METHOD, MODE><<<(unsigned)grid, bs, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
+template <typename T, int SYS, int METHOD>
+static gs_status launch_rec_inplace(RecArgs<T> a, const int32_t* order, unsigned long long* ctr, cudaStream_t st) {
+  // one resident wave; the warps take groups of 32 slots until none is left
+  const int bs = 128;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_record3_inplace<T, SYS, METHOD>, bs, 0) !=
+          cudaSuccess)
+    return GS_ECUDA;
+  const int64_t groups = (a.n + 31) / 32;
+  int64_t grid = (int64_t)(per_sm > 0 ? per_sm : 1) * sms;
+  if (grid * (bs / 32) > groups) grid = (groups + bs / 32 - 1) / (bs / 32);
+  if (cudaMemsetAsync(ctr, 0, sizeof(unsigned long long), st) != cudaSuccess) return GS_ECUDA;
+  k_record3_inplace<T, SYS, METHOD><<<(unsigned)grid, bs, 0, st>>>(a, order, ctr);
+  count_launch();
+  return launch_ok() ? GS_OK : GS_ECUDA;
+}
+
+template <typename T>
+static gs_status dispatch_rec_inplace(int sys, int method, const RecArgs<T>& a, const int32_t* order,
+                                      unsigned long long* ctr, cudaStream_t st) {
+  if (sys == GS_LORENZ && method == GS_TSIT5) return launch_rec_inplace<T, kSysLorenz, GS_TSIT5>(a, order, ctr, st);
+  if (sys == GS_LORENZ && method == GS_ROS2) return launch_rec_inplace<T, kSysLorenz, GS_ROS2>(a, order, ctr, st);
+  if (sys == GS_ROBERTSON && method == GS_TSIT5)
+    return launch_rec_inplace<T, kSysRobertson, GS_TSIT5>(a, order, ctr, st);
+  if (sys == GS_ROBERTSON && method == GS_ROS2)
+    return launch_rec_inplace<T, kSysRobertson, GS_ROS2>(a, order, ctr, st);
+  if (sys == GS_LORENZ && method == GS_ROS3) return launch_rec_inplace<T, kSysLorenz, GS_ROS3>(a, order, ctr, st);
+  if (sys == GS_ROBERTSON && method == GS_ROS3)
+    return launch_rec_inplace<T, kSysRobertson, GS_ROS3>(a, order, ctr, st);
+  if (sys == GS_KIN8 && method == GS_ROS2) return launch_rec_inplace<T, kSysKin8, GS_ROS2>(a, order, ctr, st);
+  if (sys == GS_KIN8 && method == GS_ROS3) return launch_rec_inplace<T, kSysKin8, GS_ROS3>(a, order, ctr, st);
+  return GS_EUNSUPPORTED;
 }
 
 template <typename T, int MODE>
@@ -581,6 +675,28 @@ static gs_status record3_t(const gs_problem* P, const gs_tol* tol, const gs_mesh
 
 gs_status record3(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, cudaStream_t st) {
   return P->dtype == GS_F64 ? record3_t<double>(P, tol, M, ws, st) : record3_t<float>(P, tol, M, ws, st);
+}
+
+// In-place re-record into the caller's mesh, in its slot order (no workspace
+// copy, no sort, no gather); ws holds the group counter.
+template <typename T>
+static gs_status record3_inplace_t(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws,
+                                   cudaStream_t st) {
+  RecArgs<T> a = rec_args<T>(P, tol, M->smax);
+  a.theta = tol->dense ? (T*)M->save_theta : nullptr;
+  a.h = (T*)M->h;
+  a.hcol = 1;  // step-major: step s of slot j at s * n + j
+  a.hstep = P->n;
+  a.save_idx = M->save_idx;
+  a.nsteps = M->nsteps;
+  a.status = M->status;
+  a.nreject = M->nreject;
+  return dispatch_rec_inplace<T>(P->system, P->method, a, M->order, (unsigned long long*)ws, st);
+}
+
+gs_status record3_inplace(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, cudaStream_t st) {
+  return P->dtype == GS_F64 ? record3_inplace_t<double>(P, tol, M, ws, st)
+                            : record3_inplace_t<float>(P, tol, M, ws, st);
 }
 
 gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,

@@ -30,12 +30,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 # ---- constants (mirroring include/gradsolve.h) -------------------------------
 GS_OK, GS_EINVAL, GS_ECUDA, GS_EWORKSPACE, GS_EUNSUPPORTED = 0, -1, -2, -3, -4
-TRAJ_OK, TRAJ_MAXSTEPS, TRAJ_DTMIN, TRAJ_NONFINITE, TRAJ_SINGULAR = 0, 1, 2, 3, 4
+TRAJ_OK, TRAJ_MAXSTEPS, TRAJ_DTMIN, TRAJ_NONFINITE, TRAJ_SINGULAR, TRAJ_BADORDER = 0, 1, 2, 3, 4, 5
 SYSTEMS = {"lorenz": 1, "robertson": 2, "hires": 3, "node64": 4, "kin8": 5}
 METHODS = {"tsit5": 1, "ros2": 2, "ros3": 3}
 DTYPES = {"f32": 1, "f64": 2}
 LOSSES = {"sumsq": 1, "linear": 2}
 OP_RECORD, OP_GRAD = 0, 1
+RECORD_INPLACE_WS = 8
 MAX_SAVE = 64
 TORCH_DTYPE = {"f32": torch.float32, "f64": torch.float64}
 
@@ -70,6 +71,9 @@ _lib.gs_count.argtypes = [_P(_Problem), _P(_Tol), ctypes.c_int32, ctypes.c_void_
 _lib.gs_count.restype = ctypes.c_int32
 _lib.gs_record.argtypes = [_P(_Problem), _P(_Tol), _P(_Mesh), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
 _lib.gs_record.restype = ctypes.c_int32
+_lib.gs_record_inplace.argtypes = [_P(_Problem), _P(_Tol), _P(_Mesh), ctypes.c_void_p, ctypes.c_size_t,
+                                   ctypes.c_void_p]
+_lib.gs_record_inplace.restype = ctypes.c_int32
 _lib.gs_solve.argtypes = [_P(_Problem), _P(_Mesh), ctypes.c_void_p, ctypes.c_void_p]
 _lib.gs_solve_adaptive.argtypes = [_P(_Problem), _P(_Tol), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p]
@@ -253,6 +257,18 @@ def gs_record(ens: Ensemble, mesh: Mesh, rtol: float, atol: float, h0: float = 0
         ws = workspace(need, ens.u0.device)
     _check(_lib.gs_record(ctypes.byref(ps), ctypes.byref(tol), ctypes.byref(ms), _ptr(ws), ws.numel(),
                           _stream(stream)), "gs_record")
+    return mesh
+
+
+def gs_record_inplace(ens: Ensemble, mesh: Mesh, rtol: float, atol: float, h0: float = 0.0, ws=None, stream=None,
+                      dense: bool | None = None):
+    """Re-record into mesh keeping its slot order (set by an earlier record)."""
+    dense = mesh.save_theta is not None if dense is None else dense
+    ps, ms, tol = ens._struct(), mesh._struct(), _Tol(rtol, atol, h0, int(dense))
+    if ws is None:
+        ws = workspace(RECORD_INPLACE_WS, ens.u0.device)
+    _check(_lib.gs_record_inplace(ctypes.byref(ps), ctypes.byref(tol), ctypes.byref(ms), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "gs_record_inplace")
     return mesh
 
 

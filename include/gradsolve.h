@@ -61,6 +61,7 @@ typedef int32_t gs_status;
 #define GS_TRAJ_DTMIN 2     /* step proposal fell below 16 eps |t| */
 #define GS_TRAJ_NONFINITE 3 /* non-finite input, f(u0) or initial step */
 #define GS_TRAJ_SINGULAR 4  /* zero or non-finite pivot in the Rosenbrock LU */
+#define GS_TRAJ_BADORDER 5  /* gs_record_inplace: the slot's order entry is outside [0, n) */
 
 /* Registered right-hand sides. */
 #define GS_LORENZ 1    /* d=3, np=3, p=(sigma, rho, beta): DiffEqGPU "ad" page, Lorenz listing */
@@ -218,6 +219,31 @@ GS_API gs_status gs_count(const gs_problem* prob, const gs_tol* tol, int32_t sma
  */
 GS_API gs_status gs_record(const gs_problem* prob, const gs_tol* tol, const gs_mesh* mesh, void* ws, size_t ws_bytes,
                     void* stream);
+
+/*
+ * Re-record in place: the adaptive solve of every trajectory, as gs_record
+ * runs it, into a mesh whose slot order an earlier record of this ensemble
+ * (gs_record, or this call) set.  The order is kept: mesh->order is read, not
+ * written, and must be a permutation of 0..n-1 (an entry outside [0, n) gives
+ * its slot GS_TRAJ_BADORDER and no steps; duplicates are not detected).  Each
+ * slot's steps, count, status, rejections, save indices (and save positions
+ * of a dense record) are written straight into the slot, with no workspace
+ * copy, sort or gather; h rows from the slot's new count up to its previous
+ * count (mesh->nsteps on entry, clamped to [0, smax]) are zeroed, so a mesh
+ * that was zero padded stays so.  Slots run in groups of 32 in slot order, so
+ * an order sorted by step count (what gs_record leaves) keeps the lanes of a
+ * warp on chains of about equal length.  When the trajectories' step counts
+ * changed since the order was set, the mesh is still exact, only less well
+ * sorted for gs_grad; gs_record sorts afresh.
+ *   ws        device, at least GS_RECORD_INPLACE_WS bytes, 8-byte aligned
+ *             (a work counter; gs_workspace_bytes(GS_OP_RECORD) is enough).
+ * Values equal gs_record's bit for bit (each trajectory's arithmetic does not
+ * depend on where it runs).  Same systems, methods and precisions as
+ * gs_record except GS_NODE64 (GS_EUNSUPPORTED).
+ */
+#define GS_RECORD_INPLACE_WS 8
+GS_API gs_status gs_record_inplace(const gs_problem* prob, const gs_tol* tol, const gs_mesh* mesh, void* ws,
+                                   size_t ws_bytes, void* stream);
 
 /*
  * Forward-only replay on the mesh: u_save, device [nsave][d][n] dtype, indexed

@@ -237,3 +237,27 @@ def test_kin8_validation_host_only(no_launch):
     t5 = _host_problem(system=5, method=1)
     t5.d = t5.np = 8
     assert _lib.gs_count(ctypes.byref(t5), ctypes.byref(tol), 100, ctypes.c_void_p(16), None, None) == -4
+
+
+@hidden_only
+def test_record_inplace_validation_host_only(no_launch):
+    """gs_record_inplace refuses before any launch: a missing, small or
+    misaligned workspace, the d = 64 system, a dense request without save
+    positions, bad tolerances; an empty ensemble is a no-op."""
+    from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol
+    p = _host_problem()
+    m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+    tol = _Tol(1e-6, 1e-6, 0.0)
+    call = lambda prob, mesh, t, ws, nb: _lib.gs_record_inplace(ctypes.byref(prob), ctypes.byref(t),
+                                                                ctypes.byref(mesh), ws, nb, None)
+    assert call(p, m, tol, None, 8) == -3
+    assert call(p, m, tol, ctypes.c_void_p(16), 4) == -3
+    assert call(p, m, tol, ctypes.c_void_p(20), 8) == -1
+    assert call(p, m, _Tol(-1.0, 1e-6, 0.0), ctypes.c_void_p(16), 8) == -1
+    assert call(p, m, _Tol(1e-6, 1e-6, 0.0, 1), ctypes.c_void_p(16), 8) == -1  # dense needs save_theta
+    from discrete_adjoint_b200.gradsolve import _Problem
+    node = _Problem(4, 1, 1, 64, 64, 1000, 16, 16, 16, 0.0, 10.0, 10, p._keep)
+    m64 = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+    assert call(node, m64, tol, ctypes.c_void_p(16), 8) == -4
+    assert call(p, _Mesh(100, 10, 16, None, 16, 16, 16, 16), tol, ctypes.c_void_p(16), 8) == -1  # no order
+    assert call(_host_problem(n=0), _Mesh(100, 10, None, None, None, None, None, None), tol, None, 0) == 0
