@@ -464,16 +464,28 @@ def run_single(args):
     if kind == "solve":
         attempts = int(mesh.nsteps.sum().item() + mesh.nreject.sum().item())
         flops = W["flop_attempt"] * attempts
+        # the solves run in the setup record's slot order (trajectories of
+        # equal step count side by side in a warp); --record full: in
+        # trajectory order (gs_solve_adaptive)
+        order = mesh.order.clone()
         del mesh
         u_save = torch.empty((len(prob.tsave), prob.d, n), dtype=td, device=dev)
         nsteps = torch.empty(n, dtype=torch.int32, device=dev)
         status = torch.empty(n, dtype=torch.int32, device=dev)
+        ws_solve = gs.workspace(gs.gradsolve.RECORD_INPLACE_WS, dev)
         outputs = [u_save]
-        work = {"attempted_steps": attempts}
+        ordered = args.record == "inplace"
+        work = {"attempted_steps": attempts,
+                "solve": ("gs_solve_adaptive_ordered in the slot order of a setup record of the ensemble"
+                          if ordered else "gs_solve_adaptive in trajectory order")}
 
         def step():
-            gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, smax, u_save=u_save, nsteps=nsteps, status=status,
-                                 stream=stream)
+            if ordered:
+                gs.gs_solve_adaptive_ordered(ens, prob.rtol, prob.atol, smax, order, u_save=u_save, nsteps=nsteps,
+                                             status=status, ws=ws_solve, stream=stream)
+            else:
+                gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, smax, u_save=u_save, nsteps=nsteps, status=status,
+                                     stream=stream)
     else:
         total_steps = int(mesh.nsteps.sum().item())
         flops = W["flop_step"] * total_steps

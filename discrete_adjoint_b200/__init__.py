@@ -6,9 +6,11 @@ package loads the library and fails if it has not been built.
 """
 from . import gradsolve
 from .gradsolve import (Ensemble, GradOut, Mesh, gs_count, gs_grad, gs_grad_static, gs_launch_count, gs_record,
-                        gs_record_inplace, gs_sens, gs_set_option, gs_solve, gs_solve_adaptive, gs_status_string, gs_workspace_bytes, new_grad_out, new_mesh,
+                        gs_record_inplace, gs_sens, gs_set_option, gs_solve, gs_solve_adaptive,
+                        gs_solve_adaptive_ordered, gs_status_string, gs_workspace_bytes, new_grad_out, new_mesh,
                         workspace)
 
 __all__ = ["gradsolve", "Ensemble", "GradOut", "Mesh", "gs_count", "gs_grad", "gs_grad_static", "gs_launch_count",
-           "gs_record", "gs_record_inplace", "gs_sens", "gs_set_option", "gs_solve", "gs_solve_adaptive", "gs_status_string", "gs_workspace_bytes", "new_grad_out",
-           "new_mesh", "workspace"]
+           "gs_record", "gs_record_inplace", "gs_sens", "gs_set_option", "gs_solve", "gs_solve_adaptive",
+           "gs_solve_adaptive_ordered", "gs_status_string", "gs_workspace_bytes", "new_grad_out", "new_mesh",
+           "workspace"]

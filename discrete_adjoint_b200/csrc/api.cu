@@ -16,6 +16,8 @@ gs_status count3(const gs_problem*, const gs_tol*, int32_t, int32_t*, int32_t*, 
 gs_status record3(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
 gs_status record3_inplace(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
 gs_status solve_adaptive3(const gs_problem*, const gs_tol*, int32_t, void*, int32_t*, int32_t*, cudaStream_t);
+gs_status solve_adaptive3_ordered(const gs_problem*, const gs_tol*, int32_t, const int32_t*, void*, int32_t*,
+                                  int32_t*, void*, cudaStream_t);
 size_t record_ws_bytes(int64_t n, int32_t smax, int32_t nsave, size_t tsize);
 template <typename T>
 gs_status launch_grad_tsit5_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
@@ -186,6 +188,21 @@ gs_status gs_record(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, vo
   if (!ws || ws_bytes < gs_workspace_bytes(P, M, GS_OP_RECORD)) return GS_EWORKSPACE;
   if (P->system == GS_NODE64) return record_node64(P, tol, M, ws, (cudaStream_t)stream);
   return record3(P, tol, M, ws, (cudaStream_t)stream);
+}
+
+gs_status gs_solve_adaptive_ordered(const gs_problem* P, const gs_tol* tol, int32_t smax, const int32_t* order,
+                                    void* u_save, int32_t* nsteps, int32_t* status, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  gs_status rc = check_problem(P);
+  if (rc != GS_OK) return rc;
+  if ((rc = check_tol(P, tol)) != GS_OK) return rc;
+  if (smax < 1) return GS_EINVAL;
+  if (P->system == GS_NODE64) return GS_EUNSUPPORTED;
+  if (P->n == 0) return GS_OK;
+  if (!u_save || !order) return GS_EINVAL;
+  if (!ws || ws_bytes < GS_RECORD_INPLACE_WS) return GS_EWORKSPACE;
+  if ((uintptr_t)ws % 8 != 0) return GS_EINVAL;
+  return solve_adaptive3_ordered(P, tol, smax, order, u_save, nsteps, status, ws, (cudaStream_t)stream);
 }
 
 gs_status gs_record_inplace(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, size_t ws_bytes,

@@ -324,9 +324,12 @@ __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3(RecArgs<T> a) 
 // steps, and its rows zeroed up to the previous count.  The loop ends: every
 // pass takes a group from a counter that only grows, and a group's inner loop
 // advances some chain's accepted or rejected count, both capped by smax.
-template <typename T, int SYS, int METHOD>
+// MODE kRecSolve runs the adaptive forward-only solve in the same grouped
+// order with its outputs by trajectory (an entry outside [0, n) is skipped).
+template <typename T, int SYS, int METHOD, int MODE>
 __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3_inplace(RecArgs<T> a, const int32_t* order,
                                                                          unsigned long long* next_group) {
+  static_assert(MODE == kRecMesh || MODE == kRecSolve, "grouped passes: mesh or solve");
   const unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const int64_t n = a.n;
@@ -342,14 +345,16 @@ __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3_inplace(RecArg
     bool run = false;
     int old = 0;
     if (j < n) {
-      old = a.nsteps[j];
-      old = old < 0 ? 0 : (old > a.smax ? a.smax : old);
+      if (MODE == kRecMesh) {
+        old = a.nsteps[j];
+        old = old < 0 ? 0 : (old > a.smax ? a.smax : old);
+      }
       const int32_t i = order[j];
       if (i >= 0 && i < n) {
         run = traj_start<T, SYS, METHOD>(a, i, r);
-        r.o = j;
-        if (!run) traj_finish<T, kRecMesh>(a, r);
-      } else {
+        if (MODE == kRecMesh) r.o = j;
+        if (!run) traj_finish<T, MODE>(a, r);
+      } else if (MODE == kRecMesh) {
         r.o = j;
         r.nst = r.nrej = r.kk = 0;
         r.status = GS_TRAJ_BADORDER;
@@ -357,12 +362,12 @@ __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3_inplace(RecArg
       }
     }
     while (__any_sync(kFull, run)) {
-      if (run && traj_attempt<T, SYS, METHOD, kRecMesh>(a, r, ln_floor)) {
-        traj_finish<T, kRecMesh>(a, r);
+      if (run && traj_attempt<T, SYS, METHOD, MODE>(a, r, ln_floor)) {
+        traj_finish<T, MODE>(a, r);
         run = false;
       }
     }
-    if (j < n)
+    if (MODE == kRecMesh && j < n)
       for (int s = r.nst < 0 ? 0 : r.nst; s < old; ++s) a.h[j * a.hcol + (int64_t)s * a.hstep] = cst<T>(0.0);
   }
 }
@@ -477,39 +482,40 @@ static gs_status launch_rec(RecArgs<T> a, cudaStream_t st) {
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
 
-template <typename T, int SYS, int METHOD>
+template <typename T, int SYS, int METHOD, int MODE>
 static gs_status launch_rec_inplace(RecArgs<T> a, const int32_t* order, unsigned long long* ctr, cudaStream_t st) {
   // one resident wave; the warps take groups of 32 slots until none is left
   const int bs = 128;
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
       cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_record3_inplace<T, SYS, METHOD>, bs, 0) !=
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_record3_inplace<T, SYS, METHOD, MODE>, bs, 0) !=
           cudaSuccess)
     return GS_ECUDA;
   const int64_t groups = (a.n + 31) / 32;
   int64_t grid = (int64_t)(per_sm > 0 ? per_sm : 1) * sms;
   if (grid * (bs / 32) > groups) grid = (groups + bs / 32 - 1) / (bs / 32);
   if (cudaMemsetAsync(ctr, 0, sizeof(unsigned long long), st) != cudaSuccess) return GS_ECUDA;
-  k_record3_inplace<T, SYS, METHOD><<<(unsigned)grid, bs, 0, st>>>(a, order, ctr);
+  k_record3_inplace<T, SYS, METHOD, MODE><<<(unsigned)grid, bs, 0, st>>>(a, order, ctr);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
 
-template <typename T>
+template <typename T, int MODE>
 static gs_status dispatch_rec_inplace(int sys, int method, const RecArgs<T>& a, const int32_t* order,
                                       unsigned long long* ctr, cudaStream_t st) {
-  if (sys == GS_LORENZ && method == GS_TSIT5) return launch_rec_inplace<T, kSysLorenz, GS_TSIT5>(a, order, ctr, st);
-  if (sys == GS_LORENZ && method == GS_ROS2) return launch_rec_inplace<T, kSysLorenz, GS_ROS2>(a, order, ctr, st);
+  if (sys == GS_LORENZ && method == GS_TSIT5)
+    return launch_rec_inplace<T, kSysLorenz, GS_TSIT5, MODE>(a, order, ctr, st);
+  if (sys == GS_LORENZ && method == GS_ROS2) return launch_rec_inplace<T, kSysLorenz, GS_ROS2, MODE>(a, order, ctr, st);
   if (sys == GS_ROBERTSON && method == GS_TSIT5)
-    return launch_rec_inplace<T, kSysRobertson, GS_TSIT5>(a, order, ctr, st);
+    return launch_rec_inplace<T, kSysRobertson, GS_TSIT5, MODE>(a, order, ctr, st);
   if (sys == GS_ROBERTSON && method == GS_ROS2)
-    return launch_rec_inplace<T, kSysRobertson, GS_ROS2>(a, order, ctr, st);
-  if (sys == GS_LORENZ && method == GS_ROS3) return launch_rec_inplace<T, kSysLorenz, GS_ROS3>(a, order, ctr, st);
+    return launch_rec_inplace<T, kSysRobertson, GS_ROS2, MODE>(a, order, ctr, st);
+  if (sys == GS_LORENZ && method == GS_ROS3) return launch_rec_inplace<T, kSysLorenz, GS_ROS3, MODE>(a, order, ctr, st);
   if (sys == GS_ROBERTSON && method == GS_ROS3)
-    return launch_rec_inplace<T, kSysRobertson, GS_ROS3>(a, order, ctr, st);
-  if (sys == GS_KIN8 && method == GS_ROS2) return launch_rec_inplace<T, kSysKin8, GS_ROS2>(a, order, ctr, st);
-  if (sys == GS_KIN8 && method == GS_ROS3) return launch_rec_inplace<T, kSysKin8, GS_ROS3>(a, order, ctr, st);
+    return launch_rec_inplace<T, kSysRobertson, GS_ROS3, MODE>(a, order, ctr, st);
+  if (sys == GS_KIN8 && method == GS_ROS2) return launch_rec_inplace<T, kSysKin8, GS_ROS2, MODE>(a, order, ctr, st);
+  if (sys == GS_KIN8 && method == GS_ROS3) return launch_rec_inplace<T, kSysKin8, GS_ROS3, MODE>(a, order, ctr, st);
   return GS_EUNSUPPORTED;
 }
 
@@ -556,6 +562,25 @@ gs_status solve_adaptive3(const gs_problem* P, const gs_tol* tol, int32_t smax, 
   a.status = status;
   a.u_save = (float*)u_save;
   return dispatch_rec<float, kRecSolve>(P->system, P->method, a, st);
+}
+
+// The adaptive forward-only solve in a given trajectory order (groups of 32
+// consecutive entries side by side, outputs by trajectory); ws holds the
+// group counter.
+gs_status solve_adaptive3_ordered(const gs_problem* P, const gs_tol* tol, int32_t smax, const int32_t* order,
+                                  void* u_save, int32_t* nsteps, int32_t* status, void* ws, cudaStream_t st) {
+  if (P->dtype == GS_F64) {
+    RecArgs<double> a = rec_args<double>(P, tol, smax);
+    a.nsteps = nsteps;
+    a.status = status;
+    a.u_save = (double*)u_save;
+    return dispatch_rec_inplace<double, kRecSolve>(P->system, P->method, a, order, (unsigned long long*)ws, st);
+  }
+  RecArgs<float> a = rec_args<float>(P, tol, smax);
+  a.nsteps = nsteps;
+  a.status = status;
+  a.u_save = (float*)u_save;
+  return dispatch_rec_inplace<float, kRecSolve>(P->system, P->method, a, order, (unsigned long long*)ws, st);
 }
 
 static size_t al256(size_t b) { return (b + 255) / 256 * 256; }
@@ -691,7 +716,7 @@ static gs_status record3_inplace_t(const gs_problem* P, const gs_tol* tol, const
   a.nsteps = M->nsteps;
   a.status = M->status;
   a.nreject = M->nreject;
-  return dispatch_rec_inplace<T>(P->system, P->method, a, M->order, (unsigned long long*)ws, st);
+  return dispatch_rec_inplace<T, kRecMesh>(P->system, P->method, a, M->order, (unsigned long long*)ws, st);
 }
 
 gs_status record3_inplace(const gs_problem* P, const gs_tol* tol, const gs_mesh* M, void* ws, cudaStream_t st) {

@@ -78,6 +78,10 @@ _lib.gs_solve.argtypes = [_P(_Problem), _P(_Mesh), ctypes.c_void_p, ctypes.c_voi
 _lib.gs_solve_adaptive.argtypes = [_P(_Problem), _P(_Tol), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p]
 _lib.gs_solve_adaptive.restype = ctypes.c_int32
+_lib.gs_solve_adaptive_ordered.argtypes = [_P(_Problem), _P(_Tol), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                           ctypes.c_void_p]
+_lib.gs_solve_adaptive_ordered.restype = ctypes.c_int32
 _lib.gs_set_option.argtypes = [ctypes.c_int32, ctypes.c_int32]
 _lib.gs_set_option.restype = ctypes.c_int32
 _lib.gs_sens.argtypes = [_P(_Problem), _P(_Mesh), _P(_Loss)] + [ctypes.c_void_p] * 5
@@ -243,6 +247,27 @@ def gs_solve_adaptive(ens: Ensemble, rtol: float, atol: float, smax: int, h0: fl
     ps, tol = ens._struct(), _Tol(rtol, atol, h0, int(dense))
     _check(_lib.gs_solve_adaptive(ctypes.byref(ps), ctypes.byref(tol), smax, _ptr(u_save), _ptr(nsteps),
                                   _ptr(status), _stream(stream)), "gs_solve_adaptive")
+    return u_save, nsteps, status
+
+
+def gs_solve_adaptive_ordered(ens: Ensemble, rtol: float, atol: float, smax: int, order, h0: float = 0.0,
+                              u_save=None, nsteps=None, status=None, ws=None, stream=None, dense: bool = False):
+    """gs_solve_adaptive with trajectories run in groups of 32 consecutive
+    entries of order (device int32 permutation, e.g. an earlier record's
+    mesh.order); outputs by trajectory."""
+    dev = ens.u0.device
+    if u_save is None:
+        u_save = torch.empty((len(ens.tsave), ens.d, ens.n), dtype=TORCH_DTYPE[ens.dtype], device=dev)
+    if nsteps is None:
+        nsteps = torch.empty(ens.n, dtype=torch.int32, device=dev)
+    if status is None:
+        status = torch.empty(ens.n, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(RECORD_INPLACE_WS, dev)
+    ps, tol = ens._struct(), _Tol(rtol, atol, h0, int(dense))
+    _check(_lib.gs_solve_adaptive_ordered(ctypes.byref(ps), ctypes.byref(tol), smax, _ptr(order), _ptr(u_save),
+                                          _ptr(nsteps), _ptr(status), _ptr(ws), ws.numel(), _stream(stream)),
+           "gs_solve_adaptive_ordered")
     return u_save, nsteps, status
 
 

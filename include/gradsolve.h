@@ -98,6 +98,7 @@ typedef int32_t gs_status;
 #define GS_LOSS_LINEAR 2 /* L_i = sum_k weight_ik . u_i(t_k) */
 
 #define GS_MAX_SAVE 64 /* largest nsave */
+#define GS_RECORD_INPLACE_WS 8 /* workspace bytes of gs_record_inplace and gs_solve_adaptive_ordered */
 
 /* workspace operations */
 #define GS_OP_RECORD 0
@@ -241,7 +242,6 @@ GS_API gs_status gs_record(const gs_problem* prob, const gs_tol* tol, const gs_m
  * depend on where it runs).  Same systems, methods and precisions as
  * gs_record except GS_NODE64 (GS_EUNSUPPORTED).
  */
-#define GS_RECORD_INPLACE_WS 8
 GS_API gs_status gs_record_inplace(const gs_problem* prob, const gs_tol* tol, const gs_mesh* mesh, void* ws,
                                    size_t ws_bytes, void* stream);
 
@@ -269,6 +269,21 @@ GS_API gs_status gs_solve(const gs_problem* prob, const gs_mesh* mesh, void* u_s
  */
 GS_API gs_status gs_solve_adaptive(const gs_problem* prob, const gs_tol* tol, int32_t smax, void* u_save,
                                    int32_t* nsteps, int32_t* status, void* stream);
+
+/*
+ * gs_solve_adaptive in a given trajectory order: groups of 32 consecutive
+ * entries of order (device [n] int32, a permutation of 0..n-1, e.g. the slot
+ * order of an earlier gs_record of the ensemble) run side by side in a warp,
+ * so an order sorted by step count keeps a warp's lanes on chains of about
+ * equal length.  Outputs as gs_solve_adaptive's, indexed by trajectory, bit
+ * for bit the same; an entry outside [0, n) is skipped (a trajectory that no
+ * entry names gets no output).  ws: device, at least GS_RECORD_INPLACE_WS
+ * bytes, 8-byte aligned (a work counter).  Not for GS_NODE64
+ * (GS_EUNSUPPORTED).
+ */
+GS_API gs_status gs_solve_adaptive_ordered(const gs_problem* prob, const gs_tol* tol, int32_t smax,
+                                           const int32_t* order, void* u_save, int32_t* nsteps, int32_t* status,
+                                           void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Fused replay + reverse sweep: for every trajectory, the loss of the

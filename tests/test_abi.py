@@ -261,3 +261,13 @@ def test_record_inplace_validation_host_only(no_launch):
     assert call(node, m64, tol, ctypes.c_void_p(16), 8) == -4
     assert call(p, _Mesh(100, 10, 16, None, 16, 16, 16, 16), tol, ctypes.c_void_p(16), 8) == -1  # no order
     assert call(_host_problem(n=0), _Mesh(100, 10, None, None, None, None, None, None), tol, None, 0) == 0
+    # the ordered adaptive solve: order and output required, workspace checked
+    osv = lambda prob, order, out, ws, nb: _lib.gs_solve_adaptive_ordered(
+        ctypes.byref(prob), ctypes.byref(tol), 100, order, out, None, None, ws, nb, None)
+    assert osv(p, None, ctypes.c_void_p(16), ctypes.c_void_p(16), 8) == -1
+    assert osv(p, ctypes.c_void_p(16), None, ctypes.c_void_p(16), 8) == -1
+    assert osv(p, ctypes.c_void_p(16), ctypes.c_void_p(16), None, 8) == -3
+    assert osv(p, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), 7) == -3
+    assert osv(p, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(12), 8) == -1
+    assert osv(node, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), 8) == -4
+    assert osv(_host_problem(n=0), None, None, None, 0) == 0

@@ -107,8 +107,9 @@ def test_lorenz_1m_shape(dtype, n):
 
 @pytest.mark.parametrize("dtype", ["f64", "f32"])
 def test_full_size_sampled(dtype):
-    """2**20 trajectories in the launch configuration the benchmark times; the
-    oracle checks a sample (random + the longest chains) one by one.  fp64
+    """2**20 trajectories in the launch configuration the benchmark times (the
+    in-place re-record rewrites the whole mesh bit for bit); the oracle checks
+    a sample (random + the longest chains) one by one.  fp64
     meshes equal the oracle's to 1e-10 (bitwise in practice); fp32 ones, of the
     fp32 instantiation of the oracle, have equal step counts on almost every
     trajectory and step sizes within fp32 rounding where they do."""
@@ -127,6 +128,13 @@ def test_full_size_sampled(dtype):
     gs.gs_record(ens, mesh, prob.rtol, prob.atol)
     torch.cuda.synchronize()
     assert (mesh.status == 0).all()
+    # the benchmark's steps re-record in place: the whole mesh, bit for bit
+    ref = [t.clone() for t in (mesh.h, mesh.order, mesh.nsteps, mesh.save_idx, mesh.status, mesh.nreject)]
+    gs.gs_record_inplace(ens, mesh, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    for a, b in zip(ref, (mesh.h, mesh.order, mesh.nsteps, mesh.save_idx, mesh.status, mesh.nreject)):
+        assert torch.equal(a, b)
+    del ref
     # mesh parity on the sample
     order = mesh.order.cpu().numpy()
     inv = np.empty_like(order)

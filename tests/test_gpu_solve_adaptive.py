@@ -123,3 +123,50 @@ def test_full_size_sampled():
     got = us[:, :, torch.tensor(idx, device=dev())].cpu().numpy()
     assert _rel(got, ref) <= 1e-10
     assert torch.isfinite(us).all()
+
+
+@pytest.mark.parametrize("name,method,dtype,dense,n,smax", [
+    ("lorenz_1m", None, "f64", False, 4099, 1024), ("lorenz_1m", None, "f64", True, 2051, 1024),
+    ("lorenz_1m", None, "f32", False, 2051, 1024), ("robertson", "ros2", "f64", False, 515, 20000),
+    ("robertson", "ros3", "f64", True, 515, 4096), ("kin8", "ros3", "f64", False, 333, 8192)])
+def test_ordered_equals_unordered(name, method, dtype, dense, n, smax):
+    """gs_solve_adaptive_ordered, in a record's slot order and in a random
+    order, returns gs_solve_adaptive's states, counts and statuses bit for
+    bit (each trajectory's arithmetic does not depend on where it runs)."""
+    prob = W.by_name(name, n=n)
+    if method:
+        prob.method = method
+    prob = prob.as_dtype(dtype)
+    ens = ensemble(prob)
+    ref = [t.cpu().numpy() for t in gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, smax, dense=dense)]
+    nst, _ = gs.gs_count(ens, prob.rtol, prob.atol, smax, dense=dense)
+    mesh = gs.new_mesh(n, int(nst.max().item()), len(prob.tsave), dtype, dev(), dense=dense)
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    rand = torch.tensor(np.random.default_rng(3).permutation(n), dtype=torch.int32, device=dev())
+    for order in (mesh.order, rand):
+        out = gs.gs_solve_adaptive_ordered(ens, prob.rtol, prob.atol, smax, order, dense=dense)
+        torch.cuda.synchronize()
+        for a, b in zip(ref, out):
+            assert np.array_equal(a, b.cpu().numpy(), equal_nan=True)
+
+
+def test_ordered_skips_bad_entries():
+    """Entries outside [0, n) are skipped: the trajectories no entry names
+    keep what their outputs held, the rest are solved."""
+    prob = W.lorenz_small(100)
+    ens = ensemble(prob)
+    ref = [t.cpu().numpy() for t in gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, 256)]
+    order = torch.arange(100, dtype=torch.int32, device=dev())
+    order[7] = -1
+    order[50] = 100
+    us = torch.full((len(prob.tsave), 3, 100), 7.0, dtype=torch.float64, device=dev())
+    ns = torch.full((100,), -5, dtype=torch.int32, device=dev())
+    st = torch.full((100,), -6, dtype=torch.int32, device=dev())
+    gs.gs_solve_adaptive_ordered(ens, prob.rtol, prob.atol, 256, order, u_save=us, nsteps=ns, status=st)
+    torch.cuda.synchronize()
+    us, ns, st = us.cpu().numpy(), ns.cpu().numpy(), st.cpu().numpy()
+    skipped = [7, 50]
+    keep = np.setdiff1d(np.arange(100), skipped)
+    assert (us[..., skipped] == 7.0).all() and (ns[skipped] == -5).all() and (st[skipped] == -6).all()
+    assert np.array_equal(us[..., keep], ref[0][..., keep]) and np.array_equal(ns[keep], ref[1][keep])
+    assert np.array_equal(st[keep], ref[2][keep])
