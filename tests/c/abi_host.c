@@ -81,10 +81,17 @@ int main(void) {
   CHECK(12, gs_record(&p, &tol, &m, (void*)16, 8, NULL) == GS_EWORKSPACE);
   gs_loss ls = {GS_LOSS_SUMSQ, NULL, NULL};
   CHECK(13, gs_grad(&p, &m, &ls, (void*)16, (void*)16, (void*)16, NULL, (void*)16, 8, NULL) == GS_EWORKSPACE);
+  /* the in-place re-record and the ordered solve need their 8-byte counter */
+  CHECK(17, gs_record_inplace(&p, &tol, &m, (void*)16, GS_RECORD_INPLACE_WS - 1, NULL) == GS_EWORKSPACE);
+  CHECK(18, gs_record_inplace(&p, &tol, &m, (void*)20, GS_RECORD_INPLACE_WS, NULL) == GS_EINVAL);
+  CHECK(19, gs_solve_adaptive_ordered(&p, &tol, 100, (const int32_t*)16, (void*)16, NULL, NULL, NULL, 0, NULL) ==
+                GS_EWORKSPACE);
+  CHECK(20, gs_solve_adaptive_ordered(&p, &tol, 100, NULL, (void*)16, NULL, NULL, (void*)16, 8, NULL) == GS_EINVAL);
   /* an empty ensemble is a no-op */
   p.n = 0;
   CHECK(14, gs_count(&p, &tol, 100, NULL, NULL, NULL) == GS_OK);
   CHECK(15, gs_grad(&p, &m, &ls, NULL, NULL, NULL, NULL, NULL, 0, NULL) == GS_OK);
+  CHECK(21, gs_record_inplace(&p, &tol, &m, NULL, 0, NULL) == GS_OK);
   CHECK(16, gs_launch_count() == before);
   printf("ok\n");
   return 0;
