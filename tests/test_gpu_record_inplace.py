@@ -152,3 +152,24 @@ def test_inplace_refusals():
     with pytest.raises(gs.gradsolve.GradsolveError) as e:
         gs.gs_record_inplace(e3, m3, p3.rtol, p3.atol, ws=torch.empty(4, dtype=torch.uint8, device=dev()))
     assert e.value.code == gs.gradsolve.GS_EWORKSPACE
+
+
+def test_inplace_capacity_failures_match_record():
+    """With a capacity below the longest chains, the trajectories that run
+    out end with GS_TRAJ_MAXSTEPS and a truncated mesh, the same bits as
+    gs_record's (and nothing is written past the capacity)."""
+    prob = _problem("lorenz_1m", None, "f64", 1000)
+    ens = ensemble(prob)
+    ns, _ = gs.gs_count(ens, prob.rtol, prob.atol, 4096)
+    cap = int(np.median(ns.cpu().numpy()))
+    mesh = gs.new_mesh(prob.n, cap, len(prob.tsave), "f64", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    ref = _arrays(mesh)
+    st = ref[4]
+    assert (st == gs.gradsolve.TRAJ_MAXSTEPS).sum() > 100 and (st == 0).sum() > 100
+    again = _clone(mesh)
+    gs.gs_record_inplace(ens, again, prob.rtol, prob.atol)
+    torch.cuda.synchronize()
+    for a, b in zip(ref, _arrays(again)):
+        assert np.array_equal(a, b)
