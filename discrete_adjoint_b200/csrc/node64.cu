@@ -945,8 +945,9 @@ __device__ __forceinline__ void ld16(uint32_t taddr, float (&v)[16]) {
 // One TMEM lane per trajectory: the products are M = 128 MMAs whose
 // accumulator row t is trajectory t's vector, so every element-wise step runs
 // on the thread that owns the lane, without shuffles or shared-memory round
-// trips.  A CTA has 256 threads; trajectory t = 32 (w mod 4) + lane is owned by
-// warps w and w + 4, which hold its components [0, 32) and [32, 64).
+// trips.  A CTA has NT threads; trajectory t = 32 (w mod 4) + lane is owned by
+// warps w, w + 4, ..., which hold its components in groups of HC (warp w + 4g:
+// [g HC, (g + 1) HC)).
 //   Z   = U W^T      M = 128 (t) x N = 64 (r) x K = 64 (k): A = U (rows t,
 //                    K = component), B = W (rows r, K = k)
 //   VJP = G W        M = 128 (t) x N = 64 (c) x K = 64 (r): A = G, B = W^T
@@ -965,9 +966,18 @@ __device__ __forceinline__ void ld16(uint32_t taddr, float (&v)[16]) {
 // ---------------------------------------------------------------------------
 namespace t128 {
 
+// Threads per CTA: 128 trajectories x NG component groups.  Trajectory t is
+// held by warps (t / 32) + 4 g, g = 0..NG-1, each with HC = 64 / NG of its
+// components, so every warp reads and writes only its own TMEM lane quarter.
+#ifndef GS_N64_NT
+#define GS_N64_NT 512
+#endif
 constexpr int TT = 128;                              // trajectories per CTA
-constexpr int NT = 256;                              // threads per CTA
-constexpr int HC = D / 2;                            // components per thread
+constexpr int NT = GS_N64_NT;                        // threads per CTA
+constexpr int NG = NT / TT;                          // component groups per trajectory
+constexpr int HC = D / NG;                           // components per thread
+constexpr int NQ = HC / 16;                          // 16-column passes per thread
+static_assert(NT % TT == 0 && (NG == 2 || NG == 4), "128 trajectories x 2 or 4 component groups");
 constexpr uint32_t kChunkT = (TT / 8) * 128;         // K-chunk stride, trajectory-row tile (B)
 constexpr uint32_t kChunkW = (D / 8) * 128;          // K-chunk stride, 64-row weight tiles (B)
 constexpr uint32_t kChunkC = (D / 8) * 128 + 16;     // K-chunk stride, component-row tiles, padded (B)
@@ -988,7 +998,7 @@ struct Smem {
   float Thi[TT * D], Tlo[TT * D];    // A operand of Z and the VJP: rows t, K = component
   float GChi[kTileC], GClo[kTileC];  // G^T of one half: rows c, K = trajectory
   float UEhi[kTileC], UElo[kTileC];  // U^T of one half: rows e, K = trajectory
-  float lpart[TT];                   // loss partials of the upper component halves
+  float lpart[NG - 1][TT];           // loss partials of component groups 1..NG-1
   unsigned long long bar;            // MMA completion
   uint32_t tmem;                     // TMEM base (512 columns)
   int failed;                        // an MMA wait ran out
@@ -1047,7 +1057,21 @@ __device__ __forceinline__ void product(SM& s, int tid, uint32_t& phase) {
   wait(s, phase);
 }
 
-__device__ __forceinline__ void load32(uint32_t taddr, float (&v)[HC]) { tc::ld32(taddr, v); }
+// this thread's HC columns of a TMEM row
+template <int N>
+__device__ __forceinline__ void load_hc(uint32_t taddr, float (&v)[N]) {
+  if constexpr (N == 32) {
+    tc::ld32(taddr, v);
+  } else {
+#pragma unroll
+    for (int q = 0; q < N / 16; ++q) {
+      float w[16];
+      ld16(taddr + 16 * q, w);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) v[16 * q + c] = w[c];
+    }
+  }
+}
 
 __device__ __forceinline__ void st16(uint32_t taddr, const float (&v)[16]) {
   asm volatile(
@@ -1100,7 +1124,7 @@ __device__ __forceinline__ void stage_in(SM& s, uint32_t tl, int t, int c0, floa
                               {TS_A61, TS_A62, TS_A63, TS_A64, TS_A65, 0, 0},
                               {TS_B1, TS_B2, TS_B3, TS_B4, TS_B5, TS_B6, 0}};
 #pragma unroll
-  for (int qh = 0; qh < 2; ++qh) {
+  for (int qh = 0; qh < NQ; ++qh) {
     float U[16], v[16];
     if (J == 1) {
 #pragma unroll
@@ -1132,7 +1156,7 @@ __device__ __forceinline__ void stage_in(SM& s, uint32_t tl, int t, int c0, floa
 __device__ __forceinline__ void stage_out(uint32_t tl, const float (&bias)[HC], int slot, float* gk = nullptr,
                                           int64_t n = 0) {
 #pragma unroll
-  for (int qh = 0; qh < 2; ++qh) {
+  for (int qh = 0; qh < NQ; ++qh) {
     float z[16], U[16];
     ld16(tl + kColAcc + 16 * qh, z);
     ld16(tl + kColSlot + 64 * (slot - 1) + 16 * qh, U);
@@ -1241,7 +1265,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   uint32_t phase = 0;
-  const uint32_t tl = s.tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0;  // lane t, this half
+  const uint32_t tl = s.tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0;  // lane t, this group
 
   // this thread's slot
   const int64_t j = base + t;
@@ -1318,9 +1342,14 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
 #pragma unroll
         for (int c = 0; c < HC; ++c) a.u_save[(int64_t)k * n64 + (int64_t)(c0 + c) * n + traj] = nan;
   } else {
-    if (hf == 1) s.lpart[t] = Lh;
+    if (hf > 0) s.lpart[hf - 1][t] = Lh;
     __syncthreads();
-    if (hf == 0 && traj >= 0) a.loss[traj] = (act && !bad0) ? Lh + s.lpart[t] : nan;
+    if (hf == 0 && traj >= 0) {
+      T L = Lh;
+#pragma unroll
+      for (int g = 0; g < NG - 1; ++g) L += s.lpart[g][t];
+      a.loss[traj] = (act && !bad0) ? L : nan;
+    }
 
     // -------------------------------------------------------------- reverse
     // u holds u_{st+1} at the top of iteration st
@@ -1356,7 +1385,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
       for (int jj = 0; jj < 6; ++jj) {
         const T* src = kj + (int64_t)st * kstep + (int64_t)jj * n64;
 #pragma unroll
-        for (int qh = 0; qh < 2; ++qh) {
+        for (int qh = 0; qh < NQ; ++qh) {
           T v[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) v[c] = run ? src[(int64_t)(16 * qh + c) * n] : cst<T>(0.0);
@@ -1374,7 +1403,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
 #pragma unroll 1
       for (int jj = 5; jj >= 0; --jj) {
 #pragma unroll
-        for (int qh = 0; qh < 2; ++qh) {
+        for (int qh = 0; qh < NQ; ++qh) {
           T nu[16], Uq[16], v[16];
           sweep_nu(tl, jj, qh, h, lam, nu);
           sweep_U(tl, jj, qh, h, u, Uq);
@@ -1403,7 +1432,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
         // the upper half of dW (its trajectories' g_j from slot j, U_j again)
         if (t >= TT / 2) {
 #pragma unroll
-          for (int qh = 0; qh < 2; ++qh) {
+          for (int qh = 0; qh < NQ; ++qh) {
             T g[16], Uq[16];
             ld16(tl + kColSlot + 64 * jj + 16 * qh, g);
             sweep_U(tl, jj, qh, h, u, Uq);
@@ -1419,7 +1448,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
         }
         // mu_j = W^T g_j - nu_j (the VJP completed at the previous wait)
 #pragma unroll
-        for (int qh = 0; qh < 2; ++qh) {
+        for (int qh = 0; qh < NQ; ++qh) {
           T nu[16], v[16];
           sweep_nu(tl, jj, qh, h, lam, nu);
           ld16(tl + kColAcc + 16 * qh, v);
@@ -1431,7 +1460,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
       }
       // lambda += ((mu_1 + mu_2) + (mu_3 + mu_4)) + (mu_5 + mu_6)
 #pragma unroll
-      for (int qh = 0; qh < 2; ++qh) {
+      for (int qh = 0; qh < NQ; ++qh) {
         T m1[16], m3[16], v[16];
         ld16(tl + kColSlot + 16 * qh, m1);
         ld16(tl + kColSlot + 64 + 16 * qh, v);
@@ -1463,7 +1492,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
     T v[HC];
 #pragma unroll
     for (int c = 0; c < HC; ++c) v[c] = cst<T>(0.0);
-    if (dw_acc && !bad) load32(s.tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kColDW + (uint32_t)c0, v);
+    if (dw_acc && !bad) load_hc(s.tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kColDW + (uint32_t)c0, v);
     if (lane < 16) {
       const int row = 16 * (warp & 3) + lane;
 #pragma unroll
@@ -1497,15 +1526,15 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
 // the tensor-core replay.  TMEM: the accumulator and seven stage slots (k_1 in
 // slot 1, k_j in slot j, k_7 in slot 7; an accepted step copies k_7 into slot
 // 1, FSAL).  Each trajectory's controller (starting step, error norm, PI
-// control, save points, statuses) runs on its lower-half thread with the
+// control, save points, statuses) runs on its group-0 thread with the
 // arithmetic of k_record_node64; the RMS norms keep the contract's sequential
-// sum over components 0..63 (the upper half's 32 scaled values pass through
+// sum over components 0..63 (the other groups' scaled values pass through
 // shared memory).
 // ---------------------------------------------------------------------------
 struct RecSmem {
   float Whi[D * D], Wlo[D * D];    // W: rows r, K = k
   float Thi[TT * D], Tlo[TT * D];  // stage operand: rows t, K = component
-  float red[HC][TT];               // upper halves' scaled values, for the norms
+  float red[D - HC][TT];           // scaled values of components HC..63, for the norms
   float hs[TT];                    // the attempt's step per trajectory
   int flag[TT];                    // per trajectory: finite start / accepted
   int sv[TT];                      // save point the accepted step reached, or -1
@@ -1515,20 +1544,20 @@ struct RecSmem {
 };
 
 // RMS of a trajectory's 64 scaled values in the contract's order: acc holds
-// the squares of components 0..31 (summed in order by the caller), red the
-// values of components 32..63.
+// the squares of components 0..HC-1 (summed in order by the caller), red the
+// values of components HC..63.
 __device__ __forceinline__ float rms_finish(const RecSmem& s, int t, float acc) {
-  for (int c = 0; c < HC; ++c) acc = fmaT(s.red[c][t], s.red[c][t], acc);
+  for (int c = 0; c < D - HC; ++c) acc = fmaT(s.red[c][t], s.red[c][t], acc);
   return sqrt(acc / cst<float>(64.0));
 }
 
-// Scaled values x_c / sc_c of this thread's components into the norm: the
-// lower half accumulates squares in order, the upper half stores its values.
+// Scaled values x_c / sc_c of this thread's components into the norm: group
+// 0 accumulates squares in order, the other groups store their values.
 __device__ __forceinline__ void norm_part(RecSmem& s, int t, int hf, int c, float r, float& acc) {
   if (hf == 0)
     acc = fmaT(r, r, acc);
   else
-    s.red[c][t] = r;
+    s.red[(hf - 1) * HC + c][t] = r;
 }
 
 // One stage of the recorder: state of stage J into the A operand and slot J,
@@ -1589,7 +1618,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
   __syncthreads();
   T acc0 = cst<T>(0.0), acc1 = cst<T>(0.0);
 #pragma unroll
-  for (int qh = 0; qh < 2; ++qh) {
+  for (int qh = 0; qh < NQ; ++qh) {
     T k[16];
     ld16(slot1 + 16 * qh, k);
 #pragma unroll
@@ -1603,7 +1632,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
   const T d0 = ctl ? rms_finish(s, t, acc0) : cst<T>(0.0);
   __syncthreads();
 #pragma unroll
-  for (int qh = 0; qh < 2; ++qh) {
+  for (int qh = 0; qh < NQ; ++qh) {
     T k[16];
     ld16(slot1 + 16 * qh, k);
 #pragma unroll
@@ -1624,7 +1653,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
   h0 = s.hs[t];
   // f(u0 + h0 f(u0)) into slot 2
 #pragma unroll
-  for (int qh = 0; qh < 2; ++qh) {
+  for (int qh = 0; qh < NQ; ++qh) {
     T k[16], U[16];
     ld16(slot1 + 16 * qh, k);
 #pragma unroll
@@ -1636,7 +1665,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
   stage_out(tl, bias, 2);
   T acc2 = cst<T>(0.0);
 #pragma unroll
-  for (int qh = 0; qh < 2; ++qh) {
+  for (int qh = 0; qh < NQ; ++qh) {
     T k[16], kb[16];
     ld16(slot1 + 16 * qh, k);
     ld16(slot2 + 16 * qh, kb);
@@ -1690,7 +1719,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
     {
       constexpr double E[7] = {TS_E1, TS_E2, TS_E3, TS_E4, TS_E5, TS_E6, TS_E7};
 #pragma unroll
-      for (int qh = 0; qh < 2; ++qh) {
+      for (int qh = 0; qh < NQ; ++qh) {
         T e[16], k[16];
         ld16(slot1 + 16 * qh, k);
 #pragma unroll
@@ -1723,7 +1752,7 @@ __global__ void __launch_bounds__(NT, 1) k_record_node64_t128(RecArgs64<float> a
     // slot 1 with its own choice: the TMEM address is the warp's)
     const bool acc_t = s.flag[t] != 0;
 #pragma unroll
-    for (int qh = 0; qh < 2; ++qh) {
+    for (int qh = 0; qh < NQ; ++qh) {
       T k1[16], k7[16];
       ld16(slot1 + 16 * qh, k1);
       ld16(slot7 + 16 * qh, k7);
