@@ -1392,6 +1392,22 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
           st16(tl + kColSlot + 64 * jj + 16 * qh, v);
         }
       }
+      // Step st - 1's rows into L2 while step st is transposed: its h, its
+      // 64 checkpoint rows and its 6 x 64 slope rows, the CTA's 128
+      // trajectories each (512 B, four 128-byte lines).  Every warp of the CTA
+      // reaches these loads at the same time, so nothing else would hide
+      // their DRAM latency.  Only lines of trajectories below n are touched.
+      if (st > 0) {
+        const int64_t sp = st - 1;
+        for (int row = tid; row < 1 + 64 + 6 * 64; row += NT) {
+          const T* r0 = row == 0 ? a.h + sp * n
+                                 : (row <= 64 ? a.ck + sp * n64 + (int64_t)(row - 1) * n
+                                              : a.kst + sp * kstep + (int64_t)(row - 65) * n);
+#pragma unroll
+          for (int l = 0; l < TT / 32; ++l)
+            if (base + 32 * l < n) asm volatile("prefetch.L2 [%0];" ::"l"(r0 + base + 32 * l));
+        }
+      }
 
       // transposed step, stages 6 .. 1:
       //   nu_j = h (b_j lambda + sum_{m>j} a_mj mu_m), g_j = nu_j (1 - y_j^2),
