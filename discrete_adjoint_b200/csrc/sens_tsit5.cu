@@ -22,25 +22,28 @@
 // holds (FSAL).
 //
 // Execution: one thread per (slot, NDIR directions).  The six directions of a
-// slot run in 6 / NDIR threads, each of which replays the state itself: the
-// state costs 192 flop a step against 252 per direction, and holding all six
-// tangents (7 slopes x 3 components x 6 directions) would not fit in
-// registers.  Consecutive blocks take the direction sets of one range of 128
-// slots (block b: slots 128 (b / G) .., direction set b % G, G = 6 / NDIR), so
-// the threads of a warp share one direction set and read consecutive elements
-// of the step-major mesh, and the G blocks of a range run side by side and
-// share those lines through L2 (the mesh crosses HBM once, not G times).  No
-// workspace: nothing is stored but the save-point sensitivities.
+// slot run in 6 / NDIR threads, each of which replays the state itself (192
+// flop a step against 252 per direction).  The default carries all six in one
+// thread (NDIR = 6: the state replays once; 7 slopes x 3 components x 6
+// tangents take the fp64 instance to 255 registers with a small spill), which
+// measured 1.66x faster than one direction per thread (2^20 Lorenz
+// trajectories: 25.6 ms against 42.4 ms; 3 directions: 28.9 ms) and 1.45-1.8x
+// for the dense and fp32 instances.  With NDIR < 6, consecutive blocks take
+// the direction sets of one range of 128 slots (block b: slots 128 (b / G) ..,
+// direction set b % G, G = 6 / NDIR), so the threads of a warp share one
+// direction set and read consecutive elements of the step-major mesh, and the
+// G blocks of a range share those lines through L2.  No workspace: nothing is
+// stored but the save-point sensitivities.
 #include "steps.cuh"
 #include "vec.cuh"
 
 namespace gs {
 
 #ifndef GS_SENS_NDIR
-#define GS_SENS_NDIR 1
+#define GS_SENS_NDIR 6
 #endif
 #ifndef GS_SENS_MINB
-#define GS_SENS_MINB 4
+#define GS_SENS_MINB (GS_SENS_NDIR == 6 ? 1 : (GS_SENS_NDIR == 1 ? 4 : 2))
 #endif
 
 template <typename T>
