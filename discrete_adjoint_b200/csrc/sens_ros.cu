@@ -27,11 +27,17 @@
 // and of df = J(u) du + f_p(u) w at both ends, evaluated on the steps that
 // hold such a save point.
 //
-// Execution: one thread per (slot, direction); the six directions of a slot
-// run in the six blocks of one range of 128 slots (block b: slots
-// 128 (b / 6) .., direction b % 6), which read the same mesh lines through
-// L2.  Six threads per slot give the latency-bound stiff replay six times the
-// warps of the gradient kernel.  No workspace.
+// Execution: one thread per (slot, ND directions), the state's step (its
+// Jacobian, LU and stages) taken once per thread and shared by its ND
+// tangent steps.  The default carries all six directions in one thread
+// (ND = 6, 251 registers, no spill): on the 65,536-trajectory Robertson
+// ensemble it measured 5.7 ms against 7.5 ms for one direction per thread
+// (ROS3; ROS2 59 against 87 ms, dense records 1.4-1.6x), the outputs bit for
+// bit the same -- six threads per slot gave the latency-bound stiff replay
+// more warps, but each replayed the state again.  With ND < 6 the directions
+// of a slot run in 6 / ND blocks of one range of 128 slots (block b: slots
+// 128 (b / G) .., direction set b % G), which read the same mesh lines
+// through L2.  No workspace.
 #include "steps.cuh"
 
 namespace gs {
@@ -93,11 +99,19 @@ __device__ __forceinline__ void djk3(const T u[3], const T p[3], const T v[3], c
   }
 }
 
-template <typename T, int SYS, int METHOD, bool DENSE>
-__global__ void __launch_bounds__(128) k_sens_ros(RosSensArgs<T> a) {
+#ifndef GS_SENS_ROS_NDIR
+#define GS_SENS_ROS_NDIR 6
+#endif
+#ifndef GS_SENS_ROS_MINB
+#define GS_SENS_ROS_MINB 1
+#endif
+
+template <typename T, int SYS, int METHOD, bool DENSE, int ND>
+__global__ void __launch_bounds__(128, GS_SENS_ROS_MINB) k_sens_ros(RosSensArgs<T> a) {
+  constexpr int G = 6 / ND;  // threads per slot
   const int64_t n = a.n;
-  const int64_t j = (int64_t)(blockIdx.x / 6) * blockDim.x + threadIdx.x;
-  const int dq = (int)(blockIdx.x % 6);  // this thread's direction
+  const int64_t j = (int64_t)(blockIdx.x / G) * blockDim.x + threadIdx.x;
+  const int dir0 = (int)(blockIdx.x % G) * ND;  // this thread's directions: dir0 .. dir0 + ND - 1
   if (j >= n) return;
   const int64_t i = a.order[j];
   if (i < 0 || i >= n) return;
@@ -105,112 +119,142 @@ __global__ void __launch_bounds__(128) k_sens_ros(RosSensArgs<T> a) {
   const int64_t n3 = 3 * n;
   const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
   auto fail = [&]() {
-    if (dq == 0) a.loss[i] = nan;
-    (dq < 3 ? a.dp : a.du0)[(dq % 3) * n + i] = nan;
-    if (a.sens)
-      for (int k = 0; k < a.nsave; ++k)
+    if (dir0 == 0) a.loss[i] = nan;
 #pragma unroll
-        for (int c = 0; c < 3; ++c) a.sens[(((int64_t)k * 3 + c) * 6 + dq) * n + i] = nan;
+    for (int q = 0; q < ND; ++q) {
+      const int dq = dir0 + q;
+      (dq < 3 ? a.dp : a.du0)[(dq % 3) * n + i] = nan;
+      if (a.sens)
+        for (int k = 0; k < a.nsave; ++k)
+#pragma unroll
+          for (int c = 0; c < 3; ++c) a.sens[(((int64_t)k * 3 + c) * 6 + dq) * n + i] = nan;
+    }
   };
   if (a.status[j] != GS_TRAJ_OK || S < 0 || S > a.smax) {
     fail();
     return;
   }
-  T p[3], u[3], v[3], w[3];
+  T p[3], u[3], v[ND][3], w[ND][3];
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
     p[c] = a.p[c * n + i];
     u[c] = a.u0[c * n + i];
-    w[c] = dq == c ? cst<T>(1.0) : cst<T>(0.0);
-    v[c] = dq == 3 + c ? cst<T>(1.0) : cst<T>(0.0);
+#pragma unroll
+    for (int q = 0; q < ND; ++q) {
+      w[q][c] = dir0 + q == c ? cst<T>(1.0) : cst<T>(0.0);
+      v[q][c] = dir0 + q == 3 + c ? cst<T>(1.0) : cst<T>(0.0);
+    }
   }
-  T L = cst<T>(0.0), dL = cst<T>(0.0);
+  T L = cst<T>(0.0), dL[ND];
+#pragma unroll
+  for (int q = 0; q < ND; ++q) dL[q] = cst<T>(0.0);
   int kk = 0, next = S > 0 ? a.save_idx[j] : -1;
   bool ok = true;
   const T* hq = a.h + j;
   for (int st = 0; st < S; ++st) {
     const T h = hq[(int64_t)st * n];
     if (st + 8 < S) prefetch_l2(hq + (int64_t)(st + 8) * n);
-    T LU[9], R[3], k1[3], vs[3], k2[3], k3[3], un[3], dun[3];
+    T LU[9], R[3], k1[3], vs[3], k2[3], k3[3], un[3], dun[ND][3];
     int P[3];
-    T r[3], t[3], df[3], dk1[3], dk2[3], dU[3];
-    if (METHOD == GS_ROS3) {
+    if (METHOD == GS_ROS3)
       ok = ros3_fwd<T, SYS>(u, p, h, LU, P, R, k1, vs, k2, k3, un) && ok;
-      jvp3<T, SYS>(u, p, v, w, df);
-      djk3<T, SYS>(u, p, v, w, k1, t);
-#pragma unroll
-      for (int c = 0; c < 3; ++c) r[c] = fmaT(h, t[c], df[c]);
-      lu3_solve(LU, P, R, r[0], r[1], r[2], dk1[0], dk1[1], dk1[2]);
-#pragma unroll
-      for (int c = 0; c < 3; ++c) dU[c] = fmaT(h, dk1[c], v[c]);
-      jvp3<T, SYS>(vs, p, dU, w, df);
-      djk3<T, SYS>(u, p, v, w, k2, t);
-#pragma unroll
-      for (int c = 0; c < 3; ++c) r[c] = fmaT(h, t[c], fmaT(cst<T>(ROS3_C21), dk1[c], df[c]));
-      lu3_solve(LU, P, R, r[0], r[1], r[2], dk2[0], dk2[1], dk2[2]);
-      T dk3[3];
-      djk3<T, SYS>(u, p, v, w, k3, t);
-#pragma unroll
-      for (int c = 0; c < 3; ++c)
-        r[c] = fmaT(h, t[c], fmaT(cst<T>(ROS3_C32), dk2[c], fmaT(cst<T>(ROS3_C31), dk1[c], df[c])));
-      lu3_solve(LU, P, R, r[0], r[1], r[2], dk3[0], dk3[1], dk3[2]);
-#pragma unroll
-      for (int c = 0; c < 3; ++c)
-        dun[c] = fmaT(h, fmaT(cst<T>(ROS3_M3), dk3[c], fmaT(cst<T>(ROS3_M2), dk2[c], dk1[c])), v[c]);
-    } else {
+    else
       ok = ros2_fwd<T, SYS>(u, p, h, LU, P, R, k1, vs, k2, un) && ok;
-      const T gh = cst<T>(ROS2_GAMMA) * h;
-      jvp3<T, SYS>(u, p, v, w, df);
-      djk3<T, SYS>(u, p, v, w, k1, t);
+    // the tangent step of each direction on the step's factors
 #pragma unroll
-      for (int c = 0; c < 3; ++c) r[c] = fmaT(gh, t[c], df[c]);
-      lu3_solve(LU, P, R, r[0], r[1], r[2], dk1[0], dk1[1], dk1[2]);
+    for (int q = 0; q < ND; ++q) {
+      T r[3], t[3], df[3], dk1[3], dk2[3], dU[3];
+      if (METHOD == GS_ROS3) {
+        jvp3<T, SYS>(u, p, v[q], w[q], df);
+        djk3<T, SYS>(u, p, v[q], w[q], k1, t);
 #pragma unroll
-      for (int c = 0; c < 3; ++c) dU[c] = fmaT(h, dk1[c], v[c]);
-      jvp3<T, SYS>(vs, p, dU, w, df);
-      djk3<T, SYS>(u, p, v, w, k2, t);
+        for (int c = 0; c < 3; ++c) r[c] = fmaT(h, t[c], df[c]);
+        lu3_solve(LU, P, R, r[0], r[1], r[2], dk1[0], dk1[1], dk1[2]);
 #pragma unroll
-      for (int c = 0; c < 3; ++c) r[c] = fmaT(gh, t[c], fmaT(cst<T>(-2.0), dk1[c], df[c]));
-      lu3_solve(LU, P, R, r[0], r[1], r[2], dk2[0], dk2[1], dk2[2]);
+        for (int c = 0; c < 3; ++c) dU[c] = fmaT(h, dk1[c], v[q][c]);
+        jvp3<T, SYS>(vs, p, dU, w[q], df);
+        djk3<T, SYS>(u, p, v[q], w[q], k2, t);
 #pragma unroll
-      for (int c = 0; c < 3; ++c) dun[c] = fmaT(h, fmaT(cst<T>(0.5), dk2[c], cst<T>(1.5) * dk1[c]), v[c]);
+        for (int c = 0; c < 3; ++c) r[c] = fmaT(h, t[c], fmaT(cst<T>(ROS3_C21), dk1[c], df[c]));
+        lu3_solve(LU, P, R, r[0], r[1], r[2], dk2[0], dk2[1], dk2[2]);
+        T dk3[3];
+        djk3<T, SYS>(u, p, v[q], w[q], k3, t);
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+          r[c] = fmaT(h, t[c], fmaT(cst<T>(ROS3_C32), dk2[c], fmaT(cst<T>(ROS3_C31), dk1[c], df[c])));
+        lu3_solve(LU, P, R, r[0], r[1], r[2], dk3[0], dk3[1], dk3[2]);
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+          dun[q][c] = fmaT(h, fmaT(cst<T>(ROS3_M3), dk3[c], fmaT(cst<T>(ROS3_M2), dk2[c], dk1[c])), v[q][c]);
+      } else {
+        const T gh = cst<T>(ROS2_GAMMA) * h;
+        jvp3<T, SYS>(u, p, v[q], w[q], df);
+        djk3<T, SYS>(u, p, v[q], w[q], k1, t);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) r[c] = fmaT(gh, t[c], df[c]);
+        lu3_solve(LU, P, R, r[0], r[1], r[2], dk1[0], dk1[1], dk1[2]);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) dU[c] = fmaT(h, dk1[c], v[q][c]);
+        jvp3<T, SYS>(vs, p, dU, w[q], df);
+        djk3<T, SYS>(u, p, v[q], w[q], k2, t);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) r[c] = fmaT(gh, t[c], fmaT(cst<T>(-2.0), dk1[c], df[c]));
+        lu3_solve(LU, P, R, r[0], r[1], r[2], dk2[0], dk2[1], dk2[2]);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) dun[q][c] = fmaT(h, fmaT(cst<T>(0.5), dk2[c], cst<T>(1.5) * dk1[c]), v[q][c]);
+      }
     }
     // save points of this step (a landing record: at most one, at its end)
     bool slopes = false;
-    T fs[3], fn[3], dfs[3], dfn[3];
+    T fs[3], fn[3];
     while (st + 1 == next) {
-      T ut[3] = {un[0], un[1], un[2]}, vt[3] = {dun[0], dun[1], dun[2]};
+      T ut[3] = {un[0], un[1], un[2]};
+      HermiteW<T> hw;
+      bool interp = false;
       if (DENSE) {
         const T th = a.theta[(int64_t)kk * n + j];
         if (th != cst<T>(1.0)) {
           if (!slopes) {
             rhs3<T, SYS>(u, p, fs);
             rhs3<T, SYS>(un, p, fn);
-            jvp3<T, SYS>(u, p, v, w, dfs);
-            jvp3<T, SYS>(un, p, dun, w, dfn);
             slopes = true;
           }
-          const HermiteW<T> hw = hermite_w(th);
+          hw = hermite_w(th);
+          interp = true;
 #pragma unroll
-          for (int c = 0; c < 3; ++c) {
-            ut[c] = hermite_c(hw, u[c], un[c], fs[c], fn[c], h);
-            vt[c] = hermite_c(hw, v[c], dun[c], dfs[c], dfn[c], h);
-          }
+          for (int c = 0; c < 3; ++c) ut[c] = hermite_c(hw, u[c], un[c], fs[c], fn[c], h);
         }
       }
       const int64_t o = (int64_t)kk * n3 + i;
+      T e[3];
 #pragma unroll
       for (int c = 0; c < 3; ++c) {
         if (a.loss_kind == GS_LOSS_SUMSQ) {
-          const T e = a.target ? ut[c] - a.target[o + c * n] : ut[c];
-          L = fmaT(e, e, L);
-          dL = fmaT(cst<T>(2.0) * e, vt[c], dL);
+          e[c] = a.target ? ut[c] - a.target[o + c * n] : ut[c];
+          L = fmaT(e[c], e[c], L);
         } else {
-          const T wc = a.weight[o + c * n];
-          L = fmaT(wc, ut[c], L);
-          dL = fmaT(wc, vt[c], dL);
+          e[c] = a.weight[o + c * n];
+          L = fmaT(e[c], ut[c], L);
         }
-        if (a.sens) a.sens[(((int64_t)kk * 3 + c) * 6 + dq) * n + i] = vt[c];
+      }
+#pragma unroll
+      for (int q = 0; q < ND; ++q) {
+        T vt[3] = {dun[q][0], dun[q][1], dun[q][2]};
+        if (DENSE && interp) {
+          T dfs[3], dfn[3];
+          jvp3<T, SYS>(u, p, v[q], w[q], dfs);
+          jvp3<T, SYS>(un, p, dun[q], w[q], dfn);
+#pragma unroll
+          for (int c = 0; c < 3; ++c) vt[c] = hermite_c(hw, v[q][c], dun[q][c], dfs[c], dfn[c], h);
+        }
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          if (a.loss_kind == GS_LOSS_SUMSQ)
+            dL[q] = fmaT(cst<T>(2.0) * e[c], vt[c], dL[q]);
+          else
+            dL[q] = fmaT(e[c], vt[c], dL[q]);
+          if (a.sens) a.sens[(((int64_t)kk * 3 + c) * 6 + dir0 + q) * n + i] = vt[c];
+        }
       }
       ++kk;
       next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
@@ -219,15 +263,20 @@ __global__ void __launch_bounds__(128) k_sens_ros(RosSensArgs<T> a) {
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
       u[c] = un[c];
-      v[c] = dun[c];
+#pragma unroll
+      for (int q = 0; q < ND; ++q) v[q][c] = dun[q][c];
     }
   }
   if (!ok) {
     fail();
     return;
   }
-  if (dq == 0) a.loss[i] = L;
-  (dq < 3 ? a.dp : a.du0)[(dq % 3) * n + i] = dL;
+  if (dir0 == 0) a.loss[i] = L;
+#pragma unroll
+  for (int q = 0; q < ND; ++q) {
+    const int dq = dir0 + q;
+    (dq < 3 ? a.dp : a.du0)[(dq % 3) * n + i] = dL[q];
+  }
 }
 
 template <typename T>
@@ -252,12 +301,16 @@ gs_status launch_sens_ros(const gs_problem* P, const gs_mesh* M, const gs_loss* 
   a.du0 = (T*)du0;
   a.sens = (T*)sens;
   a.theta = (const T*)M->save_theta;
-  const unsigned grid = (unsigned)((P->n + 127) / 128 * 6);
+  constexpr int ND = GS_SENS_ROS_NDIR;
+  static_assert(6 % ND == 0, "directions per thread must divide 6");
+  const unsigned grid = (unsigned)((P->n + 127) / 128 * (6 / ND));
   const bool rob = P->system == GS_ROBERTSON, ros3 = P->method == GS_ROS3, dense = a.theta != nullptr;
-  auto kern = rob ? (ros3 ? (dense ? k_sens_ros<T, GS_ROBERTSON, GS_ROS3, true> : k_sens_ros<T, GS_ROBERTSON, GS_ROS3, false>)
-                          : (dense ? k_sens_ros<T, GS_ROBERTSON, GS_ROS2, true> : k_sens_ros<T, GS_ROBERTSON, GS_ROS2, false>))
-                  : (ros3 ? (dense ? k_sens_ros<T, GS_LORENZ, GS_ROS3, true> : k_sens_ros<T, GS_LORENZ, GS_ROS3, false>)
-                          : (dense ? k_sens_ros<T, GS_LORENZ, GS_ROS2, true> : k_sens_ros<T, GS_LORENZ, GS_ROS2, false>));
+  auto kern = rob ? (ros3 ? (dense ? k_sens_ros<T, GS_ROBERTSON, GS_ROS3, true, ND>
+                                   : k_sens_ros<T, GS_ROBERTSON, GS_ROS3, false, ND>)
+                          : (dense ? k_sens_ros<T, GS_ROBERTSON, GS_ROS2, true, ND>
+                                   : k_sens_ros<T, GS_ROBERTSON, GS_ROS2, false, ND>))
+                  : (ros3 ? (dense ? k_sens_ros<T, GS_LORENZ, GS_ROS3, true, ND> : k_sens_ros<T, GS_LORENZ, GS_ROS3, false, ND>)
+                          : (dense ? k_sens_ros<T, GS_LORENZ, GS_ROS2, true, ND> : k_sens_ros<T, GS_LORENZ, GS_ROS2, false, ND>));
   kern<<<grid, 128, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
