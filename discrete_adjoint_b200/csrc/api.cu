@@ -50,7 +50,7 @@ gs_status node64_grad(const gs_problem*, const gs_mesh*, const gs_loss*, void*, 
 gs_status node64_solve(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 void node64_set_tensor(int on);
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize);
-size_t grad_tsit5_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave);
+size_t grad_tsit5_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave, bool dense);
 
 static size_t dsize(const gs_problem* P) { return P->dtype == GS_F64 ? 8 : 4; }
 
@@ -143,7 +143,7 @@ size_t gs_workspace_bytes(const gs_problem* P, const gs_mesh* M, int32_t op) {
     // one checkpointed state per step and slot (the Tsit5 Lorenz kernel adds
     // the save points' loss gradients)
     if (P->method == GS_TSIT5 && P->system == GS_LORENZ)
-      return grad_tsit5_lorenz_ws_bytes(P->dtype, P->n, M->smax, P->nsave);
+      return grad_tsit5_lorenz_ws_bytes(P->dtype, P->n, M->smax, P->nsave, M->save_theta != nullptr);
     return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
   }
   return 0;

@@ -313,7 +313,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   // components), instead of one lane at a time inside the step loop; the
   // values are bitwise those of the step loop.  The loss gradient at each
   // save point (2 (u - target) or the weights) goes to the workspace for the
-  // reverse half.  Save points are taken while their step counts stay in
+  // reverse half; for a dense save point its share of the adjoint at the
+  // step's two ends, which needs forward values only, is formed here too,
+  // so the reverse half just adds it.  Save points are taken while their step counts stay in
   // [1, S] and increase (landing) or do not decrease (dense); nvalid[q] counts
   // them (all of them for a well-formed mesh).
   int nvalid[K];
@@ -343,16 +345,21 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
           uy = c[n];
           uz = c[2 * n];
         }
+        // dense save point inside step sk - 1: its ends and slope weights
+        bool inside = false;
+        T xs, ys, zs, hs, ex = ux, ey = uy, ez = uz;
+        HermiteW<T> w;
         if (DENSE) {
           const T th = a.theta[(int64_t)k * n + j0 + q];
-          if (th != cst<T>(1.0)) {  // inside step sk - 1
+          if (th != cst<T>(1.0)) {
+            inside = true;
             const T* c = a.ck + (int64_t)(sk - 1) * nck + j0 + q;
-            const T xs = c[0], ys = c[n], zs = c[2 * n];
-            const T hs = hp[(int64_t)(sk - 1) * n + q];
+            xs = c[0], ys = c[n], zs = c[2 * n];
+            hs = hp[(int64_t)(sk - 1) * n + q];
             T fsx, fsy, fsz, fnx, fny, fnz;
             lorenz_f(xs, ys, zs, s.e[q], r.e[q], b.e[q], fsx, fsy, fsz);
             lorenz_f(ux, uy, uz, s.e[q], r.e[q], b.e[q], fnx, fny, fnz);
-            const HermiteW<T> w = hermite_w(th);
+            w = hermite_w(th);
             ux = hermite_c(w, xs, ux, fsx, fnx, hs);
             uy = hermite_c(w, ys, uy, fsy, fny, hs);
             uz = hermite_c(w, zs, uz, fsz, fnz, hs);
@@ -380,10 +387,43 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
           g2 = v2;
         }
         L.e[q] = Lq;
-        T* G = a.gsave + (int64_t)k * 3 * n + j0 + q;
-        G[0] = g0;
-        G[n] = g1;
-        G[2 * n] = g2;
+        if (!DENSE) {
+          T* G = a.gsave + (int64_t)k * 3 * n + j0 + q;
+          G[0] = g0;
+          G[n] = g1;
+          G[2 * n] = g2;
+        } else {
+          // The interpolant's cotangent g, split between the step's ends
+          // (it depends on forward values only, so it is formed here):
+          //   A = H01 g + J(u_sk)^T (h H11 g)      joins lambda at u_sk,
+          //   B = H00 g + J(u_sk-1)^T (h H10 g)    joins it at u_sk-1,
+          //   P = f_p(u_sk)^T (h H11 g) + f_p(u_sk-1)^T (h H10 g)  joins pbar;
+          // a save point at a step end has A = g, B = P = 0.
+          T A0 = g0, A1 = g1, A2 = g2, B0 = cst<T>(0.0), B1 = B0, B2 = B0, P0 = B0, P1 = B0, P2 = B0;
+          if (inside) {
+            T mx, my, mz;
+            lorenz_vjp(ex, ey, ez, s.e[q], r.e[q], b.e[q], (hs * w.h11) * g0, (hs * w.h11) * g1,
+                       (hs * w.h11) * g2, mx, my, mz, P0, P1, P2);
+            A0 = fmaT(w.h01, g0, mx);
+            A1 = fmaT(w.h01, g1, my);
+            A2 = fmaT(w.h01, g2, mz);
+            lorenz_vjp(xs, ys, zs, s.e[q], r.e[q], b.e[q], (hs * w.h10) * g0, (hs * w.h10) * g1,
+                       (hs * w.h10) * g2, mx, my, mz, P0, P1, P2);
+            B0 = fmaT(w.h00, g0, mx);
+            B1 = fmaT(w.h00, g1, my);
+            B2 = fmaT(w.h00, g2, mz);
+          }
+          T* G = a.gsave + (int64_t)k * 9 * n + j0 + q;
+          G[0] = A0;
+          G[n] = A1;
+          G[2 * n] = A2;
+          G[3 * n] = B0;
+          G[4 * n] = B1;
+          G[5 * n] = B2;
+          G[6 * n] = P0;
+          G[7 * n] = P1;
+          G[8 * n] = P2;
+        }
         nvalid[q] = k + 1;
       }
     }
@@ -422,7 +462,7 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     kk[q] = nvalid[q] - 1;
     next[q] = sp_idx(q, kk[q]);
     next2[q] = sp_idx(q, kk[q] - 1);
-    sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
+    if (!DENSE) sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
   }
   V cx = x, cy = y, cz = z, hc = vsplat<T, K>(cst<T>(0.0));
   V gx6 = x, gy6 = y, gz6 = z;
@@ -465,48 +505,39 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   cp_async_wait<kRingR - 1>();
   if (Smax > 0) take_r(Smax - 1);
   for (int st = Smax - 1; st >= 0; --st) {
-    // dense save points inside step st: the interpolant's cotangent g reaches
-    // u_{st+1} now (H01 g + J(u_{st+1})^T (h H11 g)) and u_st after the
-    // transposed step (H00 g + J(u_st)^T (h H10 g)), with the matching
-    // parameter terms f_p^T (.)
-    V pgx, pgy, pgz, pnx, pny, pnz;
+    // save points reached at u_{st+1}: landing ones add their loss gradient to
+    // lambda; dense ones add A now, B once step st is transposed (pgx..z) and
+    // P to pbar (the increments formed after the forward half)
+    V pgx, pgy, pgz;
     if (DENSE) {
       pgx = vsplat<T, K>(cst<T>(0.0));
-      pgy = pgx, pgz = pgx, pnx = pgx, pny = pgx, pnz = pgx;
+      pgy = pgx, pgz = pgx;
     }
 #pragma unroll
     for (int q = 0; q < K; ++q) {
       while (st + 1 == next[q]) {
-        T th = cst<T>(1.0);
-        HermiteW<T> w;
-        if (DENSE) {
-          th = a.theta[(int64_t)kk[q] * n + j0 + q];
-          if (th != cst<T>(1.0)) w = hermite_w(th);
-        }
-        const T gx = tv0[q], gy = tv1[q], gz = tv2[q];  // d loss_k / d u(t_k), from the forward half
-        if (!DENSE || th == cst<T>(1.0)) {
-          lx.e[q] += gx;
-          ly.e[q] += gy;
-          lz.e[q] += gz;
+        if (!DENSE) {
+          lx.e[q] += tv0[q];  // d loss_k / d u(t_k), from the forward half
+          ly.e[q] += tv1[q];
+          lz.e[q] += tv2[q];
         } else {
-          const T hh = hc.e[q];
-          T mx, my, mz;
-          lorenz_vjp(x.e[q], y.e[q], z.e[q], s.e[q], r.e[q], b.e[q], (hh * w.h11) * gx, (hh * w.h11) * gy,
-                     (hh * w.h11) * gz, mx, my, mz, ps.e[q], pr.e[q], pb.e[q]);
-          lx.e[q] = fmaT(w.h01, gx, lx.e[q] + mx);
-          ly.e[q] = fmaT(w.h01, gy, ly.e[q] + my);
-          lz.e[q] = fmaT(w.h01, gz, lz.e[q] + mz);
-          pgx.e[q] = fmaT(w.h00, gx, pgx.e[q]);
-          pgy.e[q] = fmaT(w.h00, gy, pgy.e[q]);
-          pgz.e[q] = fmaT(w.h00, gz, pgz.e[q]);
-          pnx.e[q] = fmaT(hh * w.h10, gx, pnx.e[q]);
-          pny.e[q] = fmaT(hh * w.h10, gy, pny.e[q]);
-          pnz.e[q] = fmaT(hh * w.h10, gz, pnz.e[q]);
+          const T* G = a.gsave + (int64_t)kk[q] * 9 * n + j0 + q;
+          if (kk[q] >= 0 && kk[q] < nvalid[q]) {
+            lx.e[q] += G[0];
+            ly.e[q] += G[n];
+            lz.e[q] += G[2 * n];
+            pgx.e[q] += G[3 * n];
+            pgy.e[q] += G[4 * n];
+            pgz.e[q] += G[5 * n];
+            ps.e[q] += G[6 * n];
+            pr.e[q] += G[7 * n];
+            pb.e[q] += G[8 * n];
+          }
         }
         --kk[q];
         next[q] = next2[q];
         next2[q] = sp_idx(q, kk[q] - 1);
-        sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
+        if (!DENSE) sp_g(q, kk[q], tv0[q], tv1[q], tv2[q]);
         if (!DENSE) break;
       }
     }
@@ -600,11 +631,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
     ly += ((m1y + m2y) + (m3y + m4y)) + (m5y + m6y);
     lz += ((m1z + m2z) + (m3z + m4z)) + (m5z + m6z);
     if (DENSE) {  // the interpolants' share of u_st
-      V qx, qy, qz;
-      lorenz_vjp(x, y, z, s, r, b, pnx, pny, pnz, qx, qy, qz, ps, pr, pb);
-      lx += pgx + qx;
-      ly += pgy + qy;
-      lz += pgz + qz;
+      lx += pgx;
+      ly += pgy;
+      lz += pgz;
     }
     // step st - 1's ring entries into registers only now, after the
     // transposed step: they are not live across it (3 fewer registers at its
@@ -636,11 +665,12 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
 #undef GS_C
 
 // Gradient workspace: checkpoint rows per step and slot (3, or 6 when U_6 is
-// kept), then [nsave][3][n] loss gradients of the landing save points.
-size_t grad_tsit5_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave) {
+// kept), then per save point the loss gradients of a landing record
+// ([nsave][3][n]) or the increments A, B, P of a dense one ([nsave][9][n]).
+size_t grad_tsit5_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave, bool dense) {
   const size_t rows = dtype == GS_F64 ? ck_rows<double>() : ck_rows<float>();
   const size_t tsize = dtype == GS_F64 ? 8 : 4;
-  return ((size_t)smax * rows + (size_t)nsave * 3) * (size_t)n * tsize;
+  return ((size_t)smax * rows + (size_t)nsave * (dense ? 9 : 3)) * (size_t)n * tsize;
 }
 
 template <typename T>

@@ -191,8 +191,9 @@ typedef struct gs_loss {
  * Workspace (scratch) bytes that op (GS_OP_RECORD / GS_OP_GRAD) needs for this
  * problem and mesh capacity: record -- step counts of the sizing pass and the
  * slot-ordering histograms; grad -- one checkpointed state per step and slot,
- * [smax][d][n] dtype (plus the d=64 weight-gradient partials).  Returns 0 for
- * an invalid request.  Host function; no device work.
+ * [smax][d][n] dtype (plus the d=64 weight-gradient partials; for Tsit5 on
+ * Lorenz plus 3 values per save point and slot, 9 for a dense mesh).  Returns
+ * 0 for an invalid request.  Host function; no device work.
  */
 GS_API size_t gs_workspace_bytes(const gs_problem* prob, const gs_mesh* mesh, int32_t op);
 
@@ -337,8 +338,9 @@ GS_API gs_status gs_sens(const gs_problem* prob, const gs_mesh* mesh, const gs_l
  * (32 MiB), which every GPU that loads the library holds until exit.
  *  - Problems whose gs_grad workspace exceeds GS_STATIC_SCRATCH_BYTES return
  *    GS_EWORKSPACE (d=3, fp64: (smax + nsave) * n <= 1,398,101 for Tsit5 on
- *    Lorenz, smax * n <= 1,398,101 for the Rosenbrock methods; e.g. 1,024
- *    trajectories of up to 1,355 steps with 10 save points).
+ *    Lorenz, (smax + 3 nsave) * n for a dense mesh, smax * n <= 1,398,101 for
+ *    the Rosenbrock methods; e.g. 1,024 trajectories of up to 1,355 steps
+ *    with 10 save points).
  *  - All calls share the array: calls that overlap on the GPU race.  It keeps
  *    the last call's contents; nothing in it needs clearing between calls.
  *  - Every call looks up the array's device address (cudaGetSymbolAddress)
