@@ -123,6 +123,13 @@ def test_full_size_sampled():
     got = us[:, :, torch.tensor(idx, device=dev())].cpu().numpy()
     assert _rel(got, ref) <= 1e-10
     assert torch.isfinite(us).all()
+    # the benchmark's form: the same solve in a record's slot order, bit for bit
+    ens = ensemble(prob)
+    mesh = gs.new_mesh(prob.n, int(ns_all.max()), len(prob.tsave), "f64", dev())
+    gs.gs_record(ens, mesh, prob.rtol, prob.atol)
+    uo, no, so = gs.gs_solve_adaptive_ordered(ens, prob.rtol, prob.atol, 2048, mesh.order)
+    torch.cuda.synchronize()
+    assert torch.equal(uo, us) and torch.equal(no, ns) and torch.equal(so, st)
 
 
 @pytest.mark.parametrize("name,method,dtype,dense,n,smax", [
