@@ -1445,7 +1445,23 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
         }
         dw_acc = 1u;
         wait(s, phase);
-        // the upper half of dW (its trajectories' g_j from slot j, U_j again)
+        // mu_j = W^T g_j - nu_j into slot j (the VJP completed at this wait)
+        auto mu_into_slot = [&]() {
+#pragma unroll
+          for (int qh = 0; qh < NQ; ++qh) {
+            T nu[16], v[16];
+            sweep_nu(tl, jj, qh, h, lam, nu);
+            ld16(tl + kColAcc + 16 * qh, v);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) v[c] = v[c] - nu[c];
+            st16(tl + kColSlot + 64 * jj + 16 * qh, v);
+          }
+        };
+        // The upper trajectory half writes its dW operands (its g_j from slot
+        // j, U_j again) while the lower half forms its mu_j; the upper half's
+        // mu_j follows while the upper dW products run.  Each thread touches
+        // only its own TMEM lane, so slot j holds g_j for the one half and
+        // mu_j for the other at the same time.
         if (t >= TT / 2) {
 #pragma unroll
           for (int qh = 0; qh < NQ; ++qh) {
@@ -1454,6 +1470,8 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
             sweep_U(tl, jj, qh, h, u, Uq);
             put_cols16(s, t - TT / 2, c0 + 16 * qh, g, Uq);
           }
+        } else {
+          mu_into_slot();
         }
         publish();
         if (tid == 0 && !s.failed) {
@@ -1462,16 +1480,7 @@ __global__ void __launch_bounds__(NT, 1) k_node64_t128(GradArgs64<float> a) {
                    tc::smem_u32(s.UElo), kChunkC, TT / 2 / 8, tc::idesc(D, D), 1u);
           commit(s);
         }
-        // mu_j = W^T g_j - nu_j (the VJP completed at the previous wait)
-#pragma unroll
-        for (int qh = 0; qh < NQ; ++qh) {
-          T nu[16], v[16];
-          sweep_nu(tl, jj, qh, h, lam, nu);
-          ld16(tl + kColAcc + 16 * qh, v);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) v[c] = v[c] - nu[c];
-          st16(tl + kColSlot + 64 * jj + 16 * qh, v);
-        }
+        if (t >= TT / 2) mu_into_slot();
         wait(s, phase);  // the upper-half dW products have read G^T / U^T
       }
       // lambda += ((mu_1 + mu_2) + (mu_3 + mu_4)) + (mu_5 + mu_6)
