@@ -241,7 +241,9 @@ GS_API gs_status gs_record(const gs_problem* prob, const gs_tol* tol, const gs_m
  *             (a work counter; gs_workspace_bytes(GS_OP_RECORD) is enough).
  * Values equal gs_record's bit for bit (each trajectory's arithmetic does not
  * depend on where it runs).  Same systems, methods and precisions as
- * gs_record except GS_NODE64 (GS_EUNSUPPORTED).
+ * gs_record except GS_NODE64 (GS_EUNSUPPORTED).  (Evolve.pub review,
+ * "Summary": the mesh stays fixed between re-records; this is the
+ * re-record.)
  */
 GS_API gs_status gs_record_inplace(const gs_problem* prob, const gs_tol* tol, const gs_mesh* mesh, void* ws,
                                    size_t ws_bytes, void* stream);
@@ -280,7 +282,8 @@ GS_API gs_status gs_solve_adaptive(const gs_problem* prob, const gs_tol* tol, in
  * for bit the same; an entry outside [0, n) is skipped (a trajectory that no
  * entry names gets no output).  ws: device, at least GS_RECORD_INPLACE_WS
  * bytes, 8-byte aligned (a work counter).  Not for GS_NODE64
- * (GS_EUNSUPPORTED).
+ * (GS_EUNSUPPORTED).  (The forward-only solver use of the GRADSOLVE
+ * abstract, as gs_solve_adaptive.)
  */
 GS_API gs_status gs_solve_adaptive_ordered(const gs_problem* prob, const gs_tol* tol, int32_t smax,
                                            const int32_t* order, void* u_save, int32_t* nsteps, int32_t* status,
