@@ -75,6 +75,10 @@ def lib():
         L.or_rhs.argtypes = [i32, i32, dp, dp, dp, dp, dp]
         L.or_tsit5_tableau.argtypes = [dp, dp, dp]
         L.or_tsit5_tableau.restype = None
+        L.or_tsit5_dense_coeffs.argtypes = [dp]
+        L.or_tsit5_dense_coeffs.restype = None
+        L.or_tsit5_dense_weights.argtypes = [i32, f64, dp]
+        L.or_tsit5_dense_weights.restype = None
         L.or_ros2_gamma.restype = f64
         L.or_ros3_coeffs.argtypes = [dp]
         L.or_ros3_coeffs.restype = None
@@ -127,7 +131,8 @@ def _check(rc: int, what: str):
 def record(prob, smax: int, h0: float = 0.0, nthreads: int | None = None, dense: bool = False) -> Mesh:
     """Adaptive record of every trajectory of ``prob`` (a ``workloads.Problem``).
     dense: steps do not stop at the save times; each save time is located inside
-    its step by theta (the mesh's ``theta``) and read off the Hermite interpolant."""
+    its step by theta (the mesh's ``theta``) and read off the step's dense output
+    (Tsit5: its own continuous extension; ROS2 / ROS3: the cubic Hermite one)."""
     L = lib()
     n, nsave = prob.n, len(prob.tsave)
     p, u0, W, ts = _f64(prob.p), _f64(prob.u0), _f64(prob.W), _f64(prob.tsave)
@@ -301,6 +306,20 @@ def tsit5_tableau():
     bt = np.zeros(7)
     lib().or_tsit5_tableau(_d(c), _d(A), _d(bt))
     return c, A, bt
+
+
+def tsit5_dense_coeffs():
+    """r[7][4] of Tsit5's continuous extension: b_i(theta) = sum_m r[i, m-1] theta^m."""
+    r = np.zeros((7, 4))
+    lib().or_tsit5_dense_coeffs(_d(r))
+    return r
+
+
+def tsit5_dense_weights(theta: float, dtype: str = "f64"):
+    """b_1(theta) .. b_7(theta) as the oracle's dense output forms them."""
+    bw = np.zeros(7)
+    lib().or_tsit5_dense_weights(1 if dtype == "f32" else 2, float(theta), _d(bw))
+    return bw
 
 
 def ros2_gamma() -> float:

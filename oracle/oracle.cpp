@@ -203,6 +203,24 @@ static const double TS_BT[7] = {-0.00178001105222577714, -0.0008164344596567469,
                                 -0.1447110071732629,     0.5823571654525552,     -0.45808210592918697,
                                 1.0 / 66.0};
 
+// Tsitouras' continuous extension of the pair, the dense output of Tsit5
+// (save times read off an interpolant instead of being stepped onto: the
+// gist.science summary of arXiv 2609.28458, "Methodology", "Dense Output";
+// the pages name no interpolant, so the method's own is the reading): the
+// state at t_s + theta h is u_s + h sum_i b_i(theta) k_i over the seven
+// stages (k_7 = f(u_{s+1})), b_i(theta) = sum_{m=1..4} TS_R[i][m-1] theta^m.
+// The values are recalled, not taken from the pages; the pins check that they
+// satisfy every fourth-order condition for all theta, equal b at theta = 1
+// and make the interpolant C1 across steps (b'(0) = e_1, b'(1) = e_7).
+static const double TS_R[7][4] = {
+    {1.0, -2.763706197274826, 2.9132554618219126, -1.0530884977290216},
+    {0.0, 0.13169999999999998, -0.2234, 0.1017},
+    {0.0, 3.9302962368947516, -5.941033872131505, 2.490627285651253},
+    {0.0, -12.411077166933676, 30.33818863028232, -16.548102889244902},
+    {0.0, 37.50931341651104, -88.1789048947664, 47.37952196281928},
+    {0.0, -27.896526289197286, 65.09189467479366, -34.87065786149660},
+    {0.0, 1.5, -4.0, 2.5}};
+
 // ROS2 (Verwer et al. 1999): gamma = 1 + 1/sqrt(2), L-stable choice.
 static const double ROS2_GAMMA = 1.7071067811865475;  // 1 + 1/sqrt(2) rounded to double
 
@@ -575,8 +593,9 @@ T ctrl_pow(T x, T y) {
 // when t reached tsave[k].  Starting step: Hairer, Norsett & Wanner I, II.4.
 // ---------------------------------------------------------------------------
 // ---------------------------------------------------------------------------
-// Dense output between the ends of one step (save points that steps do not
-// land on): the cubic Hermite interpolant on [t_s, t_s + h] at theta in (0, 1],
+// Dense output of the Rosenbrock methods between the ends of one step (save
+// points that steps do not land on): the cubic Hermite interpolant on
+// [t_s, t_s + h] at theta in (0, 1],
 //   u(theta) = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
 //   H01 = theta^2 (3 - 2 theta),  H00 = 1 - H01,
 //   H10 = theta (1 - theta)^2,    H11 = -theta^2 (1 - theta),
@@ -593,6 +612,61 @@ void hermite(int d, const S* us, const S* un, const S* fs, const S* fn, S h, dou
   const T H10 = (th * om) * om;
   const T H11 = -(t2 * om);
   for (int c = 0; c < d; ++c) out[c] = fma_(S(H00), us[c], fma_(S(H01), un[c], h * fma_(S(H10), fs[c], S(H11) * fn[c])));
+}
+
+// Tsit5's dense output at theta in (0, 1) inside a step of size h from u_s:
+// the stages are recomputed from u_s exactly as tsit5_step forms them (stage 7
+// is the step's end u_{s+1}, k_7 = f(u_{s+1})), then
+//   b_1 = fma(theta^2, P_1, theta),  b_i = theta^2 P_i (i >= 2),
+//   P_i = fma(fma(r_i4, theta, r_i3), theta, r_i2),
+//   u(theta) = fma(h, b_1 k_1 + b_2 k_2 + ... + b_7 k_7, u_s),
+// the weights in T and the sum an fma chain in increasing i.  theta is data.
+template <class T>
+void tsit5_dense_weights(T th, T* bw) {
+  const T t2 = th * th;
+  for (int i = 0; i < 7; ++i) {
+    const T P = std::fma(std::fma(T(TS_R[i][3]), th, T(TS_R[i][2])), th, T(TS_R[i][1]));
+    bw[i] = i == 0 ? std::fma(t2, P, th) : t2 * P;
+  }
+}
+
+template <class S>
+void tsit5_dense(int sys, int d, const S* us, const S* p, const S* W, S h, double theta, S* out) {
+  using T = typename base_of<S>::type;
+  T bw[7];
+  tsit5_dense_weights<T>(T(theta), bw);
+  S k[7][DMAX];
+  S U[DMAX];
+  rhs<S>(sys, us, p, W, k[0]);
+  for (int j = 1; j < 7; ++j) {
+    for (int c = 0; c < d; ++c) {
+      S acc = S(T(TS_A[j][0])) * k[0][c];
+      for (int m = 1; m < j; ++m) acc = fma_(S(T(TS_A[j][m])), k[m][c], acc);
+      U[c] = fma_(h, acc, us[c]);
+    }
+    rhs<S>(sys, U, p, W, k[j]);
+  }
+  for (int c = 0; c < d; ++c) {
+    S acc = S(bw[0]) * k[0][c];
+    for (int m = 1; m < 7; ++m) acc = fma_(S(bw[m]), k[m][c], acc);
+    out[c] = fma_(h, acc, us[c]);
+  }
+}
+
+// The dense output of a step of the given method at theta in (0, 1): Tsit5's
+// own continuous extension, the cubic Hermite interpolant for the Rosenbrock
+// methods (f evaluated at both ends).
+template <class S>
+void dense_value(int sys, int method, int d, const S* us, const S* un, const S* p, const S* W, S h, double theta,
+                 S* out) {
+  if (method == M_TSIT5) {
+    tsit5_dense<S>(sys, d, us, p, W, h, theta, out);
+    return;
+  }
+  S fs[DMAX], fn[DMAX];
+  rhs<S>(sys, us, p, W, fs);
+  rhs<S>(sys, un, p, W, fn);
+  hermite<S>(d, us, un, fs, fn, h, theta, out);
 }
 
 template <class T>
@@ -657,7 +731,7 @@ template <class T>
 RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, const T* W, T t0, T t1,
                         int nsave, const T* tsave, T rtol, T atol, T h0user, int smax, bool dense = false) {
   // dense: steps stop only at t1; a save time inside a step is located by its
-  // position theta in (0, 1] and read off the Hermite interpolant
+  // position theta in (0, 1] and read off the step's dense output
   RecordOut<T> out;
   out.save_idx.assign(nsave, 0);
   out.theta.assign(nsave, T(1));
@@ -711,10 +785,8 @@ RecordOut<T> record_one(int sys, int method, int d, const T* u0, const T* p, con
         while (kk < nsave && tsave[kk] <= t) {
           const T th = (tsave[kk] - tprev) / h;
           out.theta[kk] = th;
-          T fs[DMAX] = {}, fn[DMAX] = {}, ut[DMAX] = {};
-          rhs<T>(sys, u, p, W, fs);
-          rhs<T>(sys, un, p, W, fn);
-          hermite<T>(d, u, un, fs, fn, h, double(th), ut);
+          T ut[DMAX] = {};
+          if (th != T(1)) dense_value<T>(sys, method, d, u, un, p, W, h, double(th), ut);
           for (int c = 0; c < d; ++c) out.usave[(size_t)kk * d + c] = th == T(1) ? un[c] : ut[c];
           out.save_idx[kk++] = out.nsteps;
         }
@@ -767,10 +839,7 @@ S replay_loss(int sys, int method, int d, const S* u0, const S* p, const S* W, c
       S ut[DMAX];
       const S* uk = u;
       if (theta && theta[kk] != 1.0 && s > 0) {
-        S fs[DMAX], fn[DMAX];
-        rhs<S>(sys, up, p, W, fs);
-        rhs<S>(sys, u, p, W, fn);
-        hermite<S>(d, up, u, fs, fn, hs, theta[kk], ut);
+        dense_value<S>(sys, method, d, up, u, p, W, hs, theta[kk], ut);
         uk = ut;
       }
       for (int c = 0; c < d; ++c) {
@@ -1335,6 +1404,24 @@ int or_rhs(int sys, int d, const double* u, const double* p, const double* W, do
   rhs<double>(sys, u, p, W, f);
   if (J) jac<double>(sys, u, p, J);
   return 0;
+}
+
+// The continuous extension's coefficients for the pins: r[7][4], b_i(theta) =
+// sum_m r[i][m-1] theta^m; and its weights at theta as the dense output forms
+// them (dtype 2: double, 1: float).
+void or_tsit5_dense_coeffs(double* r) {
+  for (int i = 0; i < 7; ++i)
+    for (int m = 0; m < 4; ++m) r[i * 4 + m] = TS_R[i][m];
+}
+
+void or_tsit5_dense_weights(int dtype, double theta, double* bw) {
+  if (dtype == DT_F32) {
+    float w[7];
+    tsit5_dense_weights<float>(float(theta), w);
+    for (int i = 0; i < 7; ++i) bw[i] = w[i];
+  } else {
+    tsit5_dense_weights<double>(theta, bw);
+  }
 }
 
 // Tableau export for the order-condition pins: c[7], A[7][6], bt[7].
