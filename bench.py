@@ -65,12 +65,13 @@ WORKLOADS = {
                       desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, 10 save points with N(0,1) targets, "
                            "1 record + 10 gradient passes"),
     # the headline with dense-output save points: steps stop only at t1, each
-    # save time is read off the Hermite interpolant of its step (forward 27 and
-    # reverse ~75 flop more per save point)
-    "lorenz_1m_dense": dict(passes=10, flop_step=192 + 264, flop_save=18 + 102, kernel="k_grad_tsit5_lorenz",
+    # save time is read off Tsit5's continuous extension over its step's
+    # stages (per save point: the weights and the combination 82 flop, the
+    # transposed chain through the seven stages 281)
+    "lorenz_1m_dense": dict(passes=10, flop_step=192 + 264, flop_save=18 + 82 + 281, kernel="k_grad_tsit5_lorenz",
                             problem="lorenz_1m", dense=True, n=1 << 20, dtype="f64",
                             desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, dense record (steps do not stop at "
-                                 "the 10 save points; Hermite interpolant there) with N(0,1) targets, "
+                                 "the 10 save points; Tsit5's continuous extension there) with N(0,1) targets, "
                                  "1 record + 10 gradient passes"),
     "lorenz_small": dict(passes=1, flop_step=192 + 264, flop_save=12, kernel="k_grad_tsit5_lorenz", n=1024,
                          dtype="f64",

@@ -128,6 +128,72 @@ __device__ __forceinline__ void lorenz_vjp(const V& ux, const V& uy, const V& uz
   pb = fmaT(-uz, nz, pb);
 }
 
+// Tsit5's dense output inside one step of the Lorenz replay (a dense save
+// point at theta in (0, 1) of a step of size h from u_s to u_{s+1}).
+// Value: the stage states are recomputed from u_s as the forward forms them
+// (U[0] = u_s, U[j-1] = U_j for j = 2..6), and
+//   u(theta) = u_s + h sum_i b_i(theta) k_i,  k_7 = f(u_{s+1}).
+// Adjoint, for a cotangent g of u(theta) (theta and h are data): the slope at
+// the step's end gives nu_7 = h b_7 g and A = J(u_{s+1})^T nu_7 at u_{s+1};
+// the stage chain
+//   nu_j = h (b_j g + sum_{m=j+1..6} a_mj mu_m),  mu_j = J(U_j)^T nu_j,  j = 6..1,
+// gives B = g + sum_j mu_j at u_s; pbar gains P = sum_{j=1..7} f_p(U_j)^T nu_j.
+__host__ __device__ constexpr int ts_a_idx(int j, int m) { return (j - 2) * (j - 1) / 2 + (m - 1); }
+template <typename T>
+__device__ __forceinline__ T ts_a(int j, int m) {
+  return cst<T>(ts_lit(ts_a_idx(j, m)));
+}
+
+template <typename T>
+__device__ __forceinline__ void dense_point_lorenz(const T us[3], const T un[3], T s, T r, T b, T h, T th, T ut[3],
+                                                   T U[6][3], T bw[7]) {
+  T k[7][3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) U[0][c] = us[c];
+  lorenz_f(us[0], us[1], us[2], s, r, b, k[0][0], k[0][1], k[0][2]);
+#pragma unroll
+  for (int j = 2; j <= 6; ++j) {
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      T acc = ts_a<T>(j, 1) * k[0][c];
+#pragma unroll
+      for (int m = 2; m < j; ++m) acc = fmaT(ts_a<T>(j, m), k[m - 1][c], acc);
+      U[j - 1][c] = fmaT(h, acc, us[c]);
+    }
+    lorenz_f(U[j - 1][0], U[j - 1][1], U[j - 1][2], s, r, b, k[j - 1][0], k[j - 1][1], k[j - 1][2]);
+  }
+  lorenz_f(un[0], un[1], un[2], s, r, b, k[6][0], k[6][1], k[6][2]);
+  tsit5_dense_w(th, bw);
+#pragma unroll
+  for (int c = 0; c < 3; ++c)
+    ut[c] = tsit5_dense_c(bw, us[c], k[0][c], k[1][c], k[2][c], k[3][c], k[4][c], k[5][c], k[6][c], h);
+}
+
+template <typename T>
+__device__ __forceinline__ void dense_point_lorenz_vjp(const T U[6][3], const T un[3], T s, T r, T b, T h,
+                                                       const T bw[7], const T g[3], T A[3], T B[3], T P[3]) {
+  P[0] = P[1] = P[2] = cst<T>(0.0);
+  lorenz_vjp(un[0], un[1], un[2], s, r, b, (h * bw[6]) * g[0], (h * bw[6]) * g[1], (h * bw[6]) * g[2], A[0], A[1],
+             A[2], P[0], P[1], P[2]);
+  T mu[6][3];
+#pragma unroll
+  for (int j = 6; j >= 1; --j) {
+    T nu[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      T acc = bw[j - 1] * g[c];
+#pragma unroll
+      for (int m = 6; m > j; --m) acc = fmaT(ts_a<T>(m, j), mu[m - 1][c], acc);
+      nu[c] = h * acc;
+    }
+    lorenz_vjp(U[j - 1][0], U[j - 1][1], U[j - 1][2], s, r, b, nu[0], nu[1], nu[2], mu[j - 1][0], mu[j - 1][1],
+               mu[j - 1][2], P[0], P[1], P[2]);
+  }
+#pragma unroll
+  for (int c = 0; c < 3; ++c)
+    B[c] = g[c] + (((mu[0][c] + mu[1][c]) + (mu[2][c] + mu[3][c])) + (mu[4][c] + mu[5][c]));
+}
+
 // Stage state U = fma(h, acc, u) for the three components.
 #define GS_STAGE(UX, UY, UZ, AX, AY, AZ) \
   UX = fmaT(h, AX, x);                   \
@@ -307,8 +373,9 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
   cp_async_wait<0>();  // the reverse reuses the rows
   // Save points: u(t_k) is read off the checkpoints -- the state after step
   // save_idx[k] (the checkpoint of that step, or the final state) for a
-  // landing record, the Hermite interpolant of step save_idx[k] - 1 at theta_k
-  // on its checkpointed ends and their slopes for a dense one -- so every lane
+  // landing record, Tsit5's continuous extension over the stages of step
+  // save_idx[k] - 1 at theta_k (recomputed from its checkpoint) for a dense
+  // one -- so every lane
   // sums its loss here at once, in the contract's order (save points, then
   // components), instead of one lane at a time inside the step loop; the
   // values are bitwise those of the step loop.  The loss gradient at each
@@ -345,24 +412,24 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
           uy = c[n];
           uz = c[2 * n];
         }
-        // dense save point inside step sk - 1: its ends and slope weights
+        // dense save point inside step sk - 1: Tsit5's continuous extension
+        // over that step's stages, recomputed from its checkpoint
         bool inside = false;
-        T xs, ys, zs, hs, ex = ux, ey = uy, ez = uz;
-        HermiteW<T> w;
+        T hs = cst<T>(0.0);
+        const T un[3] = {ux, uy, uz};
+        T Us[6][3], bw[7];
         if (DENSE) {
           const T th = a.theta[(int64_t)k * n + j0 + q];
           if (th != cst<T>(1.0)) {
             inside = true;
             const T* c = a.ck + (int64_t)(sk - 1) * nck + j0 + q;
-            xs = c[0], ys = c[n], zs = c[2 * n];
+            const T us[3] = {c[0], c[n], c[2 * n]};
             hs = hp[(int64_t)(sk - 1) * n + q];
-            T fsx, fsy, fsz, fnx, fny, fnz;
-            lorenz_f(xs, ys, zs, s.e[q], r.e[q], b.e[q], fsx, fsy, fsz);
-            lorenz_f(ux, uy, uz, s.e[q], r.e[q], b.e[q], fnx, fny, fnz);
-            w = hermite_w(th);
-            ux = hermite_c(w, xs, ux, fsx, fnx, hs);
-            uy = hermite_c(w, ys, uy, fsy, fny, hs);
-            uz = hermite_c(w, zs, uz, fsz, fnz, hs);
+            T ut[3];
+            dense_point_lorenz(us, un, s.e[q], r.e[q], b.e[q], hs, th, ut, Us, bw);
+            ux = ut[0];
+            uy = ut[1];
+            uz = ut[2];
           }
         }
         T v0, v1, v2, g0, g1, g2;
@@ -393,36 +460,26 @@ __global__ void __launch_bounds__(GS_GRAD_BS, GS_GRAD_MINB) k_grad_tsit5_lorenz(
           G[n] = g1;
           G[2 * n] = g2;
         } else {
-          // The interpolant's cotangent g, split between the step's ends
-          // (it depends on forward values only, so it is formed here):
-          //   A = H01 g + J(u_sk)^T (h H11 g)      joins lambda at u_sk,
-          //   B = H00 g + J(u_sk-1)^T (h H10 g)    joins it at u_sk-1,
-          //   P = f_p(u_sk)^T (h H11 g) + f_p(u_sk-1)^T (h H10 g)  joins pbar;
-          // a save point at a step end has A = g, B = P = 0.
-          T A0 = g0, A1 = g1, A2 = g2, B0 = cst<T>(0.0), B1 = B0, B2 = B0, P0 = B0, P1 = B0, P2 = B0;
+          // The dense output's cotangent g, split between the step's ends
+          // (it depends on forward values only, so it is formed here): A
+          // joins lambda at u_sk, B at u_sk-1 and P joins pbar
+          // (dense_point_lorenz_vjp); a save point at a step end has A = g,
+          // B = P = 0.
+          T A[3] = {g0, g1, g2}, B[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)}, Pp[3] = {B[0], B[1], B[2]};
           if (inside) {
-            T mx, my, mz;
-            lorenz_vjp(ex, ey, ez, s.e[q], r.e[q], b.e[q], (hs * w.h11) * g0, (hs * w.h11) * g1,
-                       (hs * w.h11) * g2, mx, my, mz, P0, P1, P2);
-            A0 = fmaT(w.h01, g0, mx);
-            A1 = fmaT(w.h01, g1, my);
-            A2 = fmaT(w.h01, g2, mz);
-            lorenz_vjp(xs, ys, zs, s.e[q], r.e[q], b.e[q], (hs * w.h10) * g0, (hs * w.h10) * g1,
-                       (hs * w.h10) * g2, mx, my, mz, P0, P1, P2);
-            B0 = fmaT(w.h00, g0, mx);
-            B1 = fmaT(w.h00, g1, my);
-            B2 = fmaT(w.h00, g2, mz);
+            const T g[3] = {g0, g1, g2};
+            dense_point_lorenz_vjp(Us, un, s.e[q], r.e[q], b.e[q], hs, bw, g, A, B, Pp);
           }
           T* G = a.gsave + (int64_t)k * 9 * n + j0 + q;
-          G[0] = A0;
-          G[n] = A1;
-          G[2 * n] = A2;
-          G[3 * n] = B0;
-          G[4 * n] = B1;
-          G[5 * n] = B2;
-          G[6 * n] = P0;
-          G[7 * n] = P1;
-          G[8 * n] = P2;
+          G[0] = A[0];
+          G[n] = A[1];
+          G[2 * n] = A[2];
+          G[3 * n] = B[0];
+          G[4 * n] = B[1];
+          G[5 * n] = B[2];
+          G[6 * n] = Pp[0];
+          G[7 * n] = Pp[1];
+          G[8 * n] = Pp[2];
         }
         nvalid[q] = k + 1;
       }

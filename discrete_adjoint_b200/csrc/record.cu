@@ -53,7 +53,11 @@ struct RecArgs {
 
 // What a recorder pass writes besides the counts: nothing (the sizing pass),
 // the mesh, or the state at each save time (the adaptive forward-only solve).
-enum RecMode { kRecCount = 0, kRecMesh = 1, kRecSolve = 2 };
+enum RecMode { kRecCount = 0, kRecMesh = 1, kRecSolve = 2, kRecSolveDense = 3 };
+// the forward-only solve (states at the save times); kRecSolveDense reads a
+// dense record's save points off the steps' dense output, in an instance of
+// its own so that the landing solve carries none of that code
+template <int MODE> __host__ __device__ constexpr bool rec_solve() { return MODE == kRecSolve || MODE == kRecSolveDense; }
 
 template <typename T, int SYS, int METHOD>
 __device__ T initial_step_d(const T* u0, const T* p, T t0, T t1, T rtol, T atol) {
@@ -175,34 +179,35 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
     ++r.nst;
     const T tprev = r.t;
     r.t = clipped ? tstop : tn;
-    if (D == 3 && a.dense) {
+    if (D == 3 && a.dense && MODE != kRecSolve) {
       // every save time this step passed: its position inside the step, and
-      // (solve) the Hermite state there from u, f(u), u_new, f(u_new) -- for
-      // Tsit5 the slopes k1 and k7 it already holds, for the Rosenbrock
-      // methods two evaluations of f
+      // (solve) the state there -- for Tsit5 its continuous extension over
+      // the step's stages (recomputed from u and k1), for the Rosenbrock
+      // methods the Hermite interpolant from u, f(u), u_new, f(u_new)
       while (r.kk < a.nsave && a.tsave[r.kk] <= r.t) {
         const T th = (a.tsave[r.kk] - tprev) / h;
         if (MODE == kRecMesh) {
           a.save_idx[(int64_t)r.kk * n + r.o] = r.nst;
           a.theta[(int64_t)r.kk * n + r.o] = th;
         }
-        if (MODE == kRecSolve) {
-          const HermiteW<T> w = hermite_w(th);
-          T fs[D], fn[D];
-          if constexpr (METHOD == GS_TSIT5) {
+        if constexpr (MODE == kRecSolveDense) {
+          T ut[D];
 #pragma unroll
-            for (int c = 0; c < D; ++c) {
-              fs[c] = r.k1[c];
-              fn[c] = k7[c];
+          for (int c = 0; c < D; ++c) ut[c] = un[c];
+          if (th != cst<T>(1.0)) {
+            if constexpr (METHOD == GS_TSIT5) {
+              tsit5_dense3<T, SYS>(r.u, r.p, h, r.k1, th, ut);
+            } else {
+              const HermiteW<T> w = hermite_w(th);
+              T fs[D], fn[D];
+              rhs_s<T, SYS>(r.u, r.p, fs);
+              rhs_s<T, SYS>(un, r.p, fn);
+#pragma unroll
+              for (int c = 0; c < D; ++c) ut[c] = hermite_c(w, r.u[c], un[c], fs[c], fn[c], h);
             }
-          } else {
-            rhs_s<T, SYS>(r.u, r.p, fs);
-            rhs_s<T, SYS>(un, r.p, fn);
           }
 #pragma unroll
-          for (int c = 0; c < D; ++c)
-            a.u_save[((int64_t)r.kk * D + c) * n + r.i] =
-                th == cst<T>(1.0) ? un[c] : hermite_c(w, r.u[c], un[c], fs[c], fn[c], h);
+          for (int c = 0; c < D; ++c) a.u_save[((int64_t)r.kk * D + c) * n + r.i] = ut[c];
         }
         ++r.kk;
       }
@@ -214,7 +219,7 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
     }
     while (!a.dense && r.kk < a.nsave && r.t == a.tsave[r.kk]) {
       if (MODE == kRecMesh) a.save_idx[(int64_t)r.kk * n + r.o] = r.nst;
-      if (MODE == kRecSolve) {
+      if (rec_solve<MODE>()) {
 #pragma unroll
         for (int c = 0; c < D; ++c) a.u_save[((int64_t)r.kk * D + c) * n + r.i] = r.u[c];
       }
@@ -251,7 +256,7 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T, D
       if (a.dense) a.theta[(int64_t)k * n + r.o] = cst<T>(1.0);
     }
   }
-  if (MODE == kRecSolve && r.status != GS_TRAJ_OK) {
+  if (rec_solve<MODE>() && r.status != GS_TRAJ_OK) {
     // a failed trajectory has no solution: NaN at every save point
     const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
     for (int k = 0; k < a.nsave; ++k)
@@ -324,12 +329,12 @@ __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3(RecArgs<T> a) 
 // steps, and its rows zeroed up to the previous count.  The loop ends: every
 // pass takes a group from a counter that only grows, and a group's inner loop
 // advances some chain's accepted or rejected count, both capped by smax.
-// MODE kRecSolve runs the adaptive forward-only solve in the same grouped
+// MODE kRecSolve / kRecSolveDense runs the adaptive forward-only solve in the same grouped
 // order with its outputs by trajectory (an entry outside [0, n) is skipped).
 template <typename T, int SYS, int METHOD, int MODE>
 __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3_inplace(RecArgs<T> a, const int32_t* order,
                                                                          unsigned long long* next_group) {
-  static_assert(MODE == kRecMesh || MODE == kRecSolve, "grouped passes: mesh or solve");
+  static_assert(MODE == kRecMesh || rec_solve<MODE>(), "grouped passes: mesh or solve");
   const unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const int64_t n = a.n;
@@ -555,13 +560,15 @@ gs_status solve_adaptive3(const gs_problem* P, const gs_tol* tol, int32_t smax, 
     a.nsteps = nsteps;
     a.status = status;
     a.u_save = (double*)u_save;
-    return dispatch_rec<double, kRecSolve>(P->system, P->method, a, st);
+    return tol->dense ? dispatch_rec<double, kRecSolveDense>(P->system, P->method, a, st)
+                      : dispatch_rec<double, kRecSolve>(P->system, P->method, a, st);
   }
   RecArgs<float> a = rec_args<float>(P, tol, smax);
   a.nsteps = nsteps;
   a.status = status;
   a.u_save = (float*)u_save;
-  return dispatch_rec<float, kRecSolve>(P->system, P->method, a, st);
+  return tol->dense ? dispatch_rec<float, kRecSolveDense>(P->system, P->method, a, st)
+                    : dispatch_rec<float, kRecSolve>(P->system, P->method, a, st);
 }
 
 // The adaptive forward-only solve in a given trajectory order (groups of 32
@@ -574,13 +581,17 @@ gs_status solve_adaptive3_ordered(const gs_problem* P, const gs_tol* tol, int32_
     a.nsteps = nsteps;
     a.status = status;
     a.u_save = (double*)u_save;
-    return dispatch_rec_inplace<double, kRecSolve>(P->system, P->method, a, order, (unsigned long long*)ws, st);
+    unsigned long long* ctr = (unsigned long long*)ws;
+    return tol->dense ? dispatch_rec_inplace<double, kRecSolveDense>(P->system, P->method, a, order, ctr, st)
+                      : dispatch_rec_inplace<double, kRecSolve>(P->system, P->method, a, order, ctr, st);
   }
   RecArgs<float> a = rec_args<float>(P, tol, smax);
   a.nsteps = nsteps;
   a.status = status;
   a.u_save = (float*)u_save;
-  return dispatch_rec_inplace<float, kRecSolve>(P->system, P->method, a, order, (unsigned long long*)ws, st);
+  unsigned long long* ctr = (unsigned long long*)ws;
+  return tol->dense ? dispatch_rec_inplace<float, kRecSolveDense>(P->system, P->method, a, order, ctr, st)
+                    : dispatch_rec_inplace<float, kRecSolve>(P->system, P->method, a, order, ctr, st);
 }
 
 static size_t al256(size_t b) { return (b + 255) / 256 * 256; }

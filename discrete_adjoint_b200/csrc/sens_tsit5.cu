@@ -15,11 +15,12 @@
 // with dk_1 carried over from the previous step (FSAL, as k_1).
 //
 // Dense save points (a dense record: theta in (0, 1) inside a step): the
-// state there is the cubic Hermite interpolant of the step,
-//   u(theta) = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
-// theta and h data, so its tangent is the same combination of the end
-// tangents and the tangent slopes dk_1 of both ends, all of which the replay
-// holds (FSAL).
+// state there is Tsit5's continuous extension over the step's stages,
+//   u(theta) = u_s + h sum_i b_i(theta) k_i   (k_7 = f(u_{s+1})),
+// theta and h data, so its tangent is v_s + h sum_i b_i(theta) dk_i.  The
+// branch recomputes the step's stages and their tangents from (u_s, v_s),
+// which the dense instance keeps; k_7 and dk_7 are the FSAL slope and its
+// tangent the step has just formed.
 //
 // Execution: one thread per (slot, NDIR directions).  The six directions of a
 // slot run in 6 / NDIR threads, each of which replays the state itself (192
@@ -42,9 +43,23 @@ namespace gs {
 #ifndef GS_SENS_NDIR
 #define GS_SENS_NDIR 6
 #endif
-#ifndef GS_SENS_MINB
-#define GS_SENS_MINB (GS_SENS_NDIR == 6 ? 1 : (GS_SENS_NDIR == 1 ? 4 : 2))
+// directions per thread on dense meshes, and whether their save-point branch
+// is a call (1) or inlined (0)
+#ifndef GS_SENS_NDIR_DENSE
+#define GS_SENS_NDIR_DENSE GS_SENS_NDIR
 #endif
+#ifndef GS_SENS_DENSE_NOINLINE
+#define GS_SENS_DENSE_NOINLINE 1
+#endif
+#if GS_SENS_DENSE_NOINLINE
+#define GS_SENS_DENSE_FN __noinline__
+#else
+#define GS_SENS_DENSE_FN __forceinline__
+#endif
+template <int NDIR>
+constexpr int sens_minb() {
+  return NDIR == 6 ? 1 : (NDIR == 1 ? 4 : 2);
+}
 
 template <typename T>
 struct SensArgs {
@@ -101,8 +116,74 @@ __device__ __forceinline__ void lorenz_jvp(T x, T y, T z, T s, T r, T b, const V
   lorenz_f(Ux, Uy, Uz, s, r, b, KN##x, KN##y, KN##z);                 \
   lorenz_jvp(Ux, Uy, Uz, s, r, b, dUx, dUy, dUz, ws, wr, wb, d##KN##x, d##KN##y, d##KN##z);
 
+// A dense save point inside a step: Tsit5's continuous extension and its
+// tangent, from the step's stages and their tangents recomputed from
+// (u_s, v_s) with the step's own arithmetic; k_7 and dk_7 are the FSAL slope
+// and its tangent that the step has formed.  Not inlined: it runs only at
+// dense save points, and inlined into the step loop its stage tangents would
+// add to the register pressure of every step.
+template <typename T, int NDIR>
+struct DenseTanIn {
+  T x, y, z, k1x, k1y, k1z, k7x, k7y, k7z, s, r, b, h, th;
+  vec<T, NDIR> vx, vy, vz, dk1x, dk1y, dk1z, dk7x, dk7y, dk7z, ws, wr, wb;
+};
+template <typename T, int NDIR>
+struct DenseTanOut {
+  T ux, uy, uz;
+  vec<T, NDIR> tx, ty, tz;
+};
+
+template <typename T, int NDIR>
+__device__ GS_SENS_DENSE_FN DenseTanOut<T, NDIR> tsit5_dense_tangent(const DenseTanIn<T, NDIR> in) {
+  using V = vec<T, NDIR>;
+  const T x = in.x, y = in.y, z = in.z, k1x = in.k1x, k1y = in.k1y, k1z = in.k1z, s = in.s, r = in.r, b = in.b,
+          h = in.h;
+  const V vx = in.vx, vy = in.vy, vz = in.vz, dk1x = in.dk1x, dk1y = in.dk1y, dk1z = in.dk1z, ws = in.ws,
+          wr = in.wr, wb = in.wb;
+  T ax, ay, az, Ux, Uy, Uz;
+  V dax, day, daz, dUx, dUy, dUz;
+  T k2x, k2y, k2z, k3x, k3y, k3z, k4x, k4y, k4z, k5x, k5y, k5z, k6x, k6y, k6z;
+  V dk2x, dk2y, dk2z, dk3x, dk3y, dk3z, dk4x, dk4y, dk4z, dk5x, dk5y, dk5z, dk6x, dk6y, dk6z;
+  GS_S_ACC1(kTsA21, k1)
+  GS_S_STAGE(k2)
+  GS_S_ACC1(kTsA31, k1)
+  GS_S_ACCN(kTsA32, k2)
+  GS_S_STAGE(k3)
+  GS_S_ACC1(kTsA41, k1)
+  GS_S_ACCN(kTsA42, k2)
+  GS_S_ACCN(kTsA43, k3)
+  GS_S_STAGE(k4)
+  GS_S_ACC1(kTsA51, k1)
+  GS_S_ACCN(kTsA52, k2)
+  GS_S_ACCN(kTsA53, k3)
+  GS_S_ACCN(kTsA54, k4)
+  GS_S_STAGE(k5)
+  GS_S_ACC1(kTsA61, k1)
+  GS_S_ACCN(kTsA62, k2)
+  GS_S_ACCN(kTsA63, k3)
+  GS_S_ACCN(kTsA64, k4)
+  GS_S_ACCN(kTsA65, k5)
+  GS_S_STAGE(k6)
+  T bw[7];
+  tsit5_dense_w(in.th, bw);
+  DenseTanOut<T, NDIR> o;
+  o.ux = tsit5_dense_c(bw, x, k1x, k2x, k3x, k4x, k5x, k6x, in.k7x, h);
+  o.uy = tsit5_dense_c(bw, y, k1y, k2y, k3y, k4y, k5y, k6y, in.k7y, h);
+  o.uz = tsit5_dense_c(bw, z, k1z, k2z, k3z, k4z, k5z, k6z, in.k7z, h);
+#pragma unroll
+  for (int q = 0; q < NDIR; ++q) {
+    o.tx.e[q] = tsit5_dense_c(bw, vx.e[q], dk1x.e[q], dk2x.e[q], dk3x.e[q], dk4x.e[q], dk5x.e[q], dk6x.e[q],
+                              in.dk7x.e[q], h);
+    o.ty.e[q] = tsit5_dense_c(bw, vy.e[q], dk1y.e[q], dk2y.e[q], dk3y.e[q], dk4y.e[q], dk5y.e[q], dk6y.e[q],
+                              in.dk7y.e[q], h);
+    o.tz.e[q] = tsit5_dense_c(bw, vz.e[q], dk1z.e[q], dk2z.e[q], dk3z.e[q], dk4z.e[q], dk5z.e[q], dk6z.e[q],
+                              in.dk7z.e[q], h);
+  }
+  return o;
+}
+
 template <typename T, int NDIR, bool DENSE>
-__global__ void __launch_bounds__(128, GS_SENS_MINB) k_sens_tsit5_lorenz(SensArgs<T> a) {
+__global__ void __launch_bounds__(128, sens_minb<NDIR>()) k_sens_tsit5_lorenz(SensArgs<T> a) {
   using V = vec<T, NDIR>;
   const int64_t n = a.n;
   constexpr int G = 6 / NDIR;
@@ -207,16 +288,16 @@ __global__ void __launch_bounds__(128, GS_SENS_MINB) k_sens_tsit5_lorenz(SensArg
       if (DENSE) {
         const T th = a.theta[(int64_t)kk * n + j];
         if (th != cst<T>(1.0)) {
-          const HermiteW<T> w = hermite_w(th);
-          ux = hermite_c(w, xs, x, fsx, k1x, h);
-          uy = hermite_c(w, ys, y, fsy, k1y, h);
-          uz = hermite_c(w, zs, z, fsz, k1z, h);
-#pragma unroll
-          for (int q = 0; q < NDIR; ++q) {
-            tx.e[q] = hermite_c(w, vsx.e[q], vx.e[q], dfsx.e[q], dk1x.e[q], h);
-            ty.e[q] = hermite_c(w, vsy.e[q], vy.e[q], dfsy.e[q], dk1y.e[q], h);
-            tz.e[q] = hermite_c(w, vsz.e[q], vz.e[q], dfsz.e[q], dk1z.e[q], h);
-          }
+          DenseTanIn<T, NDIR> in;
+          in.x = xs, in.y = ys, in.z = zs, in.k1x = fsx, in.k1y = fsy, in.k1z = fsz;
+          in.k7x = k1x, in.k7y = k1y, in.k7z = k1z;  // f(u_{s+1}), the FSAL slope just formed
+          in.s = s, in.r = r, in.b = b, in.h = h, in.th = th;
+          in.vx = vsx, in.vy = vsy, in.vz = vsz, in.dk1x = dfsx, in.dk1y = dfsy, in.dk1z = dfsz;
+          in.dk7x = dk1x, in.dk7y = dk1y, in.dk7z = dk1z;
+          in.ws = ws, in.wr = wr, in.wb = wb;
+          const DenseTanOut<T, NDIR> dt = tsit5_dense_tangent<T, NDIR>(in);
+          ux = dt.ux, uy = dt.uy, uz = dt.uz;
+          tx = dt.tx, ty = dt.ty, tz = dt.tz;
         }
       }
       const int64_t o = (int64_t)kk * n3 + i;
@@ -287,13 +368,13 @@ gs_status launch_sens_tsit5_lorenz(const gs_problem* P, const gs_mesh* M, const 
   a.du0 = (T*)du0;
   a.sens = (T*)sens;
   a.theta = (const T*)M->save_theta;
-  constexpr int ND = GS_SENS_NDIR;
-  static_assert(6 % ND == 0, "directions per thread must divide 6");
-  const int64_t grid = (P->n + 127) / 128 * (6 / ND);
+  constexpr int ND = GS_SENS_NDIR, NDD = GS_SENS_NDIR_DENSE;
+  static_assert(6 % ND == 0 && 6 % NDD == 0, "directions per thread must divide 6");
+  const int64_t blocks = (P->n + 127) / 128;
   if (a.theta)
-    k_sens_tsit5_lorenz<T, ND, true><<<(unsigned)grid, 128, 0, st>>>(a);
+    k_sens_tsit5_lorenz<T, NDD, true><<<(unsigned)(blocks * (6 / NDD)), 128, 0, st>>>(a);
   else
-    k_sens_tsit5_lorenz<T, ND, false><<<(unsigned)grid, 128, 0, st>>>(a);
+    k_sens_tsit5_lorenz<T, ND, false><<<(unsigned)(blocks * (6 / ND)), 128, 0, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }

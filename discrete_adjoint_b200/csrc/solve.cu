@@ -64,14 +64,14 @@ __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
       T k7[3], e[3];
       tsit5_err_step<T, SYS>(u, p, h, k1, un, k7, e);
       if (a.theta) {
-        // dense save points inside this step: the Hermite state on u, f(u),
-        // u_new, f(u_new)
+        // dense save points inside this step: Tsit5's continuous extension
+        // over the step's stages, recomputed from u and k1
         while (st + 1 == next) {
           const T th = a.theta[(int64_t)kk * n + j];
-          const HermiteW<T> w = hermite_w(th);
+          T ut[3] = {un[0], un[1], un[2]};
+          if (th != cst<T>(1.0)) tsit5_dense3<T, SYS>(u, p, h, k1, th, ut);
 #pragma unroll
-          for (int c = 0; c < 3; ++c)
-            a.u_save[kk * n3 + c * n + i] = th == cst<T>(1.0) ? un[c] : hermite_c(w, u[c], un[c], k1[c], k7[c], h);
+          for (int c = 0; c < 3; ++c) a.u_save[kk * n3 + c * n + i] = ut[c];
           ++kk;
           next = kk < a.nsave ? a.save_idx[(int64_t)kk * n + j] : -1;
         }

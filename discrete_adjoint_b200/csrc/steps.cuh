@@ -115,8 +115,8 @@ __device__ T ctrl_pow(T x, T y) {
   return ctrl_exp<T>(y * ctrl_ln<T>(x));
 }
 
-// Dense output inside one step [t_s, t_s + h] at theta in (0, 1]: the cubic
-// Hermite interpolant on the end states and slopes,
+// Dense output of the Rosenbrock methods inside one step [t_s, t_s + h] at
+// theta in (0, 1]: the cubic Hermite interpolant on the end states and slopes,
 //   u = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
 // weights and combination in the floating-point contract's order (the same
 // operations as the CPU reference, so the values agree bit for bit).
@@ -139,6 +139,124 @@ __device__ __forceinline__ HermiteW<T> hermite_w(T th) {
 template <typename T>
 __device__ __forceinline__ T hermite_c(const HermiteW<T>& w, T us, T un, T fs, T fn, T h) {
   return fmaT(w.h00, us, fmaT(w.h01, un, h * fmaT(w.h10, fs, w.h11 * fn)));
+}
+
+// Tsit5's dense output: Tsitouras' continuous extension of the pair.  The
+// state at t_s + theta h is u_s + h sum_i b_i(theta) k_i over the seven
+// stages (k_7 = f(u_{s+1})), b_i(theta) = sum_m ts_r(i, m-1) theta^m, fourth
+// order for every theta, b(1) = b, and C1 across step ends.  Weights in the
+// contract's order:
+//   P_i = fma(fma(r_i4, theta, r_i3), theta, r_i2),
+//   b_1 = fma(theta^2, P_1, theta),  b_i = theta^2 P_i (i >= 2).
+__host__ __device__ constexpr double ts_r(int i, int m) {
+  constexpr double v[7][4] = {{1.0, -2.763706197274826, 2.9132554618219126, -1.0530884977290216},
+                              {0.0, 0.13169999999999998, -0.2234, 0.1017},
+                              {0.0, 3.9302962368947516, -5.941033872131505, 2.490627285651253},
+                              {0.0, -12.411077166933676, 30.33818863028232, -16.548102889244902},
+                              {0.0, 37.50931341651104, -88.1789048947664, 47.37952196281928},
+                              {0.0, -27.896526289197286, 65.09189467479366, -34.87065786149660},
+                              {0.0, 1.5, -4.0, 2.5}};
+  return v[i][m];
+}
+
+template <typename T>
+__device__ __forceinline__ void tsit5_dense_w(T th, T bw[7]) {
+  const T t2 = th * th;
+#pragma unroll
+  for (int i = 0; i < 7; ++i) {
+    const T P = fmaT(fmaT(cst<T>(ts_r(i, 3)), th, cst<T>(ts_r(i, 2))), th, cst<T>(ts_r(i, 1)));
+    bw[i] = i == 0 ? fmaT(t2, P, th) : t2 * P;
+  }
+}
+
+// u(theta) = fma(h, b_1 k_1 + ... + b_7 k_7, u_s), the sum an fma chain in
+// increasing i, for one component.
+template <typename T>
+__device__ __forceinline__ T tsit5_dense_c(const T bw[7], T us, T k1, T k2, T k3, T k4, T k5, T k6, T k7, T h) {
+  T acc = bw[0] * k1;
+  acc = fmaT(bw[1], k2, acc);
+  acc = fmaT(bw[2], k3, acc);
+  acc = fmaT(bw[3], k4, acc);
+  acc = fmaT(bw[4], k5, acc);
+  acc = fmaT(bw[5], k6, acc);
+  acc = fmaT(bw[6], k7, acc);
+  return fmaT(h, acc, us);
+}
+
+// The dense output of one Tsit5 step of size h from u (k1 = f(u)) at theta:
+// the stages recomputed in the step's own order (bitwise those of the step).
+// Not inlined: it runs only at a dense save point, and inlined into a
+// recorder loop its stages would raise the register pressure of every
+// attempt.  Arguments and result travel by value.
+template <typename T>
+struct Tri {
+  T v[3];
+};
+
+template <typename T, int SYS>
+__device__ __noinline__ Tri<T> tsit5_dense3_call(Tri<T> uu, Tri<T> pp, T h, Tri<T> kk1, T th) {
+  const T* u = uu.v;
+  const T* p = pp.v;
+  const T* k1 = kk1.v;
+  Tri<T> out;
+  T k2[3], k3[3], k4[3], k5[3], k6[3], k7[3], U[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, tsc<T, kTsA21>() * k1[c], u[c]);
+  rhs3<T, SYS>(U, p, k2);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) U[c] = fmaT(h, fmaT(tsc<T, kTsA32>(), k2[c], tsc<T, kTsA31>() * k1[c]), u[c]);
+  rhs3<T, SYS>(U, p, k3);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = tsc<T, kTsA41>() * k1[c];
+    acc = fmaT(tsc<T, kTsA42>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsA43>(), k3[c], acc);
+    U[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(U, p, k4);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = tsc<T, kTsA51>() * k1[c];
+    acc = fmaT(tsc<T, kTsA52>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsA53>(), k3[c], acc);
+    acc = fmaT(tsc<T, kTsA54>(), k4[c], acc);
+    U[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(U, p, k5);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = tsc<T, kTsA61>() * k1[c];
+    acc = fmaT(tsc<T, kTsA62>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsA63>(), k3[c], acc);
+    acc = fmaT(tsc<T, kTsA64>(), k4[c], acc);
+    acc = fmaT(tsc<T, kTsA65>(), k5[c], acc);
+    U[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(U, p, k6);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = tsc<T, kTsB1>() * k1[c];
+    acc = fmaT(tsc<T, kTsB2>(), k2[c], acc);
+    acc = fmaT(tsc<T, kTsB3>(), k3[c], acc);
+    acc = fmaT(tsc<T, kTsB4>(), k4[c], acc);
+    acc = fmaT(tsc<T, kTsB5>(), k5[c], acc);
+    acc = fmaT(tsc<T, kTsB6>(), k6[c], acc);
+    U[c] = fmaT(h, acc, u[c]);
+  }
+  rhs3<T, SYS>(U, p, k7);
+  T bw[7];
+  tsit5_dense_w(th, bw);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) out.v[c] = tsit5_dense_c(bw, u[c], k1[c], k2[c], k3[c], k4[c], k5[c], k6[c], k7[c], h);
+  return out;
+}
+
+template <typename T, int SYS>
+__device__ __forceinline__ void tsit5_dense3(const T u[3], const T p[3], T h, const T k1[3], T th, T out[3]) {
+  const Tri<T> r = tsit5_dense3_call<T, SYS>(Tri<T>{{u[0], u[1], u[2]}}, Tri<T>{{p[0], p[1], p[2]}}, h,
+                                             Tri<T>{{k1[0], k1[1], k1[2]}}, th);
+#pragma unroll
+  for (int c = 0; c < 3; ++c) out[c] = r.v[c];
 }
 
 // RMS of x / sc over D components (the error norm), in the contract's order.

@@ -130,18 +130,21 @@ typedef struct gs_problem {
  * is <= 1.  h0 > 0 fixes the first proposal; h0 = 0 picks it automatically
  * (Hairer, Norsett & Wanner I, II.4).
  * dense = 0: steps are shortened to land on every save time.  dense = 1 (the
- * d = 3 systems, every method): steps stop only at t1; a save time inside a step is located by
- * its position theta in (0, 1] (gs_mesh.save_theta) and the state there is the
- * cubic Hermite interpolant of the step on its end states and slopes,
- *   u = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
- *   H01 = theta^2 (3 - 2 theta), H00 = 1 - H01, H10 = theta (1 - theta)^2,
- *   H11 = -theta^2 (1 - theta).
- * The loss and its derivative then pass through that interpolant (theta, like
- * h, is data).  Tsit5 holds both slopes already (its first and FSAL stages);
- * the Rosenbrock methods evaluate f twice more on a step that holds an
- * interior save point.  Dense output (interpolated save times, as in the H200
- * forward-sensitivity study) prints no interpolant, so this cubic Hermite one
- * is this library's choice. */
+ * d = 3 systems, every method): steps stop only at t1; a save time inside a
+ * step is located by its position theta in (0, 1] (gs_mesh.save_theta) and the
+ * state there is read off the step's dense output:
+ *   Tsit5: its own continuous extension (Tsitouras 2011), fourth order,
+ *     u = u_s + h sum_{i=1..7} b_i(theta) k_i  (k_7 = f(u_{s+1})),
+ *     b_i(theta) a quartic in theta with b_i(0) = 0, b_i(1) = b_i;
+ *   ROS2, ROS3: the cubic Hermite interpolant on the end states and slopes,
+ *     u = H00 u_s + H01 u_{s+1} + h (H10 f(u_s) + H11 f(u_{s+1})),
+ *     H01 = theta^2 (3 - 2 theta), H00 = 1 - H01, H10 = theta (1 - theta)^2,
+ *     H11 = -theta^2 (1 - theta).
+ * The loss and its derivative then pass through that dense output (theta,
+ * like h, is data).  Dense output (save times interpolated instead of
+ * stepped onto: the gist.science summary of arXiv 2609.28458, "Methodology",
+ * "Dense Output") names no interpolant; the method's own is the reading for
+ * Tsit5, and the Rosenbrock methods take the Hermite one. */
 typedef struct gs_tol {
   double rtol, atol, h0;
   int32_t dense;
@@ -324,7 +327,7 @@ GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_l
  * turns singular) get NaN everywhere.  Built for GS_LORENZ with GS_TSIT5, and
  * for GS_LORENZ and GS_ROBERTSON with GS_ROS2 or GS_ROS3 (np + d = 6), fp64
  * and fp32, on landing and dense meshes (at a dense save point the matrix is
- * the tangent of the Hermite interpolant); for GS_KIN8 with GS_ROS2 or
+ * the tangent of the step's dense output); for GS_KIN8 with GS_ROS2 or
  * GS_ROS3 (np + d = 16) on landing meshes; other problems return
  * GS_EUNSUPPORTED.  (The few-parameter forward-sensitivity
  * route that the gptget summary sets beside the adjoint.)

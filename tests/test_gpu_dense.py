@@ -1,5 +1,5 @@
 """GPU <-> oracle parity for dense-output save points (steps that do not stop
-at the save times; the state there read off the cubic Hermite interpolant):
+at the save times; the state there read off Tsit5's continuous extension):
 the dense record (step counts, step sizes and save-point positions), the
 replay and the adaptive forward-only solve, and the gradient through the
 interpolant, on Lorenz with Tsit5 (ten save points strictly inside steps)."""
@@ -99,7 +99,7 @@ def test_dense_linear_loss_and_own_mesh(case):
 
 def test_dense_sensitivities(case):
     """Forward sensitivities on the dense mesh: at each save point the tangent
-    of the Hermite interpolant, against the oracle's dual numbers on the same
+    of the continuous extension, against the oracle's dual numbers on the same
     mesh, and the loss gradient equal to the adjoint's."""
     prob, om = case
     sub = prob.subset(np.arange(256))
