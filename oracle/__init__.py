@@ -30,7 +30,7 @@ _SRC = os.path.join(_HERE, "oracle.cpp")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 SYSTEMS = {"lorenz": 1, "robertson": 2, "hires": 3, "node64": 4, "linear": 5, "kin8": 6}
-METHODS = {"tsit5": 1, "ros2": 2, "ros3": 3}
+METHODS = {"tsit5": 1, "ros2": 2, "ros3": 3, "vern7": 4}
 DTYPES = {"f32": 1, "f64": 2}
 LOSSES = {"sumsq": 1, "linear": 2}
 
@@ -75,6 +75,8 @@ def lib():
         L.or_rhs.argtypes = [i32, i32, dp, dp, dp, dp, dp]
         L.or_tsit5_tableau.argtypes = [dp, dp, dp]
         L.or_tsit5_tableau.restype = None
+        L.or_vern7_tableau.argtypes = [dp, dp, dp, dp]
+        L.or_vern7_tableau.restype = None
         L.or_tsit5_dense_coeffs.argtypes = [dp]
         L.or_tsit5_dense_coeffs.restype = None
         L.or_tsit5_dense_weights.argtypes = [i32, f64, dp]
@@ -306,6 +308,13 @@ def tsit5_tableau():
     bt = np.zeros(7)
     lib().or_tsit5_tableau(_d(c), _d(A), _d(bt))
     return c, A, bt
+
+
+def vern7_tableau():
+    """Verner's 7(6) pair as the oracle holds it: c[10], A[10][9], b[10], bhat[10]."""
+    c, A, b, bh = np.zeros(10), np.zeros((10, 9)), np.zeros(10), np.zeros(10)
+    lib().or_vern7_tableau(_d(c), _d(A), _d(b), _d(bh))
+    return c, A, b, bh
 
 
 def tsit5_dense_coeffs():

@@ -23,10 +23,11 @@
 //              an independent second route to the same derivative.
 //   flops      a counting scalar (S = Cn) to count the replay's operations.
 //
-// Integrators: Tsitouras' 5(4) pair (Tsit5, Tsitouras 2011), the
-// second-order Rosenbrock method ROS2 of Verwer, Spee, Blom & Hundsdorfer
-// (1999) with gamma = 1 + 1/sqrt(2), and the third-order Rosenbrock method
-// ROS3 of Sandu, Verwer, Blom, Spee, Carmichael & Potra (1997).  Systems: Lorenz (DiffEqGPU "ad" example,
+// Integrators: Tsitouras' 5(4) pair (Tsit5, Tsitouras 2011), Verner's 7(6)
+// pair (Verner 2010), the second-order Rosenbrock method ROS2 of Verwer,
+// Spee, Blom & Hundsdorfer (1999) with gamma = 1 + 1/sqrt(2), and the
+// third-order Rosenbrock method ROS3 of Sandu, Verwer, Blom, Spee, Carmichael
+// & Potra (1997).  Systems: Lorenz (DiffEqGPU "ad" example,
 // "Forward-mode automatic differentiation" listing), Robertson kinetics
 // (mass-action form of the reaction scheme A->B (k1), 2B->B+C (k2),
 // B+C->A+C (k3)), the d=64 shared-weight system tanh(W u + b) - u, and kin8,
@@ -182,7 +183,7 @@ template <> struct base_of<Cn> { using type = double; };
 // Method constants.
 // ---------------------------------------------------------------------------
 enum { SYS_LORENZ = 1, SYS_ROBERTSON = 2, SYS_HIRES = 3, SYS_NODE64 = 4, SYS_LINEAR = 5, SYS_KIN8 = 6 };
-enum { M_TSIT5 = 1, M_ROS2 = 2, M_ROS3 = 3 };
+enum { M_TSIT5 = 1, M_ROS2 = 2, M_ROS3 = 3, M_VERN7 = 4 };
 enum { DT_F32 = 1, DT_F64 = 2 };
 enum { LOSS_SUMSQ = 1, LOSS_LINEAR = 2 };
 enum { TRAJ_OK = 0, TRAJ_MAXSTEPS = 1, TRAJ_DTMIN = 2, TRAJ_NONFINITE = 3, TRAJ_SINGULAR = 4 };
@@ -242,9 +243,43 @@ static const double ROS3_E1 = 0.5;
 static const double ROS3_E2 = -2.907955871680547;
 static const double ROS3_E3 = 0.2235406989781157;
 
+// Verner's 7(6) pair (J. H. Verner, "Numerically optimal Runge-Kutta pairs
+// with interpolants", Numer. Algorithms 53 (2010); its "most efficient" 7(6)
+// pair): ten stages, the seventh-order weights b on stages 1 and 4..9, the
+// sixth-order embedded weights bhat on 1, 4..7 and 10 (stage 10 serves only
+// the error estimate; the pair is not FSAL).  Row j of V7_A holds a_{j+1, m+1}
+// (zeros where the pair has none).  The values are recalled, not taken from
+// the pages (the gist.science summary of arXiv 2609.28458, "Results", names
+// "Verner 7" beside Tsit5 as the methods compared); the pins check every
+// order condition up to order 7 for b and 6 for bhat from these values.
+static const double V7_C[10] = {0.0, 0.005, 0.10888888888888888, 0.16333333333333333, 0.4555,
+                                0.6095094489978381, 0.884, 0.925, 1.0, 1.0};
+static const double V7_A[10][9] = {
+    {0, 0, 0, 0, 0, 0, 0, 0, 0},
+    {0.005, 0, 0, 0, 0, 0, 0, 0, 0},
+    {-1.07679012345679, 1.185679012345679, 0, 0, 0, 0, 0, 0, 0},
+    {0.04083333333333333, 0, 0.1225, 0, 0, 0, 0, 0, 0},
+    {0.6389139236255726, 0, -2.455672638223657, 2.272258714598084, 0, 0, 0, 0, 0},
+    {-2.6615773750187572, 0, 10.804513886456137, -8.3539146573962, 0.820487594956657, 0, 0, 0, 0},
+    {6.067741434696772, 0, -24.711273635911088, 20.427517930788895, -1.9061579788166472, 1.006172249242068, 0, 0,
+     0},
+    {12.054670076253203, 0, -49.75478495046899, 41.142888638604674, -4.461760149974004, 2.042334822239175,
+     -0.09834843665406107, 0, 0},
+    {10.138146522881808, 0, -42.6411360317175, 35.76384003992257, -4.3480228403929075, 2.0098622683770357,
+     0.3487490460338272, -0.27143900510483127, 0},
+    {-45.030072034298676, 0, 187.3272437654589, -154.02882369350186, 18.56465306347536, -7.141809679295079,
+     1.3088085781613787, 0, 0}};
+static const double V7_B[10] = {0.04715561848627222, 0, 0, 0.25750564298434153, 0.26216653977412624,
+                                0.15216092656738558, 0.4939969170032485, -0.29430311714032503,
+                                0.08131747232495111, 0};
+static const double V7_BH[10] = {0.044608606606341174, 0, 0, 0.26716403785713727, 0.22010183001772932,
+                                 0.2188431703143157, 0.22898717054112028, 0, 0, 0.02029518466335628};
+
 // Error order q of the step-size controller: the local error estimate of
-// Tsit5 is O(h^5), of ROS2 O(h^2), of ROS3 O(h^3).
-inline int method_order(int method) { return method == M_TSIT5 ? 5 : (method == M_ROS3 ? 3 : 2); }
+// Tsit5 is O(h^5), of ROS2 O(h^2), of ROS3 O(h^3), of Verner's 7(6) pair O(h^7).
+inline int method_order(int method) {
+  return method == M_TSIT5 ? 5 : (method == M_ROS3 ? 3 : (method == M_VERN7 ? 7 : 2));
+}
 
 constexpr int DMAX = 64;
 
@@ -508,11 +543,54 @@ bool ros3_step(int sys, int d, const S* u, const S* p, S h, S* unew, S* err) {
   return true;
 }
 
+// One step of Verner's 7(6) pair of size h from u.  Stage j state:
+// acc = a_j1 k1, then acc = fma(a_jm, k_m, acc) over the nonzero a_jm in
+// increasing m, U_j = fma(h, acc, u); u_new the same over the nonzero b_m.
+// If err != nullptr, stage 10 is formed too and the embedded error is
+// e = h * (E_1 k_1 + sum over the nonzero E_m, increasing m), E = b - bhat
+// (each a double difference of the two stored weights).
+template <class S>
+void vern7_step(int sys, int d, const S* u, const S* p, const S* W, S h, S* unew, S* err) {
+  using T = typename base_of<S>::type;
+  S k[10][DMAX];
+  S U[DMAX];
+  rhs<S>(sys, u, p, W, k[0]);
+  const int nst = err ? 10 : 9;
+  for (int j = 1; j < nst; ++j) {
+    for (int c = 0; c < d; ++c) {
+      S acc = S(T(V7_A[j][0])) * k[0][c];
+      for (int m = 1; m < j; ++m)
+        if (V7_A[j][m] != 0.0) acc = fma_(S(T(V7_A[j][m])), k[m][c], acc);
+      U[c] = fma_(h, acc, u[c]);
+    }
+    rhs<S>(sys, U, p, W, k[j]);
+  }
+  for (int c = 0; c < d; ++c) {
+    S acc = S(T(V7_B[0])) * k[0][c];
+    for (int m = 1; m < 9; ++m)
+      if (V7_B[m] != 0.0) acc = fma_(S(T(V7_B[m])), k[m][c], acc);
+    unew[c] = fma_(h, acc, u[c]);
+  }
+  if (!err) return;
+  for (int c = 0; c < d; ++c) {
+    S acc = S(T(V7_B[0] - V7_BH[0])) * k[0][c];
+    for (int m = 1; m < 10; ++m) {
+      const double e = V7_B[m] - V7_BH[m];
+      if (e != 0.0) acc = fma_(S(T(e)), k[m][c], acc);
+    }
+    err[c] = h * acc;
+  }
+}
+
 // One step of the given method (Tsit5 never fails).
 template <class S>
 bool method_step(int sys, int method, int d, const S* u, const S* p, const S* W, S h, S* unew, S* err) {
   if (method == M_TSIT5) {
     tsit5_step<S>(sys, d, u, p, W, h, unew, err);
+    return true;
+  }
+  if (method == M_VERN7) {
+    vern7_step<S>(sys, d, u, p, W, h, unew, err);
     return true;
   }
   if (method == M_ROS3) return ros3_step<S>(sys, d, u, p, h, unew, err);
@@ -1048,9 +1126,10 @@ int check_prob(const Prob& P) {
   if (P.sys == SYS_LINEAR && (P.d != 1 || P.np != 1)) return -1;
   if (P.sys == SYS_KIN8 && (P.d != 8 || P.np != 8)) return -1;
   if (P.sys < 1 || P.sys > 6) return -1;
-  if (P.method != M_TSIT5 && P.method != M_ROS2 && P.method != M_ROS3) return -1;
+  if (P.method != M_TSIT5 && P.method != M_ROS2 && P.method != M_ROS3 && P.method != M_VERN7) return -1;
   if (P.method != M_TSIT5 && P.d > 8) return -4;
   if (P.method != M_TSIT5 && P.sys == SYS_NODE64) return -4;
+  if (P.method == M_VERN7 && P.sys == SYS_KIN8) return -4;
   if (P.dtype != DT_F32 && P.dtype != DT_F64) return -1;
   return 0;
 }
@@ -1404,6 +1483,17 @@ int or_rhs(int sys, int d, const double* u, const double* p, const double* W, do
   rhs<double>(sys, u, p, W, f);
   if (J) jac<double>(sys, u, p, J);
   return 0;
+}
+
+// Verner 7(6) tableau export for the order-condition pins: c[10], A[10][9],
+// b[10], bhat[10].
+void or_vern7_tableau(double* c, double* A, double* b, double* bh) {
+  for (int i = 0; i < 10; ++i) {
+    c[i] = V7_C[i];
+    b[i] = V7_B[i];
+    bh[i] = V7_BH[i];
+    for (int j = 0; j < 9; ++j) A[i * 9 + j] = V7_A[i][j];
+  }
 }
 
 // The continuous extension's coefficients for the pins: r[7][4], b_i(theta) =

@@ -33,12 +33,18 @@ def _ros3(prob):
     return prob
 
 
+def _vern7(prob):
+    prob.method = "vern7"
+    return prob
+
+
 CASES = {
     "lorenz_small": lambda: W.lorenz_small(48),
     "lorenz_1m": lambda: W.lorenz_1m(24),
     "robertson": lambda: W.robertson(8),
     "robertson_ros3": lambda: _ros3(W.robertson(8)),
     "lorenz_ros3": lambda: _ros3(W.lorenz_small(16)),
+    "lorenz_vern7": lambda: _vern7(W.lorenz_small(16)),
 }
 
 
@@ -86,7 +92,7 @@ def test_fused_tape_matches_dual(recorded, case):
         assert not np.array_equal(gf["du0"], gt["du0"])
 
 
-@pytest.mark.parametrize("case", ["lorenz_small", "robertson", "robertson_ros3"])
+@pytest.mark.parametrize("case", ["lorenz_small", "robertson", "robertson_ros3", "lorenz_vern7"])
 def test_tape_matches_fixed_mesh_fd(recorded, case):
     prob, mesh = recorded[case]
     prob = prob.subset(range(4))

@@ -14,7 +14,13 @@
 * ROS3: the same closed-form adjoint, with R(z) = 1 + z b^T (I - z beta)^{-1} 1
   of the standard Rosenbrock form recovered from the oracle's transformed-form
   coefficients (the coefficient pins themselves are in test_oracle_ros3.py).
+* Verner's 7(6) pair: every order condition (all rooted trees up to order 7,
+  generated here, in exact rationals of the stored doubles) for b, up to
+  order 6 for the embedded weights, which fail at order 7; c = A 1; its step
+  on u' = p u equals R(z) = 1 + z b^T (I - z A)^{-1} 1; the same closed-form
+  adjoint.
 """
+import itertools
 import os
 from fractions import Fraction as Fr
 from math import factorial
@@ -71,6 +77,112 @@ def test_tsit5_order_conditions():
     assert len(res4) == 8 and max(res4) <= 8 * EPS
     # the pair really is 5(4): the embedded weights fail a fifth-order condition
     assert max(abs(v - t) for v, t in _conditions(A, c, bhat, 5)[8:]) > 1e-4
+
+
+# ---- Verner's 7(6) pair -------------------------------------------------------
+def _rooted_trees(order):
+    """All rooted trees with ``order`` nodes, each a sorted tuple of its
+    subtrees (unlabelled, so each tree appears once)."""
+    if order == 1:
+        return [()]
+    out = set()
+
+    def partitions(n, largest):
+        if n == 0:
+            yield []
+            return
+        for k in range(min(n, largest), 0, -1):
+            for rest in partitions(n - k, k):
+                yield [k] + rest
+
+    for part in partitions(order - 1, order - 1):
+        for kids in itertools.product(*[_rooted_trees(k) for k in part]):
+            out.add(tuple(sorted(kids)))
+    return sorted(out)
+
+
+def _tree_gamma(t):
+    n = 1 + sum(_tree_size(k) for k in t)
+    g = n
+    for k in t:
+        g *= _tree_gamma(k)
+    return g
+
+
+def _tree_size(t):
+    return 1 + sum(_tree_size(k) for k in t)
+
+
+def _elementary_weight(A, t):
+    """Phi_i(t) = prod over the subtrees u of (A Phi(u))_i."""
+    s = len(A)
+    v = [Fr(1)] * s
+    for k in t:
+        pk = _elementary_weight(A, k)
+        Apk = [sum(A[i][j] * pk[j] for j in range(s)) for i in range(s)]
+        v = [v[i] * Apk[i] for i in range(s)]
+    return v
+
+
+def _vern7_exact():
+    c, A9, b, bh = oracle.vern7_tableau()
+    A = [[Fr(float(A9[i, j])) if j < 9 else Fr(0) for j in range(10)] for i in range(10)]
+    return [Fr(float(x)) for x in c], A, [Fr(float(x)) for x in b], [Fr(float(x)) for x in bh]
+
+
+def test_vern7_row_sums_and_tree_count():
+    c, A, b, bh = _vern7_exact()
+    for i in range(10):
+        assert abs(float(sum(A[i]) - c[i])) <= 4 * EPS * sum(abs(float(x)) for x in A[i]), i
+    # 1, 1, 2, 4, 9, 20, 48 trees of orders 1..7 (85 conditions in all)
+    assert [len(_rooted_trees(k)) for k in range(1, 8)] == [1, 1, 2, 4, 9, 20, 48]
+
+
+def test_vern7_order_conditions():
+    c, A, b, bh = _vern7_exact()
+    worst_b7 = worst_bh6 = 0.0
+    worst_bh7 = 0.0
+    for order in range(1, 8):
+        for t in _rooted_trees(order):
+            phi = _elementary_weight(A, t)
+            want = Fr(1, _tree_gamma(t))
+            for w, kind in ((b, "b"), (bh, "bh")):
+                got = sum(w[i] * phi[i] for i in range(10))
+                mag = float(sum(abs(w[i] * phi[i]) for i in range(10)))
+                rel = abs(float(got - want)) / mag
+                if kind == "b":
+                    worst_b7 = max(worst_b7, rel)
+                elif order <= 6:
+                    worst_bh6 = max(worst_bh6, rel)
+                else:
+                    worst_bh7 = max(worst_bh7, rel)
+    assert worst_b7 <= 32 * EPS, worst_b7        # seventh order
+    assert worst_bh6 <= 64 * EPS, worst_bh6      # sixth-order embedded weights
+    assert worst_bh7 > 1e-3, worst_bh7           # ... and not seventh
+
+
+def _vern7_R_coeffs():
+    """R(z) = 1 + sum_k z^(k+1) b^T A^k 1 (A strictly lower triangular)."""
+    c, A, b, bh = _vern7_exact()
+    v = [Fr(1)] * 10
+    co = [Fr(1)]
+    for _ in range(10):
+        co.append(sum(b[i] * v[i] for i in range(10)))
+        v = [sum(A[i][j] * v[j] for j in range(10)) for i in range(10)]
+    return co
+
+
+def test_vern7_stability_function():
+    co = _vern7_R_coeffs()
+    # seventh order: R agrees with exp to z^7
+    assert all(abs(float(co[k] - Fr(1, factorial(k)))) <= 16 * EPS for k in range(8))
+    assert abs(float(co[8] - Fr(1, factorial(8)))) > 1e-9
+    # one oracle step on u' = p u multiplies u by R(p h)
+    for z in [-3.0, -1.0, -0.25, 0.1, 0.5]:
+        un, e, ok = oracle.step("linear", "vern7", "f64", np.array([1.0]), np.array([z]), 1.0)
+        R = float(_poly(co, Fr(z)))
+        terms = float(_poly([abs(x) for x in co], Fr(abs(z))))
+        assert abs(un[0] - R) <= 64 * EPS * terms, (z, un[0], R)
 
 
 def _golden():
@@ -182,9 +294,12 @@ def _ros3_R(z):
 
 
 def _R_any(method, z):
-    """(R, R') of Tsit5, ROS2 or ROS3 at z, exact."""
+    """(R, R') of Tsit5, Verner 7, ROS2 or ROS3 at z, exact."""
     if method == "tsit5":
         co = _tsit5_R_coeffs()
+        return _poly(co, z), _dpoly(co, z)
+    if method == "vern7":
+        co = _vern7_R_coeffs()
         return _poly(co, z), _dpoly(co, z)
     if method == "ros3":
         return _ros3_R(z)
@@ -223,9 +338,10 @@ def _kappa(method, p, hs):
     co = [float(x) for x in _tsit5_R_coeffs()]
     for h in hs:
         z = p * h
-        if method == "tsit5":
-            terms = sum(abs(a) * abs(z) ** k for k, a in enumerate(co))
-            R = sum(a * z**k for k, a in enumerate(co))
+        if method in ("tsit5", "vern7"):
+            cm = co if method == "tsit5" else [float(x) for x in _vern7_R_coeffs()]
+            terms = sum(abs(a) * abs(z) ** k for k, a in enumerate(cm))
+            R = sum(a * z**k for k, a in enumerate(cm))
         elif method == "ros3":
             # |terms| of R = 1 + z b^T w, with |b_i w_i| summed
             if _ROS3 is None:
@@ -245,7 +361,7 @@ def _kappa(method, p, hs):
 
 
 @pytest.mark.parametrize("method,lams", [("tsit5", [0.5, 3.0, 12.0]), ("ros2", [0.5, 50.0, 1e4]),
-                                         ("ros3", [0.5, 50.0, 1e4])])
+                                         ("ros3", [0.5, 50.0, 1e4]), ("vern7", [0.5, 3.0, 12.0])])
 @pytest.mark.parametrize("mode", ["tape", "dual"])
 def test_closed_form_decay_adjoint(method, lams, mode):
     rng = np.random.default_rng(7)
@@ -265,7 +381,7 @@ def test_closed_form_decay_adjoint(method, lams, mode):
         # size of the method's inner weights (Tsit5: |a_6m| up to ~13, so 32;
         # ROS2: 3/2, 1/2, 2 and gamma, so 8), summed over the N steps.  A
         # wrong digit or a dropped term moves these numbers by 1e-8 or more.
-        tol = N * EPS * _kappa(method, -lam, hs) * (32 if method == "tsit5" else 8)
+        tol = N * EPS * _kappa(method, -lam, hs) * {"tsit5": 32, "vern7": 128}.get(method, 8)
         assert abs(out["loss"][i] - L) <= tol * abs(L)
         assert abs(out["du0"][0, i] - gu) <= tol * abs(gu)
         assert abs(out["dp"][0, i] - gp) <= tol * abs(gp), (method, lam, out["dp"][0, i], gp)

@@ -46,7 +46,8 @@ def test_mesh_consistency(name):
             u = un
 
 
-@pytest.mark.parametrize("name,method,q", [("lorenz_small", "tsit5", 5), ("lorenz_small", "ros3", 3),
+@pytest.mark.parametrize("name,method,q", [("lorenz_small", "tsit5", 5), ("lorenz_small", "vern7", 7),
+                                           ("lorenz_small", "ros3", 3),
                                            ("robertson", "ros2", 2), ("robertson", "ros3", 3)])
 def test_controller_reproduces_recorded_steps(name, method, q):
     """The ratio of consecutive recorded steps is the PI controller's factor
@@ -100,7 +101,7 @@ def test_tight_tolerance_solution_matches_scipy():
         assert err <= 1e-7, err
 
 
-@pytest.mark.parametrize("method,order", [("tsit5", 5), ("ros2", 2), ("ros3", 3)])
+@pytest.mark.parametrize("method,order", [("tsit5", 5), ("ros2", 2), ("ros3", 3), ("vern7", 7)])
 def test_convergence_order(method, order):
     prob = W.lorenz_small(1)
     prob.method = method
