@@ -73,6 +73,14 @@ WORKLOADS = {
                             desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, dense record (steps do not stop at "
                                  "the 10 save points; Tsit5's continuous extension there) with N(0,1) targets, "
                                  "1 record + 10 gradient passes"),
+    # Verner's 7(6) pair on the headline ensemble and tolerance: the replay
+    # step 321 (18 add, 45 mul, 129 fma: oracle count) + the transposed step
+    # 420 (hand count: the nu combinations over the 30 nonzero a_mj and 7
+    # weights b_j 222, nine Lorenz VJPs of 19 flop 171, the sum into lambda 27)
+    "lorenz_1m_vern7": dict(passes=10, flop_step=321 + 420, flop_save=18, kernel="k_grad_vern7_lorenz",
+                            problem="lorenz_1m", method="vern7", n=1 << 20, dtype="f64",
+                            desc="Lorenz d=3, t in [0,10], Verner 7(6) rtol=atol=1e-6, 10 save points with N(0,1) "
+                                 "targets, 1 record + 10 gradient passes"),
     "lorenz_small": dict(passes=1, flop_step=192 + 264, flop_save=12, kernel="k_grad_tsit5_lorenz", n=1024,
                          dtype="f64",
                          desc="Lorenz d=3, t in [0,1], Tsit5 rtol=atol=1e-8, loss sum ||u(T)||^2, "
@@ -180,6 +188,8 @@ def distributed() -> bool:
 def metric_name(args) -> str:
     if args.workload == "lorenz_1m_dense":
         return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, dense save points)"
+    if args.workload == "lorenz_1m_vern7":
+        return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, Verner 7(6))"
     if args.workload == "lorenz_1m_sens":
         return f"trajectory-sensitivities/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, forward mode)"
     if args.workload == "robertson_ros3_sens":
@@ -370,7 +380,8 @@ def run_reference(args):
     W = WORKLOADS[args.workload]
     kind = W.get("kind", "grad")
     solve = kind != "grad"
-    sample = {"lorenz_1m": 256, "lorenz_1m_dense": 256, "lorenz_small": 256, "robertson": 32, "node64": 64,
+    sample = {"lorenz_1m": 256, "lorenz_1m_dense": 256, "lorenz_1m_vern7": 256, "lorenz_small": 256,
+              "robertson": 32, "node64": 64,
               "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512, "robertson_ros3": 256,
               "robertson_ros3_sens": 256, "kin8": 256, "kin8_ros2": 16}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
@@ -841,10 +852,12 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # samples sized for seconds of host work (and host memory for the
         # oracle's trajectory-major meshes)
-        sample = {"lorenz_1m": 32768, "lorenz_1m_dense": 32768, "lorenz_small": 1024, "robertson": 256,
+        sample = {"lorenz_1m": 32768, "lorenz_1m_dense": 32768, "lorenz_1m_vern7": 32768, "lorenz_small": 1024,
+                  "robertson": 256,
                   "robertson_ros3": 2048, "node64": 1024, "kin8": 2048, "kin8_ros2": 64}[args.workload]
         line["cpu_baseline"] = cpu_baseline(args, min(sample, n))
-        psample = {"lorenz_1m": 8192, "lorenz_1m_dense": 8192, "lorenz_small": 1024, "robertson": 256,
+        psample = {"lorenz_1m": 8192, "lorenz_1m_dense": 8192, "lorenz_1m_vern7": 8192, "lorenz_small": 1024,
+                   "robertson": 256,
                    "robertson_ros3": 2048, "node64": 256, "kin8": 1024, "kin8_ros2": 32}[args.workload]
         line["parity"] = parity_sample(args, min(psample, n))
     elif rank == 0 and world == 1 and args.parity_sample:
@@ -860,6 +873,7 @@ def run_ours(args):
 SECONDARY = [
     ("lorenz_1m_f32", ["--workload", "lorenz_1m", "--dtype", "f32"], 2048),
     ("lorenz_1m_dense", ["--workload", "lorenz_1m_dense"], 2048),
+    ("lorenz_1m_vern7", ["--workload", "lorenz_1m_vern7"], 2048),
     ("robertson_ros2", ["--workload", "robertson"], 128),
     ("robertson_ros3", ["--workload", "robertson_ros3"], 512),
     ("kin8_ros3", ["--workload", "kin8"], 256),

@@ -41,6 +41,9 @@ template <typename T>
 gs_status launch_grad_kin8(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                            cudaStream_t);
 template <typename T>
+gs_status launch_grad_vern7_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
+                                   cudaStream_t);
+template <typename T>
 gs_status launch_solve3(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 gs_status record_node64(const gs_problem*, const gs_tol*, const gs_mesh*, void*, cudaStream_t);
 gs_status node64_record_pass(const gs_problem*, const gs_tol*, int32_t, bool, float*, int32_t*, int32_t*, int32_t*,
@@ -51,6 +54,7 @@ gs_status node64_solve(const gs_problem*, const gs_mesh*, void*, cudaStream_t);
 void node64_set_tensor(int on);
 size_t node64_grad_ws_bytes(int64_t n, int32_t smax, size_t tsize);
 size_t grad_tsit5_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave, bool dense);
+size_t grad_vern7_lorenz_ws_bytes(int32_t dtype, int64_t n, int32_t smax, int32_t nsave);
 
 static size_t dsize(const gs_problem* P) { return P->dtype == GS_F64 ? 8 : 4; }
 
@@ -58,7 +62,8 @@ static gs_status check_problem(const gs_problem* P) {
   if (!P) return GS_EINVAL;
   if (P->n < 0 || P->n > (int64_t)INT32_MAX) return GS_EINVAL;
   if (P->dtype != GS_F32 && P->dtype != GS_F64) return GS_EINVAL;
-  if (P->method != GS_TSIT5 && P->method != GS_ROS2 && P->method != GS_ROS3) return GS_EINVAL;
+  if (P->method != GS_TSIT5 && P->method != GS_ROS2 && P->method != GS_ROS3 && P->method != GS_VERN7)
+    return GS_EINVAL;
   switch (P->system) {
     case GS_LORENZ:
     case GS_ROBERTSON:
@@ -73,7 +78,7 @@ static gs_status check_problem(const gs_problem* P) {
     case GS_KIN8:
       if (P->d != 8 || P->np != 8) return GS_EINVAL;
       // a stiff system: built for the Rosenbrock methods
-      if (P->method == GS_TSIT5) return GS_EUNSUPPORTED;
+      if (P->method == GS_TSIT5 || P->method == GS_VERN7) return GS_EUNSUPPORTED;
       break;
     case GS_HIRES:
       return GS_EUNSUPPORTED;
@@ -99,12 +104,14 @@ static gs_status check_mesh(const gs_problem* P, const gs_mesh* M) {
   return GS_OK;
 }
 
-// Tolerances; a dense record is built for the d = 3 systems (every method).
+// Tolerances; a dense record is built for the d = 3 systems (Tsit5, ROS2 and
+// ROS3; Verner's pair has landing records only).
 static gs_status check_tol(const gs_problem* P, const gs_tol* tol) {
   if (!tol || !(tol->rtol >= 0) || !(tol->atol >= 0) || !(tol->rtol + tol->atol > 0) || !(tol->h0 >= 0))
     return GS_EINVAL;
   if (tol->dense != 0 && tol->dense != 1) return GS_EINVAL;
-  if (tol->dense && (P->system == GS_NODE64 || P->system == GS_KIN8)) return GS_EUNSUPPORTED;
+  if (tol->dense && (P->system == GS_NODE64 || P->system == GS_KIN8 || P->method == GS_VERN7))
+    return GS_EUNSUPPORTED;
   return GS_OK;
 }
 
@@ -140,10 +147,12 @@ size_t gs_workspace_bytes(const gs_problem* P, const gs_mesh* M, int32_t op) {
   if (op == GS_OP_RECORD) return record_ws_bytes(P->n, M->smax, P->nsave, dsize(P));
   if (op == GS_OP_GRAD) {
     if (P->system == GS_NODE64) return node64_grad_ws_bytes(P->n, M->smax, dsize(P));
-    // one checkpointed state per step and slot (the Tsit5 Lorenz kernel adds
-    // the save points' loss gradients)
+    // one checkpointed state per step and slot (the Tsit5 and Verner Lorenz
+    // kernels add the save points' loss gradients)
     if (P->method == GS_TSIT5 && P->system == GS_LORENZ)
       return grad_tsit5_lorenz_ws_bytes(P->dtype, P->n, M->smax, P->nsave, M->save_theta != nullptr);
+    if (P->method == GS_VERN7 && P->system == GS_LORENZ)
+      return grad_vern7_lorenz_ws_bytes(P->dtype, P->n, M->smax, P->nsave);
     return (size_t)M->smax * (size_t)P->d * (size_t)P->n * dsize(P);
   }
   return 0;
@@ -223,7 +232,8 @@ gs_status gs_solve(const gs_problem* P, const gs_mesh* M, void* u_save, void* st
   gs_status rc = check_problem(P);
   if (rc != GS_OK) return rc;
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
-  if (M->save_theta && (P->system == GS_NODE64 || P->system == GS_KIN8)) return GS_EUNSUPPORTED;
+  if (M->save_theta && (P->system == GS_NODE64 || P->system == GS_KIN8 || P->method == GS_VERN7))
+    return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (!u_save) return GS_EINVAL;
   if (P->system == GS_NODE64) return node64_solve(P, M, u_save, (cudaStream_t)stream);
@@ -238,7 +248,10 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if ((rc = check_mesh(P, M)) != GS_OK) return rc;
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
   // dense save points: the d = 3 gradients (Tsit5 on Lorenz, ROS2 / ROS3 on Lorenz and Robertson)
-  if (M->save_theta && (P->system == GS_NODE64 || P->system == GS_KIN8)) return GS_EUNSUPPORTED;
+  if (M->save_theta && (P->system == GS_NODE64 || P->system == GS_KIN8 || P->method == GS_VERN7))
+    return GS_EUNSUPPORTED;
+  // Verner's pair: the Lorenz gradient
+  if (P->method == GS_VERN7 && P->system != GS_LORENZ) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;
   if (!loss || !dp || !du0) return GS_EINVAL;
@@ -248,6 +261,9 @@ gs_status gs_grad(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (P->method == GS_TSIT5 && P->system == GS_LORENZ)
     return P->dtype == GS_F64 ? launch_grad_tsit5_lorenz<double>(P, M, Ls, loss, dp, du0, ws, st)
                               : launch_grad_tsit5_lorenz<float>(P, M, Ls, loss, dp, du0, ws, st);
+  if (P->method == GS_VERN7)
+    return P->dtype == GS_F64 ? launch_grad_vern7_lorenz<double>(P, M, Ls, loss, dp, du0, ws, st)
+                              : launch_grad_vern7_lorenz<float>(P, M, Ls, loss, dp, du0, ws, st);
   if (P->system == GS_KIN8)
     return P->dtype == GS_F64 ? launch_grad_kin8<double>(P, M, Ls, loss, dp, du0, ws, st)
                               : launch_grad_kin8<float>(P, M, Ls, loss, dp, du0, ws, st);
@@ -268,7 +284,7 @@ gs_status gs_sens(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
   // Tsit5: Lorenz; ROS2 / ROS3: Lorenz and Robertson (landing or dense save
   // points) and kin8 (landing)
-  if (P->system == GS_NODE64) return GS_EUNSUPPORTED;
+  if (P->system == GS_NODE64 || P->method == GS_VERN7) return GS_EUNSUPPORTED;
   if (P->system == GS_KIN8 && M->save_theta) return GS_EUNSUPPORTED;
   if (P->method == GS_TSIT5 && P->system != GS_LORENZ) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;

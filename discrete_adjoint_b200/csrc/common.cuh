@@ -71,10 +71,47 @@ namespace gs {
 #define ROS3_E3 0.2235406989781157
 
 // Error order q of the step-size controller for each method: the local error
-// estimate of Tsit5 is O(h^5), of ROS2 O(h^2), of ROS3 O(h^3).
+// estimate of Tsit5 is O(h^5), of ROS2 O(h^2), of ROS3 O(h^3), of Verner's
+// 7(6) pair O(h^7).
 __host__ __device__ constexpr double method_order(int method) {
-  return method == GS_TSIT5 ? 5.0 : (method == GS_ROS3 ? 3.0 : 2.0);
+  return method == GS_TSIT5 ? 5.0 : (method == GS_ROS3 ? 3.0 : (method == GS_VERN7 ? 7.0 : 2.0));
 }
+
+// ---------------------------------------------------------------------------
+// Verner's 7(6) pair: v7_a(j, m) is stage j's weight on slope m (1-based,
+// m < j <= 10, zero where the pair has none), v7_b(m) the seventh-order
+// weights, v7_e(m) = b_m - bhat_m the weights of the embedded error estimate
+// (one double subtraction of the two stored weights).
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr double v7_a(int j, int m) {
+  constexpr double a[10][9] = {
+      {0, 0, 0, 0, 0, 0, 0, 0, 0},
+      {0.005, 0, 0, 0, 0, 0, 0, 0, 0},
+      {-1.07679012345679, 1.185679012345679, 0, 0, 0, 0, 0, 0, 0},
+      {0.04083333333333333, 0, 0.1225, 0, 0, 0, 0, 0, 0},
+      {0.6389139236255726, 0, -2.455672638223657, 2.272258714598084, 0, 0, 0, 0, 0},
+      {-2.6615773750187572, 0, 10.804513886456137, -8.3539146573962, 0.820487594956657, 0, 0, 0, 0},
+      {6.067741434696772, 0, -24.711273635911088, 20.427517930788895, -1.9061579788166472, 1.006172249242068, 0,
+       0, 0},
+      {12.054670076253203, 0, -49.75478495046899, 41.142888638604674, -4.461760149974004, 2.042334822239175,
+       -0.09834843665406107, 0, 0},
+      {10.138146522881808, 0, -42.6411360317175, 35.76384003992257, -4.3480228403929075, 2.0098622683770357,
+       0.3487490460338272, -0.27143900510483127, 0},
+      {-45.030072034298676, 0, 187.3272437654589, -154.02882369350186, 18.56465306347536, -7.141809679295079,
+       1.3088085781613787, 0, 0}};
+  return a[j - 1][m - 1];
+}
+__host__ __device__ constexpr double v7_b(int m) {
+  constexpr double b[10] = {0.04715561848627222, 0, 0, 0.25750564298434153, 0.26216653977412624,
+                            0.15216092656738558, 0.4939969170032485, -0.29430311714032503, 0.08131747232495111, 0};
+  return b[m - 1];
+}
+__host__ __device__ constexpr double v7_bhat(int m) {
+  constexpr double b[10] = {0.044608606606341174, 0, 0, 0.26716403785713727, 0.22010183001772932,
+                            0.2188431703143157, 0.22898717054112028, 0, 0, 0.02029518466335628};
+  return b[m - 1];
+}
+__host__ __device__ constexpr double v7_e(int m) { return v7_b(m) - v7_bhat(m); }
 
 template <typename T>
 __device__ __forceinline__ T cst(double x) {

@@ -53,11 +53,7 @@ struct RecArgs {
 
 // What a recorder pass writes besides the counts: nothing (the sizing pass),
 // the mesh, or the state at each save time (the adaptive forward-only solve).
-enum RecMode { kRecCount = 0, kRecMesh = 1, kRecSolve = 2, kRecSolveDense = 3 };
-// the forward-only solve (states at the save times); kRecSolveDense reads a
-// dense record's save points off the steps' dense output, in an instance of
-// its own so that the landing solve carries none of that code
-template <int MODE> __host__ __device__ constexpr bool rec_solve() { return MODE == kRecSolve || MODE == kRecSolveDense; }
+enum RecMode { kRecCount = 0, kRecMesh = 1, kRecSolve = 2 };
 
 template <typename T, int SYS, int METHOD>
 __device__ T initial_step_d(const T* u0, const T* p, T t0, T t1, T rtol, T atol) {
@@ -145,6 +141,9 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
   if constexpr (METHOD == GS_TSIT5) {
     static_assert(D == 3, "Tsit5 recorder: d = 3 systems");
     tsit5_err_step<T, SYS>(r.u, r.p, h, r.k1, un, k7, e);
+  } else if constexpr (METHOD == GS_VERN7) {
+    static_assert(D == 3, "Verner 7 recorder: d = 3 systems");
+    vern7_step3<T, SYS>(r.u, r.p, h, r.k1, un, e);
   } else {
     bool ok;
     if constexpr (SYS == GS_KIN8)
@@ -179,18 +178,20 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
     ++r.nst;
     const T tprev = r.t;
     r.t = clipped ? tstop : tn;
-    if (D == 3 && a.dense && MODE != kRecSolve) {
+    if (D == 3 && a.dense) {
       // every save time this step passed: its position inside the step, and
       // (solve) the state there -- for Tsit5 its continuous extension over
-      // the step's stages (recomputed from u and k1), for the Rosenbrock
-      // methods the Hermite interpolant from u, f(u), u_new, f(u_new)
+      // the step's stages (recomputed from u and k1 in a call that is not
+      // inlined, so that its registers stay out of every attempt's), for the
+      // Rosenbrock methods the Hermite interpolant from u, f(u), u_new,
+      // f(u_new)
       while (r.kk < a.nsave && a.tsave[r.kk] <= r.t) {
         const T th = (a.tsave[r.kk] - tprev) / h;
         if (MODE == kRecMesh) {
           a.save_idx[(int64_t)r.kk * n + r.o] = r.nst;
           a.theta[(int64_t)r.kk * n + r.o] = th;
         }
-        if constexpr (MODE == kRecSolveDense) {
+        if constexpr (MODE == kRecSolve) {
           T ut[D];
 #pragma unroll
           for (int c = 0; c < D; ++c) ut[c] = un[c];
@@ -217,9 +218,10 @@ __device__ __forceinline__ bool traj_attempt(const RecArgs<T>& a, Traj<T, SysDim
       r.u[c] = un[c];
       if (METHOD == GS_TSIT5) r.k1[c] = k7[c];
     }
+    if constexpr (METHOD == GS_VERN7) rhs_s<T, SYS>(r.u, r.p, r.k1);  // not FSAL: the next step's first slope
     while (!a.dense && r.kk < a.nsave && r.t == a.tsave[r.kk]) {
       if (MODE == kRecMesh) a.save_idx[(int64_t)r.kk * n + r.o] = r.nst;
-      if (rec_solve<MODE>()) {
+      if (MODE == kRecSolve) {
 #pragma unroll
         for (int c = 0; c < D; ++c) a.u_save[((int64_t)r.kk * D + c) * n + r.i] = r.u[c];
       }
@@ -256,7 +258,7 @@ __device__ __forceinline__ void traj_finish(const RecArgs<T>& a, const Traj<T, D
       if (a.dense) a.theta[(int64_t)k * n + r.o] = cst<T>(1.0);
     }
   }
-  if (rec_solve<MODE>() && r.status != GS_TRAJ_OK) {
+  if (MODE == kRecSolve && r.status != GS_TRAJ_OK) {
     // a failed trajectory has no solution: NaN at every save point
     const T nan = cst<T>(__longlong_as_double(0x7ff8000000000000ULL));
     for (int k = 0; k < a.nsave; ++k)
@@ -329,12 +331,12 @@ __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3(RecArgs<T> a) 
 // steps, and its rows zeroed up to the previous count.  The loop ends: every
 // pass takes a group from a counter that only grows, and a group's inner loop
 // advances some chain's accepted or rejected count, both capped by smax.
-// MODE kRecSolve / kRecSolveDense runs the adaptive forward-only solve in the same grouped
+// MODE kRecSolve runs the adaptive forward-only solve in the same grouped
 // order with its outputs by trajectory (an entry outside [0, n) is skipped).
 template <typename T, int SYS, int METHOD, int MODE>
 __global__ void __launch_bounds__(128, rec_minb<SYS>()) k_record3_inplace(RecArgs<T> a, const int32_t* order,
                                                                          unsigned long long* next_group) {
-  static_assert(MODE == kRecMesh || rec_solve<MODE>(), "grouped passes: mesh or solve");
+  static_assert(MODE == kRecMesh || MODE == kRecSolve, "grouped passes: mesh or solve");
   const unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const int64_t n = a.n;
@@ -521,6 +523,10 @@ static gs_status dispatch_rec_inplace(int sys, int method, const RecArgs<T>& a, 
     return launch_rec_inplace<T, kSysRobertson, GS_ROS3, MODE>(a, order, ctr, st);
   if (sys == GS_KIN8 && method == GS_ROS2) return launch_rec_inplace<T, kSysKin8, GS_ROS2, MODE>(a, order, ctr, st);
   if (sys == GS_KIN8 && method == GS_ROS3) return launch_rec_inplace<T, kSysKin8, GS_ROS3, MODE>(a, order, ctr, st);
+  if (sys == GS_LORENZ && method == GS_VERN7)
+    return launch_rec_inplace<T, kSysLorenz, GS_VERN7, MODE>(a, order, ctr, st);
+  if (sys == GS_ROBERTSON && method == GS_VERN7)
+    return launch_rec_inplace<T, kSysRobertson, GS_VERN7, MODE>(a, order, ctr, st);
   return GS_EUNSUPPORTED;
 }
 
@@ -534,6 +540,8 @@ static gs_status dispatch_rec(int sys, int method, const RecArgs<T>& a, cudaStre
   if (sys == GS_ROBERTSON && method == GS_ROS3) return launch_rec<T, kSysRobertson, GS_ROS3, MODE>(a, st);
   if (sys == GS_KIN8 && method == GS_ROS2) return launch_rec<T, kSysKin8, GS_ROS2, MODE>(a, st);
   if (sys == GS_KIN8 && method == GS_ROS3) return launch_rec<T, kSysKin8, GS_ROS3, MODE>(a, st);
+  if (sys == GS_LORENZ && method == GS_VERN7) return launch_rec<T, kSysLorenz, GS_VERN7, MODE>(a, st);
+  if (sys == GS_ROBERTSON && method == GS_VERN7) return launch_rec<T, kSysRobertson, GS_VERN7, MODE>(a, st);
   return GS_EUNSUPPORTED;
 }
 
@@ -560,15 +568,13 @@ gs_status solve_adaptive3(const gs_problem* P, const gs_tol* tol, int32_t smax, 
     a.nsteps = nsteps;
     a.status = status;
     a.u_save = (double*)u_save;
-    return tol->dense ? dispatch_rec<double, kRecSolveDense>(P->system, P->method, a, st)
-                      : dispatch_rec<double, kRecSolve>(P->system, P->method, a, st);
+    return dispatch_rec<double, kRecSolve>(P->system, P->method, a, st);
   }
   RecArgs<float> a = rec_args<float>(P, tol, smax);
   a.nsteps = nsteps;
   a.status = status;
   a.u_save = (float*)u_save;
-  return tol->dense ? dispatch_rec<float, kRecSolveDense>(P->system, P->method, a, st)
-                    : dispatch_rec<float, kRecSolve>(P->system, P->method, a, st);
+  return dispatch_rec<float, kRecSolve>(P->system, P->method, a, st);
 }
 
 // The adaptive forward-only solve in a given trajectory order (groups of 32
@@ -581,17 +587,13 @@ gs_status solve_adaptive3_ordered(const gs_problem* P, const gs_tol* tol, int32_
     a.nsteps = nsteps;
     a.status = status;
     a.u_save = (double*)u_save;
-    unsigned long long* ctr = (unsigned long long*)ws;
-    return tol->dense ? dispatch_rec_inplace<double, kRecSolveDense>(P->system, P->method, a, order, ctr, st)
-                      : dispatch_rec_inplace<double, kRecSolve>(P->system, P->method, a, order, ctr, st);
+    return dispatch_rec_inplace<double, kRecSolve>(P->system, P->method, a, order, (unsigned long long*)ws, st);
   }
   RecArgs<float> a = rec_args<float>(P, tol, smax);
   a.nsteps = nsteps;
   a.status = status;
   a.u_save = (float*)u_save;
-  unsigned long long* ctr = (unsigned long long*)ws;
-  return tol->dense ? dispatch_rec_inplace<float, kRecSolveDense>(P->system, P->method, a, order, ctr, st)
-                    : dispatch_rec_inplace<float, kRecSolve>(P->system, P->method, a, order, ctr, st);
+  return dispatch_rec_inplace<float, kRecSolve>(P->system, P->method, a, order, (unsigned long long*)ws, st);
 }
 
 static size_t al256(size_t b) { return (b + 255) / 256 * 256; }

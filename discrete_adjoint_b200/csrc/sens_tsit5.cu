@@ -43,13 +43,17 @@ namespace gs {
 #ifndef GS_SENS_NDIR
 #define GS_SENS_NDIR 6
 #endif
-// directions per thread on dense meshes, and whether their save-point branch
-// is a call (1) or inlined (0)
+// Directions per thread on dense meshes, and whether their save-point branch
+// is a call (1) or inlined (0).  At a dense save point the branch recomputes
+// the step's stages and their tangents; with six directions per thread that
+// spills heavily.  Measured on the 2^20 Lorenz dense mesh (fp64): six
+// directions, call 88 ms / inlined 68 ms; three, call 58.5 / inlined 40.3;
+// two, inlined 39.0; one, inlined 57.8 (landing meshes, six: 25.5 ms).
 #ifndef GS_SENS_NDIR_DENSE
-#define GS_SENS_NDIR_DENSE GS_SENS_NDIR
+#define GS_SENS_NDIR_DENSE 2
 #endif
 #ifndef GS_SENS_DENSE_NOINLINE
-#define GS_SENS_DENSE_NOINLINE 1
+#define GS_SENS_DENSE_NOINLINE 0
 #endif
 #if GS_SENS_DENSE_NOINLINE
 #define GS_SENS_DENSE_FN __noinline__
@@ -119,9 +123,7 @@ __device__ __forceinline__ void lorenz_jvp(T x, T y, T z, T s, T r, T b, const V
 // A dense save point inside a step: Tsit5's continuous extension and its
 // tangent, from the step's stages and their tangents recomputed from
 // (u_s, v_s) with the step's own arithmetic; k_7 and dk_7 are the FSAL slope
-// and its tangent that the step has formed.  Not inlined: it runs only at
-// dense save points, and inlined into the step loop its stage tangents would
-// add to the register pressure of every step.
+// and its tangent that the step has formed.
 template <typename T, int NDIR>
 struct DenseTanIn {
   T x, y, z, k1x, k1y, k1z, k7x, k7y, k7z, s, r, b, h, th;

@@ -1,6 +1,6 @@
 // solve.cu -- forward-only fixed-step replay on a recorded mesh, writing the
-// state at every save point (d = 3 systems with Tsit5, ROS2 or ROS3; the
-// d = 8 system with ROS2 or ROS3).  The forward-only
+// state at every save point (d = 3 systems with Tsit5, Verner 7, ROS2 or
+// ROS3; the d = 8 system with ROS2 or ROS3).  The forward-only
 // use of GRADSOLVE (arXiv 2609.02876, abstract); same arithmetic as the
 // forward half of the gradient kernels.
 #include "kin8.cuh"
@@ -60,6 +60,9 @@ __global__ void __launch_bounds__(128) k_solve3(SolveArgs<T> a) {
         kin8_ros3_fwd<T>(u, p, h, LU, P, R, q1, v, q2, q3, un);
       else
         kin8_ros2_fwd<T>(u, p, h, LU, P, R, q1, v, q2, un);
+    } else if constexpr (METHOD == GS_VERN7) {
+      vern7_step3<T, SYS>(u, p, h, k1, un, nullptr);
+      rhs3<T, SYS>(un, p, k1);  // the next step's first slope (not FSAL)
     } else if constexpr (METHOD == GS_TSIT5) {
       T k7[3], e[3];
       tsit5_err_step<T, SYS>(u, p, h, k1, un, k7, e);
@@ -145,6 +148,10 @@ gs_status launch_solve3(const gs_problem* P, const gs_mesh* M, void* u_save, cud
     k_solve3<T, kSysKin8, GS_ROS3><<<grid, 128, 0, st>>>(a);
   else if (P->system == GS_KIN8 && P->method == GS_ROS2)
     k_solve3<T, kSysKin8, GS_ROS2><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_LORENZ && P->method == GS_VERN7)
+    k_solve3<T, kSysLorenz, GS_VERN7><<<grid, 128, 0, st>>>(a);
+  else if (P->system == GS_ROBERTSON && P->method == GS_VERN7)
+    k_solve3<T, kSysRobertson, GS_VERN7><<<grid, 128, 0, st>>>(a);
   else
     k_solve3<T, kSysRobertson, GS_ROS2><<<grid, 128, 0, st>>>(a);
   count_launch();

@@ -333,6 +333,49 @@ __device__ __forceinline__ void tsit5_err_step(const T u[3], const T p[3], T h, 
   }
 }
 
+// One step of Verner's 7(6) pair (k1 = f(u) on entry): stage j's state is
+// acc = a_j1 k1, then acc = fma(a_jm, k_m, acc) over the nonzero a_jm in
+// increasing m, U_j = fma(h, acc, u); u_new the same over the nonzero b_m.
+// With E != nullptr, stage 10 and the embedded error estimate
+// e = h (E_1 k_1 + ... over the nonzero E_m), E = b - bhat.  The operation
+// order is the floating-point contract of the method.
+template <typename T, int SYS>
+__device__ __forceinline__ void vern7_step3(const T u[3], const T p[3], T h, const T k1[3], T un[3], T* e) {
+  T k[10][3], U[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) k[0][c] = k1[c];
+#pragma unroll
+  for (int j = 2; j <= 10; ++j) {
+    if (j == 10 && e == nullptr) break;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      T acc = cst<T>(v7_a(j, 1)) * k[0][c];
+#pragma unroll
+      for (int m = 2; m < j; ++m)
+        if (v7_a(j, m) != 0.0) acc = fmaT(cst<T>(v7_a(j, m)), k[m - 1][c], acc);
+      U[c] = fmaT(h, acc, u[c]);
+    }
+    rhs3<T, SYS>(U, p, k[j - 1]);
+  }
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(v7_b(1)) * k[0][c];
+#pragma unroll
+    for (int m = 2; m <= 9; ++m)
+      if (v7_b(m) != 0.0) acc = fmaT(cst<T>(v7_b(m)), k[m - 1][c], acc);
+    un[c] = fmaT(h, acc, u[c]);
+  }
+  if (e == nullptr) return;
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T acc = cst<T>(v7_e(1)) * k[0][c];
+#pragma unroll
+    for (int m = 2; m <= 10; ++m)
+      if (v7_e(m) != 0.0) acc = fmaT(cst<T>(v7_e(m)), k[m - 1][c], acc);
+    e[c] = h * acc;
+  }
+}
+
 // One ROS2 step with error estimate.  Returns false on a singular matrix.
 template <typename T, int SYS>
 __device__ __forceinline__ bool ros2_err_step(const T u[3], const T p[3], T h, T un[3], T e[3]) {

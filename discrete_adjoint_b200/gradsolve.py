@@ -32,7 +32,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 GS_OK, GS_EINVAL, GS_ECUDA, GS_EWORKSPACE, GS_EUNSUPPORTED = 0, -1, -2, -3, -4
 TRAJ_OK, TRAJ_MAXSTEPS, TRAJ_DTMIN, TRAJ_NONFINITE, TRAJ_SINGULAR, TRAJ_BADORDER = 0, 1, 2, 3, 4, 5
 SYSTEMS = {"lorenz": 1, "robertson": 2, "hires": 3, "node64": 4, "kin8": 5}
-METHODS = {"tsit5": 1, "ros2": 2, "ros3": 3}
+METHODS = {"tsit5": 1, "ros2": 2, "ros3": 3, "vern7": 4}
 DTYPES = {"f32": 1, "f64": 2}
 LOSSES = {"sumsq": 1, "linear": 2}
 OP_RECORD, OP_GRAD = 0, 1

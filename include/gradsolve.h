@@ -89,6 +89,14 @@ typedef int32_t gs_status;
  * GRADSOLVE's explicit and Rosenbrock integrators (abstract), with the
  * higher-order integrators it names as a next step ("Future directions"). */
 #define GS_ROS3 3
+/* Verner's 7(6) pair (Verner 2010, the "most efficient" 7(6) pair): ten
+ * stages, seventh-order propagating weights on stages 1 and 4..9, the
+ * sixth-order embedded weights on 1, 4..7 and 10 (stage 10 only for the error
+ * estimate; not FSAL), controller order q = 7.  The explicit high-order
+ * method the gist.science summary of arXiv 2609.28458 ("Results", "Source of
+ * Speed-up") names beside Tsit5.  d = 3 systems, landing records only; the
+ * gradient on GS_LORENZ. */
+#define GS_VERN7 4
 
 #define GS_F32 1
 #define GS_F64 2
@@ -194,8 +202,9 @@ typedef struct gs_loss {
  * Workspace (scratch) bytes that op (GS_OP_RECORD / GS_OP_GRAD) needs for this
  * problem and mesh capacity: record -- step counts of the sizing pass and the
  * slot-ordering histograms; grad -- one checkpointed state per step and slot,
- * [smax][d][n] dtype (plus the d=64 weight-gradient partials; for Tsit5 on
- * Lorenz plus 3 values per save point and slot, 9 for a dense mesh).  Returns
+ * [smax][d][n] dtype (plus the d=64 weight-gradient partials; for Tsit5 and
+ * Verner 7 on Lorenz plus 3 values per save point and slot, 9 for a dense
+ * Tsit5 mesh).  Returns
  * 0 for an invalid request.  Host function; no device work.
  */
 GS_API size_t gs_workspace_bytes(const gs_problem* prob, const gs_mesh* mesh, int32_t op);
@@ -211,14 +220,14 @@ GS_API gs_status gs_count(const gs_problem* prob, const gs_tol* tol, int32_t sma
                    void* stream);
 
 /*
- * Record: adaptive solve of every trajectory (Tsit5, ROS2 or ROS3 per prob->method)
+ * Record: adaptive solve of every trajectory (Tsit5, Verner 7, ROS2 or ROS3 per prob->method)
  * into the caller's mesh, slots ordered by decreasing step count.  Fills every
  * mesh array.  Trajectories that fail keep a status != 0 and a truncated mesh.
  * Runs the adaptive pass into the workspace (trajectory order), the slot
  * ordering and a gather into slot order, all on stream.  Built for GS_LORENZ
- * and GS_ROBERTSON with GS_TSIT5, GS_ROS2 or GS_ROS3, GS_KIN8 with GS_ROS2 or
- * GS_ROS3 (fp64 and fp32), and GS_NODE64 with GS_TSIT5 in fp32; dense records
- * for every method on the d = 3 systems.  gs_count, gs_solve and gs_solve_adaptive
+ * and GS_ROBERTSON with GS_TSIT5, GS_VERN7, GS_ROS2 or GS_ROS3, GS_KIN8 with
+ * GS_ROS2 or GS_ROS3 (fp64 and fp32), and GS_NODE64 with GS_TSIT5 in fp32;
+ * dense records for GS_TSIT5, GS_ROS2 and GS_ROS3 on the d = 3 systems.  gs_count, gs_solve and gs_solve_adaptive
  * take the same combinations.  (Evolve.pub review, "Summary": the adaptive
  * solve happens once and keeps each trajectory's accepted step sizes.)
  */
@@ -303,8 +312,9 @@ GS_API gs_status gs_solve_adaptive_ordered(const gs_problem* prob, const gs_tol*
  * All indexed by trajectory.  Slots with status != 0 get NaN loss/dp/du0 and
  * do not contribute to dshared.  Built for GS_LORENZ with GS_TSIT5, GS_ROS2
  * or GS_ROS3; GS_ROBERTSON with GS_ROS2 or GS_ROS3 (dense save points
- * included for all of these); GS_KIN8 with GS_ROS2 or GS_ROS3 (fp64 and fp32
- * for all of these); GS_NODE64 with GS_TSIT5
+ * included for all of these); GS_LORENZ with GS_VERN7 (landing save points);
+ * GS_KIN8 with GS_ROS2 or GS_ROS3 (fp64 and fp32 for all of these);
+ * GS_NODE64 with GS_TSIT5
  * in fp32.  Other combinations return GS_EUNSUPPORTED.  (Evolve.pub review,
  * "Summary": the replay is a fixed-length chain without branches, and its
  * backward sweep is the exact discrete adjoint.)

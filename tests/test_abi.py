@@ -201,9 +201,40 @@ def test_ros3_method_validation_host_only(no_launch):
         assert _lib.gs_count(ctypes.byref(e), ctypes.byref(dense), 100, None, None, None) == 0
         assert _lib.gs_sens(ctypes.byref(e), ctypes.byref(md), ctypes.byref(ls), None, None, None, None, None) == 0
         assert _lib.gs_count(ctypes.byref(e), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, None, None, None) == 0
-    bad = _host_problem(method=4)
+    bad = _host_problem(method=5)
     assert _lib.gs_count(ctypes.byref(bad), ctypes.byref(_Tol(1e-6, 1e-6, 0.0)), 100, ctypes.c_void_p(16), None,
                          None) == -1
+
+
+@hidden_only
+def test_vern7_validation_host_only(no_launch):
+    """Verner's 7(6) pair (method 4) is accepted for the d = 3 systems with
+    landing records; dense records, forward sensitivities, the d = 8 and
+    d = 64 systems and a gradient off Lorenz are not built.  The gradient
+    workspace is one checkpointed state per step and slot plus each save
+    point's loss gradient.  No call here reaches a launch."""
+    from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
+    m = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+    ls = _Loss(1, None, None)
+    tol = _Tol(1e-6, 1e-6, 0.0)
+    dense = _Tol(1e-6, 1e-6, 0.0)
+    dense.dense = 1
+    lor = _host_problem(method=4)
+    assert _lib.gs_workspace_bytes(ctypes.byref(lor), ctypes.byref(m), 1) == (100 * 3 + 10 * 3) * 1000 * 8
+    for system in (1, 2):
+        e = _host_problem(n=0, system=system, method=4)
+        assert _lib.gs_count(ctypes.byref(e), ctypes.byref(tol), 100, None, None, None) == 0
+        assert _lib.gs_count(ctypes.byref(e), ctypes.byref(dense), 100, None, None, None) == -4
+        assert _lib.gs_sens(ctypes.byref(e), ctypes.byref(m), ctypes.byref(ls), None, None, None, None, None) == -4
+        md = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
+        md.save_theta = 16
+        assert _lib.gs_solve(ctypes.byref(e), ctypes.byref(md), None, None) == -4
+    rob = _host_problem(n=0, system=2, method=4)
+    assert _lib.gs_grad(ctypes.byref(rob), ctypes.byref(m), ctypes.byref(ls), None, None, None, None, None, 0,
+                        None) == -4
+    k8 = _host_problem(n=0, system=5, method=4)
+    k8.d = k8.np = 8
+    assert _lib.gs_count(ctypes.byref(k8), ctypes.byref(tol), 100, None, None, None) == -4
 
 
 @hidden_only

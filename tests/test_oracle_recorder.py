@@ -176,6 +176,12 @@ def test_step_operation_counts():
     r = oracle.count_step("robertson", "ros2", 3, 3)
     assert r == {"add": 7, "mul": 18 + 3 + 6, "fma": 38, "div": 3, "sqrt": 0, "tanh": 0}
     assert r["add"] + r["mul"] + 2 * r["fma"] + r["div"] == 113
+    # Verner 7(6), replay step: 9 rhs evaluations (not FSAL: k1 = f(u) each
+    # step); stage sums of rows 2..9 over the pair's 30 nonzero a_jm, per
+    # component 1 mul + (n_j - 1) fma + the fma with h; u_new over 7 weights
+    v = oracle.count_step("lorenz", "vern7", 3, 3)
+    assert v == {"add": 18, "mul": 18 + 24 + 3, "fma": 18 + 90 + 21, "div": 0, "sqrt": 0, "tanh": 0}
+    assert v["add"] + v["mul"] + 2 * v["fma"] == 321
     nd = oracle.count_step("node64", "tsit5", 64, 64)
     assert nd["fma"] == 6 * 64 * 64 + 64 * 21 and nd["tanh"] == 6 * 64
 
