@@ -26,20 +26,26 @@
 // are formed: as U_j is consumed mu_j takes its place, so U and mu together
 // hold 27 values through the transposed step.
 //
-// Execution: one thread per slot; gs_record orders slots by decreasing step
-// count, so a warp's chains have nearly equal length.  h and the checkpoints
-// are step-major over slots (a warp reads 32 consecutive elements of a row);
-// each step's row is loaded one step ahead and prefetched into L2 eight steps
-// ahead.  A Verner step has about twice Tsit5's arithmetic per step of memory
-// traffic, so the loads hide behind it without the copy rings of the Tsit5
-// kernel.
+// Execution: one thread per slot (blocks of 128); gs_record orders slots by
+// decreasing step count, so a warp's chains have nearly equal length.  h and
+// the checkpoints are step-major over slots (a warp reads 32 consecutive
+// elements of a row) and stream into per-thread shared-memory rings with
+// cp.async, kV7Ring steps ahead, as in the Tsit5 kernel.
 #include "steps.cuh"
 
 namespace gs {
 
+// 4 resident blocks of 128 per SM (125 registers, no spill; 16 warps/SM):
+// 9.88-9.91 ms per pass on the 2^20 Lorenz ensemble against 9.91 ms at 3
+// blocks (165 registers); the copy rings took 10.17 ms to 9.91 (3 blocks).
 #ifndef GS_V7_MINB
-#define GS_V7_MINB 3
+#define GS_V7_MINB 4
 #endif
+#ifndef GS_V7_RING
+#define GS_V7_RING 8
+#endif
+constexpr int kV7Ring = GS_V7_RING;
+static_assert((kV7Ring & (kV7Ring - 1)) == 0 && kV7Ring >= 2, "ring depth: a power of two, at least 2");
 
 template <typename T>
 struct Vern7LorenzArgs {
@@ -98,15 +104,30 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
   const T* hp = a.h + j;
   T* cp = a.ck + j;
 
+  // Per-thread copy rings (cp.async into shared memory, each thread waiting
+  // on its own copies only): forward, row st % kV7Ring holds h of step st;
+  // reverse, rows 4 (st % kV7Ring) + c hold checkpoint row c (c < 3) and h
+  // (c = 3) of step st.  Element (row w) of a thread is rg[w * 128]:
+  // consecutive threads touch consecutive words.
+  extern __shared__ __align__(16) unsigned char v7_ring_raw[];
+  T* const rg = reinterpret_cast<T*>(v7_ring_raw) + threadIdx.x;
+
   // ---------------------------------------------------------------- forward
   {
+    auto issue_f = [&](int sf) {
+      if (sf < S) cp_async_el(rg + (sf & (kV7Ring - 1)) * 128, hp + (int64_t)sf * n);
+      cp_async_commit();
+    };
     T k1[3];
     rhs3<T, kSysLorenz>(u, pr, k1);
-    T hn = S > 0 ? hp[0] : cst<T>(0.0);
+#pragma unroll
+    for (int sf = 0; sf < kV7Ring; ++sf) issue_f(sf);
+    cp_async_wait<kV7Ring - 1>();
+    T hn = S > 0 ? rg[0] : cst<T>(0.0);
     for (int st = 0; st < S; ++st) {
       const T h = hn;
-      if (st + 1 < S) hn = hp[(int64_t)(st + 1) * n];
-      if (st + 8 < S) prefetch_l2(hp + (int64_t)(st + 8) * n);
+      cp_async_wait<kV7Ring - 2>();  // the group of step st + 1
+      if (st + 1 < S) hn = rg[((st + 1) & (kV7Ring - 1)) * 128];
 #pragma unroll
       for (int c = 0; c < 3; ++c) cp[(int64_t)st * n3 + c * n] = u[c];
       T un[3];
@@ -114,7 +135,9 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
 #pragma unroll
       for (int c = 0; c < 3; ++c) u[c] = un[c];
       rhs3<T, kSysLorenz>(u, pr, k1);
+      issue_f(st + kV7Ring);  // into the row step st has left
     }
+    cp_async_wait<0>();  // the reverse reuses the rows
   }
   // Save points: u(t_k) is the state after step save_idx[k] (its checkpoint,
   // or the final state), taken while the step counts stay in [1, S] and
@@ -159,12 +182,26 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
   T pb[3] = {cst<T>(0.0), cst<T>(0.0), cst<T>(0.0)};
   int kk = nvalid - 1;
   int next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
-  T cu[3], ch = cst<T>(0.0);
-  if (S > 0) {
+  auto issue_r = [&](int sr) {  // step sr's checkpoint rows and h
+    if (sr >= 0 && sr < S) {
+      T* d = rg + (sr & (kV7Ring - 1)) * 4 * 128;
 #pragma unroll
-    for (int c = 0; c < 3; ++c) cu[c] = cp[(int64_t)(S - 1) * n3 + c * n];
-    ch = hp[(int64_t)(S - 1) * n];
-  }
+      for (int c = 0; c < 3; ++c) cp_async_el(d + c * 128, cp + (int64_t)sr * n3 + c * n);
+      cp_async_el(d + 3 * 128, hp + (int64_t)sr * n);
+    }
+    cp_async_commit();
+  };
+  T cu[3], ch = cst<T>(0.0);
+  auto take_r = [&](int sr) {
+    const T* d = rg + (sr & (kV7Ring - 1)) * 4 * 128;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) cu[c] = d[c * 128];
+    ch = d[3 * 128];
+  };
+#pragma unroll
+  for (int i2 = 0; i2 < kV7Ring; ++i2) issue_r(S - 1 - i2);
+  cp_async_wait<kV7Ring - 1>();
+  if (S > 0) take_r(S - 1);
   for (int st = S - 1; st >= 0; --st) {
     // save points reached at u_{st+1} add their loss gradient to lambda
     while (st + 1 == next) {
@@ -177,17 +214,6 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
     T U[9][3];
 #pragma unroll
     for (int c = 0; c < 3; ++c) U[0][c] = cu[c];
-    // the next (earlier) step's checkpoint and h, one step ahead
-    if (st > 0) {
-#pragma unroll
-      for (int c = 0; c < 3; ++c) cu[c] = cp[(int64_t)(st - 1) * n3 + c * n];
-      ch = hp[(int64_t)(st - 1) * n];
-      if (st > 8) {
-        prefetch_l2(hp + (int64_t)(st - 9) * n);
-#pragma unroll
-        for (int c = 0; c < 3; ++c) prefetch_l2(cp + (int64_t)(st - 9) * n3 + c * n);
-      }
-    }
     // recompute the stage states of step st (the forward's arithmetic)
     {
       T k[8][3];
@@ -227,7 +253,15 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
       for (int jj = 2; jj <= 9; ++jj) sum += mu[jj - 1][c];
       lam[c] += sum;
     }
+    // step st - 1's ring entries, after the transposed step (not live across
+    // it); then refill the rows step st has left
+    if (st > 0) {
+      cp_async_wait<kV7Ring - 2>();  // the group of step st - 1
+      take_r(st - 1);
+    }
+    issue_r(st - kV7Ring);
   }
+  cp_async_wait<0>();
 #pragma unroll
   for (int c = 0; c < 3; ++c) {
     a.dp[c * n + i] = pb[c];
@@ -263,7 +297,12 @@ gs_status launch_grad_vern7_lorenz(const gs_problem* P, const gs_mesh* M, const 
   a.ck = (T*)ws;
   a.gsave = (T*)ws + (size_t)M->smax * 3 * (size_t)P->n;
   const int64_t grid = (P->n + 127) / 128;
-  k_grad_vern7_lorenz<T><<<(unsigned)grid, 128, 0, st>>>(a);
+  const size_t smem = (size_t)kV7Ring * 4 * 128 * sizeof(T);  // the larger (reverse) ring
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k_grad_vern7_lorenz<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return GS_ECUDA;
+  k_grad_vern7_lorenz<T><<<(unsigned)grid, 128, smem, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
