@@ -29,6 +29,9 @@ template <typename T>
 gs_status launch_sens_ros(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                           cudaStream_t);
 template <typename T>
+gs_status launch_sens_vern7_lorenz(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
+                                   cudaStream_t);
+template <typename T>
 gs_status launch_sens_kin8(const gs_problem*, const gs_mesh*, const gs_loss*, void*, void*, void*, void*,
                            cudaStream_t);
 template <typename T>
@@ -284,8 +287,10 @@ gs_status gs_sens(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (!Ls || (Ls->kind != GS_LOSS_SUMSQ && Ls->kind != GS_LOSS_LINEAR)) return GS_EINVAL;
   // Tsit5: Lorenz; ROS2 / ROS3: Lorenz and Robertson (landing or dense save
   // points) and kin8 (landing)
-  if (P->system == GS_NODE64 || P->method == GS_VERN7) return GS_EUNSUPPORTED;
+  if (P->system == GS_NODE64) return GS_EUNSUPPORTED;
   if (P->system == GS_KIN8 && M->save_theta) return GS_EUNSUPPORTED;
+  // Verner's pair: Lorenz, landing meshes
+  if (P->method == GS_VERN7 && (P->system != GS_LORENZ || M->save_theta)) return GS_EUNSUPPORTED;
   if (P->method == GS_TSIT5 && P->system != GS_LORENZ) return GS_EUNSUPPORTED;
   if (P->n == 0) return GS_OK;
   if (Ls->kind == GS_LOSS_LINEAR && !Ls->weight) return GS_EINVAL;
@@ -294,6 +299,9 @@ gs_status gs_sens(const gs_problem* P, const gs_mesh* M, const gs_loss* Ls, void
   if (P->system == GS_KIN8)
     return P->dtype == GS_F64 ? launch_sens_kin8<double>(P, M, Ls, loss, dp, du0, sens, st)
                               : launch_sens_kin8<float>(P, M, Ls, loss, dp, du0, sens, st);
+  if (P->method == GS_VERN7)
+    return P->dtype == GS_F64 ? launch_sens_vern7_lorenz<double>(P, M, Ls, loss, dp, du0, sens, st)
+                              : launch_sens_vern7_lorenz<float>(P, M, Ls, loss, dp, du0, sens, st);
   if (P->method != GS_TSIT5)
     return P->dtype == GS_F64 ? launch_sens_ros<double>(P, M, Ls, loss, dp, du0, sens, st)
                               : launch_sens_ros<float>(P, M, Ls, loss, dp, du0, sens, st);

@@ -95,7 +95,7 @@ typedef int32_t gs_status;
  * estimate; not FSAL), controller order q = 7.  The explicit high-order
  * method the gist.science summary of arXiv 2609.28458 ("Results", "Source of
  * Speed-up") names beside Tsit5.  d = 3 systems, landing records only; the
- * gradient on GS_LORENZ. */
+ * gradient and the forward sensitivities on GS_LORENZ. */
 #define GS_VERN7 4
 
 #define GS_F32 1
@@ -337,8 +337,9 @@ GS_API gs_status gs_grad(const gs_problem* prob, const gs_mesh* mesh, const gs_l
  * turns singular) get NaN everywhere.  Built for GS_LORENZ with GS_TSIT5, and
  * for GS_LORENZ and GS_ROBERTSON with GS_ROS2 or GS_ROS3 (np + d = 6), fp64
  * and fp32, on landing and dense meshes (at a dense save point the matrix is
- * the tangent of the step's dense output); for GS_KIN8 with GS_ROS2 or
- * GS_ROS3 (np + d = 16) on landing meshes; other problems return
+ * the tangent of the step's dense output); for GS_LORENZ with GS_VERN7 on
+ * landing meshes; for GS_KIN8 with GS_ROS2 or GS_ROS3 (np + d = 16) on
+ * landing meshes; other problems return
  * GS_EUNSUPPORTED.  (The few-parameter forward-sensitivity
  * route that the gptget summary sets beside the adjoint.)
  */

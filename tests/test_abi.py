@@ -209,8 +209,8 @@ def test_ros3_method_validation_host_only(no_launch):
 @hidden_only
 def test_vern7_validation_host_only(no_launch):
     """Verner's 7(6) pair (method 4) is accepted for the d = 3 systems with
-    landing records; dense records, forward sensitivities, the d = 8 and
-    d = 64 systems and a gradient off Lorenz are not built.  The gradient
+    landing records; dense records, the d = 8 and d = 64 systems, and a
+    gradient or forward sensitivities off Lorenz are not built.  The gradient
     workspace is one checkpointed state per step and slot plus each save
     point's loss gradient.  No call here reaches a launch."""
     from discrete_adjoint_b200.gradsolve import _lib, _Mesh, _Tol, _Loss
@@ -225,7 +225,8 @@ def test_vern7_validation_host_only(no_launch):
         e = _host_problem(n=0, system=system, method=4)
         assert _lib.gs_count(ctypes.byref(e), ctypes.byref(tol), 100, None, None, None) == 0
         assert _lib.gs_count(ctypes.byref(e), ctypes.byref(dense), 100, None, None, None) == -4
-        assert _lib.gs_sens(ctypes.byref(e), ctypes.byref(m), ctypes.byref(ls), None, None, None, None, None) == -4
+        assert _lib.gs_sens(ctypes.byref(e), ctypes.byref(m), ctypes.byref(ls), None, None, None, None,
+                            None) == (0 if system == 1 else -4)
         md = _Mesh(100, 10, 16, 16, 16, 16, 16, 16)
         md.save_theta = 16
         assert _lib.gs_solve(ctypes.byref(e), ctypes.byref(md), None, None) == -4

@@ -2,8 +2,10 @@
 counts, step sizes, save indices: bitwise in fp64), the sizing pass, the
 replay and the adaptive forward-only solve (bitwise), the fused gradient
 (fp64 and fp32, per-trajectory gate) on the oracle's mesh in any slot order
-and on the GPU's own record, the in-place re-record, and the 2**20 ensemble
-of the benchmark in its launch configuration on a sample."""
+and on the GPU's own record, the in-place re-record, the forward
+sensitivities (matrices against the oracle's, gradient equal to the
+adjoint's), and the 2**20 ensemble of the benchmark in its launch
+configuration on a sample."""
 import dataclasses
 
 import numpy as np
@@ -13,7 +15,7 @@ import torch
 import oracle
 import workloads as W
 import discrete_adjoint_b200 as gs
-from gpu_util import (dev, ensemble, loss_args, mesh_by_trajectory, mesh_from_oracle, parity)
+from gpu_util import (TOL, dev, ensemble, loss_args, mesh_by_trajectory, mesh_from_oracle, parity, sens_parity)
 
 pytestmark = pytest.mark.gpu
 
@@ -112,6 +114,24 @@ def test_gradient_on_own_record_and_linear_loss():
     parity(out, prob, om)
 
 
+@pytest.mark.parametrize("dtype", ["f64", "f32"])
+def test_forward_sensitivities(dtype):
+    """d u(t_k)/d(p, u0) at the ten save points of the headline ensemble's
+    first trajectories, against the oracle's wide-tape matrices with the
+    per-trajectory gate; the loss bitwise that of the oracle's replay (fp64),
+    the gradient equal to the oracle's."""
+    prob = _prob(256, dtype=dtype)
+    om = oracle.record(prob, 1024)
+    assert (om.status == 0).all()
+    out, S = gs.gs_sens(ensemble(prob), mesh_from_oracle(om, dtype), **loss_args(prob))
+    torch.cuda.synchronize()
+    sens_parity(S.double().cpu().numpy(), prob, om, TOL[dtype])
+    parity(out, prob, om)
+    if dtype == "f64":
+        loss, _ = oracle.replay(prob, om)
+        assert np.array_equal(out.loss.cpu().numpy(), loss)
+
+
 def test_unsupported_paths():
     prob = _prob(4)
     ens = ensemble(prob)
@@ -119,12 +139,12 @@ def test_unsupported_paths():
         gs.gs_count(ens, prob.rtol, prob.atol, 100, dense=True)
     mesh = gs.new_mesh(prob.n, 512, len(prob.tsave), "f64", dev())
     gs.gs_record(ens, mesh, prob.rtol, prob.atol)
-    with pytest.raises(gs.gradsolve.GradsolveError):  # no forward-sensitivity kernel for the pair
-        gs.gs_sens(ens, mesh, **loss_args(prob))
     rob = dataclasses.replace(W.robertson(4), method="vern7")
     rmesh = gs.new_mesh(rob.n, 64, 1, "f64", dev())
     with pytest.raises(gs.gradsolve.GradsolveError):  # the gradient is built for Lorenz
         gs.gs_grad(ensemble(rob), rmesh, **loss_args(rob))
+    with pytest.raises(gs.gradsolve.GradsolveError):  # and so are the forward sensitivities
+        gs.gs_sens(ensemble(rob), rmesh, **loss_args(rob))
 
 
 def test_full_size_sampled():
