@@ -137,6 +137,13 @@ WORKLOADS = {
                                 desc="Robertson d=3, t in [0,1e5], ROS3, rtol=1e-6 atol=1e-10, loss w . u(T); one "
                                      "forward-sensitivity pass per step on the recorded mesh (d u(T)/d(p,u0) + the "
                                      "loss gradient)"),
+    # forward sensitivities with Verner's 7(6) pair: the state (321) + 6
+    # directions x the tangent step (411: stage sums 204, u' 45, nine
+    # Jacobian-vector products 162; hand count)
+    "lorenz_1m_vern7_sens": dict(kind="sens", problem="lorenz_1m", method="vern7", flop_step=321 + 6 * 411,
+                                 kernel="k_sens_vern7_lorenz", n=1 << 20, dtype="f64",
+                                 desc="Lorenz d=3, t in [0,10], Verner 7(6) rtol=atol=1e-6, 10 save points with N(0,1) "
+                                      "targets; one forward-sensitivity pass per step on the recorded mesh"),
     "lorenz_1m_sens": dict(kind="sens", problem="lorenz_1m", flop_step=192 + 6 * 252, kernel="k_sens_tsit5_lorenz",
                            n=1 << 20, dtype="f64",
                            desc="Lorenz d=3, t in [0,10], Tsit5 rtol=atol=1e-6, 10 save points with N(0,1) targets; "
@@ -190,6 +197,8 @@ def metric_name(args) -> str:
         return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, dense save points)"
     if args.workload == "lorenz_1m_vern7":
         return f"trajectory-gradients/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, Verner 7(6))"
+    if args.workload == "lorenz_1m_vern7_sens":
+        return f"trajectory-sensitivities/s (Lorenz Verner 7(6) {args.dtype.replace('f', 'fp')}, forward mode)"
     if args.workload == "lorenz_1m_sens":
         return f"trajectory-sensitivities/s (Lorenz {args.dtype.replace('f', 'fp')}, 1M traj, forward mode)"
     if args.workload == "robertson_ros3_sens":
@@ -382,7 +391,7 @@ def run_reference(args):
     solve = kind != "grad"
     sample = {"lorenz_1m": 256, "lorenz_1m_dense": 256, "lorenz_1m_vern7": 256, "lorenz_small": 256,
               "robertson": 32, "node64": 64,
-              "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512, "robertson_ros3": 256,
+              "lorenz_1m_solve": 4096, "lorenz_1m_sens": 512, "lorenz_1m_vern7_sens": 512, "robertson_ros3": 256,
               "robertson_ros3_sens": 256, "kin8": 256, "kin8_ros2": 16}[args.workload]
     prob = make_problem(args).subset(np.arange(sample))
     threads = oracle.default_threads()
@@ -880,6 +889,7 @@ SECONDARY = [
     ("node64_tensor", ["--workload", "node64"], 128),
     ("lorenz_1m_solve", ["--workload", "lorenz_1m_solve"], 0),
     ("lorenz_1m_sens", ["--workload", "lorenz_1m_sens"], 0),
+    ("lorenz_1m_vern7_sens", ["--workload", "lorenz_1m_vern7_sens"], 0),
     ("robertson_ros3_sens", ["--workload", "robertson_ros3_sens"], 0),
 ]
 
