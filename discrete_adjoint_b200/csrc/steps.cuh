@@ -48,9 +48,10 @@ __device__ __forceinline__ void jac3(const T u[3], const T p[3], T J[9]) {
 // +, -, *, /, fma and the exact frexp / ldexp / rint, in a fixed order, so its
 // bits are reproducible on any IEEE machine that keeps the order:
 //   ln x : x = m 2^e, m in [sqrt(1/2), sqrt(2)); ln m = 2 atanh(s),
-//          s = (m-1)/(m+1), series s (1 + z/3 + ... + z^12/25), z = s^2;
+//          s = (m-1)/(m+1), series s (1 + z/3 + ... + z^12/25), z = s^2,
+//          the polynomial by Estrin's scheme;
 //   exp w: Cody & Waite reduction w = k ln2 + r (ln2 = 21-bit head + tail),
-//          Taylor polynomial of e^r to degree 14, times 2^k.
+//          Taylor polynomial of e^r to degree 14 by Estrin's scheme, times 2^k.
 // Accuracy: ~1 ulp for the controller's arguments (errors 1e-4..1e3, |y| <= 1).
 __device__ __forceinline__ double frexpT(double x, int* e) { return frexp(x, e); }
 __device__ __forceinline__ float frexpT(float x, int* e) { return frexpf(x, e); }
@@ -69,9 +70,16 @@ __device__ T ctrl_ln(T x) {  // x > 0 finite
   }
   const T s = (m - cst<T>(1.0)) / (m + cst<T>(1.0));
   const T z = s * s;
-  T poly = cst<T>(1.0 / 25.0);
-#pragma unroll
-  for (int k = 11; k >= 0; --k) poly = fmaT(poly, z, cst<T>(1.0 / double(2 * k + 1)));
+  // sum_{k=0..12} z^k / (2k+1), Estrin's scheme: pairs in z, then z^2, z^4,
+  // z^8 (four dependent levels)
+#define GS_LNC(k) cst<T>(1.0 / double(2 * (k) + 1))
+  const T z2 = z * z, z4 = z2 * z2, z8 = z4 * z4;
+  const T q0 = fmaT(GS_LNC(1), z, GS_LNC(0)), q1 = fmaT(GS_LNC(3), z, GS_LNC(2)), q2 = fmaT(GS_LNC(5), z, GS_LNC(4));
+  const T q3 = fmaT(GS_LNC(7), z, GS_LNC(6)), q4 = fmaT(GS_LNC(9), z, GS_LNC(8)), q5 = fmaT(GS_LNC(11), z, GS_LNC(10));
+  const T r0 = fmaT(q1, z2, q0), r1 = fmaT(q3, z2, q2), r2 = fmaT(q5, z2, q4);
+  const T s0 = fmaT(r1, z4, r0), s1 = fmaT(GS_LNC(12), z4, r2);
+  const T poly = fmaT(s1, z8, s0);
+#undef GS_LNC
   const T lnm = (s + s) * poly;
   const T ef = (T)e;
   return fmaT(ef, cst<T>(0.6931467056274414), fmaT(ef, cst<T>(4.7493250390316726e-07), lnm));
@@ -101,9 +109,15 @@ __device__ T ctrl_exp(T w) {
                                    1.0 / 479001600.0,
                                    1.0 / 6227020800.0,
                                    1.0 / 87178291200.0};
-  T p = cst<T>(inv_fact[14]);
+  // Estrin's scheme: pairs in r, then r^2, r^4, r^8 (four dependent levels)
+  const T r2 = r * r, r4 = r2 * r2, r8 = r4 * r4;
+  T q[7];
 #pragma unroll
-  for (int j = 13; j >= 0; --j) p = fmaT(p, r, cst<T>(inv_fact[j]));
+  for (int i = 0; i < 7; ++i) q[i] = fmaT(cst<T>(inv_fact[2 * i + 1]), r, cst<T>(inv_fact[2 * i]));
+  const T t0 = fmaT(q[1], r2, q[0]), t1 = fmaT(q[3], r2, q[2]), t2 = fmaT(q[5], r2, q[4]);
+  const T t3 = fmaT(cst<T>(inv_fact[14]), r2, q[6]);
+  const T u0 = fmaT(t1, r4, t0), u1 = fmaT(t3, r4, t2);
+  const T p = fmaT(u1, r8, u0);
   return ldexpT(p, (int)kf);
 }
 

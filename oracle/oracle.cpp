@@ -625,8 +625,15 @@ T ctrl_ln(T x) {  // x > 0 finite
   }
   T s = (m - T(1)) / (m + T(1));
   T z = s * s;
-  T poly = T(1.0 / 25.0);
-  for (int k = 11; k >= 0; --k) poly = std::fma(poly, z, T(1.0 / double(2 * k + 1)));
+  // sum_{k=0..12} z^k / (2k+1) by Estrin's scheme: pairs in z, then z^2,
+  // z^4, z^8 (four dependent levels instead of twelve)
+  auto c = [](int k) { return T(1.0 / double(2 * k + 1)); };
+  const T z2 = z * z, z4 = z2 * z2, z8 = z4 * z4;
+  const T q0 = std::fma(c(1), z, c(0)), q1 = std::fma(c(3), z, c(2)), q2 = std::fma(c(5), z, c(4));
+  const T q3 = std::fma(c(7), z, c(6)), q4 = std::fma(c(9), z, c(8)), q5 = std::fma(c(11), z, c(10));
+  const T r0 = std::fma(q1, z2, q0), r1 = std::fma(q3, z2, q2), r2 = std::fma(q5, z2, q4);
+  const T s0 = std::fma(r1, z4, r0), s1 = std::fma(c(12), z4, r2);
+  T poly = std::fma(s1, z8, s0);
   T lnm = (s + s) * poly;
   return std::fma(T(e), T(CP_LN2_HI), std::fma(T(e), T(CP_LN2_LO), lnm));
 }
@@ -639,13 +646,20 @@ T ctrl_exp(T w) {
   if (kf < T(-2000)) return T(0);
   T r = std::fma(-kf, T(CP_LN2_HI), w);
   r = std::fma(-kf, T(CP_LN2_LO), r);
-  // 1/j!, j = 14 .. 0
-  double fact = 87178291200.0;  // 14!
-  T p = T(1.0 / fact);
-  for (int j = 13; j >= 0; --j) {
-    fact = fact / double(j + 1);  // exact: j! is an integer below 2^53
-    p = std::fma(p, r, T(1.0 / fact));
-  }
+  // sum_{j=0..14} r^j / j! by Estrin's scheme: pairs in r, then r^2, r^4,
+  // r^8 (four dependent levels instead of fourteen); j! is exact in double
+  auto d = [](int j) {
+    double f = 1.0;
+    for (int i = 2; i <= j; ++i) f *= double(i);
+    return T(1.0 / f);
+  };
+  const T r2 = r * r, r4 = r2 * r2, r8 = r4 * r4;
+  T q[7];
+  for (int i = 0; i < 7; ++i) q[i] = std::fma(d(2 * i + 1), r, d(2 * i));
+  const T t0 = std::fma(q[1], r2, q[0]), t1 = std::fma(q[3], r2, q[2]), t2 = std::fma(q[5], r2, q[4]);
+  const T t3 = std::fma(d(14), r2, q[6]);
+  const T u0 = std::fma(t1, r4, t0), u1 = std::fma(t3, r4, t2);
+  const T p = std::fma(u1, r8, u0);
   return std::ldexp(p, int(kf));
 }
 
