@@ -45,6 +45,7 @@ namespace gs {
 #define GS_V7_RING 8
 #endif
 constexpr int kV7Ring = GS_V7_RING;
+constexpr int kV7BS = 128;  // threads per block; a thread's ring rows are kV7BS elements apart
 static_assert((kV7Ring & (kV7Ring - 1)) == 0 && kV7Ring >= 2, "ring depth: a power of two, at least 2");
 
 template <typename T>
@@ -80,7 +81,7 @@ __device__ __forceinline__ void lorenz_vjp3(const T U[3], T s, T r, T b, const T
 }
 
 template <typename T>
-__global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7LorenzArgs<T> a) {
+__global__ void __launch_bounds__(kV7BS, GS_V7_MINB) k_grad_vern7_lorenz(Vern7LorenzArgs<T> a) {
   const int64_t n = a.n;
   const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= n) return;
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
   // Per-thread copy rings (cp.async into shared memory, each thread waiting
   // on its own copies only): forward, row st % kV7Ring holds h of step st;
   // reverse, rows 4 (st % kV7Ring) + c hold checkpoint row c (c < 3) and h
-  // (c = 3) of step st.  Element (row w) of a thread is rg[w * 128]:
+  // (c = 3) of step st.  Element (row w) of a thread is rg[w * kV7BS]:
   // consecutive threads touch consecutive words.
   extern __shared__ __align__(16) unsigned char v7_ring_raw[];
   T* const rg = reinterpret_cast<T*>(v7_ring_raw) + threadIdx.x;
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
   // ---------------------------------------------------------------- forward
   {
     auto issue_f = [&](int sf) {
-      if (sf < S) cp_async_el(rg + (sf & (kV7Ring - 1)) * 128, hp + (int64_t)sf * n);
+      if (sf < S) cp_async_el(rg + (sf & (kV7Ring - 1)) * kV7BS, hp + (int64_t)sf * n);
       cp_async_commit();
     };
     T k1[3];
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
     for (int st = 0; st < S; ++st) {
       const T h = hn;
       cp_async_wait<kV7Ring - 2>();  // the group of step st + 1
-      if (st + 1 < S) hn = rg[((st + 1) & (kV7Ring - 1)) * 128];
+      if (st + 1 < S) hn = rg[((st + 1) & (kV7Ring - 1)) * kV7BS];
 #pragma unroll
       for (int c = 0; c < 3; ++c) cp[(int64_t)st * n3 + c * n] = u[c];
       T un[3];
@@ -184,19 +185,19 @@ __global__ void __launch_bounds__(128, GS_V7_MINB) k_grad_vern7_lorenz(Vern7Lore
   int next = kk >= 0 ? a.save_idx[(int64_t)kk * n + j] : -1;
   auto issue_r = [&](int sr) {  // step sr's checkpoint rows and h
     if (sr >= 0 && sr < S) {
-      T* d = rg + (sr & (kV7Ring - 1)) * 4 * 128;
+      T* d = rg + (sr & (kV7Ring - 1)) * 4 * kV7BS;
 #pragma unroll
-      for (int c = 0; c < 3; ++c) cp_async_el(d + c * 128, cp + (int64_t)sr * n3 + c * n);
-      cp_async_el(d + 3 * 128, hp + (int64_t)sr * n);
+      for (int c = 0; c < 3; ++c) cp_async_el(d + c * kV7BS, cp + (int64_t)sr * n3 + c * n);
+      cp_async_el(d + 3 * kV7BS, hp + (int64_t)sr * n);
     }
     cp_async_commit();
   };
   T cu[3], ch = cst<T>(0.0);
   auto take_r = [&](int sr) {
-    const T* d = rg + (sr & (kV7Ring - 1)) * 4 * 128;
+    const T* d = rg + (sr & (kV7Ring - 1)) * 4 * kV7BS;
 #pragma unroll
-    for (int c = 0; c < 3; ++c) cu[c] = d[c * 128];
-    ch = d[3 * 128];
+    for (int c = 0; c < 3; ++c) cu[c] = d[c * kV7BS];
+    ch = d[3 * kV7BS];
   };
 #pragma unroll
   for (int i2 = 0; i2 < kV7Ring; ++i2) issue_r(S - 1 - i2);
@@ -296,13 +297,13 @@ gs_status launch_grad_vern7_lorenz(const gs_problem* P, const gs_mesh* M, const 
   a.du0 = (T*)du0;
   a.ck = (T*)ws;
   a.gsave = (T*)ws + (size_t)M->smax * 3 * (size_t)P->n;
-  const int64_t grid = (P->n + 127) / 128;
-  const size_t smem = (size_t)kV7Ring * 4 * 128 * sizeof(T);  // the larger (reverse) ring
+  const int64_t grid = (P->n + kV7BS - 1) / kV7BS;
+  const size_t smem = (size_t)kV7Ring * 4 * kV7BS * sizeof(T);  // the larger (reverse) ring
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(k_grad_vern7_lorenz<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess)
     return GS_ECUDA;
-  k_grad_vern7_lorenz<T><<<(unsigned)grid, 128, smem, st>>>(a);
+  k_grad_vern7_lorenz<T><<<(unsigned)grid, kV7BS, smem, st>>>(a);
   count_launch();
   return launch_ok() ? GS_OK : GS_ECUDA;
 }
