@@ -132,6 +132,31 @@ def test_forward_sensitivities(dtype):
         assert np.array_equal(out.loss.cpu().numpy(), loss)
 
 
+def test_failed_trajectories_are_nan(case):
+    """Slots whose status is not OK (or whose step count is out of range) get
+    NaN loss, gradient and sensitivities; the others are unaffected."""
+    prob, om = case
+    sub = prob.subset(np.arange(8))
+    st = np.zeros(8, np.int32)
+    st[[1, 5]] = 2  # GS_TRAJ_DTMIN
+    ns = om.nsteps[:8].copy()
+    ns[6] = om.h.shape[1] + 1  # beyond the mesh capacity
+    bad = oracle.Mesh(om.h[:8], ns, om.save_idx[:8], st, om.nreject[:8])
+    good = oracle.Mesh(om.h[:8], om.nsteps[:8], om.save_idx[:8], np.zeros(8, np.int32), om.nreject[:8])
+    ens = ensemble(sub)
+    out = gs.gs_grad(ens, mesh_from_oracle(bad, "f64"), **loss_args(sub))
+    ref = gs.gs_grad(ens, mesh_from_oracle(good, "f64"), **loss_args(sub))
+    sens_out, S = gs.gs_sens(ens, mesh_from_oracle(bad, "f64"), **loss_args(sub))
+    torch.cuda.synchronize()
+    failed = np.array([1, 5, 6])
+    ok = np.setdiff1d(np.arange(8), failed)
+    for o in (out, sens_out):
+        for t in (o.loss.cpu().numpy()[None, :], o.dp.cpu().numpy(), o.du0.cpu().numpy()):
+            assert np.isnan(t[:, failed]).all() and np.isfinite(t[:, ok]).all()
+    assert np.isnan(S.cpu().numpy()[..., failed]).all()
+    assert np.array_equal(out.dp.cpu().numpy()[:, ok], ref.dp.cpu().numpy()[:, ok])
+
+
 def test_unsupported_paths():
     prob = _prob(4)
     ens = ensemble(prob)
