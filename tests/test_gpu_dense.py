@@ -113,6 +113,40 @@ def test_dense_sensitivities(case):
     assert np.abs(out.loss.cpu().numpy() - loss).max() <= 1e-14 * np.abs(loss).max()
 
 
+def test_dense_several_save_points_per_step():
+    """Save times closer than the steps (48 in t in [0.01, 0.5] on Lorenz at
+    rtol = atol = 1e-5): several fall inside one step, each read off that
+    step's continuous extension. Record, adaptive solve, replay, gradient and
+    forward sensitivities against the oracle."""
+    prob = W.lorenz_small(300)
+    prob.rtol = prob.atol = 1e-5
+    prob.t1 = 0.5
+    prob.tsave = np.linspace(0.01, 0.5, 48)
+    prob.target = np.random.default_rng(8).normal(0.0, 1.0, (48, 3, prob.n))
+    om = oracle.record(prob, 512, dense=True)
+    assert (om.status == 0).all()
+    assert (np.diff(om.save_idx, axis=1) == 0).any()  # save points sharing a step
+    ens, mesh = _record_gpu(prob, 512)
+    h, ns, si, st, _ = mesh_by_trajectory(mesh)
+    assert np.array_equal(ns, om.nsteps) and np.array_equal(si, om.save_idx)
+    assert np.abs(theta_by_trajectory(mesh) - om.theta).max() <= 1e-10
+    _, ur = oracle.replay(prob, om)
+    u = gs.gs_solve(ens, mesh_from_oracle(om, "f64")).cpu().numpy()
+    assert np.abs(u - ur).max() <= 1e-14 * np.abs(ur).max()
+    ua, na, sa = gs.gs_solve_adaptive(ens, prob.rtol, prob.atol, 512, dense=True)
+    uo, no, so = oracle.solve_adaptive(prob, 512, dense=True)
+    assert np.array_equal(ua.cpu().numpy(), uo)  # the same arithmetic: bitwise
+    out = gs.gs_grad(ens, mesh_from_oracle(om, "f64"), **loss_args(prob))
+    torch.cuda.synchronize()
+    parity(out, prob, om)
+    sub = prob.subset(np.arange(64))
+    osub = oracle.Mesh(om.h[:64], om.nsteps[:64], om.save_idx[:64], om.status[:64], om.nreject[:64],
+                       om.theta[:64])
+    sout, S = gs.gs_sens(ensemble(sub), mesh_from_oracle(osub, "f64"), **loss_args(sub))
+    torch.cuda.synchronize()
+    sens_parity(S.double().cpu().numpy(), sub, osub, TOL["f64"])
+
+
 def test_dense_unsupported_paths(case):
     k8 = W.kin8(4)  # dense records are built for the d = 3 systems
     with pytest.raises(gs.gradsolve.GradsolveError):
